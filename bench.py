@@ -1,0 +1,402 @@
+#!/usr/bin/env python
+"""Benchmark: compressed-cache decode attention on B200.
+
+One step = one decode step of the long-context workload (32 query / 8 KV heads, head_dim 128,
+batch 1, 1,048,576 cached tokens): encode + append one token per sequence, then full attention of
+all query heads over the whole compressed cache (query prep, popcount scores, online softmax,
+4-bit P.V, split merge).  The cache (872 MB compressed) is larger than L2 (126 MB), so no L2
+flush is needed between steps.
+
+    python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference] [--config c5]
+
+Prints ONE JSON line (rank 0).  With N > 1 (torchrun, one rank per GPU) every rank runs its own
+independent sequence (weak scaling, no data-path collective); time = max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "compressed-cache decode attention: KV tokens/s per head and HBM GB/s vs peak"
+UNIT = "kv_token_heads/s"
+BYTES_PER_TOKEN_HEAD = 104  # 16 B sign bits + 4 B norm + 4 B 1/C + 64 B codes + 16 B scale/min
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default="c5")
+    ap.add_argument("--engine", choices=["tensor", "cuda_core"], default="tensor")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-alt", action="store_true")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+# ------------------------------------------------------------------------------------------ clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu_index = gpu_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                                          "-lms", "200", "-i", str(self.gpu_index)], stdout=subprocess.PIPE,
+                                         stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+
+    def _read(self):
+        for ln in self.proc.stdout:
+            self.lines.append(ln.strip())
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [x.strip() for x in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------------------------------ dist
+def dist_setup():
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    else:
+        torch.cuda.set_device(0)
+    return world, rank, local
+
+
+def reduce_max(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def reduce_sum(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.SUM)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.barrier()
+
+
+# ------------------------------------------------------------------------------------------ ours
+def build_cache(cfg, extra_tokens: int, device):
+    import long_context_decode_kv1b_b200 as kv
+    from long_context_decode_kv1b_b200 import workloads as wl
+
+    cap = (cfg.L + extra_tokens + 127) // 128 * 128
+    cache = kv.Cache(cfg.B, cfg.Hkv, cap, seed=cfg.rotation_seed, device=device)
+    for start, n in wl.prefill_chunks(cfg):
+        K, V = wl.prefill_chunk(cfg, start, n, device)
+        cache.append(K, V)
+    return cache
+
+
+def cpu_baseline(cfg, steps_like: bool):
+    """Time the CPU oracle (single thread, as it stands) on a bounded sample of the workload:
+    full attention of the G query heads of one kv-head over the first S tokens of the cache."""
+    import numpy as np
+    import torch
+
+    import oracle
+    from long_context_decode_kv1b_b200 import workloads as wl
+
+    S = 1 << 18
+    K = np.zeros((S, 128), np.float32)
+    V = np.zeros((S, 128), np.float32)
+    for start, n in wl.prefill_chunks(cfg, S):
+        k, v = wl.prefill_chunk(cfg, start, n, "cpu")
+        K[start:start + n] = k[0, :, 0].float().numpy()
+        V[start:start + n] = v[0, :, 0].float().numpy()
+    D = oracle.signs(cfg.rotation_seed)
+    enc = oracle.encode(K, V, D)
+    q = wl.queries(cfg, 0, "cpu")[0, : cfg.G].float().numpy()
+    reps = 0
+    t0 = time.perf_counter()
+    while True:
+        for j in range(cfg.G):
+            oracle.attend(enc, q[j], D, cfg.scale)
+        reps += 1
+        dt = time.perf_counter() - t0
+        if dt >= 10.0 or reps >= 8:
+            break
+    return {"value": S * reps / dt, "unit": UNIT, "cores": 1, "kind": "oracle",
+            "sample": f"{cfg.name}: full attention of the {cfg.G} query heads of kv-head 0 over the first {S} "
+                      f"cached tokens, {reps} repetitions (single-threaded C++ oracle, fp64 softmax/accumulation), "
+                      f"{dt:.1f} s"}
+
+
+def run_ours(args):
+    import torch
+
+    import long_context_decode_kv1b_b200 as kv
+    from long_context_decode_kv1b_b200 import workloads as wl
+
+    world, rank, local = dist_setup()
+    dev = torch.device("cuda", local if world > 1 else 0)
+    base = wl.CONFIGS[args.config]
+    cfg = dataclasses.replace(base, seed=base.seed + 1000 * rank) if world > 1 else base
+    W, K = args.warmup, args.steps
+    n_alt = 0 if args.no_alt else 5
+    extra = W + K + (0 if args.no_e2e else K)
+    engine = kv.ATTEND_TENSOR if args.engine == "tensor" else kv.ATTEND_CUDA_CORE
+    cache = build_cache(cfg, extra, dev)
+    nsteps = W + K
+    ks, vs, qs = [], [], []
+    for i in range(nsteps + (0 if args.no_e2e else K)):
+        k, v = wl.step_kv(cfg, i, dev)
+        ks.append(k)
+        vs.append(v)
+        qs.append(wl.queries(cfg, i, dev))
+    out = torch.empty((cfg.B, cfg.Hq, 128), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+    for i in range(W):
+        cache.append(ks[i], vs[i])
+        cache.attend(qs[i], cfg.scale, out=out, engine=engine)
+    torch.cuda.synchronize()
+    barrier(world)
+    gpu_index = int(os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0]) if world == 1 and \
+        os.environ.get("CUDA_VISIBLE_DEVICES", "0").split(",")[0].isdigit() else local
+    sampler = ClockSampler(gpu_index if world == 1 else local)
+    sampler.start()
+    time.sleep(0.3)
+    a0 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    a1 = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    units = 0
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for j in range(K):
+        i = W + j
+        cache.append(ks[i], vs[i])
+        a0[j].record(stream)
+        cache.attend(qs[i], cfg.scale, out=out, engine=engine)
+        a1[j].record(stream)
+        units += cfg.B * cfg.Hkv * cache.lengths[0]
+    e1.record(stream)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    barrier(world)
+    t_ms = e0.elapsed_time(e1)
+    t_max = reduce_max(t_ms, world)
+    units_total = reduce_sum(units, world)
+    attend_ms = [a0[j].elapsed_time(a1[j]) for j in range(K)]
+    att_avg = statistics.mean(attend_ms)
+    L_mean = units / K / (cfg.B * cfg.Hkv)
+    bytes_per_attend = cfg.B * cfg.Hkv * L_mean * BYTES_PER_TOKEN_HEAD
+    peak, peak_kind = peaks()
+    achieved = bytes_per_attend / (att_avg * 1e-3) / 1e9
+    value = units_total / (t_max * 1e-3)
+
+    e2e = None
+    if not args.no_e2e:
+        qh = [q.cpu().pin_memory() for q in qs[nsteps:]]
+        kh = [k.cpu().pin_memory() for k in ks[nsteps:]]
+        vh = [v.cpu().pin_memory() for v in vs[nsteps:]]
+        outh = torch.empty((cfg.B, cfg.Hq, 128), dtype=torch.float32).pin_memory()
+        qd, kd, vd = torch.empty_like(qs[0]), torch.empty_like(ks[0]), torch.empty_like(vs[0])
+        torch.cuda.synchronize()
+        barrier(world)
+        h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        units_e = 0
+        h0.record(stream)
+        for j in range(K):
+            kv.attend_from_host(cache, qh[j], kh[j], vh[j], cfg.scale, outh, qd, kd, vd, stream=stream)
+            units_e += cfg.B * cfg.Hkv * cache.lengths[0]
+        h1.record(stream)
+        torch.cuda.synchronize()
+        barrier(world)
+        te = reduce_max(h0.elapsed_time(h1), world)
+        ue = reduce_sum(units_e, world)
+        h2d = qh[0].numel() * qh[0].element_size() + 2 * kh[0].numel() * kh[0].element_size()
+        e2e = {"value": ue / (te * 1e-3), "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": outh.numel() * outh.element_size(),
+               "path": "kv1b binding: pinned host K/V/q -> device, kv1b_encode_append, kv1b_attend, out -> host"}
+
+    alt = None
+    if n_alt:
+        other = kv.ATTEND_CUDA_CORE if engine == kv.ATTEND_TENSOR else kv.ATTEND_TENSOR
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n_alt)]
+        for x, y in ev:
+            x.record(stream)
+            cache.attend(qs[0], cfg.scale, out=out, engine=other)
+            y.record(stream)
+        torch.cuda.synchronize()
+        alt_ms = statistics.mean(x.elapsed_time(y) for x, y in ev)
+        Lc = cache.lengths[0]
+        alt = {"engine": "cuda_core" if other == kv.ATTEND_CUDA_CORE else "tensor", "attend_us": alt_ms * 1e3,
+               "achieved_gbs": cfg.B * cfg.Hkv * Lc * BYTES_PER_TOKEN_HEAD / (alt_ms * 1e-3) / 1e9}
+        alt["frac"] = alt["achieved_gbs"] / peak
+
+    result = None
+    if rank == 0:
+        result = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
+            "ms_per_step": t_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "u1 key bits / u4 value codes; int32 popcount; fp32 softmax + accumulation",
+            "data": "synthetic (seeded torch generators; see long_context_decode_kv1b_b200/workloads.py)",
+            "config": {"workload": f"{cfg.name}: {wl.DESCRIPTIONS[cfg.name]}", "batch": cfg.B, "q_heads": cfg.Hq,
+                       "kv_heads": cfg.Hkv, "head_dim": 128, "context": cfg.L,
+                       "step": "append 1 token/sequence + full attend", "engine": args.engine,
+                       "l2": "inputs larger than L2 (compressed cache %.0f MB > 126 MB); no flush" %
+                             (bytes_per_attend / 1e6), "parallelism": f"independent sequence per GPU x{world}"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None, "kernel": "kv1b_attend (attend + merge)",
+                         "attend_us": att_avg * 1e3, "peak_kind": peak_kind,
+                         "frac_of_8tbs": achieved / 8000.0},
+            "e2e": e2e,
+            "gpu_launches": 3 * K,
+            "clocks": clocks,
+        }
+        if alt:
+            result["alt_engine"] = alt
+    barrier(world)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+    if rank == 0:
+        if world == 1 and not args.no_cpu_baseline:
+            result["cpu_baseline"] = cpu_baseline(cfg, True)
+        print(json.dumps(result))
+
+
+# ------------------------------------------------------------------------------------------ reference
+def run_reference(args):
+    """The oracle, as it stands, timed on the host cores on a bounded sample of each step."""
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    import numpy as np
+
+    import oracle
+    from long_context_decode_kv1b_b200 import workloads as wl
+
+    cfg = wl.CONFIGS[args.config]
+    S = 1 << 15  # tokens of one kv-head attended by its G query heads per step
+    K = np.zeros((S, 128), np.float32)
+    V = np.zeros((S, 128), np.float32)
+    for start, n in wl.prefill_chunks(cfg, S):
+        k, v = wl.prefill_chunk(cfg, start, n, "cpu")
+        K[start:start + n] = k[0, :, 0].float().numpy()
+        V[start:start + n] = v[0, :, 0].float().numpy()
+    D = oracle.signs(cfg.rotation_seed)
+    enc = oracle.encode(K, V, D)
+    times = []
+    for i in range(args.warmup + args.steps):
+        q = wl.queries(cfg, i, "cpu")[0, : cfg.G].float().numpy()
+        t0 = time.perf_counter()
+        for j in range(cfg.G):
+            oracle.attend(enc, q[j], D, cfg.scale)
+        if i >= args.warmup:
+            times.append(time.perf_counter() - t0)
+    tot = sum(times)
+    value = S * len(times) / tot
+    sample = (f"{cfg.name}: per step, full attention of the {cfg.G} query heads of kv-head 0 over the first {S} "
+              f"cached tokens (single-threaded C++ oracle)")
+    print(json.dumps({
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": tot / len(times) * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32 steps, f64 softmax/accumulation", "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: {wl.DESCRIPTIONS[cfg.name]}"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }))
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,179 @@
+/*
+ * kv1b.h -- C ABI of the B200 (sm_100a) library for decode attention over a compressed KV cache.
+ *
+ * What the library computes (pages cited by title and section):
+ *  - Keys are kept as 1-bit sign sketches of a seeded random rotation, with a per-token norm and
+ *    correction scalar ("RaBitQCache: Rotated Binary Quantization for KVCache in Long Context LLM
+ *    Inference", abstract and core idea: randomised rotated binary quantisation; "H1B-KV: Hybrid
+ *    One-Bit Caches ...", key design: 1-bit sketch by random projection).  The rotation is
+ *    y = H * (D (.) k): H the unnormalised 128x128 Walsh-Hadamard matrix in natural order, D a
+ *    +-1 vector from SplitMix64(seed).  Bit i of word w is 1 iff y[32w+i] >= 0 (the bitmap rule of
+ *    the H1IB-KV news article, part 2 item 3: a set bit stands for +1).
+ *  - Values are 4-bit linear codes with an fp16 scale and an fp16 min per 32 channels (H1B-KV,
+ *    key design: 4-bit linear quantisation of values).
+ *  - Attention logits are estimated with binary x INT4 popcount arithmetic between the key bits
+ *    and the 4 bit-planes of the rotated, 4-bit-quantised query (RaBitQCache abstract and key
+ *    design); the output is the softmax-weighted sum of the dequantised values (H1B-KV,
+ *    technical framework), either over all tokens (kv1b_attend) or over the adaptive Top-p set
+ *    (kv1b_attend_topp; RaBitQCache abstract: adaptive Top-p retrieval).
+ *
+ * Conventions (every entry point):
+ *  - All data pointers are DEVICE pointers unless a parameter says "host".  The caller owns every
+ *    buffer; the library never allocates device memory and keeps no state outside the
+ *    kv1b_cache_t descriptor the caller holds.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Every call that
+ *    launches work is asynchronous on that stream, except kv1b_read_status (synchronous).
+ *  - Return value: KV1B_OK (0) or a negative KV1B_ERR_* code.  Arguments are validated on the
+ *    host before any launch; on error nothing is launched and no buffer is written.  No C++
+ *    exception crosses the ABI.  Conditions only the device can see (non-finite inputs, fp16
+ *    saturation of a value group) set bits in the cache's status word (kv1b_read_status).
+ *  - head_dim must be 128.  capacity must be a positive multiple of 128.  batch <= 64.
+ *    num_q_heads must be a multiple of num_kv_heads with G = num_q_heads / num_kv_heads <= 8;
+ *    query head hq reads KV head hq / G.
+ */
+#ifndef KV1B_H
+#define KV1B_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KV1B_HEAD_DIM 128
+#define KV1B_MAX_BATCH 64
+#define KV1B_MAX_GROUP 8
+#define KV1B_CAPACITY_ALIGN 128
+
+/* return codes */
+#define KV1B_OK 0
+#define KV1B_ERR_INVALID_ARG (-1)      /* null pointer, bad count, p not in (0,1], Hq % Hkv != 0 ... */
+#define KV1B_ERR_UNSUPPORTED (-2)      /* head_dim != 128, G > 8, batch > 64 */
+#define KV1B_ERR_CAPACITY (-3)         /* an append would exceed the capacity */
+#define KV1B_ERR_MISALIGNED (-4)       /* a pointer or stride breaks the alignment rule stated below */
+#define KV1B_ERR_WORKSPACE (-5)        /* workspace or cache buffer smaller than required */
+#define KV1B_ERR_CUDA (-6)             /* a CUDA launch/runtime error (cudaGetLastError) */
+
+/* element types of K, V and q */
+#define KV1B_DTYPE_F32 0
+#define KV1B_DTYPE_BF16 1
+#define KV1B_DTYPE_F16 2
+
+/* kv1b_attend flags: which engine forms the probability-weighted sum of values */
+#define KV1B_ATTEND_TENSOR 0     /* default: mma.sync (f16 codes x hi/lo-split f16 weights, fp32 accumulate) */
+#define KV1B_ATTEND_CUDA_CORE 1  /* fp32 FMA on the CUDA cores */
+
+/* status word bits (kv1b_read_status) */
+#define KV1B_STATUS_NONFINITE 1       /* a K or V element appended was NaN or Inf */
+#define KV1B_STATUS_FP16_SATURATED 2  /* a value group's min or scale left the binary16 range */
+
+/*
+ * Cache descriptor.  Filled by kv1b_cache_init; treat as opaque except for reading the fields.
+ * Device planes (carved from one caller buffer, token-major within each (sequence, kv-head)):
+ *   k_bits  u32 [batch][hkv][capacity][4]     sign bits of the rotated key (16 B / token)
+ *   k_norm  f32 [batch][hkv][capacity]        N = ||k|| (fixed pairwise tree sum of squares)
+ *   k_cinv  f32 [batch][hkv][capacity]        1/C = 128 N / sum_i |y_i| (1 when the sum is 0)
+ *   v_codes u32 [batch][hkv][capacity/16][8][32]  4-bit value codes in 16-token tiles; for tile T,
+ *           m-tile mt (channels 16mt..16mt+15) and lane l (g = l>>2, t = l&3) the word holds
+ *           bits 0-3 / 16-19:  channel 16mt+g,   tokens 16T+2t / 16T+2t+1
+ *           bits 4-7 / 20-23:  channel 16mt+g+8, tokens 16T+2t / 16T+2t+1
+ *           bits 8-11 / 24-27: channel 16mt+g,   tokens 16T+2t+8 / 16T+2t+9
+ *           bits 12-15 / 28-31: channel 16mt+g+8, tokens 16T+2t+8 / 16T+2t+9
+ *   v_sm    u32 [batch][hkv][capacity][4]     per 32-channel group: low half = fp16 scale,
+ *           high half = fp16 min; value = min + scale * code
+ *   signs   f32 [128]                         rotation signs D (+-1)
+ *   d_lengths i32 [batch]                     tokens held per sequence (device copy)
+ *   d_status  i32 [1]                         OR of KV1B_STATUS_* bits since init
+ * h_lengths is the host mirror of d_lengths; both change only through kv1b_encode_append.
+ */
+typedef struct kv1b_cache {
+  int32_t batch;
+  int32_t num_kv_heads;
+  int32_t head_dim;
+  int32_t capacity;
+  uint64_t rotation_seed;
+  uint32_t* k_bits;
+  float* k_norm;
+  float* k_cinv;
+  uint32_t* v_codes;
+  uint32_t* v_sm;
+  float* signs;
+  int32_t* d_lengths;
+  int32_t* d_status;
+  int64_t h_lengths[KV1B_MAX_BATCH];
+} kv1b_cache_t;
+
+/* Bytes of device memory a cache of this shape needs (0 if the shape is unsupported). */
+size_t kv1b_cache_bytes(int32_t batch, int32_t num_kv_heads, int32_t head_dim, int32_t capacity);
+
+/* Lay a cache out in the caller's device buffer `dev_buf` (256-byte aligned, `bytes` >=
+ * kv1b_cache_bytes), zero it, draw the rotation signs from SplitMix64(seed) and set all lengths
+ * to 0.  Writes the descriptor *cache (host memory).  Asynchronous on `stream`. */
+int kv1b_cache_init(kv1b_cache_t* cache, void* dev_buf, size_t bytes, int32_t batch, int32_t num_kv_heads,
+                    int32_t head_dim, int32_t capacity, uint64_t seed, void* stream);
+
+/* Encode and append n_new tokens to every sequence (the same n_new for all).
+ * k, v: device arrays of `dtype` (KV1B_DTYPE_*); element (b, t, h, c) of K sits at
+ * k[b*stride_b + t*stride_t + h*stride_h + c] (strides in elements, channel stride 1); V uses
+ * the same strides.  Alignment rule: k and v 16-byte aligned; stride_b, stride_t, stride_h
+ * multiples of 4 elements (so every 4-channel slice is an aligned vector).
+ * Per (sequence, token, kv-head): rotation + sign bits + N + 1/C, and 4-bit value codes with an
+ * fp16 min (rounded down) and fp16 scale (smallest with 15*scale >= range).  The tokens land at
+ * positions h_lengths[b] .. h_lengths[b]+n_new-1, then lengths advance (host mirror and device).
+ * Errors: KV1B_ERR_CAPACITY when h_lengths[b] + n_new > capacity for some b. */
+int kv1b_encode_append(kv1b_cache_t* cache, const void* k, const void* v, int32_t dtype, int32_t n_new,
+                       int64_t stride_b, int64_t stride_t, int64_t stride_h, void* stream);
+
+/* Workspace bytes kv1b_attend (mode 0) or kv1b_attend_topp (mode 1) needs for this cache and
+ * num_q_heads at any length up to the capacity.  0 on invalid arguments. */
+size_t kv1b_attend_workspace_bytes(const kv1b_cache_t* cache, int32_t num_q_heads, int32_t mode);
+
+/* Full decode attention over all cached tokens.
+ * q: [batch][num_q_heads][128] contiguous, `q_dtype`, 16-byte aligned.
+ * out: f32 [batch][num_q_heads][128].  For each (b, hq): with logits s_t estimated from the
+ * key sketch (binary x INT4 popcount) and scaled by `scale`, out = sum_t softmax(s)_t * vhat_t,
+ * vhat = min + scale_g * code.  A sequence of length 0 gives zeros.
+ * ws: device workspace, 256-byte aligned, ws_bytes >= kv1b_attend_workspace_bytes(.., 0).
+ * flags: KV1B_ATTEND_TENSOR (default) or KV1B_ATTEND_CUDA_CORE (same result within fp32
+ * rounding).  num_splits: 0 chooses the split-K factor; > 0 forces it (testing). */
+int kv1b_attend(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,
+                float* out, void* ws, size_t ws_bytes, int32_t flags, int32_t num_splits, void* stream);
+
+/* Adaptive Top-p decode attention.  Per (b, hq): integer masses u_t ~ 2^32 exp(s_t - max s)
+ * (degree-7 polynomial for 2^f, reproducible bit for bit), T = ceil(p * sum u) in fp64; the
+ * selected set is the shortest prefix of the order (s desc, index asc) whose mass reaches T.
+ * sel_idx: i32 [batch][num_q_heads][capacity] receives the selected token indices in ascending
+ * order (entries past sel_cnt are left unspecified); sel_cnt: i32 [batch][num_q_heads].
+ * out: f32 [batch][num_q_heads][128], the softmax over the selected tokens only.
+ * p must be in (0, 1].  ws_bytes >= kv1b_attend_workspace_bytes(.., 1). */
+int kv1b_attend_topp(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,
+                     float p, float* out, int32_t* sel_idx, int32_t* sel_cnt, void* ws, size_t ws_bytes,
+                     void* stream);
+
+/* Test hook for the query preparation step: planes u32 [batch][num_q_heads][4][4] (plane j,
+ * word w, bit i = bit j of the code of rotated channel 32w+i), vl / delta f32 [batch][num_q_heads]
+ * (grid origin and step), sq i32 [batch][num_q_heads] (sum of codes). */
+int kv1b_query_prep(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads,
+                    uint32_t* planes, float* vl, float* delta, int32_t* sq, void* stream);
+
+/* Test hook for the proxy score: for every (b, hq) and token t < length[b]:
+ * A = sum_j 2^j sum_w popc(k_bits_w & P_jw), Bc = sum_w popc(k_bits_w) (i32) and the fp32 logit
+ * (the exact arithmetic kv1b_attend_topp selects with).  A, Bc, s: [batch][num_q_heads][capacity];
+ * entries at t >= length[b] are left unspecified. */
+int kv1b_scores(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,
+                int32_t* A, int32_t* Bc, float* s, void* stream);
+
+/* Synchronous: waits for `stream`, then copies the cache's status word to *flags (host). */
+int kv1b_read_status(const kv1b_cache_t* cache, int32_t* flags, void* stream);
+
+/* Static string for a return code. */
+const char* kv1b_status_string(int code);
+
+/* Library version (major * 10000 + minor * 100 + patch). */
+int kv1b_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* KV1B_H */

@@ -1,0 +1,256 @@
+"""Python binding of ``libkv1b.so`` -- decode attention over a 1-bit-key / 4-bit-value KV cache.
+
+Argument marshalling only: every step of the path runs in the CUDA library (``csrc/``) behind the
+C ABI of ``include/kv1b.h``; PyTorch provides device memory and streams.  The library must have
+been built (``python -m long_context_decode_kv1b_b200.build``); there is no CPU fallback and
+importing the binding on a machine without the built library raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libkv1b.so")
+
+HEAD_DIM = 128
+MAX_BATCH = 64
+DTYPE_F32, DTYPE_BF16, DTYPE_F16 = 0, 1, 2
+ATTEND_TENSOR, ATTEND_CUDA_CORE = 0, 1
+STATUS_NONFINITE, STATUS_FP16_SATURATED = 1, 2
+ERRORS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "capacity", -4: "misaligned",
+          -5: "workspace too small", -6: "CUDA error"}
+
+# symbols declared in include/kv1b.h
+SYMBOLS = ("kv1b_cache_bytes", "kv1b_cache_init", "kv1b_encode_append", "kv1b_attend_workspace_bytes",
+           "kv1b_attend", "kv1b_attend_topp", "kv1b_query_prep", "kv1b_scores", "kv1b_read_status",
+           "kv1b_status_string", "kv1b_version")
+
+
+class Kv1bError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        super().__init__(f"{what} failed: {ERRORS.get(code, code)} ({code})")
+        self.code = code
+
+
+class CacheDesc(ctypes.Structure):
+    """Mirror of ``kv1b_cache_t``."""
+    _fields_ = [
+        ("batch", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+        ("capacity", ctypes.c_int32), ("rotation_seed", ctypes.c_uint64),
+        ("k_bits", ctypes.c_void_p), ("k_norm", ctypes.c_void_p), ("k_cinv", ctypes.c_void_p),
+        ("v_codes", ctypes.c_void_p), ("v_sm", ctypes.c_void_p), ("signs", ctypes.c_void_p),
+        ("d_lengths", ctypes.c_void_p), ("d_status", ctypes.c_void_p),
+        ("h_lengths", ctypes.c_int64 * MAX_BATCH),
+    ]
+
+
+_lib = None
+
+
+def lib() -> ctypes.CDLL:
+    """Load the CUDA library; raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: run `python -m long_context_decode_kv1b_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+        D = ctypes.POINTER(CacheDesc)
+        sig = {
+            "kv1b_cache_bytes": (sz, [i32, i32, i32, i32]),
+            "kv1b_cache_init": (ctypes.c_int, [D, P, sz, i32, i32, i32, i32, ctypes.c_uint64, P]),
+            "kv1b_encode_append": (ctypes.c_int, [D, P, P, i32, i32, i64, i64, i64, P]),
+            "kv1b_attend_workspace_bytes": (sz, [D, i32, i32]),
+            "kv1b_attend": (ctypes.c_int, [D, P, i32, i32, f32, P, P, sz, i32, i32, P]),
+            "kv1b_attend_topp": (ctypes.c_int, [D, P, i32, i32, f32, f32, P, P, P, P, sz, P]),
+            "kv1b_query_prep": (ctypes.c_int, [D, P, i32, i32, P, P, P, P, P]),
+            "kv1b_scores": (ctypes.c_int, [D, P, i32, i32, f32, P, P, P, P]),
+            "kv1b_read_status": (ctypes.c_int, [D, P, P]),
+            "kv1b_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+            "kv1b_version": (ctypes.c_int, []),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _check(code: int, what: str):
+    if code != 0:
+        raise Kv1bError(code, what)
+
+
+def _dtype_code(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return DTYPE_F32
+    if t.dtype == torch.bfloat16:
+        return DTYPE_BF16
+    if t.dtype == torch.float16:
+        return DTYPE_F16
+    raise TypeError(f"unsupported dtype {t.dtype}")
+
+
+def _stream(stream=None) -> ctypes.c_void_p:
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+class Cache:
+    """A compressed KV cache for `batch` sequences x `num_kv_heads` heads, in one device buffer."""
+
+    def __init__(self, batch: int, num_kv_heads: int, capacity: int, seed: int = 0, device="cuda",
+                 stream=None):
+        L = lib()
+        self.batch, self.num_kv_heads, self.capacity, self.seed = batch, num_kv_heads, capacity, seed
+        self.device = torch.device(device)
+        nbytes = L.kv1b_cache_bytes(batch, num_kv_heads, HEAD_DIM, capacity)
+        if nbytes == 0:
+            raise Kv1bError(-1, "kv1b_cache_bytes")
+        self.nbytes = nbytes
+        self.buffer = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
+        self.desc = CacheDesc()
+        _check(L.kv1b_cache_init(ctypes.byref(self.desc), _ptr(self.buffer), nbytes, batch, num_kv_heads, HEAD_DIM,
+                                 capacity, seed, _stream(stream)), "kv1b_cache_init")
+        self._ws = {}
+
+    # ---- views of the device planes (for tests / inspection; layout in include/kv1b.h)
+    def _view(self, addr, dtype, shape):
+        off = addr - self.buffer.data_ptr()
+        n = 1
+        for s in shape:
+            n *= s
+        esz = torch.empty((), dtype=dtype).element_size()
+        return self.buffer[off:off + n * esz].view(dtype).view(*shape)
+
+    def planes(self) -> dict:
+        B, H, C = self.batch, self.num_kv_heads, self.capacity
+        d = self.desc
+        return {
+            "k_bits": self._view(d.k_bits, torch.int32, (B, H, C, 4)),
+            "k_norm": self._view(d.k_norm, torch.float32, (B, H, C)),
+            "k_cinv": self._view(d.k_cinv, torch.float32, (B, H, C)),
+            "v_codes": self._view(d.v_codes, torch.int32, (B, H, C // 16, 8, 32)),
+            "v_sm": self._view(d.v_sm, torch.int32, (B, H, C, 4)),
+            "signs": self._view(d.signs, torch.float32, (HEAD_DIM,)),
+            "lengths": self._view(d.d_lengths, torch.int32, (B,)),
+        }
+
+    @property
+    def lengths(self):
+        return [int(self.desc.h_lengths[b]) for b in range(self.batch)]
+
+    def append(self, k: torch.Tensor, v: torch.Tensor, stream=None):
+        """k, v: [batch, n_new, num_kv_heads, 128] (channel stride 1), same dtype and strides."""
+        if k.shape != v.shape or k.stride() != v.stride() or k.dtype != v.dtype:
+            raise ValueError("k and v must have equal shapes, strides and dtypes")
+        B, n, H, D = k.shape
+        if (B, H, D) != (self.batch, self.num_kv_heads, HEAD_DIM) or k.stride(3) != 1:
+            raise ValueError("expected [batch, n_new, num_kv_heads, 128] with unit channel stride")
+        _check(lib().kv1b_encode_append(ctypes.byref(self.desc), _ptr(k), _ptr(v), _dtype_code(k), n, k.stride(0),
+                                        k.stride(1), k.stride(2), _stream(stream)), "kv1b_encode_append")
+
+    def workspace(self, num_q_heads: int, mode: int) -> torch.Tensor:
+        key = (num_q_heads, mode)
+        if key not in self._ws:
+            n = lib().kv1b_attend_workspace_bytes(ctypes.byref(self.desc), num_q_heads, mode)
+            if n == 0:
+                raise Kv1bError(-1, "kv1b_attend_workspace_bytes")
+            self._ws[key] = torch.empty(n, dtype=torch.uint8, device=self.device)
+        return self._ws[key]
+
+    def attend(self, q: torch.Tensor, scale: float, out: torch.Tensor | None = None, engine: int = ATTEND_TENSOR,
+               num_splits: int = 0, stream=None) -> torch.Tensor:
+        """q: [batch, num_q_heads, 128] contiguous.  Returns fp32 [batch, num_q_heads, 128]."""
+        B, Hq, D = q.shape
+        if not q.is_contiguous():
+            raise ValueError("q must be contiguous")
+        if out is None:
+            out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+        ws = self.workspace(Hq, 0)
+        _check(lib().kv1b_attend(ctypes.byref(self.desc), _ptr(q), _dtype_code(q), Hq, float(scale), _ptr(out),
+                                 _ptr(ws), ws.numel(), engine, num_splits, _stream(stream)), "kv1b_attend")
+        return out
+
+    def attend_topp(self, q: torch.Tensor, scale: float, p: float, stream=None):
+        """Returns (out fp32 [B, Hq, 128], sel_idx int32 [B, Hq, capacity], sel_cnt int32 [B, Hq])."""
+        B, Hq, D = q.shape
+        out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+        sel = torch.empty((B, Hq, self.capacity), dtype=torch.int32, device=q.device)
+        cnt = torch.empty((B, Hq), dtype=torch.int32, device=q.device)
+        ws = self.workspace(Hq, 1)
+        _check(lib().kv1b_attend_topp(ctypes.byref(self.desc), _ptr(q), _dtype_code(q), Hq, float(scale), float(p),
+                                      _ptr(out), _ptr(sel), _ptr(cnt), _ptr(ws), ws.numel(), _stream(stream)),
+               "kv1b_attend_topp")
+        return out, sel, cnt
+
+    def query_prep(self, q: torch.Tensor, stream=None) -> dict:
+        B, Hq, _ = q.shape
+        planes = torch.empty((B, Hq, 4, 4), dtype=torch.int32, device=q.device)
+        vl = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        dl = torch.empty((B, Hq), dtype=torch.float32, device=q.device)
+        sq = torch.empty((B, Hq), dtype=torch.int32, device=q.device)
+        _check(lib().kv1b_query_prep(ctypes.byref(self.desc), _ptr(q), _dtype_code(q), Hq, _ptr(planes), _ptr(vl),
+                                     _ptr(dl), _ptr(sq), _stream(stream)), "kv1b_query_prep")
+        return {"planes": planes, "vl": vl, "delta": dl, "Sq": sq}
+
+    def scores(self, q: torch.Tensor, scale: float, stream=None) -> dict:
+        B, Hq, _ = q.shape
+        shape = (B, Hq, self.capacity)
+        A = torch.zeros(shape, dtype=torch.int32, device=q.device)
+        Bc = torch.zeros(shape, dtype=torch.int32, device=q.device)
+        s = torch.zeros(shape, dtype=torch.float32, device=q.device)
+        _check(lib().kv1b_scores(ctypes.byref(self.desc), _ptr(q), _dtype_code(q), Hq, float(scale), _ptr(A), _ptr(Bc),
+                                 _ptr(s), _stream(stream)), "kv1b_scores")
+        return {"A": A, "Bc": Bc, "s": s}
+
+    def status(self, stream=None) -> int:
+        flags = ctypes.c_int32(0)
+        _check(lib().kv1b_read_status(ctypes.byref(self.desc), ctypes.byref(flags), _stream(stream)),
+               "kv1b_read_status")
+        return flags.value
+
+
+def attend_from_host(cache: Cache, q_host: torch.Tensor, k_new_host: torch.Tensor | None, v_new_host: torch.Tensor | None,
+                     scale: float, out_host: torch.Tensor, q_dev: torch.Tensor, k_dev: torch.Tensor | None,
+                     v_dev: torch.Tensor | None, stream=None) -> torch.Tensor:
+    """One decode step with HOST buffers: copy the new token's K/V and the query from pinned host
+    memory to the device, append, attend, copy the output back (all on one stream)."""
+    s = stream if stream is not None else torch.cuda.current_stream()
+    with torch.cuda.stream(s):
+        if k_new_host is not None:
+            k_dev.copy_(k_new_host, non_blocking=True)
+            v_dev.copy_(v_new_host, non_blocking=True)
+            cache.append(k_dev, v_dev, stream=s)
+        q_dev.copy_(q_host, non_blocking=True)
+        out = cache.attend(q_dev, scale, stream=s)
+        out_host.copy_(out, non_blocking=True)
+    return out_host
+
+
+def unpack_codes(v_codes: torch.Tensor, length: int) -> torch.Tensor:
+    """Logical codes [length, 128] (uint8) of one (sequence, kv-head) from the tiled v_codes plane
+    [capacity/16, 8, 32] (layout in include/kv1b.h)."""
+    w = v_codes.to(torch.int64) & 0xFFFFFFFF
+    ntile = (length + 15) // 16
+    w = w[:ntile]
+    out = torch.zeros((ntile * 16, HEAD_DIM), dtype=torch.uint8, device=w.device)
+    lanes = torch.arange(32, device=w.device)
+    g, t = lanes // 4, lanes % 4
+    slots = [(0, 0, 0), (16, 0, 1), (4, 8, 0), (20, 8, 1), (8, 0, 8), (24, 0, 9), (12, 8, 8), (28, 8, 9)]
+    tiles = torch.arange(ntile, device=w.device)
+    for mt in range(8):
+        for shift, choff, toff in slots:
+            nib = ((w[:, mt, :] >> shift) & 0xF).to(torch.uint8)             # [ntile, 32]
+            tok = tiles[:, None] * 16 + (2 * t)[None, :] + toff                 # [ntile, 32]
+            ch = (16 * mt + g + choff)[None, :].expand_as(tok)
+            out[tok.reshape(-1), ch.reshape(-1)] = nib.reshape(-1)
+    return out[:length]

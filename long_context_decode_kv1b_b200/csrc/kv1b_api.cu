@@ -1,0 +1,302 @@
+// kv1b_api.cu -- the extern "C" entry points declared in include/kv1b.h: argument validation on
+// the host, then kernel launches on the caller's stream.  Nothing here allocates device memory.
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <string.h>
+
+#include "kv1b.h"
+#include "kv1b_launch.h"
+
+namespace {
+
+constexpr size_t kAlign = 256;
+constexpr int kMinForcedSplits = 64;
+
+size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct Layout {
+  size_t k_bits, k_norm, k_cinv, v_codes, v_sm, signs, lengths, status, total;
+};
+
+bool shape_ok(int32_t batch, int32_t hkv, int32_t head_dim, int32_t capacity) {
+  return batch >= 1 && batch <= KV1B_MAX_BATCH && hkv >= 1 && head_dim == KV1B_HEAD_DIM && capacity >= 1 &&
+         capacity % KV1B_CAPACITY_ALIGN == 0;
+}
+
+Layout layout(int32_t batch, int32_t hkv, int32_t capacity) {
+  const size_t tok = static_cast<size_t>(batch) * hkv * capacity;
+  Layout l;
+  size_t off = 0;
+  l.k_bits = off;  off += align_up(tok * 16);
+  l.k_norm = off;  off += align_up(tok * 4);
+  l.k_cinv = off;  off += align_up(tok * 4);
+  l.v_codes = off; off += align_up(tok * 64);
+  l.v_sm = off;    off += align_up(tok * 16);
+  l.signs = off;   off += align_up(KV1B_HEAD_DIM * 4);
+  l.lengths = off; off += align_up(KV1B_MAX_BATCH * 4);
+  l.status = off;  off += align_up(4);
+  l.total = off;
+  return l;
+}
+
+bool aligned(const void* ptr, size_t a) { return (reinterpret_cast<uintptr_t>(ptr) % a) == 0; }
+
+int num_sms() {
+  static int cached[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (cached[dev] == 0) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+kv1b::CacheView view(const kv1b_cache_t* c) {
+  kv1b::CacheView v;
+  v.k_bits = c->k_bits;
+  v.k_norm = c->k_norm;
+  v.k_cinv = c->k_cinv;
+  v.v_codes = c->v_codes;
+  v.v_sm = c->v_sm;
+  v.signs = c->signs;
+  v.B = c->batch;
+  v.Hkv = c->num_kv_heads;
+  v.cap = c->capacity;
+  return v;
+}
+
+bool cache_ok(const kv1b_cache_t* c) {
+  return c && shape_ok(c->batch, c->num_kv_heads, c->head_dim, c->capacity) && c->k_bits && c->v_codes &&
+         c->signs && c->d_lengths && c->d_status;
+}
+
+bool dtype_ok(int32_t dt) { return dt == KV1B_DTYPE_F32 || dt == KV1B_DTYPE_BF16 || dt == KV1B_DTYPE_F16; }
+
+int64_t max_length(const kv1b_cache_t* c) {
+  int64_t m = 0;
+  for (int b = 0; b < c->batch; ++b) m = c->h_lengths[b] > m ? c->h_lengths[b] : m;
+  return m;
+}
+
+int heads_check(const kv1b_cache_t* c, int32_t num_q_heads) {
+  if (num_q_heads < 1 || num_q_heads % c->num_kv_heads != 0) return KV1B_ERR_INVALID_ARG;
+  if (num_q_heads / c->num_kv_heads > KV1B_MAX_GROUP) return KV1B_ERR_UNSUPPORTED;
+  return KV1B_OK;
+}
+
+int32_t max_splits(const kv1b_cache_t* c) {
+  const int auto_max = kv1b_pick_splits(c->batch, c->num_kv_heads, c->capacity, num_sms());
+  return auto_max > kMinForcedSplits ? auto_max : kMinForcedSplits;
+}
+
+int cuda_status(cudaError_t e) { return e == cudaSuccess ? KV1B_OK : KV1B_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t kv1b_cache_bytes(int32_t batch, int32_t num_kv_heads, int32_t head_dim, int32_t capacity) {
+  if (!shape_ok(batch, num_kv_heads, head_dim, capacity)) return 0;
+  return layout(batch, num_kv_heads, capacity).total;
+}
+
+int kv1b_cache_init(kv1b_cache_t* cache, void* dev_buf, size_t bytes, int32_t batch, int32_t num_kv_heads,
+                    int32_t head_dim, int32_t capacity, uint64_t seed, void* stream) {
+  if (!cache || !dev_buf) return KV1B_ERR_INVALID_ARG;
+  if (head_dim != KV1B_HEAD_DIM || batch > KV1B_MAX_BATCH) return KV1B_ERR_UNSUPPORTED;
+  if (!shape_ok(batch, num_kv_heads, head_dim, capacity)) return KV1B_ERR_INVALID_ARG;
+  if (!aligned(dev_buf, kAlign)) return KV1B_ERR_MISALIGNED;
+  const Layout l = layout(batch, num_kv_heads, capacity);
+  if (bytes < l.total) return KV1B_ERR_WORKSPACE;
+  uint8_t* base = static_cast<uint8_t*>(dev_buf);
+  kv1b_cache_t c;
+  memset(&c, 0, sizeof(c));
+  c.batch = batch;
+  c.num_kv_heads = num_kv_heads;
+  c.head_dim = head_dim;
+  c.capacity = capacity;
+  c.rotation_seed = seed;
+  c.k_bits = reinterpret_cast<uint32_t*>(base + l.k_bits);
+  c.k_norm = reinterpret_cast<float*>(base + l.k_norm);
+  c.k_cinv = reinterpret_cast<float*>(base + l.k_cinv);
+  c.v_codes = reinterpret_cast<uint32_t*>(base + l.v_codes);
+  c.v_sm = reinterpret_cast<uint32_t*>(base + l.v_sm);
+  c.signs = reinterpret_cast<float*>(base + l.signs);
+  c.d_lengths = reinterpret_cast<int32_t*>(base + l.lengths);
+  c.d_status = reinterpret_cast<int32_t*>(base + l.status);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(dev_buf, 0, l.total, s);
+  if (e != cudaSuccess) return KV1B_ERR_CUDA;
+  e = kv1b_launch_init(seed, c.signs, c.d_lengths, batch, c.d_status, s);
+  if (e != cudaSuccess) return KV1B_ERR_CUDA;
+  *cache = c;
+  return KV1B_OK;
+}
+
+int kv1b_encode_append(kv1b_cache_t* cache, const void* k, const void* v, int32_t dtype, int32_t n_new,
+                       int64_t stride_b, int64_t stride_t, int64_t stride_h, void* stream) {
+  if (!cache_ok(cache) || !k || !v || !dtype_ok(dtype) || n_new < 1) return KV1B_ERR_INVALID_ARG;
+  if (stride_b < 0 || stride_t < 0 || stride_h < 0) return KV1B_ERR_INVALID_ARG;
+  if (!aligned(k, 16) || !aligned(v, 16) || stride_b % 4 || stride_t % 4 || stride_h % 4) return KV1B_ERR_MISALIGNED;
+  for (int b = 0; b < cache->batch; ++b)
+    if (cache->h_lengths[b] + n_new > cache->capacity) return KV1B_ERR_CAPACITY;
+  kv1b::EncodeParams p;
+  memset(&p, 0, sizeof(p));
+  p.k = k;
+  p.v = v;
+  p.dtype = dtype;
+  p.n_new = n_new;
+  p.sb = stride_b;
+  p.st = stride_t;
+  p.sh = stride_h;
+  p.B = cache->batch;
+  p.Hkv = cache->num_kv_heads;
+  p.cap = cache->capacity;
+  p.k_bits = cache->k_bits;
+  p.k_norm = cache->k_norm;
+  p.k_cinv = cache->k_cinv;
+  p.v_codes = cache->v_codes;
+  p.v_sm = cache->v_sm;
+  p.signs = cache->signs;
+  p.lengths = cache->d_lengths;
+  p.status = cache->d_status;
+  int64_t max_tiles = 0;
+  for (int b = 0; b < cache->batch; ++b) {
+    p.L0[b] = cache->h_lengths[b];
+    const int64_t nt = (p.L0[b] + n_new - 1) / 16 - p.L0[b] / 16 + 1;
+    max_tiles = nt > max_tiles ? nt : max_tiles;
+  }
+  const cudaError_t e = kv1b_launch_encode(p, max_tiles, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return KV1B_ERR_CUDA;
+  for (int b = 0; b < cache->batch; ++b) cache->h_lengths[b] += n_new;
+  return KV1B_OK;
+}
+
+size_t kv1b_attend_workspace_bytes(const kv1b_cache_t* cache, int32_t num_q_heads, int32_t mode) {
+  if (!cache_ok(cache) || heads_check(cache, num_q_heads) != KV1B_OK) return 0;
+  const size_t rows = static_cast<size_t>(cache->batch) * num_q_heads;
+  if (mode == 0) return align_up(rows * static_cast<size_t>(max_splits(cache)) * kv1b::kPartStride * 4);
+  if (mode == 1) return align_up(rows * static_cast<size_t>(cache->capacity) * 4);
+  return 0;
+}
+
+int kv1b_attend(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,
+                float* out, void* ws, size_t ws_bytes, int32_t flags, int32_t num_splits, void* stream) {
+  if (!cache_ok(cache) || !q || !out || !ws || !dtype_ok(q_dtype)) return KV1B_ERR_INVALID_ARG;
+  const int hc = heads_check(cache, num_q_heads);
+  if (hc != KV1B_OK) return hc;
+  if (flags != KV1B_ATTEND_TENSOR && flags != KV1B_ATTEND_CUDA_CORE) return KV1B_ERR_INVALID_ARG;
+  if (num_splits < 0 || num_splits > max_splits(cache)) return KV1B_ERR_INVALID_ARG;
+  if (!(scale == scale)) return KV1B_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(ws, kAlign) || !aligned(out, 16)) return KV1B_ERR_MISALIGNED;
+  if (ws_bytes < kv1b_attend_workspace_bytes(cache, num_q_heads, 0)) return KV1B_ERR_WORKSPACE;
+  const int64_t maxlen = max_length(cache);
+  kv1b::AttendParams p;
+  memset(&p, 0, sizeof(p));
+  p.c = view(cache);
+  p.q = q;
+  p.q_dtype = q_dtype;
+  p.Hq = num_q_heads;
+  p.scale = scale;
+  p.nsplit = num_splits > 0 ? num_splits : kv1b_pick_splits(cache->batch, cache->num_kv_heads, maxlen, num_sms());
+  p.part = static_cast<float*>(ws);
+  p.out = out;
+  for (int b = 0; b < cache->batch; ++b) p.len[b] = static_cast<int32_t>(cache->h_lengths[b]);
+  const int G = num_q_heads / cache->num_kv_heads;
+  return cuda_status(kv1b_launch_attend(p, G, flags, static_cast<int32_t>(maxlen), static_cast<cudaStream_t>(stream)));
+}
+
+int kv1b_attend_topp(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,
+                     float p, float* out, int32_t* sel_idx, int32_t* sel_cnt, void* ws, size_t ws_bytes,
+                     void* stream) {
+  if (!cache_ok(cache) || !q || !out || !sel_idx || !sel_cnt || !ws || !dtype_ok(q_dtype)) return KV1B_ERR_INVALID_ARG;
+  const int hc = heads_check(cache, num_q_heads);
+  if (hc != KV1B_OK) return hc;
+  if (!(p > 0.0f && p <= 1.0f) || !(scale == scale)) return KV1B_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(ws, kAlign)) return KV1B_ERR_MISALIGNED;
+  if (ws_bytes < kv1b_attend_workspace_bytes(cache, num_q_heads, 1)) return KV1B_ERR_WORKSPACE;
+  const int G = num_q_heads / cache->num_kv_heads;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  kv1b::ScoresParams sp;
+  memset(&sp, 0, sizeof(sp));
+  sp.c = view(cache);
+  sp.q = q;
+  sp.q_dtype = q_dtype;
+  sp.Hq = num_q_heads;
+  sp.scale = scale;
+  sp.s = static_cast<float*>(ws);
+  for (int b = 0; b < cache->batch; ++b) sp.len[b] = static_cast<int32_t>(cache->h_lengths[b]);
+  cudaError_t e = kv1b_launch_scores(sp, G, static_cast<int32_t>(max_length(cache)), s);
+  if (e != cudaSuccess) return KV1B_ERR_CUDA;
+  kv1b::ToppParams tp;
+  memset(&tp, 0, sizeof(tp));
+  tp.c = view(cache);
+  tp.Hq = num_q_heads;
+  tp.p = p;
+  tp.s = static_cast<const float*>(ws);
+  tp.out = out;
+  tp.sel_idx = sel_idx;
+  tp.sel_cnt = sel_cnt;
+  memcpy(tp.len, sp.len, sizeof(tp.len));
+  return cuda_status(kv1b_launch_topp(tp, s));
+}
+
+int kv1b_query_prep(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, uint32_t* planes,
+                    float* vl, float* delta, int32_t* sq, void* stream) {
+  if (!cache_ok(cache) || !q || !planes || !vl || !delta || !sq || !dtype_ok(q_dtype)) return KV1B_ERR_INVALID_ARG;
+  const int hc = heads_check(cache, num_q_heads);
+  if (hc != KV1B_OK) return hc;
+  if (!aligned(q, 16)) return KV1B_ERR_MISALIGNED;
+  return cuda_status(kv1b_launch_query_prep(view(cache), q, q_dtype, num_q_heads, planes, vl, delta, sq,
+                                            static_cast<cudaStream_t>(stream)));
+}
+
+int kv1b_scores(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,
+                int32_t* A, int32_t* Bc, float* s, void* stream) {
+  if (!cache_ok(cache) || !q || !s || !dtype_ok(q_dtype)) return KV1B_ERR_INVALID_ARG;
+  const int hc = heads_check(cache, num_q_heads);
+  if (hc != KV1B_OK) return hc;
+  if (!aligned(q, 16)) return KV1B_ERR_MISALIGNED;
+  kv1b::ScoresParams sp;
+  memset(&sp, 0, sizeof(sp));
+  sp.c = view(cache);
+  sp.q = q;
+  sp.q_dtype = q_dtype;
+  sp.Hq = num_q_heads;
+  sp.scale = scale;
+  sp.A = A;
+  sp.Bc = Bc;
+  sp.s = s;
+  for (int b = 0; b < cache->batch; ++b) sp.len[b] = static_cast<int32_t>(cache->h_lengths[b]);
+  return cuda_status(kv1b_launch_scores(sp, num_q_heads / cache->num_kv_heads, static_cast<int32_t>(max_length(cache)),
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+int kv1b_read_status(const kv1b_cache_t* cache, int32_t* flags, void* stream) {
+  if (!cache_ok(cache) || !flags) return KV1B_ERR_INVALID_ARG;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t h = 0;
+  if (cudaMemcpyAsync(&h, cache->d_status, sizeof(h), cudaMemcpyDeviceToHost, s) != cudaSuccess) return KV1B_ERR_CUDA;
+  if (cudaStreamSynchronize(s) != cudaSuccess) return KV1B_ERR_CUDA;
+  *flags = h;
+  return KV1B_OK;
+}
+
+const char* kv1b_status_string(int code) {
+  switch (code) {
+    case KV1B_OK: return "ok";
+    case KV1B_ERR_INVALID_ARG: return "invalid argument";
+    case KV1B_ERR_UNSUPPORTED: return "unsupported shape (head_dim must be 128, G <= 8, batch <= 64)";
+    case KV1B_ERR_CAPACITY: return "append would exceed the cache capacity";
+    case KV1B_ERR_MISALIGNED: return "misaligned pointer or stride";
+    case KV1B_ERR_WORKSPACE: return "buffer or workspace too small";
+    case KV1B_ERR_CUDA: return "CUDA error";
+    default: return "unknown status";
+  }
+}
+
+int kv1b_version(void) { return 100; }
+
+}  // extern "C"

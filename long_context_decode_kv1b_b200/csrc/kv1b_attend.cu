@@ -1,0 +1,510 @@
+// kv1b_attend.cu -- split-K decode attention over the compressed cache, its merge, and the
+// query-preparation / proxy-score test hooks.
+//
+// Per (sequence b, kv-head, split) one CTA of 256 threads walks its token range in chunks of 256:
+//   phase S  (thread = token): binary x INT4 popcount scores of the G query heads of this kv-head
+//            ("RaBitQCache", abstract / key design), online-softmax update in log2 units, and the
+//            per-(token, group, head) weights p * scale written to shared memory;
+//   phase PV (warp = 16-channel m-tile): the probability-weighted sum of the 4-bit values
+//            ("H1B-KV", technical framework: weights from the sketch, then the 4-bit values),
+//            either on the tensor cores (mma.sync m16n8k16: codes are exact fp16 integers c - 8,
+//            weights split into fp16 hi + lo, fp32 accumulation) or on the CUDA cores (fp32 FMA).
+// The dequantised value is min + scale*code = mid + scale*(code - 8) with mid = min + 8 scale;
+// the mid term is accumulated per (head, group) in fp32 by phase S.
+#include "kv1b_device.cuh"
+#include "kv1b_launch.h"
+
+namespace kv1b {
+
+constexpr int kThreads = 256;  // = tokens per chunk
+constexpr int kNoExp = 1 << 20;
+constexpr float kLog2e = 0x1.715476p+0f;  // log2(e) rounded to fp32
+
+__device__ __forceinline__ void mma16816(float d[4], const uint32_t a[4], const uint32_t b0, const uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x2_trans(uint32_t& b0, uint32_t& b1, uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];" : "=r"(b0), "=r"(b1) : "r"(addr));
+}
+
+__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// One code word (see the v_codes layout) -> the m16n8k16 A fragment.  Rows g: exact fp16 (c - 8);
+// rows g + 8: exact fp16 16 (c - 8) (their nibbles sit 4 bits higher), undone in the epilogue.
+__device__ __forceinline__ void codes_to_afrag(uint32_t w, uint32_t a[4]) {
+  const uint32_t w8 = w >> 8;
+  a[0] = hsub2((w & 0x000F000Fu) | 0x64006400u, 0x64086408u);   // (1024 + c) - 1032
+  a[1] = hsub2((w & 0x00F000F0u) | 0x64006400u, 0x64806480u);   // (1024 + 16c) - 1152
+  a[2] = hsub2((w8 & 0x000F000Fu) | 0x64006400u, 0x64086408u);
+  a[3] = hsub2((w8 & 0x00F000F0u) | 0x64006400u, 0x64806480u);
+}
+
+__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
+  const uint32_t l = __half_as_ushort(__float2half_rn(lo));
+  const uint32_t h = __half_as_ushort(__float2half_rn(hi));
+  return l | (h << 16);
+}
+
+__device__ __forceinline__ float exp2_of_int(int e) { return __int_as_float((e + 127) << 23); }
+
+template <int G>
+__device__ __forceinline__ float select_head(const float (&v)[G], int h) {
+  float r = v[0];
+  #pragma unroll
+  for (int i = 1; i < G; ++i)
+    if (h == i) r = v[i];
+  return r;
+}
+
+__device__ __forceinline__ void tile_range(int L, int nsplit, int split, int64_t& tok_begin, int64_t& tok_end) {
+  const int64_t ntiles = (static_cast<int64_t>(L) + 15) / 16;
+  const int64_t t0 = ntiles * split / nsplit, t1 = ntiles * (split + 1) / nsplit;
+  tok_begin = 16 * t0;
+  tok_end = (16 * t1 < L) ? 16 * t1 : L;
+  if (tok_begin > tok_end) tok_begin = tok_end;
+}
+
+template <int G, bool TENSOR>
+__global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendParams p) {
+  constexpr int NT = (2 * G + 7) / 8;                       // n-tiles of 8 columns: (head, hi/lo)
+  constexpr int ROWH = TENSOR ? 8 * NT : 2 * G;             // halves (tensor) or 2*floats per row
+  extern __shared__ __align__(16) uint8_t smem_dyn[];       // [4 groups][256 tokens][row]
+  __shared__ __align__(16) uint32_t s_planes[G][4][4];
+  __shared__ float s_vl[G], s_dl[G];
+  __shared__ int s_sq[G];
+  __shared__ float s_red[kThreads / 32][G + 4];
+
+  const int b = blockIdx.z, kvh = blockIdx.y, split = blockIdx.x;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int L = p.len[b];
+  const CacheView& c = p.c;
+  int64_t tok_begin, tok_end;
+  tile_range(L, p.nsplit, split, tok_begin, tok_end);
+
+  // ---- prologue: query preparation of the G heads of this kv-head (warp h -> head h)
+  if (warp < G) {
+    const int hq = kvh * G + warp;
+    const QueryPrep qp = query_prep_warp(p.q, (static_cast<int64_t>(b) * p.Hq + hq) * kD, p.q_dtype, c.signs);
+    if (lane == 0) {
+      #pragma unroll
+      for (int j = 0; j < 4; ++j)
+        #pragma unroll
+        for (int w = 0; w < 4; ++w) s_planes[warp][j][w] = qp.planes[j][w];
+      s_vl[warp] = qp.vl;
+      s_dl[warp] = qp.delta;
+      s_sq[warp] = qp.sq;
+    }
+  }
+  __syncthreads();
+  uint32_t P[G][4][4];
+  float vl[G], dl[G];
+  int sq[G];
+  #pragma unroll
+  for (int h = 0; h < G; ++h) {
+    #pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint4 pw = *reinterpret_cast<const uint4*>(&s_planes[h][j][0]);
+      P[h][j][0] = pw.x; P[h][j][1] = pw.y; P[h][j][2] = pw.z; P[h][j][3] = pw.w;
+    }
+    vl[h] = s_vl[h];
+    dl[h] = s_dl[h];
+    sq[h] = s_sq[h];
+  }
+  const float qs = __fdiv_rn(p.scale, static_cast<float>(kD));
+
+  const int64_t head_tok = (static_cast<int64_t>(b) * c.Hkv + kvh) * c.cap;  // token-major base
+  const uint4* kb4 = reinterpret_cast<const uint4*>(c.k_bits) + head_tok;
+  const float* kn = c.k_norm + head_tok;
+  const float* kc = c.k_cinv + head_tok;
+  const uint4* sm4 = reinterpret_cast<const uint4*>(c.v_sm) + head_tok;
+  const uint32_t* vcw = c.v_codes + head_tok * 16;  // 16 words per token, tile-major
+
+  float m_run[G], l_acc[G], mid_acc[G][4];
+  #pragma unroll
+  for (int h = 0; h < G; ++h) {
+    m_run[h] = -INFINITY;
+    l_acc[h] = 0.0f;
+    #pragma unroll
+    for (int g = 0; g < 4; ++g) mid_acc[h][g] = 0.0f;
+  }
+  int E_run[4] = {kNoExp, kNoExp, kNoExp, kNoExp};
+  float D[NT][4];      // tensor engine accumulators
+  float acc[G][2];     // CUDA-core engine accumulators (2 channels per lane)
+  #pragma unroll
+  for (int n = 0; n < NT; ++n)
+    #pragma unroll
+    for (int i = 0; i < 4; ++i) D[n][i] = 0.0f;
+  #pragma unroll
+  for (int h = 0; h < G; ++h) acc[h][0] = acc[h][1] = 0.0f;
+
+  const int gw = warp >> 1;           // value group owned by this warp in phase PV
+  const int g8 = lane >> 2, t4 = lane & 3;
+  const uint32_t smem_base = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dyn));
+
+  for (int64_t c0 = tok_begin; c0 < tok_end; c0 += kThreads) {
+    // ================= phase S: thread = token
+    const int64_t tau = c0 + threadIdx.x;
+    const bool valid = tau < tok_end;
+    float s2[G], sc[4], mid[4];
+    if (valid) {
+      const uint4 kb = __ldg(kb4 + tau);
+      const float nc = __fmul_rn(__ldg(kn + tau), __ldg(kc + tau));
+      const uint4 smv = __ldg(sm4 + tau);
+      const uint32_t smw[4] = {smv.x, smv.y, smv.z, smv.w};
+      const int32_t Bc = popc_Bc(kb);
+      #pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const int32_t A = popc_A(kb, P[h]);
+        s2[h] = __fmul_rn(logit_from_ints(A, Bc, sq[h], vl[h], dl[h], nc, qs), kLog2e);
+      }
+      #pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        sc[g] = __half2float(__ushort_as_half(static_cast<unsigned short>(smw[g] & 0xffffu)));
+        const float mn = __half2float(__ushort_as_half(static_cast<unsigned short>(smw[g] >> 16)));
+        mid[g] = __fmaf_rn(8.0f, sc[g], mn);
+      }
+    } else {
+      #pragma unroll
+      for (int h = 0; h < G; ++h) s2[h] = -INFINITY;
+      #pragma unroll
+      for (int g = 0; g < 4; ++g) sc[g] = mid[g] = 0.0f;
+    }
+    // chunk maxima of the logits (per head) and of the scales (per group)
+    float red[G + 4];
+    #pragma unroll
+    for (int h = 0; h < G; ++h) red[h] = s2[h];
+    #pragma unroll
+    for (int g = 0; g < 4; ++g) red[G + g] = sc[g];
+    #pragma unroll
+    for (int m = 16; m >= 1; m >>= 1)
+      #pragma unroll
+      for (int i = 0; i < G + 4; ++i) red[i] = fmaxf(red[i], __shfl_xor_sync(kFull, red[i], m));
+    if (lane == 0)
+      #pragma unroll
+      for (int i = 0; i < G + 4; ++i) s_red[warp][i] = red[i];
+    __syncthreads();
+    #pragma unroll
+    for (int i = 0; i < G + 4; ++i) {
+      float v = s_red[0][i];
+      #pragma unroll
+      for (int w = 1; w < kThreads / 32; ++w) v = fmaxf(v, s_red[w][i]);
+      red[i] = v;
+    }
+    float alpha[G], pr[G];
+    #pragma unroll
+    for (int h = 0; h < G; ++h) {
+      const float m_new = fmaxf(m_run[h], red[h]);
+      alpha[h] = (m_new == -INFINITY) ? 1.0f : exp2f(m_run[h] - m_new);
+      pr[h] = (valid && m_new != -INFINITY) ? exp2f(s2[h] - m_new) : 0.0f;
+      m_run[h] = m_new;
+      l_acc[h] = __fmaf_rn(l_acc[h], alpha[h], pr[h]);
+      #pragma unroll
+      for (int g = 0; g < 4; ++g) mid_acc[h][g] = __fmaf_rn(pr[h], mid[g], __fmul_rn(mid_acc[h][g], alpha[h]));
+    }
+    // per-group power-of-two shift keeping every fp16 weight p*scale*2^E below 2^15
+    float beta[4], shift[4];
+    #pragma unroll
+    for (int g = 0; g < 4; ++g) {
+      int e_new = E_run[g];
+      if (red[G + g] > 0.0f) {
+        const int cand = 14 - ilogbf(red[G + g]);
+        e_new = cand < e_new ? cand : e_new;
+      }
+      beta[g] = (E_run[g] == kNoExp || e_new == E_run[g]) ? 1.0f : exp2_of_int(e_new - E_run[g]);
+      E_run[g] = e_new;
+      shift[g] = (e_new == kNoExp) ? 0.0f : exp2_of_int(e_new);
+    }
+    // weights of this token
+    if (TENSOR) {
+      #pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const float f = __fmul_rn(sc[g], shift[g]);
+        uint32_t row[4 * NT];
+        #pragma unroll
+        for (int h = 0; h < 4 * NT; ++h) {
+          if (h < G) {
+            const float w = __fmul_rn(pr[h], f);
+            const float hi = __half2float(__float2half_rn(w));
+            row[h] = pack_half2(hi, __fsub_rn(w, hi));
+          } else {
+            row[h] = 0u;
+          }
+        }
+        uint4* dst = reinterpret_cast<uint4*>(smem_dyn + ((g * kThreads + threadIdx.x) * ROWH) * 2);
+        #pragma unroll
+        for (int n = 0; n < NT; ++n) dst[n] = make_uint4(row[4 * n], row[4 * n + 1], row[4 * n + 2], row[4 * n + 3]);
+      }
+    } else {
+      #pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        float* dst = reinterpret_cast<float*>(smem_dyn) + (g * kThreads + threadIdx.x) * G;
+        #pragma unroll
+        for (int h = 0; h < G; ++h) dst[h] = __fmul_rn(pr[h], sc[g]);
+      }
+    }
+    __syncthreads();
+    // ================= phase PV: warp = m-tile (channels 16 warp .. 16 warp + 15)
+    const int nsteps = static_cast<int>((tok_end - c0 + 15) / 16) < 16 ? static_cast<int>((tok_end - c0 + 15) / 16) : 16;
+    const uint32_t* tilew = vcw + (c0 / 16) * 256 + warp * 32 + lane;
+    if (TENSOR) {
+      #pragma unroll
+      for (int n = 0; n < NT; ++n) {
+        const int head = 4 * n + t4;
+        const float f = (head < G ? select_head<G>(alpha, head) : 1.0f) * beta[gw];
+        #pragma unroll
+        for (int i = 0; i < 4; ++i) D[n][i] = __fmul_rn(D[n][i], f);
+      }
+      const uint32_t brow = smem_base + ((gw * kThreads + (lane & 15)) * ROWH) * 2;
+      #pragma unroll 4
+      for (int ks = 0; ks < nsteps; ++ks) {
+        uint32_t a[4];
+        codes_to_afrag(__ldg(tilew + ks * 256), a);
+        #pragma unroll
+        for (int n = 0; n < NT; ++n) {
+          uint32_t b0, b1;
+          ldsm_x2_trans(b0, b1, brow + (ks * 16 * ROWH + 8 * n) * 2);
+          mma16816(D[n], a, b0, b1);
+        }
+      }
+    } else {
+      #pragma unroll
+      for (int h = 0; h < G; ++h) {
+        acc[h][0] = __fmul_rn(acc[h][0], alpha[h]);
+        acc[h][1] = __fmul_rn(acc[h][1], alpha[h]);
+      }
+      const float* wbase = reinterpret_cast<const float*>(smem_dyn) + gw * kThreads * G;
+      #pragma unroll 2
+      for (int ks = 0; ks < nsteps; ++ks) {
+        const uint32_t w = __ldg(tilew + ks * 256);
+        // slot -> (channel row 0/1, token within the 16-token tile)
+        const int shifts[8] = {0, 16, 4, 20, 8, 24, 12, 28};
+        const int rowsel[8] = {0, 0, 1, 1, 0, 0, 1, 1};
+        const int toks[8] = {2 * t4, 2 * t4 + 1, 2 * t4, 2 * t4 + 1, 2 * t4 + 8, 2 * t4 + 9, 2 * t4 + 8, 2 * t4 + 9};
+        #pragma unroll
+        for (int i = 0; i < 8; ++i) {
+          const float cv = __int_as_float(0x4B000000 | ((w >> shifts[i]) & 0xFu)) - 8388616.0f;  // c - 8, exact
+          const float* wt = wbase + (ks * 16 + toks[i]) * G;
+          #pragma unroll
+          for (int h = 0; h < G; ++h) acc[h][rowsel[i]] = __fmaf_rn(wt[h], cv, acc[h][rowsel[i]]);
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  // ================= epilogue: CTA sums of l and of the mid terms, then this split's partial
+  __shared__ float s_sum[kThreads / 32][G * 5];
+  {
+    float v[G * 5];
+    #pragma unroll
+    for (int h = 0; h < G; ++h) {
+      v[h * 5] = l_acc[h];
+      #pragma unroll
+      for (int g = 0; g < 4; ++g) v[h * 5 + 1 + g] = mid_acc[h][g];
+    }
+    #pragma unroll
+    for (int m = 16; m >= 1; m >>= 1)
+      #pragma unroll
+      for (int i = 0; i < G * 5; ++i) v[i] += __shfl_xor_sync(kFull, v[i], m);
+    if (lane == 0)
+      #pragma unroll
+      for (int i = 0; i < G * 5; ++i) s_sum[warp][i] = v[i];
+  }
+  __syncthreads();
+  const int64_t part_row0 = (static_cast<int64_t>(b) * p.Hq + kvh * G) * p.nsplit + split;  // head 0
+  auto part_ptr = [&](int h) { return p.part + (part_row0 + static_cast<int64_t>(h) * p.nsplit) * kPartStride; };
+  auto total = [&](int i) {
+    float t = 0.0f;
+    #pragma unroll
+    for (int w = 0; w < kThreads / 32; ++w) t += s_sum[w][i];
+    return t;
+  };
+  if (threadIdx.x < G) {
+    const int h = threadIdx.x;
+    part_ptr(h)[0] = select_head<G>(m_run, h);
+    part_ptr(h)[1] = total(h * 5);
+  }
+  const int ch0 = 16 * warp + g8, ch1 = ch0 + 8;
+  const float unshift = (E_run[gw] == kNoExp) ? 0.0f : exp2_of_int(-E_run[gw]);
+  if (TENSOR) {
+    #pragma unroll
+    for (int n = 0; n < NT; ++n) {
+      const int head = 4 * n + t4;
+      if (head < G) {
+        const float midt = total(head * 5 + 1 + gw);
+        float* dst = part_ptr(head) + 2;
+        dst[ch0] = __fmaf_rn(__fadd_rn(D[n][0], D[n][1]), unshift, midt);
+        dst[ch1] = __fmaf_rn(__fadd_rn(D[n][2], D[n][3]), unshift * 0.0625f, midt);
+      }
+    }
+  } else {
+    #pragma unroll
+    for (int h = 0; h < G; ++h) {
+      #pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        acc[h][r] += __shfl_xor_sync(kFull, acc[h][r], 1);
+        acc[h][r] += __shfl_xor_sync(kFull, acc[h][r], 2);
+      }
+    }
+    if (t4 == 0) {
+      #pragma unroll
+      for (int h = 0; h < G; ++h) {
+        const float midt = total(h * 5 + 1 + gw);
+        float* dst = part_ptr(h) + 2;
+        dst[ch0] = __fadd_rn(acc[h][0], midt);
+        dst[ch1] = __fadd_rn(acc[h][1], midt);
+      }
+    }
+  }
+}
+
+// log-sum-exp merge of the split partials; one block of 128 threads (channels) per (b, hq).
+__global__ void __launch_bounds__(128) merge_kernel(const float* __restrict__ part, float* __restrict__ out,
+                                                    int nsplit) {
+  const int64_t row = blockIdx.x;  // b * Hq + hq
+  const float* pr = part + row * nsplit * kPartStride;
+  float M = -INFINITY;
+  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, pr[s * kPartStride]);
+  float den = 0.0f, num = 0.0f;
+  if (M != -INFINITY) {
+    for (int s = 0; s < nsplit; ++s) {
+      const float ms = pr[s * kPartStride];
+      if (ms == -INFINITY) continue;
+      const float w = exp2f(ms - M);
+      den = __fmaf_rn(w, pr[s * kPartStride + 1], den);
+      num = __fmaf_rn(w, pr[s * kPartStride + 2 + threadIdx.x], num);
+    }
+  }
+  out[row * kD + threadIdx.x] = den > 0.0f ? __fdiv_rn(num, den) : 0.0f;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Test hooks.
+__global__ void __launch_bounds__(32) query_prep_kernel(const CacheView c, const void* q, int q_dtype, int Hq,
+                                                        uint32_t* planes, float* vl, float* delta, int32_t* sq) {
+  const int64_t row = blockIdx.x;  // b * Hq + hq
+  const QueryPrep qp = query_prep_warp(q, row * kD, q_dtype, c.signs);
+  if (threadIdx.x < 16) planes[row * 16 + threadIdx.x] = qp.planes[threadIdx.x >> 2][threadIdx.x & 3];
+  if (threadIdx.x == 0) {
+    vl[row] = qp.vl;
+    delta[row] = qp.delta;
+    sq[row] = qp.sq;
+  }
+}
+
+// Scores of every token of every query head (grid: token blocks x kv-heads x sequences).
+__global__ void __launch_bounds__(256) scores_kernel(const ScoresParams p, int G) {
+  __shared__ __align__(16) uint32_t s_planes[KV1B_MAX_GROUP][4][4];
+  __shared__ float s_vl[KV1B_MAX_GROUP], s_dl[KV1B_MAX_GROUP];
+  __shared__ int s_sq[KV1B_MAX_GROUP];
+  const int b = blockIdx.z, kvh = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const CacheView& c = p.c;
+  if (warp < G) {
+    const QueryPrep qp =
+        query_prep_warp(p.q, (static_cast<int64_t>(b) * p.Hq + kvh * G + warp) * kD, p.q_dtype, c.signs);
+    if (lane == 0) {
+      for (int j = 0; j < 4; ++j)
+        for (int w = 0; w < 4; ++w) s_planes[warp][j][w] = qp.planes[j][w];
+      s_vl[warp] = qp.vl;
+      s_dl[warp] = qp.delta;
+      s_sq[warp] = qp.sq;
+    }
+  }
+  __syncthreads();
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * 256 + threadIdx.x;
+  if (t >= p.len[b]) return;
+  const int64_t head_tok = (static_cast<int64_t>(b) * c.Hkv + kvh) * c.cap;
+  const uint4 kb = __ldg(reinterpret_cast<const uint4*>(c.k_bits) + head_tok + t);
+  const float nc = __fmul_rn(__ldg(c.k_norm + head_tok + t), __ldg(c.k_cinv + head_tok + t));
+  const int32_t Bc = popc_Bc(kb);
+  const float qs = __fdiv_rn(p.scale, static_cast<float>(kD));
+  for (int h = 0; h < G; ++h) {
+    uint32_t P[4][4];
+    for (int j = 0; j < 4; ++j)
+      for (int w = 0; w < 4; ++w) P[j][w] = s_planes[h][j][w];
+    const int32_t A = popc_A(kb, P);
+    const int64_t o = (static_cast<int64_t>(b) * p.Hq + kvh * G + h) * c.cap + t;
+    if (p.A) p.A[o] = A;
+    if (p.Bc) p.Bc[o] = Bc;
+    p.s[o] = logit_from_ints(A, Bc, s_sq[h], s_vl[h], s_dl[h], nc, qs);
+  }
+}
+
+template <int G, bool TENSOR>
+static cudaError_t launch_attend_t(const AttendParams& p, cudaStream_t stream) {
+  constexpr int NT = (2 * G + 7) / 8;
+  const size_t smem = TENSOR ? static_cast<size_t>(4) * kThreads * 8 * NT * 2 : static_cast<size_t>(4) * kThreads * G * 4;
+  auto kern = attend_kernel<G, TENSOR>;
+  static bool configured = false;  // per template instance
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  dim3 grid(p.nsplit, p.c.Hkv, p.c.B);
+  kern<<<grid, kThreads, smem, stream>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace kv1b
+
+using namespace kv1b;
+
+int kv1b_pick_splits(int32_t B, int32_t Hkv, int64_t max_len, int num_sms) {
+  const int64_t units = static_cast<int64_t>(B) * Hkv;
+  int64_t ns = (2LL * num_sms) / (units > 0 ? units : 1);
+  const int64_t by_len = max_len / 512;
+  if (ns > by_len) ns = by_len;
+  if (ns < 1) ns = 1;
+  if (ns > 1024) ns = 1024;
+  return static_cast<int>(ns);
+}
+
+cudaError_t kv1b_launch_attend(const AttendParams& p, int32_t G, int32_t engine, int32_t max_len,
+                               cudaStream_t stream) {
+  (void)max_len;
+  cudaError_t e = cudaSuccess;
+  const bool tensor = engine == KV1B_ATTEND_TENSOR;
+#define KV1B_CASE(GG)                                                                     \
+  case GG:                                                                                \
+    e = tensor ? launch_attend_t<GG, true>(p, stream) : launch_attend_t<GG, false>(p, stream); \
+    break;
+  switch (G) {
+    KV1B_CASE(1)
+    KV1B_CASE(2)
+    KV1B_CASE(3)
+    KV1B_CASE(4)
+    KV1B_CASE(5)
+    KV1B_CASE(6)
+    KV1B_CASE(7)
+    KV1B_CASE(8)
+    default:
+      return cudaErrorInvalidValue;
+  }
+#undef KV1B_CASE
+  if (e != cudaSuccess) return e;
+  merge_kernel<<<p.c.B * p.Hq, 128, 0, stream>>>(p.part, p.out, p.nsplit);
+  return cudaGetLastError();
+}
+
+cudaError_t kv1b_launch_query_prep(const CacheView& c, const void* q, int32_t q_dtype, int32_t Hq, uint32_t* planes,
+                                   float* vl, float* delta, int32_t* sq, cudaStream_t stream) {
+  query_prep_kernel<<<c.B * Hq, 32, 0, stream>>>(c, q, q_dtype, Hq, planes, vl, delta, sq);
+  return cudaGetLastError();
+}
+
+cudaError_t kv1b_launch_scores(const ScoresParams& p, int32_t G, int32_t max_len, cudaStream_t stream) {
+  if (max_len <= 0) return cudaSuccess;
+  dim3 grid(static_cast<unsigned>((max_len + 255) / 256), p.c.Hkv, p.c.B);
+  scores_kernel<<<grid, 256, 0, stream>>>(p, G);
+  return cudaGetLastError();
+}

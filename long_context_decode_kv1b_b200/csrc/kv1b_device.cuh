@@ -1,0 +1,201 @@
+// kv1b_device.cuh -- device-side building blocks shared by the encode, attend and Top-p kernels.
+//
+// Warp convention used throughout: a warp owns one 128-channel vector; lane l holds channels
+// 4l .. 4l+3 in registers x[0..3].
+//
+// Every floating-point step that decides a stored bit, code or integer is written with explicit
+// round-to-nearest intrinsics (__fadd_rn, __fmul_rn, __fdiv_rn, __fsqrt_rn) so the compiler can
+// neither contract nor reorder it; the library is also compiled with --fmad=false.
+#pragma once
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kv1b.h"
+
+namespace kv1b {
+
+constexpr int kD = 128;
+constexpr unsigned kFull = 0xffffffffu;
+
+// ---------------------------------------------------------------------------------------------
+// Loads: 4 consecutive channels of an fp32 / bf16 / fp16 row as fp32 (exact conversions).
+__device__ __forceinline__ void load4(const void* base, int64_t elem_off, int dtype, float x[4]) {
+  if (dtype == KV1B_DTYPE_F32) {
+    const float4 v = __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(base) + elem_off));
+    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+  } else {
+    const uint2 u = __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(base) + elem_off));
+    const uint32_t h[4] = {u.x & 0xffffu, u.x >> 16, u.y & 0xffffu, u.y >> 16};
+    #pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      if (dtype == KV1B_DTYPE_BF16) x[r] = __uint_as_float(h[r] << 16);
+      else x[r] = __half2float(__ushort_as_half(static_cast<unsigned short>(h[r])));
+    }
+  }
+}
+
+// ---------------------------------------------------------------------------------------------
+// Random-sign Walsh-Hadamard rotation ("RaBitQCache": randomised rotation before binarisation).
+// y = H (D (.) x), H the unnormalised Hadamard matrix in natural (Sylvester) order, computed with
+// butterfly stages h = 1, 2, 4, ..., 64; each stage maps the pair (a at index i, c at i + h) to
+// (a + c, a - c).  Stages 1 and 2 are inside a lane, stages 4..64 pair lane l with lane l ^ (h/4).
+__device__ __forceinline__ void rotate128(float x[4], const float sgn[4]) {
+  #pragma unroll
+  for (int r = 0; r < 4; ++r) x[r] = (sgn[r] < 0.0f) ? -x[r] : x[r];
+  const float a0 = __fadd_rn(x[0], x[1]), a1 = __fsub_rn(x[0], x[1]);
+  const float a2 = __fadd_rn(x[2], x[3]), a3 = __fsub_rn(x[2], x[3]);
+  x[0] = __fadd_rn(a0, a2);
+  x[2] = __fsub_rn(a0, a2);
+  x[1] = __fadd_rn(a1, a3);
+  x[3] = __fsub_rn(a1, a3);
+  const int lane = threadIdx.x & 31;
+  #pragma unroll
+  for (int m = 1; m < 32; m <<= 1) {
+    const bool upper = (lane & m) != 0;
+    #pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float o = __shfl_xor_sync(kFull, x[r], m);
+      x[r] = upper ? __fsub_rn(o, x[r]) : __fadd_rn(x[r], o);
+    }
+  }
+}
+
+// Fixed pairwise tree over the 128 channels: for h = 64, 32, ..., 1: a[i] += a[i + h] (i < h).
+// Returns a[0] on every lane.
+__device__ __forceinline__ float tree_sum128(const float a_in[4]) {
+  float a[4] = {a_in[0], a_in[1], a_in[2], a_in[3]};
+  #pragma unroll
+  for (int off = 16; off >= 1; off >>= 1) {  // h = 64, 32, 16, 8, 4  <->  lane offsets 16..1
+    #pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const float o = __shfl_down_sync(kFull, a[r], off);
+      a[r] = __fadd_rn(a[r], o);
+    }
+  }
+  // lane 0 now holds a[0..3] after the h = 4 stage
+  a[0] = __fadd_rn(a[0], a[2]);  // h = 2
+  a[1] = __fadd_rn(a[1], a[3]);
+  a[0] = __fadd_rn(a[0], a[1]);  // h = 1
+  return __shfl_sync(kFull, a[0], 0);
+}
+
+// Pack one bit per channel: bit i of word w = bit of channel 32w + i ("H1IB-KV" bitmap order).
+// nib = this lane's 4 bits (bit r = channel 4l + r).  Returns word (lane >> 3) on every lane.
+__device__ __forceinline__ uint32_t pack_word(uint32_t nib) {
+  const int lane = threadIdx.x & 31;
+  uint32_t v = nib << (4 * (lane & 7));
+  v |= __shfl_xor_sync(kFull, v, 1);
+  v |= __shfl_xor_sync(kFull, v, 2);
+  v |= __shfl_xor_sync(kFull, v, 4);
+  return v;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Query preparation for one head (one warp): rotate, quantise to 4 bits between min and max,
+// and build the 4 bit-planes ("RaBitQCache": binary x INT4 arithmetic).
+struct QueryPrep {
+  uint32_t planes[4][4];  // [plane j][word w], valid on every lane
+  float vl, delta;
+  int32_t sq;
+};
+
+__device__ __forceinline__ QueryPrep query_prep_warp(const void* q, int64_t row_off, int dtype, const float* signs) {
+  const int lane = threadIdx.x & 31;
+  float x[4], sg[4];
+  load4(q, row_off + 4 * lane, dtype, x);
+  #pragma unroll
+  for (int r = 0; r < 4; ++r) sg[r] = signs[4 * lane + r];
+  rotate128(x, sg);
+  float lo = fminf(fminf(x[0], x[1]), fminf(x[2], x[3]));
+  float hi = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
+  #pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) {
+    lo = fminf(lo, __shfl_xor_sync(kFull, lo, m));
+    hi = fmaxf(hi, __shfl_xor_sync(kFull, hi, m));
+  }
+  const float dl = __fdiv_rn(__fsub_rn(hi, lo), 15.0f);
+  int code[4];
+  int csum = 0;
+  #pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    int c = 0;
+    if (dl > 0.0f) {
+      const float fl = floorf(__fadd_rn(__fdiv_rn(__fsub_rn(x[r], lo), dl), 0.5f));
+      c = !(fl > 0.0f) ? 0 : (fl >= 15.0f ? 15 : static_cast<int>(fl));
+    }
+    code[r] = c;
+    csum += c;
+  }
+  QueryPrep qp;
+  #pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    uint32_t nib = 0;
+    #pragma unroll
+    for (int r = 0; r < 4; ++r) nib |= static_cast<uint32_t>((code[r] >> j) & 1) << r;
+    const uint32_t word = pack_word(nib);
+    #pragma unroll
+    for (int w = 0; w < 4; ++w) qp.planes[j][w] = __shfl_sync(kFull, word, 8 * w);
+  }
+  qp.vl = lo;
+  qp.delta = dl;
+  qp.sq = __reduce_add_sync(kFull, csum);
+  return qp;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Proxy score of one (token, head): binary x INT4 popcounts, then the fp32 logit in the fixed
+// order  dot = fl(fl(delta * I2) + fl(vl * I1)),  s = fl(fl(dot * fl(N * cinv)) * qs),
+// I1 = 2 Bc - 128, I2 = 2 A - Sq, qs = scale / 128.
+__device__ __forceinline__ int32_t popc_A(const uint4 b, const uint32_t P[4][4]) {
+  int32_t A = 0;
+  #pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int32_t pj = __popc(b.x & P[j][0]) + __popc(b.y & P[j][1]) + __popc(b.z & P[j][2]) + __popc(b.w & P[j][3]);
+    A += pj << j;
+  }
+  return A;
+}
+
+__device__ __forceinline__ int32_t popc_Bc(const uint4 b) {
+  return __popc(b.x) + __popc(b.y) + __popc(b.z) + __popc(b.w);
+}
+
+__device__ __forceinline__ float logit_from_ints(int32_t A, int32_t Bc, int32_t sq, float vl, float delta, float nc,
+                                                 float qs) {
+  const int32_t I1 = 2 * Bc - kD;
+  const int32_t I2 = 2 * A - sq;
+  const float dot = __fadd_rn(__fmul_rn(delta, static_cast<float>(I2)), __fmul_rn(vl, static_cast<float>(I1)));
+  return __fmul_rn(__fmul_rn(dot, nc), qs);
+}
+
+// ---------------------------------------------------------------------------------------------
+// binary16 helpers for the value quantiser.
+__device__ __forceinline__ double half_bits_to_double(uint32_t hb) {
+  return static_cast<double>(__half2float(__ushort_as_half(static_cast<unsigned short>(hb))));
+}
+
+// Smallest non-negative finite binary16 h with 15*h >= D (15*h is exact in fp64); 0x7bff and
+// *sat on overflow.  Starts next to the answer and walks at most a few steps.
+__device__ __forceinline__ uint32_t half_scale_up(double D, int* sat) {
+  if (!(D > 0.0)) return 0u;
+  if (D > 15.0 * 65504.0) { *sat = 1; return 0x7bffu; }
+  uint32_t hb = __half_as_ushort(__float2half_rz(__double2float_rz(D / 15.0)));
+  if (hb > 0x7bffu) hb = 0x7bffu;
+  #pragma unroll 1
+  for (int i = 0; i < 8 && 15.0 * half_bits_to_double(hb) < D; ++i) ++hb;
+  #pragma unroll 1
+  for (int i = 0; i < 8 && hb > 0u && 15.0 * half_bits_to_double(hb - 1u) >= D; ++i) --hb;
+  return hb;
+}
+
+// Largest finite binary16 <= x (saturates at -65504 with *sat).
+__device__ __forceinline__ uint32_t half_round_down(float x, int* sat) {
+  uint32_t hb = __half_as_ushort(__float2half_rd(x));
+  if (hb == 0xfc00u) { *sat = 1; return 0xfbffu; }  // -inf: below the binary16 range
+  if (hb == 0x8000u) hb = 0u;                      // -0 -> +0
+  return hb;
+}
+
+}  // namespace kv1b

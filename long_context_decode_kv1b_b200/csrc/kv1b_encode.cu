@@ -1,0 +1,153 @@
+// kv1b_encode.cu -- cache initialisation and the encode/append kernel.
+//
+// Keys ("RaBitQCache", abstract / core idea: randomised rotation, then binary quantisation;
+// "H1B-KV", key design: a 1-bit sketch by random projection): y = H (D (.) k), one sign bit per
+// channel, N = ||k|| and 1/C = 128 N / sum|y_i| for RaBitQ's unbiased estimator.
+// Values ("H1B-KV", key design: 4-bit linear quantisation): groups of 32 channels, fp16 min
+// rounded down, fp16 scale the smallest with 15 scale >= range, codes = round-half-up.
+#include "kv1b_device.cuh"
+#include "kv1b_launch.h"
+
+namespace kv1b {
+
+// SplitMix64 (Steele, Lea & Flood, OOPSLA 2014) draws the rotation signs: D_i = -1 iff the top bit
+// of the i-th output is set.  One thread; runs once per cache.
+__global__ void init_kernel(uint64_t seed, float* signs, int32_t* lengths, int32_t batch, int32_t* status) {
+  if (threadIdx.x == 0 && blockIdx.x == 0) {
+    uint64_t st = seed;
+    for (int i = 0; i < kD; ++i) {
+      st += 0x9E3779B97F4A7C15ull;
+      uint64_t z = st;
+      z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+      z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+      z ^= (z >> 31);
+      signs[i] = (z >> 63) ? -1.0f : 1.0f;
+    }
+    *status = 0;
+  }
+  if (blockIdx.x == 0 && threadIdx.x < batch) lengths[threadIdx.x] = 0;
+}
+
+// One block per (16-token tile touched by the append, kv-head, sequence); warp r handles tile
+// slot r.  Keys and v_sm are token-major and written directly; the 4-bit codes of the tile are
+// staged in shared memory and then written as whole 32-bit words in the mma A-fragment order
+// (read-modify-write keeps the nibbles of tokens already in the tile).
+__global__ void __launch_bounds__(512) encode_kernel(const EncodeParams p) {
+  __shared__ uint8_t codes[16][kD];
+  __shared__ int s_new[16];
+  const int b = blockIdx.z, h = blockIdx.y;
+  const int64_t L0 = p.L0[b];
+  const int64_t first_tile = L0 / 16, last_tile = (L0 + p.n_new - 1) / 16;
+  const int64_t tile = first_tile + blockIdx.x;
+  if (tile > last_tile) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t pos = tile * 16 + warp;
+  const bool is_new = pos >= L0 && pos < L0 + p.n_new;
+  if (lane == 0) s_new[warp] = is_new;
+  const int64_t head_base = (static_cast<int64_t>(b) * p.Hkv + h) * p.cap;  // token index base
+
+  if (is_new) {
+    const int64_t t = pos - L0;
+    const int64_t row = static_cast<int64_t>(b) * p.sb + t * p.st + static_cast<int64_t>(h) * p.sh;
+    int flags = 0;
+    // ---- key sketch
+    float x[4], sg[4], sq[4], y[4], ab[4];
+    load4(p.k, row + 4 * lane, p.dtype, x);
+    #pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      sg[r] = p.signs[4 * lane + r];
+      sq[r] = __fmul_rn(x[r], x[r]);
+      if (!isfinite(x[r])) flags |= KV1B_STATUS_NONFINITE;
+      y[r] = x[r];
+    }
+    const float nrm = __fsqrt_rn(tree_sum128(sq));
+    rotate128(y, sg);
+    uint32_t nib = 0;
+    #pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      nib |= static_cast<uint32_t>(y[r] >= 0.0f) << r;
+      ab[r] = fabsf(y[r]);
+    }
+    const uint32_t word = pack_word(nib);
+    const float sabs = tree_sum128(ab);
+    const float cinv = (sabs > 0.0f) ? __fdiv_rn(__fmul_rn(static_cast<float>(kD), nrm), sabs) : 1.0f;
+    if ((lane & 7) == 0) p.k_bits[(head_base + pos) * 4 + (lane >> 3)] = word;
+    if (lane == 0) {
+      p.k_norm[head_base + pos] = nrm;
+      p.k_cinv[head_base + pos] = cinv;
+    }
+    // ---- value codes
+    float v[4];
+    load4(p.v, row + 4 * lane, p.dtype, v);
+    float mn = fminf(fminf(v[0], v[1]), fminf(v[2], v[3]));
+    float mx = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
+    #pragma unroll
+    for (int m = 1; m <= 4; m <<= 1) {  // reduce over the 8 lanes of this 32-channel group
+      mn = fminf(mn, __shfl_xor_sync(kFull, mn, m));
+      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
+    }
+    int sat = 0;
+    #pragma unroll
+    for (int r = 0; r < 4; ++r)
+      if (!isfinite(v[r])) flags |= KV1B_STATUS_NONFINITE;
+    const uint32_t min_bits = half_round_down(mn, &sat);
+    const double range = static_cast<double>(mx) - half_bits_to_double(min_bits);
+    const uint32_t scale_bits = half_scale_up(range, &sat);
+    if (sat) flags |= KV1B_STATUS_FP16_SATURATED;
+    const float sf = __half2float(__ushort_as_half(static_cast<unsigned short>(scale_bits)));
+    const float mf = __half2float(__ushort_as_half(static_cast<unsigned short>(min_bits)));
+    #pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      int c = 0;
+      if (sf > 0.0f) {
+        const float fl = floorf(__fadd_rn(__fdiv_rn(__fsub_rn(v[r], mf), sf), 0.5f));
+        c = !(fl > 0.0f) ? 0 : (fl >= 15.0f ? 15 : static_cast<int>(fl));
+      }
+      codes[warp][4 * lane + r] = static_cast<uint8_t>(c);
+    }
+    if ((lane & 7) == 0) p.v_sm[(head_base + pos) * 4 + (lane >> 3)] = scale_bits | (min_bits << 16);
+    flags = static_cast<int>(__reduce_or_sync(kFull, static_cast<unsigned>(flags)));
+    if (lane == 0 && flags) atomicOr(p.status, flags);
+  }
+  __syncthreads();
+  // ---- assemble the tile's code words: thread = (m-tile, lane) of the A fragment
+  if (threadIdx.x < 256) {
+    const int mt = threadIdx.x >> 5, l = threadIdx.x & 31;
+    const int g = l >> 2, t = l & 3;
+    // slot order: bits 0,16,4,20,8,24,12,28  <->  (channel offset, token) pairs
+    const int ch_off[8] = {0, 0, 8, 8, 0, 0, 8, 8};
+    const int tok[8] = {2 * t, 2 * t + 1, 2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9, 2 * t + 8, 2 * t + 9};
+    const int shift[8] = {0, 16, 4, 20, 8, 24, 12, 28};
+    uint32_t* dst = p.v_codes + ((static_cast<int64_t>(b) * p.Hkv + h) * (p.cap / 16) + tile) * 256 + mt * 32 + l;
+    bool all_new = true;
+    #pragma unroll
+    for (int i = 0; i < 8; ++i) all_new = all_new && s_new[tok[i]];
+    uint32_t w = all_new ? 0u : *dst;
+    #pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      if (s_new[tok[i]]) {
+        const uint32_t c = codes[tok[i]][16 * mt + g + ch_off[i]];
+        w = (w & ~(0xfu << shift[i])) | (c << shift[i]);
+      }
+    }
+    *dst = w;
+  }
+  if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x < p.B)
+    p.lengths[threadIdx.x] = static_cast<int32_t>(p.L0[threadIdx.x] + p.n_new);
+}
+
+}  // namespace kv1b
+
+using namespace kv1b;
+
+cudaError_t kv1b_launch_init(uint64_t seed, float* signs, int32_t* lengths, int32_t batch, int32_t* status,
+                             cudaStream_t stream) {
+  init_kernel<<<1, 64, 0, stream>>>(seed, signs, lengths, batch, status);
+  return cudaGetLastError();
+}
+
+cudaError_t kv1b_launch_encode(const EncodeParams& p, int64_t max_tiles, cudaStream_t stream) {
+  dim3 grid(static_cast<unsigned>(max_tiles), p.Hkv, p.B);
+  encode_kernel<<<grid, 512, 0, stream>>>(p);
+  return cudaGetLastError();
+}

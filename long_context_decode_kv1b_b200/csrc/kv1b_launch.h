@@ -1,0 +1,86 @@
+// kv1b_launch.h -- internal host<->device interface: kernel parameter blocks and launchers.
+#pragma once
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kv1b.h"
+
+namespace kv1b {
+
+struct EncodeParams {
+  const void* k;
+  const void* v;
+  int32_t dtype;
+  int32_t n_new;
+  int64_t sb, st, sh;  // element strides of K/V: sequence, token, kv-head
+  int32_t B, Hkv, cap;
+  uint32_t* k_bits;
+  float* k_norm;
+  float* k_cinv;
+  uint32_t* v_codes;
+  uint32_t* v_sm;
+  const float* signs;
+  int32_t* lengths;
+  int32_t* status;
+  int64_t L0[KV1B_MAX_BATCH];  // write position per sequence (host mirror before the append)
+};
+
+struct CacheView {
+  const uint32_t* k_bits;
+  const float* k_norm;
+  const float* k_cinv;
+  const uint32_t* v_codes;
+  const uint32_t* v_sm;
+  const float* signs;
+  int32_t B, Hkv, cap;
+};
+
+struct AttendParams {
+  CacheView c;
+  const void* q;
+  int32_t q_dtype;
+  int32_t Hq;
+  float scale;
+  int32_t nsplit;
+  float* part;   // [B][Hq][nsplit][2 + 128]: m (log2 units), l, o[128]
+  float* out;    // [B][Hq][128]
+  int32_t len[KV1B_MAX_BATCH];
+};
+
+struct ScoresParams {
+  CacheView c;
+  const void* q;
+  int32_t q_dtype;
+  int32_t Hq;
+  float scale;
+  int32_t* A;    // optional [B][Hq][cap]
+  int32_t* Bc;   // optional [B][Hq][cap]
+  float* s;      // [B][Hq][cap]
+  int32_t len[KV1B_MAX_BATCH];
+};
+
+struct ToppParams {
+  CacheView c;
+  int32_t Hq;
+  float p;
+  const float* s;  // [B][Hq][cap] logits
+  float* out;
+  int32_t* sel_idx;
+  int32_t* sel_cnt;
+  int32_t len[KV1B_MAX_BATCH];
+};
+
+constexpr int kPartStride = 2 + 128;
+
+}  // namespace kv1b
+
+cudaError_t kv1b_launch_init(uint64_t seed, float* signs, int32_t* lengths, int32_t batch, int32_t* status,
+                             cudaStream_t stream);
+cudaError_t kv1b_launch_encode(const kv1b::EncodeParams& p, int64_t max_tiles, cudaStream_t stream);
+cudaError_t kv1b_launch_attend(const kv1b::AttendParams& p, int32_t G, int32_t engine, int32_t max_len,
+                               cudaStream_t stream);
+cudaError_t kv1b_launch_query_prep(const kv1b::CacheView& c, const void* q, int32_t q_dtype, int32_t Hq,
+                                   uint32_t* planes, float* vl, float* delta, int32_t* sq, cudaStream_t stream);
+cudaError_t kv1b_launch_scores(const kv1b::ScoresParams& p, int32_t G, int32_t max_len, cudaStream_t stream);
+cudaError_t kv1b_launch_topp(const kv1b::ToppParams& p, cudaStream_t stream);
+int kv1b_pick_splits(int32_t B, int32_t Hkv, int64_t max_len, int num_sms);

@@ -80,8 +80,8 @@ uint16_t half_round_down(double x, int* sat) {
 /* Smallest non-negative finite half h with 15*h >= D (15*h is exact in fp64); saturates. */
 uint16_t half_scale_up(double D, int* sat) {
   const auto& t = finite_halves();
-  std::size_t i = 0;
-  while (i < t.size() && t[i].first < 0.0) ++i;  // first non-negative (+0)
+  static const std::size_t i = static_cast<std::size_t>(
+      std::lower_bound(t.begin(), t.end(), std::make_pair(0.0, static_cast<uint16_t>(0))) - t.begin());  // +0
   if (15.0 * t.back().first < D) { *sat = 1; return t.back().second; }
   std::size_t lo = i, hi = t.size() - 1;  // answer in [lo, hi]
   while (lo < hi) {

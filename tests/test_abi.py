@@ -1,0 +1,63 @@
+"""CPU-only checks of the boundary: the C-ABI library loads and exports every symbol that
+include/kv1b.h declares; host-only size queries behave; the binding's struct mirrors the header.
+No kernel is launched here."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import long_context_decode_kv1b_b200 as kv
+from long_context_decode_kv1b_b200 import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "kv1b.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(kv1b_[a-z_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build.build()
+    return kv.lib()
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(lib, n), n
+    assert sorted(kv.SYMBOLS) == names
+
+
+def test_version_and_status_strings(lib):
+    assert lib.kv1b_version() == 100
+    assert lib.kv1b_status_string(0) == b"ok"
+    assert b"capacity" in lib.kv1b_status_string(-3)
+
+
+def test_cache_bytes_host_rules(lib):
+    n = lib.kv1b_cache_bytes(1, 8, 128, 1024)
+    # 104 bytes per token-kv-head plus small aligned extras
+    assert 104 * 8 * 1024 <= n <= 104 * 8 * 1024 + 4096
+    assert lib.kv1b_cache_bytes(1, 8, 64, 1024) == 0      # head_dim must be 128
+    assert lib.kv1b_cache_bytes(1, 8, 128, 1000) == 0     # capacity multiple of 128
+    assert lib.kv1b_cache_bytes(65, 8, 128, 1024) == 0    # batch <= 64
+
+
+def test_descriptor_layout_matches_header():
+    # int32 x4, u64, 8 pointers, int64[64]
+    assert ctypes.sizeof(kv.CacheDesc) == 16 + 8 + 8 * 8 + 8 * 64
+
+
+def test_init_rejects_bad_arguments_without_launching(lib):
+    d = kv.CacheDesc()
+    # null buffer / misaligned buffer / short buffer are refused on the host
+    assert lib.kv1b_cache_init(ctypes.byref(d), None, 0, 1, 1, 128, 128, 0, None) == -1
+    assert lib.kv1b_cache_init(ctypes.byref(d), ctypes.c_void_p(0x1001), 1 << 20, 1, 1, 128, 128, 0, None) == -4
+    assert lib.kv1b_cache_init(ctypes.byref(d), ctypes.c_void_p(0x10000), 16, 1, 1, 128, 128, 0, None) == -5
+    assert lib.kv1b_cache_init(ctypes.byref(d), ctypes.c_void_p(0x10000), 1 << 20, 1, 1, 96, 128, 0, None) == -2

@@ -1,0 +1,248 @@
+"""GPU parity: every step of the CUDA path, called through the C ABI, against the CPU oracle.
+
+Bit-exact: key bits, N, 1/C, value codes, fp16 scale/min, query planes and grid, popcount
+integers, logits, Top-p index sets.  Attention outputs: <= 1e-3 relative per row (max and l2).
+"""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import long_context_decode_kv1b_b200 as kv
+from parity_utils import HostKV, assert_planes_equal, assert_rows_close, gpu_head_planes, oracle_attend_all, to_np32
+
+pytestmark = pytest.mark.gpu
+DEV = "cuda"
+
+
+def rand_kv(g, B, n, H, dtype, scale=1.0):
+    K = (torch.randn((B, n, H, 128), generator=g, device=DEV) * scale).to(dtype)
+    V = (torch.randn((B, n, H, 128), generator=g, device=DEV) * scale).to(dtype)
+    return K, V
+
+
+def build_cache(B, Hkv, appends, dtype, seed=0, data_seed=1, vscale=1.0, cap=None):
+    total = sum(appends)
+    cap = cap or (total + 127) // 128 * 128
+    cache = kv.Cache(B, Hkv, cap, seed=seed)
+    host = HostKV(B, Hkv, cap)
+    g = torch.Generator(device=DEV).manual_seed(data_seed)
+    for n in appends:
+        K, V = rand_kv(g, B, n, Hkv, dtype)
+        V = (V.float() * vscale).to(dtype)
+        cache.append(K, V)
+        host.add(K, V)
+    return cache, host
+
+
+# ------------------------------------------------------------------------------------- encode
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
+def test_encode_bit_exact_ragged_appends(dtype):
+    B, H = 2, 3
+    appends = [37, 1, 16, 5, 70]
+    cache, host = build_cache(B, H, appends, dtype, seed=123)
+    torch.cuda.synchronize()
+    D = oracle.signs(123)
+    assert np.array_equal(cache.planes()["signs"].cpu().numpy(), D)
+    assert cache.lengths == [sum(appends)] * B
+    assert cache.planes()["lengths"].cpu().tolist() == [sum(appends)] * B
+    for b in range(B):
+        for h in range(H):
+            assert_planes_equal(gpu_head_planes(cache, b, h, host.n), host.encode(b, h, D), f"b{b} h{h}")
+    assert cache.status() == 0
+
+
+def test_encode_strided_inputs_and_special_values():
+    B, H, n = 1, 2, 48
+    g = torch.Generator(device=DEV).manual_seed(5)
+    big = torch.randn((B, n, H, 256), generator=g, device=DEV)  # padded last dim -> strided view
+    K = big[..., :128].clone()
+    K[0, 3, 0, :] = 0.0                       # zero key: every sign bit 1, cinv = 1
+    K[0, 4, 1, 10:20] = 0.0                   # exact zeros inside a key
+    Vb = big.clone()
+    Vb[0, 5, 0, :128] = 0.25                  # constant (binary16-exact) group values
+    Vb[0, 6, 1, 0:32] = 3.0e4                 # large but representable
+    K = K.contiguous()
+    V = Vb[..., :128]                         # non-contiguous view, unit channel stride
+    Kb = torch.empty_like(Vb)
+    Kb[..., :128] = K
+    Kv = Kb[..., :128]
+    cache = kv.Cache(B, H, 128, seed=9)
+    cache.append(Kv, V)
+    host = HostKV(B, H, 128)
+    host.add(Kv, V)
+    D = oracle.signs(9)
+    for h in range(H):
+        assert_planes_equal(gpu_head_planes(cache, 0, h, n), host.encode(0, h, D), f"h{h}")
+    assert cache.status() == 0
+
+
+def test_encode_status_flags():
+    cache = kv.Cache(1, 1, 128, seed=0)
+    K = torch.zeros((1, 1, 1, 128), device=DEV)
+    V = torch.zeros((1, 1, 1, 128), device=DEV)
+    V[0, 0, 0, 5] = 1e7                       # beyond min + 15 * 65504: saturation
+    cache.append(K, V)
+    assert cache.status() & kv.STATUS_FP16_SATURATED
+    V2 = torch.zeros_like(V)
+    V2[0, 0, 0, 7] = float("nan")
+    cache.append(K, V2)
+    assert cache.status() & kv.STATUS_NONFINITE
+
+
+def test_capacity_and_argument_errors():
+    cache = kv.Cache(1, 1, 128, seed=0)
+    K = torch.zeros((1, 100, 1, 128), device=DEV)
+    cache.append(K, K)
+    with pytest.raises(kv.Kv1bError) as e:
+        cache.append(K, K)
+    assert e.value.code == -3
+    assert cache.lengths == [100]
+    q = torch.zeros((1, 3, 128), device=DEV)   # 3 % 1 == 0 but G = 3 fine; 9 heads -> G 9 > 8
+    with pytest.raises(kv.Kv1bError):
+        cache.attend(torch.zeros((1, 9, 128), device=DEV), 0.1)
+    with pytest.raises(kv.Kv1bError):
+        cache.attend_topp(q, 0.1, 0.0)
+    with pytest.raises(kv.Kv1bError):
+        cache.attend_topp(q, 0.1, 1.5)
+
+
+# ------------------------------------------------------------------------------------- query / scores
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_query_prep_and_scores_bit_exact(dtype):
+    B, Hkv, G = 2, 3, 2
+    cache, host = build_cache(B, Hkv, [300], dtype, seed=77)
+    g = torch.Generator(device=DEV).manual_seed(3)
+    q = (torch.randn((B, Hkv * G, 128), generator=g, device=DEV) * 2.0).to(dtype)
+    q[0, 1] = 0.0                                # flat query: delta = 0, all codes 0
+    qp = cache.query_prep(q)
+    sc = cache.scores(q, 0.125)
+    torch.cuda.synchronize()
+    D = oracle.signs(77)
+    qn = to_np32(q)
+    for b in range(B):
+        for hq in range(Hkv * G):
+            r = oracle.query_prep(qn[b, hq], D)
+            assert np.array_equal(qp["planes"][b, hq].cpu().numpy().view(np.uint32), r["planes"])
+            assert qp["vl"][b, hq].item() == r["vl"] and qp["delta"][b, hq].item() == r["delta"]
+            assert qp["Sq"][b, hq].item() == r["Sq"]
+            enc = host.encode(b, hq // G, D)
+            A, Bc = oracle.score_ints(enc["bits"], r["planes"])
+            s = oracle.logits(enc, r, 0.125)
+            assert np.array_equal(sc["A"][b, hq, :300].cpu().numpy(), A)
+            assert np.array_equal(sc["Bc"][b, hq, :300].cpu().numpy(), Bc)
+            assert np.array_equal(sc["s"][b, hq, :300].cpu().numpy().view(np.uint32), s.view(np.uint32))
+
+
+# ------------------------------------------------------------------------------------- attend
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("engine", [kv.ATTEND_TENSOR, kv.ATTEND_CUDA_CORE])
+def test_attend_parity_group_sizes(G, engine):
+    B, Hkv = 2, 2
+    cache, host = build_cache(B, Hkv, [700, 3], torch.bfloat16, seed=5, data_seed=G)
+    g = torch.Generator(device=DEV).manual_seed(100 + G)
+    q = torch.randn((B, Hkv * G, 128), generator=g, device=DEV).to(torch.bfloat16)
+    out = cache.attend(q, 1 / math.sqrt(128), engine=engine)
+    ref = oracle_attend_all(host, q, oracle.signs(5), 1 / math.sqrt(128), G)
+    assert_rows_close(out.cpu().numpy(), ref, where=f"G{G} e{engine}")
+
+
+@pytest.mark.parametrize("L", [1, 15, 16, 17, 255, 256, 257, 1000, 4099])
+@pytest.mark.parametrize("splits", [0, 1, 3, 7])
+def test_attend_parity_lengths_and_splits(L, splits):
+    B, Hkv, G = 1, 2, 4
+    cache, host = build_cache(B, Hkv, [L], torch.float32, seed=11, data_seed=L)
+    g = torch.Generator(device=DEV).manual_seed(L)
+    q = torch.randn((B, Hkv * G, 128), generator=g, device=DEV)
+    ref = oracle_attend_all(host, q, oracle.signs(11), 0.2, G)
+    for engine in (kv.ATTEND_TENSOR, kv.ATTEND_CUDA_CORE):
+        out = cache.attend(q, 0.2, engine=engine, num_splits=splits)
+        assert_rows_close(out.cpu().numpy(), ref, where=f"L{L} s{splits} e{engine}")
+
+
+def test_attend_empty_cache_gives_zeros():
+    cache = kv.Cache(2, 2, 128, seed=0)
+    q = torch.randn((2, 8, 128), device=DEV)
+    for engine in (kv.ATTEND_TENSOR, kv.ATTEND_CUDA_CORE):
+        assert torch.count_nonzero(cache.attend(q, 0.1, engine=engine)).item() == 0
+    out, sel, cnt = cache.attend_topp(q, 0.1, 0.9)
+    assert torch.count_nonzero(out).item() == 0 and torch.count_nonzero(cnt).item() == 0
+
+
+@pytest.mark.parametrize("vscale", [1e-4, 1e-2, 30.0, 1e3])
+def test_attend_value_magnitudes(vscale):
+    B, Hkv, G = 1, 1, 4
+    cache, host = build_cache(B, Hkv, [2000], torch.float32, seed=3, data_seed=7, vscale=vscale)
+    q = torch.randn((B, G, 128), device=DEV, generator=torch.Generator(device=DEV).manual_seed(1))
+    ref = oracle_attend_all(host, q, oracle.signs(3), 0.09, G)
+    for engine in (kv.ATTEND_TENSOR, kv.ATTEND_CUDA_CORE):
+        assert_rows_close(cache.attend(q, 0.09, engine=engine).cpu().numpy(), ref, where=f"v{vscale} e{engine}")
+
+
+def test_attend_peaked_softmax():
+    # a large softmax scale concentrates the mass on a few tokens (online rescaling exercised)
+    B, Hkv, G = 1, 2, 4
+    cache, host = build_cache(B, Hkv, [3000], torch.float32, seed=8, data_seed=2)
+    q = torch.randn((B, Hkv * G, 128), device=DEV, generator=torch.Generator(device=DEV).manual_seed(4))
+    ref = oracle_attend_all(host, q, oracle.signs(8), 3.0, G)
+    for engine in (kv.ATTEND_TENSOR, kv.ATTEND_CUDA_CORE):
+        for splits in (0, 5):
+            out = cache.attend(q, 3.0, engine=engine, num_splits=splits)
+            assert_rows_close(out.cpu().numpy(), ref, where=f"peaked e{engine} s{splits}")
+
+
+def test_attend_deterministic_reruns():
+    cache, host = build_cache(1, 2, [5000], torch.bfloat16, seed=1)
+    q = torch.randn((1, 8, 128), device=DEV).to(torch.bfloat16)
+    a = cache.attend(q, 0.1).clone()
+    b = cache.attend(q, 0.1)
+    assert torch.equal(a, b)
+
+
+# ------------------------------------------------------------------------------------- Top-p
+def topp_check(cache, host, q, scale, p, G, signs, rows=None):
+    out, sel, cnt = cache.attend_topp(q, scale, p)
+    torch.cuda.synchronize()
+    qn = to_np32(q)
+    B, Hq, _ = qn.shape
+    encs = {}
+    for b in range(B):
+        for hq in range(Hq):
+            if rows is not None and (b, hq) not in rows:
+                continue
+            kvh = hq // G
+            if (b, kvh) not in encs:
+                encs[(b, kvh)] = host.encode(b, kvh, signs)
+            rs, ro = oracle.attend_topp(encs[(b, kvh)], qn[b, hq], signs, scale, p)
+            n = cnt[b, hq].item()
+            assert n == len(rs), f"b{b} hq{hq}: count {n} vs {len(rs)}"
+            assert np.array_equal(sel[b, hq, :n].cpu().numpy(), rs), f"b{b} hq{hq}: index sets differ"
+            assert_rows_close(out[b, hq].cpu().numpy(), ro, where=f"topp b{b} hq{hq}")
+    return cnt
+
+
+@pytest.mark.parametrize("p", [0.05, 0.5, 0.9, 0.999, 1.0])
+def test_topp_parity(p):
+    B, Hkv, G = 2, 2, 2
+    cache, host = build_cache(B, Hkv, [1500, 37], torch.bfloat16, seed=21, data_seed=3)
+    q = torch.randn((B, Hkv * G, 128), device=DEV, generator=torch.Generator(device=DEV).manual_seed(9))
+    q = q.to(torch.bfloat16)
+    topp_check(cache, host, q, 0.5, p, G, oracle.signs(21))
+
+
+def test_topp_ties_take_lowest_indices():
+    # many identical keys -> identical logits; the selection must take them in index order
+    B, Hkv, G, L = 1, 1, 1, 600
+    cache = kv.Cache(B, Hkv, 640, seed=4)
+    host = HostKV(B, Hkv, 640)
+    g = torch.Generator(device=DEV).manual_seed(0)
+    K = torch.randn((B, L, Hkv, 128), generator=g, device=DEV)
+    K[:, 100:500] = K[:, 50:51]                # 401 equal keys (positions 50 and 100..499)
+    V = torch.randn((B, L, Hkv, 128), generator=g, device=DEV)
+    cache.append(K, V)
+    host.add(K, V)
+    q = K[:, 50, :, :].clone().view(B, 1, 128) * 0.3
+    for p in (0.3, 0.6, 0.95):
+        topp_check(cache, host, q, 0.3, p, G, oracle.signs(4))
