@@ -140,6 +140,25 @@ size_t kv1b_attend_workspace_bytes(const kv1b_cache_t* cache, int32_t num_q_head
 int kv1b_attend(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,
                 float* out, void* ws, size_t ws_bytes, int32_t flags, int32_t num_splits, void* stream);
 
+/* Fixed size of the device array behind kv1b_attend_noalloc (4 MiB on every GPU that loads the
+ * library, held until the process exits). */
+#define KV1B_NOALLOC_SCRATCH_BYTES (4u << 20)
+
+/* kv1b_attend without a workspace and without any allocation.  (The pages describe nothing like
+ * it; it exists for this library's users.)  For callers that can neither allocate device memory
+ * (their framework's allocator owns it, or cudaMalloc/cudaFree would synchronise a
+ * latency-critical decode loop) nor pass a workspace buffer (a fixed ABI with inputs and outputs
+ * only).  Same arguments, result and rules as kv1b_attend minus ws / ws_bytes / num_splits; the
+ * split-K partials go to a file-scope device array of KV1B_NOALLOC_SCRATCH_BYTES instead.
+ * The first call on a device looks up that array's device address (cudaGetSymbolAddress, with
+ * the device current) and caches it; make that first call before any stream capture.
+ * Every call shares the array: calls whose kernels may overlap on the GPU race, so order them on
+ * one stream (or otherwise).  The split count is lowered when needed to fit the array; a shape
+ * whose partials do not fit even unsplit (batch * num_q_heads * 520 bytes > the array) returns
+ * KV1B_ERR_WORKSPACE before launching anything.  Calls no cudaMalloc / cudaFree. */
+int kv1b_attend_noalloc(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,
+                        float* out, int32_t flags, void* stream);
+
 /* Adaptive Top-p decode attention.  Per (b, hq): integer masses u_t ~ 2^32 exp(s_t - max s)
  * (degree-7 polynomial for 2^f, reproducible bit for bit), T = ceil(p * sum u) in fp64; the
  * selected set is the shortest prefix of the order (s desc, index asc) whose mass reaches T.

@@ -25,8 +25,8 @@ ERRORS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "capacity", -4
 
 # symbols declared in include/kv1b.h
 SYMBOLS = ("kv1b_cache_bytes", "kv1b_cache_init", "kv1b_encode_append", "kv1b_attend_workspace_bytes",
-           "kv1b_attend", "kv1b_attend_topp", "kv1b_query_prep", "kv1b_scores", "kv1b_read_status",
-           "kv1b_status_string", "kv1b_version")
+           "kv1b_attend", "kv1b_attend_noalloc", "kv1b_attend_topp", "kv1b_query_prep", "kv1b_scores",
+           "kv1b_read_status", "kv1b_status_string", "kv1b_version")
 
 
 class Kv1bError(RuntimeError):
