@@ -67,6 +67,7 @@ extern "C" {
 /* status word bits (kv1b_read_status) */
 #define KV1B_STATUS_NONFINITE 1       /* a K or V element appended was NaN or Inf */
 #define KV1B_STATUS_FP16_SATURATED 2  /* a value group's min or scale left the binary16 range */
+#define KV1B_STATUS_TIMEOUT 4         /* an attend kernel's bounded pipeline wait ran out (results invalid) */
 
 /*
  * Cache descriptor.  Filled by kv1b_cache_init; treat as opaque except for reading the fields.

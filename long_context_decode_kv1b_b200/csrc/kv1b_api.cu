@@ -93,6 +93,23 @@ int32_t max_splits(const kv1b_cache_t* c) {
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? KV1B_OK : KV1B_ERR_CUDA; }
 
+// Partial slots of the persistent kernel: segments x pieces x G x (6 + 128) floats; the piece
+// count per segment does not depend on the length, so the capacity-sized plan bounds every call.
+size_t ws_bytes_needed(const kv1b_cache_t* c, int32_t num_q_heads) {
+  const int G = num_q_heads / c->num_kv_heads;
+  if (!kv1b_ws_supported(G)) return 0;
+  int64_t T, Lt;
+  int ncta, pieces;
+  kv1b_ws_plan(c->batch, c->num_kv_heads, G, c->capacity, num_sms(), &T, &Lt, &ncta, &pieces);
+  return static_cast<size_t>(c->batch) * c->num_kv_heads * pieces * G * kv1b::kPartStride * 4;
+}
+
+bool equal_lengths(const kv1b_cache_t* c) {
+  for (int b = 1; b < c->batch; ++b)
+    if (c->h_lengths[b] != c->h_lengths[0]) return false;
+  return true;
+}
+
 }  // namespace
 
 extern "C" {
@@ -177,7 +194,11 @@ int kv1b_encode_append(kv1b_cache_t* cache, const void* k, const void* v, int32_
 size_t kv1b_attend_workspace_bytes(const kv1b_cache_t* cache, int32_t num_q_heads, int32_t mode) {
   if (!cache_ok(cache) || heads_check(cache, num_q_heads) != KV1B_OK) return 0;
   const size_t rows = static_cast<size_t>(cache->batch) * num_q_heads;
-  if (mode == 0) return align_up(rows * static_cast<size_t>(max_splits(cache)) * kv1b::kPartStride * 4);
+  if (mode == 0) {
+    const size_t split_bytes = rows * static_cast<size_t>(max_splits(cache)) * kv1b::kPartStride * 4;
+    return align_up(split_bytes > ws_bytes_needed(cache, num_q_heads) ? split_bytes
+                                                                      : ws_bytes_needed(cache, num_q_heads));
+  }
   if (mode == 1) return align_up(rows * static_cast<size_t>(cache->capacity) * 4);
   return 0;
 }
@@ -193,6 +214,31 @@ int kv1b_attend(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32
   if (!aligned(q, 16) || !aligned(ws, kAlign) || !aligned(out, 16)) return KV1B_ERR_MISALIGNED;
   if (ws_bytes < kv1b_attend_workspace_bytes(cache, num_q_heads, 0)) return KV1B_ERR_WORKSPACE;
   const int64_t maxlen = max_length(cache);
+  const int G = num_q_heads / cache->num_kv_heads;
+  if (flags == KV1B_ATTEND_TENSOR && num_splits == 0 && kv1b_ws_supported(G) && equal_lengths(cache) && maxlen > 0) {
+    kv1b::AttendWsParams w;
+    memset(&w, 0, sizeof(w));
+    w.c = view(cache);
+    w.q = q;
+    w.q_dtype = q_dtype;
+    w.Hq = num_q_heads;
+    w.scale = scale;
+    w.L = static_cast<int32_t>(maxlen);
+    int ncta = 0, pieces = 0;
+    kv1b_ws_plan(cache->batch, cache->num_kv_heads, G, maxlen, num_sms(), &w.T, &w.Lt, &ncta, &pieces);
+    int64_t Tc, Ltc;
+    int nc, pieces_cap;
+    kv1b_ws_plan(cache->batch, cache->num_kv_heads, G, cache->capacity, num_sms(), &Tc, &Ltc, &nc, &pieces_cap);
+    w.ncta = ncta;
+    w.max_pieces = pieces_cap > pieces ? pieces_cap : pieces;
+    if (w.max_pieces > 256 ||
+        static_cast<size_t>(cache->batch) * cache->num_kv_heads * w.max_pieces * G * kv1b::kPartStride * 4 > ws_bytes)
+      return KV1B_ERR_WORKSPACE;
+    w.part = static_cast<float*>(ws);
+    w.out = out;
+    w.status = cache->d_status;
+    return cuda_status(kv1b_launch_attend_ws(w, G, static_cast<cudaStream_t>(stream)));
+  }
   kv1b::AttendParams p;
   memset(&p, 0, sizeof(p));
   p.c = view(cache);
@@ -204,7 +250,6 @@ int kv1b_attend(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32
   p.part = static_cast<float*>(ws);
   p.out = out;
   for (int b = 0; b < cache->batch; ++b) p.len[b] = static_cast<int32_t>(cache->h_lengths[b]);
-  const int G = num_q_heads / cache->num_kv_heads;
   return cuda_status(kv1b_launch_attend(p, G, flags, static_cast<int32_t>(maxlen), static_cast<cudaStream_t>(stream)));
 }
 

@@ -367,22 +367,38 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendParams 
 }
 
 // log-sum-exp merge of the split partials; one block of 128 threads (channels) per (b, hq).
+// Split maxima and weights are formed in parallel, then each channel sums the splits with
+// independent loads (nsplit <= 1024).
 __global__ void __launch_bounds__(128) merge_kernel(const float* __restrict__ part, float* __restrict__ out,
                                                     int nsplit) {
+  __shared__ float s_w[1024];
+  __shared__ float s_red[4];
   const int64_t row = blockIdx.x;  // b * Hq + hq
   const float* pr = part + row * nsplit * kPartStride;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   float M = -INFINITY;
-  for (int s = 0; s < nsplit; ++s) M = fmaxf(M, pr[s * kPartStride]);
-  float den = 0.0f, num = 0.0f;
-  if (M != -INFINITY) {
-    for (int s = 0; s < nsplit; ++s) {
-      const float ms = pr[s * kPartStride];
-      if (ms == -INFINITY) continue;
-      const float w = exp2f(ms - M);
-      den = __fmaf_rn(w, pr[s * kPartStride + 1], den);
-      num = __fmaf_rn(w, pr[s * kPartStride + 2 + threadIdx.x], num);
-    }
+  for (int k = threadIdx.x; k < nsplit; k += 128) M = fmaxf(M, pr[k * kPartStride]);
+  #pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, m));
+  if (lane == 0) s_red[warp] = M;
+  __syncthreads();
+  M = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
+  __syncthreads();
+  float den = 0.0f;
+  for (int k = threadIdx.x; k < nsplit; k += 128) {
+    const float ms = pr[k * kPartStride];
+    const float w = (ms != -INFINITY && M != -INFINITY) ? exp2f(ms - M) : 0.0f;
+    s_w[k] = w;
+    den = __fmaf_rn(w, pr[k * kPartStride + 1], den);
   }
+  #pragma unroll
+  for (int m = 16; m >= 1; m >>= 1) den += __shfl_xor_sync(kFull, den, m);
+  if (lane == 0) s_red[warp] = den;
+  __syncthreads();
+  den = (s_red[0] + s_red[1]) + (s_red[2] + s_red[3]);
+  float num = 0.0f;
+  #pragma unroll 8
+  for (int k = 0; k < nsplit; ++k) num = __fmaf_rn(s_w[k], pr[k * kPartStride + 2 + threadIdx.x], num);
   out[row * kD + threadIdx.x] = den > 0.0f ? __fdiv_rn(num, den) : 0.0f;
 }
 

@@ -72,6 +72,24 @@ struct ToppParams {
 
 constexpr int kPartStride = 2 + 128;
 
+// persistent warp-specialised attend (kv1b_attend_ws.cu)
+struct AttendWsParams {
+  CacheView c;
+  const void* q;
+  int32_t q_dtype;
+  int32_t Hq;
+  float scale;
+  int32_t L;           // tokens per sequence (equal for every sequence)
+  int64_t T;           // total 16-token tiles over all (sequence, kv-head) segments
+  int64_t Lt;          // tiles per segment
+  int32_t ncta;        // CTAs (one per SM)
+  int32_t max_pieces;  // partial slots per segment
+  float* part;         // [segments][max_pieces][warps][G][6 + 128]: m, l, mid[4], o[128]
+  float* out;          // [B][Hq][128]
+  int32_t* status;     // cache status word (timeout flag)
+};
+constexpr int kPartStrideWs = 6 + 128;
+
 }  // namespace kv1b
 
 cudaError_t kv1b_launch_init(uint64_t seed, float* signs, int32_t* lengths, int32_t batch, int32_t* status,
@@ -84,3 +102,8 @@ cudaError_t kv1b_launch_query_prep(const kv1b::CacheView& c, const void* q, int3
 cudaError_t kv1b_launch_scores(const kv1b::ScoresParams& p, int32_t G, int32_t max_len, cudaStream_t stream);
 cudaError_t kv1b_launch_topp(const kv1b::ToppParams& p, cudaStream_t stream);
 int kv1b_pick_splits(int32_t B, int32_t Hkv, int64_t max_len, int num_sms);
+bool kv1b_ws_supported(int32_t G);
+int kv1b_ws_rows_per_piece();
+void kv1b_ws_plan(int32_t B, int32_t Hkv, int32_t G, int64_t L, int num_sms, int64_t* T, int64_t* Lt, int* ncta,
+                  int* max_pieces);
+cudaError_t kv1b_launch_attend_ws(const kv1b::AttendWsParams& p, int32_t G, cudaStream_t stream);

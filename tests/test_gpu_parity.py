@@ -147,6 +147,7 @@ def test_attend_parity_group_sizes(G, engine):
     out = cache.attend(q, 1 / math.sqrt(128), engine=engine)
     ref = oracle_attend_all(host, q, oracle.signs(5), 1 / math.sqrt(128), G)
     assert_rows_close(out.cpu().numpy(), ref, where=f"G{G} e{engine}")
+    assert cache.status() == 0
 
 
 @pytest.mark.parametrize("L", [1, 15, 16, 17, 255, 256, 257, 1000, 4099])
@@ -160,6 +161,7 @@ def test_attend_parity_lengths_and_splits(L, splits):
     for engine in (kv.ATTEND_TENSOR, kv.ATTEND_CUDA_CORE):
         out = cache.attend(q, 0.2, engine=engine, num_splits=splits)
         assert_rows_close(out.cpu().numpy(), ref, where=f"L{L} s{splits} e{engine}")
+    assert cache.status() == 0
 
 
 def test_attend_empty_cache_gives_zeros():
