@@ -2,23 +2,28 @@
 //
 // Work split: all (sequence, kv-head) segments are laid end to end in 16-token tiles and cut into
 // one equal contiguous range per CTA, so every SM streams the same number of compressed bytes
-// whatever the batch / head / context mix.  Each CTA walks its range in 512-token chunks that a
-// 3-stage shared-memory ring receives by cp.async.bulk (plain bulk copies, no multicast); an
-// mbarrier per stage tracks the bytes, and the last warp to finish a stage refills it.
+// whatever the batch / head / context mix.  Each CTA walks its range in 512-token chunks; every
+// warp owns a 64-token slice of each chunk and streams that slice into its own 3-stage
+// shared-memory ring with cp.async.bulk (plain bulk copies, no multicast), tracked by its own
+// mbarriers and refilled by itself, so warps never wait on one another inside a segment.
 //
-// Each of the 16 warps owns a 32-token slice of every chunk and does all of the work for it, so
-// warps never wait on one another inside a segment:
-//   lane = token: binary x INT4 popcount proxy scores of the G query heads sharing this kv-head
-//   ("RaBitQCache", abstract / key design), a warp-local online softmax in log2 units whose
-//   reference maximum is raised only when a logit exceeds it by 8 (then the warp's sums are
-//   rescaled), and the weights p * scale written as fp16 hi + lo rows;
-//   then 2 k-steps x 8 m-tiles of mma.sync m16n8k16: the codes as exact fp16 subnormals straight
+// Each warp does all of the work for its slice, one 16-token tile at a time:
+//   the binary x INT4 proxy scores of the G query heads sharing this kv-head ("RaBitQCache",
+//   abstract / key design) as integer tensor-core products: the key sign bits are the A operand
+//   (one AND per register, bits masked in place), the query's 4-bit codes with a per-channel
+//   power-of-two correction the B operand, so the s32 accumulator holds 8 * sum_i bit_i * code_i
+//   exactly, plus 8 * Bc in the spare columns; lane (g, t) then owns token g + 8 (t >> 1) and two
+//   head slots of the tile;
+//   a warp-local online softmax in log2 units whose reference maximum is raised only when a logit
+//   exceeds it by 8 (then the warp's sums are rescaled), and the weights p * scale written as
+//   fp16 hi + lo rows;
+//   then 4 k-steps x 8 m-tiles of mma.sync m16n8k16: the codes as exact fp16 subnormals straight
 //   from the staged code tiles (one AND per register), ldmatrix'd weight B fragments; each chunk's
 //   tensor-core partial is added into fp32 accumulators on the CUDA cores (round to nearest), so
 //   accumulation error does not build up inside the tensor core ("H1B-KV", technical framework:
 //   weights from the sketch, then the 4-bit values).  value = min + scale * code, the min term is
 //   summed per (head, group) in fp32 by the score lanes.
-// At the end of a segment piece the 16 warps' partials are combined in shared memory and the CTA
+// At the end of a segment piece the 8 warps' partials are combined in shared memory and the CTA
 // writes one row (m, l, o[128]) per query head; a merge kernel combines the CTA rows of a head
 // by log-sum-exp.
 //
@@ -31,26 +36,28 @@
 namespace kv1b {
 namespace ws {
 
-constexpr int kWarps = 16;
-constexpr int kThreads = kWarps * 32;            // 512
-constexpr int kChunkTiles = 2 * kWarps;          // 32 tiles = 512 tokens per chunk
-constexpr int kChunkTok = kChunkTiles * 16;
+constexpr int kWarps = 8;
+constexpr int kTPL = 2;                          // tokens per lane per chunk
+constexpr int kThreads = kWarps * 32;            // 256
+constexpr int kWarpTiles = 2 * kTPL;             // 16-token tiles per warp per chunk
+constexpr int kChunkTiles = kWarpTiles * kWarps; // 32 tiles = 512 tokens per chunk
 constexpr int kStages = 3;
 constexpr float kTau = 8.0f;                     // lazy-max threshold (log2 units): p <= 2^8
 constexpr int kNoExp = 1 << 20;
 constexpr long long kSpinLimit = 1LL << 24;
 
-// stage layout (bytes)
-constexpr int kOffBits = 0;                                   // u32 [512][4]
-constexpr int kOffNorm = kOffBits + kChunkTok * 16;           // f32 [512]
-constexpr int kOffCinv = kOffNorm + kChunkTok * 4;            // f32 [512]
-constexpr int kOffSm = kOffCinv + kChunkTok * 4;              // u32 [512][4]
-constexpr int kOffCodes = kOffSm + kChunkTok * 16;            // u32 [32 tiles][256]
-constexpr int kStageBytes = kOffCodes + kChunkTiles * 1024;   // 53248
-constexpr int kBRowsPerWarp = 4 * 32 * 16;                    // [4 groups][32 tokens][16 B]
+// Per-warp stage layout (bytes): the warp's 64-token slice of one chunk.
+constexpr int kWarpTok = kWarpTiles * 16;                     // 64
+constexpr int kOffBits = 0;                                   // u32 [64][4]
+constexpr int kOffNorm = kOffBits + kWarpTok * 16;            // f32 [64]
+constexpr int kOffCinv = kOffNorm + kWarpTok * 4;             // f32 [64]
+constexpr int kOffSm = kOffCinv + kWarpTok * 4;               // u32 [64][4]
+constexpr int kOffCodes = kOffSm + kWarpTok * 16;             // u32 [4 tiles][256]
+constexpr int kStageBytes = kOffCodes + kWarpTiles * 1024;    // 6656
+constexpr int kBRowsPerWarp = 4 * kWarpTok * 16;              // [4 groups][64 tokens][16 B]
 constexpr int kRowF = 6 + 128;                                // per-warp partial: m, l, mid[4], o[128]
-constexpr int kPartSmemBytes = kWarps * 4 * kRowF * 4;        // [16 warps][G <= 4 heads][134] floats
-constexpr int kSmemBytes = kStages * kStageBytes + kWarps * kBRowsPerWarp + kPartSmemBytes;
+constexpr int kPartSmemBytes = kWarps * 4 * kRowF * 4;        // [8 warps][G <= 4 heads][134] floats
+constexpr int kSmemBytes = kWarps * kStages * kStageBytes + kWarps * kBRowsPerWarp + kPartSmemBytes;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 
@@ -70,19 +77,27 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
+// try_wait that lets the hardware suspend the warp (up to ~0.5 ms per try) instead of spinning,
+// so waiting warps give their issue slots to working ones.
+__device__ __forceinline__ bool mbar_try_sleep(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p; mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3; selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(500000u)
+      : "memory");
+  return ok != 0;
+}
+constexpr int kWaitTries = 4096;
 // Bounded wait.  Returns false when the CTA has given up (then the caller proceeds on garbage
 // data; the status word records the failure and no further copies are issued).
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  long long spins = 0;
-  while (!mbar_try(bar, parity)) {
+  for (int tries = 0; tries < kWaitTries; ++tries) {
+    if (mbar_try_sleep(bar, parity)) return true;
     if (*abort_flag) return false;
-    if (++spins > kSpinLimit) {
-      *abort_flag = 1;
-      return false;
-    }
-    if (spins > 32) __nanosleep(32);
   }
-  return true;
+  *abort_flag = 1;
+  return false;
 }
 __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
@@ -122,25 +137,34 @@ __device__ __forceinline__ void mma16816_zc(float d[4], const uint32_t a[4], uin
       : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
 }
+// Integer tensor-core step of the binary x INT4 product: D (s32) += A (16 tokens x 32 channels,
+// s8) * B (32 channels x 8 columns, s8).
+__device__ __forceinline__ void imma16832(int d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// Score MMA over one 16-token tile.  Lane (g, t) holds word t of the sign bits of tokens g and
+// g + 8.  K-block kb (32 channels) takes, from each word, the bits at positions 8j + 2kb (k = 4t+j)
+// and 8j + 2kb + 1 (k = 16+4t+j), j = 0..3, each masked in place so that the byte is
+// bit * 2^((2kb + hi) & 3); the query operand carries code * 2^(3 - that), so every product is
+// 8 * bit * code and D = 8 * sum_i bit_i * code_i exactly (the integer A of the popcount form;
+// the column of ones gives 8 * Bc).
+__device__ __forceinline__ void score_tile(int d[4], uint32_t wg, uint32_t wg8, const uint32_t (&bq)[4][2]) {
+  d[0] = d[1] = d[2] = d[3] = 0;
+  const uint32_t xg[2] = {wg, wg >> 4}, xg8[2] = {wg8, wg8 >> 4};
+  #pragma unroll
+  for (int kb = 0; kb < 4; ++kb) {
+    const uint32_t mlo = 0x01010101u << (2 * (kb & 1)), mhi = mlo << 1;
+    const uint32_t a[4] = {xg[kb >> 1] & mlo, xg8[kb >> 1] & mlo, xg[kb >> 1] & mhi, xg8[kb >> 1] & mhi};
+    imma16832(d, a, bq[kb][0], bq[kb][1]);
+  }
+}
 __device__ __forceinline__ float exp2i(int e) { return __int_as_float((e + 127) << 23); }
 __device__ __forceinline__ int ilog2_pos(float x) { return static_cast<int>((__float_as_uint(x) >> 23) & 0xff) - 127; }
 // exact int -> float for |x| < 2^22 without the quarter-rate conversion unit
 __device__ __forceinline__ float i2f_exact(int x) { return __int_as_float(x + 0x4B400000) - 12582912.0f; }
-
-// Binary x INT4 integer A = sum_j 2^j sum_w popc(b_w & P_jw); the four words of a plane are first
-// folded by a carry-save adder (3 popcounts per plane instead of 4).
-__device__ __forceinline__ int popc_A_csa(const uint4 b, const uint4* P) {
-  int A = 0;
-  #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const uint4 pj = P[j];
-    const uint32_t x0 = b.x & pj.x, x1 = b.y & pj.y, x2 = b.z & pj.z, x3 = b.w & pj.w;
-    const uint32_t s = x0 ^ x1 ^ x2;
-    const uint32_t c = (x0 & x1) | (x2 & (x0 | x1));
-    A += (__popc(s) + __popc(x3) + 2 * __popc(c)) << j;
-  }
-  return A;
-}
 
 struct Work {
   int64_t T;   // total tiles
@@ -164,10 +188,15 @@ __device__ __forceinline__ Chunk chunk_at(const Work& wk, int64_t t, int64_t t_e
   return ch;
 }
 
-__device__ __forceinline__ void issue_chunk(const CacheView& c, const Chunk& ch, uint8_t* st, uint64_t* bar) {
-  const int64_t tok = static_cast<int64_t>(ch.seg) * c.cap + static_cast<int64_t>(ch.lt) * 16;
-  const uint32_t ntok = ch.nt * 16;
+// Copy warp `w`'s tiles of chunk `ch` into its stage (one lane); zero tiles still arrive on the
+// barrier so its phases stay in step with the chunk sequence.
+__device__ __forceinline__ void issue_slice(const CacheView& c, const Chunk& ch, int w, uint8_t* st, uint64_t* bar) {
+  int n = ch.nt - kWarpTiles * w;
+  n = n < 0 ? 0 : (n > kWarpTiles ? kWarpTiles : n);
+  const uint32_t ntok = n * 16;
   mbar_expect_tx(bar, ntok * 104u);
+  if (n == 0) return;
+  const int64_t tok = static_cast<int64_t>(ch.seg) * c.cap + static_cast<int64_t>(ch.lt + kWarpTiles * w) * 16;
   bulk_g2s(st + kOffBits, c.k_bits + tok * 4, ntok * 16, bar);
   bulk_g2s(st + kOffNorm, c.k_norm + tok, ntok * 4, bar);
   bulk_g2s(st + kOffCinv, c.k_cinv + tok, ntok * 4, bar);
@@ -216,8 +245,7 @@ template <int G>
 __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsParams p) {
   static_assert(G == 1 || G == 2 || G == 4, "one n-tile: (head, hi/lo) columns <= 8");
   extern __shared__ __align__(1024) uint8_t smem[];
-  __shared__ __align__(8) uint64_t full_bar[kStages];
-  __shared__ int s_cnt[kStages];
+  __shared__ __align__(8) uint64_t full_bar[kWarps][kStages];
   __shared__ __align__(16) uint4 s_planes[2][G][4];  // double-buffered by segment parity
   __shared__ float s_vl[2][G], s_dl[2][G];
   __shared__ int s_sq[2][G];
@@ -231,15 +259,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
   const int L = p.L;
   const float qsl = __fmul_rn(__fdiv_rn(p.scale, static_cast<float>(kD)), 0x1.715476p+0f);  // scale/128*log2e
   const int g8 = lane >> 2, t4 = lane & 3;
-  uint8_t* brows = smem + kStages * kStageBytes + warp * kBRowsPerWarp;
-  const int tloc = warp * 32 + lane;  // this lane's token within every chunk
+  uint8_t* stages = smem + warp * kStages * kStageBytes;  // this warp's ring
+  uint8_t* brows = smem + kWarps * kStages * kStageBytes + warp * kBRowsPerWarp;
+  uint64_t* bars = full_bar[warp];
 
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&full_bar[s], 1);
-      s_cnt[s] = 0;
-    }
-    s_abort = 0;
+  if (lane == 0) {
+    for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
+    if (warp == 0) s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -251,22 +277,39 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
   int issued = 0;
   for (int s = 0; s < kStages && is.rem > 0; ++s) {
     const int n = is.nt(Lt);
-    if (threadIdx.x == 0) issue_chunk(c, Chunk{is.seg, is.lt, n}, smem + s * kStageBytes, &full_bar[s]);
+    if (lane == 0) issue_slice(c, Chunk{is.seg, is.lt, n}, warp, stages + s * kStageBytes, &bars[s]);
     is.advance(n, Lt);
     ++issued;
   }
 
-  float m_w[G], l_acc[G], mid_acc[G][4];
+  // Score lanes: lane (g, t) takes token g + 8 (t >> 1) of each tile and the head slots
+  // hs0 = 2 (t & 1), hs0 + 1 (a slot >= G is empty).
+  const int hs0 = 2 * (t4 & 1);
+  const int tokr = g8 + 8 * (t4 >> 1);
+  const bool upper = (t4 >> 1) != 0;
+
+  float m_w[G], m_thr[G];        // warp-uniform reference maximum and its rare-path threshold
+  float m_my[2], thr_my[2];      // the same for this lane's two head slots
+  float l_acc[2], mid_acc[2][4]; // this lane's slots: sum p, sum p * min per value group
   float smax[4];
   int E_w[4];
   float D[8][4];
+  uint32_t bq[4][2];             // score-MMA query operand of this segment
+  float vl_my[2], dl_my[2];
+  int sq_my[2];
   auto reset = [&]() {
     #pragma unroll
     for (int h = 0; h < G; ++h) {
       m_w[h] = -INFINITY;
-      l_acc[h] = 0.0f;
+      m_thr[h] = -INFINITY;
+    }
+    #pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      m_my[e] = -INFINITY;
+      thr_my[e] = -INFINITY;
+      l_acc[e] = 0.0f;
       #pragma unroll
-      for (int g = 0; g < 4; ++g) mid_acc[h][g] = 0.0f;
+      for (int g = 0; g < 4; ++g) mid_acc[e][g] = 0.0f;
     }
     #pragma unroll
     for (int g = 0; g < 4; ++g) {
@@ -280,38 +323,37 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
   };
 
   // Segment piece done: each warp puts its partial (m, l, mid[4], o[128]) per head in shared
-  // memory; then thread (head, channel) combines the 16 warps by log-sum-exp and writes the CTA's
+  // memory; then thread (head, channel) combines the warps by log-sum-exp and writes the CTA's
   // row (m, l, o[128] with the mid term folded in) for slot (segment, piece).  Every warp reaches
   // this at the same chunk.
-  float* spart = reinterpret_cast<float*>(smem + kStages * kStageBytes + kWarps * kBRowsPerWarp);
+  float* spart = reinterpret_cast<float*>(smem + kWarps * kStages * kStageBytes + kWarps * kBRowsPerWarp);
   auto flush = [&](int seg) {
-    float v[G * 5];
+    float v[2][5];
     #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      v[h * 5] = l_acc[h];
+    for (int e = 0; e < 2; ++e) {
+      v[e][0] = l_acc[e];
       #pragma unroll
-      for (int g = 0; g < 4; ++g) v[h * 5 + 1 + g] = mid_acc[h][g];
+      for (int g = 0; g < 4; ++g) v[e][1 + g] = mid_acc[e][g];
     }
     #pragma unroll
-    for (int m = 16; m >= 1; m >>= 1)
+    for (int m = 16; m >= 2; m >>= 1)  // lanes with the same t & 1 hold the same head slots
       #pragma unroll
-      for (int k = 0; k < G * 5; ++k) v[k] += __shfl_xor_sync(kFull, v[k], m);
+      for (int e = 0; e < 2; ++e)
+        #pragma unroll
+        for (int k = 0; k < 5; ++k) v[e][k] += __shfl_xor_sync(kFull, v[e][k], m);
     float* mine = spart + warp * 4 * kRowF;
-    if (lane < G) {
-      float* r = mine + lane * kRowF;
-      float mh = m_w[0], lh = v[0], md[4] = {v[1], v[2], v[3], v[4]};
+    if (lane < 2) {
       #pragma unroll
-      for (int h = 1; h < G; ++h)
-        if (lane == h) {
-          mh = m_w[h];
-          lh = v[h * 5];
+      for (int e = 0; e < 2; ++e) {
+        const int h = 2 * lane + e;
+        if (h < G) {
+          float* r = mine + h * kRowF;
+          r[0] = m_my[e];
+          r[1] = v[e][0];
           #pragma unroll
-          for (int g = 0; g < 4; ++g) md[g] = v[h * 5 + 1 + g];
+          for (int g = 0; g < 4; ++g) r[2 + g] = v[e][1 + g];
         }
-      r[0] = mh;
-      r[1] = lh;
-      #pragma unroll
-      for (int g = 0; g < 4; ++g) r[2 + g] = md[g];
+      }
     }
     if (t4 < G) {  // D columns 2 t4, 2 t4 + 1 = head t4, hi and lo parts
       float* o = mine + t4 * kRowF + 6;
@@ -324,8 +366,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
       }
     }
     named_bar(1, kThreads);
-    const int h = threadIdx.x >> 7, ch = threadIdx.x & 127;
-    if (h < G) {
+    const int ch = threadIdx.x & 127;
+    for (int h = threadIdx.x >> 7; h < G; h += kThreads / 128) {
       float M = -INFINITY;
       #pragma unroll
       for (int w = 0; w < kWarps; ++w) M = fmaxf(M, spart[(w * 4 + h) * kRowF]);
@@ -351,7 +393,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
     named_bar(1, kThreads);  // the shared partials may be rewritten by the next flush
   };
 
-  // query preparation of a segment's G heads (warp h -> head h) into buffer seg & 1
+  // Query preparation of a segment's G heads (warp h -> head h) into buffer seg & 1, then every
+  // lane builds its score-MMA operand: column n = g of B holds head n's codes (n < G), ones
+  // (n >= 4, giving Bc) or zeros; k-row 4t + j of k-block kb is channel 32t + 8j + 2kb (+1 for
+  // k-rows 16..31), scaled by 2^(3 - ((2kb + hi) & 3)) to undo the in-place bit position.
   auto prep = [&](int seg) {
     const int par = seg & 1;
     if (warp < G) {
@@ -368,6 +413,30 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
       }
     }
     named_bar(1, kThreads);  // reached by every warp at the same chunk
+    uint32_t pw[4] = {0u, 0u, 0u, 0u};
+    if (g8 < G) {
+      #pragma unroll
+      for (int j = 0; j < 4; ++j) pw[j] = reinterpret_cast<const uint32_t*>(&s_planes[par][g8][j])[t4];
+    }
+    #pragma unroll
+    for (int kb = 0; kb < 4; ++kb)
+      #pragma unroll
+      for (int hi = 0; hi < 2; ++hi) {
+        const int r = 2 * kb + hi;
+        const int sh = 3 - (r & 3);
+        uint32_t code = 0u;
+        #pragma unroll
+        for (int j = 0; j < 4; ++j) code |= ((pw[j] >> r) & 0x01010101u) << j;
+        bq[kb][hi] = (g8 < G) ? (code << sh) : (g8 >= 4 ? (0x01010101u << sh) : 0u);
+      }
+    #pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int h = hs0 + e;
+      const bool ok = h < G;
+      vl_my[e] = ok ? s_vl[par][ok ? h : 0] : 0.0f;
+      dl_my[e] = ok ? s_dl[par][ok ? h : 0] : 0.0f;
+      sq_my[e] = ok ? s_sq[par][ok ? h : 0] : 0;
+    }
   };
 
   reset();
@@ -384,56 +453,79 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
       cur_seg = it.seg;
       prep(cur_seg);
     }
-    const int par = cur_seg & 1;
-    mbar_wait(&full_bar[s], phase, &s_abort);
-    const uint8_t* st = smem + s * kStageBytes;
+    mbar_wait(&bars[s], phase, &s_abort);
+    const uint8_t* st = stages + s * kStageBytes;
+    const int my_tiles = nt - kWarpTiles * warp;  // tiles of this chunk owned by this warp (may be <= 0)
 
-    // ---------------- scores of this lane's token (invalid lanes read token 0 and are masked)
-    const bool valid = tloc < nt * 16 && it.lt * 16 + tloc < L;
-    const int tk = valid ? tloc : 0;
-    const uint4 kb = *reinterpret_cast<const uint4*>(st + kOffBits + tk * 16);
-    const float nc = __fmul_rn(__fmul_rn(reinterpret_cast<const float*>(st + kOffNorm)[tk],
-                                         reinterpret_cast<const float*>(st + kOffCinv)[tk]), qsl);
-    const uint4 smv = *reinterpret_cast<const uint4*>(st + kOffSm + tk * 16);
-    const float i1 = i2f_exact(2 * popc_Bc(kb) - kD);
-    float s2[G];
+    // ---------------- scores: one integer MMA chain per tile, then lane (g, t) takes its token's
+    // two head slots and Bc from the accumulator columns (heads in columns 0..3, Bc in 4..7)
+    bool valid[kWarpTiles];
+    float s2[kWarpTiles][2], sc[kWarpTiles][4], mid[kWarpTiles][4];
     #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      const int A = popc_A_csa(kb, s_planes[par][h]);
-      const float dot = __fmaf_rn(s_vl[par][h], i1, __fmul_rn(s_dl[par][h], i2f_exact(2 * A - s_sq[par][h])));
-      s2[h] = valid ? __fmul_rn(dot, nc) : -INFINITY;
-    }
-    float sc[4], mid[4];
-    {
+    for (int kk = 0; kk < kWarpTiles; ++kk) {
+      const int tt = kk * 16 + tokr;  // token within the warp slice
+      valid[kk] = kk < my_tiles && it.lt * 16 + kWarpTok * warp + tt < L;
+      const uint32_t* kbits = reinterpret_cast<const uint32_t*>(st + kOffBits) + kk * 64 + t4;
+      int d[4];
+      score_tile(d, kbits[g8 * 4], kbits[(g8 + 8) * 4], bq);
+      const int x0 = __shfl_xor_sync(kFull, d[0], 2);
+      const int x2 = __shfl_xor_sync(kFull, d[2], 2);
+      const int x3 = __shfl_xor_sync(kFull, d[3], 2);
+      const int a0 = upper ? x2 : d[0], a1 = upper ? x3 : d[1], bc8 = upper ? d[2] : x0;
+      const float nc = __fmul_rn(__fmul_rn(reinterpret_cast<const float*>(st + kOffNorm)[tt],
+                                           reinterpret_cast<const float*>(st + kOffCinv)[tt]), qsl);
+      const float i1 = i2f_exact((bc8 >> 2) - kD);  // 2 Bc - 128
+      const int aa[2] = {a0, a1};
+      #pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        const float dot = __fmaf_rn(vl_my[e], i1, __fmul_rn(dl_my[e], i2f_exact((aa[e] >> 2) - sq_my[e])));
+        s2[kk][e] = (valid[kk] && hs0 + e < G) ? __fmul_rn(dot, nc) : -INFINITY;
+      }
+      const uint4 smv = *reinterpret_cast<const uint4*>(st + kOffSm + tt * 16);
       const uint32_t smw[4] = {smv.x, smv.y, smv.z, smv.w};
       #pragma unroll
       for (int g = 0; g < 4; ++g) {
         const float scg = __half2float(__ushort_as_half(static_cast<unsigned short>(smw[g] & 0xffffu)));
         const float mn = __half2float(__ushort_as_half(static_cast<unsigned short>(smw[g] >> 16)));
-        sc[g] = valid ? scg : 0.0f;
-        mid[g] = mn;
+        sc[kk][g] = valid[kk] ? scg : 0.0f;
+        mid[kk][g] = valid[kk] ? mn : 0.0f;  // invalid lanes may read a stage slot never filled
       }
     }
 
     // ---------------- warp-local lazy online softmax: rare path when a logit passes its
-    // reference by kTau or a value scale passes the group's running maximum
+    // reference by kTau or a value scale passes the group's power-of-two headroom
     bool rare = false;
     #pragma unroll
-    for (int h = 0; h < G; ++h) rare |= s2[h] > m_w[h] + kTau;
-    #pragma unroll
-    for (int g = 0; g < 4; ++g) rare |= sc[g] > smax[g];  // smax = current power-of-two headroom
+    for (int kk = 0; kk < kWarpTiles; ++kk) {
+      #pragma unroll
+      for (int e = 0; e < 2; ++e) rare |= s2[kk][e] > thr_my[e];
+      #pragma unroll
+      for (int g = 0; g < 4; ++g) rare |= sc[kk][g] > smax[g];
+    }
     if (__any_sync(kFull, rare)) {
+      float lm[2];
+      #pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        lm[e] = s2[0][e];
+        #pragma unroll
+        for (int kk = 1; kk < kWarpTiles; ++kk) lm[e] = fmaxf(lm[e], s2[kk][e]);
+      }
       #pragma unroll
       for (int h = 0; h < G; ++h) {
-        float mx = s2[h];
+        // lanes whose slot (h & 1) is head h contribute; the rest give -inf
+        float mx = (hs0 == (h & ~1)) ? lm[h & 1] : -INFINITY;
         #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
-        if (mx > m_w[h] + kTau) {  // warp-uniform
+        if (mx > m_thr[h]) {  // warp-uniform
           const float alpha = (m_w[h] == -INFINITY) ? 0.0f : ex2(m_w[h] - mx);
           m_w[h] = mx;
-          l_acc[h] = __fmul_rn(l_acc[h], alpha);
-          #pragma unroll
-          for (int g = 0; g < 4; ++g) mid_acc[h][g] = __fmul_rn(mid_acc[h][g], alpha);
+          m_thr[h] = mx + kTau;
+          if (hs0 == (h & ~1)) {
+            const int e = h & 1;
+            l_acc[e] = __fmul_rn(l_acc[e], alpha);
+            #pragma unroll
+            for (int g = 0; g < 4; ++g) mid_acc[e][g] = __fmul_rn(mid_acc[e][g], alpha);
+          }
           const float f = (t4 == h) ? alpha : 1.0f;
           #pragma unroll
           for (int mt = 0; mt < 8; ++mt)
@@ -442,8 +534,19 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
         }
       }
       #pragma unroll
+      for (int e = 0; e < 2; ++e) {  // slot e is head e (t & 1 == 0) or head 2 + e
+        const float mlo = (e < G) ? m_w[e < G ? e : 0] : -INFINITY;
+        const float tlo = (e < G) ? m_thr[e < G ? e : 0] : -INFINITY;
+        const float mhi = (2 + e < G) ? m_w[2 + e < G ? 2 + e : 0] : -INFINITY;
+        const float thi = (2 + e < G) ? m_thr[2 + e < G ? 2 + e : 0] : -INFINITY;
+        m_my[e] = hs0 ? mhi : mlo;
+        thr_my[e] = hs0 ? thi : tlo;
+      }
+      #pragma unroll
       for (int g = 0; g < 4; ++g) {
-        float mx = sc[g];
+        float mx = sc[0][g];
+        #pragma unroll
+        for (int kk = 1; kk < kWarpTiles; ++kk) mx = fmaxf(mx, sc[kk][g]);
         #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
         if (mx > smax[g]) {  // warp-uniform
@@ -463,79 +566,67 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
         }
       }
     }
-    float pr[G];
     #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      pr[h] = valid ? ex2(s2[h] - m_w[h]) : 0.0f;
-      l_acc[h] = __fadd_rn(l_acc[h], pr[h]);
+    for (int kk = 0; kk < kWarpTiles; ++kk) {
+      float pr[2];
       #pragma unroll
-      for (int g = 0; g < 4; ++g) mid_acc[h][g] = __fmaf_rn(pr[h], mid[g], mid_acc[h][g]);
-    }
-    // ---------------- this token's B rows: [group][token][(head, hi/lo) x 8 halves]
-    #pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      const float f = (E_w[g] == kNoExp) ? 0.0f : __fmul_rn(sc[g], exp2i(E_w[g]));
-      uint32_t row[4] = {0u, 0u, 0u, 0u};
-      #pragma unroll
-      for (int h = 0; h < G; h += 2) {
-        if (h + 1 < G) {
-          const uint64_t w2 = mul2(f2pack(pr[h], pr[h + 1]), f2pack(f, f));
-          const uint64_t hi2 = w2 & 0xFFFFE000FFFFE000ull;  // 11 significant bits each
-          const uint64_t lo2 = sub2(w2, hi2);
-          asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(row[h]) : "f"(__uint_as_float(static_cast<uint32_t>(lo2))),
-              "f"(__uint_as_float(static_cast<uint32_t>(hi2))));
-          asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(row[h + 1]) : "f"(__uint_as_float(static_cast<uint32_t>(lo2 >> 32))),
-              "f"(__uint_as_float(static_cast<uint32_t>(hi2 >> 32))));
-        } else {
-          const float w = __fmul_rn(pr[h], f);
-          const float hi = __uint_as_float(__float_as_uint(w) & 0xFFFFE000u);
-          asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(row[h]) : "f"(__fsub_rn(w, hi)), "f"(hi));
-        }
+      for (int e = 0; e < 2; ++e) {
+        pr[e] = (s2[kk][e] != -INFINITY) ? ex2(s2[kk][e] - m_my[e]) : 0.0f;
+        l_acc[e] = __fadd_rn(l_acc[e], pr[e]);
+        #pragma unroll
+        for (int g = 0; g < 4; ++g) mid_acc[e][g] = __fmaf_rn(pr[e], mid[kk][g], mid_acc[e][g]);
       }
-      *reinterpret_cast<uint4*>(brows + (g * 32 + lane) * 16) = make_uint4(row[0], row[1], row[2], row[3]);
+      // this token's B rows, columns (head, hi/lo) of its two head slots:
+      // [group][token][8 halves], this lane writes halves 4 (t & 1) .. 4 (t & 1) + 3
+      #pragma unroll
+      for (int g = 0; g < 4; ++g) {
+        const float f = (E_w[g] == kNoExp) ? 0.0f : __fmul_rn(sc[kk][g], exp2i(E_w[g]));
+        const uint64_t w2 = mul2(f2pack(pr[0], pr[1]), f2pack(f, f));
+        const uint64_t hi2 = w2 & 0xFFFFE000FFFFE000ull;  // 11 significant bits each
+        const uint64_t lo2 = sub2(w2, hi2);
+        uint32_t r0, r1;
+        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r0) : "f"(__uint_as_float(static_cast<uint32_t>(lo2))),
+            "f"(__uint_as_float(static_cast<uint32_t>(hi2))));
+        asm("cvt.rn.f16x2.f32 %0, %1, %2;"
+            : "=r"(r1)
+            : "f"(__uint_as_float(static_cast<uint32_t>(lo2 >> 32))), "f"(__uint_as_float(static_cast<uint32_t>(hi2 >> 32))));
+        *reinterpret_cast<uint2*>(brows + (g * kWarpTok + kk * 16 + tokr) * 16 + (t4 & 1) * 8) = make_uint2(r0, r1);
+      }
     }
     __syncwarp();
 
-    // ---------------- P.V: this warp's 2 tiles x 8 m-tiles, chunk partial flushed into D
-    const uint32_t* codes = reinterpret_cast<const uint32_t*>(st + kOffCodes) + warp * 512 + lane;
-    const int my_tiles = nt - 2 * warp;  // tiles of this chunk owned by this warp (may be <= 0)
+    // ---------------- P.V: this warp's kWarpTiles tiles x 8 m-tiles, chunk partial flushed into D
+    const uint32_t* codes = reinterpret_cast<const uint32_t*>(st + kOffCodes) + lane;
     if (my_tiles > 0) {
-      uint32_t bf[4][2][2];
+      float tmp[8][4];
       #pragma unroll
-      for (int g = 0; g < 4; ++g)
-        #pragma unroll
-        for (int kk = 0; kk < 2; ++kk) ldsm_x2_trans(bf[g][kk][0], bf[g][kk][1], bbase + (g * 32 + kk * 16) * 16);
-      const bool two = my_tiles > 1;
-      #pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        uint32_t a[4];
-        float tmp[4];
-        codes_to_afrag(codes[mt * 32], a);
-        mma16816_zc(tmp, a, bf[mt >> 1][0][0], bf[mt >> 1][0][1]);
-        if (two) {
-          codes_to_afrag(codes[256 + mt * 32], a);
-          mma16816(tmp, a, bf[mt >> 1][1][0], bf[mt >> 1][1][1]);
+      for (int kk = 0; kk < kWarpTiles; ++kk) {
+        if (kk < my_tiles) {
+          uint32_t bf[4][2];
+          #pragma unroll
+          for (int g = 0; g < 4; ++g) ldsm_x2_trans(bf[g][0], bf[g][1], bbase + (g * kWarpTok + kk * 16) * 16);
+          #pragma unroll
+          for (int mt = 0; mt < 8; ++mt) {
+            uint32_t a[4];
+            codes_to_afrag(codes[kk * 256 + mt * 32], a);
+            if (kk == 0) mma16816_zc(tmp[mt], a, bf[mt >> 1][0], bf[mt >> 1][1]);
+            else mma16816(tmp[mt], a, bf[mt >> 1][0], bf[mt >> 1][1]);
+          }
         }
-        #pragma unroll
-        for (int k = 0; k < 4; ++k) D[mt][k] = __fadd_rn(D[mt][k], tmp[k]);
       }
+      #pragma unroll
+      for (int mt = 0; mt < 8; ++mt)
+        #pragma unroll
+        for (int k = 0; k < 4; ++k) D[mt][k] = __fadd_rn(D[mt][k], tmp[mt][k]);
     }
     __syncwarp();
 
-    // ---------------- release the stage; the last warp refills it with the chunk kStages ahead
-    if (lane == 0) {
-      __threadfence_block();
-      const int old = atomicAdd(&s_cnt[s], 1);
-      if (old == kWarps - 1) {
-        s_cnt[s] = 0;
-        if (is.rem > 0 && !s_abort) {
-          asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-          issue_chunk(c, Chunk{is.seg, is.lt, is.nt(Lt)}, smem + s * kStageBytes, &full_bar[s]);
-        }
-      }
-    }
+    // ---------------- refill this warp's stage with the slice kStages chunks ahead
     if (is.rem > 0) {
-      is.advance(is.nt(Lt), Lt);
+      const int n = is.nt(Lt);
+      if (lane == 0 && !s_abort)  // the warp's reads of this slot completed before __syncwarp
+        issue_slice(c, Chunk{is.seg, is.lt, n}, warp, stages + s * kStageBytes, &bars[s]);
+      is.advance(n, Lt);
       ++issued;
     }
     it.advance(nt, Lt);
@@ -546,14 +637,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
   }
   if (t_end > t_begin) flush(cur_seg);
   if (s_abort && lane == 0) atomicOr(p.status, KV1B_STATUS_TIMEOUT);
-  // before the CTA's shared memory is released, every copy issued into the ring must have landed
-  __syncthreads();
-  if (threadIdx.x == 0) {
+  // before the CTA's shared memory is released, every copy issued into this warp's ring must
+  // have landed
+  if (lane == 0) {
     for (int j = (issued - kStages > 0 ? issued - kStages : 0); j < issued; ++j) {
       long long spins = 0;
-      while (!mbar_try(&full_bar[j % kStages], (j / kStages) & 1) && ++spins < kSpinLimit) __nanosleep(64);
+      while (!mbar_try(&bars[j % kStages], (j / kStages) & 1) && ++spins < kSpinLimit) __nanosleep(64);
     }
   }
+  __syncwarp();
 }
 
 // Merge: one block of 128 threads (channels) per (b, hq): log-sum-exp over the CTA pieces of the
