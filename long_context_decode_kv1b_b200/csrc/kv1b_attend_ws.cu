@@ -2,10 +2,11 @@
 //
 // Work split: all (sequence, kv-head) segments are laid end to end in 16-token tiles and cut into
 // one equal contiguous range per CTA, so every SM streams the same number of compressed bytes
-// whatever the batch / head / context mix.  Each CTA walks its range in 512-token chunks; every
-// warp owns a 64-token slice of each chunk and streams that slice into its own 3-stage
-// shared-memory ring with cp.async.bulk (plain bulk copies, no multicast), tracked by its own
-// mbarriers and refilled by itself, so warps never wait on one another inside a segment.
+// whatever the batch / head / context mix.  Each CTA walks its range in 512-token chunks
+// streamed into a 3-stage shared-memory ring with cp.async.bulk (five plain bulk copies per chunk,
+// one per cache plane, no multicast) and mbarrier completion; every warp owns a 64-token slice of
+// each chunk.  A warp done with a stage counts itself out on a shared counter; the warp that
+// counts out last issues the refill, so no warp waits for the others except through the ring.
 //
 // Each warp does all of the work for its slice, one 16-token tile at a time:
 //   the binary x INT4 proxy scores of the G query heads sharing this kv-head ("RaBitQCache",
@@ -36,28 +37,32 @@
 namespace kv1b {
 namespace ws {
 
-constexpr int kWarps = 8;
+constexpr int kWarps = 8;                        // consumer warps; one more warp issues the copies
 constexpr int kTPL = 2;                          // tokens per lane per chunk
-constexpr int kThreads = kWarps * 32;            // 256
+constexpr int kThreads = kWarps * 32;            // 256 consumer threads
+constexpr int kBlock = kThreads + 32;            // + the producer warp
 constexpr int kWarpTiles = 2 * kTPL;             // 16-token tiles per warp per chunk
 constexpr int kChunkTiles = kWarpTiles * kWarps; // 32 tiles = 512 tokens per chunk
 constexpr int kStages = 3;
 constexpr float kTau = 8.0f;                     // lazy-max threshold (log2 units): p <= 2^8
-constexpr int kNoExp = 1 << 20;
+constexpr int kNoExp = 100;                     // group exponent before any scale was seen (finite:
+                                                 // every product with it meets a zero)
+constexpr float kNoMax = -1e30f;                 // reference maximum before any logit was seen
 constexpr long long kSpinLimit = 1LL << 24;
 
-// Per-warp stage layout (bytes): the warp's 64-token slice of one chunk.
+// Stage layout (bytes): one 512-token chunk; warp w uses tokens 64w .. 64w + 63 of it.
+constexpr int kChunkTok = kChunkTiles * 16;                   // 512
 constexpr int kWarpTok = kWarpTiles * 16;                     // 64
-constexpr int kOffBits = 0;                                   // u32 [64][4]
-constexpr int kOffNorm = kOffBits + kWarpTok * 16;            // f32 [64]
-constexpr int kOffCinv = kOffNorm + kWarpTok * 4;             // f32 [64]
-constexpr int kOffSm = kOffCinv + kWarpTok * 4;               // u32 [64][4]
-constexpr int kOffCodes = kOffSm + kWarpTok * 16;             // u32 [4 tiles][256]
-constexpr int kStageBytes = kOffCodes + kWarpTiles * 1024;    // 6656
+constexpr int kOffBits = 0;                                   // u32 [512][4]
+constexpr int kOffNorm = kOffBits + kChunkTok * 16;           // f32 [512]
+constexpr int kOffCinv = kOffNorm + kChunkTok * 4;            // f32 [512]
+constexpr int kOffSm = kOffCinv + kChunkTok * 4;              // u32 [512][4]
+constexpr int kOffCodes = kOffSm + kChunkTok * 16;            // u32 [32 tiles][256]
+constexpr int kStageBytes = kOffCodes + kChunkTiles * 1024;   // 53248
 constexpr int kBRowsPerWarp = 4 * kWarpTok * 16;              // [4 groups][64 tokens][16 B]
 constexpr int kRowF = 6 + 128;                                // per-warp partial: m, l, mid[4], o[128]
-constexpr int kPartSmemBytes = kWarps * 4 * kRowF * 4;        // [8 warps][G <= 4 heads][134] floats
-constexpr int kSmemBytes = kWarps * kStages * kStageBytes + kWarps * kBRowsPerWarp + kPartSmemBytes;
+static_assert(4 * kRowF * 4 <= kBRowsPerWarp, "a warp's flush partial reuses its B-row area");
+constexpr int kSmemBytes = kStages * kStageBytes + kWarps * kBRowsPerWarp;
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 
@@ -67,6 +72,9 @@ __device__ __forceinline__ void mbar_init(uint64_t* bar, int count) {
 __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes)
                : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
@@ -125,7 +133,7 @@ __device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
 // subnormals: rows g get c * 2^-24 (nibbles at bits 0-3 / 16-19 of a half), rows g + 8 get
 // 16 c * 2^-24 (their nibbles sit 4 bits higher).  Both scale factors are undone at the end.
 __device__ __forceinline__ void codes_to_afrag(uint32_t w, uint32_t a[4]) {
-  const uint32_t w8 = w >> 8;
+  const uint32_t w8 = __umulhi(w, 1u << 24);  // w >> 8 on the multiply pipe (the logic pipe is the busy one)
   a[0] = w & 0x000F000Fu;
   a[1] = w & 0x00F000F0u;
   a[2] = w8 & 0x000F000Fu;
@@ -151,14 +159,20 @@ __device__ __forceinline__ void imma16832(int d[4], const uint32_t a[4], uint32_
 // bit * 2^((2kb + hi) & 3); the query operand carries code * 2^(3 - that), so every product is
 // 8 * bit * code and D = 8 * sum_i bit_i * code_i exactly (the integer A of the popcount form;
 // the column of ones gives 8 * Bc).
+__device__ __forceinline__ void imma16832_zc(int d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0));
+}
 __device__ __forceinline__ void score_tile(int d[4], uint32_t wg, uint32_t wg8, const uint32_t (&bq)[4][2]) {
-  d[0] = d[1] = d[2] = d[3] = 0;
-  const uint32_t xg[2] = {wg, wg >> 4}, xg8[2] = {wg8, wg8 >> 4};
+  const uint32_t xg[2] = {wg, __umulhi(wg, 1u << 28)}, xg8[2] = {wg8, __umulhi(wg8, 1u << 28)};  // >> 4
   #pragma unroll
   for (int kb = 0; kb < 4; ++kb) {
     const uint32_t mlo = 0x01010101u << (2 * (kb & 1)), mhi = mlo << 1;
     const uint32_t a[4] = {xg[kb >> 1] & mlo, xg8[kb >> 1] & mlo, xg[kb >> 1] & mhi, xg8[kb >> 1] & mhi};
-    imma16832(d, a, bq[kb][0], bq[kb][1]);
+    if (kb == 0) imma16832_zc(d, a, bq[kb][0], bq[kb][1]);
+    else imma16832(d, a, bq[kb][0], bq[kb][1]);
   }
 }
 __device__ __forceinline__ float exp2i(int e) { return __int_as_float((e + 127) << 23); }
@@ -188,15 +202,11 @@ __device__ __forceinline__ Chunk chunk_at(const Work& wk, int64_t t, int64_t t_e
   return ch;
 }
 
-// Copy warp `w`'s tiles of chunk `ch` into its stage (one lane); zero tiles still arrive on the
-// barrier so its phases stay in step with the chunk sequence.
-__device__ __forceinline__ void issue_slice(const CacheView& c, const Chunk& ch, int w, uint8_t* st, uint64_t* bar) {
-  int n = ch.nt - kWarpTiles * w;
-  n = n < 0 ? 0 : (n > kWarpTiles ? kWarpTiles : n);
-  const uint32_t ntok = n * 16;
+// Copy chunk `ch` (contiguous tiles of one segment) into a stage: five bulk copies, one per plane.
+__device__ __forceinline__ void issue_chunk(const CacheView& c, const Chunk& ch, uint8_t* st, uint64_t* bar) {
+  const uint32_t ntok = ch.nt * 16;
   mbar_expect_tx(bar, ntok * 104u);
-  if (n == 0) return;
-  const int64_t tok = static_cast<int64_t>(ch.seg) * c.cap + static_cast<int64_t>(ch.lt + kWarpTiles * w) * 16;
+  const int64_t tok = static_cast<int64_t>(ch.seg) * c.cap + static_cast<int64_t>(ch.lt) * 16;
   bulk_g2s(st + kOffBits, c.k_bits + tok * 4, ntok * 16, bar);
   bulk_g2s(st + kOffNorm, c.k_norm + tok, ntok * 4, bar);
   bulk_g2s(st + kOffCinv, c.k_cinv + tok, ntok * 4, bar);
@@ -242,10 +252,11 @@ struct TileIt {
 };
 
 template <int G>
-__global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsParams p) {
+__global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsParams p) {
   static_assert(G == 1 || G == 2 || G == 4, "one n-tile: (head, hi/lo) columns <= 8");
   extern __shared__ __align__(1024) uint8_t smem[];
-  __shared__ __align__(8) uint64_t full_bar[kWarps][kStages];
+  __shared__ __align__(8) uint64_t full_bar[kStages];
+  __shared__ __align__(8) uint64_t empty_bar[kStages];  // all consumer warps released the stage
   __shared__ __align__(16) uint4 s_planes[2][G][4];  // double-buffered by segment parity
   __shared__ float s_vl[2][G], s_dl[2][G];
   __shared__ int s_sq[2][G];
@@ -259,13 +270,15 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
   const int L = p.L;
   const float qsl = __fmul_rn(__fdiv_rn(p.scale, static_cast<float>(kD)), 0x1.715476p+0f);  // scale/128*log2e
   const int g8 = lane >> 2, t4 = lane & 3;
-  uint8_t* stages = smem + warp * kStages * kStageBytes;  // this warp's ring
-  uint8_t* brows = smem + kWarps * kStages * kStageBytes + warp * kBRowsPerWarp;
-  uint64_t* bars = full_bar[warp];
+  uint8_t* brows = smem + kStages * kStageBytes + warp * kBRowsPerWarp;
+  uint64_t* bars = full_bar;
 
-  if (lane == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(&bars[s], 1);
-    if (warp == 0) s_abort = 0;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&bars[s], 1);
+      mbar_init(&empty_bar[s], kWarps);
+    }
+    s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
@@ -273,13 +286,26 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
   it.seg = static_cast<int>(t_begin / p.Lt);
   it.lt = static_cast<int>(t_begin - static_cast<int64_t>(it.seg) * p.Lt);
   it.rem = static_cast<int>(t_end - t_begin);
-  TileIt is = it;  // issue position (identical on every warp)
-  int issued = 0;
-  for (int s = 0; s < kStages && is.rem > 0; ++s) {
-    const int n = is.nt(Lt);
-    if (lane == 0) issue_slice(c, Chunk{is.seg, is.lt, n}, warp, stages + s * kStageBytes, &bars[s]);
-    is.advance(n, Lt);
-    ++issued;
+  if (warp == kWarps) {  // producer: one lane streams the CTA's chunks through the ring
+    if (lane == 0) {
+      TileIt is = it;
+      int j = 0;  // chunks issued
+      while (is.rem > 0 && !s_abort) {
+        const int st = j % kStages;
+        if (j >= kStages && !mbar_wait(&empty_bar[st], ((j / kStages) - 1) & 1, &s_abort)) break;
+        const int n = is.nt(Lt);
+        issue_chunk(c, Chunk{is.seg, is.lt, n}, smem + st * kStageBytes, &bars[st]);
+        is.advance(n, Lt);
+        ++j;
+      }
+      // the CTA's shared memory must outlive every copy issued into it (the consumers wait for
+      // all of them unless the CTA gave up)
+      for (int k = (j - kStages > 0 ? j - kStages : 0); k < j; ++k) {
+        long long spins = 0;
+        while (!mbar_try(&bars[k % kStages], (k / kStages) & 1) && ++spins < kSpinLimit) __nanosleep(64);
+      }
+    }
+    return;
   }
 
   // Score lanes: lane (g, t) takes token g + 8 (t >> 1) of each tile and the head slots
@@ -300,13 +326,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
   auto reset = [&]() {
     #pragma unroll
     for (int h = 0; h < G; ++h) {
-      m_w[h] = -INFINITY;
-      m_thr[h] = -INFINITY;
+      m_w[h] = kNoMax;
+      m_thr[h] = kNoMax;
     }
     #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      m_my[e] = -INFINITY;
-      thr_my[e] = -INFINITY;
+      m_my[e] = kNoMax;
+      thr_my[e] = kNoMax;
       l_acc[e] = 0.0f;
       #pragma unroll
       for (int g = 0; g < 4; ++g) mid_acc[e][g] = 0.0f;
@@ -326,7 +352,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
   // memory; then thread (head, channel) combines the warps by log-sum-exp and writes the CTA's
   // row (m, l, o[128] with the mid term folded in) for slot (segment, piece).  Every warp reaches
   // this at the same chunk.
-  float* spart = reinterpret_cast<float*>(smem + kWarps * kStages * kStageBytes + kWarps * kBRowsPerWarp);
+  auto part_of = [&](int w) { return reinterpret_cast<float*>(smem + kStages * kStageBytes + w * kBRowsPerWarp); };
   auto flush = [&](int seg) {
     float v[2][5];
     #pragma unroll
@@ -341,14 +367,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
       for (int e = 0; e < 2; ++e)
         #pragma unroll
         for (int k = 0; k < 5; ++k) v[e][k] += __shfl_xor_sync(kFull, v[e][k], m);
-    float* mine = spart + warp * 4 * kRowF;
+    float* mine = part_of(warp);  // this warp's P.V is done with its B rows
     if (lane < 2) {
       #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int h = 2 * lane + e;
         if (h < G) {
           float* r = mine + h * kRowF;
-          r[0] = m_my[e];
+          r[0] = m_my[e] == kNoMax ? -INFINITY : m_my[e];
           r[1] = v[e][0];
           #pragma unroll
           for (int g = 0; g < 4; ++g) r[2 + g] = v[e][1 + g];
@@ -359,8 +385,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
       float* o = mine + t4 * kRowF + 6;
       #pragma unroll
       for (int mt = 0; mt < 8; ++mt) {
-        const int e = E_w[mt >> 1];
-        const float un = (e == kNoExp) ? 0.0f : exp2i(24 - e);  // codes were c * 2^-24
+        const float un = exp2i(24 - E_w[mt >> 1]);  // codes were c * 2^-24
         o[16 * mt + g8] = __fmul_rn(__fadd_rn(D[mt][0], D[mt][1]), un);
         o[16 * mt + g8 + 8] = __fmul_rn(__fadd_rn(D[mt][2], D[mt][3]), un * 0.0625f);
       }
@@ -370,12 +395,12 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
     for (int h = threadIdx.x >> 7; h < G; h += kThreads / 128) {
       float M = -INFINITY;
       #pragma unroll
-      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, spart[(w * 4 + h) * kRowF]);
+      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, part_of(w)[h * kRowF]);
       float num = 0.0f, den = 0.0f;
       if (M != -INFINITY) {
         #pragma unroll
         for (int w = 0; w < kWarps; ++w) {
-          const float* r = spart + (w * 4 + h) * kRowF;
+          const float* r = part_of(w) + h * kRowF;
           if (r[0] == -INFINITY) continue;
           const float wt = exp2f(r[0] - M);
           den = __fmaf_rn(wt, r[1], den);
@@ -454,8 +479,13 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
       prep(cur_seg);
     }
     mbar_wait(&bars[s], phase, &s_abort);
-    const uint8_t* st = stages + s * kStageBytes;
+    const uint8_t* st = smem + s * kStageBytes;
     const int my_tiles = nt - kWarpTiles * warp;  // tiles of this chunk owned by this warp (may be <= 0)
+
+    // tokens of this warp's slice below `lim` are real (beyond: other warps' tiles, a ragged
+    // segment end, or slots of the stage that were not filled)
+    int lim = L - (it.lt * 16 + kWarpTok * warp);
+    lim = lim < my_tiles * 16 ? lim : my_tiles * 16;
 
     // ---------------- scores: one integer MMA chain per tile, then lane (g, t) takes its token's
     // two head slots and Bc from the accumulator columns (heads in columns 0..3, Bc in 4..7)
@@ -464,16 +494,16 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
     #pragma unroll
     for (int kk = 0; kk < kWarpTiles; ++kk) {
       const int tt = kk * 16 + tokr;  // token within the warp slice
-      valid[kk] = kk < my_tiles && it.lt * 16 + kWarpTok * warp + tt < L;
-      const uint32_t* kbits = reinterpret_cast<const uint32_t*>(st + kOffBits) + kk * 64 + t4;
+      valid[kk] = tt < lim;
+      const uint32_t* kbits = reinterpret_cast<const uint32_t*>(st + kOffBits + warp * kWarpTok * 16) + kk * 64 + t4;
       int d[4];
       score_tile(d, kbits[g8 * 4], kbits[(g8 + 8) * 4], bq);
       const int x0 = __shfl_xor_sync(kFull, d[0], 2);
       const int x2 = __shfl_xor_sync(kFull, d[2], 2);
       const int x3 = __shfl_xor_sync(kFull, d[3], 2);
       const int a0 = upper ? x2 : d[0], a1 = upper ? x3 : d[1], bc8 = upper ? d[2] : x0;
-      const float nc = __fmul_rn(__fmul_rn(reinterpret_cast<const float*>(st + kOffNorm)[tt],
-                                           reinterpret_cast<const float*>(st + kOffCinv)[tt]), qsl);
+      const float nc = __fmul_rn(__fmul_rn(reinterpret_cast<const float*>(st + kOffNorm)[kWarpTok * warp + tt],
+                                           reinterpret_cast<const float*>(st + kOffCinv)[kWarpTok * warp + tt]), qsl);
       const float i1 = i2f_exact((bc8 >> 2) - kD);  // 2 Bc - 128
       const int aa[2] = {a0, a1};
       #pragma unroll
@@ -481,14 +511,14 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
         const float dot = __fmaf_rn(vl_my[e], i1, __fmul_rn(dl_my[e], i2f_exact((aa[e] >> 2) - sq_my[e])));
         s2[kk][e] = (valid[kk] && hs0 + e < G) ? __fmul_rn(dot, nc) : -INFINITY;
       }
-      const uint4 smv = *reinterpret_cast<const uint4*>(st + kOffSm + tt * 16);
-      const uint32_t smw[4] = {smv.x, smv.y, smv.z, smv.w};
+      const uint4 smv = *reinterpret_cast<const uint4*>(st + kOffSm + (kWarpTok * warp + tt) * 16);
+      // invalid tokens may read a stage slot never filled: their (scale, min) become zeros
+      const uint32_t smw[4] = {valid[kk] ? smv.x : 0u, valid[kk] ? smv.y : 0u, valid[kk] ? smv.z : 0u,
+                               valid[kk] ? smv.w : 0u};
       #pragma unroll
       for (int g = 0; g < 4; ++g) {
-        const float scg = __half2float(__ushort_as_half(static_cast<unsigned short>(smw[g] & 0xffffu)));
-        const float mn = __half2float(__ushort_as_half(static_cast<unsigned short>(smw[g] >> 16)));
-        sc[kk][g] = valid[kk] ? scg : 0.0f;
-        mid[kk][g] = valid[kk] ? mn : 0.0f;  // invalid lanes may read a stage slot never filled
+        sc[kk][g] = __half2float(__ushort_as_half(static_cast<unsigned short>(smw[g] & 0xffffu)));
+        mid[kk][g] = __half2float(__ushort_as_half(static_cast<unsigned short>(smw[g] >> 16)));
       }
     }
 
@@ -517,7 +547,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
         #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
         if (mx > m_thr[h]) {  // warp-uniform
-          const float alpha = (m_w[h] == -INFINITY) ? 0.0f : ex2(m_w[h] - mx);
+          const float alpha = ex2(m_w[h] - mx);  // 0 while m_w is still kNoMax
           m_w[h] = mx;
           m_thr[h] = mx + kTau;
           if (hs0 == (h & ~1)) {
@@ -535,10 +565,10 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
       }
       #pragma unroll
       for (int e = 0; e < 2; ++e) {  // slot e is head e (t & 1 == 0) or head 2 + e
-        const float mlo = (e < G) ? m_w[e < G ? e : 0] : -INFINITY;
-        const float tlo = (e < G) ? m_thr[e < G ? e : 0] : -INFINITY;
-        const float mhi = (2 + e < G) ? m_w[2 + e < G ? 2 + e : 0] : -INFINITY;
-        const float thi = (2 + e < G) ? m_thr[2 + e < G ? 2 + e : 0] : -INFINITY;
+        const float mlo = (e < G) ? m_w[e < G ? e : 0] : kNoMax;
+        const float tlo = (e < G) ? m_thr[e < G ? e : 0] : kNoMax;
+        const float mhi = (2 + e < G) ? m_w[2 + e < G ? 2 + e : 0] : kNoMax;
+        const float thi = (2 + e < G) ? m_thr[2 + e < G ? 2 + e : 0] : kNoMax;
         m_my[e] = hs0 ? mhi : mlo;
         thr_my[e] = hs0 ? thi : tlo;
       }
@@ -553,13 +583,11 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
           const int e_new = 6 - ilog2_pos(mx);
           smax[g] = exp2i(7 - e_new);  // scales up to 2^(7-E) keep p * scale * 2^E <= 2^15
           if (e_new < E_w[g]) {
-            if (E_w[g] != kNoExp) {
-              const float beta = exp2i(e_new - E_w[g]);
-              #pragma unroll
-              for (int k = 0; k < 4; ++k) {
-                D[2 * g][k] = __fmul_rn(D[2 * g][k], beta);
-                D[2 * g + 1][k] = __fmul_rn(D[2 * g + 1][k], beta);
-              }
+            const float beta = exp2i(e_new - E_w[g]);  // D is still 0 while E_w is kNoExp
+            #pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              D[2 * g][k] = __fmul_rn(D[2 * g][k], beta);
+              D[2 * g + 1][k] = __fmul_rn(D[2 * g + 1][k], beta);
             }
             E_w[g] = e_new;
           }
@@ -571,7 +599,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
       float pr[2];
       #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        pr[e] = (s2[kk][e] != -INFINITY) ? ex2(s2[kk][e] - m_my[e]) : 0.0f;
+        pr[e] = ex2(s2[kk][e] - m_my[e]);  // -inf for invalid tokens and empty slots -> 0
         l_acc[e] = __fadd_rn(l_acc[e], pr[e]);
         #pragma unroll
         for (int g = 0; g < 4; ++g) mid_acc[e][g] = __fmaf_rn(pr[e], mid[kk][g], mid_acc[e][g]);
@@ -580,7 +608,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
       // [group][token][8 halves], this lane writes halves 4 (t & 1) .. 4 (t & 1) + 3
       #pragma unroll
       for (int g = 0; g < 4; ++g) {
-        const float f = (E_w[g] == kNoExp) ? 0.0f : __fmul_rn(sc[kk][g], exp2i(E_w[g]));
+        const float f = __fmul_rn(sc[kk][g], exp2i(E_w[g]));
         const uint64_t w2 = mul2(f2pack(pr[0], pr[1]), f2pack(f, f));
         const uint64_t hi2 = w2 & 0xFFFFE000FFFFE000ull;  // 11 significant bits each
         const uint64_t lo2 = sub2(w2, hi2);
@@ -596,7 +624,7 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
     __syncwarp();
 
     // ---------------- P.V: this warp's kWarpTiles tiles x 8 m-tiles, chunk partial flushed into D
-    const uint32_t* codes = reinterpret_cast<const uint32_t*>(st + kOffCodes) + lane;
+    const uint32_t* codes = reinterpret_cast<const uint32_t*>(st + kOffCodes + warp * kWarpTiles * 1024) + lane;
     if (my_tiles > 0) {
       float tmp[8][4];
       #pragma unroll
@@ -621,14 +649,8 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
     }
     __syncwarp();
 
-    // ---------------- refill this warp's stage with the slice kStages chunks ahead
-    if (is.rem > 0) {
-      const int n = is.nt(Lt);
-      if (lane == 0 && !s_abort)  // the warp's reads of this slot completed before __syncwarp
-        issue_slice(c, Chunk{is.seg, is.lt, n}, warp, stages + s * kStageBytes, &bars[s]);
-      is.advance(n, Lt);
-      ++issued;
-    }
+    // ---------------- release the stage to the producer
+    if (lane == 0) mbar_arrive(&empty_bar[s]);  // the warp's reads of the stage completed before __syncwarp
     it.advance(nt, Lt);
     if (++s == kStages) {
       s = 0;
@@ -637,15 +659,6 @@ __global__ void __launch_bounds__(kThreads, 1) attend_ws_kernel(const AttendWsPa
   }
   if (t_end > t_begin) flush(cur_seg);
   if (s_abort && lane == 0) atomicOr(p.status, KV1B_STATUS_TIMEOUT);
-  // before the CTA's shared memory is released, every copy issued into this warp's ring must
-  // have landed
-  if (lane == 0) {
-    for (int j = (issued - kStages > 0 ? issued - kStages : 0); j < issued; ++j) {
-      long long spins = 0;
-      while (!mbar_try(&bars[j % kStages], (j / kStages) & 1) && ++spins < kSpinLimit) __nanosleep(64);
-    }
-  }
-  __syncwarp();
 }
 
 // Merge: one block of 128 threads (channels) per (b, hq): log-sum-exp over the CTA pieces of the
@@ -712,7 +725,7 @@ static cudaError_t launch_t(const AttendWsParams& p, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  attend_ws_kernel<G><<<p.ncta, kThreads, kSmemBytes, stream>>>(p);
+  attend_ws_kernel<G><<<p.ncta, kBlock, kSmemBytes, stream>>>(p);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   merge_ws_kernel<<<p.c.B * p.Hq, 128, 0, stream>>>(p, G);
