@@ -3,8 +3,8 @@
 
 One step = one decode step of the long-context workload (32 query / 8 KV heads, head_dim 128,
 batch 1, 1,048,576 cached tokens): encode + append one token per sequence, then full attention of
-all query heads over the whole compressed cache (query prep, popcount scores, online softmax,
-4-bit P.V, split merge).  The cache (872 MB compressed) is larger than L2 (126 MB), so no L2
+all query heads over the whole compressed cache (query prep, binary x INT4 scores, online
+softmax, 4-bit P.V, split merge).  The cache (872 MB compressed) is larger than L2 (126 MB), so no L2
 flush is needed between steps.
 
     python bench.py [--gpus N --steps K --warmup W] [--impl ours|reference] [--config c5]
@@ -32,6 +32,12 @@ METRIC = "compressed-cache decode attention: KV tokens/s per head and HBM GB/s v
 UNIT = "kv_token_heads/s"
 BYTES_PER_TOKEN_HEAD = 104  # 16 B sign bits + 4 B norm + 4 B 1/C + 64 B codes + 16 B scale/min
 FALLBACK_HBM_GBS = 6650.0
+ATTEND_SRC = os.path.join(ROOT, "long_context_decode_kv1b_b200", "csrc", "kv1b_attend_ws.cu")
+# DRAM bytes (read + write) per token x kv-head of one attend kernel launch, from an ncu capture of
+# the c3 workload (same head grouping, cache 218 MB > L2) scaled by the tokens x kv-heads it
+# processed; valid only for the attend source with this SHA-256 (profiles/attend_ws_c3_ncu_full.txt).
+TRAFFIC = {"bytes_per_token_head": 222420480 / 2097408,
+           "source_sha256": "78e51c26d081d32adf9a5ce16b4bada5eb982ff9e5cc00e28775c851940079d6"}
 
 
 def parse_args():
@@ -46,6 +52,19 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-alt", action="store_true")
     return ap.parse_args()
+
+
+def traffic_per_launch(token_heads: float):
+    import hashlib
+
+    try:
+        with open(ATTEND_SRC, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except OSError:
+        return None
+    if TRAFFIC["bytes_per_token_head"] is None or sha != TRAFFIC["source_sha256"]:
+        return None  # the kernel changed since the counters were taken
+    return TRAFFIC["bytes_per_token_head"] * token_heads
 
 
 def peaks():
@@ -250,6 +269,7 @@ def run_ours(args):
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     units = 0
     torch.cuda.synchronize()
+    torch.cuda.nvtx.range_push("timed")  # lets a profiler select exactly the timed launches
     e0.record(stream)
     for j in range(K):
         i = W + j
@@ -259,6 +279,7 @@ def run_ours(args):
         a1[j].record(stream)
         units += cfg.B * cfg.Hkv * cache.lengths[0]
     e1.record(stream)
+    torch.cuda.nvtx.range_pop()
     torch.cuda.synchronize()
     clocks = sampler.stop()
     barrier(world)
@@ -318,7 +339,7 @@ def run_ours(args):
         result = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
             "ms_per_step": t_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "u1 key bits / u4 value codes; int32 popcount; fp32 softmax + accumulation",
+            "dtype": "u1 key bits / u4 value codes; s8 x s8 -> s32 scores; f16 x f16 -> f32 P.V; fp32 softmax",
             "data": "synthetic (seeded torch generators; see long_context_decode_kv1b_b200/workloads.py)",
             "config": {"workload": f"{cfg.name}: {wl.DESCRIPTIONS[cfg.name]}", "batch": cfg.B, "q_heads": cfg.Hq,
                        "kv_heads": cfg.Hkv, "head_dim": 128, "context": cfg.L,
@@ -326,7 +347,8 @@ def run_ours(args):
                        "l2": "inputs larger than L2 (compressed cache %.0f MB > 126 MB); no flush" %
                              (bytes_per_attend / 1e6), "parallelism": f"independent sequence per GPU x{world}"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None, "kernel": "kv1b_attend (attend + merge)",
+                         "frac": achieved / peak, "traffic": traffic_per_launch(cfg.B * cfg.Hkv * L_mean),
+                         "kernel": "kv1b_attend: attend_ws_kernel + merge_ws_kernel, CUDA events around both",
                          "attend_us": att_avg * 1e3, "peak_kind": peak_kind,
                          "frac_of_8tbs": achieved / 8000.0},
             "e2e": e2e,
