@@ -13,8 +13,8 @@
 //   abstract / key design) as integer tensor-core products: the key sign bits are the A operand
 //   (one AND per register, bits masked in place), the query's 4-bit codes with a per-channel
 //   power-of-two correction the B operand, so the s32 accumulator holds 8 * sum_i bit_i * code_i
-//   exactly, plus 8 * Bc in the spare columns; lane (g, t) then owns token g + 8 (t >> 1) and two
-//   head slots of the tile;
+//   exactly, plus 8 * Bc in the spare columns; each lane then owns one token of the tile and two
+//   head slots (and, for the weights, two of the four value groups);
 //   a warp-local online softmax in log2 units whose reference maximum is raised only when a logit
 //   exceeds it by 8 (then the warp's sums are rescaled), and the weights p * scale written as
 //   fp16 hi + lo rows;
@@ -59,7 +59,8 @@ constexpr int kOffCinv = kOffNorm + kChunkTok * 4;            // f32 [512]
 constexpr int kOffSm = kOffCinv + kChunkTok * 4;              // u32 [512][4]
 constexpr int kOffCodes = kOffSm + kChunkTok * 16;            // u32 [32 tiles][256]
 constexpr int kStageBytes = kOffCodes + kChunkTiles * 1024;   // 53248
-constexpr int kBRowsPerWarp = 4 * kWarpTok * 16;              // [4 groups][64 tokens][16 B]
+constexpr int kGroupRows = kWarpTok + 1;                      // 16-B B rows per group (+1 pad: bank shift)
+constexpr int kBRowsPerWarp = 4 * kGroupRows * 16;            // [4 groups][65 rows][16 B]
 constexpr int kRowF = 6 + 128;                                // per-warp partial: m, l, mid[4], o[128]
 static_assert(4 * kRowF * 4 <= kBRowsPerWarp, "a warp's flush partial reuses its B-row area");
 constexpr int kSmemBytes = kStages * kStageBytes + kWarps * kBRowsPerWarp;
@@ -308,21 +309,28 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsPara
     return;
   }
 
-  // Score lanes: lane (g, t) takes token g + 8 (t >> 1) of each tile and the head slots
-  // hs0 = 2 (t & 1), hs0 + 1 (a slot >= G is empty).
-  const int hs0 = 2 * (t4 & 1);
-  const int tokr = g8 + 8 * (t4 >> 1);
+  // Score lanes.  MMA row g of a tile holds token g + 8 (g >> 2) and row g + 8 holds token g + 4,
+  // so that each half-warp's tokens fill 128 contiguous bytes of a B-row group (conflict-free
+  // stores) while the key-word loads stay conflict-free too.  Lane (g, t) takes row g (t < 2) or
+  // row g + 8 (t >= 2) and the head slots hs0 = 2 (t & 1), hs0 + 1 of the scores (a slot >= G is
+  // empty); for the weights the lane pair (t, t ^ 1), which shares the token, splits the value
+  // groups: lane t takes groups 2q, 2q + 1 with q = t & 1.
+  const int q1 = t4 & 1;
+  const int hs0 = 2 * q1;
   const bool upper = (t4 >> 1) != 0;
+  const int row_lo = g8 + 8 * (g8 >> 2), row_hi = g8 + 4;
+  const int tokr = upper ? row_hi : row_lo;
 
   float m_w[G], m_thr[G];        // warp-uniform reference maximum and its rare-path threshold
   float m_my[2], thr_my[2];      // the same for this lane's two head slots
-  float l_acc[2], mid_acc[2][4]; // this lane's slots: sum p, sum p * min per value group
-  float smax[4];
+  float l_acc[2];                // sum p of this lane's head slots
+  float mid_acc[4][2];           // sum p * min, heads 0..3 x this lane's groups 2q, 2q + 1
+  float smax[4];                 // per group: scales up to this keep p * scale * 2^E in fp16 range
   int E_w[4];
+  float smax_my[2], ef_my[2];    // smax and 2^E of this lane's groups
   float D[8][4];
   uint32_t bq[4][2];             // score-MMA query operand of this segment
-  float vl_my[2], dl_my[2];
-  int sq_my[2];
+  float vl_my[2], dl4_my[2], kq_my[2];
   auto reset = [&]() {
     #pragma unroll
     for (int h = 0; h < G; ++h) {
@@ -334,9 +342,11 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsPara
       m_my[e] = kNoMax;
       thr_my[e] = kNoMax;
       l_acc[e] = 0.0f;
-      #pragma unroll
-      for (int g = 0; g < 4; ++g) mid_acc[e][g] = 0.0f;
+      smax_my[e] = 0.0f;
+      ef_my[e] = exp2i(kNoExp);
     }
+    #pragma unroll
+    for (int h = 0; h < 4; ++h) mid_acc[h][0] = mid_acc[h][1] = 0.0f;
     #pragma unroll
     for (int g = 0; g < 4; ++g) {
       smax[g] = 0.0f;
@@ -354,31 +364,32 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsPara
   // this at the same chunk.
   auto part_of = [&](int w) { return reinterpret_cast<float*>(smem + kStages * kStageBytes + w * kBRowsPerWarp); };
   auto flush = [&](int seg) {
-    float v[2][5];
+    float v[10];  // l of the own head slots, then mid[head][own group]
+    v[0] = l_acc[0];
+    v[1] = l_acc[1];
     #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      v[e][0] = l_acc[e];
-      #pragma unroll
-      for (int g = 0; g < 4; ++g) v[e][1 + g] = mid_acc[e][g];
+    for (int h = 0; h < 4; ++h) {
+      v[2 + 2 * h] = mid_acc[h][0];
+      v[3 + 2 * h] = mid_acc[h][1];
     }
     #pragma unroll
-    for (int m = 16; m >= 2; m >>= 1)  // lanes with the same t & 1 hold the same head slots
+    for (int m = 16; m >= 2; m >>= 1)  // lanes with the same t & 1 hold the same slots and groups
       #pragma unroll
-      for (int e = 0; e < 2; ++e)
-        #pragma unroll
-        for (int k = 0; k < 5; ++k) v[e][k] += __shfl_xor_sync(kFull, v[e][k], m);
+      for (int k = 0; k < 10; ++k) v[k] += __shfl_xor_sync(kFull, v[k], m);
     float* mine = part_of(warp);  // this warp's P.V is done with its B rows
-    if (lane < 2) {
+    if (lane < 2) {  // lane q: head slots 2q, 2q + 1 and value groups 2q, 2q + 1
       #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const int h = 2 * lane + e;
         if (h < G) {
-          float* r = mine + h * kRowF;
-          r[0] = m_my[e] == kNoMax ? -INFINITY : m_my[e];
-          r[1] = v[e][0];
-          #pragma unroll
-          for (int g = 0; g < 4; ++g) r[2 + g] = v[e][1 + g];
+          mine[h * kRowF] = m_my[e] == kNoMax ? -INFINITY : m_my[e];
+          mine[h * kRowF + 1] = v[e];
         }
+      }
+      #pragma unroll
+      for (int h = 0; h < G; ++h) {
+        mine[h * kRowF + 2 + 2 * lane] = v[2 + 2 * h];
+        mine[h * kRowF + 3 + 2 * lane] = v[3 + 2 * h];
       }
     }
     if (t4 < G) {  // D columns 2 t4, 2 t4 + 1 = head t4, hi and lo parts
@@ -458,9 +469,10 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsPara
     for (int e = 0; e < 2; ++e) {
       const int h = hs0 + e;
       const bool ok = h < G;
+      const float dl = ok ? s_dl[par][ok ? h : 0] : 0.0f;
       vl_my[e] = ok ? s_vl[par][ok ? h : 0] : 0.0f;
-      dl_my[e] = ok ? s_dl[par][ok ? h : 0] : 0.0f;
-      sq_my[e] = ok ? s_sq[par][ok ? h : 0] : 0;
+      dl4_my[e] = 0.25f * dl;
+      kq_my[e] = -dl * static_cast<float>(ok ? s_sq[par][ok ? h : 0] : 0);
     }
   };
 
@@ -490,35 +502,35 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsPara
     // ---------------- scores: one integer MMA chain per tile, then lane (g, t) takes its token's
     // two head slots and Bc from the accumulator columns (heads in columns 0..3, Bc in 4..7)
     bool valid[kWarpTiles];
-    float s2[kWarpTiles][2], sc[kWarpTiles][4], mid[kWarpTiles][4];
+    float s2[kWarpTiles][2], sc[kWarpTiles][2], mid[kWarpTiles][2];
     #pragma unroll
     for (int kk = 0; kk < kWarpTiles; ++kk) {
       const int tt = kk * 16 + tokr;  // token within the warp slice
       valid[kk] = tt < lim;
       const uint32_t* kbits = reinterpret_cast<const uint32_t*>(st + kOffBits + warp * kWarpTok * 16) + kk * 64 + t4;
       int d[4];
-      score_tile(d, kbits[g8 * 4], kbits[(g8 + 8) * 4], bq);
+      score_tile(d, kbits[row_lo * 4], kbits[row_hi * 4], bq);
       const int x0 = __shfl_xor_sync(kFull, d[0], 2);
       const int x2 = __shfl_xor_sync(kFull, d[2], 2);
       const int x3 = __shfl_xor_sync(kFull, d[3], 2);
       const int a0 = upper ? x2 : d[0], a1 = upper ? x3 : d[1], bc8 = upper ? d[2] : x0;
       const float nc = __fmul_rn(__fmul_rn(reinterpret_cast<const float*>(st + kOffNorm)[kWarpTok * warp + tt],
                                            reinterpret_cast<const float*>(st + kOffCinv)[kWarpTok * warp + tt]), qsl);
-      const float i1 = i2f_exact((bc8 >> 2) - kD);  // 2 Bc - 128
+      // the accumulators hold 8 A and 8 Bc: dot = (delta / 4) 8A + (vl (2 Bc - 128) - delta Sq)
+      const float i1 = __fmaf_rn(0.25f, __int2float_rn(bc8), -128.0f);
       const int aa[2] = {a0, a1};
       #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        const float dot = __fmaf_rn(vl_my[e], i1, __fmul_rn(dl_my[e], i2f_exact((aa[e] >> 2) - sq_my[e])));
+        const float dot = __fmaf_rn(dl4_my[e], __int2float_rn(aa[e]), __fmaf_rn(vl_my[e], i1, kq_my[e]));
         s2[kk][e] = (valid[kk] && hs0 + e < G) ? __fmul_rn(dot, nc) : -INFINITY;
       }
-      const uint4 smv = *reinterpret_cast<const uint4*>(st + kOffSm + (kWarpTok * warp + tt) * 16);
-      // invalid tokens may read a stage slot never filled: their (scale, min) become zeros
-      const uint32_t smw[4] = {valid[kk] ? smv.x : 0u, valid[kk] ? smv.y : 0u, valid[kk] ? smv.z : 0u,
-                               valid[kk] ? smv.w : 0u};
+      // (scale, min) of this lane's two groups; invalid tokens may read a stage slot never filled
+      const uint2 smv = *reinterpret_cast<const uint2*>(st + kOffSm + (kWarpTok * warp + tt) * 16 + q1 * 8);
+      const uint32_t smw[2] = {valid[kk] ? smv.x : 0u, valid[kk] ? smv.y : 0u};
       #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        sc[kk][g] = __half2float(__ushort_as_half(static_cast<unsigned short>(smw[g] & 0xffffu)));
-        mid[kk][g] = __half2float(__ushort_as_half(static_cast<unsigned short>(smw[g] >> 16)));
+      for (int j = 0; j < 2; ++j) {
+        sc[kk][j] = __half2float(__ushort_as_half(static_cast<unsigned short>(smw[j] & 0xffffu)));
+        mid[kk][j] = __half2float(__ushort_as_half(static_cast<unsigned short>(smw[j] >> 16)));
       }
     }
 
@@ -530,7 +542,7 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsPara
       #pragma unroll
       for (int e = 0; e < 2; ++e) rare |= s2[kk][e] > thr_my[e];
       #pragma unroll
-      for (int g = 0; g < 4; ++g) rare |= sc[kk][g] > smax[g];
+      for (int j = 0; j < 2; ++j) rare |= sc[kk][j] > smax_my[j];
     }
     if (__any_sync(kFull, rare)) {
       float lm[2];
@@ -550,12 +562,9 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsPara
           const float alpha = ex2(m_w[h] - mx);  // 0 while m_w is still kNoMax
           m_w[h] = mx;
           m_thr[h] = mx + kTau;
-          if (hs0 == (h & ~1)) {
-            const int e = h & 1;
-            l_acc[e] = __fmul_rn(l_acc[e], alpha);
-            #pragma unroll
-            for (int g = 0; g < 4; ++g) mid_acc[e][g] = __fmul_rn(mid_acc[e][g], alpha);
-          }
+          if (hs0 == (h & ~1)) l_acc[h & 1] = __fmul_rn(l_acc[h & 1], alpha);
+          mid_acc[h][0] = __fmul_rn(mid_acc[h][0], alpha);
+          mid_acc[h][1] = __fmul_rn(mid_acc[h][1], alpha);
           const float f = (t4 == h) ? alpha : 1.0f;
           #pragma unroll
           for (int mt = 0; mt < 8; ++mt)
@@ -574,9 +583,11 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsPara
       }
       #pragma unroll
       for (int g = 0; g < 4; ++g) {
-        float mx = sc[0][g];
-        #pragma unroll
-        for (int kk = 1; kk < kWarpTiles; ++kk) mx = fmaxf(mx, sc[kk][g]);
+        float mx = 0.0f;  // lanes holding group g contribute their scales
+        if (q1 == (g >> 1)) {
+          #pragma unroll
+          for (int kk = 0; kk < kWarpTiles; ++kk) mx = fmaxf(mx, sc[kk][g & 1]);
+        }
         #pragma unroll
         for (int m = 16; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
         if (mx > smax[g]) {  // warp-uniform
@@ -593,6 +604,11 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsPara
           }
         }
       }
+      #pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        smax_my[j] = q1 ? smax[2 + j] : smax[j];
+        ef_my[j] = exp2i(q1 ? E_w[2 + j] : E_w[j]);
+      }
     }
     #pragma unroll
     for (int kk = 0; kk < kWarpTiles; ++kk) {
@@ -601,24 +617,37 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsPara
       for (int e = 0; e < 2; ++e) {
         pr[e] = ex2(s2[kk][e] - m_my[e]);  // -inf for invalid tokens and empty slots -> 0
         l_acc[e] = __fadd_rn(l_acc[e], pr[e]);
-        #pragma unroll
-        for (int g = 0; g < 4; ++g) mid_acc[e][g] = __fmaf_rn(pr[e], mid[kk][g], mid_acc[e][g]);
       }
-      // this token's B rows, columns (head, hi/lo) of its two head slots:
-      // [group][token][8 halves], this lane writes halves 4 (t & 1) .. 4 (t & 1) + 3
+      // p of all four heads for this token: heads 0, 1 from the pair's even lane, 2, 3 from the odd
+      float ph[4];
+      ph[0] = __shfl_sync(kFull, pr[0], lane & ~1);
+      ph[1] = __shfl_sync(kFull, pr[1], lane & ~1);
+      ph[2] = G > 2 ? __shfl_sync(kFull, pr[0], lane | 1) : 0.0f;
+      ph[3] = G > 2 ? __shfl_sync(kFull, pr[1], lane | 1) : 0.0f;
       #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const float f = __fmul_rn(sc[kk][g], exp2i(E_w[g]));
-        const uint64_t w2 = mul2(f2pack(pr[0], pr[1]), f2pack(f, f));
-        const uint64_t hi2 = w2 & 0xFFFFE000FFFFE000ull;  // 11 significant bits each
-        const uint64_t lo2 = sub2(w2, hi2);
-        uint32_t r0, r1;
-        asm("cvt.rn.f16x2.f32 %0, %1, %2;" : "=r"(r0) : "f"(__uint_as_float(static_cast<uint32_t>(lo2))),
-            "f"(__uint_as_float(static_cast<uint32_t>(hi2))));
-        asm("cvt.rn.f16x2.f32 %0, %1, %2;"
-            : "=r"(r1)
-            : "f"(__uint_as_float(static_cast<uint32_t>(lo2 >> 32))), "f"(__uint_as_float(static_cast<uint32_t>(hi2 >> 32))));
-        *reinterpret_cast<uint2*>(brows + (g * kWarpTok + kk * 16 + tokr) * 16 + (t4 & 1) * 8) = make_uint2(r0, r1);
+      for (int h = 0; h < G; ++h) {
+        mid_acc[h][0] = __fmaf_rn(ph[h], mid[kk][0], mid_acc[h][0]);
+        mid_acc[h][1] = __fmaf_rn(ph[h], mid[kk][1], mid_acc[h][1]);
+      }
+      // this token's B rows of the lane's two groups: 8 halves (head, hi/lo)
+      #pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const float f = __fmul_rn(sc[kk][j], ef_my[j]);
+        uint32_t row[4];
+        #pragma unroll
+        for (int hp = 0; hp < 2; ++hp) {
+          const uint64_t w2 = mul2(f2pack(ph[2 * hp], ph[2 * hp + 1]), f2pack(f, f));
+          const uint64_t hi2 = w2 & 0xFFFFE000FFFFE000ull;  // 11 significant bits each
+          const uint64_t lo2 = sub2(w2, hi2);
+          asm("cvt.rn.f16x2.f32 %0, %1, %2;"
+              : "=r"(row[2 * hp])
+              : "f"(__uint_as_float(static_cast<uint32_t>(lo2))), "f"(__uint_as_float(static_cast<uint32_t>(hi2))));
+          asm("cvt.rn.f16x2.f32 %0, %1, %2;"
+              : "=r"(row[2 * hp + 1])
+              : "f"(__uint_as_float(static_cast<uint32_t>(lo2 >> 32))), "f"(__uint_as_float(static_cast<uint32_t>(hi2 >> 32))));
+        }
+        *reinterpret_cast<uint4*>(brows + ((2 * q1 + j) * kGroupRows + kk * 16 + tokr) * 16) =
+            make_uint4(row[0], row[1], row[2], row[3]);
       }
     }
     __syncwarp();
@@ -632,7 +661,7 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsPara
         if (kk < my_tiles) {
           uint32_t bf[4][2];
           #pragma unroll
-          for (int g = 0; g < 4; ++g) ldsm_x2_trans(bf[g][0], bf[g][1], bbase + (g * kWarpTok + kk * 16) * 16);
+          for (int g = 0; g < 4; ++g) ldsm_x2_trans(bf[g][0], bf[g][1], bbase + (g * kGroupRows + kk * 16) * 16);
           #pragma unroll
           for (int mt = 0; mt < 8; ++mt) {
             uint32_t a[4];
