@@ -154,26 +154,25 @@ def dist_setup():
     return world, rank, local
 
 
-def reduce_max(x: float, world: int) -> float:
+def _all_reduce(x: float, world: int, op_name: str) -> float:
+    """All-reduce one float over the ranks (on the GPU under NCCL, on the host under gloo)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
 
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=getattr(dist.ReduceOp, op_name))
     return float(t.item())
+
+
+def reduce_max(x: float, world: int) -> float:
+    return _all_reduce(x, world, "MAX")
 
 
 def reduce_sum(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch
-    import torch.distributed as dist
-
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
-    dist.all_reduce(t, op=dist.ReduceOp.SUM)
-    return float(t.item())
+    return _all_reduce(x, world, "SUM")
 
 
 def barrier(world: int):
