@@ -36,8 +36,8 @@ ATTEND_SRC = os.path.join(ROOT, "long_context_decode_kv1b_b200", "csrc", "kv1b_a
 # DRAM bytes (read + write) per token x kv-head of one attend kernel launch, from an ncu capture of
 # the c3 workload (same head grouping, cache 218 MB > L2) scaled by the tokens x kv-heads it
 # processed; valid only for the attend source with this SHA-256 (profiles/attend_ws_c3_ncu_full.txt).
-TRAFFIC = {"bytes_per_token_head": 222420480 / 2097408,
-           "source_sha256": "78e51c26d081d32adf9a5ce16b4bada5eb982ff9e5cc00e28775c851940079d6"}
+TRAFFIC = {"bytes_per_token_head": 223290112 / 2097408,
+           "source_sha256": "b7de00c40f372ec09d87bba489129348bcd95d0d488806f6859558eba76c8d2a"}
 
 
 def parse_args():
