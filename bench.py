@@ -347,11 +347,11 @@ def run_ours(args):
                              (bytes_per_attend / 1e6), "parallelism": f"independent sequence per GPU x{world}"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic_per_launch(cfg.B * cfg.Hkv * L_mean),
-                         "kernel": "kv1b_attend: attend_ws_kernel + merge_ws_kernel, CUDA events around both",
+                         "kernel": "kv1b_attend: counter memset + attend_ws_kernel (merge fused), CUDA events around both",
                          "attend_us": att_avg * 1e3, "peak_kind": peak_kind,
                          "frac_of_8tbs": achieved / 8000.0},
             "e2e": e2e,
-            "gpu_launches": 3 * K,
+            "gpu_launches": 2 * K,  # encode + attend per step (plus one 32-byte counter memset)
             "clocks": clocks,
         }
         if alt:

@@ -104,6 +104,16 @@ size_t ws_bytes_needed(const kv1b_cache_t* c, int32_t num_q_heads) {
   return static_cast<size_t>(c->batch) * c->num_kv_heads * pieces * G * kv1b::kPartStride * 4;
 }
 
+// kv1b_attend's workspace: the partial rows of either attend kernel, then one merge counter per
+// (sequence, kv-head) for the persistent kernel.
+size_t ws_counter_bytes(const kv1b_cache_t* c) { return sizeof(unsigned) * c->batch * c->num_kv_heads; }
+size_t ws_counters_offset(const kv1b_cache_t* c, int32_t num_q_heads) {
+  const size_t rows = static_cast<size_t>(c->batch) * num_q_heads;
+  const size_t split_bytes = rows * static_cast<size_t>(max_splits(c)) * kv1b::kPartStride * 4;
+  const size_t ws = ws_bytes_needed(c, num_q_heads);
+  return align_up(split_bytes > ws ? split_bytes : ws);
+}
+
 bool equal_lengths(const kv1b_cache_t* c) {
   for (int b = 1; b < c->batch; ++b)
     if (c->h_lengths[b] != c->h_lengths[0]) return false;
@@ -194,11 +204,7 @@ int kv1b_encode_append(kv1b_cache_t* cache, const void* k, const void* v, int32_
 size_t kv1b_attend_workspace_bytes(const kv1b_cache_t* cache, int32_t num_q_heads, int32_t mode) {
   if (!cache_ok(cache) || heads_check(cache, num_q_heads) != KV1B_OK) return 0;
   const size_t rows = static_cast<size_t>(cache->batch) * num_q_heads;
-  if (mode == 0) {
-    const size_t split_bytes = rows * static_cast<size_t>(max_splits(cache)) * kv1b::kPartStride * 4;
-    return align_up(split_bytes > ws_bytes_needed(cache, num_q_heads) ? split_bytes
-                                                                      : ws_bytes_needed(cache, num_q_heads));
-  }
+  if (mode == 0) return ws_counters_offset(cache, num_q_heads) + align_up(ws_counter_bytes(cache));
   if (mode == 1) return align_up(rows * static_cast<size_t>(cache->capacity) * 4);
   return 0;
 }
@@ -231,12 +237,13 @@ int kv1b_attend(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32
     kv1b_ws_plan(cache->batch, cache->num_kv_heads, G, cache->capacity, num_sms(), &Tc, &Ltc, &nc, &pieces_cap);
     w.ncta = ncta;
     w.max_pieces = pieces_cap > pieces ? pieces_cap : pieces;
-    if (w.max_pieces > 256 ||
-        static_cast<size_t>(cache->batch) * cache->num_kv_heads * w.max_pieces * G * kv1b::kPartStride * 4 > ws_bytes)
+    if (w.max_pieces > 256 || static_cast<size_t>(cache->batch) * cache->num_kv_heads * w.max_pieces * G *
+                                      kv1b::kPartStride * 4 > ws_counters_offset(cache, num_q_heads))
       return KV1B_ERR_WORKSPACE;
     w.part = static_cast<float*>(ws);
     w.out = out;
     w.status = cache->d_status;
+    w.counters = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + ws_counters_offset(cache, num_q_heads));
     return cuda_status(kv1b_launch_attend_ws(w, G, static_cast<cudaStream_t>(stream)));
   }
   kv1b::AttendParams p;

@@ -25,8 +25,8 @@
 //   weights from the sketch, then the 4-bit values).  value = min + scale * code, the min term is
 //   summed per (head, group) in fp32 by the score lanes.
 // At the end of a segment piece the 8 warps' partials are combined in shared memory and the CTA
-// writes one row (m, l, o[128]) per query head; a merge kernel combines the CTA rows of a head
-// by log-sum-exp.
+// writes one row (m, l, o[128]) per query head; the CTA that writes a segment's last row merges
+// the segment's rows by log-sum-exp into the output (one kernel per attend).
 //
 // Every mbarrier wait is bounded: a wait that runs out sets KV1B_STATUS_TIMEOUT in the cache's
 // status word; the CTA then stops issuing copies, later waits return at once, and thread 0
@@ -262,6 +262,7 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsPara
   __shared__ float s_vl[2][G], s_dl[2][G];
   __shared__ int s_sq[2][G];
   __shared__ volatile int s_abort;
+  __shared__ int s_merge;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const CacheView& c = p.c;
@@ -363,6 +364,59 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsPara
   // row (m, l, o[128] with the mid term folded in) for slot (segment, piece).  Every warp reaches
   // this at the same chunk.
   auto part_of = [&](int w) { return reinterpret_cast<float*>(smem + kStages * kStageBytes + w * kBRowsPerWarp); };
+
+  // Log-sum-exp merge of the n CTA rows of segment `seg` (per query head) into the output; the
+  // CTA's shared partials are free by now and hold the piece maxima, sums and weights.  All heads
+  // at once: thread t takes channel t & 127 of heads (t >> 7) + 2i, with the pieces' loads
+  // independent of one another.
+  static_assert(kThreads == 256, "two threads per channel in the merge");
+  auto merge_segment = [&](int seg, int n) {
+    float* sm_m = part_of(0);       // [G][256] piece maxima, then weights
+    float* sm_l = sm_m + 4 * 256;   // [G][256] piece sums
+    float* sm_d = sm_l + 4 * 256;   // [G] denominators
+    const int b = seg / c.Hkv, kvh = seg - b * c.Hkv;
+    const int64_t stride = static_cast<int64_t>(G) * kPartStride;  // between pieces
+    const float* base = p.part + static_cast<int64_t>(seg) * p.max_pieces * G * kPartStride;
+    for (int i = threadIdx.x; i < G * n; i += kThreads) {
+      const int h = i / n, k = i - h * n;
+      sm_m[h * 256 + k] = base[k * stride + h * kPartStride];
+      sm_l[h * 256 + k] = base[k * stride + h * kPartStride + 1];
+    }
+    named_bar(1, kThreads);
+    if (warp < G) {
+      float* mw = sm_m + warp * 256;
+      const float* lw = sm_l + warp * 256;
+      float M = -INFINITY;
+      for (int k = lane; k < n; k += 32) M = fmaxf(M, mw[k]);
+      #pragma unroll
+      for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, m));
+      float den = 0.0f;
+      for (int k = lane; k < n; k += 32) {
+        const float wt = (mw[k] == -INFINITY || M == -INFINITY) ? 0.0f : exp2f(mw[k] - M);
+        den = __fmaf_rn(wt, lw[k], den);
+        mw[k] = wt;
+      }
+      #pragma unroll
+      for (int m = 16; m >= 1; m >>= 1) den += __shfl_xor_sync(kFull, den, m);
+      if (lane == 0) sm_d[warp] = den;
+    }
+    named_bar(1, kThreads);
+    const int ch = threadIdx.x & 127;
+    for (int h = threadIdx.x >> 7; h < G; h += 2) {
+      const float* w = sm_m + h * 256;
+      const float* o = base + h * kPartStride + 2 + ch;
+      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      int k = 0;
+      for (; k + 4 <= n; k += 4) {
+        #pragma unroll
+        for (int u = 0; u < 4; ++u) acc[u] = __fmaf_rn(w[k + u], o[(k + u) * stride], acc[u]);
+      }
+      for (; k < n; ++k) acc[0] = __fmaf_rn(w[k], o[k * stride], acc[0]);
+      const float den = sm_d[h];
+      p.out[(static_cast<int64_t>(b) * p.Hq + kvh * G + h) * kD + ch] =
+          den > 0.0f ? __fdiv_rn(__fadd_rn(__fadd_rn(acc[0], acc[1]), __fadd_rn(acc[2], acc[3])), den) : 0.0f;
+    }
+  };
   auto flush = [&](int seg) {
     float v[10];  // l of the own head slots, then mid[head][own group]
     v[0] = l_acc[0];
@@ -425,6 +479,22 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsPara
         row[1] = den;
       }
       row[2 + ch] = num;
+    }
+    // The CTA that writes a segment's last piece merges the segment: ticket after the rows are
+    // visible device-wide (the counters are zeroed on the stream before the launch).
+    __threadfence();
+    named_bar(1, kThreads);
+    if (threadIdx.x == 0) {
+      const int64_t c0 = cta_of_tile(wk, static_cast<int64_t>(seg) * wk.Lt);
+      const int64_t c1 = cta_of_tile(wk, static_cast<int64_t>(seg + 1) * wk.Lt - 1);
+      const unsigned n = static_cast<unsigned>(c1 - c0 + 1);
+      s_merge = (atomicAdd(p.counters + seg, 1u) == n - 1u) ? static_cast<int>(n) : 0;
+    }
+    named_bar(1, kThreads);
+    const int npieces = s_merge;
+    if (npieces > 0) {
+      __threadfence();
+      merge_segment(seg, npieces);
     }
     named_bar(1, kThreads);  // the shared partials may be rewritten by the next flush
   };
@@ -690,62 +760,6 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsPara
   if (s_abort && lane == 0) atomicOr(p.status, KV1B_STATUS_TIMEOUT);
 }
 
-// Merge: one block of 128 threads (channels) per (b, hq): log-sum-exp over the CTA pieces of the
-// query head's segment.  Row maxima and weights are formed in parallel, then every channel sums
-// the pieces with independent loads.
-__global__ void __launch_bounds__(128) merge_ws_kernel(const AttendWsParams p, int G) {
-  __shared__ float s_w[256];
-  __shared__ float s_red[4];
-  const int row = blockIdx.x;  // b * Hq + hq
-  const int b = row / p.Hq, hq = row - b * p.Hq;
-  const int kvh = hq / G, h = hq - kvh * G;
-  const int seg = b * p.c.Hkv + kvh;
-  const Work wk{p.T, p.Lt, p.ncta};
-  float* out = p.out + static_cast<int64_t>(row) * kD;
-  if (p.Lt == 0 || p.T == 0) {
-    out[threadIdx.x] = 0.0f;
-    return;
-  }
-  const int64_t c0 = cta_of_tile(wk, static_cast<int64_t>(seg) * wk.Lt);
-  const int64_t c1 = cta_of_tile(wk, static_cast<int64_t>(seg + 1) * wk.Lt - 1);
-  const int n = static_cast<int>(c1 - c0 + 1);  // <= max_pieces <= 256 (host-checked)
-  const float* base = p.part + (static_cast<int64_t>(seg) * p.max_pieces * G + h) * kPartStride;
-  const int stride = G * kPartStride;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  float mk[2], lk[2];
-  float M = -INFINITY;
-  #pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int k = threadIdx.x + 128 * u;
-    mk[u] = k < n ? base[static_cast<int64_t>(k) * stride] : -INFINITY;
-    lk[u] = k < n ? base[static_cast<int64_t>(k) * stride + 1] : 0.0f;
-    M = fmaxf(M, mk[u]);
-  }
-  #pragma unroll
-  for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, m));
-  if (lane == 0) s_red[warp] = M;
-  __syncthreads();
-  M = fmaxf(fmaxf(s_red[0], s_red[1]), fmaxf(s_red[2], s_red[3]));
-  __syncthreads();
-  float den = 0.0f;
-  #pragma unroll
-  for (int u = 0; u < 2; ++u) {
-    const int k = threadIdx.x + 128 * u;
-    const float wt = (k < n && mk[u] != -INFINITY && M != -INFINITY) ? exp2f(mk[u] - M) : 0.0f;
-    if (k < n) s_w[k] = wt;
-    den = __fmaf_rn(wt, lk[u], den);
-  }
-  #pragma unroll
-  for (int m = 16; m >= 1; m >>= 1) den += __shfl_xor_sync(0xffffffffu, den, m);
-  if (lane == 0) s_red[warp] = den;
-  __syncthreads();
-  den = (s_red[0] + s_red[1]) + (s_red[2] + s_red[3]);
-  float num = 0.0f;
-  #pragma unroll 8
-  for (int k = 0; k < n; ++k) num = __fmaf_rn(s_w[k], base[static_cast<int64_t>(k) * stride + 2 + threadIdx.x], num);
-  out[threadIdx.x] = den > 0.0f ? __fdiv_rn(num, den) : 0.0f;
-}
-
 template <int G>
 static cudaError_t launch_t(const AttendWsParams& p, cudaStream_t stream) {
   static bool configured = false;
@@ -754,10 +768,9 @@ static cudaError_t launch_t(const AttendWsParams& p, cudaStream_t stream) {
     if (e != cudaSuccess) return e;
     configured = true;
   }
-  attend_ws_kernel<G><<<p.ncta, kBlock, kSmemBytes, stream>>>(p);
-  cudaError_t e = cudaGetLastError();
+  cudaError_t e = cudaMemsetAsync(p.counters, 0, sizeof(unsigned) * p.c.B * p.c.Hkv, stream);
   if (e != cudaSuccess) return e;
-  merge_ws_kernel<<<p.c.B * p.Hq, 128, 0, stream>>>(p, G);
+  attend_ws_kernel<G><<<p.ncta, kBlock, kSmemBytes, stream>>>(p);
   return cudaGetLastError();
 }
 
@@ -781,8 +794,6 @@ void kv1b_ws_plan(int32_t B, int32_t Hkv, int32_t G, int64_t L, int num_sms, int
   *max_pieces = tot > 0 ? static_cast<int>((lt * n + tot - 1) / tot + 1) : 1;
   (void)G;
 }
-
-int kv1b_ws_rows_per_piece() { return ws::kWarps; }
 
 cudaError_t kv1b_launch_attend_ws(const AttendWsParams& p, int32_t G, cudaStream_t stream) {
   switch (G) {

@@ -87,6 +87,7 @@ struct AttendWsParams {
   float* part;         // [segments][max_pieces][warps][G][6 + 128]: m, l, mid[4], o[128]
   float* out;          // [B][Hq][128]
   int32_t* status;     // cache status word (timeout flag)
+  unsigned* counters;  // [B * Hkv] pieces of each segment written so far (zeroed before the launch)
 };
 constexpr int kPartStrideWs = 6 + 128;
 
@@ -103,7 +104,6 @@ cudaError_t kv1b_launch_scores(const kv1b::ScoresParams& p, int32_t G, int32_t m
 cudaError_t kv1b_launch_topp(const kv1b::ToppParams& p, cudaStream_t stream);
 int kv1b_pick_splits(int32_t B, int32_t Hkv, int64_t max_len, int num_sms);
 bool kv1b_ws_supported(int32_t G);
-int kv1b_ws_rows_per_piece();
 void kv1b_ws_plan(int32_t B, int32_t Hkv, int32_t G, int64_t L, int num_sms, int64_t* T, int64_t* Lt, int* ncta,
                   int* max_pieces);
 cudaError_t kv1b_launch_attend_ws(const kv1b::AttendWsParams& p, int32_t G, cudaStream_t stream);
