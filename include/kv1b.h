@@ -61,8 +61,10 @@ extern "C" {
 #define KV1B_DTYPE_F16 2
 
 /* kv1b_attend flags: which engine forms the probability-weighted sum of values */
-#define KV1B_ATTEND_TENSOR 0     /* default: mma.sync (f16 codes x hi/lo-split f16 weights, fp32 accumulate) */
-#define KV1B_ATTEND_CUDA_CORE 1  /* fp32 FMA on the CUDA cores */
+#define KV1B_ATTEND_TENSOR 0     /* default: integer mma.sync (u8 codes x 23-bit fixed-point weights, exact s32
+                                    accumulation) in a persistent kernel, for G in {1, 2, 4}, equal sequence
+                                    lengths and an automatic split count; other shapes run the CUDA-core engine */
+#define KV1B_ATTEND_CUDA_CORE 1  /* fp32 FMA on the CUDA cores (split-K grid, any shape) */
 
 /* status word bits (kv1b_read_status) */
 #define KV1B_STATUS_NONFINITE 1       /* a K or V element appended was NaN or Inf */
@@ -75,12 +77,10 @@ extern "C" {
  *   k_bits  u32 [batch][hkv][capacity][4]     sign bits of the rotated key (16 B / token)
  *   k_norm  f32 [batch][hkv][capacity]        N = ||k|| (fixed pairwise tree sum of squares)
  *   k_cinv  f32 [batch][hkv][capacity]        1/C = 128 N / sum_i |y_i| (1 when the sum is 0)
- *   v_codes u32 [batch][hkv][capacity/16][8][32]  4-bit value codes in 16-token tiles; for tile T,
- *           m-tile mt (channels 16mt..16mt+15) and lane l (g = l>>2, t = l&3) the word holds
- *           bits 0-3 / 16-19:  channel 16mt+g,   tokens 16T+2t / 16T+2t+1
- *           bits 4-7 / 20-23:  channel 16mt+g+8, tokens 16T+2t / 16T+2t+1
- *           bits 8-11 / 24-27: channel 16mt+g,   tokens 16T+2t+8 / 16T+2t+9
- *           bits 12-15 / 28-31: channel 16mt+g+8, tokens 16T+2t+8 / 16T+2t+9
+ *   v_codes u32 [batch][hkv][capacity/128][128][16]  4-bit value codes in 128-token tiles, one
+ *           64-byte row per channel: nibble j (bits 4j..4j+3) of word w of row (tile T, channel c)
+ *           is the code of token 128T + 8w + j, channel c.  One tile is one TMA box of 4-bit
+ *           elements that the tensor-core engine expands to a byte per code in shared memory.
  *   v_sm    u32 [batch][hkv][capacity][4]     per 32-channel group: low half = fp16 scale,
  *           high half = fp16 min; value = min + scale * code
  *   signs   f32 [128]                         rotation signs D (+-1)

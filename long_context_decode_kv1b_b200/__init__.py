@@ -138,7 +138,7 @@ class Cache:
             "k_bits": self._view(d.k_bits, torch.int32, (B, H, C, 4)),
             "k_norm": self._view(d.k_norm, torch.float32, (B, H, C)),
             "k_cinv": self._view(d.k_cinv, torch.float32, (B, H, C)),
-            "v_codes": self._view(d.v_codes, torch.int32, (B, H, C // 16, 8, 32)),
+            "v_codes": self._view(d.v_codes, torch.int32, (B, H, C // 128, HEAD_DIM, 16)),
             "v_sm": self._view(d.v_sm, torch.int32, (B, H, C, 4)),
             "signs": self._view(d.signs, torch.float32, (HEAD_DIM,)),
             "lengths": self._view(d.d_lengths, torch.int32, (B,)),
@@ -237,20 +237,13 @@ def attend_from_host(cache: Cache, q_host: torch.Tensor, k_new_host: torch.Tenso
 
 
 def unpack_codes(v_codes: torch.Tensor, length: int) -> torch.Tensor:
-    """Logical codes [length, 128] (uint8) of one (sequence, kv-head) from the tiled v_codes plane
-    [capacity/16, 8, 32] (layout in include/kv1b.h)."""
-    w = v_codes.to(torch.int64) & 0xFFFFFFFF
-    ntile = (length + 15) // 16
+    """Logical codes [length, 128] (uint8) of one (sequence, kv-head) from the code plane
+    [capacity/128, 128, 16] (128-token tiles, channel-major rows; nibble j of word w of a row is
+    token 8w + j of the tile; layout in include/kv1b.h)."""
+    w = v_codes.to(torch.int64) & 0xFFFFFFFF                       # [tiles, 128 ch, 16 words]
+    ntile = (length + 127) // 128
     w = w[:ntile]
-    out = torch.zeros((ntile * 16, HEAD_DIM), dtype=torch.uint8, device=w.device)
-    lanes = torch.arange(32, device=w.device)
-    g, t = lanes // 4, lanes % 4
-    slots = [(0, 0, 0), (16, 0, 1), (4, 8, 0), (20, 8, 1), (8, 0, 8), (24, 0, 9), (12, 8, 8), (28, 8, 9)]
-    tiles = torch.arange(ntile, device=w.device)
-    for mt in range(8):
-        for shift, choff, toff in slots:
-            nib = ((w[:, mt, :] >> shift) & 0xF).to(torch.uint8)             # [ntile, 32]
-            tok = tiles[:, None] * 16 + (2 * t)[None, :] + toff                 # [ntile, 32]
-            ch = (16 * mt + g + choff)[None, :].expand_as(tok)
-            out[tok.reshape(-1), ch.reshape(-1)] = nib.reshape(-1)
-    return out[:length]
+    shifts = torch.arange(8, device=w.device, dtype=torch.int64) * 4
+    nib = (w[..., None] >> shifts) & 0xF                             # [tiles, 128 ch, 16 words, 8]
+    out = nib.permute(0, 2, 3, 1).reshape(ntile * 128, HEAD_DIM)     # token = 128 tile + 8 word + j
+    return out[:length].to(torch.uint8)

@@ -5,53 +5,20 @@
 //   phase S  (thread = token): binary x INT4 popcount scores of the G query heads of this kv-head
 //            ("RaBitQCache", abstract / key design), online-softmax update in log2 units, and the
 //            per-(token, group, head) weights p * scale written to shared memory;
-//   phase PV (warp = 16-channel m-tile): the probability-weighted sum of the 4-bit values
-//            ("H1B-KV", technical framework: weights from the sketch, then the 4-bit values),
-//            either on the tensor cores (mma.sync m16n8k16: codes are exact fp16 integers c - 8,
-//            weights split into fp16 hi + lo, fp32 accumulation) or on the CUDA cores (fp32 FMA).
+//   phase PV (warp = 16 channels, lane = channel x half of each 16-token step): the
+//            probability-weighted sum of the 4-bit values on the CUDA cores in fp32 ("H1B-KV",
+//            technical framework: weights from the sketch, then the 4-bit values).
 // The dequantised value is min + scale*code = mid + scale*(code - 8) with mid = min + 8 scale;
-// the mid term is accumulated per (head, group) in fp32 by phase S.
+// the mid term is accumulated per (head, group) in fp32 by phase S.  This kernel serves every
+// shape (any G <= 8, unequal lengths, a forced split count); the persistent tensor-core kernel
+// (kv1b_attend_ws.cu) takes the common shapes.
 #include "kv1b_device.cuh"
 #include "kv1b_launch.h"
 
 namespace kv1b {
 
 constexpr int kThreads = 256;  // = tokens per chunk
-constexpr int kNoExp = 1 << 20;
 constexpr float kLog2e = 0x1.715476p+0f;  // log2(e) rounded to fp32
-
-__device__ __forceinline__ void mma16816(float d[4], const uint32_t a[4], const uint32_t b0, const uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ void ldsm_x2_trans(uint32_t& b0, uint32_t& b1, uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];" : "=r"(b0), "=r"(b1) : "r"(addr));
-}
-
-__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-
-// One code word (see the v_codes layout) -> the m16n8k16 A fragment.  Rows g: exact fp16 (c - 8);
-// rows g + 8: exact fp16 16 (c - 8) (their nibbles sit 4 bits higher), undone in the epilogue.
-__device__ __forceinline__ void codes_to_afrag(uint32_t w, uint32_t a[4]) {
-  const uint32_t w8 = w >> 8;
-  a[0] = hsub2((w & 0x000F000Fu) | 0x64006400u, 0x64086408u);   // (1024 + c) - 1032
-  a[1] = hsub2((w & 0x00F000F0u) | 0x64006400u, 0x64806480u);   // (1024 + 16c) - 1152
-  a[2] = hsub2((w8 & 0x000F000Fu) | 0x64006400u, 0x64086408u);
-  a[3] = hsub2((w8 & 0x00F000F0u) | 0x64006400u, 0x64806480u);
-}
-
-__device__ __forceinline__ uint32_t pack_half2(float lo, float hi) {
-  const uint32_t l = __half_as_ushort(__float2half_rn(lo));
-  const uint32_t h = __half_as_ushort(__float2half_rn(hi));
-  return l | (h << 16);
-}
 
 __device__ __forceinline__ float exp2_of_int(int e) { return __int_as_float((e + 127) << 23); }
 
@@ -72,11 +39,9 @@ __device__ __forceinline__ void tile_range(int L, int nsplit, int split, int64_t
   if (tok_begin > tok_end) tok_begin = tok_end;
 }
 
-template <int G, bool TENSOR>
+template <int G>
 __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendParams p) {
-  constexpr int NT = (2 * G + 7) / 8;                       // n-tiles of 8 columns: (head, hi/lo)
-  constexpr int ROWH = TENSOR ? 8 * NT : 2 * G;             // halves (tensor) or 2*floats per row
-  extern __shared__ __align__(16) uint8_t smem_dyn[];       // [4 groups][256 tokens][row]
+  extern __shared__ __align__(16) uint8_t smem_dyn[];       // [4 groups][256 tokens][G] weights p * scale
   __shared__ __align__(16) uint32_t s_planes[G][4][4];
   __shared__ float s_vl[G], s_dl[G];
   __shared__ int s_sq[G];
@@ -125,7 +90,7 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendParams 
   const float* kn = c.k_norm + head_tok;
   const float* kc = c.k_cinv + head_tok;
   const uint4* sm4 = reinterpret_cast<const uint4*>(c.v_sm) + head_tok;
-  const uint32_t* vcw = c.v_codes + head_tok * 16;  // 16 words per token, tile-major
+  const uint32_t* vcw = c.v_codes + head_tok * 16;  // 128-token tiles of [128 channels][16 words]
 
   float m_run[G], l_acc[G], mid_acc[G][4];
   #pragma unroll
@@ -135,19 +100,12 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendParams 
     #pragma unroll
     for (int g = 0; g < 4; ++g) mid_acc[h][g] = 0.0f;
   }
-  int E_run[4] = {kNoExp, kNoExp, kNoExp, kNoExp};
-  float D[NT][4];      // tensor engine accumulators
-  float acc[G][2];     // CUDA-core engine accumulators (2 channels per lane)
+  float acc[G];        // this lane's channel, its half of every 16-token step
   #pragma unroll
-  for (int n = 0; n < NT; ++n)
-    #pragma unroll
-    for (int i = 0; i < 4; ++i) D[n][i] = 0.0f;
-  #pragma unroll
-  for (int h = 0; h < G; ++h) acc[h][0] = acc[h][1] = 0.0f;
+  for (int h = 0; h < G; ++h) acc[h] = 0.0f;
 
   const int gw = warp >> 1;           // value group owned by this warp in phase PV
-  const int g8 = lane >> 2, t4 = lane & 3;
-  const uint32_t smem_base = static_cast<uint32_t>(__cvta_generic_to_shared(smem_dyn));
+  const int ch = 16 * warp + (lane & 15), hf = lane >> 4;
 
   for (int64_t c0 = tok_begin; c0 < tok_end; c0 += kThreads) {
     // ================= phase S: thread = token
@@ -209,40 +167,8 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendParams 
       #pragma unroll
       for (int g = 0; g < 4; ++g) mid_acc[h][g] = __fmaf_rn(pr[h], mid[g], __fmul_rn(mid_acc[h][g], alpha[h]));
     }
-    // per-group power-of-two shift keeping every fp16 weight p*scale*2^E below 2^15
-    float beta[4], shift[4];
-    #pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      int e_new = E_run[g];
-      if (red[G + g] > 0.0f) {
-        const int cand = 14 - ilogbf(red[G + g]);
-        e_new = cand < e_new ? cand : e_new;
-      }
-      beta[g] = (E_run[g] == kNoExp || e_new == E_run[g]) ? 1.0f : exp2_of_int(e_new - E_run[g]);
-      E_run[g] = e_new;
-      shift[g] = (e_new == kNoExp) ? 0.0f : exp2_of_int(e_new);
-    }
     // weights of this token
-    if (TENSOR) {
-      #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        const float f = __fmul_rn(sc[g], shift[g]);
-        uint32_t row[4 * NT];
-        #pragma unroll
-        for (int h = 0; h < 4 * NT; ++h) {
-          if (h < G) {
-            const float w = __fmul_rn(pr[h], f);
-            const float hi = __half2float(__float2half_rn(w));
-            row[h] = pack_half2(hi, __fsub_rn(w, hi));
-          } else {
-            row[h] = 0u;
-          }
-        }
-        uint4* dst = reinterpret_cast<uint4*>(smem_dyn + ((g * kThreads + threadIdx.x) * ROWH) * 2);
-        #pragma unroll
-        for (int n = 0; n < NT; ++n) dst[n] = make_uint4(row[4 * n], row[4 * n + 1], row[4 * n + 2], row[4 * n + 3]);
-      }
-    } else {
+    {
       #pragma unroll
       for (int g = 0; g < 4; ++g) {
         float* dst = reinterpret_cast<float*>(smem_dyn) + (g * kThreads + threadIdx.x) * G;
@@ -251,50 +177,21 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendParams 
       }
     }
     __syncthreads();
-    // ================= phase PV: warp = m-tile (channels 16 warp .. 16 warp + 15)
+    // ================= phase PV: warp = channels 16 warp .. 16 warp + 15; lane = (channel, token half)
     const int nsteps = static_cast<int>((tok_end - c0 + 15) / 16) < 16 ? static_cast<int>((tok_end - c0 + 15) / 16) : 16;
-    const uint32_t* tilew = vcw + (c0 / 16) * 256 + warp * 32 + lane;
-    if (TENSOR) {
+    #pragma unroll
+    for (int h = 0; h < G; ++h) acc[h] = __fmul_rn(acc[h], alpha[h]);
+    const float* wbase = reinterpret_cast<const float*>(smem_dyn) + gw * kThreads * G;
+    #pragma unroll 2
+    for (int ks = 0; ks < nsteps; ++ks) {
+      const int64_t t8 = c0 + 16 * ks + 8 * hf;  // first of this lane's 8 tokens (a multiple of 8)
+      const uint32_t w = __ldg(vcw + ((t8 >> 7) * kD + ch) * 16 + ((t8 & 127) >> 3));
       #pragma unroll
-      for (int n = 0; n < NT; ++n) {
-        const int head = 4 * n + t4;
-        const float f = (head < G ? select_head<G>(alpha, head) : 1.0f) * beta[gw];
+      for (int j = 0; j < 8; ++j) {
+        const float cv = __int_as_float(0x4B000000 | ((w >> (4 * j)) & 0xFu)) - 8388616.0f;  // c - 8, exact
+        const float* wt = wbase + (16 * ks + 8 * hf + j) * G;
         #pragma unroll
-        for (int i = 0; i < 4; ++i) D[n][i] = __fmul_rn(D[n][i], f);
-      }
-      const uint32_t brow = smem_base + ((gw * kThreads + (lane & 15)) * ROWH) * 2;
-      #pragma unroll 4
-      for (int ks = 0; ks < nsteps; ++ks) {
-        uint32_t a[4];
-        codes_to_afrag(__ldg(tilew + ks * 256), a);
-        #pragma unroll
-        for (int n = 0; n < NT; ++n) {
-          uint32_t b0, b1;
-          ldsm_x2_trans(b0, b1, brow + (ks * 16 * ROWH + 8 * n) * 2);
-          mma16816(D[n], a, b0, b1);
-        }
-      }
-    } else {
-      #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        acc[h][0] = __fmul_rn(acc[h][0], alpha[h]);
-        acc[h][1] = __fmul_rn(acc[h][1], alpha[h]);
-      }
-      const float* wbase = reinterpret_cast<const float*>(smem_dyn) + gw * kThreads * G;
-      #pragma unroll 2
-      for (int ks = 0; ks < nsteps; ++ks) {
-        const uint32_t w = __ldg(tilew + ks * 256);
-        // slot -> (channel row 0/1, token within the 16-token tile)
-        const int shifts[8] = {0, 16, 4, 20, 8, 24, 12, 28};
-        const int rowsel[8] = {0, 0, 1, 1, 0, 0, 1, 1};
-        const int toks[8] = {2 * t4, 2 * t4 + 1, 2 * t4, 2 * t4 + 1, 2 * t4 + 8, 2 * t4 + 9, 2 * t4 + 8, 2 * t4 + 9};
-        #pragma unroll
-        for (int i = 0; i < 8; ++i) {
-          const float cv = __int_as_float(0x4B000000 | ((w >> shifts[i]) & 0xFu)) - 8388616.0f;  // c - 8, exact
-          const float* wt = wbase + (ks * 16 + toks[i]) * G;
-          #pragma unroll
-          for (int h = 0; h < G; ++h) acc[h][rowsel[i]] = __fmaf_rn(wt[h], cv, acc[h][rowsel[i]]);
-        }
+        for (int h = 0; h < G; ++h) acc[h] = __fmaf_rn(wt[h], cv, acc[h]);
       }
     }
     __syncthreads();
@@ -332,37 +229,11 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendParams 
     part_ptr(h)[0] = select_head<G>(m_run, h);
     part_ptr(h)[1] = total(h * 5);
   }
-  const int ch0 = 16 * warp + g8, ch1 = ch0 + 8;
-  const float unshift = (E_run[gw] == kNoExp) ? 0.0f : exp2_of_int(-E_run[gw]);
-  if (TENSOR) {
+  #pragma unroll
+  for (int h = 0; h < G; ++h) acc[h] = __fadd_rn(acc[h], __shfl_xor_sync(kFull, acc[h], 16));
+  if (hf == 0) {
     #pragma unroll
-    for (int n = 0; n < NT; ++n) {
-      const int head = 4 * n + t4;
-      if (head < G) {
-        const float midt = total(head * 5 + 1 + gw);
-        float* dst = part_ptr(head) + 2;
-        dst[ch0] = __fmaf_rn(__fadd_rn(D[n][0], D[n][1]), unshift, midt);
-        dst[ch1] = __fmaf_rn(__fadd_rn(D[n][2], D[n][3]), unshift * 0.0625f, midt);
-      }
-    }
-  } else {
-    #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        acc[h][r] += __shfl_xor_sync(kFull, acc[h][r], 1);
-        acc[h][r] += __shfl_xor_sync(kFull, acc[h][r], 2);
-      }
-    }
-    if (t4 == 0) {
-      #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        const float midt = total(h * 5 + 1 + gw);
-        float* dst = part_ptr(h) + 2;
-        dst[ch0] = __fadd_rn(acc[h][0], midt);
-        dst[ch1] = __fadd_rn(acc[h][1], midt);
-      }
-    }
+    for (int h = 0; h < G; ++h) part_ptr(h)[2 + ch] = __fadd_rn(acc[h], total(h * 5 + 1 + gw));
   }
 }
 
@@ -455,11 +326,10 @@ __global__ void __launch_bounds__(256) scores_kernel(const ScoresParams p, int G
   }
 }
 
-template <int G, bool TENSOR>
+template <int G>
 static cudaError_t launch_attend_t(const AttendParams& p, cudaStream_t stream) {
-  constexpr int NT = (2 * G + 7) / 8;
-  const size_t smem = TENSOR ? static_cast<size_t>(4) * kThreads * 8 * NT * 2 : static_cast<size_t>(4) * kThreads * G * 4;
-  auto kern = attend_kernel<G, TENSOR>;
+  const size_t smem = static_cast<size_t>(4) * kThreads * G * 4;
+  auto kern = attend_kernel<G>;
   static bool configured = false;  // per template instance
   if (!configured) {
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
@@ -488,11 +358,11 @@ int kv1b_pick_splits(int32_t B, int32_t Hkv, int64_t max_len, int num_sms) {
 cudaError_t kv1b_launch_attend(const AttendParams& p, int32_t G, int32_t engine, int32_t max_len,
                                cudaStream_t stream) {
   (void)max_len;
+  (void)engine;
   cudaError_t e = cudaSuccess;
-  const bool tensor = engine == KV1B_ATTEND_TENSOR;
-#define KV1B_CASE(GG)                                                                     \
-  case GG:                                                                                \
-    e = tensor ? launch_attend_t<GG, true>(p, stream) : launch_attend_t<GG, false>(p, stream); \
+#define KV1B_CASE(GG)                      \
+  case GG:                                 \
+    e = launch_attend_t<GG>(p, stream);    \
     break;
   switch (G) {
     KV1B_CASE(1)

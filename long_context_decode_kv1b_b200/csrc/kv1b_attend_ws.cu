@@ -1,35 +1,43 @@
-// kv1b_attend_ws.cu -- persistent split-K decode attention with tensor-core P.V, one CTA per SM.
+// kv1b_attend_ws.cu -- persistent split-K decode attention on the integer tensor cores, one CTA per SM.
 //
-// Work split: all (sequence, kv-head) segments are laid end to end in 16-token tiles and cut into
+// Work split: all (sequence, kv-head) segments are laid end to end in 128-token tiles and cut into
 // one equal contiguous range per CTA, so every SM streams the same number of compressed bytes
-// whatever the batch / head / context mix.  Each CTA walks its range in 512-token chunks
-// streamed into a 3-stage shared-memory ring with cp.async.bulk (five plain bulk copies per chunk,
-// one per cache plane, no multicast) and mbarrier completion; every warp owns a 64-token slice of
-// each chunk.  A warp done with a stage counts itself out on a shared counter; the warp that
-// counts out last issues the refill, so no warp waits for the others except through the ring.
+// whatever the batch / head / context mix.  A producer warp walks the CTA's range in stages of up
+// to two tiles (256 tokens) of one segment through a 4-deep shared-memory ring: one TMA tensor load
+// per tile brings the tile's 4-bit value codes ([128 channels][128 tokens], data type 16U4_ALIGN16B:
+// every 8 bytes of packed codes land in a 16-byte slot, 128-byte swizzle), and four plain bulk
+// copies bring the key bits, N, 1/C and the fp16 (scale, min) pairs.  Completion is tracked by
+// mbarriers with transaction bytes; the 8 compute warps release a stage by arriving on its "empty"
+// barrier.  Compute warp w owns tokens 32 (w & 3) .. + 31 of the stage's tile w >> 2.
 //
-// Each warp does all of the work for its slice, one 16-token tile at a time:
-//   the binary x INT4 proxy scores of the G query heads sharing this kv-head ("RaBitQCache",
-//   abstract / key design) as integer tensor-core products: the key sign bits are the A operand
-//   (one AND per register, bits masked in place), the query's 4-bit codes with a per-channel
-//   power-of-two correction the B operand, so the s32 accumulator holds 8 * sum_i bit_i * code_i
-//   exactly, plus 8 * Bc in the spare columns; each lane then owns one token of the tile and two
-//   head slots (and, for the weights, two of the four value groups);
-//   a warp-local online softmax in log2 units whose reference maximum is raised only when a logit
-//   exceeds it by 8 (then the warp's sums are rescaled), and the weights p * scale written as
-//   fp16 hi + lo rows;
-//   then 4 k-steps x 8 m-tiles of mma.sync m16n8k16: the codes as exact fp16 subnormals straight
-//   from the staged code tiles (one AND per register), ldmatrix'd weight B fragments; each chunk's
-//   tensor-core partial is added into fp32 accumulators on the CUDA cores (round to nearest), so
-//   accumulation error does not build up inside the tensor core ("H1B-KV", technical framework:
-//   weights from the sketch, then the 4-bit values).  value = min + scale * code, the min term is
-//   summed per (head, group) in fp32 by the score lanes.
+// Per 32-token slice a warp computes, for the G <= 4 query heads of the segment:
+//   scores ("RaBitQCache", abstract / key design: binary x INT4 arithmetic): per 16 tokens, four
+//     mma.m16n8k32 s8 products of the key sign bits (A, one AND per register: each byte keeps one
+//     bit in place) with the query's 4-bit codes (B, column 2h = head h scaled to undo the bit
+//     position, column 2h + 1 = ones), so lane (g, t) receives 8 A and 8 Bc of tokens g and g + 8
+//     for head t exactly -- the integers of the popcount form;
+//   softmax: lane (g, t) turns them into head t's logits (log2 units) and probabilities against a
+//     warp-uniform reference maximum that is raised only when a logit passes it by kTau (then the
+//     accumulators are rescaled), so every p <= 2^kTau;
+//   weights ("H1B-KV", technical framework: weights from the sketch, then the 4-bit values): lane
+//     (g, t) takes value group t of its tokens for all heads (the heads' p by shuffles within the
+//     lane quad) and forms W = p * scale * 2^E rounded to an unsigned 32-bit integer; E is a
+//     per-group power of two kept in step with the largest scale seen, so W < 2^32 and the weights
+//     of tokens far below the maximum keep many significant bits (a fixed point with fewer bits
+//     would round the long tail of a wide softmax to zero and bias the sum).  stmatrix (.trans, b8)
+//     writes the four bytes of every W into a per-warp buffer; ldmatrix gathers them as the A
+//     operand (rows = (head, byte));
+//   P.V: ldmatrix .b8x16.b4x16_p64 expands the staged codes to one byte per code (the B operand,
+//     k = tokens), and mma.m16n8k32 u8 x u8 -> s32 accumulates sum_t W * code per (head, byte,
+//     channel) EXACTLY in 32-bit integers; value = min + scale * code, the min term is summed per
+//     (head, group) in fp32.  The integer accumulators are converted (and rescaled) only when the
+//     reference maximum or a group exponent moves, and at the end of a segment piece.
 // At the end of a segment piece the 8 warps' partials are combined in shared memory and the CTA
 // writes one row (m, l, o[128]) per query head; the CTA that writes a segment's last row merges
 // the segment's rows by log-sum-exp into the output (one kernel per attend).
 //
 // Every mbarrier wait is bounded: a wait that runs out sets KV1B_STATUS_TIMEOUT in the cache's
-// status word; the CTA then stops issuing copies, later waits return at once, and thread 0
+// status word; the CTA then stops issuing copies, later waits return at once, and the producer
 // drains the copies already in flight before the CTA exits.
 #include "kv1b_device.cuh"
 #include "kv1b_launch.h"
@@ -37,33 +45,38 @@
 namespace kv1b {
 namespace ws {
 
-constexpr int kWarps = 8;                        // consumer warps; one more warp issues the copies
-constexpr int kTPL = 2;                          // tokens per lane per chunk
-constexpr int kThreads = kWarps * 32;            // 256 consumer threads
-constexpr int kBlock = kThreads + 32;            // + the producer warp
-constexpr int kWarpTiles = 2 * kTPL;             // 16-token tiles per warp per chunk
-constexpr int kChunkTiles = kWarpTiles * kWarps; // 32 tiles = 512 tokens per chunk
-constexpr int kStages = 3;
-constexpr float kTau = 8.0f;                     // lazy-max threshold (log2 units): p <= 2^8
-constexpr int kNoExp = 100;                     // group exponent before any scale was seen (finite:
-                                                 // every product with it meets a zero)
-constexpr float kNoMax = -1e30f;                 // reference maximum before any logit was seen
+constexpr int kWarps = 8;                   // compute warps; one more warp issues the copies
+constexpr int kThreads = kWarps * 32;       // 256 compute threads
+constexpr int kBlock = kThreads + 32;       // + the producer warp
+constexpr int kTileTok = 128;               // tokens per code tile (one TMA box)
+constexpr int kStageTiles = 2;
+constexpr int kStageTok = kStageTiles * kTileTok;
+constexpr int kStages = 4;
+constexpr int kTau = 2;                     // lazy-max threshold (log2 units): p <= 2^kTau
+constexpr int kNoExp = 100;                 // group exponent before any scale was seen
+constexpr float kNoMax = -1e30f;            // reference maximum before any logit was seen
+constexpr int kMaxAccStages = 8192;         // int32 headroom: 255 * 15 * 32 * 8192 < 2^31
 constexpr long long kSpinLimit = 1LL << 24;
 
-// Stage layout (bytes): one 512-token chunk; warp w uses tokens 64w .. 64w + 63 of it.
-constexpr int kChunkTok = kChunkTiles * 16;                   // 512
-constexpr int kWarpTok = kWarpTiles * 16;                     // 64
-constexpr int kOffBits = 0;                                   // u32 [512][4]
-constexpr int kOffNorm = kOffBits + kChunkTok * 16;           // f32 [512]
-constexpr int kOffCinv = kOffNorm + kChunkTok * 4;            // f32 [512]
-constexpr int kOffSm = kOffCinv + kChunkTok * 4;              // u32 [512][4]
-constexpr int kOffCodes = kOffSm + kChunkTok * 16;            // u32 [32 tiles][256]
-constexpr int kStageBytes = kOffCodes + kChunkTiles * 1024;   // 53248
-constexpr int kGroupRows = kWarpTok + 1;                      // 16-B B rows per group (+1 pad: bank shift)
-constexpr int kBRowsPerWarp = 4 * kGroupRows * 16;            // [4 groups][65 rows][16 B]
-constexpr int kRowF = 6 + 128;                                // per-warp partial: m, l, mid[4], o[128]
-static_assert(4 * kRowF * 4 <= kBRowsPerWarp, "a warp's flush partial reuses its B-row area");
-constexpr int kSmemBytes = kStages * kStageBytes + kWarps * kBRowsPerWarp;
+// Stage layout (bytes).
+constexpr int kTileSmem = kTileTok * 128;                  // 128 channels x 128 B (8 B codes + 8 B gap per 16 tokens)
+constexpr int kOffCodes = 0;
+constexpr int kOffBits = kStageTiles * kTileSmem;          // u32 [256][4]
+constexpr int kOffNorm = kOffBits + kStageTok * 16;        // f32 [256]
+constexpr int kOffCinv = kOffNorm + kStageTok * 4;         // f32 [256]
+constexpr int kOffSm = kOffCinv + kStageTok * 4;           // u32 [256][4]
+constexpr int kStageBytes = (kOffSm + kStageTok * 16 + 1023) / 1024 * 1024;
+constexpr int kWBytes = 16 * 128;                          // per warp: 16 byte matrices of 8 rows x 16 tokens
+constexpr int kOffW = kStages * kStageBytes;
+constexpr int kRowF = 6 + 128;                             // per-warp partial row: m, l, mid[4], o[128]
+constexpr int kPartBytes = 4 * kRowF * 4;
+constexpr int kOffPart = kOffW + kWarps * kWBytes;
+constexpr int kSmemUsed = kOffPart + kWarps * kPartBytes;
+constexpr int kSmemBytes = kSmemUsed + 1024;               // + slack to align the base to 1024 B
+constexpr uint32_t kTxPerTile = kTileTok * 104;            // packed codes 64 B + 40 B of the other planes per token
+static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
+static_assert(kOffW % 1024 == 0 && kStageBytes % 1024 == 0, "TMA 128B-swizzle destinations are 1024-B aligned");
+static_assert(2 * 4 * 256 * 4 + 64 <= kWarps * kPartBytes, "the segment merge reuses the partial area");
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 
@@ -86,8 +99,7 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-// try_wait that lets the hardware suspend the warp (up to ~0.5 ms per try) instead of spinning,
-// so waiting warps give their issue slots to working ones.
+// try_wait that lets the hardware suspend the warp (up to ~0.5 ms per try) instead of spinning.
 __device__ __forceinline__ bool mbar_try_sleep(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -114,72 +126,87 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
                "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
 }
+// One 128-token code tile: box [128 tokens, 128 channels, 1 tile] at tile index z (no multicast).
+__device__ __forceinline__ void tma_codes(void* dst, const CUtensorMap* map, int z, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3, %4}], [%5];" ::"r"(
+          smem_u32(dst)),
+      "l"(map), "r"(0), "r"(0), "r"(z), "r"(smem_u32(bar))
+      : "memory");
+}
 __device__ __forceinline__ void named_bar(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
 
-__device__ __forceinline__ void mma16816(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
+// Integer tensor-core products (m16n8k32: A 16 x 32, B 32 x 8, D 16 x 8 s32).
+__device__ __forceinline__ void imma_s8(int d[4], const uint32_t a[4], uint32_t b0, uint32_t b1, bool zero) {
+  if (zero)
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
+        : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0));
+  else
+    asm volatile(
+        "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+        : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ void imma_u8(int d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
   asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
-      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-__device__ __forceinline__ void ldsm_x2_trans(uint32_t& b0, uint32_t& b1, uint32_t addr) {
-  asm volatile("ldmatrix.sync.aligned.m8n8.x2.trans.shared.b16 {%0,%1}, [%2];" : "=r"(b0), "=r"(b1) : "r"(addr));
-}
-__device__ __forceinline__ uint32_t hsub2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-// One code word (v_codes layout) -> m16n8k16 A fragment holding the codes as exact fp16
-// subnormals: rows g get c * 2^-24 (nibbles at bits 0-3 / 16-19 of a half), rows g + 8 get
-// 16 c * 2^-24 (their nibbles sit 4 bits higher).  Both scale factors are undone at the end.
-__device__ __forceinline__ void codes_to_afrag(uint32_t w, uint32_t a[4]) {
-  const uint32_t w8 = __umulhi(w, 1u << 24);  // w >> 8 on the multiply pipe (the logic pipe is the busy one)
-  a[0] = w & 0x000F000Fu;
-  a[1] = w & 0x00F000F0u;
-  a[2] = w8 & 0x000F000Fu;
-  a[3] = w8 & 0x00F000F0u;
-}
-__device__ __forceinline__ void mma16816_zc(float d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
-      : "=f"(d[0]), "=f"(d[1]), "=f"(d[2]), "=f"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "f"(0.0f));
-}
-// Integer tensor-core step of the binary x INT4 product: D (s32) += A (16 tokens x 32 channels,
-// s8) * B (32 channels x 8 columns, s8).
-__device__ __forceinline__ void imma16832(int d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      "mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
       : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+// Four 8 x 16-byte matrices; lane i addresses row i & 7 of matrix i >> 3; register j of lane
+// (g, t) receives bytes 4t .. 4t + 3 of row g of matrix j.
+__device__ __forceinline__ void ldsm_x4(uint32_t r[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+// Same with rows of 16 packed 4-bit values (8 data bytes, then an 8-byte gap): element e of a row
+// becomes byte e of the row, value in bits 0-3 (low nibble = even element).
+__device__ __forceinline__ void ldsm_x4_u4(uint32_t r[4], uint32_t addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n16.x4.shared.b8x16.b4x16_p64 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(addr));
+}
+// Four 16 x 8 byte matrices stored transposed: byte b of register m of lane (g, t) goes to row
+// 2t + (b & 1), column g + 8 (b >> 1) of matrix m, whose 16-byte rows lanes 8m .. 8m + 7 address.
+__device__ __forceinline__ void stsm_x4_t8(uint32_t addr, const uint32_t r[4]) {
+  asm volatile("stmatrix.sync.aligned.m16n8.x4.trans.shared.b8 [%0], {%1,%2,%3,%4};" ::"r"(addr), "r"(r[0]), "r"(r[1]),
+               "r"(r[2]), "r"(r[3])
+               : "memory");
+}
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
 }
 // Score MMA over one 16-token tile.  Lane (g, t) holds word t of the sign bits of tokens g and
 // g + 8.  K-block kb (32 channels) takes, from each word, the bits at positions 8j + 2kb (k = 4t+j)
 // and 8j + 2kb + 1 (k = 16+4t+j), j = 0..3, each masked in place so that the byte is
 // bit * 2^((2kb + hi) & 3); the query operand carries code * 2^(3 - that), so every product is
 // 8 * bit * code and D = 8 * sum_i bit_i * code_i exactly (the integer A of the popcount form;
-// the column of ones gives 8 * Bc).
-__device__ __forceinline__ void imma16832_zc(int d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
-      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
-      : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
-      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0));
-}
+// the columns of ones give 8 * Bc).
 __device__ __forceinline__ void score_tile(int d[4], uint32_t wg, uint32_t wg8, const uint32_t (&bq)[4][2]) {
   const uint32_t xg[2] = {wg, __umulhi(wg, 1u << 28)}, xg8[2] = {wg8, __umulhi(wg8, 1u << 28)};  // >> 4
   #pragma unroll
   for (int kb = 0; kb < 4; ++kb) {
     const uint32_t mlo = 0x01010101u << (2 * (kb & 1)), mhi = mlo << 1;
     const uint32_t a[4] = {xg[kb >> 1] & mlo, xg8[kb >> 1] & mlo, xg[kb >> 1] & mhi, xg8[kb >> 1] & mhi};
-    if (kb == 0) imma16832_zc(d, a, bq[kb][0], bq[kb][1]);
-    else imma16832(d, a, bq[kb][0], bq[kb][1]);
+    imma_s8(d, a, bq[kb][0], bq[kb][1], kb == 0);
   }
 }
 __device__ __forceinline__ float exp2i(int e) { return __int_as_float((e + 127) << 23); }
 __device__ __forceinline__ int ilog2_pos(float x) { return static_cast<int>((__float_as_uint(x) >> 23) & 0xff) - 127; }
-// exact int -> float for |x| < 2^22 without the quarter-rate conversion unit
-__device__ __forceinline__ float i2f_exact(int x) { return __int_as_float(x + 0x4B400000) - 12582912.0f; }
+__device__ __forceinline__ float ex2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+template <typename T>
+__device__ __forceinline__ T sel4(const T (&v)[4], int i) {
+  return i == 0 ? v[0] : (i == 1 ? v[1] : (i == 2 ? v[2] : v[3]));
+}
 
 struct Work {
   int64_t T;   // total tiles
@@ -189,58 +216,13 @@ struct Work {
 __device__ __host__ __forceinline__ int64_t tile_begin(const Work& w, int64_t c) { return c * w.T / w.n; }
 __device__ __host__ __forceinline__ int64_t cta_of_tile(const Work& w, int64_t t) { return ((t + 1) * w.n - 1) / w.T; }
 
-struct Chunk {
-  int seg, lt, nt;
-};
-__device__ __forceinline__ Chunk chunk_at(const Work& wk, int64_t t, int64_t t_end) {
-  Chunk ch;
-  ch.seg = static_cast<int>(t / wk.Lt);
-  ch.lt = static_cast<int>(t - static_cast<int64_t>(ch.seg) * wk.Lt);
-  int64_t lim = static_cast<int64_t>(ch.seg + 1) * wk.Lt;
-  if (lim > t_end) lim = t_end;
-  const int64_t n = lim - t;
-  ch.nt = static_cast<int>(n < kChunkTiles ? n : kChunkTiles);
-  return ch;
-}
-
-// Copy chunk `ch` (contiguous tiles of one segment) into a stage: five bulk copies, one per plane.
-__device__ __forceinline__ void issue_chunk(const CacheView& c, const Chunk& ch, uint8_t* st, uint64_t* bar) {
-  const uint32_t ntok = ch.nt * 16;
-  mbar_expect_tx(bar, ntok * 104u);
-  const int64_t tok = static_cast<int64_t>(ch.seg) * c.cap + static_cast<int64_t>(ch.lt) * 16;
-  bulk_g2s(st + kOffBits, c.k_bits + tok * 4, ntok * 16, bar);
-  bulk_g2s(st + kOffNorm, c.k_norm + tok, ntok * 4, bar);
-  bulk_g2s(st + kOffCinv, c.k_cinv + tok, ntok * 4, bar);
-  bulk_g2s(st + kOffSm, c.v_sm + tok * 4, ntok * 16, bar);
-  bulk_g2s(st + kOffCodes, c.v_codes + tok * 16, ntok * 64, bar);
-}
-
-__device__ __forceinline__ float ex2(float x) {
-  float y;
-  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
-  return y;
-}
-__device__ __forceinline__ uint64_t f2pack(float a, float b) {
-  return static_cast<uint64_t>(__float_as_uint(a)) | (static_cast<uint64_t>(__float_as_uint(b)) << 32);
-}
-__device__ __forceinline__ uint64_t mul2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t sub2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-
 // Tile iterator over a CTA's range: (segment, tile within segment, tiles left), no divisions.
 struct TileIt {
   int seg, lt, rem;
   __device__ __forceinline__ int nt(int Lt) const {
     int n = Lt - lt;
     n = n < rem ? n : rem;
-    return n < kChunkTiles ? n : kChunkTiles;
+    return n < kStageTiles ? n : kStageTiles;
   }
   __device__ __forceinline__ void advance(int n, int Lt) {
     lt += n;
@@ -252,32 +234,43 @@ struct TileIt {
   }
 };
 
+// Copy a stage: n tiles of segment `seg` starting at tile `lt`.
+__device__ __forceinline__ void issue_stage(const AttendWsParams& p, int seg, int lt, int n, uint8_t* st, uint64_t* bar) {
+  const CacheView& c = p.c;
+  mbar_expect_tx(bar, n * kTxPerTile);
+  const int tiles_per_seg = c.cap / kTileTok;
+  for (int i = 0; i < n; ++i) tma_codes(st + kOffCodes + i * kTileSmem, &p.codes_map, seg * tiles_per_seg + lt + i, bar);
+  const int64_t tok = static_cast<int64_t>(seg) * c.cap + static_cast<int64_t>(lt) * kTileTok;
+  const uint32_t ntok = n * kTileTok;
+  bulk_g2s(st + kOffBits, c.k_bits + tok * 4, ntok * 16, bar);
+  bulk_g2s(st + kOffNorm, c.k_norm + tok, ntok * 4, bar);
+  bulk_g2s(st + kOffCinv, c.k_cinv + tok, ntok * 4, bar);
+  bulk_g2s(st + kOffSm, c.v_sm + tok * 4, ntok * 16, bar);
+}
+
 template <int G>
-__global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsParams p) {
-  static_assert(G == 1 || G == 2 || G == 4, "one n-tile: (head, hi/lo) columns <= 8");
-  extern __shared__ __align__(1024) uint8_t smem[];
+__global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_constant__ AttendWsParams p) {
+  static_assert(G == 1 || G == 2 || G == 4, "head t of lane (g, t) for t < G");
+  extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kStages];
-  __shared__ __align__(8) uint64_t empty_bar[kStages];  // all consumer warps released the stage
-  __shared__ __align__(16) uint4 s_planes[2][G][4];  // double-buffered by segment parity
-  __shared__ float s_vl[2][G], s_dl[2][G];
-  __shared__ int s_sq[2][G];
+  __shared__ __align__(8) uint64_t empty_bar[kStages];  // all compute warps released the stage
+  __shared__ __align__(16) uint4 s_planes[2][4][4];     // double-buffered by segment parity
+  __shared__ float s_vl[2][4], s_dl[2][4];
+  __shared__ int s_sq[2][4];
   __shared__ volatile int s_abort;
   __shared__ int s_merge;
 
+  uint8_t* smem = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const CacheView& c = p.c;
   const Work wk{p.T, p.Lt, static_cast<int>(gridDim.x)};
   const int64_t t_begin = tile_begin(wk, blockIdx.x), t_end = tile_begin(wk, blockIdx.x + 1);
   const int Lt = static_cast<int>(p.Lt);
   const int L = p.L;
-  const float qsl = __fmul_rn(__fdiv_rn(p.scale, static_cast<float>(kD)), 0x1.715476p+0f);  // scale/128*log2e
-  const int g8 = lane >> 2, t4 = lane & 3;
-  uint8_t* brows = smem + kStages * kStageBytes + warp * kBRowsPerWarp;
-  uint64_t* bars = full_bar;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
-      mbar_init(&bars[s], 1);
+      mbar_init(&full_bar[s], 1);
       mbar_init(&empty_bar[s], kWarps);
     }
     s_abort = 0;
@@ -288,87 +281,111 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsPara
   it.seg = static_cast<int>(t_begin / p.Lt);
   it.lt = static_cast<int>(t_begin - static_cast<int64_t>(it.seg) * p.Lt);
   it.rem = static_cast<int>(t_end - t_begin);
-  if (warp == kWarps) {  // producer: one lane streams the CTA's chunks through the ring
+  if (warp == kWarps) {  // producer: one lane streams the CTA's stages through the ring
     if (lane == 0) {
       TileIt is = it;
-      int j = 0;  // chunks issued
+      int j = 0;  // stages issued
       while (is.rem > 0 && !s_abort) {
         const int st = j % kStages;
         if (j >= kStages && !mbar_wait(&empty_bar[st], ((j / kStages) - 1) & 1, &s_abort)) break;
         const int n = is.nt(Lt);
-        issue_chunk(c, Chunk{is.seg, is.lt, n}, smem + st * kStageBytes, &bars[st]);
+        issue_stage(p, is.seg, is.lt, n, smem + st * kStageBytes, &full_bar[st]);
         is.advance(n, Lt);
         ++j;
       }
-      // the CTA's shared memory must outlive every copy issued into it (the consumers wait for
-      // all of them unless the CTA gave up)
+      // the CTA's shared memory must outlive every copy issued into it (the compute warps wait
+      // for all of them unless the CTA gave up)
       for (int k = (j - kStages > 0 ? j - kStages : 0); k < j; ++k) {
         long long spins = 0;
-        while (!mbar_try(&bars[k % kStages], (k / kStages) & 1) && ++spins < kSpinLimit) __nanosleep(64);
+        while (!mbar_try(&full_bar[k % kStages], (k / kStages) & 1) && ++spins < kSpinLimit) __nanosleep(64);
       }
     }
     return;
   }
 
-  // Score lanes.  MMA row g of a tile holds token g + 8 (g >> 2) and row g + 8 holds token g + 4,
-  // so that each half-warp's tokens fill 128 contiguous bytes of a B-row group (conflict-free
-  // stores) while the key-word loads stay conflict-free too.  Lane (g, t) takes row g (t < 2) or
-  // row g + 8 (t >= 2) and the head slots hs0 = 2 (t & 1), hs0 + 1 of the scores (a slot >= G is
-  // empty); for the weights the lane pair (t, t ^ 1), which shares the token, splits the value
-  // groups: lane t takes groups 2q, 2q + 1 with q = t & 1.
-  const int q1 = t4 & 1;
-  const int hs0 = 2 * q1;
-  const bool upper = (t4 >> 1) != 0;
-  const int row_lo = g8 + 8 * (g8 >> 2), row_hi = g8 + 4;
-  const int tokr = upper ? row_hi : row_lo;
+  const int g = lane >> 2, t = lane & 3;
+  const int hh = g & 3;                  // head of this lane's P.V accumulator rows
+  const bool lo_bytes = (g >> 2) == 0;   // rows g / g + 8 hold bytes 0 / 2 (else bytes 1 / 3)
+  const float qsl = __fmul_rn(__fdiv_rn(p.scale, static_cast<float>(kD)), 0x1.715476p+0f);  // scale/128 * log2 e
+  uint8_t* wbuf = smem + kOffW + warp * kWBytes;
+  const uint32_t wbase = smem_u32(wbuf);
+  // stmatrix row address of this lane: matrix (kk, head m = lane >> 3, lo/hi), row rho = lane & 7
+  // kept in slot (rho + 2 m) & 7 so that the A-operand gathers below are free of bank conflicts
+  const uint32_t st_off = static_cast<uint32_t>((lane >> 3) * 2 * 128 + (((lane & 7) + 2 * (lane >> 3)) & 7) * 16);
+  // A-operand gather for group grp: lane i addresses A row r = (i & 7) + 8 ((i >> 3) & 1) of
+  // k-half kk = i >> 4; row r = (head r & 3, byte r >> 2)
+  const int a_r = (lane & 7) + 8 * ((lane >> 3) & 1), a_kk = lane >> 4;
+  const int a_head = a_r & 3, a_byte = a_r >> 2;
+  const uint32_t a_off0 = static_cast<uint32_t>(((a_kk * 4 + a_head) * 2 + (a_byte >> 1)) * 128);
+  const int a_rho0 = (a_byte & 1) + 2 * a_head;
 
-  float m_w[G], m_thr[G];        // warp-uniform reference maximum and its rare-path threshold
-  float m_my[2], thr_my[2];      // the same for this lane's two head slots
-  float l_acc[2];                // sum p of this lane's head slots
-  float mid_acc[4][2];           // sum p * min, heads 0..3 x this lane's groups 2q, 2q + 1
-  float smax[4];                 // per group: scales up to this keep p * scale * 2^E in fp16 range
-  int E_w[4];
-  float smax_my[2], ef_my[2];    // smax and 2^E of this lane's groups
-  float D[8][4];
-  uint32_t bq[4][2];             // score-MMA query operand of this segment
-  float vl_my[2], dl4_my[2], kq_my[2];
+  // per-lane state
+  float m_w[4], smax_w[4];  // warp-uniform: reference maximum per head, scale bound per group
+  int E_w[4];               // warp-uniform: weight exponent per group
+  float m_t, thr_t, s2e_t, smax_t;  // the same for this lane's head t / group t
+  float l_t;                // sum p of head t over this lane's tokens
+  float mid[4];             // sum p * min of group t, heads 0..3
+  int D[16][4];             // P.V integer accumulators: n-tile (8 channels) x (rows g, g + 8) x 2 channels
+  // converted P.V sums live in the warp's partial rows in shared memory: o[head][channel]
+  uint32_t bq[4][2];        // score-MMA query operand of this segment
+  float c1_t, c2_t, c0_t;   // head t logit constants
+  bool hv_t;                // head t exists
+  int nacc = 0;             // stages accumulated in D since the last conversion
+
+  auto part_of = [&](int w) { return reinterpret_cast<float*>(smem + kOffPart + w * kPartBytes); };
+
   auto reset = [&]() {
     #pragma unroll
-    for (int h = 0; h < G; ++h) {
-      m_w[h] = kNoMax;
-      m_thr[h] = kNoMax;
+    for (int i = 0; i < 4; ++i) {
+      m_w[i] = kNoMax;
+      smax_w[i] = 0.0f;
+      E_w[i] = kNoExp;
+      mid[i] = 0.0f;
     }
+    m_t = kNoMax;
+    thr_t = kNoMax;
+    s2e_t = exp2i(kNoExp);
+    smax_t = 0.0f;
+    l_t = 0.0f;
     #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      m_my[e] = kNoMax;
-      thr_my[e] = kNoMax;
-      l_acc[e] = 0.0f;
-      smax_my[e] = 0.0f;
-      ef_my[e] = exp2i(kNoExp);
-    }
+    for (int n = 0; n < 16; ++n) D[n][0] = D[n][1] = D[n][2] = D[n][3] = 0;
+    float* o = part_of(warp);
+    for (int i = lane; i < 4 * 128; i += 32) o[(i >> 7) * kRowF + 6 + (i & 127)] = 0.0f;
+    __syncwarp();
+    nacc = 0;
+  };
+  // Convert the integer accumulators (old exponents) and add them to the warp's o rows in shared
+  // memory, then scale head h's row by alpha[h]: lanes g and g + 4 hold bytes {0, 2} and {1, 3} of
+  // the same head and channels; lane g < 4 owns head g, channels 8n + 2t + e.
+  auto drain = [&](const float (&alpha)[4]) {
+    const float wb0 = lo_bytes ? 1.0f : 256.0f, wb2 = lo_bytes ? 65536.0f : 16777216.0f;
+    const float al = sel4(alpha, hh);
+    float* o = part_of(warp) + hh * kRowF + 6 + 2 * t;
     #pragma unroll
-    for (int h = 0; h < 4; ++h) mid_acc[h][0] = mid_acc[h][1] = 0.0f;
-    #pragma unroll
-    for (int g = 0; g < 4; ++g) {
-      smax[g] = 0.0f;
-      E_w[g] = kNoExp;
-    }
-    #pragma unroll
-    for (int mt = 0; mt < 8; ++mt)
+    for (int n = 0; n < 16; ++n) {
+      const float inv = exp2i(-E_w[n >> 2]);
+      float x[2];
       #pragma unroll
-      for (int k = 0; k < 4; ++k) D[mt][k] = 0.0f;
+      for (int e = 0; e < 2; ++e) {
+        x[e] = __fmaf_rn(wb2, static_cast<float>(D[n][2 + e]), __fmul_rn(wb0, static_cast<float>(D[n][e])));
+        x[e] = __fadd_rn(x[e], __shfl_xor_sync(kFull, x[e], 16));
+        D[n][e] = 0;
+        D[n][2 + e] = 0;
+      }
+      if (lo_bytes && hh < G) {
+        float2 v = *reinterpret_cast<float2*>(o + 8 * n);
+        v.x = __fmul_rn(__fmaf_rn(x[0], inv, v.x), al);
+        v.y = __fmul_rn(__fmaf_rn(x[1], inv, v.y), al);
+        *reinterpret_cast<float2*>(o + 8 * n) = v;
+      }
+    }
+    __syncwarp();
+    nacc = 0;
   };
 
-  // Segment piece done: each warp puts its partial (m, l, mid[4], o[128]) per head in shared
-  // memory; then thread (head, channel) combines the warps by log-sum-exp and writes the CTA's
-  // row (m, l, o[128] with the mid term folded in) for slot (segment, piece).  Every warp reaches
-  // this at the same chunk.
-  auto part_of = [&](int w) { return reinterpret_cast<float*>(smem + kStages * kStageBytes + w * kBRowsPerWarp); };
-
-  // Log-sum-exp merge of the n CTA rows of segment `seg` (per query head) into the output; the
-  // CTA's shared partials are free by now and hold the piece maxima, sums and weights.  All heads
-  // at once: thread t takes channel t & 127 of heads (t >> 7) + 2i, with the pieces' loads
-  // independent of one another.
+  // Log-sum-exp merge of the n CTA rows of segment `seg` (per query head) into the output; uses
+  // the shared partial area.  All heads at once: thread t takes channel t & 127 of heads
+  // (t >> 7) + 2i, with the pieces' loads independent of one another.
   static_assert(kThreads == 256, "two threads per channel in the merge");
   auto merge_segment = [&](int seg, int n) {
     float* sm_m = part_of(0);       // [G][256] piece maxima, then weights
@@ -417,43 +434,27 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsPara
           den > 0.0f ? __fdiv_rn(__fadd_rn(__fadd_rn(acc[0], acc[1]), __fadd_rn(acc[2], acc[3])), den) : 0.0f;
     }
   };
+
+  // Segment piece done: each warp puts its partial (m, l, mid[4], o[128]) per head in shared
+  // memory; then thread (head, channel) combines the warps by log-sum-exp and writes the CTA's
+  // row (m, l, o[128] with the mid term folded in) for slot (segment, piece).  Every warp reaches
+  // this at the same stage.
   auto flush = [&](int seg) {
-    float v[10];  // l of the own head slots, then mid[head][own group]
-    v[0] = l_acc[0];
-    v[1] = l_acc[1];
+    const float ones[4] = {1.0f, 1.0f, 1.0f, 1.0f};
+    drain(ones);
+    float v[5] = {l_t, mid[0], mid[1], mid[2], mid[3]};
     #pragma unroll
-    for (int h = 0; h < 4; ++h) {
-      v[2 + 2 * h] = mid_acc[h][0];
-      v[3 + 2 * h] = mid_acc[h][1];
-    }
-    #pragma unroll
-    for (int m = 16; m >= 2; m >>= 1)  // lanes with the same t & 1 hold the same slots and groups
+    for (int m = 4; m <= 16; m <<= 1)  // sum over the 8 lanes with the same t
       #pragma unroll
-      for (int k = 0; k < 10; ++k) v[k] += __shfl_xor_sync(kFull, v[k], m);
-    float* mine = part_of(warp);  // this warp's P.V is done with its B rows
-    if (lane < 2) {  // lane q: head slots 2q, 2q + 1 and value groups 2q, 2q + 1
-      #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const int h = 2 * lane + e;
-        if (h < G) {
-          mine[h * kRowF] = m_my[e] == kNoMax ? -INFINITY : m_my[e];
-          mine[h * kRowF + 1] = v[e];
-        }
+      for (int k = 0; k < 5; ++k) v[k] = __fadd_rn(v[k], __shfl_xor_sync(kFull, v[k], m));
+    float* mine = part_of(warp);
+    if (g == 0) {  // lane t: head t's m and l, group t's mid of every head
+      if (t < G) {
+        mine[t * kRowF] = m_t == kNoMax ? -INFINITY : m_t;
+        mine[t * kRowF + 1] = v[0];
       }
       #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        mine[h * kRowF + 2 + 2 * lane] = v[2 + 2 * h];
-        mine[h * kRowF + 3 + 2 * lane] = v[3 + 2 * h];
-      }
-    }
-    if (t4 < G) {  // D columns 2 t4, 2 t4 + 1 = head t4, hi and lo parts
-      float* o = mine + t4 * kRowF + 6;
-      #pragma unroll
-      for (int mt = 0; mt < 8; ++mt) {
-        const float un = exp2i(24 - E_w[mt >> 1]);  // codes were c * 2^-24
-        o[16 * mt + g8] = __fmul_rn(__fadd_rn(D[mt][0], D[mt][1]), un);
-        o[16 * mt + g8 + 8] = __fmul_rn(__fadd_rn(D[mt][2], D[mt][3]), un * 0.0625f);
-      }
+      for (int h = 0; h < G; ++h) mine[h * kRowF + 2 + t] = v[1 + h];
     }
     named_bar(1, kThreads);
     const int ch = threadIdx.x & 127;
@@ -500,9 +501,10 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsPara
   };
 
   // Query preparation of a segment's G heads (warp h -> head h) into buffer seg & 1, then every
-  // lane builds its score-MMA operand: column n = g of B holds head n's codes (n < G), ones
-  // (n >= 4, giving Bc) or zeros; k-row 4t + j of k-block kb is channel 32t + 8j + 2kb (+1 for
-  // k-rows 16..31), scaled by 2^(3 - ((2kb + hi) & 3)) to undo the in-place bit position.
+  // lane builds its score-MMA operand: column n = g of B holds head g / 2's codes (g even, head
+  // < G), ones (g odd, giving Bc) or zeros; k-row 4t + j of k-block kb is channel
+  // 32t + 8j + 2kb (+1 for k-rows 16..31), scaled by 2^(3 - ((2kb + hi) & 3)) to undo the
+  // in-place bit position.
   auto prep = [&](int seg) {
     const int par = seg & 1;
     if (warp < G) {
@@ -518,11 +520,13 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsPara
         s_sq[par][warp] = qp.sq;
       }
     }
-    named_bar(1, kThreads);  // reached by every warp at the same chunk
+    named_bar(1, kThreads);  // reached by every warp at the same stage
+    const int hb = g >> 1;
+    const bool code_col = (g & 1) == 0 && hb < G;
     uint32_t pw[4] = {0u, 0u, 0u, 0u};
-    if (g8 < G) {
+    if (code_col) {
       #pragma unroll
-      for (int j = 0; j < 4; ++j) pw[j] = reinterpret_cast<const uint32_t*>(&s_planes[par][g8][j])[t4];
+      for (int j = 0; j < 4; ++j) pw[j] = reinterpret_cast<const uint32_t*>(&s_planes[par][hb][j])[t];
     }
     #pragma unroll
     for (int kb = 0; kb < 4; ++kb)
@@ -533,24 +537,23 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsPara
         uint32_t code = 0u;
         #pragma unroll
         for (int j = 0; j < 4; ++j) code |= ((pw[j] >> r) & 0x01010101u) << j;
-        bq[kb][hi] = (g8 < G) ? (code << sh) : (g8 >= 4 ? (0x01010101u << sh) : 0u);
+        bq[kb][hi] = code_col ? (code << sh) : ((g & 1) ? (0x01010101u << sh) : 0u);
       }
-    #pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const int h = hs0 + e;
-      const bool ok = h < G;
-      const float dl = ok ? s_dl[par][ok ? h : 0] : 0.0f;
-      vl_my[e] = ok ? s_vl[par][ok ? h : 0] : 0.0f;
-      dl4_my[e] = 0.25f * dl;
-      kq_my[e] = -dl * static_cast<float>(ok ? s_sq[par][ok ? h : 0] : 0);
-    }
+    hv_t = t < G;
+    const int hs = hv_t ? t : 0;
+    const float dl = hv_t ? s_dl[par][hs] : 0.0f, vl = hv_t ? s_vl[par][hs] : 0.0f;
+    const float sq = hv_t ? static_cast<float>(s_sq[par][hs]) : 0.0f;
+    // dot = delta (2A - Sq) + vl (2Bc - 128) = (delta / 4) 8A + (vl / 4) 8Bc - (delta Sq + 128 vl)
+    c1_t = __fmul_rn(0.25f * dl, qsl);
+    c2_t = __fmul_rn(0.25f * vl, qsl);
+    c0_t = __fmul_rn(-__fadd_rn(__fmul_rn(dl, sq), 128.0f * vl), qsl);
   };
 
   reset();
   int cur_seg = it.seg;
   if (it.rem > 0) prep(cur_seg);
-  const uint32_t bbase = smem_u32(brows) + (lane & 15) * 16;
-  int s = 0;           // stage of the current chunk
+  const int tl = warp >> 2, tw = (warp & 3) * 32;  // this warp's tile in the stage and token offset in it
+  int s = 0;           // stage of the current step
   uint32_t phase = 0;  // parity of the stage's expected completion
   while (it.rem > 0) {
     const int nt = it.nt(Lt);
@@ -560,194 +563,136 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const AttendWsPara
       cur_seg = it.seg;
       prep(cur_seg);
     }
-    mbar_wait(&bars[s], phase, &s_abort);
+    mbar_wait(&full_bar[s], phase, &s_abort);
     const uint8_t* st = smem + s * kStageBytes;
-    const int my_tiles = nt - kWarpTiles * warp;  // tiles of this chunk owned by this warp (may be <= 0)
-
-    // tokens of this warp's slice below `lim` are real (beyond: other warps' tiles, a ragged
-    // segment end, or slots of the stage that were not filled)
-    int lim = L - (it.lt * 16 + kWarpTok * warp);
-    lim = lim < my_tiles * 16 ? lim : my_tiles * 16;
-
-    // ---------------- scores: one integer MMA chain per tile, then lane (g, t) takes its token's
-    // two head slots and Bc from the accumulator columns (heads in columns 0..3, Bc in 4..7)
-    bool valid[kWarpTiles];
-    float s2[kWarpTiles][2], sc[kWarpTiles][2], mid[kWarpTiles][2];
-    #pragma unroll
-    for (int kk = 0; kk < kWarpTiles; ++kk) {
-      const int tt = kk * 16 + tokr;  // token within the warp slice
-      valid[kk] = tt < lim;
-      const uint32_t* kbits = reinterpret_cast<const uint32_t*>(st + kOffBits + warp * kWarpTok * 16) + kk * 64 + t4;
-      int d[4];
-      score_tile(d, kbits[row_lo * 4], kbits[row_hi * 4], bq);
-      const int x0 = __shfl_xor_sync(kFull, d[0], 2);
-      const int x2 = __shfl_xor_sync(kFull, d[2], 2);
-      const int x3 = __shfl_xor_sync(kFull, d[3], 2);
-      const int a0 = upper ? x2 : d[0], a1 = upper ? x3 : d[1], bc8 = upper ? d[2] : x0;
-      const float nc = __fmul_rn(__fmul_rn(reinterpret_cast<const float*>(st + kOffNorm)[kWarpTok * warp + tt],
-                                           reinterpret_cast<const float*>(st + kOffCinv)[kWarpTok * warp + tt]), qsl);
-      // the accumulators hold 8 A and 8 Bc: dot = (delta / 4) 8A + (vl (2 Bc - 128) - delta Sq)
-      const float i1 = __fmaf_rn(0.25f, __int2float_rn(bc8), -128.0f);
-      const int aa[2] = {a0, a1};
-      #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        const float dot = __fmaf_rn(dl4_my[e], __int2float_rn(aa[e]), __fmaf_rn(vl_my[e], i1, kq_my[e]));
-        s2[kk][e] = (valid[kk] && hs0 + e < G) ? __fmul_rn(dot, nc) : -INFINITY;
+    int lim = L - (it.lt * kTileTok + tl * kTileTok + tw);  // real tokens of this warp's slice
+    lim = tl < nt ? (lim < 32 ? lim : 32) : 0;
+    if (lim > 0) {
+      if (nacc >= kMaxAccStages) {
+        const float ones[4] = {1.0f, 1.0f, 1.0f, 1.0f};
+        drain(ones);
       }
-      // (scale, min) of this lane's two groups; invalid tokens may read a stage slot never filled
-      const uint2 smv = *reinterpret_cast<const uint2*>(st + kOffSm + (kWarpTok * warp + tt) * 16 + q1 * 8);
-      const uint32_t smw[2] = {valid[kk] ? smv.x : 0u, valid[kk] ? smv.y : 0u};
+      ++nacc;
+      const int tbase = tl * kTileTok + tw;  // slice start within the stage
+      const uint32_t* kbits = reinterpret_cast<const uint32_t*>(st + kOffBits) + tbase * 4 + t;
+      const float* knorm = reinterpret_cast<const float*>(st + kOffNorm) + tbase;
+      const float* kcinv = reinterpret_cast<const float*>(st + kOffCinv) + tbase;
+      const uint32_t* vsm = reinterpret_cast<const uint32_t*>(st + kOffSm) + tbase * 4 + t;
+      // ---------------- scores of head t for tokens 16 kk + g + 8 e
+      float s2[2][2], sc[2][2], mn[2][2];
+      bool rare = false;
       #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        sc[kk][j] = __half2float(__ushort_as_half(static_cast<unsigned short>(smw[j] & 0xffffu)));
-        mid[kk][j] = __half2float(__ushort_as_half(static_cast<unsigned short>(smw[j] >> 16)));
-      }
-    }
-
-    // ---------------- warp-local lazy online softmax: rare path when a logit passes its
-    // reference by kTau or a value scale passes the group's power-of-two headroom
-    bool rare = false;
-    #pragma unroll
-    for (int kk = 0; kk < kWarpTiles; ++kk) {
-      #pragma unroll
-      for (int e = 0; e < 2; ++e) rare |= s2[kk][e] > thr_my[e];
-      #pragma unroll
-      for (int j = 0; j < 2; ++j) rare |= sc[kk][j] > smax_my[j];
-    }
-    if (__any_sync(kFull, rare)) {
-      float lm[2];
-      #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        lm[e] = s2[0][e];
+      for (int kk = 0; kk < 2; ++kk) {
+        int d[4];
+        score_tile(d, kbits[(16 * kk + g) * 4], kbits[(16 * kk + g + 8) * 4], bq);
         #pragma unroll
-        for (int kk = 1; kk < kWarpTiles; ++kk) lm[e] = fmaxf(lm[e], s2[kk][e]);
-      }
-      #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        // lanes whose slot (h & 1) is head h contribute; the rest give -inf
-        float mx = (hs0 == (h & ~1)) ? lm[h & 1] : -INFINITY;
-        #pragma unroll
-        for (int m = 16; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
-        if (mx > m_thr[h]) {  // warp-uniform
-          const float alpha = ex2(m_w[h] - mx);  // 0 while m_w is still kNoMax
-          m_w[h] = mx;
-          m_thr[h] = mx + kTau;
-          if (hs0 == (h & ~1)) l_acc[h & 1] = __fmul_rn(l_acc[h & 1], alpha);
-          mid_acc[h][0] = __fmul_rn(mid_acc[h][0], alpha);
-          mid_acc[h][1] = __fmul_rn(mid_acc[h][1], alpha);
-          const float f = (t4 == h) ? alpha : 1.0f;
-          #pragma unroll
-          for (int mt = 0; mt < 8; ++mt)
-            #pragma unroll
-            for (int k = 0; k < 4; ++k) D[mt][k] = __fmul_rn(D[mt][k], f);
+        for (int e = 0; e < 2; ++e) {
+          const int tt = 16 * kk + g + 8 * e;
+          const bool valid = tt < lim;
+          const float nc = __fmul_rn(knorm[tt], kcinv[tt]);
+          const float dot = __fmaf_rn(c1_t, static_cast<float>(d[2 * e]), __fmaf_rn(c2_t, static_cast<float>(d[2 * e + 1]), c0_t));
+          s2[kk][e] = (valid && hv_t) ? __fmul_rn(dot, nc) : -INFINITY;
+          const uint32_t smw = valid ? vsm[tt * 4] : 0u;  // (scale, min) of group t
+          sc[kk][e] = __half2float(__ushort_as_half(static_cast<unsigned short>(smw & 0xffffu)));
+          mn[kk][e] = __half2float(__ushort_as_half(static_cast<unsigned short>(smw >> 16)));
+          rare |= (s2[kk][e] > thr_t) | (sc[kk][e] > smax_t);
         }
       }
-      #pragma unroll
-      for (int e = 0; e < 2; ++e) {  // slot e is head e (t & 1 == 0) or head 2 + e
-        const float mlo = (e < G) ? m_w[e < G ? e : 0] : kNoMax;
-        const float tlo = (e < G) ? m_thr[e < G ? e : 0] : kNoMax;
-        const float mhi = (2 + e < G) ? m_w[2 + e < G ? 2 + e : 0] : kNoMax;
-        const float thi = (2 + e < G) ? m_thr[2 + e < G ? 2 + e : 0] : kNoMax;
-        m_my[e] = hs0 ? mhi : mlo;
-        thr_my[e] = hs0 ? thi : tlo;
-      }
-      #pragma unroll
-      for (int g = 0; g < 4; ++g) {
-        float mx = 0.0f;  // lanes holding group g contribute their scales
-        if (q1 == (g >> 1)) {
-          #pragma unroll
-          for (int kk = 0; kk < kWarpTiles; ++kk) mx = fmaxf(mx, sc[kk][g & 1]);
-        }
+      // ---------------- rare path: raise a head's reference maximum or a group's scale bound
+      if (__any_sync(kFull, rare)) {
+        float mx = fmaxf(fmaxf(s2[0][0], s2[0][1]), fmaxf(s2[1][0], s2[1][1]));
+        float sx = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
         #pragma unroll
-        for (int m = 16; m >= 1; m >>= 1) mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
-        if (mx > smax[g]) {  // warp-uniform
-          const int e_new = 6 - ilog2_pos(mx);
-          smax[g] = exp2i(7 - e_new);  // scales up to 2^(7-E) keep p * scale * 2^E <= 2^15
-          if (e_new < E_w[g]) {
-            const float beta = exp2i(e_new - E_w[g]);  // D is still 0 while E_w is kNoExp
-            #pragma unroll
-            for (int k = 0; k < 4; ++k) {
-              D[2 * g][k] = __fmul_rn(D[2 * g][k], beta);
-              D[2 * g + 1][k] = __fmul_rn(D[2 * g + 1][k], beta);
-            }
-            E_w[g] = e_new;
+        for (int m = 4; m <= 16; m <<= 1) {
+          mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
+          sx = fmaxf(sx, __shfl_xor_sync(kFull, sx, m));
+        }
+        float alpha[4];
+        bool changed = false;
+        int E_new[4];
+        #pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          const float mh = __shfl_sync(kFull, mx, h);  // lane h has t = h
+          const float sh = __shfl_sync(kFull, sx, h);
+          alpha[h] = 1.0f;
+          if (mh > m_w[h] + static_cast<float>(kTau)) {  // warp-uniform
+            alpha[h] = (m_w[h] == kNoMax) ? 0.0f : ex2(m_w[h] - mh);
+            m_w[h] = mh;
+            changed = true;
+          }
+          E_new[h] = E_w[h];
+          if (sh > smax_w[h]) {  // warp-uniform; group h
+            const int k = ilog2_pos(sh);
+            smax_w[h] = exp2i(k + 1);  // scales < 2^(k+1) keep W = p scale 2^E < 2^kTau 2^(k+1) 2^E = 2^32
+            E_new[h] = 31 - kTau - k;
+            changed |= E_new[h] != E_w[h];
           }
         }
-      }
-      #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        smax_my[j] = q1 ? smax[2 + j] : smax[j];
-        ef_my[j] = exp2i(q1 ? E_w[2 + j] : E_w[j]);
-      }
-    }
-    #pragma unroll
-    for (int kk = 0; kk < kWarpTiles; ++kk) {
-      float pr[2];
-      #pragma unroll
-      for (int e = 0; e < 2; ++e) {
-        pr[e] = ex2(s2[kk][e] - m_my[e]);  // -inf for invalid tokens and empty slots -> 0
-        l_acc[e] = __fadd_rn(l_acc[e], pr[e]);
-      }
-      // p of all four heads for this token: heads 0, 1 from the pair's even lane, 2, 3 from the odd
-      float ph[4];
-      ph[0] = __shfl_sync(kFull, pr[0], lane & ~1);
-      ph[1] = __shfl_sync(kFull, pr[1], lane & ~1);
-      ph[2] = G > 2 ? __shfl_sync(kFull, pr[0], lane | 1) : 0.0f;
-      ph[3] = G > 2 ? __shfl_sync(kFull, pr[1], lane | 1) : 0.0f;
-      #pragma unroll
-      for (int h = 0; h < G; ++h) {
-        mid_acc[h][0] = __fmaf_rn(ph[h], mid[kk][0], mid_acc[h][0]);
-        mid_acc[h][1] = __fmaf_rn(ph[h], mid[kk][1], mid_acc[h][1]);
-      }
-      // this token's B rows of the lane's two groups: 8 halves (head, hi/lo)
-      #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const float f = __fmul_rn(sc[kk][j], ef_my[j]);
-        uint32_t row[4];
-        #pragma unroll
-        for (int hp = 0; hp < 2; ++hp) {
-          const uint64_t w2 = mul2(f2pack(ph[2 * hp], ph[2 * hp + 1]), f2pack(f, f));
-          const uint64_t hi2 = w2 & 0xFFFFE000FFFFE000ull;  // 11 significant bits each
-          const uint64_t lo2 = sub2(w2, hi2);
-          asm("cvt.rn.f16x2.f32 %0, %1, %2;"
-              : "=r"(row[2 * hp])
-              : "f"(__uint_as_float(static_cast<uint32_t>(lo2))), "f"(__uint_as_float(static_cast<uint32_t>(hi2))));
-          asm("cvt.rn.f16x2.f32 %0, %1, %2;"
-              : "=r"(row[2 * hp + 1])
-              : "f"(__uint_as_float(static_cast<uint32_t>(lo2 >> 32))), "f"(__uint_as_float(static_cast<uint32_t>(hi2 >> 32))));
+        if (changed) {
+          drain(alpha);
+          #pragma unroll
+          for (int h = 0; h < 4; ++h) E_w[h] = E_new[h];
         }
-        *reinterpret_cast<uint4*>(brows + ((2 * q1 + j) * kGroupRows + kk * 16 + tokr) * 16) =
-            make_uint4(row[0], row[1], row[2], row[3]);
+        l_t = __fmul_rn(l_t, sel4(alpha, t));
+        #pragma unroll
+        for (int h = 0; h < 4; ++h) mid[h] = __fmul_rn(mid[h], alpha[h]);
+        m_t = sel4(m_w, t);
+        thr_t = m_t + static_cast<float>(kTau);
+        s2e_t = exp2i(sel4(E_w, t));
+        smax_t = sel4(smax_w, t);
+      }
+      // ---------------- probabilities of head t, then every head's p for this lane's tokens
+      float ph[2][2][4];
+      #pragma unroll
+      for (int kk = 0; kk < 2; ++kk)
+        #pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float pr = ex2(s2[kk][e] - m_t);  // -inf for invalid tokens and absent heads -> 0
+          l_t = __fadd_rn(l_t, pr);
+          #pragma unroll
+          for (int h = 0; h < 4; ++h) ph[kk][e][h] = (h < G) ? __shfl_sync(kFull, pr, (lane & ~3) | h) : 0.0f;
+        }
+      // ---------------- weights of group t: W = rint(p scale 2^E) < 2^32
+      #pragma unroll
+      for (int kk = 0; kk < 2; ++kk) {
+        uint32_t W[2][4];
+        #pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const float s2g = __fmul_rn(sc[kk][e], s2e_t);
+          #pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            W[e][h] = __float2uint_rn(__fmul_rn(ph[kk][e][h], s2g));
+            mid[h] = __fmaf_rn(ph[kk][e][h], mn[kk][e], mid[h]);
+          }
+        }
+        uint32_t rlo[4], rhi[4];
+        #pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          rlo[h] = prmt(W[0][h], W[1][h], 0x5410);  // bytes 0, 1 of tokens g, g + 8
+          rhi[h] = prmt(W[0][h], W[1][h], 0x7632);  // bytes 2, 3
+        }
+        stsm_x4_t8(wbase + (kk * 4 * 2) * 128 + st_off, rlo);
+        stsm_x4_t8(wbase + (kk * 4 * 2 + 1) * 128 + st_off, rhi);
+      }
+      __syncwarp();
+      // ---------------- P.V: per group, A = weight bytes (rows (head, byte)), B = codes (8 channels)
+      const uint32_t ctile = smem_u32(st + kOffCodes + tl * kTileSmem);
+      const int c_row = lane & 7, c_ntile = (lane >> 4), c_k16 = (tw >> 4) + ((lane >> 3) & 1);
+      #pragma unroll
+      for (int grp = 0; grp < 4; ++grp) {
+        uint32_t a[4];
+        ldsm_x4(a, wbase + a_off0 + (((a_rho0 + 2 * grp) & 7) * 16));
+        #pragma unroll
+        for (int pr = 0; pr < 2; ++pr) {
+          const int ch = 8 * (4 * grp + 2 * pr + c_ntile) + c_row;
+          uint32_t b[4];
+          ldsm_x4_u4(b, ctile + ch * 128 + ((c_k16 ^ (ch & 7)) << 4));
+          imma_u8(D[4 * grp + 2 * pr], a, b[0], b[1]);
+          imma_u8(D[4 * grp + 2 * pr + 1], a, b[2], b[3]);
+        }
       }
     }
     __syncwarp();
-
-    // ---------------- P.V: this warp's kWarpTiles tiles x 8 m-tiles, chunk partial flushed into D
-    const uint32_t* codes = reinterpret_cast<const uint32_t*>(st + kOffCodes + warp * kWarpTiles * 1024) + lane;
-    if (my_tiles > 0) {
-      float tmp[8][4];
-      #pragma unroll
-      for (int kk = 0; kk < kWarpTiles; ++kk) {
-        if (kk < my_tiles) {
-          uint32_t bf[4][2];
-          #pragma unroll
-          for (int g = 0; g < 4; ++g) ldsm_x2_trans(bf[g][0], bf[g][1], bbase + (g * kGroupRows + kk * 16) * 16);
-          #pragma unroll
-          for (int mt = 0; mt < 8; ++mt) {
-            uint32_t a[4];
-            codes_to_afrag(codes[kk * 256 + mt * 32], a);
-            if (kk == 0) mma16816_zc(tmp[mt], a, bf[mt >> 1][0], bf[mt >> 1][1]);
-            else mma16816(tmp[mt], a, bf[mt >> 1][0], bf[mt >> 1][1]);
-          }
-        }
-      }
-      #pragma unroll
-      for (int mt = 0; mt < 8; ++mt)
-        #pragma unroll
-        for (int k = 0; k < 4; ++k) D[mt][k] = __fadd_rn(D[mt][k], tmp[mt][k]);
-    }
-    __syncwarp();
-
     // ---------------- release the stage to the producer
     if (lane == 0) mbar_arrive(&empty_bar[s]);  // the warp's reads of the stage completed before __syncwarp
     it.advance(nt, Lt);
@@ -774,6 +719,31 @@ static cudaError_t launch_t(const AttendWsParams& p, cudaStream_t stream) {
   return cudaGetLastError();
 }
 
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+// The code plane as a 3-D tensor of 4-bit elements: [tiles][128 channels][128 tokens], one box per
+// tile.  Host-only (no device work); the driver function is looked up once through the runtime.
+static cudaError_t encode_codes_map(CUtensorMap* map, const uint32_t* v_codes, int64_t tiles) {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    cudaDriverEntryPointQueryResult q;
+    void* f = nullptr;
+    cudaError_t e = cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q);
+    if (e != cudaSuccess || q != cudaDriverEntryPointSuccess || !f) return e != cudaSuccess ? e : cudaErrorNotSupported;
+    fn = reinterpret_cast<EncodeTiledFn>(f);
+  }
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(kTileTok), 128, static_cast<cuuint64_t>(tiles)};
+  const cuuint64_t strides[2] = {kTileTok / 2, kTileTok / 2 * 128};  // bytes: one channel row, one tile
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(kTileTok), 128, 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_16U4_ALIGN16B, 3, const_cast<uint32_t*>(v_codes), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? cudaSuccess : cudaErrorInvalidValue;
+}
+
 }  // namespace ws
 }  // namespace kv1b
 
@@ -781,10 +751,11 @@ using namespace kv1b;
 
 bool kv1b_ws_supported(int32_t G) { return G == 1 || G == 2 || G == 4; }
 
-// CTAs = SMs (fewer when there are fewer tiles); partial rows per segment = pieces x 16 warps.
+// CTAs = SMs (fewer when there are fewer tiles); T, Lt in 128-token tiles; partial rows per
+// segment = the most CTAs one segment can touch.
 void kv1b_ws_plan(int32_t B, int32_t Hkv, int32_t G, int64_t L, int num_sms, int64_t* T, int64_t* Lt, int* ncta,
                   int* max_pieces) {
-  const int64_t lt = (L + 15) / 16;
+  const int64_t lt = (L + ws::kTileTok - 1) / ws::kTileTok;
   const int64_t tot = static_cast<int64_t>(B) * Hkv * lt;
   int n = num_sms;
   if (tot < n) n = static_cast<int>(tot > 0 ? tot : 1);
@@ -795,7 +766,10 @@ void kv1b_ws_plan(int32_t B, int32_t Hkv, int32_t G, int64_t L, int num_sms, int
   (void)G;
 }
 
-cudaError_t kv1b_launch_attend_ws(const AttendWsParams& p, int32_t G, cudaStream_t stream) {
+cudaError_t kv1b_launch_attend_ws(AttendWsParams& p, int32_t G, cudaStream_t stream) {
+  const int64_t tiles = static_cast<int64_t>(p.c.B) * p.c.Hkv * (p.c.cap / ws::kTileTok);
+  const cudaError_t e = ws::encode_codes_map(&p.codes_map, p.c.v_codes, tiles);
+  if (e != cudaSuccess) return e;
   switch (G) {
     case 1: return ws::launch_t<1>(p, stream);
     case 2: return ws::launch_t<2>(p, stream);

@@ -30,7 +30,7 @@ __global__ void init_kernel(uint64_t seed, float* signs, int32_t* lengths, int32
 
 // One block per (16-token tile touched by the append, kv-head, sequence); warp r handles tile
 // slot r.  Keys and v_sm are token-major and written directly; the 4-bit codes of the tile are
-// staged in shared memory and then written as whole 32-bit words in the mma A-fragment order
+// staged in shared memory and then written as whole 32-bit words of the channel-major code plane
 // (read-modify-write keeps the nibbles of tokens already in the tile).
 __global__ void __launch_bounds__(512) encode_kernel(const EncodeParams p) {
   __shared__ uint8_t codes[16][kD];
@@ -110,24 +110,22 @@ __global__ void __launch_bounds__(512) encode_kernel(const EncodeParams p) {
     if (lane == 0 && flags) atomicOr(p.status, flags);
   }
   __syncthreads();
-  // ---- assemble the tile's code words: thread = (m-tile, lane) of the A fragment
+  // ---- write the tile's codes: thread = (channel, half of the 16 tokens); the 8 tokens' nibbles
+  // form one 32-bit word of the channel's 64-byte row in its 128-token tile (nibble j = token j
+  // of the 8), read-modify-write keeps the nibbles of tokens already in the cache.
   if (threadIdx.x < 256) {
-    const int mt = threadIdx.x >> 5, l = threadIdx.x & 31;
-    const int g = l >> 2, t = l & 3;
-    // slot order: bits 0,16,4,20,8,24,12,28  <->  (channel offset, token) pairs
-    const int ch_off[8] = {0, 0, 8, 8, 0, 0, 8, 8};
-    const int tok[8] = {2 * t, 2 * t + 1, 2 * t, 2 * t + 1, 2 * t + 8, 2 * t + 9, 2 * t + 8, 2 * t + 9};
-    const int shift[8] = {0, 16, 4, 20, 8, 24, 12, 28};
-    uint32_t* dst = p.v_codes + ((static_cast<int64_t>(b) * p.Hkv + h) * (p.cap / 16) + tile) * 256 + mt * 32 + l;
+    const int ch = threadIdx.x >> 1, half = threadIdx.x & 1;
+    const int64_t seg = static_cast<int64_t>(b) * p.Hkv + h;
+    uint32_t* dst = p.v_codes + ((seg * (p.cap / 128) + tile / 8) * kD + ch) * 16 + (tile & 7) * 2 + half;
     bool all_new = true;
     #pragma unroll
-    for (int i = 0; i < 8; ++i) all_new = all_new && s_new[tok[i]];
+    for (int j = 0; j < 8; ++j) all_new = all_new && s_new[8 * half + j];
     uint32_t w = all_new ? 0u : *dst;
     #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      if (s_new[tok[i]]) {
-        const uint32_t c = codes[tok[i]][16 * mt + g + ch_off[i]];
-        w = (w & ~(0xfu << shift[i])) | (c << shift[i]);
+    for (int j = 0; j < 8; ++j) {
+      if (s_new[8 * half + j]) {
+        const uint32_t c = codes[8 * half + j][ch];
+        w = (w & ~(0xfu << (4 * j))) | (c << (4 * j));
       }
     }
     *dst = w;

@@ -1,5 +1,6 @@
 // kv1b_launch.h -- internal host<->device interface: kernel parameter blocks and launchers.
 #pragma once
+#include <cuda.h>  // CUtensorMap (the descriptor type only; encoded through the runtime entry point)
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -72,24 +73,24 @@ struct ToppParams {
 
 constexpr int kPartStride = 2 + 128;
 
-// persistent warp-specialised attend (kv1b_attend_ws.cu)
-struct AttendWsParams {
+// persistent attend on the integer tensor cores (kv1b_attend_ws.cu)
+struct alignas(64) AttendWsParams {
+  CUtensorMap codes_map;  // v_codes as [tiles][128 channels][128 4-bit tokens], 16U4_ALIGN16B, 128B swizzle
   CacheView c;
   const void* q;
   int32_t q_dtype;
   int32_t Hq;
   float scale;
   int32_t L;           // tokens per sequence (equal for every sequence)
-  int64_t T;           // total 16-token tiles over all (sequence, kv-head) segments
+  int64_t T;           // total 128-token tiles over all (sequence, kv-head) segments
   int64_t Lt;          // tiles per segment
   int32_t ncta;        // CTAs (one per SM)
   int32_t max_pieces;  // partial slots per segment
-  float* part;         // [segments][max_pieces][warps][G][6 + 128]: m, l, mid[4], o[128]
+  float* part;         // [segments][max_pieces][G][2 + 128]: m (log2 units), l, o[128]
   float* out;          // [B][Hq][128]
   int32_t* status;     // cache status word (timeout flag)
   unsigned* counters;  // [B * Hkv] pieces of each segment written so far (zeroed before the launch)
 };
-constexpr int kPartStrideWs = 6 + 128;
 
 }  // namespace kv1b
 
@@ -106,4 +107,4 @@ int kv1b_pick_splits(int32_t B, int32_t Hkv, int64_t max_len, int num_sms);
 bool kv1b_ws_supported(int32_t G);
 void kv1b_ws_plan(int32_t B, int32_t Hkv, int32_t G, int64_t L, int num_sms, int64_t* T, int64_t* Lt, int* ncta,
                   int* max_pieces);
-cudaError_t kv1b_launch_attend_ws(const kv1b::AttendWsParams& p, int32_t G, cudaStream_t stream);
+cudaError_t kv1b_launch_attend_ws(kv1b::AttendWsParams& p, int32_t G, cudaStream_t stream);

@@ -170,25 +170,20 @@ __global__ void __launch_bounds__(kToppThreads) topp_kernel(const ToppParams p) 
   const uint32_t* vsm = c.v_sm + head_tok * 4;
   float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
   float lsum = 0.0f;
-  const int mt = lane >> 2;                 // m-tile of channels 4l..4l+3
   const int grp = lane >> 3;                // 32-channel group
   for (int i = warp; i < base; i += kToppWarps) {
     const int64_t t = sel[i];
     const float e = exp2f(__fmul_rn(__fsub_rn(s[t], m), kL2e));
     lsum += e;
-    const int64_t tile = t >> 4;
-    const int r16 = static_cast<int>(t & 15);
-    const int tq = (r16 & 7) >> 1, second = r16 >> 3, odd = r16 & 1;
+    // code plane: 128-token tiles, channel-major rows of 16 words, nibble j of word w = token 8w + j
+    const uint32_t* row = vcw + ((t >> 7) * kD + 4 * lane) * 16 + ((t & 127) >> 3);
+    const int shift = 4 * static_cast<int>(t & 7);
     const uint32_t smw = vsm[t * 4 + grp];
     const float scl = __half2float(__ushort_as_half(static_cast<unsigned short>(smw & 0xffffu)));
     const float mnv = __half2float(__ushort_as_half(static_cast<unsigned short>(smw >> 16)));
     #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      const int cm = 4 * (lane & 3) + r;    // channel within the m-tile
-      const int g = cm & 7, upper = cm >> 3;
-      const uint32_t word = vcw[tile * 256 + mt * 32 + g * 4 + tq];
-      const int shift = 8 * second + 4 * upper + 16 * odd;
-      const float code = static_cast<float>((word >> shift) & 0xFu);
+      const float code = static_cast<float>((row[16 * r] >> shift) & 0xFu);
       acc[r] = __fmaf_rn(e, __fmaf_rn(scl, code, mnv), acc[r]);
     }
   }
