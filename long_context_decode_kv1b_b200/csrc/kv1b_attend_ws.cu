@@ -3,36 +3,38 @@
 // Work split: all (sequence, kv-head) segments are laid end to end in 128-token tiles and cut into
 // one equal contiguous range per CTA, so every SM streams the same number of compressed bytes
 // whatever the batch / head / context mix.  A producer warp walks the CTA's range in stages of up
-// to two tiles (256 tokens) of one segment through a 4-deep shared-memory ring: one TMA tensor load
-// per tile brings the tile's 4-bit value codes ([128 channels][128 tokens], data type 16U4_ALIGN16B:
-// every 8 bytes of packed codes land in a 16-byte slot, 128-byte swizzle), and four plain bulk
-// copies bring the key bits, N, 1/C and the fp16 (scale, min) pairs.  Completion is tracked by
-// mbarriers with transaction bytes; the 8 compute warps release a stage by arriving on its "empty"
-// barrier.  Compute warp w owns tokens 32 (w & 3) .. + 31 of the stage's tile w >> 2.
+// to three tiles (384 tokens) of one segment through a 3-deep shared-memory ring: one TMA tensor
+// load per tile brings the tile's 4-bit value codes ([128 channels][128 tokens], data type
+// 16U4_ALIGN16B: every 8 bytes of packed codes land in a 16-byte slot, 128-byte swizzle), and four
+// plain bulk copies bring the key bits, N, 1/C and the fp16 (scale, min) pairs.  Completion is
+// tracked by mbarriers with transaction bytes; the 12 compute warps release a stage by arriving on
+// its "empty" barrier.  The producer's warpgroup gives most of its registers to the compute
+// warpgroups (setmaxnreg), so three compute warps share each SM sub-partition.
 //
-// Per 32-token slice a warp computes, for the G <= 4 query heads of the segment:
+// The compute warps work in 6 pairs; pair p owns 64 tokens of a stage (tile p >> 1, tokens
+// 64 (p & 1) ..), warp half j of the pair owns the 32-token slice j of them for the scores and
+// channels 64 j .. 64 j + 63 for the P.V:
 //   scores ("RaBitQCache", abstract / key design: binary x INT4 arithmetic): per 16 tokens, four
 //     mma.m16n8k32 s8 products of the key sign bits (A, one AND per register: each byte keeps one
 //     bit in place) with the query's 4-bit codes (B, column 2h = head h scaled to undo the bit
 //     position, column 2h + 1 = ones), so lane (g, t) receives 8 A and 8 Bc of tokens g and g + 8
 //     for head t exactly -- the integers of the popcount form;
 //   softmax: lane (g, t) turns them into head t's logits (log2 units) and probabilities against a
-//     warp-uniform reference maximum that is raised only when a logit passes it by kTau (then the
+//     reference maximum shared by the pair and raised only when a logit passes it by kTau (then the
 //     accumulators are rescaled), so every p <= 2^kTau;
 //   weights ("H1B-KV", technical framework: weights from the sketch, then the 4-bit values): lane
 //     (g, t) takes value group t of its tokens for all heads (the heads' p by shuffles within the
-//     lane quad) and forms W = p * scale * 2^E rounded to an unsigned 32-bit integer; E is a
-//     per-group power of two kept in step with the largest scale seen, so W < 2^32 and the weights
-//     of tokens far below the maximum keep many significant bits (a fixed point with fewer bits
-//     would round the long tail of a wide softmax to zero and bias the sum).  stmatrix (.trans, b8)
-//     writes the four bytes of every W into a per-warp buffer; ldmatrix gathers them as the A
-//     operand (rows = (head, byte));
+//     lane quad) and forms W = rint(p * scale * 2^E) < 2^32; E is a per-group power of two kept in
+//     step with the largest scale seen (the pair shares it), so the weights of tokens far below the
+//     maximum keep many significant bits (a fixed point with fewer bits would round the long tail
+//     of a wide softmax to zero and bias the sum).  stmatrix (.trans, b8) writes the four bytes of
+//     every W into the pair's buffer; ldmatrix gathers them as the A operand (rows = (head, byte));
 //   P.V: ldmatrix .b8x16.b4x16_p64 expands the staged codes to one byte per code (the B operand,
 //     k = tokens), and mma.m16n8k32 u8 x u8 -> s32 accumulates sum_t W * code per (head, byte,
 //     channel) EXACTLY in 32-bit integers; value = min + scale * code, the min term is summed per
 //     (head, group) in fp32.  The integer accumulators are converted (and rescaled) only when the
 //     reference maximum or a group exponent moves, and at the end of a segment piece.
-// At the end of a segment piece the 8 warps' partials are combined in shared memory and the CTA
+// At the end of a segment piece the pairs' partials are combined in shared memory and the CTA
 // writes one row (m, l, o[128]) per query head; the CTA that writes a segment's last row merges
 // the segment's rows by log-sum-exp into the output (one kernel per attend).
 //
@@ -45,38 +47,43 @@
 namespace kv1b {
 namespace ws {
 
-constexpr int kWarps = 8;                   // compute warps; one more warp issues the copies
-constexpr int kThreads = kWarps * 32;       // 256 compute threads
-constexpr int kBlock = kThreads + 32;       // + the producer warp
+constexpr int kPairs = 6;
+constexpr int kWarps = 2 * kPairs;          // compute warps
+constexpr int kThreads = kWarps * 32;       // 384 compute threads
+constexpr int kBlock = kThreads + 128;      // + the producer warpgroup
+constexpr int kComputeRegs = 152;           // setmaxnreg: 384 x 152 + 128 x 40 <= 512 x 128 registers
+constexpr int kProducerRegs = 40;
+static_assert(kThreads * kComputeRegs + 128 * kProducerRegs <= 65536, "register split within the launch's registers");
 constexpr int kTileTok = 128;               // tokens per code tile (one TMA box)
-constexpr int kStageTiles = 2;
+constexpr int kStageTiles = 3;
 constexpr int kStageTok = kStageTiles * kTileTok;
-constexpr int kStages = 4;
-constexpr int kTau = 2;                     // lazy-max threshold (log2 units): p <= 2^kTau
+constexpr int kStages = 3;
+constexpr int kTau = 4;                     // lazy-max threshold (log2 units): p <= 2^kTau
+constexpr int kScaleRoom = 2;               // bits of headroom above the largest scale seen
 constexpr int kNoExp = 100;                 // group exponent before any scale was seen
 constexpr float kNoMax = -1e30f;            // reference maximum before any logit was seen
-constexpr int kMaxAccStages = 8192;         // int32 headroom: 255 * 15 * 32 * 8192 < 2^31
+constexpr int kMaxAccStages = 8192;         // int32 headroom: 255 * 15 * 64 tokens * 8192 < 2^31
 constexpr long long kSpinLimit = 1LL << 24;
 
 // Stage layout (bytes).
 constexpr int kTileSmem = kTileTok * 128;                  // 128 channels x 128 B (8 B codes + 8 B gap per 16 tokens)
 constexpr int kOffCodes = 0;
-constexpr int kOffBits = kStageTiles * kTileSmem;          // u32 [256][4]
-constexpr int kOffNorm = kOffBits + kStageTok * 16;        // f32 [256]
-constexpr int kOffCinv = kOffNorm + kStageTok * 4;         // f32 [256]
-constexpr int kOffSm = kOffCinv + kStageTok * 4;           // u32 [256][4]
+constexpr int kOffBits = kStageTiles * kTileSmem;          // u32 [384][4]
+constexpr int kOffNorm = kOffBits + kStageTok * 16;        // f32 [384]
+constexpr int kOffCinv = kOffNorm + kStageTok * 4;         // f32 [384]
+constexpr int kOffSm = kOffCinv + kStageTok * 4;           // u32 [384][4]
 constexpr int kStageBytes = (kOffSm + kStageTok * 16 + 1023) / 1024 * 1024;
-constexpr int kWBytes = 16 * 128;                          // per warp: 16 byte matrices of 8 rows x 16 tokens
+constexpr int kWSlice = 16 * 128;                          // one warp's 32 tokens: 16 byte matrices of 8 rows x 16 tokens
+constexpr int kWPair = 2 * kWSlice;
 constexpr int kOffW = kStages * kStageBytes;
-constexpr int kRowF = 6 + 128;                             // per-warp partial row: m, l, mid[4], o[128]
-constexpr int kPartBytes = 4 * kRowF * 4;
-constexpr int kOffPart = kOffW + kWarps * kWBytes;
-constexpr int kSmemUsed = kOffPart + kWarps * kPartBytes;
+constexpr int kRowP = 140;                                 // pair partial row per head: m, l0, l1, -, mid0[4], mid1[4], o[128]
+constexpr int kSmemUsed = kOffW + kPairs * kWPair;
 constexpr int kSmemBytes = kSmemUsed + 1024;               // + slack to align the base to 1024 B
 constexpr uint32_t kTxPerTile = kTileTok * 104;            // packed codes 64 B + 40 B of the other planes per token
 static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 static_assert(kOffW % 1024 == 0 && kStageBytes % 1024 == 0, "TMA 128B-swizzle destinations are 1024-B aligned");
-static_assert(2 * 4 * 256 * 4 + 64 <= kWarps * kPartBytes, "the segment merge reuses the partial area");
+static_assert(4 * kRowP * 4 <= kWPair, "a pair's partial rows fit its weight buffer");
+static_assert(2 * 4 * 256 * 4 + 64 <= kPairs * kWPair, "the segment merge reuses the weight buffers");
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 
@@ -257,6 +264,8 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
   __shared__ __align__(16) uint4 s_planes[2][4][4];     // double-buffered by segment parity
   __shared__ float s_vl[2][4], s_dl[2][4];
   __shared__ int s_sq[2][4];
+  __shared__ int s_rflag[kPairs][2];                     // a warp of the pair needs a rescale
+  __shared__ float s_xchg[kPairs][2][8];                 // its slice maxima: logits per head, scales per group
   __shared__ volatile int s_abort;
   __shared__ int s_merge;
 
@@ -281,8 +290,9 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
   it.seg = static_cast<int>(t_begin / p.Lt);
   it.lt = static_cast<int>(t_begin - static_cast<int64_t>(it.seg) * p.Lt);
   it.rem = static_cast<int>(t_end - t_begin);
-  if (warp == kWarps) {  // producer: one lane streams the CTA's stages through the ring
-    if (lane == 0) {
+  if (warp >= kWarps) {  // producer warpgroup: one lane streams the CTA's stages through the ring
+    asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kProducerRegs));
+    if (warp == kWarps && lane == 0) {
       TileIt is = it;
       int j = 0;  // stages issued
       while (is.rem > 0 && !s_abort) {
@@ -302,37 +312,47 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
     }
     return;
   }
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kComputeRegs));
 
   const int g = lane >> 2, t = lane & 3;
-  const int hh = g & 3;                  // head of this lane's P.V accumulator rows
-  const bool lo_bytes = (g >> 2) == 0;   // rows g / g + 8 hold bytes 0 / 2 (else bytes 1 / 3)
+  const int pr_ = warp >> 1, jh = warp & 1;  // pair, half
+  const int hh = g & 3;                      // head of this lane's P.V accumulator rows
+  const bool lo_bytes = (g >> 2) == 0;       // rows g / g + 8 hold bytes 0 / 2 (else bytes 1 / 3)
   const float qsl = __fmul_rn(__fdiv_rn(p.scale, static_cast<float>(kD)), 0x1.715476p+0f);  // scale/128 * log2 e
-  uint8_t* wbuf = smem + kOffW + warp * kWBytes;
-  const uint32_t wbase = smem_u32(wbuf);
+  const int tl = pr_ >> 1;                                  // the pair's tile in the stage
+  const int pbase = tl * kTileTok + (pr_ & 1) * 64;         // the pair's first token in the stage
+  const int sbase = pbase + 32 * jh;                        // this warp's score slice
+  uint8_t* wpair = smem + kOffW + pr_ * kWPair;
+  const uint32_t wpair_s = smem_u32(wpair);
   // stmatrix row address of this lane: matrix (kk, head m = lane >> 3, lo/hi), row rho = lane & 7
   // kept in slot (rho + 2 m) & 7 so that the A-operand gathers below are free of bank conflicts
-  const uint32_t st_off = static_cast<uint32_t>((lane >> 3) * 2 * 128 + (((lane & 7) + 2 * (lane >> 3)) & 7) * 16);
+  const uint32_t st_addr = wpair_s + jh * kWSlice +
+                           static_cast<uint32_t>((lane >> 3) * 2 * 128 + (((lane & 7) + 2 * (lane >> 3)) & 7) * 16);
   // A-operand gather for group grp: lane i addresses A row r = (i & 7) + 8 ((i >> 3) & 1) of
   // k-half kk = i >> 4; row r = (head r & 3, byte r >> 2)
   const int a_r = (lane & 7) + 8 * ((lane >> 3) & 1), a_kk = lane >> 4;
   const int a_head = a_r & 3, a_byte = a_r >> 2;
-  const uint32_t a_off0 = static_cast<uint32_t>(((a_kk * 4 + a_head) * 2 + (a_byte >> 1)) * 128);
+  const uint32_t a_addr = wpair_s + static_cast<uint32_t>(((a_kk * 4 + a_head) * 2 + (a_byte >> 1)) * 128);
   const int a_rho0 = (a_byte & 1) + 2 * a_head;
+  // code-tile gathers: lanes 8m .. 8m + 7 address channel rows 64 jh + 8 (2 np + (m >> 1)) + (lane & 7)
+  // of 16-token chunk k16 = (pair chunk) + 2 ks + (m & 1); 128-byte swizzle: chunk ^ (row & 7)
+  const uint32_t c_off = static_cast<uint32_t>(tl * kTileSmem + (64 * jh + 8 * (lane >> 4) + (lane & 7)) * 128);
+  uint32_t c_kx[2];
+  #pragma unroll
+  for (int ks = 0; ks < 2; ++ks) c_kx[ks] = static_cast<uint32_t>(((4 * (pr_ & 1) + 2 * ks + ((lane >> 3) & 1)) ^ (lane & 7)) << 4);
 
   // per-lane state
-  float m_w[4], smax_w[4];  // warp-uniform: reference maximum per head, scale bound per group
-  int E_w[4];               // warp-uniform: weight exponent per group
+  float m_w[4], smax_w[4];  // pair-uniform: reference maximum per head, scale bound per group
+  int E_w[4];               // pair-uniform: weight exponent per group
   float m_t, thr_t, s2e_t, smax_t;  // the same for this lane's head t / group t
   float l_t;                // sum p of head t over this lane's tokens
   float mid[4];             // sum p * min of group t, heads 0..3
-  int D[16][4];             // P.V integer accumulators: n-tile (8 channels) x (rows g, g + 8) x 2 channels
-  // converted P.V sums live in the warp's partial rows in shared memory: o[head][channel]
+  int D[8][4];              // P.V integer accumulators: n-tile (8 channels) x (rows g, g + 8) x 2 channels
+  float F[8][2];            // converted P.V sums of this lane's rows
   uint32_t bq[4][2];        // score-MMA query operand of this segment
   float c1_t, c2_t, c0_t;   // head t logit constants
   bool hv_t;                // head t exists
   int nacc = 0;             // stages accumulated in D since the last conversion
-
-  auto part_of = [&](int w) { return reinterpret_cast<float*>(smem + kOffPart + w * kPartBytes); };
 
   auto reset = [&]() {
     #pragma unroll
@@ -348,49 +368,39 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
     smax_t = 0.0f;
     l_t = 0.0f;
     #pragma unroll
-    for (int n = 0; n < 16; ++n) D[n][0] = D[n][1] = D[n][2] = D[n][3] = 0;
-    float* o = part_of(warp);
-    for (int i = lane; i < 4 * 128; i += 32) o[(i >> 7) * kRowF + 6 + (i & 127)] = 0.0f;
-    __syncwarp();
+    for (int n = 0; n < 8; ++n) {
+      D[n][0] = D[n][1] = D[n][2] = D[n][3] = 0;
+      F[n][0] = F[n][1] = 0.0f;
+    }
     nacc = 0;
   };
-  // Convert the integer accumulators (old exponents) and add them to the warp's o rows in shared
-  // memory, then scale head h's row by alpha[h]: lanes g and g + 4 hold bytes {0, 2} and {1, 3} of
-  // the same head and channels; lane g < 4 owns head g, channels 8n + 2t + e.
-  auto drain = [&](const float (&alpha)[4]) {
+  // Convert the integer accumulators into F (old exponents), then scale F by alpha of this lane's head.
+  auto drain = [&](float al) {
     const float wb0 = lo_bytes ? 1.0f : 256.0f, wb2 = lo_bytes ? 65536.0f : 16777216.0f;
-    const float al = sel4(alpha, hh);
-    float* o = part_of(warp) + hh * kRowF + 6 + 2 * t;
+    const float inv0 = exp2i(-(jh ? E_w[2] : E_w[0])), inv1 = exp2i(-(jh ? E_w[3] : E_w[1]));
     #pragma unroll
-    for (int n = 0; n < 16; ++n) {
-      const float inv = exp2i(-E_w[n >> 2]);
-      float x[2];
+    for (int n = 0; n < 8; ++n) {
+      const float inv = n < 4 ? inv0 : inv1;
       #pragma unroll
       for (int e = 0; e < 2; ++e) {
-        x[e] = __fmaf_rn(wb2, static_cast<float>(D[n][2 + e]), __fmul_rn(wb0, static_cast<float>(D[n][e])));
-        x[e] = __fadd_rn(x[e], __shfl_xor_sync(kFull, x[e], 16));
+        const float x = __fmaf_rn(wb2, static_cast<float>(D[n][2 + e]), __fmul_rn(wb0, static_cast<float>(D[n][e])));
+        F[n][e] = __fmul_rn(__fmaf_rn(x, inv, F[n][e]), al);
         D[n][e] = 0;
         D[n][2 + e] = 0;
       }
-      if (lo_bytes && hh < G) {
-        float2 v = *reinterpret_cast<float2*>(o + 8 * n);
-        v.x = __fmul_rn(__fmaf_rn(x[0], inv, v.x), al);
-        v.y = __fmul_rn(__fmaf_rn(x[1], inv, v.y), al);
-        *reinterpret_cast<float2*>(o + 8 * n) = v;
-      }
     }
-    __syncwarp();
     nacc = 0;
   };
 
+  auto prow = [&](int pp, int h) { return reinterpret_cast<float*>(smem + kOffW + pp * kWPair) + h * kRowP; };
+
   // Log-sum-exp merge of the n CTA rows of segment `seg` (per query head) into the output; uses
-  // the shared partial area.  All heads at once: thread t takes channel t & 127 of heads
-  // (t >> 7) + 2i, with the pieces' loads independent of one another.
-  static_assert(kThreads == 256, "two threads per channel in the merge");
+  // the weight buffers as scratch.  All heads at once: thread i takes channel i & 127 of heads
+  // (i >> 7) + 3k, with the pieces' loads independent of one another.
   auto merge_segment = [&](int seg, int n) {
-    float* sm_m = part_of(0);       // [G][256] piece maxima, then weights
-    float* sm_l = sm_m + 4 * 256;   // [G][256] piece sums
-    float* sm_d = sm_l + 4 * 256;   // [G] denominators
+    float* sm_m = reinterpret_cast<float*>(smem + kOffW);  // [G][256] piece maxima, then weights
+    float* sm_l = sm_m + 4 * 256;                          // [G][256] piece sums
+    float* sm_d = sm_l + 4 * 256;                          // [G] denominators
     const int b = seg / c.Hkv, kvh = seg - b * c.Hkv;
     const int64_t stride = static_cast<int64_t>(G) * kPartStride;  // between pieces
     const float* base = p.part + static_cast<int64_t>(seg) * p.max_pieces * G * kPartStride;
@@ -419,7 +429,7 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
     }
     named_bar(1, kThreads);
     const int ch = threadIdx.x & 127;
-    for (int h = threadIdx.x >> 7; h < G; h += 2) {
+    for (int h = threadIdx.x >> 7; h < G; h += kThreads / 128) {
       const float* w = sm_m + h * 256;
       const float* o = base + h * kPartStride + 2 + ch;
       float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
@@ -435,42 +445,50 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
     }
   };
 
-  // Segment piece done: each warp puts its partial (m, l, mid[4], o[128]) per head in shared
-  // memory; then thread (head, channel) combines the warps by log-sum-exp and writes the CTA's
-  // row (m, l, o[128] with the mid term folded in) for slot (segment, piece).  Every warp reaches
-  // this at the same stage.
+  // Segment piece done: each warp puts its share of the pair's partial (m, l, mid, o) per head in
+  // the pair's weight buffer; then thread (head, channel) combines the pairs by log-sum-exp and
+  // writes the CTA's row (m, l, o[128] with the mid terms folded in) for slot (segment, piece).
+  // Every compute warp reaches this at the same stage.
   auto flush = [&](int seg) {
-    const float ones[4] = {1.0f, 1.0f, 1.0f, 1.0f};
-    drain(ones);
+    drain(1.0f);
+    #pragma unroll
+    for (int n = 0; n < 8; ++n)  // rows g (g < 4) and g + 4 of the same head: bytes {0, 2} and {1, 3}
+      #pragma unroll
+      for (int e = 0; e < 2; ++e) F[n][e] = __fadd_rn(F[n][e], __shfl_xor_sync(kFull, F[n][e], 16));
     float v[5] = {l_t, mid[0], mid[1], mid[2], mid[3]};
     #pragma unroll
     for (int m = 4; m <= 16; m <<= 1)  // sum over the 8 lanes with the same t
       #pragma unroll
       for (int k = 0; k < 5; ++k) v[k] = __fadd_rn(v[k], __shfl_xor_sync(kFull, v[k], m));
-    float* mine = part_of(warp);
-    if (g == 0) {  // lane t: head t's m and l, group t's mid of every head
+    named_bar(1, kThreads);  // every pair is done with its weight buffer
+    if (g == 0) {  // lane t: head t's m and l of this slice, group t's mid of every head
       if (t < G) {
-        mine[t * kRowF] = m_t == kNoMax ? -INFINITY : m_t;
-        mine[t * kRowF + 1] = v[0];
+        if (jh == 0) prow(pr_, t)[0] = m_t == kNoMax ? -INFINITY : m_t;
+        prow(pr_, t)[1 + jh] = v[0];
       }
       #pragma unroll
-      for (int h = 0; h < G; ++h) mine[h * kRowF + 2 + t] = v[1 + h];
+      for (int h = 0; h < G; ++h) prow(pr_, h)[4 + 4 * jh + t] = v[1 + h];
+    }
+    if (g < G) {  // head g: channels 64 jh + 8n + 2t + e
+      float* o = prow(pr_, g) + 12 + 64 * jh + 2 * t;
+      #pragma unroll
+      for (int n = 0; n < 8; ++n) *reinterpret_cast<float2*>(o + 8 * n) = make_float2(F[n][0], F[n][1]);
     }
     named_bar(1, kThreads);
     const int ch = threadIdx.x & 127;
     for (int h = threadIdx.x >> 7; h < G; h += kThreads / 128) {
       float M = -INFINITY;
       #pragma unroll
-      for (int w = 0; w < kWarps; ++w) M = fmaxf(M, part_of(w)[h * kRowF]);
+      for (int q = 0; q < kPairs; ++q) M = fmaxf(M, prow(q, h)[0]);
       float num = 0.0f, den = 0.0f;
       if (M != -INFINITY) {
         #pragma unroll
-        for (int w = 0; w < kWarps; ++w) {
-          const float* r = part_of(w) + h * kRowF;
+        for (int q = 0; q < kPairs; ++q) {
+          const float* r = prow(q, h);
           if (r[0] == -INFINITY) continue;
           const float wt = exp2f(r[0] - M);
-          den = __fmaf_rn(wt, r[1], den);
-          num = __fmaf_rn(wt, __fadd_rn(r[6 + ch], r[2 + (ch >> 5)]), num);
+          den = __fmaf_rn(wt, __fadd_rn(r[1], r[2]), den);
+          num = __fmaf_rn(wt, __fadd_rn(r[12 + ch], __fadd_rn(r[4 + (ch >> 5)], r[8 + (ch >> 5)])), num);
         }
       }
       const int64_t piece = blockIdx.x - cta_of_tile(wk, static_cast<int64_t>(seg) * wk.Lt);
@@ -497,7 +515,7 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
       __threadfence();
       merge_segment(seg, npieces);
     }
-    named_bar(1, kThreads);  // the shared partials may be rewritten by the next flush
+    named_bar(1, kThreads);  // the buffers may be rewritten by the next segment
   };
 
   // Query preparation of a segment's G heads (warp h -> head h) into buffer seg & 1, then every
@@ -520,7 +538,7 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
         s_sq[par][warp] = qp.sq;
       }
     }
-    named_bar(1, kThreads);  // reached by every warp at the same stage
+    named_bar(1, kThreads);  // reached by every compute warp at the same stage
     const int hb = g >> 1;
     const bool code_col = (g & 1) == 0 && hb < G;
     uint32_t pw[4] = {0u, 0u, 0u, 0u};
@@ -552,7 +570,6 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
   reset();
   int cur_seg = it.seg;
   if (it.rem > 0) prep(cur_seg);
-  const int tl = warp >> 2, tw = (warp & 3) * 32;  // this warp's tile in the stage and token offset in it
   int s = 0;           // stage of the current step
   uint32_t phase = 0;  // parity of the stage's expected completion
   while (it.rem > 0) {
@@ -565,20 +582,18 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
     }
     mbar_wait(&full_bar[s], phase, &s_abort);
     const uint8_t* st = smem + s * kStageBytes;
-    int lim = L - (it.lt * kTileTok + tl * kTileTok + tw);  // real tokens of this warp's slice
-    lim = tl < nt ? (lim < 32 ? lim : 32) : 0;
-    if (lim > 0) {
-      if (nacc >= kMaxAccStages) {
-        const float ones[4] = {1.0f, 1.0f, 1.0f, 1.0f};
-        drain(ones);
-      }
+    const int rel = it.lt * kTileTok + sbase;          // this slice's first token in the segment
+    const bool pair_on = tl < nt && L > rel - 32 * jh;  // the pair has real tokens in this stage
+    if (pair_on) {
+      int lim = L - rel;                                // real tokens of this slice (may be <= 0)
+      lim = lim < 32 ? lim : 32;
+      if (nacc >= kMaxAccStages) drain(1.0f);
       ++nacc;
-      const int tbase = tl * kTileTok + tw;  // slice start within the stage
-      const uint32_t* kbits = reinterpret_cast<const uint32_t*>(st + kOffBits) + tbase * 4 + t;
-      const float* knorm = reinterpret_cast<const float*>(st + kOffNorm) + tbase;
-      const float* kcinv = reinterpret_cast<const float*>(st + kOffCinv) + tbase;
-      const uint32_t* vsm = reinterpret_cast<const uint32_t*>(st + kOffSm) + tbase * 4 + t;
-      // ---------------- scores of head t for tokens 16 kk + g + 8 e
+      const uint32_t* kbits = reinterpret_cast<const uint32_t*>(st + kOffBits) + sbase * 4 + t;
+      const float* knorm = reinterpret_cast<const float*>(st + kOffNorm) + sbase;
+      const float* kcinv = reinterpret_cast<const float*>(st + kOffCinv) + sbase;
+      const uint32_t* vsm = reinterpret_cast<const uint32_t*>(st + kOffSm) + sbase * 4 + t;
+      // ---------------- scores of head t for tokens 16 kk + g + 8 e of the slice
       float s2[2][2], sc[2][2], mn[2][2];
       bool rare = false;
       #pragma unroll
@@ -588,18 +603,22 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
         #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const int tt = 16 * kk + g + 8 * e;
-          const bool valid = tt < lim;
+          const bool valid = tt < lim && hv_t;
           const float nc = __fmul_rn(knorm[tt], kcinv[tt]);
           const float dot = __fmaf_rn(c1_t, static_cast<float>(d[2 * e]), __fmaf_rn(c2_t, static_cast<float>(d[2 * e + 1]), c0_t));
-          s2[kk][e] = (valid && hv_t) ? __fmul_rn(dot, nc) : -INFINITY;
-          const uint32_t smw = valid ? vsm[tt * 4] : 0u;  // (scale, min) of group t
+          s2[kk][e] = valid ? __fmul_rn(dot, nc) : -INFINITY;
+          const uint32_t smw = vsm[tt * 4];  // (scale, min) of group t; zeros past the end of the cache
           sc[kk][e] = __half2float(__ushort_as_half(static_cast<unsigned short>(smw & 0xffffu)));
-          mn[kk][e] = __half2float(__ushort_as_half(static_cast<unsigned short>(smw >> 16)));
-          rare |= (s2[kk][e] > thr_t) | (sc[kk][e] > smax_t);
+          mn[kk][e] = tt < lim ? __half2float(__ushort_as_half(static_cast<unsigned short>(smw >> 16))) : 0.0f;
         }
       }
-      // ---------------- rare path: raise a head's reference maximum or a group's scale bound
-      if (__any_sync(kFull, rare)) {
+      rare = (fmaxf(fmaxf(s2[0][0], s2[0][1]), fmaxf(s2[1][0], s2[1][1])) > thr_t) |
+             (fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1])) > smax_t);
+      const bool rare_w = __any_sync(kFull, rare);
+      if (lane == 0) s_rflag[pr_][jh] = rare_w;
+      named_bar(2 + pr_, 64);  // the pair's flags are posted; both warps are done with the weight buffer
+      // ---------------- rare path (pair-uniform): raise a head's reference maximum or a group's scale bound
+      if (rare_w || s_rflag[pr_][jh ^ 1]) {
         float mx = fmaxf(fmaxf(s2[0][0], s2[0][1]), fmaxf(s2[1][0], s2[1][1]));
         float sx = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
         #pragma unroll
@@ -607,6 +626,13 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
           mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
           sx = fmaxf(sx, __shfl_xor_sync(kFull, sx, m));
         }
+        if (g == 0) {
+          s_xchg[pr_][jh][t] = mx;
+          s_xchg[pr_][jh][4 + t] = sx;
+        }
+        named_bar(2 + pr_, 64);
+        mx = fmaxf(mx, s_xchg[pr_][jh ^ 1][t]);
+        sx = fmaxf(sx, s_xchg[pr_][jh ^ 1][4 + t]);
         float alpha[4];
         bool changed = false;
         int E_new[4];
@@ -615,21 +641,21 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
           const float mh = __shfl_sync(kFull, mx, h);  // lane h has t = h
           const float sh = __shfl_sync(kFull, sx, h);
           alpha[h] = 1.0f;
-          if (mh > m_w[h] + static_cast<float>(kTau)) {  // warp-uniform
+          if (mh > m_w[h] + static_cast<float>(kTau)) {  // pair-uniform
             alpha[h] = (m_w[h] == kNoMax) ? 0.0f : ex2(m_w[h] - mh);
             m_w[h] = mh;
             changed = true;
           }
           E_new[h] = E_w[h];
-          if (sh > smax_w[h]) {  // warp-uniform; group h
+          if (sh > smax_w[h]) {  // pair-uniform; group h
             const int k = ilog2_pos(sh);
-            smax_w[h] = exp2i(k + 1);  // scales < 2^(k+1) keep W = p scale 2^E < 2^kTau 2^(k+1) 2^E = 2^32
-            E_new[h] = 31 - kTau - k;
+            smax_w[h] = exp2i(k + 1 + kScaleRoom);  // W = p scale 2^E < 2^kTau 2^(k+1+room) 2^E = 2^32
+            E_new[h] = 31 - kTau - kScaleRoom - k;
             changed |= E_new[h] != E_w[h];
           }
         }
         if (changed) {
-          drain(alpha);
+          drain(sel4(alpha, hh));
           #pragma unroll
           for (int h = 0; h < 4; ++h) E_w[h] = E_new[h];
         }
@@ -671,24 +697,27 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
           rlo[h] = prmt(W[0][h], W[1][h], 0x5410);  // bytes 0, 1 of tokens g, g + 8
           rhi[h] = prmt(W[0][h], W[1][h], 0x7632);  // bytes 2, 3
         }
-        stsm_x4_t8(wbase + (kk * 4 * 2) * 128 + st_off, rlo);
-        stsm_x4_t8(wbase + (kk * 4 * 2 + 1) * 128 + st_off, rhi);
+        stsm_x4_t8(st_addr + (kk * 8) * 128, rlo);
+        stsm_x4_t8(st_addr + (kk * 8 + 1) * 128, rhi);
       }
-      __syncwarp();
-      // ---------------- P.V: per group, A = weight bytes (rows (head, byte)), B = codes (8 channels)
-      const uint32_t ctile = smem_u32(st + kOffCodes + tl * kTileSmem);
-      const int c_row = lane & 7, c_ntile = (lane >> 4), c_k16 = (tw >> 4) + ((lane >> 3) & 1);
+      named_bar(8 + pr_, 64);  // both slices' weights are in the pair's buffer
+      // ---------------- P.V: channels 64 jh .. + 63 over the pair's 64 tokens
+      const uint32_t ctile = smem_u32(st) + c_off;
       #pragma unroll
-      for (int grp = 0; grp < 4; ++grp) {
-        uint32_t a[4];
-        ldsm_x4(a, wbase + a_off0 + (((a_rho0 + 2 * grp) & 7) * 16));
+      for (int ks = 0; ks < 2; ++ks) {
         #pragma unroll
-        for (int pr = 0; pr < 2; ++pr) {
-          const int ch = 8 * (4 * grp + 2 * pr + c_ntile) + c_row;
-          uint32_t b[4];
-          ldsm_x4_u4(b, ctile + ch * 128 + ((c_k16 ^ (ch & 7)) << 4));
-          imma_u8(D[4 * grp + 2 * pr], a, b[0], b[1]);
-          imma_u8(D[4 * grp + 2 * pr + 1], a, b[2], b[3]);
+        for (int gi = 0; gi < 2; ++gi) {
+          const int grp = 2 * jh + gi;
+          uint32_t a[4];
+          ldsm_x4(a, a_addr + ks * kWSlice + (((a_rho0 + 2 * grp) & 7) * 16));
+          #pragma unroll
+          for (int np2 = 0; np2 < 2; ++np2) {
+            const int np = 2 * gi + np2;  // n-tiles 2 np, 2 np + 1
+            uint32_t b[4];
+            ldsm_x4_u4(b, ctile + np * 2048 + c_kx[ks]);
+            imma_u8(D[2 * np], a, b[0], b[1]);
+            imma_u8(D[2 * np + 1], a, b[2], b[3]);
+          }
         }
       }
     }
