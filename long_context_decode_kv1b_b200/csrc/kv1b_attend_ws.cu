@@ -51,8 +51,8 @@ constexpr int kPairs = 6;
 constexpr int kWarps = 2 * kPairs;          // compute warps
 constexpr int kThreads = kWarps * 32;       // 384 compute threads
 constexpr int kBlock = kThreads + 128;      // + the producer warpgroup
-constexpr int kComputeRegs = 152;           // setmaxnreg: 384 x 152 + 128 x 40 <= 512 x 128 registers
-constexpr int kProducerRegs = 40;
+constexpr int kComputeRegs = 160;           // setmaxnreg: 384 x 160 + 128 x 24 <= 512 x 128 registers (the producer thread may spill)
+constexpr int kProducerRegs = 24;
 static_assert(kThreads * kComputeRegs + 128 * kProducerRegs <= 65536, "register split within the launch's registers");
 constexpr int kTileTok = 128;               // tokens per code tile (one TMA box)
 constexpr int kStageTiles = 3;
@@ -334,6 +334,9 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
   const int a_head = a_r & 3, a_byte = a_r >> 2;
   const uint32_t a_addr = wpair_s + static_cast<uint32_t>(((a_kk * 4 + a_head) * 2 + (a_byte >> 1)) * 128);
   const int a_rho0 = (a_byte & 1) + 2 * a_head;
+  uint32_t a_pre[2];
+  #pragma unroll
+  for (int gi = 0; gi < 2; ++gi) a_pre[gi] = a_addr + (((a_rho0 + 2 * (2 * jh + gi)) & 7) * 16);
   // code-tile gathers: lanes 8m .. 8m + 7 address channel rows 64 jh + 8 (2 np + (m >> 1)) + (lane & 7)
   // of 16-token chunk k16 = (pair chunk) + 2 ks + (m & 1); 128-byte swizzle: chunk ^ (row & 7)
   const uint32_t c_off = static_cast<uint32_t>(tl * kTileSmem + (64 * jh + 8 * (lane >> 4) + (lane & 7)) * 128);
@@ -580,7 +583,7 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
       cur_seg = it.seg;
       prep(cur_seg);
     }
-    mbar_wait(&full_bar[s], phase, &s_abort);
+    if (!mbar_try(&full_bar[s], phase)) mbar_wait(&full_bar[s], phase, &s_abort);
     const uint8_t* st = smem + s * kStageBytes;
     const int rel = it.lt * kTileTok + sbase;          // this slice's first token in the segment
     const bool pair_on = tl < nt && L > rel - 32 * jh;  // the pair has real tokens in this stage
@@ -705,16 +708,16 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
       const uint32_t ctile = smem_u32(st) + c_off;
       #pragma unroll
       for (int ks = 0; ks < 2; ++ks) {
+        const uint32_t cks = ctile + c_kx[ks];
         #pragma unroll
         for (int gi = 0; gi < 2; ++gi) {
-          const int grp = 2 * jh + gi;
           uint32_t a[4];
-          ldsm_x4(a, a_addr + ks * kWSlice + (((a_rho0 + 2 * grp) & 7) * 16));
+          ldsm_x4(a, a_pre[gi] + ks * kWSlice);
           #pragma unroll
           for (int np2 = 0; np2 < 2; ++np2) {
             const int np = 2 * gi + np2;  // n-tiles 2 np, 2 np + 1
             uint32_t b[4];
-            ldsm_x4_u4(b, ctile + np * 2048 + c_kx[ks]);
+            ldsm_x4_u4(b, cks + np * 2048);
             imma_u8(D[2 * np], a, b[0], b[1]);
             imma_u8(D[2 * np + 1], a, b[2], b[3]);
           }
