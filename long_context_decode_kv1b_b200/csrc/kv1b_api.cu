@@ -205,7 +205,7 @@ size_t kv1b_attend_workspace_bytes(const kv1b_cache_t* cache, int32_t num_q_head
   if (!cache_ok(cache) || heads_check(cache, num_q_heads) != KV1B_OK) return 0;
   const size_t rows = static_cast<size_t>(cache->batch) * num_q_heads;
   if (mode == 0) return ws_counters_offset(cache, num_q_heads) + align_up(ws_counter_bytes(cache));
-  if (mode == 1) return align_up(rows * static_cast<size_t>(cache->capacity) * 4);
+  if (mode == 1) return align_up(kv1b_topp_workspace_bytes(static_cast<int32_t>(rows), cache->capacity));
   return 0;
 }
 
@@ -270,29 +270,21 @@ int kv1b_attend_topp(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, 
   if (!aligned(q, 16) || !aligned(ws, kAlign)) return KV1B_ERR_MISALIGNED;
   if (ws_bytes < kv1b_attend_workspace_bytes(cache, num_q_heads, 1)) return KV1B_ERR_WORKSPACE;
   const int G = num_q_heads / cache->num_kv_heads;
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
-  kv1b::ScoresParams sp;
-  memset(&sp, 0, sizeof(sp));
-  sp.c = view(cache);
-  sp.q = q;
-  sp.q_dtype = q_dtype;
-  sp.Hq = num_q_heads;
-  sp.scale = scale;
-  sp.s = static_cast<float*>(ws);
-  for (int b = 0; b < cache->batch; ++b) sp.len[b] = static_cast<int32_t>(cache->h_lengths[b]);
-  cudaError_t e = kv1b_launch_scores(sp, G, static_cast<int32_t>(max_length(cache)), s);
-  if (e != cudaSuccess) return KV1B_ERR_CUDA;
   kv1b::ToppParams tp;
   memset(&tp, 0, sizeof(tp));
   tp.c = view(cache);
+  tp.q = q;
+  tp.q_dtype = q_dtype;
   tp.Hq = num_q_heads;
   tp.p = p;
-  tp.s = static_cast<const float*>(ws);
+  tp.scale = scale;
   tp.out = out;
   tp.sel_idx = sel_idx;
   tp.sel_cnt = sel_cnt;
-  memcpy(tp.len, sp.len, sizeof(tp.len));
-  return cuda_status(kv1b_launch_topp(tp, s));
+  for (int b = 0; b < cache->batch; ++b) tp.len[b] = static_cast<int32_t>(cache->h_lengths[b]);
+  kv1b_topp_carve(&tp, ws, cache->batch * num_q_heads, cache->capacity);
+  return cuda_status(
+      kv1b_launch_topp(tp, G, static_cast<int32_t>(max_length(cache)), static_cast<cudaStream_t>(stream)));
 }
 
 int kv1b_query_prep(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, uint32_t* planes,

@@ -60,11 +60,34 @@ struct ScoresParams {
   int32_t len[KV1B_MAX_BATCH];
 };
 
+// Top-p pipeline (kv1b_topp.cu): per row r = b * Hq + hq of the query heads.
+struct ToppRowState {
+  uint32_t maxkey;           // order-preserving key of the row's largest logit (atomicMax)
+  uint32_t ncand;            // tokens in the threshold bucket
+  int32_t bstar;             // threshold bucket (-1: the row is empty)
+  uint32_t pad0;
+  unsigned long long U;      // total integer mass
+  unsigned long long rem;    // mass still needed inside the threshold bucket
+  unsigned long long kstar;  // largest selected 64-bit key of the threshold bucket
+  unsigned long long pad1[3];
+};
+constexpr int kToppBuckets = 1024;  // masses by t = (s - m) log2 e: bucket floor(-16 t) for t >= -40
+constexpr int kToppChunk = 4096;    // tokens per block of the streaming kernels
+
 struct ToppParams {
   CacheView c;
+  const void* q;
+  int32_t q_dtype;
   int32_t Hq;
   float p;
-  const float* s;  // [B][Hq][cap] logits
+  float scale;
+  float* s;                  // [R][cap] logits
+  int32_t* cand;             // [R][cap] threshold-bucket candidates (any order)
+  ToppRowState* rows;        // [R]
+  unsigned long long* hist;  // [R][kToppBuckets] masses per bucket
+  uint32_t* chunk_cnt;       // [R][nchunk] selected tokens per chunk
+  float* part;               // [R][nchunk][kPartStride] gather partials per chunk
+  int32_t nchunk;
   float* out;
   int32_t* sel_idx;
   int32_t* sel_cnt;
@@ -102,7 +125,9 @@ cudaError_t kv1b_launch_attend(const kv1b::AttendParams& p, int32_t G, int32_t e
 cudaError_t kv1b_launch_query_prep(const kv1b::CacheView& c, const void* q, int32_t q_dtype, int32_t Hq,
                                    uint32_t* planes, float* vl, float* delta, int32_t* sq, cudaStream_t stream);
 cudaError_t kv1b_launch_scores(const kv1b::ScoresParams& p, int32_t G, int32_t max_len, cudaStream_t stream);
-cudaError_t kv1b_launch_topp(const kv1b::ToppParams& p, cudaStream_t stream);
+cudaError_t kv1b_launch_topp(const kv1b::ToppParams& p, int32_t G, int32_t max_len, cudaStream_t stream);
+size_t kv1b_topp_workspace_bytes(int32_t rows, int32_t cap);
+void kv1b_topp_carve(kv1b::ToppParams* p, void* ws, int32_t rows, int32_t cap);
 int kv1b_pick_splits(int32_t B, int32_t Hkv, int64_t max_len, int num_sms);
 bool kv1b_ws_supported(int32_t G);
 void kv1b_ws_plan(int32_t B, int32_t Hkv, int32_t G, int64_t L, int num_sms, int64_t* T, int64_t* Lt, int* ncta,

@@ -248,3 +248,15 @@ def test_topp_ties_take_lowest_indices():
     q = K[:, 50, :, :].clone().view(B, 1, 128) * 0.3
     for p in (0.3, 0.6, 0.95):
         topp_check(cache, host, q, 0.3, p, G, oracle.signs(4))
+
+
+@pytest.mark.parametrize("scale", [0.005, 0.5, 4.0])
+def test_topp_multi_chunk_ragged(scale):
+    # 9097 tokens in two appends: several 4096-token chunks and a ragged tail; a tiny scale puts
+    # nearly every token in the threshold bucket, a large one leaves most tokens massless
+    B, Hkv, G = 2, 1, 4
+    cache, host = build_cache(B, Hkv, [5000, 4097], torch.bfloat16, seed=5, data_seed=6)
+    q = torch.randn((B, Hkv * G, 128), device=DEV, generator=torch.Generator(device=DEV).manual_seed(2))
+    q = q.to(torch.bfloat16)
+    for p in (0.5, 0.99):
+        topp_check(cache, host, q, scale, p, G, oracle.signs(5))
