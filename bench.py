@@ -51,6 +51,7 @@ def parse_args():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-alt", action="store_true")
+    ap.add_argument("--no-topp", action="store_true")
     return ap.parse_args()
 
 
@@ -333,6 +334,32 @@ def run_ours(args):
                "achieved_gbs": cfg.B * cfg.Hkv * Lc * BYTES_PER_TOKEN_HEAD / (alt_ms * 1e-3) / 1e9}
         alt["frac"] = alt["achieved_gbs"] / peak
 
+    topp = None
+    if not args.no_topp:
+        # Top-p attend (selection + gather-attend) on the same cache and query, after the timed region
+        p_top = cfg.p or 0.9
+        Lc = cache.lengths[0]
+        tout = torch.empty((cfg.B, cfg.Hq, 128), dtype=torch.float32, device=dev)
+        tsel = torch.empty((cfg.B, cfg.Hq, cache.capacity), dtype=torch.int32, device=dev)
+        tcnt = torch.empty((cfg.B, cfg.Hq), dtype=torch.int32, device=dev)
+        for _ in range(3):
+            cache.attend_topp(qs[0], cfg.scale, p_top, out=tout, sel=tsel, cnt=tcnt)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
+        for x, y in ev:
+            x.record(stream)
+            cache.attend_topp(qs[0], cfg.scale, p_top, out=tout, sel=tsel, cnt=tcnt)
+            y.record(stream)
+        torch.cuda.synchronize()
+        t_ms = statistics.median(x.elapsed_time(y) for x, y in ev)
+        cnt_f = tcnt.double()
+        alg = cfg.B * cfg.Hkv * Lc * 24 + 80 * int(tcnt.sum().item())
+        topp = {"p": p_top, "us": t_ms * 1e3, "context": Lc, "sel_mean": cnt_f.mean().item(),
+                "sel_min": int(tcnt.min().item()), "sel_max": int(tcnt.max().item()),
+                "algorithmic_bytes": alg, "achieved_gbs": alg / (t_ms * 1e-3) / 1e9,
+                "bytes_rule": "24 B per token x kv-head (scores) + 80 B per selected token x query head (gather)",
+                "kernels": "memset + scores, mass, threshold, cand, resolve, count, write_gather, merge (median of 5)"}
+        topp["frac"] = topp["achieved_gbs"] / peak
+
     result = None
     if rank == 0:
         result = {
@@ -356,6 +383,8 @@ def run_ours(args):
         }
         if alt:
             result["alt_engine"] = alt
+        if topp:
+            result["topp"] = topp
     barrier(world)
     if world > 1:
         import torch.distributed as dist

@@ -85,6 +85,11 @@ def _check(code: int, what: str):
         raise Kv1bError(code, what)
 
 
+def _check_buf(t: torch.Tensor, shape, dtype, name: str):
+    if tuple(t.shape) != tuple(shape) or t.dtype != dtype or not t.is_contiguous():
+        raise ValueError(f"{name} must be a contiguous {dtype} tensor of shape {tuple(shape)}")
+
+
 def _dtype_code(t: torch.Tensor) -> int:
     if t.dtype == torch.float32:
         return DTYPE_F32
@@ -180,12 +185,19 @@ class Cache:
                                  _ptr(ws), ws.numel(), engine, num_splits, _stream(stream)), "kv1b_attend")
         return out
 
-    def attend_topp(self, q: torch.Tensor, scale: float, p: float, stream=None):
-        """Returns (out fp32 [B, Hq, 128], sel_idx int32 [B, Hq, capacity], sel_cnt int32 [B, Hq])."""
+    def attend_topp(self, q: torch.Tensor, scale: float, p: float, out=None, sel=None, cnt=None, stream=None):
+        """Returns (out fp32 [B, Hq, 128], sel_idx int32 [B, Hq, capacity], sel_cnt int32 [B, Hq]);
+        out / sel / cnt may be passed in (contiguous, those shapes and dtypes) to reuse buffers."""
         B, Hq, D = q.shape
-        out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
-        sel = torch.empty((B, Hq, self.capacity), dtype=torch.int32, device=q.device)
-        cnt = torch.empty((B, Hq), dtype=torch.int32, device=q.device)
+        if out is None:
+            out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+        if sel is None:
+            sel = torch.empty((B, Hq, self.capacity), dtype=torch.int32, device=q.device)
+        if cnt is None:
+            cnt = torch.empty((B, Hq), dtype=torch.int32, device=q.device)
+        _check_buf(out, (B, Hq, D), torch.float32, "out")
+        _check_buf(sel, (B, Hq, self.capacity), torch.int32, "sel")
+        _check_buf(cnt, (B, Hq), torch.int32, "cnt")
         ws = self.workspace(Hq, 1)
         _check(lib().kv1b_attend_topp(ctypes.byref(self.desc), _ptr(q), _dtype_code(q), Hq, float(scale), float(p),
                                       _ptr(out), _ptr(sel), _ptr(cnt), _ptr(ws), ws.numel(), _stream(stream)),

@@ -71,7 +71,7 @@ struct ToppRowState {
   unsigned long long kstar;  // largest selected 64-bit key of the threshold bucket
   unsigned long long pad1[3];
 };
-constexpr int kToppBuckets = 1024;  // masses by t = (s - m) log2 e: bucket floor(-16 t) for t >= -40
+constexpr int kToppBuckets = 2048;  // masses by t = (s - m) log2 e: bucket floor(-64 t), t >= -40
 constexpr int kToppChunk = 4096;    // tokens per block of the streaming kernels
 
 struct ToppParams {
@@ -81,11 +81,15 @@ struct ToppParams {
   int32_t Hq;
   float p;
   float scale;
+  uint32_t* planes;          // [R][4][4] query bit-planes, then grid origin, step and code sum per row
+  float* qvl;
+  float* qdl;
+  int32_t* qsq;
   float* s;                  // [R][cap] logits
   int32_t* cand;             // [R][cap] threshold-bucket candidates (any order)
   ToppRowState* rows;        // [R]
   unsigned long long* hist;  // [R][kToppBuckets] masses per bucket
-  uint32_t* chunk_cnt;       // [R][nchunk] selected tokens per chunk
+  uint32_t* chunk_cnt;       // [R][nchunk] selected tokens per chunk (lower buckets, then candidates)
   float* part;               // [R][nchunk][kPartStride] gather partials per chunk
   int32_t nchunk;
   float* out;

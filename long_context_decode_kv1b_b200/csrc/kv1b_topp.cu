@@ -3,22 +3,25 @@
 // grid-wide kernels so that a long context is spread over every SM.  Per row r = (sequence,
 // query head), with the reproducible integer masses u_t ~ 2^32 2^((s_t - m) log2 e) (degree-7
 // polynomial of 2^f, bit for bit the same as the CPU reference) and T = ceil(p U) in fp64:
-//  1. scores: binary x INT4 popcount logits of every token for the G heads of a kv-head (bit-exact
-//     arithmetic), written to the workspace; the row maximum m by atomicMax on an order-preserving
-//     key;
-//  2. masses: u_t, the row total U, and a histogram of masses over 640 buckets of
-//     t = (s - m) log2 e (bucket floor(-16 t), monotone in s; t < -40 has no mass);
+//  0. query preparation (rotation, 4-bit codes, bit-planes) once per row;
+//  1. scores: the binary x INT4 integers A = sum_i bit_i code_i and Bc = sum_i bit_i of every token
+//     on the integer tensor cores (exact), then the fp32 logit in the fixed operation order; the row
+//     maximum m by atomicMax on an order-preserving key;
+//  2. masses: u_t, the row total U, and a histogram of masses over 2048 buckets of
+//     t = (s - m) log2 e (bucket floor(-64 t), monotone in s, the last one also holding
+//     t in [-40, -32); t < -40 has no mass);
 //  3. threshold: the first bucket b* where the cumulative mass reaches T; rem = the mass still
 //     needed inside b*;
-//  4. candidates: the tokens of bucket b* (any order);
+//  4. candidates: the tokens of bucket b* (any order), and per chunk the count of tokens in lower
+//     buckets (all of them selected);
 //  5. resolve: a block-wide radix select over the candidates' unique 64-bit keys
 //     (order-preserving descending code of s) << 32 | t finds the smallest key K* whose cumulative
-//     candidate mass reaches rem;
+//     candidate mass reaches rem, and adds the selected candidates to their chunks' counts;
 //  6. the selected set {t : bucket(t) < b*} U {t in b* : key_t <= K*} -- the shortest prefix of the
-//     order (s desc, index asc) whose mass reaches T -- is compacted in ascending index order
-//     (chunk counts, then ordered writes);
-//  7. gather-attend, fused with the compaction: the softmax over the selected tokens' logits with
-//     the 4-bit values dequantised on the fly, fp32 partials per chunk, summed in chunk order.
+//     order (s desc, index asc) whose mass reaches T -- is written in ascending index order (chunk
+//     offsets from the counts), and in the same pass the chunk's selected tokens are gathered: the
+//     softmax numerator and denominator against m, 4-bit values dequantised on the fly, fp32;
+//  7. merge: the chunk partials summed in chunk order.
 #include "kv1b_device.cuh"
 #include "kv1b_launch.h"
 
@@ -26,6 +29,13 @@ namespace kv1b {
 
 constexpr float kL2e = 0x1.715476p+0f;  // log2(e) rounded to fp32
 constexpr int kStreamThreads = 256;
+constexpr int kStreamWarps = kStreamThreads / 32;
+constexpr int kTokPerThread = kToppChunk / kStreamThreads;  // contiguous tokens per thread
+static_assert(kTokPerThread == 16, "the streaming kernels hold 16 tokens per thread");
+constexpr int kScoreTok = 2048;          // tokens per block of the score kernel
+constexpr int kResolveThreads = 1024;
+constexpr int kResolveSmemCand = 12288;  // candidates whose keys and masses the resolve keeps on chip
+constexpr size_t kResolveSmem = static_cast<size_t>(kResolveSmemCand) * 16;
 
 // (ln 2)^k / k!, k = 0..7, each rounded to the nearest fp32 (Taylor coefficients of 2^f).
 __constant__ float kExp2Coef[8] = {0x1p+0f,         0x1.62e43p-1f,   0x1.ebfbep-3f,   0x1.c6b08ep-5f,
@@ -45,11 +55,12 @@ __device__ __forceinline__ uint64_t topp_mass_t(float t) {
   return __float2ull_rz(scaled);
 }
 
-// Bucket of t = (s - m) log2 e: floor(-16 t) for t in [-40, 0] (639 at most), 640 below.
+// Bucket of t = (s - m) log2 e: floor(-64 t) for t in [-40, 0], at most kToppBuckets - 1 (a
+// non-decreasing function of -t, hence of the key order); kToppBuckets below -40 (no mass there).
 __device__ __forceinline__ int topp_bucket(float t) {
-  if (!(t >= -40.0f)) return 640;
-  const int b = static_cast<int>(__fmul_rn(-t, 16.0f));
-  return b < 639 ? b : 639;
+  if (!(t >= -40.0f)) return kToppBuckets;
+  const int b = static_cast<int>(__fmul_rn(-t, 64.0f));
+  return b < kToppBuckets - 1 ? b : kToppBuckets - 1;
 }
 
 __device__ __forceinline__ uint64_t topp_key(float s, int64_t t) {
@@ -70,105 +81,213 @@ __device__ __forceinline__ T warp_sum(T v) {
   for (int m = 16; m >= 1; m >>= 1) v += __shfl_xor_sync(kFull, v, m);
   return v;
 }
+__device__ __forceinline__ unsigned warp_incl_scan(unsigned v) {
+  const int lane = threadIdx.x & 31;
+  #pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const unsigned x = __shfl_up_sync(kFull, v, o);
+    if (lane >= o) v += x;
+  }
+  return v;
+}
 
 __device__ __forceinline__ int row_len(const ToppParams& p, int64_t r) { return p.len[r / p.Hq]; }
 
+// 16 logits t0 .. t0 + 15 of a row (t0 a multiple of 16; the row holds cap floats, cap a multiple
+// of 128, so whole float4s stay inside it); entries at or past t1 are left unspecified.
+__device__ __forceinline__ void load16(const float* s, int64_t t0, int64_t t1, float v[16]) {
+  #pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    float4 x = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    if (t0 + 4 * q < t1) x = *reinterpret_cast<const float4*>(s + t0 + 4 * q);
+    v[4 * q] = x.x;
+    v[4 * q + 1] = x.y;
+    v[4 * q + 2] = x.z;
+    v[4 * q + 3] = x.w;
+  }
+}
+
 // ---------------------------------------------------------------- 1. logits and row maxima
-// grid (token blocks of 256, kv-heads, sequences); thread = token, loops over the G heads.
-__global__ void __launch_bounds__(kStreamThreads) topp_scores_kernel(const ToppParams p, int G) {
-  __shared__ __align__(16) uint32_t s_planes[KV1B_MAX_GROUP][4][4];
-  __shared__ float s_vl[KV1B_MAX_GROUP], s_dl[KV1B_MAX_GROUP];
-  __shared__ int s_sq[KV1B_MAX_GROUP];
-  __shared__ float s_max[kStreamThreads / 32][KV1B_MAX_GROUP];
-  const int b = blockIdx.z, kvh = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const CacheView& c = p.c;
-  if (warp < G) {
-    const QueryPrep qp =
-        query_prep_warp(p.q, (static_cast<int64_t>(b) * p.Hq + kvh * G + warp) * kD, p.q_dtype, c.signs);
-    if (lane == 0) {
-      for (int j = 0; j < 4; ++j)
-        for (int w = 0; w < 4; ++w) s_planes[warp][j][w] = qp.planes[j][w];
-      s_vl[warp] = qp.vl;
-      s_dl[warp] = qp.delta;
-      s_sq[warp] = qp.sq;
+// Integer MMA D += A B (16 x 32 s8 by 32 x 8 s8 -> s32).
+__device__ __forceinline__ void mma_s8(int d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%0,%1,%2,%3};"
+      : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+      : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+// Sign bits of 16 tokens against 8 operand columns.  Lane (g, t) holds word t (channels 32t..32t+31)
+// of tokens g and g + 8.  K-block kb uses the bits at positions 8j + 2kb and 8j + 2kb + 1 of the word
+// (after a 4-bit shift for kb >= 2), masked in place so each byte is bit * 2^(position & 3); the
+// query column carries code * 2^(3 - (position & 3)) for the same channel, so every product is
+// 8 * bit * code and D = 8 * sum_i bit_i code_i exactly (columns of ones give 8 * Bc).
+__device__ __forceinline__ void bits_mma(int d[4], uint32_t w0, uint32_t w8, const uint32_t (&bq)[4][2]) {
+  d[0] = d[1] = d[2] = d[3] = 0;
+  const uint32_t x0[2] = {w0, w0 >> 4}, x8[2] = {w8, w8 >> 4};
+  #pragma unroll
+  for (int kb = 0; kb < 4; ++kb) {
+    const uint32_t mlo = 0x01010101u << (2 * (kb & 1)), mhi = mlo << 1;
+    const uint32_t a[4] = {x0[kb >> 1] & mlo, x8[kb >> 1] & mlo, x0[kb >> 1] & mhi, x8[kb >> 1] & mhi};
+    mma_s8(d, a, bq[kb][0], bq[kb][1]);
+  }
+}
+
+// Query operand of lane (g, t): column g, k = 4t..4t+3 (register 0) and 16+4t..16+4t+3 (register 1)
+// of each k-block.  planes_row: the head's bit-planes for a code column, nullptr otherwise.
+__device__ __forceinline__ void build_bq(uint32_t (&bq)[4][2], const uint32_t* planes_row, int t, bool ones_col) {
+  uint32_t pw[4] = {0u, 0u, 0u, 0u};
+  if (planes_row) {
+    #pragma unroll
+    for (int j = 0; j < 4; ++j) pw[j] = planes_row[4 * j + t];
+  }
+  #pragma unroll
+  for (int kb = 0; kb < 4; ++kb)
+    #pragma unroll
+    for (int hi = 0; hi < 2; ++hi) {
+      const int r = 2 * kb + hi;
+      const int sh = 3 - (r & 3);
+      uint32_t code = 0u;
+      #pragma unroll
+      for (int j = 0; j < 4; ++j) code |= ((pw[j] >> r) & 0x01010101u) << j;
+      bq[kb][hi] = planes_row ? (code << sh) : (ones_col ? (0x01010101u << sh) : 0u);
     }
-  }
-  __syncthreads();
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * kStreamThreads + threadIdx.x;
-  const bool valid = t < p.len[b];
-  const int64_t head_tok = (static_cast<int64_t>(b) * c.Hkv + kvh) * c.cap;
-  uint4 kb = make_uint4(0u, 0u, 0u, 0u);
-  float nc = 0.0f;
-  if (valid) {
-    kb = __ldg(reinterpret_cast<const uint4*>(c.k_bits) + head_tok + t);
-    nc = __fmul_rn(__ldg(c.k_norm + head_tok + t), __ldg(c.k_cinv + head_tok + t));
-  }
-  const int32_t Bc = popc_Bc(kb);
+}
+
+// grid (token blocks of kScoreTok, kv-heads, sequences); warp = 64 tokens at a time, up to 4 NG
+// heads as NG groups of 4 operand-column pairs.
+template <int NG>
+__global__ void __launch_bounds__(kStreamThreads) topp_scores_kernel(const ToppParams p, int G) {
+  __shared__ float s_max[kStreamWarps][8];
+  const CacheView& c = p.c;
+  const int b = blockIdx.z, kvh = blockIdx.y;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
+  const int L = p.len[b];
+  const int64_t row0 = static_cast<int64_t>(b) * p.Hq + static_cast<int64_t>(kvh) * G;
   const float qs = __fdiv_rn(p.scale, static_cast<float>(kD));
-  for (int h = 0; h < G; ++h) {
-    uint32_t P[4][4];
-    for (int j = 0; j < 4; ++j)
-      for (int w = 0; w < 4; ++w) P[j][w] = s_planes[h][j][w];
-    float sv = -INFINITY;
-    if (valid) {
-      const int32_t A = popc_A(kb, P);
-      sv = logit_from_ints(A, Bc, s_sq[h], s_vl[h], s_dl[h], nc, qs);
-      p.s[(static_cast<int64_t>(b) * p.Hq + kvh * G + h) * c.cap + t] = sv;
+  uint32_t bq[NG][4][2];
+  float cdl[NG], cvl[NG];
+  int32_t csq[NG];
+  bool hv[NG];
+  #pragma unroll
+  for (int hg = 0; hg < NG; ++hg) {
+    const int hc = 4 * hg + (g >> 1);  // head of this lane's operand column
+    const bool code_col = (g & 1) == 0 && hc < G;
+    build_bq(bq[hg], code_col ? p.planes + (row0 + hc) * 16 : nullptr, t, (g & 1) != 0);
+    const int ht = 4 * hg + t;  // head of this lane's output column
+    hv[hg] = ht < G;
+    cdl[hg] = hv[hg] ? p.qdl[row0 + ht] : 0.0f;
+    cvl[hg] = hv[hg] ? p.qvl[row0 + ht] : 0.0f;
+    csq[hg] = hv[hg] ? p.qsq[row0 + ht] : 0;
+  }
+  float mx[NG];
+  #pragma unroll
+  for (int hg = 0; hg < NG; ++hg) mx[hg] = -INFINITY;
+  const int64_t head_tok = (static_cast<int64_t>(b) * c.Hkv + kvh) * c.cap;
+  const uint32_t* kw = c.k_bits + head_tok * 4;
+  const float* kn = c.k_norm + head_tok;
+  const float* ki = c.k_cinv + head_tok;
+  const int64_t tb0 = static_cast<int64_t>(blockIdx.x) * kScoreTok;
+  const int64_t tend = tb0 + kScoreTok < L ? tb0 + kScoreTok : L;
+  for (int64_t base = tb0 + 64 * warp; base < tend; base += 64 * kStreamWarps) {  // warp-uniform
+    uint32_t w[8];
+    float nc[8];
+    #pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const int64_t tok = base + g + 8 * i;
+      const bool v = tok < tend;
+      w[i] = v ? __ldg(kw + tok * 4 + t) : 0u;
+      nc[i] = v ? __fmul_rn(__ldg(kn + tok), __ldg(ki + tok)) : 0.0f;
     }
     #pragma unroll
-    for (int o = 16; o >= 1; o >>= 1) sv = fmaxf(sv, __shfl_xor_sync(kFull, sv, o));
-    if (lane == 0) s_max[warp][h] = sv;
+    for (int hg = 0; hg < NG; ++hg) {
+      #pragma unroll
+      for (int kk = 0; kk < 4; ++kk) {
+        int d[4];
+        bits_mma(d, w[2 * kk], w[2 * kk + 1], bq[hg]);
+        #pragma unroll
+        for (int e = 0; e < 2; ++e) {
+          const int64_t tok = base + 16 * kk + g + 8 * e;
+          if (hv[hg] && tok < tend) {
+            const float sv =
+                logit_from_ints(d[2 * e] >> 3, d[2 * e + 1] >> 3, csq[hg], cvl[hg], cdl[hg], nc[2 * kk + e], qs);
+            p.s[(row0 + 4 * hg + t) * c.cap + tok] = sv;
+            mx[hg] = fmaxf(mx[hg], sv);
+          }
+        }
+      }
+    }
+  }
+  #pragma unroll
+  for (int hg = 0; hg < NG; ++hg) {
+    #pragma unroll
+    for (int o = 4; o <= 16; o <<= 1) mx[hg] = fmaxf(mx[hg], __shfl_xor_sync(kFull, mx[hg], o));
+    if (g == 0) s_max[warp][4 * hg + t] = mx[hg];
   }
   __syncthreads();
   if (threadIdx.x < G) {
-    float mx = s_max[0][threadIdx.x];
-    for (int w = 1; w < kStreamThreads / 32; ++w) mx = fmaxf(mx, s_max[w][threadIdx.x]);
-    if (mx != -INFINITY) atomicMax(&p.rows[static_cast<int64_t>(b) * p.Hq + kvh * G + threadIdx.x].maxkey, fkey(mx));
+    float m = s_max[0][threadIdx.x];
+    for (int w = 1; w < kStreamWarps; ++w) m = fmaxf(m, s_max[w][threadIdx.x]);
+    if (m != -INFINITY) atomicMax(&p.rows[row0 + threadIdx.x].maxkey, fkey(m));
   }
 }
 
 // ---------------------------------------------------------------- 2. masses and bucket histogram
-// grid (chunks of kToppChunk tokens, rows)
+// grid (chunks of kToppChunk tokens, rows); thread = 16 contiguous tokens.  The block histogram keeps
+// each bucket's 64-bit sum as a wrapping 32-bit low word plus a count of carries (32-bit shared
+// atomics); the block then adds its non-empty buckets to the row's 64-bit histogram.
 __global__ void __launch_bounds__(kStreamThreads) topp_mass_kernel(const ToppParams p) {
-  __shared__ unsigned long long sh[kToppBuckets];
-  __shared__ unsigned long long s_u[kStreamThreads / 32];
+  __shared__ uint32_t s_lo[kToppBuckets], s_hi[kToppBuckets];
+  __shared__ unsigned long long s_u[kStreamWarps];
   const int64_t r = blockIdx.y;
   const int L = row_len(p, r);
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kToppChunk;
   if (t0 >= L) return;
   const int64_t t1 = t0 + kToppChunk < L ? t0 + kToppChunk : L;
-  for (int i = threadIdx.x; i < kToppBuckets; i += kStreamThreads) sh[i] = 0ull;
+  const int64_t tt0 = t0 + kTokPerThread * threadIdx.x;
+  float v[16];
+  load16(p.s + r * p.c.cap, tt0, t1, v);
+  for (int i = threadIdx.x; i < kToppBuckets; i += kStreamThreads) {
+    s_lo[i] = 0u;
+    s_hi[i] = 0u;
+  }
   __syncthreads();
   const float m = fkey_inv(p.rows[r].maxkey);
-  const float* s = p.s + r * p.c.cap;
   unsigned long long usum = 0ull;
-  for (int64_t t = t0 + threadIdx.x; t < t1; t += kStreamThreads) {
-    const float tt = topp_t(s[t], m);
-    const uint64_t u = topp_mass_t(tt);
-    if (u) {
-      atomicAdd(&sh[topp_bucket(tt)], static_cast<unsigned long long>(u));
-      usum += u;
+  #pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    if (tt0 + i < t1) {
+      const float tt = topp_t(v[i], m);
+      const uint64_t u = topp_mass_t(tt);
+      if (u) {
+        const int bk = topp_bucket(tt);
+        const uint32_t ulo = static_cast<uint32_t>(u);
+        const uint32_t old = atomicAdd(&s_lo[bk], ulo);
+        const uint32_t inc = static_cast<uint32_t>(u >> 32) + (old + ulo < old ? 1u : 0u);
+        if (inc) atomicAdd(&s_hi[bk], inc);
+        usum += u;
+      }
     }
   }
   usum = warp_sum(usum);
   if ((threadIdx.x & 31) == 0) s_u[threadIdx.x >> 5] = usum;
   __syncthreads();
   unsigned long long* hist = p.hist + r * kToppBuckets;
-  for (int i = threadIdx.x; i < 640; i += kStreamThreads)
-    if (sh[i]) atomicAdd(&hist[i], sh[i]);
+  for (int i = threadIdx.x; i < kToppBuckets; i += kStreamThreads) {
+    const unsigned long long h = (static_cast<unsigned long long>(s_hi[i]) << 32) | s_lo[i];
+    if (h) atomicAdd(&hist[i], h);
+  }
   if (threadIdx.x == 0) {
     unsigned long long tot = 0ull;
-    for (int w = 0; w < kStreamThreads / 32; ++w) tot += s_u[w];
+    for (int w = 0; w < kStreamWarps; ++w) tot += s_u[w];
     atomicAdd(&p.rows[r].U, tot);
   }
 }
 
 // ---------------------------------------------------------------- 3. threshold bucket
-// grid (rows), 1024 threads: thread i owns bucket i.
-__global__ void __launch_bounds__(kToppBuckets) topp_threshold_kernel(const ToppParams p) {
-  __shared__ unsigned long long s_w[kToppBuckets / 32];
-  __shared__ int s_first;
+// grid (rows), 1024 threads: thread i owns buckets 2i and 2i + 1.
+constexpr int kThresholdThreads = kToppBuckets / 2;
+__global__ void __launch_bounds__(kThresholdThreads) topp_threshold_kernel(const ToppParams p) {
+  __shared__ unsigned long long s_w[kThresholdThreads / 32];
   const int64_t r = blockIdx.x;
   ToppRowState& rs = p.rows[r];
   const unsigned long long U = rs.U;
@@ -180,15 +299,15 @@ __global__ void __launch_bounds__(kToppBuckets) topp_threshold_kernel(const Topp
   if (T > U) T = U;
   if (T < 1) T = 1;
   const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
-  const unsigned long long h = p.hist[r * kToppBuckets + i];
-  unsigned long long incl = h;
+  const unsigned long long h0 = p.hist[r * kToppBuckets + 2 * i], h1 = p.hist[r * kToppBuckets + 2 * i + 1];
+  const unsigned long long loc = h0 + h1;
+  unsigned long long incl = loc;
   #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
     const unsigned long long v = __shfl_up_sync(kFull, incl, o);
     if (lane >= o) incl += v;
   }
   if (lane == 31) s_w[warp] = incl;
-  if (i == 0) s_first = kToppBuckets;
   __syncthreads();
   if (warp == 0) {
     unsigned long long w = s_w[lane];
@@ -201,78 +320,130 @@ __global__ void __launch_bounds__(kToppBuckets) topp_threshold_kernel(const Topp
   }
   __syncthreads();
   incl += warp ? s_w[warp - 1] : 0ull;
-  if (incl >= T && incl - h < T) atomicMin(&s_first, i);  // exactly one bucket crosses T
-  __syncthreads();
-  if (i == s_first) {
-    rs.bstar = i;
-    rs.rem = T - (incl - h);
+  const unsigned long long excl = incl - loc;
+  // exactly one bucket crosses T (it has mass > 0)
+  if (excl < T && T <= excl + h0) {
+    rs.bstar = 2 * i;
+    rs.rem = T - excl;
+  } else if (excl + h0 < T && T <= incl) {
+    rs.bstar = 2 * i + 1;
+    rs.rem = T - excl - h0;
   }
 }
 
-// ---------------------------------------------------------------- 4. candidates of bucket b*
+// ---------------------------------------------------------------- 4. candidates and lower-bucket counts
+// grid (chunks, rows); thread = 16 contiguous tokens.
 __global__ void __launch_bounds__(kStreamThreads) topp_cand_kernel(const ToppParams p) {
+  __shared__ unsigned s_c[kStreamWarps];
   const int64_t r = blockIdx.y;
   const int L = row_len(p, r);
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kToppChunk;
-  const int bstar = p.rows[r].bstar;
+  ToppRowState& rs = p.rows[r];
+  const int bstar = rs.bstar;
   if (t0 >= L || bstar < 0) return;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t t1 = t0 + kToppChunk < L ? t0 + kToppChunk : L;
-  const float m = fkey_inv(p.rows[r].maxkey);
-  const float* s = p.s + r * p.c.cap;
-  int32_t* cand = p.cand + r * p.c.cap;
-  const int lane = threadIdx.x & 31;
-  for (int64_t tb = t0; tb < t1; tb += kStreamThreads) {
-    const int64_t t = tb + threadIdx.x;
-    const bool f = t < t1 && topp_bucket(topp_t(s[t], m)) == bstar;
-    const unsigned ball = __ballot_sync(kFull, f);
-    if (ball) {
-      unsigned base = 0;
-      if (lane == 0) base = atomicAdd(&p.rows[r].ncand, static_cast<unsigned>(__popc(ball)));
-      base = __shfl_sync(kFull, base, 0);
-      if (f) cand[base + __popc(ball & ((1u << lane) - 1u))] = static_cast<int32_t>(t);
+  const int64_t tt0 = t0 + kTokPerThread * threadIdx.x;
+  float v[16];
+  load16(p.s + r * p.c.cap, tt0, t1, v);
+  const float m = fkey_inv(rs.maxkey);
+  unsigned lo = 0, cmask = 0;
+  #pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    if (tt0 + i < t1) {
+      const int bk = topp_bucket(topp_t(v[i], m));
+      lo += bk < bstar;
+      cmask |= static_cast<unsigned>(bk == bstar) << i;
     }
+  }
+  const unsigned nc = __popc(cmask);
+  const unsigned incl = warp_incl_scan(nc);
+  unsigned wbase = 0;
+  if (lane == 31 && incl) wbase = atomicAdd(&rs.ncand, incl);
+  wbase = __shfl_sync(kFull, wbase, 31);
+  int32_t* cand = p.cand + r * p.c.cap + (wbase + incl - nc);
+  while (cmask) {
+    const int i = __ffs(cmask) - 1;
+    cmask &= cmask - 1u;
+    *cand++ = static_cast<int32_t>(tt0 + i);
+  }
+  lo = warp_sum(lo);
+  if (lane == 0) s_c[warp] = lo;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    unsigned tot = 0;
+    for (int w = 0; w < kStreamWarps; ++w) tot += s_c[w];
+    p.chunk_cnt[r * p.nchunk + blockIdx.x] = tot;
   }
 }
 
 // ---------------------------------------------------------------- 5. exact resolution inside b*
 // grid (rows), 1024 threads: radix select, 8 passes of 8 bits (most significant first), over the
 // candidates' unique keys with per-bin mass histograms; K* = the smallest key whose cumulative
-// mass (in key order) reaches rem.
-constexpr int kResolveThreads = 1024;
+// mass (in key order) reaches rem.  Up to kResolveSmemCand candidates keep key and mass on chip.
 __global__ void __launch_bounds__(kResolveThreads) topp_resolve_kernel(const ToppParams p) {
-  __shared__ unsigned long long hist[256];
+  extern __shared__ unsigned long long s_kv[];  // [kResolveSmemCand] keys, then masses
+  __shared__ uint32_t h_lo[256], h_hi[256];     // bin masses: wrapping low word + carries
   __shared__ unsigned long long s_prefix, s_rem;
   const int64_t r = blockIdx.x;
   ToppRowState& rs = p.rows[r];
   if (rs.bstar < 0) return;
   const int n = static_cast<int>(rs.ncand);
+  const bool on_chip = n <= kResolveSmemCand;
   const float m = fkey_inv(rs.maxkey);
   const float* s = p.s + r * p.c.cap;
   const int32_t* cand = p.cand + r * p.c.cap;
+  unsigned long long* skey = s_kv;
+  unsigned long long* smass = s_kv + kResolveSmemCand;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (on_chip) {
+    for (int i = threadIdx.x; i < n; i += kResolveThreads) {
+      const int64_t t = cand[i];
+      const float st = s[t];
+      skey[i] = topp_key(st, t);
+      smass[i] = topp_mass_t(topp_t(st, m));
+    }
+  }
   if (threadIdx.x == 0) {
     s_prefix = 0;
     s_rem = rs.rem;
   }
   for (int d = 7; d >= 0; --d) {
-    if (threadIdx.x < 256) hist[threadIdx.x] = 0;
+    if (threadIdx.x < 256) {
+      h_lo[threadIdx.x] = 0u;
+      h_hi[threadIdx.x] = 0u;
+    }
     __syncthreads();
     const unsigned long long prefix = s_prefix;
     for (int i = threadIdx.x; i < n; i += kResolveThreads) {
-      const int64_t t = cand[i];
-      const float st = s[t];
-      const uint64_t key = topp_key(st, t);
-      if (d == 7 || (key >> (8 * (d + 1))) == prefix) {
-        const uint64_t u = topp_mass_t(topp_t(st, m));
-        if (u) atomicAdd(&hist[(key >> (8 * d)) & 255u], static_cast<unsigned long long>(u));
+      unsigned long long key, u;
+      if (on_chip) {
+        key = skey[i];
+        u = smass[i];
+      } else {
+        const int64_t t = cand[i];
+        const float st = s[t];
+        key = topp_key(st, t);
+        u = topp_mass_t(topp_t(st, m));
+      }
+      if (u && (d == 7 || (key >> (8 * (d + 1))) == prefix)) {
+        const int bin = static_cast<int>((key >> (8 * d)) & 255u);
+        const uint32_t ulo = static_cast<uint32_t>(u);
+        const uint32_t old = atomicAdd(&h_lo[bin], ulo);
+        const uint32_t inc = static_cast<uint32_t>(u >> 32) + (old + ulo < old ? 1u : 0u);
+        if (inc) atomicAdd(&h_hi[bin], inc);
       }
     }
     __syncthreads();
     if (warp == 0) {
       const unsigned long long rem = s_rem;
       unsigned long long loc = 0;
+      unsigned long long hb[8];
       #pragma unroll
-      for (int i = 0; i < 8; ++i) loc += hist[8 * lane + i];
+      for (int i = 0; i < 8; ++i) {
+        hb[i] = (static_cast<unsigned long long>(h_hi[8 * lane + i]) << 32) | h_lo[8 * lane + i];
+        loc += hb[i];
+      }
       unsigned long long incl = loc;
       #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
@@ -286,12 +457,11 @@ __global__ void __launch_bounds__(kResolveThreads) topp_resolve_kernel(const Top
         unsigned long long cum = excl;
         int bin = 8 * lane + 7;
         for (int i = 0; i < 8; ++i) {
-          const unsigned long long hb = hist[8 * lane + i];
-          if (cum + hb >= rem) {
+          if (cum + hb[i] >= rem) {
             bin = 8 * lane + i;
             break;
           }
-          cum += hb;
+          cum += hb[i];
         }
         s_rem = rem - cum;
         s_prefix = (prefix << 8) | static_cast<unsigned long long>(bin);
@@ -299,160 +469,231 @@ __global__ void __launch_bounds__(kResolveThreads) topp_resolve_kernel(const Top
     }
     __syncthreads();
   }
-  if (threadIdx.x == 0) rs.kstar = s_prefix;
-}
-
-// ---------------------------------------------------------------- 6. ascending compaction
-__device__ __forceinline__ bool topp_selected(const ToppRowState& rs, const float* s, float m, int64_t t) {
-  const float st = s[t];
-  const int bk = topp_bucket(topp_t(st, m));
-  return bk < rs.bstar || (bk == rs.bstar && topp_key(st, t) <= rs.kstar);
-}
-
-__global__ void __launch_bounds__(kStreamThreads) topp_count_kernel(const ToppParams p) {
-  __shared__ unsigned s_c[kStreamThreads / 32];
-  const int64_t r = blockIdx.y;
-  const int L = row_len(p, r);
-  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kToppChunk;
-  const ToppRowState& rs = p.rows[r];
-  unsigned cnt = 0;
-  if (t0 < L && rs.bstar >= 0) {
-    const int64_t t1 = t0 + kToppChunk < L ? t0 + kToppChunk : L;
-    const float m = fkey_inv(rs.maxkey);
-    const float* s = p.s + r * p.c.cap;
-    for (int64_t t = t0 + threadIdx.x; t < t1; t += kStreamThreads) cnt += topp_selected(rs, s, m, t);
-  }
-  cnt = warp_sum(cnt);
-  if ((threadIdx.x & 31) == 0) s_c[threadIdx.x >> 5] = cnt;
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    unsigned tot = 0;
-    for (int w = 0; w < kStreamThreads / 32; ++w) tot += s_c[w];
-    p.chunk_cnt[r * p.nchunk + blockIdx.x] = tot;
+  const unsigned long long kstar = s_prefix;
+  if (threadIdx.x == 0) rs.kstar = kstar;
+  // selected candidates join their chunks' counts (one atomic per chunk and warp)
+  uint32_t* cc = p.chunk_cnt + r * p.nchunk;
+  for (int i0 = 0; i0 < n; i0 += kResolveThreads) {  // block-uniform trip count
+    const int i = i0 + threadIdx.x;
+    int ck = -1;
+    if (i < n) {
+      const int64_t t = cand[i];
+      const unsigned long long key = on_chip ? skey[i] : topp_key(s[t], t);
+      if (key <= kstar) ck = static_cast<int>(t / kToppChunk);
+    }
+    const unsigned same = __match_any_sync(kFull, ck);
+    if (ck >= 0 && lane == __ffs(same) - 1) atomicAdd(&cc[ck], static_cast<unsigned>(__popc(same)));
   }
 }
 
-// 6b + 7. ordered writes of the selected indices, fused with the gather-attend of the chunk's selected
-// tokens.  grid (G, chunks, B * Hkv): the G query heads of a kv-head and chunk are adjacent in launch
-// order, so their value reads share L2.  Warp w owns the 32-token slice tb + 32 w; when any token of
-// the slice is selected, lane l loads the slice's 4-bit codes of channels 4l..4l+3 (one 16-byte word
-// group per channel) and accumulates e (scale code + min) for every selected token.  The chunk's
-// partial (numerator, denominator) against the row maximum goes to part[row][chunk]; the merge sums
-// the chunks in order.
+// ---------------------------------------------------------------- 6. ordered writes + gather-attend
+// grid (chunks, B * Hkv): one block serves the G query heads of a kv-head, so each code tile of the
+// chunk is read once for all of them.  Thread = 16 contiguous tokens.  Per head: selection mask,
+// block scan, ordered index writes, softmax weights of the selected tokens into shared memory.
+// Then warp w gathers its 512 tokens in slices of 32 (lanes 2k, 2k + 1): for each slice where any
+// head selects a token, lane l loads the slice's 4-bit codes of channels 4l..4l+3 (one 16-byte group
+// per channel), the next such slice's loads in flight meanwhile, and accumulates, per head,
+// e * (scale * code + min) over that head's selected tokens.  Each head's (numerator, denominator)
+// against its row maximum goes to part[row][chunk].
+template <int GM>
 __global__ void __launch_bounds__(kStreamThreads) topp_write_gather_kernel(const ToppParams p, int G) {
-  constexpr int kW = kStreamThreads / 32;
-  __shared__ unsigned s_c[kW];
-  __shared__ unsigned s_base;
-  __shared__ float s_e[kW][32];
-  __shared__ __align__(16) uint32_t s_smw[kW][32][4];  // written as uint4
+  constexpr int kW = kStreamWarps;
+  extern __shared__ float s_e[];  // [G][kToppChunk] weights of the selected tokens
+  __shared__ unsigned s_c[kW][GM];
+  __shared__ unsigned s_base[GM];
+  __shared__ __align__(16) float s_scl[kW][32][4];  // per slice token: group scales and minima as fp32
+  __shared__ __align__(16) float s_mnv[kW][32][4];
   __shared__ float s_acc[kW][kD];
-  __shared__ float s_l[kW];
+  __shared__ float s_l[kW][GM];
   const CacheView& c = p.c;
-  const int z = blockIdx.z;  // b * Hkv + kvh
-  const int64_t r = static_cast<int64_t>(z) * G + blockIdx.x;
-  const int chunk = blockIdx.y;
+  const int z = blockIdx.y;  // b * Hkv + kvh
+  const int64_t row0 = static_cast<int64_t>(z) * G;
+  const int chunk = blockIdx.x;
   const int L = p.len[z / c.Hkv];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const ToppRowState& rs = p.rows[r];
-  const uint32_t* cc = p.chunk_cnt + r * p.nchunk;
-  // offset of this chunk = selected tokens of the chunks before it
-  unsigned before = 0;
-  for (int k = threadIdx.x; k < chunk; k += kStreamThreads) before += cc[k];
-  before = warp_sum(before);
-  if (lane == 0) s_c[warp] = before;
+  // offsets of this chunk = selected tokens of the row's chunks before it
+  #pragma unroll
+  for (int h = 0; h < GM; ++h) {
+    if (h < G) {
+      const uint32_t* cc = p.chunk_cnt + (row0 + h) * p.nchunk;
+      unsigned before = 0;
+      for (int k = threadIdx.x; k < chunk; k += kStreamThreads) before += cc[k];
+      before = warp_sum(before);
+      if (lane == 0) s_c[warp][h] = before;
+    }
+  }
   __syncthreads();
-  if (threadIdx.x == 0) {
+  if (threadIdx.x < G) {
+    const int h = threadIdx.x;
     unsigned tot = 0;
-    for (int w = 0; w < kW; ++w) tot += s_c[w];
-    s_base = tot;
-    if (chunk == p.nchunk - 1) p.sel_cnt[r] = static_cast<int32_t>(tot + cc[chunk]);
+    for (int w = 0; w < kW; ++w) tot += s_c[w][h];
+    s_base[h] = tot;
+    if (chunk == p.nchunk - 1) p.sel_cnt[row0 + h] = static_cast<int32_t>(tot + p.chunk_cnt[(row0 + h) * p.nchunk + chunk]);
   }
   __syncthreads();
   const int64_t t0 = static_cast<int64_t>(chunk) * kToppChunk;
-  if (t0 >= L || rs.bstar < 0) return;
+  if (t0 >= L) return;  // block-uniform
   const int64_t t1 = t0 + kToppChunk < L ? t0 + kToppChunk : L;
-  const float m = fkey_inv(rs.maxkey);
-  const float* s = p.s + r * c.cap;
-  int32_t* sel = p.sel_idx + r * c.cap;
+  const int64_t tt0 = t0 + kTokPerThread * threadIdx.x;
+  unsigned mask[GM];
+  float lsum[GM];
+  #pragma unroll
+  for (int h = 0; h < GM; ++h) {
+    mask[h] = 0u;
+    lsum[h] = 0.0f;
+    if (h < G) {
+      const int64_t r = row0 + h;
+      const ToppRowState& rs = p.rows[r];
+      const int bstar = rs.bstar;  // >= 0: the row is not empty
+      const unsigned long long kstar = rs.kstar;
+      const float m = fkey_inv(rs.maxkey);
+      float v[16];
+      load16(p.s + r * c.cap, tt0, t1, v);
+      #pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if (tt0 + i < t1) {
+          const int bk = topp_bucket(topp_t(v[i], m));
+          const bool f = bk < bstar || (bk == bstar && topp_key(v[i], tt0 + i) <= kstar);
+          mask[h] |= static_cast<unsigned>(f) << i;
+        }
+      }
+      const unsigned cnt = __popc(mask[h]);
+      const unsigned incl = warp_incl_scan(cnt);
+      __syncthreads();  // s_c is reused
+      if (lane == 31) s_c[warp][0] = incl;
+      __syncthreads();
+      unsigned off = s_base[h] + incl - cnt;
+      for (int w = 0; w < warp; ++w) off += s_c[w][0];
+      int32_t* sel = p.sel_idx + r * c.cap;
+      unsigned mm = mask[h];
+      while (mm) {
+        const int i = __ffs(mm) - 1;
+        mm &= mm - 1u;
+        sel[off++] = static_cast<int32_t>(tt0 + i);
+      }
+      float* eh = s_e + h * kToppChunk + kTokPerThread * threadIdx.x;
+      #pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        if ((mask[h] >> i) & 1u) {
+          const float e = exp2f(__fmul_rn(__fsub_rn(v[i], m), kL2e));
+          eh[i] = e;
+          lsum[h] += e;
+        }
+      }
+    }
+  }
+  __syncwarp();
+  // gather over the warp's slices where any head selects a token
   const int64_t head_tok = static_cast<int64_t>(z) * c.cap;
   const uint32_t* vcw = c.v_codes + head_tok * 16;
   const uint4* vsm4 = reinterpret_cast<const uint4*>(c.v_sm) + head_tok;
   const int grp = lane >> 3;  // 32-channel group of this lane's channels
-  float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-  float accm = 0.0f, lsum = 0.0f;
-  unsigned base = s_base;
-  for (int64_t tb = t0; tb < t1; tb += kStreamThreads) {
-    const int64_t t = tb + threadIdx.x;
-    const bool f = t < t1 && topp_selected(rs, s, m, t);
-    const unsigned ball = __ballot_sync(kFull, f);
-    __syncthreads();  // the previous round's counts are read
-    if (lane == 0) s_c[warp] = __popc(ball);
-    __syncthreads();
-    unsigned off = 0, tot = 0;
-    for (int w = 0; w < kW; ++w) {
-      off += (w < warp) ? s_c[w] : 0u;
-      tot += s_c[w];
+  unsigned pair[GM];          // slice masks per head, on even lanes
+  unsigned any = 0u;
+  #pragma unroll
+  for (int h = 0; h < GM; ++h) {
+    pair[h] = mask[h] | (__shfl_down_sync(kFull, mask[h], 1) << 16);
+    any |= pair[h];
+  }
+  unsigned active = __ballot_sync(kFull, (lane & 1) == 0 && any != 0u);
+  const int64_t wt0 = t0 + 32 * kTokPerThread * warp;
+  float acc[GM][4], accm[GM];
+  #pragma unroll
+  for (int h = 0; h < GM; ++h) {
+    accm[h] = 0.0f;
+    #pragma unroll
+    for (int q = 0; q < 4; ++q) acc[h][q] = 0.0f;
+  }
+  uint4 cw_n[4], sm_n = make_uint4(0u, 0u, 0u, 0u);
+  int src = active ? __ffs(active) - 1 : -1;
+  auto load_slice = [&](int sl) {
+    const int64_t ts = wt0 + kTokPerThread * sl;  // slice start: a multiple of 32 inside one 128-token tile
+    const unsigned ball_any = __shfl_sync(kFull, any, sl);
+    const uint32_t* cp = vcw + ((ts >> 7) * kD + 4 * lane) * 16 + ((ts & 127) >> 3);
+    #pragma unroll
+    for (int q = 0; q < 4; ++q) cw_n[q] = __ldg(reinterpret_cast<const uint4*>(cp + 16 * q));
+    sm_n = ((ball_any >> lane) & 1u) ? __ldg(vsm4 + ts + lane) : make_uint4(0u, 0u, 0u, 0u);
+  };
+  if (src >= 0) load_slice(src);
+  while (src >= 0) {  // warp-uniform
+    const int cur = src;
+    uint4 cw[4];
+    #pragma unroll
+    for (int q = 0; q < 4; ++q) cw[q] = cw_n[q];
+    {
+      float4 sc, mn;
+      sc.x = __half2float(__ushort_as_half(static_cast<unsigned short>(sm_n.x & 0xffffu)));
+      sc.y = __half2float(__ushort_as_half(static_cast<unsigned short>(sm_n.y & 0xffffu)));
+      sc.z = __half2float(__ushort_as_half(static_cast<unsigned short>(sm_n.z & 0xffffu)));
+      sc.w = __half2float(__ushort_as_half(static_cast<unsigned short>(sm_n.w & 0xffffu)));
+      mn.x = __half2float(__ushort_as_half(static_cast<unsigned short>(sm_n.x >> 16)));
+      mn.y = __half2float(__ushort_as_half(static_cast<unsigned short>(sm_n.y >> 16)));
+      mn.z = __half2float(__ushort_as_half(static_cast<unsigned short>(sm_n.z >> 16)));
+      mn.w = __half2float(__ushort_as_half(static_cast<unsigned short>(sm_n.w >> 16)));
+      *reinterpret_cast<float4*>(&s_scl[warp][lane][0]) = sc;
+      *reinterpret_cast<float4*>(&s_mnv[warp][lane][0]) = mn;
     }
-    if (f) sel[base + off + __popc(ball & ((1u << lane) - 1u))] = static_cast<int32_t>(t);
-    base += tot;
-    if (ball) {  // warp-uniform: gather this slice's selected tokens
-      float e = 0.0f;
-      uint4 smv = make_uint4(0u, 0u, 0u, 0u);
-      if (f) {
-        e = exp2f(__fmul_rn(__fsub_rn(s[t], m), kL2e));
-        smv = __ldg(vsm4 + t);
-      }
-      lsum += e;
-      s_e[warp][lane] = e;
-      *reinterpret_cast<uint4*>(&s_smw[warp][lane][0]) = smv;
-      const int64_t ts = tb + 32 * warp;  // slice start: a multiple of 32 inside one 128-token tile
-      const uint32_t* cp = vcw + ((ts >> 7) * kD + 4 * lane) * 16 + ((ts & 127) >> 3);
-      uint4 cw[4];
-      #pragma unroll
-      for (int q = 0; q < 4; ++q) cw[q] = __ldg(reinterpret_cast<const uint4*>(cp + 16 * q));
-      __syncwarp();
-      #pragma unroll
-      for (int w = 0; w < 4; ++w) {
-        unsigned bits = (ball >> (8 * w)) & 0xffu;
-        while (bits) {
-          const int jj = __ffs(bits) - 1;
-          bits &= bits - 1u;
-          const int j = 8 * w + jj;
-          const float ej = s_e[warp][j];
-          const uint32_t smw = s_smw[warp][j][grp];
-          const float scl = __half2float(__ushort_as_half(static_cast<unsigned short>(smw & 0xffffu)));
-          const float mnv = __half2float(__ushort_as_half(static_cast<unsigned short>(smw >> 16)));
-          const float es = __fmul_rn(ej, scl);
-          accm = __fmaf_rn(ej, mnv, accm);
-          #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint32_t word = w == 0 ? cw[q].x : (w == 1 ? cw[q].y : (w == 2 ? cw[q].z : cw[q].w));
-            acc[q] = __fmaf_rn(es, static_cast<float>((word >> (4 * jj)) & 0xFu), acc[q]);
+    active &= active - 1u;
+    src = active ? __ffs(active) - 1 : -1;
+    if (src >= 0) load_slice(src);  // next slice in flight
+    __syncwarp();
+    #pragma unroll
+    for (int h = 0; h < GM; ++h) {
+      if (h < G) {
+        const unsigned ball = __shfl_sync(kFull, pair[h], cur);
+        const float* ew = s_e + h * kToppChunk + 32 * kTokPerThread * warp + kTokPerThread * cur;
+        #pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          unsigned bits = (ball >> (8 * w)) & 0xffu;
+          while (bits) {
+            const int jj = __ffs(bits) - 1;
+            bits &= bits - 1u;
+            const int j = 8 * w + jj;
+            const float ej = ew[j];
+            const float es = __fmul_rn(ej, s_scl[warp][j][grp]);
+            accm[h] = __fmaf_rn(ej, s_mnv[warp][j][grp], accm[h]);
+            #pragma unroll
+            for (int q = 0; q < 4; ++q) {
+              const uint32_t word = w == 0 ? cw[q].x : (w == 1 ? cw[q].y : (w == 2 ? cw[q].z : cw[q].w));
+              // 2^23 + code as a float (exact), minus 2^23: the code as fp32 without an int conversion
+              const float code = __fsub_rn(__uint_as_float(((word >> (4 * jj)) & 0xFu) | 0x4B000000u), 8388608.0f);
+              acc[h][q] = __fmaf_rn(es, code, acc[h][q]);
+            }
           }
         }
       }
-      __syncwarp();  // s_e / s_smw are rewritten by the next slice
     }
+    __syncwarp();  // s_scl / s_mnv are rewritten for the next slice
   }
   #pragma unroll
-  for (int q = 0; q < 4; ++q) s_acc[warp][4 * lane + q] = acc[q] + accm;
-  lsum = warp_sum(lsum);
-  if (lane == 0) s_l[warp] = lsum;
-  __syncthreads();
-  if (threadIdx.x < kD) {
-    float* row = p.part + (r * p.nchunk + chunk) * kPartStride;
-    float num = 0.0f;
-    for (int w = 0; w < kW; ++w) num += s_acc[w][threadIdx.x];
-    row[2 + threadIdx.x] = num;
-    if (threadIdx.x == 0) {
-      float den = 0.0f;
-      for (int w = 0; w < kW; ++w) den += s_l[w];
-      row[0] = 0.0f;  // every chunk of the row uses the same reference maximum
-      row[1] = den;
+  for (int h = 0; h < GM; ++h) {
+    const float l = warp_sum(lsum[h]);
+    if (lane == 0) s_l[warp][h] = l;
+  }
+  #pragma unroll
+  for (int h = 0; h < GM; ++h) {
+    if (h < G) {
+      __syncthreads();  // s_acc is free
+      #pragma unroll
+      for (int q = 0; q < 4; ++q) s_acc[warp][4 * lane + q] = acc[h][q] + accm[h];
+      __syncthreads();
+      if (threadIdx.x < kD) {
+        float* row = p.part + ((row0 + h) * p.nchunk + chunk) * kPartStride;
+        float num = 0.0f;
+        for (int w = 0; w < kW; ++w) num += s_acc[w][threadIdx.x];
+        row[2 + threadIdx.x] = num;
+        if (threadIdx.x == 0) {
+          float den = 0.0f;
+          for (int w = 0; w < kW; ++w) den += s_l[w][h];
+          row[0] = 0.0f;  // every chunk of the row uses the same reference maximum
+          row[1] = den;
+        }
+      }
     }
   }
 }
 
+// ---------------------------------------------------------------- 7. merge
 // Sum of the row's chunk partials in chunk order; rows with nothing selected give zeros.
 __global__ void __launch_bounds__(kD) topp_merge_kernel(const ToppParams p) {
   const int64_t r = blockIdx.x;
@@ -461,6 +702,7 @@ __global__ void __launch_bounds__(kD) topp_merge_kernel(const ToppParams p) {
   const int nch = p.rows[r].bstar >= 0 ? (L + kToppChunk - 1) / kToppChunk : 0;
   const float* base = p.part + r * p.nchunk * kPartStride;
   float num = 0.0f, den = 0.0f;
+  #pragma unroll 8
   for (int k = 0; k < nch; ++k) {
     num += base[k * kPartStride + 2 + ch];
     den += base[k * kPartStride + 1];
@@ -474,56 +716,90 @@ using namespace kv1b;
 
 namespace {
 size_t al256(size_t x) { return (x + 255) / 256 * 256; }
+struct ToppLayout {
+  size_t planes, qvl, qdl, qsq, s, cand, rows, hist, chunk_cnt, part, total, state_bytes;
+};
+ToppLayout topp_layout(int32_t rows, int32_t cap) {
+  const size_t R = static_cast<size_t>(rows), C = static_cast<size_t>(cap);
+  const size_t nchunk = (C + kToppChunk - 1) / kToppChunk;
+  ToppLayout l;
+  size_t o = 0;
+  l.planes = o;    o += al256(R * 16 * 4);
+  l.qvl = o;       o += al256(R * 4);
+  l.qdl = o;       o += al256(R * 4);
+  l.qsq = o;       o += al256(R * 4);
+  l.s = o;         o += al256(R * C * 4);
+  l.cand = o;      o += al256(R * C * 4);
+  l.rows = o;      o += al256(R * sizeof(ToppRowState));  // rows, hist and chunk_cnt: one memset
+  l.hist = o;      o += al256(R * kToppBuckets * 8);
+  l.chunk_cnt = o; o += al256(R * nchunk * 4);
+  l.state_bytes = o - l.rows;
+  l.part = o;      o += al256(R * nchunk * kPartStride * 4);
+  l.total = o;
+  return l;
+}
 }  // namespace
 
-// Workspace of kv1b_attend_topp: logits, candidates, row states, bucket histograms, chunk counts,
-// gather partials (rows = batch x query heads, capacity tokens each).
-size_t kv1b_topp_workspace_bytes(int32_t rows, int32_t cap) {
-  const size_t R = static_cast<size_t>(rows), C = static_cast<size_t>(cap);
-  const size_t nchunk = (C + kToppChunk - 1) / kToppChunk;
-  return al256(R * C * 4) + al256(R * C * 4) + al256(R * sizeof(ToppRowState)) + al256(R * kToppBuckets * 8) +
-         al256(R * nchunk * 4) + al256(R * nchunk * kPartStride * 4);
-}
+// Workspace of kv1b_attend_topp (rows = batch x query heads, capacity tokens each).
+size_t kv1b_topp_workspace_bytes(int32_t rows, int32_t cap) { return topp_layout(rows, cap).total; }
 
 void kv1b_topp_carve(ToppParams* p, void* ws, int32_t rows, int32_t cap) {
-  const size_t R = static_cast<size_t>(rows), C = static_cast<size_t>(cap);
-  const size_t nchunk = (C + kToppChunk - 1) / kToppChunk;
+  const ToppLayout l = topp_layout(rows, cap);
   char* w = static_cast<char*>(ws);
-  p->s = reinterpret_cast<float*>(w);
-  w += al256(R * C * 4);
-  p->cand = reinterpret_cast<int32_t*>(w);
-  w += al256(R * C * 4);
-  p->rows = reinterpret_cast<ToppRowState*>(w);  // row states and histograms are contiguous: one memset
-  w += al256(R * sizeof(ToppRowState));
-  p->hist = reinterpret_cast<unsigned long long*>(w);
-  w += al256(R * kToppBuckets * 8);
-  p->chunk_cnt = reinterpret_cast<uint32_t*>(w);
-  w += al256(R * nchunk * 4);
-  p->part = reinterpret_cast<float*>(w);
-  p->nchunk = static_cast<int32_t>(nchunk);
+  p->planes = reinterpret_cast<uint32_t*>(w + l.planes);
+  p->qvl = reinterpret_cast<float*>(w + l.qvl);
+  p->qdl = reinterpret_cast<float*>(w + l.qdl);
+  p->qsq = reinterpret_cast<int32_t*>(w + l.qsq);
+  p->s = reinterpret_cast<float*>(w + l.s);
+  p->cand = reinterpret_cast<int32_t*>(w + l.cand);
+  p->rows = reinterpret_cast<ToppRowState*>(w + l.rows);
+  p->hist = reinterpret_cast<unsigned long long*>(w + l.hist);
+  p->chunk_cnt = reinterpret_cast<uint32_t*>(w + l.chunk_cnt);
+  p->part = reinterpret_cast<float*>(w + l.part);
+  p->nchunk = static_cast<int32_t>((static_cast<size_t>(cap) + kToppChunk - 1) / kToppChunk);
 }
 
 cudaError_t kv1b_launch_topp(const ToppParams& p, int32_t G, int32_t max_len, cudaStream_t stream) {
   const int R = p.c.B * p.Hq;
-  if (p.nchunk > 65535) return cudaErrorInvalidValue;  // grid y limit: capacity above 2^28 tokens
-  const size_t state_bytes = al256(static_cast<size_t>(R) * sizeof(ToppRowState)) + static_cast<size_t>(R) * kToppBuckets * 8;
-  cudaError_t e = cudaMemsetAsync(p.rows, 0, state_bytes, stream);
+  if (p.nchunk > 65535 || G > 8) return cudaErrorInvalidValue;  // grid x limit of the row kernels; 8 heads
+  const size_t e_smem = static_cast<size_t>(G) * kToppChunk * 4;
+  static bool configured = false;
+  if (!configured) {
+    cudaError_t e = cudaFuncSetAttribute(topp_resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(kResolveSmem));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(topp_write_gather_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               4 * kToppChunk * 4);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(topp_write_gather_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               8 * kToppChunk * 4);
+    if (e != cudaSuccess) return e;
+    configured = true;
+  }
+  const ToppLayout l = topp_layout(R, p.c.cap);
+  cudaError_t e = cudaMemsetAsync(p.rows, 0, l.state_bytes, stream);
   if (e != cudaSuccess) return e;
   const dim3 sg(static_cast<unsigned>(p.nchunk), static_cast<unsigned>(R));
   if (max_len > 0) {
-    topp_scores_kernel<<<dim3((max_len + kStreamThreads - 1) / kStreamThreads, p.c.Hkv, p.c.B), kStreamThreads, 0,
-                         stream>>>(p, G);
+    e = kv1b_launch_query_prep(p.c, p.q, p.q_dtype, p.Hq, p.planes, p.qvl, p.qdl, p.qsq, stream);
+    if (e != cudaSuccess) return e;
+    const dim3 grid((max_len + kScoreTok - 1) / kScoreTok, p.c.Hkv, p.c.B);
+    if (G <= 4)
+      topp_scores_kernel<1><<<grid, kStreamThreads, 0, stream>>>(p, G);
+    else
+      topp_scores_kernel<2><<<grid, kStreamThreads, 0, stream>>>(p, G);
     topp_mass_kernel<<<sg, kStreamThreads, 0, stream>>>(p);
   }
-  topp_threshold_kernel<<<R, kToppBuckets, 0, stream>>>(p);
+  topp_threshold_kernel<<<R, kThresholdThreads, 0, stream>>>(p);
   if (max_len > 0) {
     topp_cand_kernel<<<sg, kStreamThreads, 0, stream>>>(p);
-    topp_resolve_kernel<<<R, kResolveThreads, 0, stream>>>(p);
+    topp_resolve_kernel<<<R, kResolveThreads, kResolveSmem, stream>>>(p);
   }
-  topp_count_kernel<<<sg, kStreamThreads, 0, stream>>>(p);
-  topp_write_gather_kernel<<<dim3(static_cast<unsigned>(G), static_cast<unsigned>(p.nchunk),
-                              static_cast<unsigned>(p.c.B * p.c.Hkv)),
-                         kStreamThreads, 0, stream>>>(p, G);
+  const dim3 gg(static_cast<unsigned>(p.nchunk), static_cast<unsigned>(p.c.B * p.c.Hkv));
+  if (G <= 4)
+    topp_write_gather_kernel<4><<<gg, kStreamThreads, e_smem, stream>>>(p, G);
+  else
+    topp_write_gather_kernel<8><<<gg, kStreamThreads, e_smem, stream>>>(p, G);
   topp_merge_kernel<<<R, kD, 0, stream>>>(p);
   return cudaGetLastError();
 }

@@ -260,3 +260,13 @@ def test_topp_multi_chunk_ragged(scale):
     q = q.to(torch.bfloat16)
     for p in (0.5, 0.99):
         topp_check(cache, host, q, scale, p, G, oracle.signs(5))
+
+
+@pytest.mark.parametrize("G,qdt", [(1, torch.float32), (3, torch.float16), (8, torch.bfloat16)])
+def test_topp_group_sizes(G, qdt):
+    # one, a non-power-of-two and the largest number of query heads per kv-head (two operand groups)
+    B, Hkv = 1, 2
+    cache, host = build_cache(B, Hkv, [4500], torch.bfloat16, seed=13, data_seed=8)
+    q = torch.randn((B, Hkv * G, 128), device=DEV, generator=torch.Generator(device=DEV).manual_seed(5)).to(qdt)
+    for p in (0.3, 0.95):
+        topp_check(cache, host, q, 0.4, p, G, oracle.signs(13))
