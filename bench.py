@@ -357,7 +357,7 @@ def run_ours(args):
                 "sel_min": int(tcnt.min().item()), "sel_max": int(tcnt.max().item()),
                 "algorithmic_bytes": alg, "achieved_gbs": alg / (t_ms * 1e-3) / 1e9,
                 "bytes_rule": "24 B per token x kv-head (scores) + 80 B per selected token x query head (gather)",
-                "kernels": "memset + scores, mass, threshold, cand, resolve, count, write_gather, merge (median of 5)"}
+                "kernels": "memset + query prep, scores, mass, threshold, cand, resolve, write_gather, merge (median of 5)"}
         topp["frac"] = topp["achieved_gbs"] / peak
 
     result = None

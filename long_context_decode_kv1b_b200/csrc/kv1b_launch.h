@@ -65,7 +65,7 @@ struct ToppRowState {
   uint32_t maxkey;           // order-preserving key of the row's largest logit (atomicMax)
   uint32_t ncand;            // tokens in the threshold bucket
   int32_t bstar;             // threshold bucket (-1: the row is empty)
-  uint32_t pad0;
+  uint32_t merged;           // merge blocks of the row done (atomic ticket)
   unsigned long long U;      // total integer mass
   unsigned long long rem;    // mass still needed inside the threshold bucket
   unsigned long long kstar;  // largest selected 64-bit key of the threshold bucket
@@ -73,6 +73,8 @@ struct ToppRowState {
 };
 constexpr int kToppBuckets = 2048;  // masses by t = (s - m) log2 e: bucket floor(-64 t), t >= -40
 constexpr int kToppChunk = 4096;    // tokens per block of the streaming kernels
+constexpr int kToppSub = 1024;      // tokens per selected-count entry and per compaction+gather block
+constexpr int kToppMergeSplit = 8;  // first-level merge blocks per row
 
 struct ToppParams {
   CacheView c;
@@ -89,9 +91,11 @@ struct ToppParams {
   int32_t* cand;             // [R][cap] threshold-bucket candidates (any order)
   ToppRowState* rows;        // [R]
   unsigned long long* hist;  // [R][kToppBuckets] masses per bucket
-  uint32_t* chunk_cnt;       // [R][nchunk] selected tokens per chunk (lower buckets, then candidates)
-  float* part;               // [R][nchunk][kPartStride] gather partials per chunk
+  uint32_t* sub_cnt;         // [R][nsub] selected tokens per sub-chunk (lower buckets, then candidates)
+  float* part;               // [R][nsub][kPartStride] gather partials per sub-chunk
+  float* part2;              // [R][kToppMergeSplit][kPartStride] first-level merge sums
   int32_t nchunk;
+  int32_t nsub;
   float* out;
   int32_t* sel_idx;
   int32_t* sel_cnt;

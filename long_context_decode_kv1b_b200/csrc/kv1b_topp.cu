@@ -107,6 +107,11 @@ __device__ __forceinline__ void load16(const float* s, int64_t t0, int64_t t1, f
   }
 }
 
+// Programmatic dependent launch: a kernel launched with the programmatic-serialization attribute may
+// be scheduled while its predecessor in the stream is still running; griddepcontrol.wait returns once
+// every prerequisite grid has completed and its memory is visible (a no-op for a plain launch).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 // ---------------------------------------------------------------- 1. logits and row maxima
 // Integer MMA D += A B (16 x 32 s8 by 32 x 8 s8 -> s32).
 __device__ __forceinline__ void mma_s8(int d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
@@ -157,6 +162,7 @@ __device__ __forceinline__ void build_bq(uint32_t (&bq)[4][2], const uint32_t* p
 // heads as NG groups of 4 operand-column pairs.
 template <int NG>
 __global__ void __launch_bounds__(kStreamThreads) topp_scores_kernel(const ToppParams p, int G) {
+  pdl_wait();
   __shared__ float s_max[kStreamWarps][8];
   const CacheView& c = p.c;
   const int b = blockIdx.z, kvh = blockIdx.y;
@@ -232,11 +238,13 @@ __global__ void __launch_bounds__(kStreamThreads) topp_scores_kernel(const ToppP
 }
 
 // ---------------------------------------------------------------- 2. masses and bucket histogram
-// grid (chunks of kToppChunk tokens, rows); thread = 16 contiguous tokens.  The block histogram keeps
-// each bucket's 64-bit sum as a wrapping 32-bit low word plus a count of carries (32-bit shared
-// atomics); the block then adds its non-empty buckets to the row's 64-bit histogram.
+// grid (chunks of kToppChunk tokens, rows); thread = 16 contiguous tokens.  u < 2^33 is split as
+// uh 2^16 + ul (ul < 2^16, uh < 2^17); per bucket the block sums ul and uh separately with 32-bit
+// shared reductions (at most 4096 tokens: no overflow), then adds each non-empty bucket's
+// (sum uh) 2^16 + sum ul to the row's 64-bit histogram.
 __global__ void __launch_bounds__(kStreamThreads) topp_mass_kernel(const ToppParams p) {
-  __shared__ uint32_t s_lo[kToppBuckets], s_hi[kToppBuckets];
+  pdl_wait();
+  __shared__ uint32_t s_lo[kToppBuckets], s_hi[kToppBuckets];  // sums of ul and of uh per bucket
   __shared__ unsigned long long s_u[kStreamWarps];
   const int64_t r = blockIdx.y;
   const int L = row_len(p, r);
@@ -260,10 +268,8 @@ __global__ void __launch_bounds__(kStreamThreads) topp_mass_kernel(const ToppPar
       const uint64_t u = topp_mass_t(tt);
       if (u) {
         const int bk = topp_bucket(tt);
-        const uint32_t ulo = static_cast<uint32_t>(u);
-        const uint32_t old = atomicAdd(&s_lo[bk], ulo);
-        const uint32_t inc = static_cast<uint32_t>(u >> 32) + (old + ulo < old ? 1u : 0u);
-        if (inc) atomicAdd(&s_hi[bk], inc);
+        atomicAdd(&s_lo[bk], static_cast<uint32_t>(u & 0xffffu));
+        atomicAdd(&s_hi[bk], static_cast<uint32_t>(u >> 16));
         usum += u;
       }
     }
@@ -273,7 +279,7 @@ __global__ void __launch_bounds__(kStreamThreads) topp_mass_kernel(const ToppPar
   __syncthreads();
   unsigned long long* hist = p.hist + r * kToppBuckets;
   for (int i = threadIdx.x; i < kToppBuckets; i += kStreamThreads) {
-    const unsigned long long h = (static_cast<unsigned long long>(s_hi[i]) << 32) | s_lo[i];
+    const unsigned long long h = (static_cast<unsigned long long>(s_hi[i]) << 16) + s_lo[i];
     if (h) atomicAdd(&hist[i], h);
   }
   if (threadIdx.x == 0) {
@@ -287,6 +293,7 @@ __global__ void __launch_bounds__(kStreamThreads) topp_mass_kernel(const ToppPar
 // grid (rows), 1024 threads: thread i owns buckets 2i and 2i + 1.
 constexpr int kThresholdThreads = kToppBuckets / 2;
 __global__ void __launch_bounds__(kThresholdThreads) topp_threshold_kernel(const ToppParams p) {
+  pdl_wait();
   __shared__ unsigned long long s_w[kThresholdThreads / 32];
   const int64_t r = blockIdx.x;
   ToppRowState& rs = p.rows[r];
@@ -332,8 +339,10 @@ __global__ void __launch_bounds__(kThresholdThreads) topp_threshold_kernel(const
 }
 
 // ---------------------------------------------------------------- 4. candidates and lower-bucket counts
+static_assert(kToppChunk % kToppSub == 0 && kToppSub % (32 * kTokPerThread) == 0, "sub-chunks are whole warps");
 // grid (chunks, rows); thread = 16 contiguous tokens.
 __global__ void __launch_bounds__(kStreamThreads) topp_cand_kernel(const ToppParams p) {
+  pdl_wait();
   __shared__ unsigned s_c[kStreamWarps];
   const int64_t r = blockIdx.y;
   const int L = row_len(p, r);
@@ -370,10 +379,12 @@ __global__ void __launch_bounds__(kStreamThreads) topp_cand_kernel(const ToppPar
   lo = warp_sum(lo);
   if (lane == 0) s_c[warp] = lo;
   __syncthreads();
-  if (threadIdx.x == 0) {
+  constexpr int kSubsPerChunk = kToppChunk / kToppSub, kWarpsPerSub = kStreamWarps / kSubsPerChunk;
+  if (threadIdx.x < kSubsPerChunk) {
+    const int64_t sb = static_cast<int64_t>(blockIdx.x) * kSubsPerChunk + threadIdx.x;
     unsigned tot = 0;
-    for (int w = 0; w < kStreamWarps; ++w) tot += s_c[w];
-    p.chunk_cnt[r * p.nchunk + blockIdx.x] = tot;
+    for (int w = 0; w < kWarpsPerSub; ++w) tot += s_c[kWarpsPerSub * threadIdx.x + w];
+    if (sb < p.nsub) p.sub_cnt[r * p.nsub + sb] = tot;
   }
 }
 
@@ -382,6 +393,7 @@ __global__ void __launch_bounds__(kStreamThreads) topp_cand_kernel(const ToppPar
 // candidates' unique keys with per-bin mass histograms; K* = the smallest key whose cumulative
 // mass (in key order) reaches rem.  Up to kResolveSmemCand candidates keep key and mass on chip.
 __global__ void __launch_bounds__(kResolveThreads) topp_resolve_kernel(const ToppParams p) {
+  pdl_wait();
   extern __shared__ unsigned long long s_kv[];  // [kResolveSmemCand] keys, then masses
   __shared__ uint32_t h_lo[256], h_hi[256];     // bin masses: wrapping low word + carries
   __shared__ unsigned long long s_prefix, s_rem;
@@ -471,15 +483,15 @@ __global__ void __launch_bounds__(kResolveThreads) topp_resolve_kernel(const Top
   }
   const unsigned long long kstar = s_prefix;
   if (threadIdx.x == 0) rs.kstar = kstar;
-  // selected candidates join their chunks' counts (one atomic per chunk and warp)
-  uint32_t* cc = p.chunk_cnt + r * p.nchunk;
+  // selected candidates join their sub-chunks' counts (one atomic per sub-chunk and warp)
+  uint32_t* cc = p.sub_cnt + r * p.nsub;
   for (int i0 = 0; i0 < n; i0 += kResolveThreads) {  // block-uniform trip count
     const int i = i0 + threadIdx.x;
     int ck = -1;
     if (i < n) {
       const int64_t t = cand[i];
       const unsigned long long key = on_chip ? skey[i] : topp_key(s[t], t);
-      if (key <= kstar) ck = static_cast<int>(t / kToppChunk);
+      if (key <= kstar) ck = static_cast<int>(t / kToppSub);
     }
     const unsigned same = __match_any_sync(kFull, ck);
     if (ck >= 0 && lane == __ffs(same) - 1) atomicAdd(&cc[ck], static_cast<unsigned>(__popc(same)));
@@ -487,116 +499,140 @@ __global__ void __launch_bounds__(kResolveThreads) topp_resolve_kernel(const Top
 }
 
 // ---------------------------------------------------------------- 6. ordered writes + gather-attend
-// grid (chunks, B * Hkv): one block serves the G query heads of a kv-head, so each code tile of the
-// chunk is read once for all of them.  Thread = 16 contiguous tokens.  Per head: selection mask,
-// block scan, ordered index writes, softmax weights of the selected tokens into shared memory.
-// Then warp w gathers its 512 tokens in slices of 32 (lanes 2k, 2k + 1): for each slice where any
-// head selects a token, lane l loads the slice's 4-bit codes of channels 4l..4l+3 (one 16-byte group
-// per channel), the next such slice's loads in flight meanwhile, and accumulates, per head,
-// e * (scale * code + min) over that head's selected tokens.  Each head's (numerator, denominator)
-// against its row maximum goes to part[row][chunk].
+// grid (sub-chunks of kToppSub tokens, B * Hkv): one block serves the G query heads of a kv-head, so
+// each code tile is read once for all of them.  Thread = 4 contiguous tokens, warp = one 128-token
+// code tile.  Per head: selection mask, block scan, ordered index writes, softmax weights of the
+// selected tokens into shared memory.  Then each warp gathers its tile in slices of 32 tokens (lanes
+// 8k .. 8k + 7): for each slice where any head selects a token, lane l loads the slice's 4-bit codes
+// of channels 4l..4l+3 (one 16-byte group per channel), the next such slice's loads in flight
+// meanwhile, and accumulates, per head, e * (scale * code + min) over that head's selected tokens.
+// Each head's (numerator, denominator) against its row maximum goes to part[row][sub-chunk].
 template <int GM>
-__global__ void __launch_bounds__(kStreamThreads) topp_write_gather_kernel(const ToppParams p, int G) {
+__global__ void __launch_bounds__(kStreamThreads, GM <= 4 ? 3 : 2) topp_write_gather_kernel(const ToppParams p, int G) {
+  pdl_wait();
   constexpr int kW = kStreamWarps;
-  extern __shared__ float s_e[];  // [G][kToppChunk] weights of the selected tokens
-  __shared__ unsigned s_c[kW][GM];
-  __shared__ unsigned s_base[GM];
+  constexpr int kTok = kToppSub / kStreamThreads;  // contiguous tokens per thread
+  constexpr int kPk = (GM + 1) / 2;                // per-thread counts, two heads per 32-bit word
+  static_assert(kTok == 4 && kTok * 32 == 128, "a warp covers one 128-token code tile");
+  static_assert(kW * kD == kToppSub, "the weight buffer doubles as the cross-warp reduction buffer");
+  __shared__ float s_e[GM][kToppSub];               // weights of the selected tokens, then partial sums
+  __shared__ unsigned s_before[kW][GM];
+  __shared__ unsigned s_cnt[kW][kPk];
   __shared__ __align__(16) float s_scl[kW][32][4];  // per slice token: group scales and minima as fp32
   __shared__ __align__(16) float s_mnv[kW][32][4];
-  __shared__ float s_acc[kW][kD];
   __shared__ float s_l[kW][GM];
   const CacheView& c = p.c;
   const int z = blockIdx.y;  // b * Hkv + kvh
   const int64_t row0 = static_cast<int64_t>(z) * G;
-  const int chunk = blockIdx.x;
+  const int sub = blockIdx.x;
   const int L = p.len[z / c.Hkv];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  // offsets of this chunk = selected tokens of the row's chunks before it
+  const int64_t t0 = static_cast<int64_t>(sub) * kToppSub;
+  const int64_t t1 = t0 + kToppSub < L ? t0 + kToppSub : L;
+  const int64_t tt0 = t0 + kTok * threadIdx.x;
+  // independent global reads first: earlier sub-chunks' counts, row states, this thread's logits
+  unsigned before[GM], mask[GM];
+  float4 x4[GM];
+  float mrow[GM];
   #pragma unroll
   for (int h = 0; h < GM; ++h) {
+    before[h] = 0u;
+    mask[h] = 0u;
+    x4[h] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    mrow[h] = 0.0f;
     if (h < G) {
-      const uint32_t* cc = p.chunk_cnt + (row0 + h) * p.nchunk;
-      unsigned before = 0;
-      for (int k = threadIdx.x; k < chunk; k += kStreamThreads) before += cc[k];
-      before = warp_sum(before);
-      if (lane == 0) s_c[warp][h] = before;
+      const uint32_t* cc = p.sub_cnt + (row0 + h) * p.nsub;
+      for (int k = threadIdx.x; k < sub; k += kStreamThreads) before[h] += cc[k];
+      if (tt0 < t1) x4[h] = *reinterpret_cast<const float4*>(p.s + (row0 + h) * c.cap + tt0);  // inside the row
     }
   }
-  __syncthreads();
-  if (threadIdx.x < G) {
-    const int h = threadIdx.x;
-    unsigned tot = 0;
-    for (int w = 0; w < kW; ++w) tot += s_c[w][h];
-    s_base[h] = tot;
-    if (chunk == p.nchunk - 1) p.sel_cnt[row0 + h] = static_cast<int32_t>(tot + p.chunk_cnt[(row0 + h) * p.nchunk + chunk]);
-  }
-  __syncthreads();
-  const int64_t t0 = static_cast<int64_t>(chunk) * kToppChunk;
-  if (t0 >= L) return;  // block-uniform
-  const int64_t t1 = t0 + kToppChunk < L ? t0 + kToppChunk : L;
-  const int64_t tt0 = t0 + kTokPerThread * threadIdx.x;
-  unsigned mask[GM];
-  float lsum[GM];
   #pragma unroll
   for (int h = 0; h < GM; ++h) {
-    mask[h] = 0u;
-    lsum[h] = 0.0f;
-    if (h < G) {
-      const int64_t r = row0 + h;
-      const ToppRowState& rs = p.rows[r];
+    if (h < G && tt0 < t1) {
+      const ToppRowState& rs = p.rows[row0 + h];
       const int bstar = rs.bstar;  // >= 0: the row is not empty
       const unsigned long long kstar = rs.kstar;
       const float m = fkey_inv(rs.maxkey);
-      float v[16];
-      load16(p.s + r * c.cap, tt0, t1, v);
+      mrow[h] = m;
+      const float v[4] = {x4[h].x, x4[h].y, x4[h].z, x4[h].w};
       #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < kTok; ++i) {
         if (tt0 + i < t1) {
           const int bk = topp_bucket(topp_t(v[i], m));
           const bool f = bk < bstar || (bk == bstar && topp_key(v[i], tt0 + i) <= kstar);
           mask[h] |= static_cast<unsigned>(f) << i;
         }
       }
-      const unsigned cnt = __popc(mask[h]);
-      const unsigned incl = warp_incl_scan(cnt);
-      __syncthreads();  // s_c is reused
-      if (lane == 31) s_c[warp][0] = incl;
-      __syncthreads();
-      unsigned off = s_base[h] + incl - cnt;
-      for (int w = 0; w < warp; ++w) off += s_c[w][0];
-      int32_t* sel = p.sel_idx + r * c.cap;
-      unsigned mm = mask[h];
-      while (mm) {
-        const int i = __ffs(mm) - 1;
-        mm &= mm - 1u;
-        sel[off++] = static_cast<int32_t>(tt0 + i);
+    }
+  }
+  // one block scan for all heads (counts <= kToppSub fit 16 bits)
+  unsigned pk[kPk], incl[kPk];
+  #pragma unroll
+  for (int w = 0; w < kPk; ++w) pk[w] = 0u;
+  #pragma unroll
+  for (int h = 0; h < GM; ++h) pk[h >> 1] |= static_cast<unsigned>(__popc(mask[h])) << (16 * (h & 1));
+  #pragma unroll
+  for (int w = 0; w < kPk; ++w) {
+    incl[w] = warp_incl_scan(pk[w]);
+    if (lane == 31) s_cnt[warp][w] = incl[w];
+  }
+  #pragma unroll
+  for (int h = 0; h < GM; ++h) {
+    if (h < G) {
+      const unsigned bsum = warp_sum(before[h]);
+      if (lane == 0) s_before[warp][h] = bsum;
+    }
+  }
+  __syncthreads();
+  float lsum[GM];
+  #pragma unroll
+  for (int h = 0; h < GM; ++h) {
+    lsum[h] = 0.0f;
+    if (h < G) {
+      const int sh = 16 * (h & 1);
+      unsigned base = 0, prior = 0, tot = 0;
+      for (int w = 0; w < kW; ++w) {
+        base += s_before[w][h];
+        const unsigned cw = (s_cnt[w][h >> 1] >> sh) & 0xffffu;
+        prior += (w < warp) ? cw : 0u;
+        tot += cw;
       }
-      float* eh = s_e + h * kToppChunk + kTokPerThread * threadIdx.x;
+      if (sub == p.nsub - 1 && threadIdx.x == 0) p.sel_cnt[row0 + h] = static_cast<int32_t>(base + tot);
+      const unsigned cnt = __popc(mask[h]);
+      unsigned off = base + prior + ((incl[h >> 1] >> sh) & 0xffffu) - cnt;
+      int32_t* sel = p.sel_idx + (row0 + h) * c.cap;
+      const float v[4] = {x4[h].x, x4[h].y, x4[h].z, x4[h].w};
       #pragma unroll
-      for (int i = 0; i < 16; ++i) {
+      for (int i = 0; i < kTok; ++i) {
         if ((mask[h] >> i) & 1u) {
-          const float e = exp2f(__fmul_rn(__fsub_rn(v[i], m), kL2e));
-          eh[i] = e;
+          sel[off++] = static_cast<int32_t>(tt0 + i);
+          const float e = exp2f(__fmul_rn(__fsub_rn(v[i], mrow[h]), kL2e));
+          s_e[h][kTok * threadIdx.x + i] = e;
           lsum[h] += e;
         }
       }
     }
   }
+  if (t0 >= L) return;  // block-uniform; nothing to gather
   __syncwarp();
   // gather over the warp's slices where any head selects a token
   const int64_t head_tok = static_cast<int64_t>(z) * c.cap;
   const uint32_t* vcw = c.v_codes + head_tok * 16;
   const uint4* vsm4 = reinterpret_cast<const uint4*>(c.v_sm) + head_tok;
   const int grp = lane >> 3;  // 32-channel group of this lane's channels
-  unsigned pair[GM];          // slice masks per head, on even lanes
+  unsigned pair[GM];          // 32-token slice masks per head, on every lane of the slice's 8 lanes
   unsigned any = 0u;
   #pragma unroll
   for (int h = 0; h < GM; ++h) {
-    pair[h] = mask[h] | (__shfl_down_sync(kFull, mask[h], 1) << 16);
-    any |= pair[h];
+    unsigned x = mask[h] << (kTok * (lane & 7));
+    x |= __shfl_xor_sync(kFull, x, 1);
+    x |= __shfl_xor_sync(kFull, x, 2);
+    x |= __shfl_xor_sync(kFull, x, 4);
+    pair[h] = x;
+    any |= x;
   }
-  unsigned active = __ballot_sync(kFull, (lane & 1) == 0 && any != 0u);
-  const int64_t wt0 = t0 + 32 * kTokPerThread * warp;
+  unsigned active = __ballot_sync(kFull, (lane & 7) == 0 && any != 0u);
+  const int64_t wt0 = t0 + 32 * kTok * warp;
   float acc[GM][4], accm[GM];
   #pragma unroll
   for (int h = 0; h < GM; ++h) {
@@ -607,7 +643,7 @@ __global__ void __launch_bounds__(kStreamThreads) topp_write_gather_kernel(const
   uint4 cw_n[4], sm_n = make_uint4(0u, 0u, 0u, 0u);
   int src = active ? __ffs(active) - 1 : -1;
   auto load_slice = [&](int sl) {
-    const int64_t ts = wt0 + kTokPerThread * sl;  // slice start: a multiple of 32 inside one 128-token tile
+    const int64_t ts = wt0 + kTok * sl;  // slice start: a multiple of 32 inside the warp's tile
     const unsigned ball_any = __shfl_sync(kFull, any, sl);
     const uint32_t* cp = vcw + ((ts >> 7) * kD + 4 * lane) * 16 + ((ts & 127) >> 3);
     #pragma unroll
@@ -641,7 +677,7 @@ __global__ void __launch_bounds__(kStreamThreads) topp_write_gather_kernel(const
     for (int h = 0; h < GM; ++h) {
       if (h < G) {
         const unsigned ball = __shfl_sync(kFull, pair[h], cur);
-        const float* ew = s_e + h * kToppChunk + 32 * kTokPerThread * warp + kTokPerThread * cur;
+        const float* ew = &s_e[h][32 * kTok * warp + kTok * cur];
         #pragma unroll
         for (int w = 0; w < 4; ++w) {
           unsigned bits = (ball >> (8 * w)) & 0xffu;
@@ -670,42 +706,69 @@ __global__ void __launch_bounds__(kStreamThreads) topp_write_gather_kernel(const
     const float l = warp_sum(lsum[h]);
     if (lane == 0) s_l[warp][h] = l;
   }
+  __syncthreads();  // every warp is done with the weights: s_e becomes [head][warp][channel] sums
   #pragma unroll
   for (int h = 0; h < GM; ++h) {
     if (h < G) {
-      __syncthreads();  // s_acc is free
       #pragma unroll
-      for (int q = 0; q < 4; ++q) s_acc[warp][4 * lane + q] = acc[h][q] + accm[h];
-      __syncthreads();
-      if (threadIdx.x < kD) {
-        float* row = p.part + ((row0 + h) * p.nchunk + chunk) * kPartStride;
-        float num = 0.0f;
-        for (int w = 0; w < kW; ++w) num += s_acc[w][threadIdx.x];
-        row[2 + threadIdx.x] = num;
-        if (threadIdx.x == 0) {
-          float den = 0.0f;
-          for (int w = 0; w < kW; ++w) den += s_l[w][h];
-          row[0] = 0.0f;  // every chunk of the row uses the same reference maximum
-          row[1] = den;
-        }
-      }
+      for (int q = 0; q < 4; ++q) s_e[h][kD * warp + 4 * lane + q] = acc[h][q] + accm[h];
+    }
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < G * kD; i += kStreamThreads) {
+    const int h = i / kD, ch = i % kD;
+    float* row = p.part + ((row0 + h) * p.nsub + sub) * kPartStride;
+    float num = 0.0f;
+    for (int w = 0; w < kW; ++w) num += s_e[h][kD * w + ch];
+    row[2 + ch] = num;
+    if (ch == 0) {
+      float den = 0.0f;
+      for (int w = 0; w < kW; ++w) den += s_l[w][h];
+      row[0] = 0.0f;  // every sub-chunk of the row uses the same reference maximum
+      row[1] = den;
     }
   }
 }
 
 // ---------------------------------------------------------------- 7. merge
-// Sum of the row's chunk partials in chunk order; rows with nothing selected give zeros.
+// grid (kToppMergeSplit, rows), 128 threads: block j sums the row's sub-chunk partials
+// [j n / M, (j + 1) n / M) in order into part2[row][j]; the row's last block to finish (atomic ticket
+// after a fence) sums the M first-level sums in order and writes out = numerator / denominator.
+// Rows with nothing selected give zeros.
 __global__ void __launch_bounds__(kD) topp_merge_kernel(const ToppParams p) {
-  const int64_t r = blockIdx.x;
+  pdl_wait();
+  constexpr int M = kToppMergeSplit;
+  __shared__ bool s_last;
+  const int64_t r = blockIdx.y;
+  const int j = blockIdx.x;
   const int ch = threadIdx.x;
   const int L = row_len(p, r);
-  const int nch = p.rows[r].bstar >= 0 ? (L + kToppChunk - 1) / kToppChunk : 0;
-  const float* base = p.part + r * p.nchunk * kPartStride;
+  const int n = p.rows[r].bstar >= 0 ? (L + kToppSub - 1) / kToppSub : 0;
+  const int k0 = static_cast<int>(static_cast<int64_t>(n) * j / M);
+  const int k1 = static_cast<int>(static_cast<int64_t>(n) * (j + 1) / M);
+  const float* base = p.part + r * p.nsub * kPartStride;
   float num = 0.0f, den = 0.0f;
   #pragma unroll 8
-  for (int k = 0; k < nch; ++k) {
+  for (int k = k0; k < k1; ++k) {
     num += base[k * kPartStride + 2 + ch];
     den += base[k * kPartStride + 1];
+  }
+  float* q2 = p.part2 + (r * M + j) * kPartStride;
+  q2[2 + ch] = num;
+  if (ch == 0) q2[1] = den;
+  __threadfence();
+  __syncthreads();
+  if (ch == 0) s_last = atomicAdd(&p.rows[r].merged, 1u) == M - 1;
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  const float* b2 = p.part2 + r * M * kPartStride;
+  num = 0.0f;
+  den = 0.0f;
+  #pragma unroll
+  for (int k = 0; k < M; ++k) {
+    num += __ldcg(b2 + k * kPartStride + 2 + ch);
+    den += __ldcg(b2 + k * kPartStride + 1);
   }
   p.out[r * kD + ch] = den > 0.0f ? __fdiv_rn(num, den) : 0.0f;
 }
@@ -716,12 +779,29 @@ using namespace kv1b;
 
 namespace {
 size_t al256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Launch with programmatic stream serialization (the kernel starts with pdl_wait()).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
 struct ToppLayout {
-  size_t planes, qvl, qdl, qsq, s, cand, rows, hist, chunk_cnt, part, total, state_bytes;
+  size_t planes, qvl, qdl, qsq, s, cand, rows, hist, sub_cnt, part, part2, total, state_bytes;
 };
 ToppLayout topp_layout(int32_t rows, int32_t cap) {
   const size_t R = static_cast<size_t>(rows), C = static_cast<size_t>(cap);
-  const size_t nchunk = (C + kToppChunk - 1) / kToppChunk;
+  const size_t nsub = (C + kToppSub - 1) / kToppSub;
   ToppLayout l;
   size_t o = 0;
   l.planes = o;    o += al256(R * 16 * 4);
@@ -730,11 +810,12 @@ ToppLayout topp_layout(int32_t rows, int32_t cap) {
   l.qsq = o;       o += al256(R * 4);
   l.s = o;         o += al256(R * C * 4);
   l.cand = o;      o += al256(R * C * 4);
-  l.rows = o;      o += al256(R * sizeof(ToppRowState));  // rows, hist and chunk_cnt: one memset
+  l.rows = o;      o += al256(R * sizeof(ToppRowState));  // rows, hist and sub_cnt: one memset
   l.hist = o;      o += al256(R * kToppBuckets * 8);
-  l.chunk_cnt = o; o += al256(R * nchunk * 4);
+  l.sub_cnt = o;   o += al256(R * nsub * 4);
   l.state_bytes = o - l.rows;
-  l.part = o;      o += al256(R * nchunk * kPartStride * 4);
+  l.part = o;      o += al256(R * nsub * kPartStride * 4);
+  l.part2 = o;     o += al256(R * kToppMergeSplit * kPartStride * 4);
   l.total = o;
   return l;
 }
@@ -754,25 +835,20 @@ void kv1b_topp_carve(ToppParams* p, void* ws, int32_t rows, int32_t cap) {
   p->cand = reinterpret_cast<int32_t*>(w + l.cand);
   p->rows = reinterpret_cast<ToppRowState*>(w + l.rows);
   p->hist = reinterpret_cast<unsigned long long*>(w + l.hist);
-  p->chunk_cnt = reinterpret_cast<uint32_t*>(w + l.chunk_cnt);
+  p->sub_cnt = reinterpret_cast<uint32_t*>(w + l.sub_cnt);
   p->part = reinterpret_cast<float*>(w + l.part);
+  p->part2 = reinterpret_cast<float*>(w + l.part2);
   p->nchunk = static_cast<int32_t>((static_cast<size_t>(cap) + kToppChunk - 1) / kToppChunk);
+  p->nsub = static_cast<int32_t>((static_cast<size_t>(cap) + kToppSub - 1) / kToppSub);
 }
 
 cudaError_t kv1b_launch_topp(const ToppParams& p, int32_t G, int32_t max_len, cudaStream_t stream) {
   const int R = p.c.B * p.Hq;
-  if (p.nchunk > 65535 || G > 8) return cudaErrorInvalidValue;  // grid x limit of the row kernels; 8 heads
-  const size_t e_smem = static_cast<size_t>(G) * kToppChunk * 4;
+  if (R > 65535 || G > 8) return cudaErrorInvalidValue;  // grid y of the row kernels; two groups of 4 heads
   static bool configured = false;
   if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(topp_resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(kResolveSmem));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(topp_write_gather_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               4 * kToppChunk * 4);
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(topp_write_gather_kernel<8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               8 * kToppChunk * 4);
+    const cudaError_t e = cudaFuncSetAttribute(topp_resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(kResolveSmem));
     if (e != cudaSuccess) return e;
     configured = true;
   }
@@ -780,26 +856,27 @@ cudaError_t kv1b_launch_topp(const ToppParams& p, int32_t G, int32_t max_len, cu
   cudaError_t e = cudaMemsetAsync(p.rows, 0, l.state_bytes, stream);
   if (e != cudaSuccess) return e;
   const dim3 sg(static_cast<unsigned>(p.nchunk), static_cast<unsigned>(R));
+  const dim3 bs(kStreamThreads);
+  // the first kernel after the memset is a plain launch; the rest overlap their predecessor's tail
   if (max_len > 0) {
     e = kv1b_launch_query_prep(p.c, p.q, p.q_dtype, p.Hq, p.planes, p.qvl, p.qdl, p.qsq, stream);
     if (e != cudaSuccess) return e;
     const dim3 grid((max_len + kScoreTok - 1) / kScoreTok, p.c.Hkv, p.c.B);
-    if (G <= 4)
-      topp_scores_kernel<1><<<grid, kStreamThreads, 0, stream>>>(p, G);
-    else
-      topp_scores_kernel<2><<<grid, kStreamThreads, 0, stream>>>(p, G);
-    topp_mass_kernel<<<sg, kStreamThreads, 0, stream>>>(p);
+    e = G <= 4 ? launch_pdl(topp_scores_kernel<1>, grid, bs, 0, stream, p, G)
+               : launch_pdl(topp_scores_kernel<2>, grid, bs, 0, stream, p, G);
+    if (e == cudaSuccess) e = launch_pdl(topp_mass_kernel, sg, bs, 0, stream, p);
+    if (e == cudaSuccess) e = launch_pdl(topp_threshold_kernel, dim3(R), dim3(kThresholdThreads), 0, stream, p);
+    if (e == cudaSuccess) e = launch_pdl(topp_cand_kernel, sg, bs, 0, stream, p);
+    if (e == cudaSuccess) e = launch_pdl(topp_resolve_kernel, dim3(R), dim3(kResolveThreads), kResolveSmem, stream, p);
+  } else {
+    topp_threshold_kernel<<<R, kThresholdThreads, 0, stream>>>(p);  // marks every row empty
+    e = cudaGetLastError();
   }
-  topp_threshold_kernel<<<R, kThresholdThreads, 0, stream>>>(p);
-  if (max_len > 0) {
-    topp_cand_kernel<<<sg, kStreamThreads, 0, stream>>>(p);
-    topp_resolve_kernel<<<R, kResolveThreads, kResolveSmem, stream>>>(p);
-  }
-  const dim3 gg(static_cast<unsigned>(p.nchunk), static_cast<unsigned>(p.c.B * p.c.Hkv));
-  if (G <= 4)
-    topp_write_gather_kernel<4><<<gg, kStreamThreads, e_smem, stream>>>(p, G);
-  else
-    topp_write_gather_kernel<8><<<gg, kStreamThreads, e_smem, stream>>>(p, G);
-  topp_merge_kernel<<<R, kD, 0, stream>>>(p);
+  if (e != cudaSuccess) return e;
+  const dim3 gg(static_cast<unsigned>(p.nsub), static_cast<unsigned>(p.c.B * p.c.Hkv));
+  e = G <= 4 ? launch_pdl(topp_write_gather_kernel<4>, gg, bs, 0, stream, p, G)
+             : launch_pdl(topp_write_gather_kernel<8>, gg, bs, 0, stream, p, G);
+  if (e == cudaSuccess) e = launch_pdl(topp_merge_kernel, dim3(kToppMergeSplit, R), dim3(kD), 0, stream, p);
+  if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
