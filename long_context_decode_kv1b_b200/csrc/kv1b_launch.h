@@ -88,6 +88,7 @@ struct ToppParams {
   float* qdl;
   int32_t* qsq;
   float* s;                  // [R][cap] logits
+  uint16_t* bk;              // [R][cap] mass bucket of each token (kToppBuckets: no mass)
   int32_t* cand;             // [R][cap] threshold-bucket candidates (any order)
   ToppRowState* rows;        // [R]
   unsigned long long* hist;  // [R][kToppBuckets] masses per bucket

@@ -37,30 +37,38 @@ constexpr int kResolveThreads = 1024;
 constexpr int kResolveSmemCand = 12288;  // candidates whose keys and masses the resolve keeps on chip
 constexpr size_t kResolveSmem = static_cast<size_t>(kResolveSmemCand) * 16;
 
-// (ln 2)^k / k!, k = 0..7, each rounded to the nearest fp32 (Taylor coefficients of 2^f).
-__constant__ float kExp2Coef[8] = {0x1p+0f,         0x1.62e43p-1f,   0x1.ebfbep-3f,   0x1.c6b08ep-5f,
-                                   0x1.3b2ab6p-7f,  0x1.5d87fep-10f, 0x1.430912p-13f, 0x1.ffcbfcp-17f};
-
 __device__ __forceinline__ float topp_t(float s, float m) { return __fmul_rn(__fsub_rn(s, m), kL2e); }
 
+// u = trunc(P(f) 2^(32 + n)), n = rint(t), f = t - n, P the degree-7 Taylor polynomial of 2^f with
+// coefficients (ln 2)^k / k! each rounded to the nearest fp32 (Horner, fused multiply-adds); 0 for
+// t < -40.  Branch-free: for t in [-40, 0], n in [-40, 0] converts through the 1.5 * 2^23 rounding
+// constant (exact), the scaling by 2^(32 + n) is exact, and P 2^(32 + n) <= 2^32 (equal only at
+// t = 0, where P(0) = 1), so a 32-bit truncation plus that one case gives the 64-bit value.
 __device__ __forceinline__ uint64_t topp_mass_t(float t) {
-  if (!(t >= -40.0f)) return 0ull;
-  const float n = rintf(t);
-  const float f = __fsub_rn(t, n);
-  float P = kExp2Coef[7];
-  #pragma unroll
-  for (int k = 6; k >= 0; --k) P = __fmaf_rn(P, f, kExp2Coef[k]);
-  const int e = 32 + static_cast<int>(n);                          // in [-8, 32]
-  const float scaled = __fmul_rn(P, __int_as_float((e + 127) << 23)); // exact power-of-two scaling
-  return __float2ull_rz(scaled);
+  const float tc = fmaxf(t, -40.0f);
+  const float r = __fadd_rn(tc, 12582912.0f);  // 1.5 * 2^23 + rint(tc)
+  const float n = __fsub_rn(r, 12582912.0f);
+  const float f = __fsub_rn(tc, n);
+  float P = 0x1.ffcbfcp-17f;                   // (ln 2)^7 / 7!
+  P = __fmaf_rn(P, f, 0x1.430912p-13f);        // (ln 2)^6 / 6!
+  P = __fmaf_rn(P, f, 0x1.5d87fep-10f);        // (ln 2)^5 / 5!
+  P = __fmaf_rn(P, f, 0x1.3b2ab6p-7f);         // (ln 2)^4 / 4!
+  P = __fmaf_rn(P, f, 0x1.c6b08ep-5f);         // (ln 2)^3 / 3!
+  P = __fmaf_rn(P, f, 0x1.ebfbep-3f);          // (ln 2)^2 / 2!
+  P = __fmaf_rn(P, f, 0x1.62e43p-1f);          // ln 2
+  P = __fmaf_rn(P, f, 1.0f);
+  const int ni = __float_as_int(r) - 0x4B400000;                      // rint(tc) as an integer
+  const float scaled = __fmul_rn(P, __int_as_float((ni + 32 + 127) << 23)); // exact power-of-two scaling
+  const uint64_t u = scaled >= 4294967296.0f ? (1ull << 32) : static_cast<uint64_t>(__float2uint_rz(scaled));
+  return t >= -40.0f ? u : 0ull;
 }
 
 // Bucket of t = (s - m) log2 e: floor(-64 t) for t in [-40, 0], at most kToppBuckets - 1 (a
 // non-decreasing function of -t, hence of the key order); kToppBuckets below -40 (no mass there).
 __device__ __forceinline__ int topp_bucket(float t) {
-  if (!(t >= -40.0f)) return kToppBuckets;
-  const int b = static_cast<int>(__fmul_rn(-t, 64.0f));
-  return b < kToppBuckets - 1 ? b : kToppBuckets - 1;
+  // floor(-64 t) for -64 t in [0, 2560]: 2^23 + x rounded toward zero is 2^23 + floor(x)
+  const int b = __float_as_int(__fadd_rz(__fmul_rn(-fmaxf(t, -40.0f), 64.0f), 8388608.0f)) - 0x4B000000;
+  return t >= -40.0f ? (b < kToppBuckets - 1 ? b : kToppBuckets - 1) : kToppBuckets;
 }
 
 __device__ __forceinline__ uint64_t topp_key(float s, int64_t t) {
@@ -161,7 +169,7 @@ __device__ __forceinline__ void build_bq(uint32_t (&bq)[4][2], const uint32_t* p
 // grid (token blocks of kScoreTok, kv-heads, sequences); warp = 64 tokens at a time, up to 4 NG
 // heads as NG groups of 4 operand-column pairs.
 template <int NG>
-__global__ void __launch_bounds__(kStreamThreads) topp_scores_kernel(const ToppParams p, int G) {
+__global__ void __launch_bounds__(kStreamThreads, NG == 1 ? 4 : 2) topp_scores_kernel(const ToppParams p, int G) {
   pdl_wait();
   __shared__ float s_max[kStreamWarps][8];
   const CacheView& c = p.c;
@@ -186,22 +194,27 @@ __global__ void __launch_bounds__(kStreamThreads) topp_scores_kernel(const ToppP
     csq[hg] = hv[hg] ? p.qsq[row0 + ht] : 0;
   }
   float mx[NG];
+  float* srow[NG];  // this lane's output row per head group
   #pragma unroll
-  for (int hg = 0; hg < NG; ++hg) mx[hg] = -INFINITY;
+  for (int hg = 0; hg < NG; ++hg) {
+    mx[hg] = -INFINITY;
+    srow[hg] = p.s + (row0 + (hv[hg] ? 4 * hg + t : 0)) * c.cap;
+  }
   const int64_t head_tok = (static_cast<int64_t>(b) * c.Hkv + kvh) * c.cap;
-  const uint32_t* kw = c.k_bits + head_tok * 4;
+  const uint32_t* kw = c.k_bits + head_tok * 4 + t;
   const float* kn = c.k_norm + head_tok;
   const float* ki = c.k_cinv + head_tok;
-  const int64_t tb0 = static_cast<int64_t>(blockIdx.x) * kScoreTok;
-  const int64_t tend = tb0 + kScoreTok < L ? tb0 + kScoreTok : L;
-  for (int64_t base = tb0 + 64 * warp; base < tend; base += 64 * kStreamWarps) {  // warp-uniform
+  const int tb0 = blockIdx.x * kScoreTok;
+  const int tend = tb0 + kScoreTok < L ? tb0 + kScoreTok : L;
+  for (int base = tb0 + 64 * warp; base < tend; base += 64 * kStreamWarps) {  // warp-uniform
     uint32_t w[8];
     float nc[8];
+    const int nvt = tend - base - g;  // token base + g + 8 i is valid for 8 i < nvt
     #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const int64_t tok = base + g + 8 * i;
-      const bool v = tok < tend;
-      w[i] = v ? __ldg(kw + tok * 4 + t) : 0u;
+      const int tok = base + g + 8 * i;
+      const bool v = 8 * i < nvt;
+      w[i] = v ? __ldg(kw + 4 * tok) : 0u;
       nc[i] = v ? __fmul_rn(__ldg(kn + tok), __ldg(ki + tok)) : 0.0f;
     }
     #pragma unroll
@@ -212,11 +225,11 @@ __global__ void __launch_bounds__(kStreamThreads) topp_scores_kernel(const ToppP
         bits_mma(d, w[2 * kk], w[2 * kk + 1], bq[hg]);
         #pragma unroll
         for (int e = 0; e < 2; ++e) {
-          const int64_t tok = base + 16 * kk + g + 8 * e;
-          if (hv[hg] && tok < tend) {
+          const int i = 2 * kk + e;  // token base + g + 8 i
+          if (hv[hg] && 8 * i < nvt) {
             const float sv =
-                logit_from_ints(d[2 * e] >> 3, d[2 * e + 1] >> 3, csq[hg], cvl[hg], cdl[hg], nc[2 * kk + e], qs);
-            p.s[(row0 + 4 * hg + t) * c.cap + tok] = sv;
+                logit_from_ints(d[2 * e] >> 3, d[2 * e + 1] >> 3, csq[hg], cvl[hg], cdl[hg], nc[i], qs);
+            srow[hg][base + g + 8 * i] = sv;
             mx[hg] = fmaxf(mx[hg], sv);
           }
         }
@@ -261,18 +274,28 @@ __global__ void __launch_bounds__(kStreamThreads) topp_mass_kernel(const ToppPar
   __syncthreads();
   const float m = fkey_inv(p.rows[r].maxkey);
   unsigned long long usum = 0ull;
+  const int nv = static_cast<int>(t1 - tt0);  // valid tokens of this thread (may be <= 0)
+  uint32_t bkw[8];                             // the 16 buckets as 16-bit pairs
   #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    if (tt0 + i < t1) {
+    int bk = kToppBuckets;
+    if (i < nv) {
       const float tt = topp_t(v[i], m);
       const uint64_t u = topp_mass_t(tt);
+      bk = topp_bucket(tt);
       if (u) {
-        const int bk = topp_bucket(tt);
         atomicAdd(&s_lo[bk], static_cast<uint32_t>(u & 0xffffu));
         atomicAdd(&s_hi[bk], static_cast<uint32_t>(u >> 16));
         usum += u;
       }
     }
+    if (i & 1) bkw[i >> 1] |= static_cast<uint32_t>(bk) << 16;
+    else bkw[i >> 1] = static_cast<uint32_t>(bk);
+  }
+  if (nv > 0) {  // whole 32-byte groups stay inside the row (cap % 128 == 0)
+    uint4* bo = reinterpret_cast<uint4*>(p.bk + r * p.c.cap + tt0);
+    bo[0] = make_uint4(bkw[0], bkw[1], bkw[2], bkw[3]);
+    bo[1] = make_uint4(bkw[4], bkw[5], bkw[6], bkw[7]);
   }
   usum = warp_sum(usum);
   if ((threadIdx.x & 31) == 0) s_u[threadIdx.x >> 5] = usum;
@@ -353,14 +376,19 @@ __global__ void __launch_bounds__(kStreamThreads) topp_cand_kernel(const ToppPar
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t t1 = t0 + kToppChunk < L ? t0 + kToppChunk : L;
   const int64_t tt0 = t0 + kTokPerThread * threadIdx.x;
-  float v[16];
-  load16(p.s + r * p.c.cap, tt0, t1, v);
-  const float m = fkey_inv(rs.maxkey);
+  uint32_t bkw[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+  const int nv = static_cast<int>(t1 - tt0);  // valid tokens of this thread (may be <= 0)
+  if (nv > 0) {
+    const uint4* bi = reinterpret_cast<const uint4*>(p.bk + r * p.c.cap + tt0);
+    const uint4 a = bi[0], b = bi[1];
+    bkw[0] = a.x; bkw[1] = a.y; bkw[2] = a.z; bkw[3] = a.w;
+    bkw[4] = b.x; bkw[5] = b.y; bkw[6] = b.z; bkw[7] = b.w;
+  }
   unsigned lo = 0, cmask = 0;
   #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    if (tt0 + i < t1) {
-      const int bk = topp_bucket(topp_t(v[i], m));
+    if (i < nv) {
+      const int bk = static_cast<int>((bkw[i >> 1] >> (16 * (i & 1))) & 0xffffu);
       lo += bk < bstar;
       cmask |= static_cast<unsigned>(bk == bstar) << i;
     }
@@ -532,34 +560,37 @@ __global__ void __launch_bounds__(kStreamThreads, GM <= 4 ? 3 : 2) topp_write_ga
   const int64_t tt0 = t0 + kTok * threadIdx.x;
   // independent global reads first: earlier sub-chunks' counts, row states, this thread's logits
   unsigned before[GM], mask[GM];
-  float4 x4[GM];
+  uint2 bk4[GM];    // this thread's 4 buckets per head (16 bits each)
+  float v[GM][4];   // their logits, loaded where the bucket is at most b*
   float mrow[GM];
+  const int nv = static_cast<int>(t1 - tt0);
   #pragma unroll
   for (int h = 0; h < GM; ++h) {
     before[h] = 0u;
     mask[h] = 0u;
-    x4[h] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    bk4[h] = make_uint2(0xffffffffu, 0xffffffffu);
     mrow[h] = 0.0f;
     if (h < G) {
       const uint32_t* cc = p.sub_cnt + (row0 + h) * p.nsub;
       for (int k = threadIdx.x; k < sub; k += kStreamThreads) before[h] += cc[k];
-      if (tt0 < t1) x4[h] = *reinterpret_cast<const float4*>(p.s + (row0 + h) * c.cap + tt0);  // inside the row
+      if (nv > 0) bk4[h] = *reinterpret_cast<const uint2*>(p.bk + (row0 + h) * c.cap + tt0);  // inside the row
     }
   }
   #pragma unroll
   for (int h = 0; h < GM; ++h) {
-    if (h < G && tt0 < t1) {
+    if (h < G && nv > 0) {
       const ToppRowState& rs = p.rows[row0 + h];
       const int bstar = rs.bstar;  // >= 0: the row is not empty
       const unsigned long long kstar = rs.kstar;
-      const float m = fkey_inv(rs.maxkey);
-      mrow[h] = m;
-      const float v[4] = {x4[h].x, x4[h].y, x4[h].z, x4[h].w};
+      mrow[h] = fkey_inv(rs.maxkey);
+      const float* srow = p.s + (row0 + h) * c.cap + tt0;
       #pragma unroll
       for (int i = 0; i < kTok; ++i) {
-        if (tt0 + i < t1) {
-          const int bk = topp_bucket(topp_t(v[i], m));
-          const bool f = bk < bstar || (bk == bstar && topp_key(v[i], tt0 + i) <= kstar);
+        const int bk = static_cast<int>(((i < 2 ? bk4[h].x : bk4[h].y) >> (16 * (i & 1))) & 0xffffu);
+        v[h][i] = 0.0f;
+        if (i < nv && bk <= bstar) {
+          v[h][i] = srow[i];
+          const bool f = bk < bstar || topp_key(v[h][i], tt0 + i) <= kstar;
           mask[h] |= static_cast<unsigned>(f) << i;
         }
       }
@@ -590,23 +621,21 @@ __global__ void __launch_bounds__(kStreamThreads, GM <= 4 ? 3 : 2) topp_write_ga
     lsum[h] = 0.0f;
     if (h < G) {
       const int sh = 16 * (h & 1);
-      unsigned base = 0, prior = 0, tot = 0;
-      for (int w = 0; w < kW; ++w) {
-        base += s_before[w][h];
-        const unsigned cw = (s_cnt[w][h >> 1] >> sh) & 0xffffu;
-        prior += (w < warp) ? cw : 0u;
-        tot += cw;
-      }
+      // lane w < kW holds warp w's values: chunk base, this warp's prior count, the block total
+      const unsigned bw = lane < kW ? s_before[lane][h] : 0u;
+      const unsigned cw = lane < kW ? (s_cnt[lane][h >> 1] >> sh) & 0xffffu : 0u;
+      const unsigned base = __reduce_add_sync(kFull, bw);
+      const unsigned prior = __reduce_add_sync(kFull, lane < warp ? cw : 0u);
+      const unsigned tot = __reduce_add_sync(kFull, cw);
       if (sub == p.nsub - 1 && threadIdx.x == 0) p.sel_cnt[row0 + h] = static_cast<int32_t>(base + tot);
       const unsigned cnt = __popc(mask[h]);
       unsigned off = base + prior + ((incl[h >> 1] >> sh) & 0xffffu) - cnt;
       int32_t* sel = p.sel_idx + (row0 + h) * c.cap;
-      const float v[4] = {x4[h].x, x4[h].y, x4[h].z, x4[h].w};
       #pragma unroll
       for (int i = 0; i < kTok; ++i) {
         if ((mask[h] >> i) & 1u) {
           sel[off++] = static_cast<int32_t>(tt0 + i);
-          const float e = exp2f(__fmul_rn(__fsub_rn(v[i], mrow[h]), kL2e));
+          const float e = exp2f(__fmul_rn(__fsub_rn(v[h][i], mrow[h]), kL2e));
           s_e[h][kTok * threadIdx.x + i] = e;
           lsum[h] += e;
         }
@@ -731,13 +760,13 @@ __global__ void __launch_bounds__(kStreamThreads, GM <= 4 ? 3 : 2) topp_write_ga
 }
 
 // ---------------------------------------------------------------- 7. merge
-// grid (kToppMergeSplit, rows), 128 threads: block j sums the row's sub-chunk partials
+// grid (M <= kToppMergeSplit, rows), 128 threads: block j sums the row's sub-chunk partials
 // [j n / M, (j + 1) n / M) in order into part2[row][j]; the row's last block to finish (atomic ticket
 // after a fence) sums the M first-level sums in order and writes out = numerator / denominator.
 // Rows with nothing selected give zeros.
 __global__ void __launch_bounds__(kD) topp_merge_kernel(const ToppParams p) {
   pdl_wait();
-  constexpr int M = kToppMergeSplit;
+  const int M = gridDim.x;
   __shared__ bool s_last;
   const int64_t r = blockIdx.y;
   const int j = blockIdx.x;
@@ -765,7 +794,6 @@ __global__ void __launch_bounds__(kD) topp_merge_kernel(const ToppParams p) {
   const float* b2 = p.part2 + r * M * kPartStride;
   num = 0.0f;
   den = 0.0f;
-  #pragma unroll
   for (int k = 0; k < M; ++k) {
     num += __ldcg(b2 + k * kPartStride + 2 + ch);
     den += __ldcg(b2 + k * kPartStride + 1);
@@ -797,7 +825,7 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 struct ToppLayout {
-  size_t planes, qvl, qdl, qsq, s, cand, rows, hist, sub_cnt, part, part2, total, state_bytes;
+  size_t planes, qvl, qdl, qsq, s, bk, cand, rows, hist, sub_cnt, part, part2, total, state_bytes;
 };
 ToppLayout topp_layout(int32_t rows, int32_t cap) {
   const size_t R = static_cast<size_t>(rows), C = static_cast<size_t>(cap);
@@ -809,6 +837,7 @@ ToppLayout topp_layout(int32_t rows, int32_t cap) {
   l.qdl = o;       o += al256(R * 4);
   l.qsq = o;       o += al256(R * 4);
   l.s = o;         o += al256(R * C * 4);
+  l.bk = o;        o += al256(R * C * 2);
   l.cand = o;      o += al256(R * C * 4);
   l.rows = o;      o += al256(R * sizeof(ToppRowState));  // rows, hist and sub_cnt: one memset
   l.hist = o;      o += al256(R * kToppBuckets * 8);
@@ -832,6 +861,7 @@ void kv1b_topp_carve(ToppParams* p, void* ws, int32_t rows, int32_t cap) {
   p->qdl = reinterpret_cast<float*>(w + l.qdl);
   p->qsq = reinterpret_cast<int32_t*>(w + l.qsq);
   p->s = reinterpret_cast<float*>(w + l.s);
+  p->bk = reinterpret_cast<uint16_t*>(w + l.bk);
   p->cand = reinterpret_cast<int32_t*>(w + l.cand);
   p->rows = reinterpret_cast<ToppRowState*>(w + l.rows);
   p->hist = reinterpret_cast<unsigned long long*>(w + l.hist);
@@ -876,7 +906,11 @@ cudaError_t kv1b_launch_topp(const ToppParams& p, int32_t G, int32_t max_len, cu
   const dim3 gg(static_cast<unsigned>(p.nsub), static_cast<unsigned>(p.c.B * p.c.Hkv));
   e = G <= 4 ? launch_pdl(topp_write_gather_kernel<4>, gg, bs, 0, stream, p, G)
              : launch_pdl(topp_write_gather_kernel<8>, gg, bs, 0, stream, p, G);
-  if (e == cudaSuccess) e = launch_pdl(topp_merge_kernel, dim3(kToppMergeSplit, R), dim3(kD), 0, stream, p);
+  // first-level merge blocks per row: one per 16 sub-chunk partials, at most kToppMergeSplit
+  const int nsub_used = (max_len + kToppSub - 1) / kToppSub;
+  int msplit = (nsub_used + 15) / 16;
+  msplit = msplit < 1 ? 1 : (msplit > kToppMergeSplit ? kToppMergeSplit : msplit);
+  if (e == cudaSuccess) e = launch_pdl(topp_merge_kernel, dim3(msplit, R), dim3(kD), 0, stream, p);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }
