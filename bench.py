@@ -184,16 +184,28 @@ def barrier(world: int):
 
 
 # ------------------------------------------------------------------------------------------ ours
-def build_cache(cfg, extra_tokens: int, device):
+def build_cache(cfg, extra_tokens: int, device, keep_exact: bool = False):
+    """The compressed cache of the workload; with keep_exact also the exact bf16 keys / values it
+    was built from ([B, capacity, Hkv, 128] in the workload's dtype, for the exact attention over a
+    Top-p set)."""
+    import torch
+
     import long_context_decode_kv1b_b200 as kv
     from long_context_decode_kv1b_b200 import workloads as wl
 
     cap = (cfg.L + extra_tokens + 127) // 128 * 128
     cache = kv.Cache(cfg.B, cfg.Hkv, cap, seed=cfg.rotation_seed, device=device)
+    Kx = Vx = None
+    if keep_exact:
+        Kx = torch.zeros((cfg.B, cap, cfg.Hkv, 128), dtype=cfg.dtype, device=device)
+        Vx = torch.zeros_like(Kx)
     for start, n in wl.prefill_chunks(cfg):
         K, V = wl.prefill_chunk(cfg, start, n, device)
         cache.append(K, V)
-    return cache
+        if keep_exact:
+            Kx[:, start:start + n] = K
+            Vx[:, start:start + n] = V
+    return cache, Kx, Vx
 
 
 def cpu_baseline(cfg, steps_like: bool):
@@ -244,7 +256,7 @@ def run_ours(args):
     n_alt = 0 if args.no_alt else 5
     extra = W + K + (0 if args.no_e2e else K)
     engine = kv.ATTEND_TENSOR if args.engine == "tensor" else kv.ATTEND_CUDA_CORE
-    cache = build_cache(cfg, extra, dev)
+    cache, Kx, Vx = build_cache(cfg, extra, dev, keep_exact=not args.no_topp)
     nsteps = W + K
     ks, vs, qs = [], [], []
     for i in range(nsteps + (0 if args.no_e2e else K)):
@@ -359,6 +371,26 @@ def run_ours(args):
                 "bytes_rule": "24 B per token x kv-head (scores) + 80 B per selected token x query head (gather)",
                 "kernels": "memset + query prep, scores, mass, threshold, cand, resolve, write_gather, merge (median of 5)"}
         topp["frac"] = topp["achieved_gbs"] / peak
+        # exact attention over the same selected sets with the exact bf16 keys / values (the appended
+        # step tokens are copied in here, outside the timed region)
+        for i in range(cache.lengths[0] - cfg.L):  # every appended step token, in order
+            Kx[:, cfg.L + i] = ks[i][:, 0]
+            Vx[:, cfg.L + i] = vs[i][:, 0]
+        xout = torch.empty_like(tout)
+        for _ in range(3):
+            cache.attend_selected_exact(qs[0], cfg.scale, Kx, Vx, tsel, tcnt, out=xout)
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(5)]
+        for x, y in ev:
+            x.record(stream)
+            cache.attend_selected_exact(qs[0], cfg.scale, Kx, Vx, tsel, tcnt, out=xout)
+            y.record(stream)
+        torch.cuda.synchronize()
+        x_ms = statistics.median(x.elapsed_time(y) for x, y in ev)
+        xbytes = 2 * 128 * Kx.element_size() * int(tcnt.sum().item())
+        topp["exact"] = {"us": x_ms * 1e3, "algorithmic_bytes": xbytes, "achieved_gbs": xbytes / (x_ms * 1e-3) / 1e9,
+                         "frac": xbytes / (x_ms * 1e-3) / 1e9 / peak,
+                         "bytes_rule": "2 x 128 x element size (key + value row) per selected token x query head",
+                         "kernels": "exact_kernel + split merge (median of 5)"}
 
     result = None
     if rank == 0:

@@ -61,7 +61,7 @@ extern "C" {
 #define KV1B_DTYPE_F16 2
 
 /* kv1b_attend flags: which engine forms the probability-weighted sum of values */
-#define KV1B_ATTEND_TENSOR 0     /* default: integer mma.sync (u8 codes x 23-bit fixed-point weights, exact s32
+#define KV1B_ATTEND_TENSOR 0     /* default: integer mma.sync (u8 codes x 32-bit fixed-point weights, exact s32
                                     accumulation) in a persistent kernel, for G in {1, 2, 4}, equal sequence
                                     lengths and an automatic split count; other shapes run the CUDA-core engine */
 #define KV1B_ATTEND_CUDA_CORE 1  /* fp32 FMA on the CUDA cores (split-K grid, any shape) */
@@ -70,6 +70,8 @@ extern "C" {
 #define KV1B_STATUS_NONFINITE 1       /* a K or V element appended was NaN or Inf */
 #define KV1B_STATUS_FP16_SATURATED 2  /* a value group's min or scale left the binary16 range */
 #define KV1B_STATUS_TIMEOUT 4         /* an attend kernel's bounded pipeline wait ran out (results invalid) */
+#define KV1B_STATUS_BAD_INDEX 8       /* kv1b_attend_selected_exact met a selected index outside the valid
+                                         tokens; that entry was skipped */
 
 /*
  * Cache descriptor.  Filled by kv1b_cache_init; treat as opaque except for reading the fields.
@@ -126,7 +128,8 @@ int kv1b_cache_init(kv1b_cache_t* cache, void* dev_buf, size_t bytes, int32_t ba
 int kv1b_encode_append(kv1b_cache_t* cache, const void* k, const void* v, int32_t dtype, int32_t n_new,
                        int64_t stride_b, int64_t stride_t, int64_t stride_h, void* stream);
 
-/* Workspace bytes kv1b_attend (mode 0) or kv1b_attend_topp (mode 1) needs for this cache and
+/* Workspace bytes kv1b_attend (mode 0), kv1b_attend_topp (mode 1) or kv1b_attend_selected_exact
+ * (mode 2) needs for this cache and
  * num_q_heads at any length up to the capacity.  0 on invalid arguments. */
 size_t kv1b_attend_workspace_bytes(const kv1b_cache_t* cache, int32_t num_q_heads, int32_t mode);
 
@@ -170,6 +173,27 @@ int kv1b_attend_noalloc(const kv1b_cache_t* cache, const void* q, int32_t q_dtyp
 int kv1b_attend_topp(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,
                      float p, float* out, int32_t* sel_idx, int32_t* sel_cnt, void* ws, size_t ws_bytes,
                      void* stream);
+
+/* Exact attention over a selected token set ("RaBitQCache", abstract / core idea: the binary x INT4
+ * proxy scores retrieve the tokens -- e.g. kv1b_attend_topp's sel_idx / sel_cnt -- and attention
+ * over them uses the exact keys and values).  For each (b, hq), with S = sel_idx[b][hq][0 ..
+ * sel_cnt[b][hq]) and kv-head kvh = hq / (num_q_heads / num_kv_heads):
+ *   z_t = scale * sum_c q_c k_{b,t,kvh,c},  out[b][hq] = sum_{t in S} softmax(z)_t v_{b,t,kvh}
+ * in fp32 (logits in log2 units, online softmax, fixed-order log-sum-exp merge); zeros when S is
+ * empty.
+ * k, v: the exact keys and values, `kv_dtype` (KV1B_DTYPE_*); element (b, t, h, c) at offset
+ *   b*stride_b + t*stride_t + h*stride_h + c elements (channels contiguous); device memory or host
+ *   memory the device can address (mapped pinned / managed).  Base addresses 16-byte aligned and
+ *   strides multiples of 8 elements; kv_tokens = tokens per sequence the arrays hold.
+ * q: [batch][num_q_heads][128] contiguous, `q_dtype`, 16-byte aligned.
+ * sel_idx: i32 [batch][num_q_heads][capacity]; sel_cnt: i32 [batch][num_q_heads] (<= capacity).
+ *   An index outside [0, min(length[b], kv_tokens)) is skipped and sets KV1B_STATUS_BAD_INDEX.
+ * out: f32 [batch][num_q_heads][128].  ws: kv1b_attend_workspace_bytes(.., 2) bytes, 256-aligned.
+ * The caller owns every buffer; the call only launches work on `stream`. */
+int kv1b_attend_selected_exact(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads,
+                               float scale, const void* k, const void* v, int32_t kv_dtype, int64_t kv_tokens,
+                               int64_t stride_b, int64_t stride_t, int64_t stride_h, const int32_t* sel_idx,
+                               const int32_t* sel_cnt, float* out, void* ws, size_t ws_bytes, void* stream);
 
 /* Test hook for the query preparation step: planes u32 [batch][num_q_heads][4][4] (plane j,
  * word w, bit i = bit j of the code of rotated channel 32w+i), vl / delta f32 [batch][num_q_heads]

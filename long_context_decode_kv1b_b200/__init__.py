@@ -25,7 +25,8 @@ ERRORS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "capacity", -4
 
 # symbols declared in include/kv1b.h
 SYMBOLS = ("kv1b_cache_bytes", "kv1b_cache_init", "kv1b_encode_append", "kv1b_attend_workspace_bytes",
-           "kv1b_attend", "kv1b_attend_noalloc", "kv1b_attend_topp", "kv1b_query_prep", "kv1b_scores",
+           "kv1b_attend", "kv1b_attend_noalloc", "kv1b_attend_topp", "kv1b_attend_selected_exact",
+           "kv1b_query_prep", "kv1b_scores",
            "kv1b_read_status", "kv1b_status_string", "kv1b_version")
 
 
@@ -66,6 +67,8 @@ def lib() -> ctypes.CDLL:
             "kv1b_attend_workspace_bytes": (sz, [D, i32, i32]),
             "kv1b_attend": (ctypes.c_int, [D, P, i32, i32, f32, P, P, sz, i32, i32, P]),
             "kv1b_attend_topp": (ctypes.c_int, [D, P, i32, i32, f32, f32, P, P, P, P, sz, P]),
+            "kv1b_attend_selected_exact": (ctypes.c_int, [D, P, i32, i32, f32, P, P, i32, i64, i64, i64, i64, P, P,
+                                                          P, P, sz, P]),
             "kv1b_query_prep": (ctypes.c_int, [D, P, i32, i32, P, P, P, P, P]),
             "kv1b_scores": (ctypes.c_int, [D, P, i32, i32, f32, P, P, P, P]),
             "kv1b_read_status": (ctypes.c_int, [D, P, P]),
@@ -203,6 +206,31 @@ class Cache:
                                       _ptr(out), _ptr(sel), _ptr(cnt), _ptr(ws), ws.numel(), _stream(stream)),
                "kv1b_attend_topp")
         return out, sel, cnt
+
+    def attend_selected_exact(self, q: torch.Tensor, scale: float, k: torch.Tensor, v: torch.Tensor,
+                              sel: torch.Tensor, cnt: torch.Tensor, out=None, stream=None) -> torch.Tensor:
+        """Exact attention over selected tokens (e.g. attend_topp's sel / cnt) with the caller's exact keys
+        and values k, v: [batch, tokens, num_kv_heads, 128], equal strides and dtype, unit channel stride
+        (device memory, or host memory the device can address).  Returns fp32 [batch, num_q_heads, 128]."""
+        B, Hq, D = q.shape
+        if not q.is_contiguous():
+            raise ValueError("q must be contiguous")
+        if k.shape != v.shape or k.stride() != v.stride() or k.dtype != v.dtype:
+            raise ValueError("k and v must have equal shapes, strides and dtypes")
+        if k.dim() != 4 or (k.shape[0], k.shape[2], k.shape[3]) != (self.batch, self.num_kv_heads, HEAD_DIM) \
+                or k.stride(3) != 1:
+            raise ValueError("expected k, v of [batch, tokens, num_kv_heads, 128] with unit channel stride")
+        _check_buf(sel, (B, Hq, self.capacity), torch.int32, "sel")
+        _check_buf(cnt, (B, Hq), torch.int32, "cnt")
+        if out is None:
+            out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+        _check_buf(out, (B, Hq, D), torch.float32, "out")
+        ws = self.workspace(Hq, 2)
+        _check(lib().kv1b_attend_selected_exact(ctypes.byref(self.desc), _ptr(q), _dtype_code(q), Hq, float(scale),
+                                                _ptr(k), _ptr(v), _dtype_code(k), k.shape[1], k.stride(0),
+                                                k.stride(1), k.stride(2), _ptr(sel), _ptr(cnt), _ptr(out), _ptr(ws),
+                                                ws.numel(), _stream(stream)), "kv1b_attend_selected_exact")
+        return out
 
     def query_prep(self, q: torch.Tensor, stream=None) -> dict:
         B, Hq, _ = q.shape

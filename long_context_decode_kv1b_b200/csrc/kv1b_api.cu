@@ -206,6 +206,7 @@ size_t kv1b_attend_workspace_bytes(const kv1b_cache_t* cache, int32_t num_q_head
   const size_t rows = static_cast<size_t>(cache->batch) * num_q_heads;
   if (mode == 0) return ws_counters_offset(cache, num_q_heads) + align_up(ws_counter_bytes(cache));
   if (mode == 1) return align_up(kv1b_topp_workspace_bytes(static_cast<int32_t>(rows), cache->capacity));
+  if (mode == 2) return align_up(kv1b_exact_workspace_bytes(static_cast<int32_t>(rows), cache->capacity));
   return 0;
 }
 
@@ -285,6 +286,45 @@ int kv1b_attend_topp(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, 
   kv1b_topp_carve(&tp, ws, cache->batch * num_q_heads, cache->capacity);
   return cuda_status(
       kv1b_launch_topp(tp, G, static_cast<int32_t>(max_length(cache)), static_cast<cudaStream_t>(stream)));
+}
+
+int kv1b_attend_selected_exact(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads,
+                               float scale, const void* k, const void* v, int32_t kv_dtype, int64_t kv_tokens,
+                               int64_t stride_b, int64_t stride_t, int64_t stride_h, const int32_t* sel_idx,
+                               const int32_t* sel_cnt, float* out, void* ws, size_t ws_bytes, void* stream) {
+  if (!cache_ok(cache) || !q || !k || !v || !sel_idx || !sel_cnt || !out || !ws || !dtype_ok(q_dtype) ||
+      !dtype_ok(kv_dtype))
+    return KV1B_ERR_INVALID_ARG;
+  const int hc = heads_check(cache, num_q_heads);
+  if (hc != KV1B_OK) return hc;
+  if (!(scale == scale) || kv_tokens < 0 || stride_b < 0 || stride_t < 0 || stride_h < 0) return KV1B_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(ws, kAlign) || stride_b % 8 != 0 ||
+      stride_t % 8 != 0 || stride_h % 8 != 0)
+    return KV1B_ERR_MISALIGNED;
+  if (ws_bytes < kv1b_attend_workspace_bytes(cache, num_q_heads, 2)) return KV1B_ERR_WORKSPACE;
+  kv1b::ExactParams p;
+  memset(&p, 0, sizeof(p));
+  p.q = q;
+  p.q_dtype = q_dtype;
+  p.Hq = num_q_heads;
+  p.Hkv = cache->num_kv_heads;
+  p.qscale = scale * 1.4426950408889634f;
+  p.k = k;
+  p.v = v;
+  p.kv_dtype = kv_dtype;
+  p.sb = stride_b;
+  p.st = stride_t;
+  p.sh = stride_h;
+  p.kv_tokens = kv_tokens;
+  p.sel = sel_idx;
+  p.cnt = sel_cnt;
+  p.cap = cache->capacity;
+  p.out = out;
+  p.status = cache->d_status;
+  for (int b = 0; b < cache->batch; ++b) p.len[b] = static_cast<int32_t>(cache->h_lengths[b]);
+  kv1b_exact_carve(&p, ws, cache->batch * num_q_heads);
+  return cuda_status(
+      kv1b_launch_exact(p, cache->batch * num_q_heads, num_sms(), static_cast<cudaStream_t>(stream)));
 }
 
 int kv1b_query_prep(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, uint32_t* planes,

@@ -382,6 +382,13 @@ cudaError_t kv1b_launch_attend(const AttendParams& p, int32_t G, int32_t engine,
   return cudaGetLastError();
 }
 
+// Log-sum-exp merge of nsplit partial rows (m in log2 units, l, o[128]) per row: [rows][nsplit][2 + 128].
+cudaError_t kv1b_launch_merge(const float* part, float* out, int32_t rows, int32_t nsplit, cudaStream_t stream) {
+  if (nsplit < 1 || nsplit > 1024 || rows < 1) return cudaErrorInvalidValue;
+  merge_kernel<<<rows, 128, 0, stream>>>(part, out, nsplit);
+  return cudaGetLastError();
+}
+
 cudaError_t kv1b_launch_query_prep(const CacheView& c, const void* q, int32_t q_dtype, int32_t Hq, uint32_t* planes,
                                    float* vl, float* delta, int32_t* sq, cudaStream_t stream) {
   query_prep_kernel<<<c.B * Hq, 32, 0, stream>>>(c, q, q_dtype, Hq, planes, vl, delta, sq);

@@ -105,6 +105,28 @@ struct ToppParams {
 
 constexpr int kPartStride = 2 + 128;
 
+// exact attention over a selected token set (kv1b_exact.cu)
+constexpr int kExactItem = 256;  // selected entries per work item
+struct ExactParams {
+  const void* q;
+  int32_t q_dtype;
+  int32_t Hq, Hkv;
+  float qscale;              // scale * log2(e)
+  const void* k;             // exact keys / values: element (b, t, h, c) at b sb + t st + h sh + c
+  const void* v;
+  int32_t kv_dtype;
+  int64_t sb, st, sh;
+  int64_t kv_tokens;         // tokens per sequence the key / value arrays hold
+  const int32_t* sel;        // [R][cap] selected indices
+  const int32_t* cnt;        // [R]
+  int32_t cap;
+  int32_t* item_off;         // [R + 1] first work item of each row
+  float* part;               // [items][kPartStride]
+  float* out;                // [R][128]
+  int32_t* status;
+  int32_t len[KV1B_MAX_BATCH];
+};
+
 // persistent attend on the integer tensor cores (kv1b_attend_ws.cu)
 struct alignas(64) AttendWsParams {
   CUtensorMap codes_map;  // v_codes as [tiles][128 channels][128 4-bit tokens], 16U4_ALIGN16B, 128B swizzle
@@ -138,6 +160,10 @@ cudaError_t kv1b_launch_topp(const kv1b::ToppParams& p, int32_t G, int32_t max_l
 size_t kv1b_topp_workspace_bytes(int32_t rows, int32_t cap);
 void kv1b_topp_carve(kv1b::ToppParams* p, void* ws, int32_t rows, int32_t cap);
 int kv1b_pick_splits(int32_t B, int32_t Hkv, int64_t max_len, int num_sms);
+cudaError_t kv1b_launch_merge(const float* part, float* out, int32_t rows, int32_t nsplit, cudaStream_t stream);
+size_t kv1b_exact_workspace_bytes(int32_t rows, int32_t cap);
+void kv1b_exact_carve(kv1b::ExactParams* p, void* ws, int32_t rows);
+cudaError_t kv1b_launch_exact(const kv1b::ExactParams& p, int32_t rows, int32_t num_sms, cudaStream_t stream);
 bool kv1b_ws_supported(int32_t G);
 void kv1b_ws_plan(int32_t B, int32_t Hkv, int32_t G, int64_t L, int num_sms, int64_t* T, int64_t* Lt, int* ncta,
                   int* max_pieces);

@@ -62,6 +62,7 @@ def lib() -> ctypes.CDLL:
             "ref_topp_weight": (u64, [f32, f32]),
             "ref_topp_select": (i64, [P, i64, f32, P]),
             "ref_attend_topp_head": (i64, [P, P, P, P, P, i64, P, P, f32, f32, ctypes.c_int, P, P]),
+            "ref_attend_exact_selected": (ctypes.c_int, [P, P, P, i64, ctypes.c_int, P, i64, f32, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -244,3 +245,20 @@ def attend_topp(enc: dict, q, sgn, scale: float, p: float):
     if n < 0:
         raise ValueError("invalid Top-p arguments")
     return sel[:n].copy(), out
+
+
+def attend_exact_selected(q, K, V, sel, scale: float) -> np.ndarray:
+    """Exact attention of one query head over the selected tokens: q [d]; K, V [L, d] (exact
+    values, converted to fp32 without rounding from bf16 / fp16 / fp32); sel: indices into [0, L).
+    Returns fp64 [d] (zeros for an empty selection)."""
+    q = _f32(q)
+    K = _f32(K)
+    V = _f32(V)
+    L, d = K.shape
+    sel = np.ascontiguousarray(np.asarray(sel, dtype=np.int64).reshape(-1))
+    out = np.empty(d, np.float64)
+    rc = lib().ref_attend_exact_selected(_p(q), _p(K), _p(V), L, d, _p(sel) if sel.size else None, sel.size,
+                                         float(scale), _p(out))
+    if rc != 0:
+        raise ValueError("selected index out of range")
+    return out

@@ -425,4 +425,32 @@ int64_t ref_attend_topp_head(const uint32_t* bits, const float* norm, const floa
   return n;
 }
 
+/* RaBitQCache abstract / core idea: after the proxy scores pick the token set, attention is taken
+ * over that set alone with the exact keys and values (sparse attention).  Plain fp64 softmax. */
+int ref_attend_exact_selected(const float* q, const float* K, const float* V, int64_t L, int d, const int64_t* sel,
+                              int64_t n, float scale, double* out) {
+  if (d <= 0) return -1;
+  for (int c = 0; c < d; ++c) out[c] = 0.0;
+  for (int64_t i = 0; i < n; ++i)
+    if (sel[i] < 0 || sel[i] >= L) return -1;
+  if (n <= 0) return 0;
+  std::vector<double> z(n);
+  for (int64_t i = 0; i < n; ++i) {
+    double dot = 0.0;
+    for (int c = 0; c < d; ++c) dot += static_cast<double>(q[c]) * static_cast<double>(K[sel[i] * d + c]);
+    z[i] = static_cast<double>(scale) * dot;
+  }
+  double m = z[0];
+  for (int64_t i = 1; i < n; ++i) m = std::max(m, z[i]);
+  double l = 0.0;
+  std::vector<double> acc(d, 0.0);
+  for (int64_t i = 0; i < n; ++i) {
+    const double e = std::exp(z[i] - m);
+    l += e;
+    for (int c = 0; c < d; ++c) acc[c] += e * static_cast<double>(V[sel[i] * d + c]);
+  }
+  for (int c = 0; c < d; ++c) out[c] = acc[c] / l;
+  return 0;
+}
+
 }  // extern "C"

@@ -109,6 +109,15 @@ int64_t ref_attend_topp_head(const uint32_t* bits, const float* norm, const floa
                              const uint32_t* sm, int64_t L, const float* q, const float* signs, float scale,
                              float p, int d, int64_t* sel, double* out);
 
+/* Exact attention over a selected token set (RaBitQCache, abstract / core idea: the proxy scores
+ * retrieve the tokens, attention over them is then sparse attention with the exact keys and
+ * values).  q: [d]; K, V: [L][d] as fp32 (the exact values of the caller's keys and values);
+ * sel: n indices into [0, L) (any order, no repeats).  z_t = scale * sum_c q_c K_tc in fp64;
+ * out = sum_t softmax(z)_t V_t in fp64 over t in sel; zeros when n == 0.  Returns 0, or -1 when an
+ * index is out of range or d is not positive. */
+int ref_attend_exact_selected(const float* q, const float* K, const float* V, int64_t L, int d, const int64_t* sel,
+                              int64_t n, float scale, double* out);
+
 #ifdef __cplusplus
 }
 #endif

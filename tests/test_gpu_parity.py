@@ -270,3 +270,86 @@ def test_topp_group_sizes(G, qdt):
     q = torch.randn((B, Hkv * G, 128), device=DEV, generator=torch.Generator(device=DEV).manual_seed(5)).to(qdt)
     for p in (0.3, 0.95):
         topp_check(cache, host, q, 0.4, p, G, oracle.signs(13))
+
+
+# ------------------------------------------------------------------ exact attention over a selected set
+def cache_with_exact(B, Hkv, L, dtype, seed, data_seed):
+    """A compressed cache plus the exact keys / values it was built from ([B, L, Hkv, 128] on the GPU)."""
+    cap = (L + 127) // 128 * 128
+    cache = kv.Cache(B, Hkv, cap, seed=seed)
+    g = torch.Generator(device=DEV).manual_seed(data_seed)
+    K, V = rand_kv(g, B, L, Hkv, dtype)
+    cache.append(K, V)
+    return cache, K, V
+
+
+def exact_check(cache, q, scale, K, V, sel, cnt, G, where=""):
+    out = cache.attend_selected_exact(q, scale, K, V, sel, cnt)
+    torch.cuda.synchronize()
+    qn, Kn, Vn = to_np32(q), to_np32(K), to_np32(V)
+    B, Hq, _ = qn.shape
+    L = min(cache.lengths[0], K.shape[1])
+    for b in range(B):
+        for hq in range(Hq):
+            n = int(cnt[b, hq].item())
+            s = sel[b, hq, :n].cpu().numpy().astype(np.int64)
+            s = s[(s >= 0) & (s < L)]  # out-of-range entries are skipped
+            ref = oracle.attend_exact_selected(qn[b, hq], Kn[b, :, hq // G], Vn[b, :, hq // G], s, scale)
+            if s.size == 0:
+                assert torch.count_nonzero(out[b, hq]).item() == 0, f"{where} b{b} hq{hq}: empty set"
+            else:
+                assert_rows_close(out[b, hq].cpu().numpy(), ref, where=f"{where} b{b} hq{hq}")
+    return out
+
+
+@pytest.mark.parametrize("p", [0.5, 0.95])
+def test_exact_over_topp_selection(p):
+    B, Hkv, G, L = 2, 2, 4, 5000
+    cache, K, V = cache_with_exact(B, Hkv, L, torch.bfloat16, seed=31, data_seed=4)
+    q = torch.randn((B, Hkv * G, 128), device=DEV, generator=torch.Generator(device=DEV).manual_seed(6))
+    q = q.to(torch.bfloat16)
+    _, sel, cnt = cache.attend_topp(q, 0.3, p)
+    exact_check(cache, q, 0.3, K, V, sel, cnt, G, where=f"p{p}")
+    assert cache.status() == 0
+
+
+def test_exact_hand_made_sets_and_bad_indices():
+    B, Hkv, G, L = 1, 1, 4, 700
+    cache, K, V = cache_with_exact(B, Hkv, L, torch.bfloat16, seed=2, data_seed=9)
+    cap = cache.capacity
+    q = torch.randn((B, G, 128), device=DEV, generator=torch.Generator(device=DEV).manual_seed(1))
+    sel = torch.zeros((B, G, cap), dtype=torch.int32, device=DEV)
+    cnt = torch.zeros((B, G), dtype=torch.int32, device=DEV)
+    # head 0: empty; head 1: one token; head 2: every token; head 3: random subset
+    sel[0, 1, 0] = 345
+    cnt[0, 1] = 1
+    sel[0, 2, :L] = torch.arange(L, dtype=torch.int32, device=DEV)
+    cnt[0, 2] = L
+    sub = torch.randperm(L, generator=torch.Generator().manual_seed(3))[:123].sort().values.to(torch.int32)
+    sel[0, 3, :123] = sub.to(DEV)
+    cnt[0, 3] = 123
+    exact_check(cache, q, 0.2, K, V, sel, cnt, G, where="hand")
+    assert cache.status() == 0
+    # indices past the sequence are skipped and flagged
+    sel[0, 1, 1] = L + 5
+    sel[0, 1, 2] = -3
+    cnt[0, 1] = 3
+    exact_check(cache, q, 0.2, K, V, sel, cnt, G, where="bad")
+    assert cache.status() & 8
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.float16])
+def test_exact_kv_dtypes_and_strides(dtype):
+    # keys / values as column slices of wider rows (token stride 2 x 2 x 128 elements, head stride 256)
+    B, Hkv, G, L = 2, 2, 2, 1800
+    cap = (L + 127) // 128 * 128
+    cache = kv.Cache(B, Hkv, cap, seed=5)
+    g = torch.Generator(device=DEV).manual_seed(12)
+    wide = torch.randn((B, L, Hkv, 2, 128), generator=g, device=DEV).to(dtype)
+    K, V = wide[:, :, :, 0, :], wide[:, :, :, 1, :]  # equal strides (L: 512, head: 256, channel: 1)
+    Kc, Vc = K.contiguous(), V.contiguous()
+    cache.append(Kc, Vc)
+    q = torch.randn((B, Hkv * G, 128), device=DEV, generator=torch.Generator(device=DEV).manual_seed(2))
+    _, sel, cnt = cache.attend_topp(q, 0.25, 0.8)
+    exact_check(cache, q, 0.25, K, V, sel, cnt, G, where=f"{dtype} strided")
+    exact_check(cache, q, 0.25, Kc, Vc, sel, cnt, G, where=f"{dtype} contiguous")

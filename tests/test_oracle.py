@@ -496,3 +496,70 @@ def test_attend_topp_matches_softmax_over_selected():
     sel1, out1 = oracle.attend_topp(enc, q, D, sc, 1.0)
     if len(sel1) == 200:
         assert np.allclose(out1, oracle.attend(enc, q, D, sc), rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------------ exact attention over a selected set
+# RaBitQCache (abstract / core idea): the proxy scores pick the tokens, attention over them uses the
+# exact keys and values.  Pinned by closed forms, invariants and a worked two-token example.
+def _exact_inputs(L=40, d=128, seed=3):
+    rng = np.random.default_rng(seed)
+    return (rng.standard_normal(d).astype(np.float32), rng.standard_normal((L, d)).astype(np.float32),
+            rng.standard_normal((L, d)).astype(np.float32))
+
+
+def test_exact_selected_single_token_and_empty():
+    q, K, V = _exact_inputs()
+    for t in (0, 17, 39):
+        assert np.array_equal(oracle.attend_exact_selected(q, K, V, [t], 0.3), V[t].astype(np.float64))
+    assert np.count_nonzero(oracle.attend_exact_selected(q, K, V, [], 0.3)) == 0
+    with pytest.raises(ValueError):
+        oracle.attend_exact_selected(q, K, V, [40], 0.3)
+    with pytest.raises(ValueError):
+        oracle.attend_exact_selected(q, K, V, [-1], 0.3)
+
+
+def test_exact_selected_equal_logits_give_the_mean():
+    q, K, V = _exact_inputs()
+    sel = [2, 5, 11, 30]
+    out = oracle.attend_exact_selected(np.zeros_like(q), K, V, sel, 0.3)  # q = 0: every logit is 0
+    ref = V[sel].astype(np.float64).sum(0) / len(sel)
+    assert np.allclose(out, ref, rtol=1e-13, atol=1e-15)
+
+
+def test_exact_selected_two_token_worked_example():
+    # q = e_0, k_a = 0, k_b = c e_0 with scale * c = ln 3 (up to the fp32 rounding of c): weights 1/4, 3/4
+    d, scale = 128, 0.5
+    q = np.zeros(d, np.float32)
+    q[0] = 1.0
+    K = np.zeros((2, d), np.float32)
+    K[1, 0] = np.float32(2.0 * math.log(3.0))
+    V = np.zeros((2, d), np.float32)
+    V[0, :] = 4.0
+    V[1, :] = -8.0
+    out = oracle.attend_exact_selected(q, K, V, [0, 1], scale)
+    assert np.allclose(out, 0.25 * 4.0 + 0.75 * -8.0, rtol=1e-6)  # = -5
+
+
+def test_exact_selected_invariants():
+    q, K, V = _exact_inputs(seed=8)
+    sel = [1, 4, 9, 16, 25, 36]
+    out = oracle.attend_exact_selected(q, K, V, sel, 0.2)
+    # the order of the selected list does not matter
+    assert np.allclose(oracle.attend_exact_selected(q, K, V, sel[::-1], 0.2), out, rtol=1e-13, atol=1e-15)
+    # a convex combination of the selected values
+    assert np.all(out <= V[sel].max(0) + 1e-12) and np.all(out >= V[sel].min(0) - 1e-12)
+    # adding a constant vector to every value adds it to the output; scaling the values scales it
+    c = np.linspace(-3, 3, 128).astype(np.float32)
+    assert np.allclose(oracle.attend_exact_selected(q, K, V + c, sel, 0.2), out + c, rtol=1e-6, atol=1e-6)
+    assert np.allclose(oracle.attend_exact_selected(q, K, 2 * V, sel, 0.2), 2 * out, rtol=1e-13, atol=1e-15)
+    # tokens outside the set do not matter
+    V2 = V.copy()
+    V2[0] = 1e6
+    K2 = K.copy()
+    K2[0] = 1e3
+    assert np.array_equal(oracle.attend_exact_selected(q, K2, V2, sel, 0.2), out)
+    # a dominant logit takes the whole mass
+    K3 = K.copy()
+    K3[9] = 50.0 * q / np.linalg.norm(q)
+    out3 = oracle.attend_exact_selected(q, K3, V, sel, 1.0)
+    assert np.allclose(out3, V[9], rtol=1e-9, atol=1e-9)
