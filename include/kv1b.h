@@ -66,6 +66,10 @@ extern "C" {
                                     lengths and an automatic split count; other shapes run the CUDA-core engine */
 #define KV1B_ATTEND_CUDA_CORE 1  /* fp32 FMA on the CUDA cores (split-K grid, any shape) */
 
+/* kv1b_attend_select modes */
+#define KV1B_SELECT_TOPP 0  /* smallest set reaching a fraction p of the estimated attention mass */
+#define KV1B_SELECT_TOPK 1  /* a fixed budget of k tokens */
+
 /* status word bits (kv1b_read_status) */
 #define KV1B_STATUS_NONFINITE 1       /* a K or V element appended was NaN or Inf */
 #define KV1B_STATUS_FP16_SATURATED 2  /* a value group's min or scale left the binary16 range */
@@ -173,6 +177,23 @@ int kv1b_attend_noalloc(const kv1b_cache_t* cache, const void* q, int32_t q_dtyp
 int kv1b_attend_topp(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,
                      float p, float* out, int32_t* sel_idx, int32_t* sel_cnt, void* ws, size_t ws_bytes,
                      void* stream);
+
+/* Top-p or Top-k selection plus an always-kept window, then attention over the set.
+ * (RaBitQCache abstract: adaptive Top-p, contrasted with a fixed Top-k budget; H1IB-KV article part 2
+ * item 1: a high-precision layer for important tokens, read here as the first `sink` and the last
+ * `recent` tokens of each sequence.)  Per (b, hq), with W = {t < sink} U {t >= length[b] - recent}
+ * and the order (s desc, index asc) of the other tokens:
+ *   KV1B_SELECT_TOPP: masses u_t as kv1b_attend_topp (m = max over all tokens), T = ceil(p U) in
+ *     fp64 over all tokens, clamped to [1, U]; the set is W plus the shortest prefix of the other
+ *     tokens whose mass reaches T - mass(W) (nothing when W already reaches T);
+ *   KV1B_SELECT_TOPK: W plus the first min(k, number of other tokens) of them.
+ * Outputs and workspace as kv1b_attend_topp (sel_idx ascending, sel_cnt, out = the softmax over the
+ * set of the estimated logits with the 4-bit values; ws >= kv1b_attend_workspace_bytes(.., 1)).
+ * mode must be one of the two; p in (0, 1] for Top-p; k >= 0 for Top-k; sink, recent >= 0.
+ * kv1b_attend_topp(.., p, ..) is kv1b_attend_select(.., KV1B_SELECT_TOPP, p, 0, 0, 0, ..). */
+int kv1b_attend_select(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,
+                       int32_t mode, float p, int32_t k, int32_t sink, int32_t recent, float* out, int32_t* sel_idx,
+                       int32_t* sel_cnt, void* ws, size_t ws_bytes, void* stream);
 
 /* Exact attention over a selected token set ("RaBitQCache", abstract / core idea: the binary x INT4
  * proxy scores retrieve the tokens -- e.g. kv1b_attend_topp's sel_idx / sel_cnt -- and attention

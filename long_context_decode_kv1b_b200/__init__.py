@@ -25,7 +25,8 @@ ERRORS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "capacity", -4
 
 # symbols declared in include/kv1b.h
 SYMBOLS = ("kv1b_cache_bytes", "kv1b_cache_init", "kv1b_encode_append", "kv1b_attend_workspace_bytes",
-           "kv1b_attend", "kv1b_attend_noalloc", "kv1b_attend_topp", "kv1b_attend_selected_exact",
+           "kv1b_attend", "kv1b_attend_noalloc", "kv1b_attend_topp", "kv1b_attend_select",
+           "kv1b_attend_selected_exact",
            "kv1b_query_prep", "kv1b_scores",
            "kv1b_read_status", "kv1b_status_string", "kv1b_version")
 
@@ -67,6 +68,7 @@ def lib() -> ctypes.CDLL:
             "kv1b_attend_workspace_bytes": (sz, [D, i32, i32]),
             "kv1b_attend": (ctypes.c_int, [D, P, i32, i32, f32, P, P, sz, i32, i32, P]),
             "kv1b_attend_topp": (ctypes.c_int, [D, P, i32, i32, f32, f32, P, P, P, P, sz, P]),
+            "kv1b_attend_select": (ctypes.c_int, [D, P, i32, i32, f32, i32, f32, i32, i32, i32, P, P, P, P, sz, P]),
             "kv1b_attend_selected_exact": (ctypes.c_int, [D, P, i32, i32, f32, P, P, i32, i64, i64, i64, i64, P, P,
                                                           P, P, sz, P]),
             "kv1b_query_prep": (ctypes.c_int, [D, P, i32, i32, P, P, P, P, P]),
@@ -110,6 +112,9 @@ def _stream(stream=None) -> ctypes.c_void_p:
 
 def _ptr(t) -> ctypes.c_void_p:
     return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+SELECT_TOPP, SELECT_TOPK = 0, 1
 
 
 class Cache:
@@ -205,6 +210,27 @@ class Cache:
         _check(lib().kv1b_attend_topp(ctypes.byref(self.desc), _ptr(q), _dtype_code(q), Hq, float(scale), float(p),
                                       _ptr(out), _ptr(sel), _ptr(cnt), _ptr(ws), ws.numel(), _stream(stream)),
                "kv1b_attend_topp")
+        return out, sel, cnt
+
+    def attend_select(self, q: torch.Tensor, scale: float, mode: int, p: float = 1.0, k: int = 0, sink: int = 0,
+                      recent: int = 0, out=None, sel=None, cnt=None, stream=None):
+        """Top-p (mode SELECT_TOPP, fraction p) or Top-k (SELECT_TOPK, budget k) selection plus the
+        always-kept first `sink` / last `recent` tokens, then attention over the set.  Returns
+        (out fp32 [B, Hq, 128], sel_idx int32 [B, Hq, capacity], sel_cnt int32 [B, Hq])."""
+        B, Hq, D = q.shape
+        if out is None:
+            out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+        if sel is None:
+            sel = torch.empty((B, Hq, self.capacity), dtype=torch.int32, device=q.device)
+        if cnt is None:
+            cnt = torch.empty((B, Hq), dtype=torch.int32, device=q.device)
+        _check_buf(out, (B, Hq, D), torch.float32, "out")
+        _check_buf(sel, (B, Hq, self.capacity), torch.int32, "sel")
+        _check_buf(cnt, (B, Hq), torch.int32, "cnt")
+        ws = self.workspace(Hq, 1)
+        _check(lib().kv1b_attend_select(ctypes.byref(self.desc), _ptr(q), _dtype_code(q), Hq, float(scale), int(mode),
+                                        float(p), int(k), int(sink), int(recent), _ptr(out), _ptr(sel), _ptr(cnt),
+                                        _ptr(ws), ws.numel(), _stream(stream)), "kv1b_attend_select")
         return out, sel, cnt
 
     def attend_selected_exact(self, q: torch.Tensor, scale: float, k: torch.Tensor, v: torch.Tensor,

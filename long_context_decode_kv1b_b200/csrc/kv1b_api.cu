@@ -261,13 +261,16 @@ int kv1b_attend(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32
   return cuda_status(kv1b_launch_attend(p, G, flags, static_cast<int32_t>(maxlen), static_cast<cudaStream_t>(stream)));
 }
 
-int kv1b_attend_topp(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,
-                     float p, float* out, int32_t* sel_idx, int32_t* sel_cnt, void* ws, size_t ws_bytes,
-                     void* stream) {
+int kv1b_attend_select(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,
+                       int32_t mode, float p, int32_t k, int32_t sink, int32_t recent, float* out, int32_t* sel_idx,
+                       int32_t* sel_cnt, void* ws, size_t ws_bytes, void* stream) {
   if (!cache_ok(cache) || !q || !out || !sel_idx || !sel_cnt || !ws || !dtype_ok(q_dtype)) return KV1B_ERR_INVALID_ARG;
   const int hc = heads_check(cache, num_q_heads);
   if (hc != KV1B_OK) return hc;
-  if (!(p > 0.0f && p <= 1.0f) || !(scale == scale)) return KV1B_ERR_INVALID_ARG;
+  if (mode != KV1B_SELECT_TOPP && mode != KV1B_SELECT_TOPK) return KV1B_ERR_INVALID_ARG;
+  if (mode == KV1B_SELECT_TOPP && !(p > 0.0f && p <= 1.0f)) return KV1B_ERR_INVALID_ARG;
+  if (mode == KV1B_SELECT_TOPK && k < 0) return KV1B_ERR_INVALID_ARG;
+  if (sink < 0 || recent < 0 || !(scale == scale)) return KV1B_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(ws, kAlign)) return KV1B_ERR_MISALIGNED;
   if (ws_bytes < kv1b_attend_workspace_bytes(cache, num_q_heads, 1)) return KV1B_ERR_WORKSPACE;
   const int G = num_q_heads / cache->num_kv_heads;
@@ -277,8 +280,12 @@ int kv1b_attend_topp(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, 
   tp.q = q;
   tp.q_dtype = q_dtype;
   tp.Hq = num_q_heads;
-  tp.p = p;
+  tp.p = mode == KV1B_SELECT_TOPP ? p : 1.0f;
   tp.scale = scale;
+  tp.mode = mode;
+  tp.k = k;
+  tp.sink = sink;
+  tp.recent = recent;
   tp.out = out;
   tp.sel_idx = sel_idx;
   tp.sel_cnt = sel_cnt;
@@ -286,6 +293,13 @@ int kv1b_attend_topp(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, 
   kv1b_topp_carve(&tp, ws, cache->batch * num_q_heads, cache->capacity);
   return cuda_status(
       kv1b_launch_topp(tp, G, static_cast<int32_t>(max_length(cache)), static_cast<cudaStream_t>(stream)));
+}
+
+int kv1b_attend_topp(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,
+                     float p, float* out, int32_t* sel_idx, int32_t* sel_cnt, void* ws, size_t ws_bytes,
+                     void* stream) {
+  return kv1b_attend_select(cache, q, q_dtype, num_q_heads, scale, KV1B_SELECT_TOPP, p, 0, 0, 0, out, sel_idx, sel_cnt,
+                            ws, ws_bytes, stream);
 }
 
 int kv1b_attend_selected_exact(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads,

@@ -64,14 +64,16 @@ struct ScoresParams {
 struct ToppRowState {
   uint32_t maxkey;           // order-preserving key of the row's largest logit (atomicMax)
   uint32_t ncand;            // tokens in the threshold bucket
-  int32_t bstar;             // threshold bucket (-1: the row is empty)
+  int32_t bstar;             // threshold bucket (-1: the row is empty; -2: the kept window alone suffices)
   uint32_t merged;           // merge blocks of the row done (atomic ticket)
-  unsigned long long U;      // total integer mass
+  unsigned long long U;      // integer mass of the tokens outside the kept window (Top-k: their count)
   unsigned long long rem;    // mass still needed inside the threshold bucket
   unsigned long long kstar;  // largest selected 64-bit key of the threshold bucket
-  unsigned long long pad1[3];
+  unsigned long long Uw;     // integer mass of the kept window (Top-p)
+  unsigned long long pad1[2];
 };
 constexpr int kToppBuckets = 2048;  // masses by t = (s - m) log2 e: bucket floor(-64 t), t >= -40
+constexpr int kToppWinBucket = 0xffff;  // bucket-plane mark of a token of the kept window
 constexpr int kToppChunk = 4096;    // tokens per block of the streaming kernels
 constexpr int kToppSub = 1024;      // tokens per selected-count entry and per compaction+gather block
 constexpr int kToppMergeSplit = 8;  // first-level merge blocks per row
@@ -83,6 +85,9 @@ struct ToppParams {
   int32_t Hq;
   float p;
   float scale;
+  int32_t mode;              // KV1B_SELECT_TOPP or KV1B_SELECT_TOPK
+  int32_t k;                 // Top-k budget (tokens outside the window)
+  int32_t sink, recent;      // kept window: the first `sink` and the last `recent` tokens
   uint32_t* planes;          // [R][4][4] query bit-planes, then grid origin, step and code sum per row
   float* qvl;
   float* qdl;

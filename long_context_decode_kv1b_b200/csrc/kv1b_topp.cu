@@ -258,7 +258,7 @@ __global__ void __launch_bounds__(kStreamThreads, NG == 1 ? 4 : 2) topp_scores_k
 __global__ void __launch_bounds__(kStreamThreads) topp_mass_kernel(const ToppParams p) {
   pdl_wait();
   __shared__ uint32_t s_lo[kToppBuckets], s_hi[kToppBuckets];  // sums of ul and of uh per bucket
-  __shared__ unsigned long long s_u[kStreamWarps];
+  __shared__ unsigned long long s_u[kStreamWarps], s_w[kStreamWarps];
   const int64_t r = blockIdx.y;
   const int L = row_len(p, r);
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kToppChunk;
@@ -273,20 +273,30 @@ __global__ void __launch_bounds__(kStreamThreads) topp_mass_kernel(const ToppPar
   }
   __syncthreads();
   const float m = fkey_inv(p.rows[r].maxkey);
-  unsigned long long usum = 0ull;
+  unsigned long long usum = 0ull, wsum = 0ull;
   const int nv = static_cast<int>(t1 - tt0);  // valid tokens of this thread (may be <= 0)
+  const bool topk = p.mode == KV1B_SELECT_TOPK;
+  const int64_t win_hi = static_cast<int64_t>(L) - p.recent;  // tokens >= win_hi (and < sink) are kept
   uint32_t bkw[8];                             // the 16 buckets as 16-bit pairs
   #pragma unroll
   for (int i = 0; i < 16; ++i) {
     int bk = kToppBuckets;
     if (i < nv) {
       const float tt = topp_t(v[i], m);
-      const uint64_t u = topp_mass_t(tt);
-      bk = topp_bucket(tt);
-      if (u) {
-        atomicAdd(&s_lo[bk], static_cast<uint32_t>(u & 0xffffu));
-        atomicAdd(&s_hi[bk], static_cast<uint32_t>(u >> 16));
-        usum += u;
+      const int64_t tok = tt0 + i;
+      if (tok < p.sink || tok >= win_hi) {  // kept window: outside the histogram
+        bk = kToppWinBucket;
+        if (!topk) wsum += topp_mass_t(tt);
+      } else {
+        // Top-k: every token has unit mass, and the tokens below 2^-40 share the last bucket
+        const uint64_t u = topk ? 1ull : topp_mass_t(tt);
+        bk = topp_bucket(tt);
+        if (topk && bk > kToppBuckets - 1) bk = kToppBuckets - 1;
+        if (u) {
+          atomicAdd(&s_lo[bk], static_cast<uint32_t>(u & 0xffffu));
+          atomicAdd(&s_hi[bk], static_cast<uint32_t>(u >> 16));
+          usum += u;
+        }
       }
     }
     if (i & 1) bkw[i >> 1] |= static_cast<uint32_t>(bk) << 16;
@@ -298,7 +308,11 @@ __global__ void __launch_bounds__(kStreamThreads) topp_mass_kernel(const ToppPar
     bo[1] = make_uint4(bkw[4], bkw[5], bkw[6], bkw[7]);
   }
   usum = warp_sum(usum);
-  if ((threadIdx.x & 31) == 0) s_u[threadIdx.x >> 5] = usum;
+  wsum = warp_sum(wsum);
+  if ((threadIdx.x & 31) == 0) {
+    s_u[threadIdx.x >> 5] = usum;
+    s_w[threadIdx.x >> 5] = wsum;
+  }
   __syncthreads();
   unsigned long long* hist = p.hist + r * kToppBuckets;
   for (int i = threadIdx.x; i < kToppBuckets; i += kStreamThreads) {
@@ -306,9 +320,13 @@ __global__ void __launch_bounds__(kStreamThreads) topp_mass_kernel(const ToppPar
     if (h) atomicAdd(&hist[i], h);
   }
   if (threadIdx.x == 0) {
-    unsigned long long tot = 0ull;
-    for (int w = 0; w < kStreamWarps; ++w) tot += s_u[w];
-    atomicAdd(&p.rows[r].U, tot);
+    unsigned long long tot = 0ull, wtot = 0ull;
+    for (int w = 0; w < kStreamWarps; ++w) {
+      tot += s_u[w];
+      wtot += s_w[w];
+    }
+    if (tot) atomicAdd(&p.rows[r].U, tot);
+    if (wtot) atomicAdd(&p.rows[r].Uw, wtot);
   }
 }
 
@@ -320,14 +338,25 @@ __global__ void __launch_bounds__(kThresholdThreads) topp_threshold_kernel(const
   __shared__ unsigned long long s_w[kThresholdThreads / 32];
   const int64_t r = blockIdx.x;
   ToppRowState& rs = p.rows[r];
-  const unsigned long long U = rs.U;
-  if (U == 0ull || row_len(p, r) == 0) {  // empty row
+  if (row_len(p, r) == 0) {  // empty row
     if (threadIdx.x == 0) rs.bstar = -1;
     return;
   }
-  unsigned long long T = static_cast<unsigned long long>(ceil(static_cast<double>(p.p) * static_cast<double>(U)));
-  if (T > U) T = U;
-  if (T < 1) T = 1;
+  const unsigned long long U = rs.U, Uw = rs.Uw;
+  unsigned long long T;  // mass (Top-k: count) still needed from outside the kept window
+  if (p.mode == KV1B_SELECT_TOPK) {
+    T = static_cast<unsigned long long>(p.k) < U ? static_cast<unsigned long long>(p.k) : U;
+  } else {
+    const unsigned long long Ua = U + Uw;
+    unsigned long long Tp = static_cast<unsigned long long>(ceil(static_cast<double>(p.p) * static_cast<double>(Ua)));
+    if (Tp > Ua) Tp = Ua;
+    if (Tp < 1) Tp = 1;
+    T = Uw >= Tp ? 0ull : Tp - Uw;
+  }
+  if (T == 0ull) {  // the kept window alone is the set
+    if (threadIdx.x == 0) rs.bstar = -2;
+    return;
+  }
   const int i = threadIdx.x, lane = i & 31, warp = i >> 5;
   const unsigned long long h0 = p.hist[r * kToppBuckets + 2 * i], h1 = p.hist[r * kToppBuckets + 2 * i + 1];
   const unsigned long long loc = h0 + h1;
@@ -372,7 +401,7 @@ __global__ void __launch_bounds__(kStreamThreads) topp_cand_kernel(const ToppPar
   const int64_t t0 = static_cast<int64_t>(blockIdx.x) * kToppChunk;
   ToppRowState& rs = p.rows[r];
   const int bstar = rs.bstar;
-  if (t0 >= L || bstar < 0) return;
+  if (t0 >= L || bstar == -1) return;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int64_t t1 = t0 + kToppChunk < L ? t0 + kToppChunk : L;
   const int64_t tt0 = t0 + kTokPerThread * threadIdx.x;
@@ -389,7 +418,7 @@ __global__ void __launch_bounds__(kStreamThreads) topp_cand_kernel(const ToppPar
   for (int i = 0; i < 16; ++i) {
     if (i < nv) {
       const int bk = static_cast<int>((bkw[i >> 1] >> (16 * (i & 1))) & 0xffffu);
-      lo += bk < bstar;
+      lo += (bk < bstar) | (bk == kToppWinBucket);  // lower buckets and the kept window are selected
       cmask |= static_cast<unsigned>(bk == bstar) << i;
     }
   }
@@ -430,6 +459,7 @@ __global__ void __launch_bounds__(kResolveThreads) topp_resolve_kernel(const Top
   if (rs.bstar < 0) return;
   const int n = static_cast<int>(rs.ncand);
   const bool on_chip = n <= kResolveSmemCand;
+  const bool topk = p.mode == KV1B_SELECT_TOPK;
   const float m = fkey_inv(rs.maxkey);
   const float* s = p.s + r * p.c.cap;
   const int32_t* cand = p.cand + r * p.c.cap;
@@ -441,7 +471,7 @@ __global__ void __launch_bounds__(kResolveThreads) topp_resolve_kernel(const Top
       const int64_t t = cand[i];
       const float st = s[t];
       skey[i] = topp_key(st, t);
-      smass[i] = topp_mass_t(topp_t(st, m));
+      smass[i] = topk ? 1ull : topp_mass_t(topp_t(st, m));
     }
   }
   if (threadIdx.x == 0) {
@@ -464,7 +494,7 @@ __global__ void __launch_bounds__(kResolveThreads) topp_resolve_kernel(const Top
         const int64_t t = cand[i];
         const float st = s[t];
         key = topp_key(st, t);
-        u = topp_mass_t(topp_t(st, m));
+        u = topk ? 1ull : topp_mass_t(topp_t(st, m));
       }
       if (u && (d == 7 || (key >> (8 * (d + 1))) == prefix)) {
         const int bin = static_cast<int>((key >> (8 * d)) & 255u);
@@ -580,7 +610,7 @@ __global__ void __launch_bounds__(kStreamThreads, GM <= 4 ? 3 : 2) topp_write_ga
   for (int h = 0; h < GM; ++h) {
     if (h < G && nv > 0) {
       const ToppRowState& rs = p.rows[row0 + h];
-      const int bstar = rs.bstar;  // >= 0: the row is not empty
+      const int bstar = rs.bstar;  // >= 0, or -2 (window only): the row is not empty
       const unsigned long long kstar = rs.kstar;
       mrow[h] = fkey_inv(rs.maxkey);
       const float* srow = p.s + (row0 + h) * c.cap + tt0;
@@ -588,9 +618,10 @@ __global__ void __launch_bounds__(kStreamThreads, GM <= 4 ? 3 : 2) topp_write_ga
       for (int i = 0; i < kTok; ++i) {
         const int bk = static_cast<int>(((i < 2 ? bk4[h].x : bk4[h].y) >> (16 * (i & 1))) & 0xffffu);
         v[h][i] = 0.0f;
-        if (i < nv && bk <= bstar) {
+        const bool win = bk == kToppWinBucket;
+        if (i < nv && (win || bk <= bstar)) {
           v[h][i] = srow[i];
-          const bool f = bk < bstar || topp_key(v[h][i], tt0 + i) <= kstar;
+          const bool f = win || bk < bstar || topp_key(v[h][i], tt0 + i) <= kstar;
           mask[h] |= static_cast<unsigned>(f) << i;
         }
       }
@@ -772,7 +803,7 @@ __global__ void __launch_bounds__(kD) topp_merge_kernel(const ToppParams p) {
   const int j = blockIdx.x;
   const int ch = threadIdx.x;
   const int L = row_len(p, r);
-  const int n = p.rows[r].bstar >= 0 ? (L + kToppSub - 1) / kToppSub : 0;
+  const int n = p.rows[r].bstar != -1 ? (L + kToppSub - 1) / kToppSub : 0;
   const int k0 = static_cast<int>(static_cast<int64_t>(n) * j / M);
   const int k1 = static_cast<int>(static_cast<int64_t>(n) * (j + 1) / M);
   const float* base = p.part + r * p.nsub * kPartStride;

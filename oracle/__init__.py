@@ -63,6 +63,9 @@ def lib() -> ctypes.CDLL:
             "ref_topp_select": (i64, [P, i64, f32, P]),
             "ref_attend_topp_head": (i64, [P, P, P, P, P, i64, P, P, f32, f32, ctypes.c_int, P, P]),
             "ref_attend_exact_selected": (ctypes.c_int, [P, P, P, i64, ctypes.c_int, P, i64, f32, P]),
+            "ref_select": (i64, [P, i64, ctypes.c_int, f32, i64, i64, i64, P]),
+            "ref_attend_select_head": (i64, [P, P, P, P, P, i64, P, P, f32, ctypes.c_int, f32, i64, i64, i64,
+                                             ctypes.c_int, P, P]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -244,6 +247,35 @@ def attend_topp(enc: dict, q, sgn, scale: float, p: float):
     n = lib().ref_attend_topp_head(*ptrs, L, _p(q), _p(sgn), float(scale), float(p), d, _p(sel), _p(out))
     if n < 0:
         raise ValueError("invalid Top-p arguments")
+    return sel[:n].copy(), out
+
+
+SELECT_TOPP, SELECT_TOPK = 0, 1
+
+
+def select(s, mode: int, p: float = 1.0, k: int = 0, sink: int = 0, recent: int = 0) -> np.ndarray:
+    """Top-p (mode 0) or Top-k (mode 1) selection plus the always-kept first `sink` / last `recent`
+    tokens; ascending indices."""
+    s = _f32(s)
+    sel = np.empty(max(1, s.shape[0]), np.int64)
+    n = lib().ref_select(_p(s), s.shape[0], int(mode), float(p), int(k), int(sink), int(recent), _p(sel))
+    if n < 0:
+        raise ValueError("invalid selection arguments")
+    return sel[:n].copy()
+
+
+def attend_select(enc: dict, q, sgn, scale: float, mode: int, p: float = 1.0, k: int = 0, sink: int = 0,
+                  recent: int = 0):
+    """Attention of one query head over a `select` set; returns (indices ascending, fp64 out)."""
+    keep, ptrs, L, d = _enc_ptrs(enc)
+    q = _f32(q)
+    sgn = _f32(sgn)
+    out = np.empty(d, np.float64)
+    sel = np.empty(max(1, L), np.int64)
+    n = lib().ref_attend_select_head(*ptrs, L, _p(q), _p(sgn), float(scale), int(mode), float(p), int(k), int(sink),
+                                     int(recent), d, _p(sel), _p(out))
+    if n < 0:
+        raise ValueError("invalid selection arguments")
     return sel[:n].copy(), out
 
 

@@ -425,6 +425,88 @@ int64_t ref_attend_topp_head(const uint32_t* bits, const float* norm, const floa
   return n;
 }
 
+/* RaBitQCache abstract (adaptive Top-p, and the fixed Top-k budget it is contrasted with) and the
+ * H1IB-KV article, part 2 item 1 (a high-precision layer for important tokens; here the first
+ * `sink` and last `recent` tokens are always kept). */
+int64_t ref_select(const float* s, int64_t L, int mode, float p, int64_t k, int64_t sink, int64_t recent,
+                   int64_t* sel) {
+  if (mode != 0 && mode != 1) return -1;
+  if (mode == 0 && !(p > 0.0f && p <= 1.0f)) return -1;
+  if (mode == 1 && k < 0) return -1;
+  if (sink < 0 || recent < 0) return -1;
+  if (L <= 0) return 0;
+  std::vector<char> win(L, 0);
+  for (int64_t t = 0; t < L; ++t) win[t] = (t < sink || t >= L - recent) ? 1 : 0;
+  std::vector<int64_t> order;
+  for (int64_t t = 0; t < L; ++t)
+    if (!win[t]) order.push_back(t);
+  std::sort(order.begin(), order.end(), [&](int64_t a, int64_t b) {
+    if (s[a] != s[b]) return s[a] > s[b];
+    return a < b;
+  });
+  int64_t n_extra = 0;
+  if (mode == 1) {
+    n_extra = std::min<int64_t>(k, static_cast<int64_t>(order.size()));
+  } else {
+    float m = s[0];
+    for (int64_t t = 1; t < L; ++t) m = std::max(m, s[t]);
+    uint64_t U = 0, Uw = 0;
+    for (int64_t t = 0; t < L; ++t) {
+      const uint64_t u = ref_topp_weight(s[t], m);
+      U += u;
+      if (win[t]) Uw += u;
+    }
+    uint64_t T = static_cast<uint64_t>(std::ceil(static_cast<double>(p) * static_cast<double>(U)));
+    if (T > U) T = U;
+    if (T < 1) T = 1;
+    if (Uw < T) {
+      const uint64_t need = T - Uw;
+      uint64_t acc = 0;
+      while (n_extra < static_cast<int64_t>(order.size())) {
+        acc += ref_topp_weight(s[order[n_extra]], m);
+        ++n_extra;
+        if (acc >= need) break;
+      }
+    }
+  }
+  std::vector<int64_t> chosen(order.begin(), order.begin() + n_extra);
+  for (int64_t t = 0; t < L; ++t)
+    if (win[t]) chosen.push_back(t);
+  std::sort(chosen.begin(), chosen.end());
+  for (size_t i = 0; i < chosen.size(); ++i) sel[i] = chosen[i];
+  return static_cast<int64_t>(chosen.size());
+}
+
+int64_t ref_attend_select_head(const uint32_t* bits, const float* norm, const float* cinv, const uint32_t* codes,
+                               const uint32_t* sm, int64_t L, const float* q, const float* signs, float scale,
+                               int mode, float p, int64_t k, int64_t sink, int64_t recent, int d, int64_t* sel,
+                               double* out) {
+  for (int c = 0; c < d; ++c) out[c] = 0.0;
+  if (!valid_d(d)) return -1;
+  if (L <= 0) return ref_select(nullptr, 0, mode, p, k, sink, recent, sel);
+  std::vector<uint32_t> planes(4 * (d / 32));
+  float vl, dl;
+  int32_t Sq;
+  ref_query_prep(q, signs, d, planes.data(), &vl, &dl, &Sq, nullptr, nullptr);
+  std::vector<float> s(L);
+  ref_logits(bits, norm, cinv, L, planes.data(), vl, dl, Sq, scale, d, s.data());
+  const int64_t n = ref_select(s.data(), L, mode, p, k, sink, recent, sel);
+  if (n <= 0) return n;
+  double m = s[sel[0]];
+  for (int64_t i = 1; i < n; ++i) m = std::max(m, static_cast<double>(s[sel[i]]));
+  std::vector<double> acc(d, 0.0), vh(d);
+  double l = 0.0;
+  for (int64_t i = 0; i < n; ++i) {
+    const int64_t t = sel[i];
+    const double e = std::exp(static_cast<double>(s[t]) - m);
+    l += e;
+    ref_dequant_value(codes + t * (d / 8), sm + t * (d / 32), d, vh.data());
+    for (int c = 0; c < d; ++c) acc[c] += e * vh[c];
+  }
+  for (int c = 0; c < d; ++c) out[c] = acc[c] / l;
+  return n;
+}
+
 /* RaBitQCache abstract / core idea: after the proxy scores pick the token set, attention is taken
  * over that set alone with the exact keys and values (sparse attention).  Plain fp64 softmax. */
 int ref_attend_exact_selected(const float* q, const float* K, const float* V, int64_t L, int d, const int64_t* sel,

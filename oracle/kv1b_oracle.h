@@ -109,6 +109,25 @@ int64_t ref_attend_topp_head(const uint32_t* bits, const float* norm, const floa
                              const uint32_t* sm, int64_t L, const float* q, const float* signs, float scale,
                              float p, int d, int64_t* sel, double* out);
 
+/* Token selection with a mass threshold or a fixed budget, plus an always-kept window (RaBitQCache
+ * abstract: adaptive Top-p against a fixed Top-k budget; H1IB-KV article part 2 item 1: a
+ * high-precision layer for the important tokens -- read here as the first `sink` and the last
+ * `recent` tokens).  W = {t < sink} U {t >= L - recent}.  mode 0 (Top-p): masses u_t as
+ * ref_topp_weight with m = max over all L tokens, T = ceil(p U) clamped to [1, U],
+ * need = T - sum_{t in W} u_t; the shortest prefix of the other tokens in (s desc, index asc) order
+ * whose mass reaches need (nothing when need <= 0).  mode 1 (Top-k): the first min(k, L - |W|) other
+ * tokens in that order.  sel receives W and the chosen tokens in ascending order; returns their
+ * number, or -1 on an invalid mode / p / k / sink / recent. */
+int64_t ref_select(const float* s, int64_t L, int mode, float p, int64_t k, int64_t sink, int64_t recent,
+                   int64_t* sel);
+
+/* Attention over a ref_select set for one query head: fp64 softmax over the selected tokens'
+ * estimated logits and dequantised values (as ref_attend_topp_head).  Returns the set size or -1. */
+int64_t ref_attend_select_head(const uint32_t* bits, const float* norm, const float* cinv, const uint32_t* codes,
+                               const uint32_t* sm, int64_t L, const float* q, const float* signs, float scale,
+                               int mode, float p, int64_t k, int64_t sink, int64_t recent, int d, int64_t* sel,
+                               double* out);
+
 /* Exact attention over a selected token set (RaBitQCache, abstract / core idea: the proxy scores
  * retrieve the tokens, attention over them is then sparse attention with the exact keys and
  * values).  q: [d]; K, V: [L][d] as fp32 (the exact values of the caller's keys and values);

@@ -353,3 +353,60 @@ def test_exact_kv_dtypes_and_strides(dtype):
     _, sel, cnt = cache.attend_topp(q, 0.25, 0.8)
     exact_check(cache, q, 0.25, K, V, sel, cnt, G, where=f"{dtype} strided")
     exact_check(cache, q, 0.25, Kc, Vc, sel, cnt, G, where=f"{dtype} contiguous")
+
+
+# ------------------------------------------------------------------ Top-k budget and the kept window
+def select_check(cache, host, q, scale, G, signs, mode, p=1.0, k=0, sink=0, recent=0, where=""):
+    out, sel, cnt = cache.attend_select(q, scale, mode, p=p, k=k, sink=sink, recent=recent)
+    torch.cuda.synchronize()
+    qn = to_np32(q)
+    B, Hq, _ = qn.shape
+    encs = {}
+    for b in range(B):
+        for hq in range(Hq):
+            kvh = hq // G
+            if (b, kvh) not in encs:
+                encs[(b, kvh)] = host.encode(b, kvh, signs)
+            rs, ro = oracle.attend_select(encs[(b, kvh)], qn[b, hq], signs, scale, mode, p=p, k=k, sink=sink,
+                                          recent=recent)
+            n = cnt[b, hq].item()
+            assert n == len(rs), f"{where} b{b} hq{hq}: count {n} vs {len(rs)}"
+            assert np.array_equal(sel[b, hq, :n].cpu().numpy(), rs), f"{where} b{b} hq{hq}: index sets differ"
+            assert_rows_close(out[b, hq].cpu().numpy(), ro, where=f"{where} b{b} hq{hq}")
+    return cnt
+
+
+@pytest.mark.parametrize("k", [0, 1, 37, 5000, 9999])
+def test_topk_parity(k):
+    # 5097 tokens over two chunks and a ragged tail; k = 0 and k above the length included
+    B, Hkv, G = 1, 2, 4
+    cache, host = build_cache(B, Hkv, [5000, 97], torch.bfloat16, seed=17, data_seed=4)
+    q = torch.randn((B, Hkv * G, 128), device=DEV, generator=torch.Generator(device=DEV).manual_seed(8))
+    cnt = select_check(cache, host, q.to(torch.bfloat16), 0.4, G, oracle.signs(17), kv.SELECT_TOPK, k=k,
+                       where=f"k{k}")
+    assert torch.all(cnt == min(k, 5097)).item()
+
+
+@pytest.mark.parametrize("mode,p,k", [(0, 0.5, 0), (0, 0.99, 0), (1, 0, 20)])
+@pytest.mark.parametrize("sink,recent", [(4, 0), (0, 64), (16, 300), (3000, 3000)])
+def test_select_with_kept_window(mode, p, k, sink, recent):
+    B, Hkv, G = 2, 1, 2
+    cache, host = build_cache(B, Hkv, [4200], torch.bfloat16, seed=23, data_seed=5)
+    q = torch.randn((B, Hkv * G, 128), device=DEV, generator=torch.Generator(device=DEV).manual_seed(3))
+    select_check(cache, host, q, 0.5, G, oracle.signs(23), mode, p=p, k=k, sink=sink, recent=recent,
+                 where=f"m{mode} s{sink} r{recent}")
+
+
+def test_topk_ties_take_lowest_indices():
+    B, Hkv, G, L = 1, 1, 1, 600
+    cache = kv.Cache(B, Hkv, 640, seed=4)
+    host = HostKV(B, Hkv, 640)
+    g = torch.Generator(device=DEV).manual_seed(0)
+    K = torch.randn((B, L, Hkv, 128), generator=g, device=DEV)
+    K[:, 100:500] = K[:, 50:51]  # 401 equal keys -> equal logits
+    V = torch.randn((B, L, Hkv, 128), generator=g, device=DEV)
+    cache.append(K, V)
+    host.add(K, V)
+    q = K[:, 50, :, :].clone().view(B, 1, 128) * 0.3
+    for k in (10, 200, 450):
+        select_check(cache, host, q, 0.3, G, oracle.signs(4), kv.SELECT_TOPK, k=k, where=f"ties k{k}")

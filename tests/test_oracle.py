@@ -563,3 +563,60 @@ def test_exact_selected_invariants():
     K3[9] = 50.0 * q / np.linalg.norm(q)
     out3 = oracle.attend_exact_selected(q, K3, V, sel, 1.0)
     assert np.allclose(out3, V[9], rtol=1e-9, atol=1e-9)
+
+
+# ------------------------------------------------------------------ Top-k budget and the kept window
+# RaBitQCache abstract (adaptive Top-p vs a fixed Top-k budget) and the H1IB-KV article's high-precision
+# layer, read as an always-kept first `sink` / last `recent` window.
+def _key_order(s):
+    """(s desc, index asc) order by numpy's lexsort (a library sort, independent of the oracle)."""
+    return np.lexsort((np.arange(len(s)), -s.astype(np.float64)))
+
+
+def test_select_topk_is_the_first_k_in_key_order():
+    rng = np.random.default_rng(12)
+    for L in (1, 7, 40, 300):
+        s = np.round(rng.standard_normal(L) * 3, 1).astype(np.float32)  # many equal logits
+        order = _key_order(s)
+        for k in (0, 1, 5, L, L + 3):
+            sel = oracle.select(s, oracle.SELECT_TOPK, k=k)
+            assert np.array_equal(sel, np.sort(order[:min(k, L)]))
+
+
+def test_select_window_is_always_kept_and_budget_applies_to_the_rest():
+    rng = np.random.default_rng(13)
+    L = 200
+    s = rng.standard_normal(L).astype(np.float32)
+    s[3] = 50.0  # a dominant token inside the sink
+    for sink, recent in ((0, 0), (4, 0), (0, 16), (4, 16), (150, 60)):
+        win = [t for t in range(L) if t < sink or t >= L - recent]
+        rest = np.array([t for t in range(L) if t not in win], np.int64)
+        order = rest[_key_order(s[rest])] if rest.size else rest
+        for k in (0, 3, 10):
+            sel = oracle.select(s, oracle.SELECT_TOPK, k=k, sink=sink, recent=recent)
+            assert np.array_equal(sel, np.sort(np.concatenate([win, order[:k]]).astype(np.int64)))
+        for p in (0.3, 0.9, 1.0):
+            sel = oracle.select(s, oracle.SELECT_TOPP, p=p, sink=sink, recent=recent)
+            assert set(win) <= set(sel.tolist())
+            m = s.max()
+            u = np.array([oracle.topp_weight(x, m) for x in s], dtype=object)
+            T = min(max(int(math.ceil(float(np.float32(p)) * float(sum(u)))), 1), int(sum(u)))
+            extra = [t for t in sel.tolist() if t not in win]
+            mass = sum(u[t] for t in sel.tolist())
+            if extra:
+                # the extra tokens are a prefix of the key order, and the shortest one reaching T
+                assert extra == sorted(order[:len(extra)].tolist())
+                last = order[len(extra) - 1]
+                assert mass >= T and mass - u[last] < T
+            else:
+                assert sum(u[t] for t in win) >= T or len(rest) == 0
+    # with no window, Top-p equals the plain Top-p selection
+    assert np.array_equal(oracle.select(s, oracle.SELECT_TOPP, p=0.7), oracle.topp_select(s, 0.7))
+    # a window covering everything keeps everything
+    assert np.array_equal(oracle.select(s, oracle.SELECT_TOPK, k=0, sink=120, recent=120), np.arange(L))
+    with pytest.raises(ValueError):
+        oracle.select(s, 2)
+    with pytest.raises(ValueError):
+        oracle.select(s, oracle.SELECT_TOPK, k=-1)
+    with pytest.raises(ValueError):
+        oracle.select(s, oracle.SELECT_TOPP, p=0.0)
