@@ -44,6 +44,7 @@ extern "C" {
 #define KV1B_HEAD_DIM 128
 #define KV1B_MAX_BATCH 64
 #define KV1B_MAX_GROUP 8
+#define KV1B_MAX_ROUNDS 3  /* rotation rounds H * diag(D_r) a cache may use (kv1b_cache_init_rounds) */
 #define KV1B_CAPACITY_ALIGN 128
 
 /* return codes */
@@ -89,7 +90,8 @@ extern "C" {
  *           elements that the tensor-core engine expands to a byte per code in shared memory.
  *   v_sm    u32 [batch][hkv][capacity][4]     per 32-channel group: low half = fp16 scale,
  *           high half = fp16 min; value = min + scale * code
- *   signs   f32 [128]                         rotation signs D (+-1)
+ *   signs   f32 [3][128]                      rotation signs D_r (+-1) of each round; 0 for the
+ *                                             rounds past rotation_rounds
  *   d_lengths i32 [batch]                     tokens held per sequence (device copy)
  *   d_status  i32 [1]                         OR of KV1B_STATUS_* bits since init
  * h_lengths is the host mirror of d_lengths; both change only through kv1b_encode_append.
@@ -109,6 +111,8 @@ typedef struct kv1b_cache {
   int32_t* d_lengths;
   int32_t* d_status;
   int64_t h_lengths[KV1B_MAX_BATCH];
+  int32_t rotation_rounds;  /* 1 (kv1b_cache_init) to KV1B_MAX_ROUNDS (kv1b_cache_init_rounds) */
+  int32_t reserved;
 } kv1b_cache_t;
 
 /* Bytes of device memory a cache of this shape needs (0 if the shape is unsupported). */
@@ -119,6 +123,15 @@ size_t kv1b_cache_bytes(int32_t batch, int32_t num_kv_heads, int32_t head_dim, i
  * to 0.  Writes the descriptor *cache (host memory).  Asynchronous on `stream`. */
 int kv1b_cache_init(kv1b_cache_t* cache, void* dev_buf, size_t bytes, int32_t batch, int32_t num_kv_heads,
                     int32_t head_dim, int32_t capacity, uint64_t seed, void* stream);
+
+/* kv1b_cache_init with a stronger rotation: `rounds` (1..KV1B_MAX_ROUNDS) successive H * diag(D_r)
+ * applied to keys and queries (a closer stand-in for RaBitQ's random orthogonal rotation, whose
+ * unbiasedness the RaBitQCache abstract relies on).  Round r's signs are outputs 128 r .. 128 r + 127
+ * of the same SplitMix64(seed) stream, so rounds = 1 is kv1b_cache_init.  The estimator needs no
+ * other change: C^-1 = 128 N / sum|y| and the query grid both scale with the rotation.  Every later
+ * call reads the rounds from the cache.  KV1B_ERR_INVALID_ARG for rounds outside 1..3. */
+int kv1b_cache_init_rounds(kv1b_cache_t* cache, void* dev_buf, size_t bytes, int32_t batch, int32_t num_kv_heads,
+                           int32_t head_dim, int32_t capacity, uint64_t seed, int32_t rounds, void* stream);
 
 /* Encode and append n_new tokens to every sequence (the same n_new for all).
  * k, v: device arrays of `dtype` (KV1B_DTYPE_*); element (b, t, h, c) of K sits at

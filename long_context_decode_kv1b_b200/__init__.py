@@ -24,7 +24,7 @@ ERRORS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "capacity", -4
           -5: "workspace too small", -6: "CUDA error"}
 
 # symbols declared in include/kv1b.h
-SYMBOLS = ("kv1b_cache_bytes", "kv1b_cache_init", "kv1b_encode_append", "kv1b_attend_workspace_bytes",
+SYMBOLS = ("kv1b_cache_bytes", "kv1b_cache_init", "kv1b_cache_init_rounds", "kv1b_encode_append", "kv1b_attend_workspace_bytes",
            "kv1b_attend", "kv1b_attend_noalloc", "kv1b_attend_topp", "kv1b_attend_select",
            "kv1b_attend_selected_exact",
            "kv1b_query_prep", "kv1b_scores",
@@ -46,6 +46,7 @@ class CacheDesc(ctypes.Structure):
         ("v_codes", ctypes.c_void_p), ("v_sm", ctypes.c_void_p), ("signs", ctypes.c_void_p),
         ("d_lengths", ctypes.c_void_p), ("d_status", ctypes.c_void_p),
         ("h_lengths", ctypes.c_int64 * MAX_BATCH),
+        ("rotation_rounds", ctypes.c_int32), ("reserved", ctypes.c_int32),
     ]
 
 
@@ -64,6 +65,7 @@ def lib() -> ctypes.CDLL:
         sig = {
             "kv1b_cache_bytes": (sz, [i32, i32, i32, i32]),
             "kv1b_cache_init": (ctypes.c_int, [D, P, sz, i32, i32, i32, i32, ctypes.c_uint64, P]),
+            "kv1b_cache_init_rounds": (ctypes.c_int, [D, P, sz, i32, i32, i32, i32, ctypes.c_uint64, i32, P]),
             "kv1b_encode_append": (ctypes.c_int, [D, P, P, i32, i32, i64, i64, i64, P]),
             "kv1b_attend_workspace_bytes": (sz, [D, i32, i32]),
             "kv1b_attend": (ctypes.c_int, [D, P, i32, i32, f32, P, P, sz, i32, i32, P]),
@@ -121,9 +123,11 @@ class Cache:
     """A compressed KV cache for `batch` sequences x `num_kv_heads` heads, in one device buffer."""
 
     def __init__(self, batch: int, num_kv_heads: int, capacity: int, seed: int = 0, device="cuda",
-                 stream=None):
+                 stream=None, rounds: int = 1):
+        """rounds: rotation rounds H * diag(D_r) (1 .. 3; see kv1b_cache_init_rounds)."""
         L = lib()
         self.batch, self.num_kv_heads, self.capacity, self.seed = batch, num_kv_heads, capacity, seed
+        self.rounds = rounds
         self.device = torch.device(device)
         nbytes = L.kv1b_cache_bytes(batch, num_kv_heads, HEAD_DIM, capacity)
         if nbytes == 0:
@@ -131,8 +135,8 @@ class Cache:
         self.nbytes = nbytes
         self.buffer = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
         self.desc = CacheDesc()
-        _check(L.kv1b_cache_init(ctypes.byref(self.desc), _ptr(self.buffer), nbytes, batch, num_kv_heads, HEAD_DIM,
-                                 capacity, seed, _stream(stream)), "kv1b_cache_init")
+        _check(L.kv1b_cache_init_rounds(ctypes.byref(self.desc), _ptr(self.buffer), nbytes, batch, num_kv_heads,
+                                        HEAD_DIM, capacity, seed, rounds, _stream(stream)), "kv1b_cache_init_rounds")
         self._ws = {}
 
     # ---- views of the device planes (for tests / inspection; layout in include/kv1b.h)
@@ -153,7 +157,8 @@ class Cache:
             "k_cinv": self._view(d.k_cinv, torch.float32, (B, H, C)),
             "v_codes": self._view(d.v_codes, torch.int32, (B, H, C // 128, HEAD_DIM, 16)),
             "v_sm": self._view(d.v_sm, torch.int32, (B, H, C, 4)),
-            "signs": self._view(d.signs, torch.float32, (HEAD_DIM,)),
+            "signs": self._view(d.signs, torch.float32, (HEAD_DIM,)),  # round 0
+            "signs_rounds": self._view(d.signs, torch.float32, (3, HEAD_DIM)),
             "lengths": self._view(d.d_lengths, torch.int32, (B,)),
         }
 

@@ -32,7 +32,7 @@ Layout layout(int32_t batch, int32_t hkv, int32_t capacity) {
   l.k_cinv = off;  off += align_up(tok * 4);
   l.v_codes = off; off += align_up(tok * 64);
   l.v_sm = off;    off += align_up(tok * 16);
-  l.signs = off;   off += align_up(KV1B_HEAD_DIM * 4);
+  l.signs = off;   off += align_up(KV1B_MAX_ROUNDS * KV1B_HEAD_DIM * 4);
   l.lengths = off; off += align_up(KV1B_MAX_BATCH * 4);
   l.status = off;  off += align_up(4);
   l.total = off;
@@ -131,7 +131,12 @@ size_t kv1b_cache_bytes(int32_t batch, int32_t num_kv_heads, int32_t head_dim, i
 
 int kv1b_cache_init(kv1b_cache_t* cache, void* dev_buf, size_t bytes, int32_t batch, int32_t num_kv_heads,
                     int32_t head_dim, int32_t capacity, uint64_t seed, void* stream) {
-  if (!cache || !dev_buf) return KV1B_ERR_INVALID_ARG;
+  return kv1b_cache_init_rounds(cache, dev_buf, bytes, batch, num_kv_heads, head_dim, capacity, seed, 1, stream);
+}
+
+int kv1b_cache_init_rounds(kv1b_cache_t* cache, void* dev_buf, size_t bytes, int32_t batch, int32_t num_kv_heads,
+                           int32_t head_dim, int32_t capacity, uint64_t seed, int32_t rounds, void* stream) {
+  if (!cache || !dev_buf || rounds < 1 || rounds > KV1B_MAX_ROUNDS) return KV1B_ERR_INVALID_ARG;
   if (head_dim != KV1B_HEAD_DIM || batch > KV1B_MAX_BATCH) return KV1B_ERR_UNSUPPORTED;
   if (!shape_ok(batch, num_kv_heads, head_dim, capacity)) return KV1B_ERR_INVALID_ARG;
   if (!aligned(dev_buf, kAlign)) return KV1B_ERR_MISALIGNED;
@@ -145,6 +150,7 @@ int kv1b_cache_init(kv1b_cache_t* cache, void* dev_buf, size_t bytes, int32_t ba
   c.head_dim = head_dim;
   c.capacity = capacity;
   c.rotation_seed = seed;
+  c.rotation_rounds = rounds;
   c.k_bits = reinterpret_cast<uint32_t*>(base + l.k_bits);
   c.k_norm = reinterpret_cast<float*>(base + l.k_norm);
   c.k_cinv = reinterpret_cast<float*>(base + l.k_cinv);
@@ -156,7 +162,7 @@ int kv1b_cache_init(kv1b_cache_t* cache, void* dev_buf, size_t bytes, int32_t ba
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   cudaError_t e = cudaMemsetAsync(dev_buf, 0, l.total, s);
   if (e != cudaSuccess) return KV1B_ERR_CUDA;
-  e = kv1b_launch_init(seed, c.signs, c.d_lengths, batch, c.d_status, s);
+  e = kv1b_launch_init(seed, rounds, c.signs, c.d_lengths, batch, c.d_status, s);
   if (e != cudaSuccess) return KV1B_ERR_CUDA;
   *cache = c;
   return KV1B_OK;

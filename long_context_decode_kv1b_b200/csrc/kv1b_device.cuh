@@ -62,6 +62,21 @@ __device__ __forceinline__ void rotate128(float x[4], const float sgn[4]) {
   }
 }
 
+// Several rounds y <- H (D_r (.) y) (a stronger rotation): signs holds KV1B_MAX_ROUNDS x 128 entries
+// and a round whose first sign is 0 ends the rotation (one round unless the cache asked for more).
+__device__ __forceinline__ void rotate_rounds(float x[4], const float* signs) {
+  const int lane = threadIdx.x & 31;
+  #pragma unroll 1
+  for (int r = 0; r < KV1B_MAX_ROUNDS; ++r) {
+    const float* sr = signs + r * kD;
+    if (sr[0] == 0.0f) break;  // the same address for every lane: warp-uniform
+    float sg[4];
+    #pragma unroll
+    for (int j = 0; j < 4; ++j) sg[j] = sr[4 * lane + j];
+    rotate128(x, sg);
+  }
+}
+
 // Fixed pairwise tree over the 128 channels: for h = 64, 32, ..., 1: a[i] += a[i + h] (i < h).
 // Returns a[0] on every lane.
 __device__ __forceinline__ float tree_sum128(const float a_in[4]) {
@@ -103,11 +118,9 @@ struct QueryPrep {
 
 __device__ __forceinline__ QueryPrep query_prep_warp(const void* q, int64_t row_off, int dtype, const float* signs) {
   const int lane = threadIdx.x & 31;
-  float x[4], sg[4];
+  float x[4];
   load4(q, row_off + 4 * lane, dtype, x);
-  #pragma unroll
-  for (int r = 0; r < 4; ++r) sg[r] = signs[4 * lane + r];
-  rotate128(x, sg);
+  rotate_rounds(x, signs);
   float lo = fminf(fminf(x[0], x[1]), fminf(x[2], x[3]));
   float hi = fmaxf(fmaxf(x[0], x[1]), fmaxf(x[2], x[3]));
   #pragma unroll

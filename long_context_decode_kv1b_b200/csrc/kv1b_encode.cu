@@ -11,11 +11,17 @@
 namespace kv1b {
 
 // SplitMix64 (Steele, Lea & Flood, OOPSLA 2014) draws the rotation signs: D_i = -1 iff the top bit
-// of the i-th output is set.  One thread; runs once per cache.
-__global__ void init_kernel(uint64_t seed, float* signs, int32_t* lengths, int32_t batch, int32_t* status) {
+// of the i-th output is set; round r of a stronger rotation takes outputs 128 r .. 128 r + 127 of the
+// same stream, and the rounds past `rounds` are zero.  One thread; runs once per cache.
+__global__ void init_kernel(uint64_t seed, int rounds, float* signs, int32_t* lengths, int32_t batch,
+                            int32_t* status) {
   if (threadIdx.x == 0 && blockIdx.x == 0) {
     uint64_t st = seed;
-    for (int i = 0; i < kD; ++i) {
+    for (int i = 0; i < KV1B_MAX_ROUNDS * kD; ++i) {
+      if (i >= rounds * kD) {
+        signs[i] = 0.0f;
+        continue;
+      }
       st += 0x9E3779B97F4A7C15ull;
       uint64_t z = st;
       z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
@@ -51,17 +57,16 @@ __global__ void __launch_bounds__(512) encode_kernel(const EncodeParams p) {
     const int64_t row = static_cast<int64_t>(b) * p.sb + t * p.st + static_cast<int64_t>(h) * p.sh;
     int flags = 0;
     // ---- key sketch
-    float x[4], sg[4], sq[4], y[4], ab[4];
+    float x[4], sq[4], y[4], ab[4];
     load4(p.k, row + 4 * lane, p.dtype, x);
     #pragma unroll
     for (int r = 0; r < 4; ++r) {
-      sg[r] = p.signs[4 * lane + r];
       sq[r] = __fmul_rn(x[r], x[r]);
       if (!isfinite(x[r])) flags |= KV1B_STATUS_NONFINITE;
       y[r] = x[r];
     }
     const float nrm = __fsqrt_rn(tree_sum128(sq));
-    rotate128(y, sg);
+    rotate_rounds(y, p.signs);
     uint32_t nib = 0;
     #pragma unroll
     for (int r = 0; r < 4; ++r) {
@@ -138,9 +143,10 @@ __global__ void __launch_bounds__(512) encode_kernel(const EncodeParams p) {
 
 using namespace kv1b;
 
-cudaError_t kv1b_launch_init(uint64_t seed, float* signs, int32_t* lengths, int32_t batch, int32_t* status,
+cudaError_t kv1b_launch_init(uint64_t seed, int32_t rounds, float* signs, int32_t* lengths, int32_t batch,
+                             int32_t* status,
                              cudaStream_t stream) {
-  init_kernel<<<1, 64, 0, stream>>>(seed, signs, lengths, batch, status);
+  init_kernel<<<1, 64, 0, stream>>>(seed, rounds, signs, lengths, batch, status);
   return cudaGetLastError();
 }
 

@@ -153,7 +153,8 @@ struct alignas(64) AttendWsParams {
 
 }  // namespace kv1b
 
-cudaError_t kv1b_launch_init(uint64_t seed, float* signs, int32_t* lengths, int32_t batch, int32_t* status,
+cudaError_t kv1b_launch_init(uint64_t seed, int32_t rounds, float* signs, int32_t* lengths, int32_t batch,
+                             int32_t* status,
                              cudaStream_t stream);
 cudaError_t kv1b_launch_encode(const kv1b::EncodeParams& p, int64_t max_tiles, cudaStream_t stream);
 cudaError_t kv1b_launch_attend(const kv1b::AttendParams& p, int32_t G, int32_t engine, int32_t max_len,

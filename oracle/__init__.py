@@ -45,6 +45,7 @@ def lib() -> ctypes.CDLL:
         sig = {
             "ref_splitmix64_next": (u64, [P]),
             "ref_rotation_signs": (None, [u64, ctypes.c_int, P]),
+            "ref_rotation_signs_rounds": (None, [u64, ctypes.c_int, ctypes.c_int, P]),
             "ref_fwht": (None, [P, ctypes.c_int]),
             "ref_tree_sum": (f32, [P, ctypes.c_int]),
             "ref_encode_key": (None, [P, P, ctypes.c_int, P, P, P]),
@@ -90,9 +91,26 @@ def splitmix64(seed: int, n: int) -> np.ndarray:
     return np.array([lib().ref_splitmix64_next(ctypes.byref(st)) for _ in range(n)], dtype=np.uint64)
 
 
-def signs(seed: int, d: int = 128) -> np.ndarray:
-    out = np.empty(d, np.float32)
-    lib().ref_rotation_signs(seed, d, _p(out))
+MAX_ROUNDS = 3
+
+
+def signs(seed: int, d: int = 128, rounds: int = 1) -> np.ndarray:
+    """Rotation signs: [d] for one round, else [rounds * d] (round r = the next d draws)."""
+    if rounds == 1:
+        out = np.empty(d, np.float32)
+        lib().ref_rotation_signs(seed, d, _p(out))
+        return out
+    out = np.empty(MAX_ROUNDS * d, np.float32)
+    lib().ref_rotation_signs_rounds(seed, d, rounds, _p(out))
+    return out[:rounds * d].copy()
+
+
+def _sg(sgn, d: int) -> np.ndarray:
+    """Signs as the C oracle reads them: MAX_ROUNDS x d entries, rounds after the given ones zero."""
+    sgn = _f32(sgn).reshape(-1)
+    assert sgn.size % d == 0 and 0 < sgn.size // d <= MAX_ROUNDS
+    out = np.zeros(MAX_ROUNDS * d, np.float32)
+    out[:sgn.size] = sgn
     return out
 
 
@@ -112,7 +130,7 @@ def encode(K, V, sgn) -> dict:
     K = _f32(K)
     V = _f32(V)
     L, d = K.shape
-    sgn = _f32(sgn)
+    sgn = _sg(sgn, d)
     bits = np.empty((L, d // 32), np.uint32)
     norm = np.empty(L, np.float32)
     cinv = np.empty(L, np.float32)
@@ -145,7 +163,7 @@ def query_prep(q, sgn) -> dict:
     single = q.ndim == 1
     q2 = q.reshape(-1, q.shape[-1])
     H, d = q2.shape
-    sgn = _f32(sgn)
+    sgn = _sg(sgn, d)
     planes = np.empty((H, 4, d // 32), np.uint32)
     vl = np.empty(H, np.float32)
     dl = np.empty(H, np.float32)
@@ -214,7 +232,7 @@ def attend(enc: dict, q, sgn, scale: float) -> np.ndarray:
     """Full attention of one query head (q: [d]) over one encoded (sequence, kv-head); fp64 out."""
     keep, ptrs, L, d = _enc_ptrs(enc)
     q = _f32(q)
-    sgn = _f32(sgn)
+    sgn = _sg(sgn, d)
     out = np.empty(d, np.float64)
     lib().ref_attend_head(*ptrs, L, _p(q), _p(sgn), float(scale), d, _p(out))
     return out
@@ -241,7 +259,7 @@ def attend_topp(enc: dict, q, sgn, scale: float, p: float):
     """Top-p attention of one query head; returns (selected indices ascending, fp64 out)."""
     keep, ptrs, L, d = _enc_ptrs(enc)
     q = _f32(q)
-    sgn = _f32(sgn)
+    sgn = _sg(sgn, d)
     out = np.empty(d, np.float64)
     sel = np.empty(max(1, L), np.int64)
     n = lib().ref_attend_topp_head(*ptrs, L, _p(q), _p(sgn), float(scale), float(p), d, _p(sel), _p(out))
@@ -269,7 +287,7 @@ def attend_select(enc: dict, q, sgn, scale: float, mode: int, p: float = 1.0, k:
     """Attention of one query head over a `select` set; returns (indices ascending, fp64 out)."""
     keep, ptrs, L, d = _enc_ptrs(enc)
     q = _f32(q)
-    sgn = _f32(sgn)
+    sgn = _sg(sgn, d)
     out = np.empty(d, np.float64)
     sel = np.empty(max(1, L), np.int64)
     n = lib().ref_attend_select_head(*ptrs, L, _p(q), _p(sgn), float(scale), int(mode), float(p), int(k), int(sink),

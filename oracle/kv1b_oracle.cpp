@@ -91,9 +91,18 @@ uint16_t half_scale_up(double D, int* sat) {
   return t[lo].second;
 }
 
+// Up to kRefMaxRounds rounds y <- H (D_r (.) y); signs holds kRefMaxRounds x d entries, and a
+// round whose signs are 0 ends the rotation (one round unless a stronger rotation was asked for).
+constexpr int kRefMaxRounds = 3;
+
 void rotate(const float* x, const float* signs, int d, float* y) {
-  for (int i = 0; i < d; ++i) y[i] = (signs[i] < 0.0f) ? -x[i] : x[i];
-  ref_fwht(y, d);
+  for (int i = 0; i < d; ++i) y[i] = x[i];
+  for (int r = 0; r < kRefMaxRounds; ++r) {
+    const float* sg = signs + static_cast<int64_t>(r) * d;
+    if (sg[0] == 0.0f) break;
+    for (int i = 0; i < d; ++i) y[i] = (sg[i] < 0.0f) ? -y[i] : y[i];
+    ref_fwht(y, d);
+  }
 }
 
 }  // namespace
@@ -115,6 +124,17 @@ uint64_t ref_splitmix64_next(uint64_t* state) {
 void ref_rotation_signs(uint64_t seed, int d, float* signs) {
   uint64_t st = seed;
   for (int i = 0; i < d; ++i) signs[i] = (ref_splitmix64_next(&st) >> 63) ? -1.0f : 1.0f;
+}
+
+/* Stronger rotation (reading of SURVEY NEXT-4 / RaBitQ's random orthogonal rotation): `rounds`
+ * successive H * diag(D_r), the signs of round r being outputs r d .. r d + d - 1 of the same
+ * SplitMix64 stream (round 0 equals ref_rotation_signs).  signs: kRefMaxRounds x d entries, the
+ * unused rounds zero. */
+void ref_rotation_signs_rounds(uint64_t seed, int d, int rounds, float* signs) {
+  uint64_t st = seed;
+  for (int r = 0; r < kRefMaxRounds; ++r)
+    for (int i = 0; i < d; ++i)
+      signs[r * d + i] = r < rounds ? ((ref_splitmix64_next(&st) >> 63) ? -1.0f : 1.0f) : 0.0f;
 }
 
 /* Walsh-Hadamard transform, natural order, unnormalised (H H = d I). */

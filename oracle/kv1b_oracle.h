@@ -35,6 +35,11 @@ uint64_t ref_splitmix64_next(uint64_t* state);
 /* Rotation signs D[0..d): state = seed; D[i] = (next() >> 63) ? -1 : +1. */
 void ref_rotation_signs(uint64_t seed, int d, float* signs);
 
+/* Stronger rotation: `rounds` (1..3) successive H * diag(D_r); signs receives 3 x d entries, round r
+ * = outputs r d .. r d + d - 1 of one SplitMix64 stream, unused rounds 0.  Every function below
+ * that takes `signs` reads 3 x d entries and applies the rounds up to the first all-zero one. */
+void ref_rotation_signs_rounds(uint64_t seed, int d, int rounds, float* signs);
+
 /* Unnormalised Walsh-Hadamard transform in natural (Sylvester) order, in place, fp32,
  * butterfly stages h = 1, 2, 4, ..., d/2, each (a, c) -> (a + c, a - c). */
 void ref_fwht(float* x, int d);

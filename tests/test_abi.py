@@ -50,8 +50,15 @@ def test_cache_bytes_host_rules(lib):
 
 
 def test_descriptor_layout_matches_header():
-    # int32 x4, u64, 8 pointers, int64[64]
-    assert ctypes.sizeof(kv.CacheDesc) == 16 + 8 + 8 * 8 + 8 * 64
+    # int32 x4, u64, 8 pointers, int64[64], int32 rotation_rounds + reserved
+    assert ctypes.sizeof(kv.CacheDesc) == 16 + 8 + 8 * 8 + 8 * 64 + 8
+
+
+def test_init_rounds_rejects_bad_round_counts_without_launching(lib):
+    d = kv.CacheDesc()
+    for rounds in (0, 4, -1):
+        assert lib.kv1b_cache_init_rounds(ctypes.byref(d), ctypes.c_void_p(0x10000), 1 << 20, 1, 1, 128, 128, 0, rounds,
+                                          None) == -1
 
 
 def test_init_rejects_bad_arguments_without_launching(lib):

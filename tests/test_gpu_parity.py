@@ -23,10 +23,10 @@ def rand_kv(g, B, n, H, dtype, scale=1.0):
     return K, V
 
 
-def build_cache(B, Hkv, appends, dtype, seed=0, data_seed=1, vscale=1.0, cap=None):
+def build_cache(B, Hkv, appends, dtype, seed=0, data_seed=1, vscale=1.0, cap=None, rounds=1):
     total = sum(appends)
     cap = cap or (total + 127) // 128 * 128
-    cache = kv.Cache(B, Hkv, cap, seed=seed)
+    cache = kv.Cache(B, Hkv, cap, seed=seed, rounds=rounds)
     host = HostKV(B, Hkv, cap)
     g = torch.Generator(device=DEV).manual_seed(data_seed)
     for n in appends:
@@ -410,3 +410,32 @@ def test_topk_ties_take_lowest_indices():
     q = K[:, 50, :, :].clone().view(B, 1, 128) * 0.3
     for k in (10, 200, 450):
         select_check(cache, host, q, 0.3, G, oracle.signs(4), kv.SELECT_TOPK, k=k, where=f"ties k{k}")
+
+
+# ------------------------------------------------------------------ stronger rotation (3 rounds of H D)
+def test_rotation_rounds_signs_plane():
+    c1 = kv.Cache(1, 1, 128, seed=77)
+    c3 = kv.Cache(1, 1, 128, seed=77, rounds=3)
+    s1 = c1.planes()["signs_rounds"].cpu().numpy()
+    s3 = c3.planes()["signs_rounds"].cpu().numpy()
+    assert np.array_equal(s1[0], oracle.signs(77)) and np.count_nonzero(s1[1:]) == 0
+    assert np.array_equal(s3.reshape(-1), oracle.signs(77, rounds=3))
+    with pytest.raises(kv.Kv1bError):
+        kv.Cache(1, 1, 128, seed=77, rounds=4)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_three_rounds_encode_bit_exact_and_attend(dtype):
+    B, Hkv, G = 2, 2, 4
+    cache, host = build_cache(B, Hkv, [700, 1, 33], dtype, seed=41, data_seed=2, rounds=3)
+    D = oracle.signs(41, rounds=3)
+    L = cache.lengths[0]
+    for b in range(B):
+        for h in range(Hkv):
+            assert_planes_equal(gpu_head_planes(cache, b, h, L), host.encode(b, h, D), where=f"3 rounds b{b} h{h}")
+    q = torch.randn((B, Hkv * G, 128), device=DEV, generator=torch.Generator(device=DEV).manual_seed(4)).to(dtype)
+    ref = oracle_attend_all(host, q, D, 0.3, G)
+    for engine in (kv.ATTEND_TENSOR, kv.ATTEND_CUDA_CORE):
+        assert_rows_close(cache.attend(q, 0.3, engine=engine).cpu().numpy(), ref, where=f"3 rounds e{engine}")
+    topp_check(cache, host, q, 0.3, 0.9, G, D)
+    assert cache.status() == 0

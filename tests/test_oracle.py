@@ -620,3 +620,63 @@ def test_select_window_is_always_kept_and_budget_applies_to_the_rest():
         oracle.select(s, oracle.SELECT_TOPK, k=-1)
     with pytest.raises(ValueError):
         oracle.select(s, oracle.SELECT_TOPP, p=0.0)
+
+
+# ------------------------------------------------------------------ stronger rotation (several H D rounds)
+def test_rotation_rounds_signs_continue_one_stream():
+    d = 128
+    s3 = oracle.signs(7, d, rounds=3)
+    assert s3.shape == (3 * d,) and set(np.unique(s3)) <= {-1.0, 1.0}
+    assert np.array_equal(s3[:d], oracle.signs(7, d))  # round 0 is the single-round rotation
+    draws = oracle.splitmix64(7, 3 * d)  # round r = the next d draws of the same stream
+    assert np.array_equal(s3, np.where(draws >> np.uint64(63), -1.0, 1.0).astype(np.float32))
+    assert np.array_equal(oracle.signs(7, d, rounds=2), s3[:2 * d])
+
+
+def test_three_round_key_sketch_against_fp64_matrix():
+    d = 128
+    rng = np.random.default_rng(21)
+    S = oracle.signs(3, d, rounds=3).reshape(3, d).astype(np.float64)
+    H = sylvester(d).astype(np.float64)
+    R = np.eye(d)
+    for r in range(3):
+        R = H @ np.diag(S[r]) @ R  # y = H D_3 H D_2 H D_1 k
+    assert np.allclose(R.T @ R, d ** 3 * np.eye(d))  # orthogonal up to the scale d^3
+    K = rng.standard_normal((150, d)).astype(np.float32)
+    enc = oracle.encode(K, np.zeros_like(K), S.reshape(-1).astype(np.float32))
+    for t in range(K.shape[0]):
+        y = R @ K[t].astype(np.float64)
+        bits = np.array([(enc["bits"][t, i // 32] >> (i % 32)) & 1 for i in range(d)])
+        sure = np.abs(y) > 1e-4 * np.linalg.norm(y)
+        assert np.array_equal(bits[sure], (y[sure] >= 0).astype(bits.dtype))
+        n = np.linalg.norm(K[t].astype(np.float64))
+        cinv = d * n / np.abs(y).sum()  # the same definition for any number of rounds
+        assert abs(enc["cinv"][t] - cinv) <= 1e-5 * cinv
+
+
+def test_three_round_estimator_nearly_unbiased_and_scale_free():
+    d = 128
+    rng = np.random.default_rng(13)
+    k = rng.standard_normal(d).astype(np.float32)
+    q = rng.standard_normal(d).astype(np.float32)
+    qk = float(np.dot(q.astype(np.float64), k.astype(np.float64)))
+    ests = []
+    for seed in range(1000):
+        D = oracle.signs(seed, d, rounds=3)
+        enc = oracle.encode(k[None, :], np.zeros((1, d), np.float32), D)
+        qp = oracle.query_prep(q, D)
+        A, Bc = oracle.score_ints(enc["bits"], qp["planes"])
+        ests.append(oracle.logit(A[0], Bc[0], qp["Sq"], qp["vl"], qp["delta"], enc["norm"][0], enc["cinv"][0], 1.0, d))
+    ests = np.array(ests)
+    sem = ests.std() / math.sqrt(len(ests))
+    assert abs(ests.mean() - qk) <= 4 * sem + 0.02 * abs(qk) + 0.05, (ests.mean(), qk, sem)
+    # a key whose three-round transform has all |y_i| equal: ||y|| = d^1.5 ||k||, so
+    # C = sum|y| / (d ||k||) = d (the single-round value 1 times the extra scale d of two more rounds)
+    S = oracle.signs(5, d, rounds=3)
+    H = sylvester(d).astype(np.float64)
+    R = np.eye(d)
+    for r in range(3):
+        R = H @ np.diag(S[r * d:(r + 1) * d].astype(np.float64)) @ R
+    kk = (R.T @ np.ones(d) / d ** 3).astype(np.float32)  # R kk = (1, ..., 1) up to fp32 rounding
+    enc = oracle.encode(kk[None, :], np.zeros((1, d), np.float32), S)
+    assert abs(1.0 / enc["cinv"][0] - d) <= 1e-4 * d
