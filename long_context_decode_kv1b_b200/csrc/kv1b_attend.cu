@@ -330,12 +330,9 @@ template <int G>
 static cudaError_t launch_attend_t(const AttendParams& p, cudaStream_t stream) {
   const size_t smem = static_cast<size_t>(4) * kThreads * G * 4;
   auto kern = attend_kernel<G>;
-  static bool configured = false;  // per template instance
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<unsigned long long> configured{0};  // per template instance, bit per device
+  const cudaError_t e = configure_smem(reinterpret_cast<const void*>(kern), static_cast<int>(smem), &configured);
+  if (e != cudaSuccess) return e;
   dim3 grid(p.nsplit, p.c.Hkv, p.c.B);
   kern<<<grid, kThreads, smem, stream>>>(p);
   return cudaGetLastError();

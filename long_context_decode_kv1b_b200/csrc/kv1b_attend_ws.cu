@@ -739,13 +739,10 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
 
 template <int G>
 static cudaError_t launch_t(const AttendWsParams& p, cudaStream_t stream) {
-  static bool configured = false;
-  if (!configured) {
-    cudaError_t e = cudaFuncSetAttribute(attend_ws_kernel<G>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
-  cudaError_t e = cudaMemsetAsync(p.counters, 0, sizeof(unsigned) * p.c.B * p.c.Hkv, stream);
+  static std::atomic<unsigned long long> configured{0};  // bit per device
+  cudaError_t e = configure_smem(reinterpret_cast<const void*>(attend_ws_kernel<G>), kSmemBytes, &configured);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(p.counters, 0, sizeof(unsigned) * p.c.B * p.c.Hkv, stream);
   if (e != cudaSuccess) return e;
   attend_ws_kernel<G><<<p.ncta, kBlock, kSmemBytes, stream>>>(p);
   return cudaGetLastError();

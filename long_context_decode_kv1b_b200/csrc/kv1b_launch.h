@@ -1,5 +1,6 @@
 // kv1b_launch.h -- internal host<->device interface: kernel parameter blocks and launchers.
 #pragma once
+#include <atomic>
 #include <cuda.h>  // CUtensorMap (the descriptor type only; encoded through the runtime entry point)
 #include <cuda_runtime.h>
 #include <stdint.h>
@@ -109,6 +110,19 @@ struct ToppParams {
 };
 
 constexpr int kPartStride = 2 + 128;
+
+// cudaFuncSetAttribute(MaxDynamicSharedMemorySize) for `func` once per device of the calling thread
+// (bit d of *done marks device d; devices past 63 set it on every call).
+inline cudaError_t configure_smem(const void* func, int bytes, std::atomic<unsigned long long>* done) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const unsigned long long bit = (dev >= 0 && dev < 64) ? (1ull << dev) : 0ull;
+  if (bit && (done->load(std::memory_order_acquire) & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(func, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && bit) done->fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 // exact attention over a selected token set (kv1b_exact.cu)
 constexpr int kExactItem = 256;  // selected entries per work item

@@ -906,15 +906,12 @@ void kv1b_topp_carve(ToppParams* p, void* ws, int32_t rows, int32_t cap) {
 cudaError_t kv1b_launch_topp(const ToppParams& p, int32_t G, int32_t max_len, cudaStream_t stream) {
   const int R = p.c.B * p.Hq;
   if (R > 65535 || G > 8) return cudaErrorInvalidValue;  // grid y of the row kernels; two groups of 4 heads
-  static bool configured = false;
-  if (!configured) {
-    const cudaError_t e = cudaFuncSetAttribute(topp_resolve_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(kResolveSmem));
-    if (e != cudaSuccess) return e;
-    configured = true;
-  }
+  static std::atomic<unsigned long long> configured{0};  // bit per device
+  cudaError_t e = configure_smem(reinterpret_cast<const void*>(topp_resolve_kernel), static_cast<int>(kResolveSmem),
+                                 &configured);
+  if (e != cudaSuccess) return e;
   const ToppLayout l = topp_layout(R, p.c.cap);
-  cudaError_t e = cudaMemsetAsync(p.rows, 0, l.state_bytes, stream);
+  e = cudaMemsetAsync(p.rows, 0, l.state_bytes, stream);
   if (e != cudaSuccess) return e;
   const dim3 sg(static_cast<unsigned>(p.nchunk), static_cast<unsigned>(R));
   const dim3 bs(kStreamThreads);
