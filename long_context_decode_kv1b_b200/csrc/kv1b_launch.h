@@ -99,6 +99,7 @@ struct ToppParams {
   ToppRowState* rows;        // [R]
   unsigned long long* hist;  // [R][kToppBuckets] masses per bucket
   uint32_t* sub_cnt;         // [R][nsub] selected tokens per sub-chunk (lower buckets, then candidates)
+  uint32_t* sub_off;         // [R][nsub + 1] exclusive prefix of sub_cnt (first output slot per sub-chunk)
   float* part;               // [R][nsub][kPartStride] gather partials per sub-chunk
   float* part2;              // [R][kToppMergeSplit][kPartStride] first-level merge sums
   int32_t nchunk;

@@ -71,6 +71,15 @@ __device__ __forceinline__ int topp_bucket(float t) {
   return t >= -40.0f ? (b < kToppBuckets - 1 ? b : kToppBuckets - 1) : kToppBuckets;
 }
 
+// Top-k bucket (unit masses, so the logit range matters, not the mass range): the float bits of
+// d = m - s >= 0 (non-increasing in s, so non-decreasing in the key order), 128 buckets per binade
+// for d in [2^-8, 2^8); smaller d -> 0, larger -> the last bucket.
+__device__ __forceinline__ int topk_bucket(float s, float m) {
+  const float d = __fsub_rn(m, s);
+  const int b = static_cast<int>(__float_as_uint(d) >> 16) - ((127 - 8) << 7);
+  return b < 0 ? 0 : (b > kToppBuckets - 1 ? kToppBuckets - 1 : b);
+}
+
 __device__ __forceinline__ uint64_t topp_key(float s, int64_t t) {
   const uint32_t u = __float_as_uint(__fadd_rn(s, 0.0f));  // -0 -> +0 so equal logits tie
   const uint32_t asc = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
@@ -255,7 +264,9 @@ __global__ void __launch_bounds__(kStreamThreads, NG == 1 ? 4 : 2) topp_scores_k
 // uh 2^16 + ul (ul < 2^16, uh < 2^17); per bucket the block sums ul and uh separately with 32-bit
 // shared reductions (at most 4096 tokens: no overflow), then adds each non-empty bucket's
 // (sum uh) 2^16 + sum ul to the row's 64-bit histogram.
+template <int MODE>
 __global__ void __launch_bounds__(kStreamThreads) topp_mass_kernel(const ToppParams p) {
+  constexpr bool topk = MODE == KV1B_SELECT_TOPK;
   pdl_wait();
   __shared__ uint32_t s_lo[kToppBuckets], s_hi[kToppBuckets];  // sums of ul and of uh per bucket
   __shared__ unsigned long long s_u[kStreamWarps], s_w[kStreamWarps];
@@ -275,32 +286,54 @@ __global__ void __launch_bounds__(kStreamThreads) topp_mass_kernel(const ToppPar
   const float m = fkey_inv(p.rows[r].maxkey);
   unsigned long long usum = 0ull, wsum = 0ull;
   const int nv = static_cast<int>(t1 - tt0);  // valid tokens of this thread (may be <= 0)
-  const bool topk = p.mode == KV1B_SELECT_TOPK;
-  const int64_t win_hi = static_cast<int64_t>(L) - p.recent;  // tokens >= win_hi (and < sink) are kept
-  uint32_t bkw[8];                             // the 16 buckets as 16-bit pairs
-  #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    int bk = kToppBuckets;
-    if (i < nv) {
-      const float tt = topp_t(v[i], m);
-      const int64_t tok = tt0 + i;
-      if (tok < p.sink || tok >= win_hi) {  // kept window: outside the histogram
-        bk = kToppWinBucket;
-        if (!topk) wsum += topp_mass_t(tt);
-      } else {
-        // Top-k: every token has unit mass, and the tokens below 2^-40 share the last bucket
-        const uint64_t u = topk ? 1ull : topp_mass_t(tt);
-        bk = topp_bucket(tt);
-        if (topk && bk > kToppBuckets - 1) bk = kToppBuckets - 1;
-        if (u) {
-          atomicAdd(&s_lo[bk], static_cast<uint32_t>(u & 0xffffu));
-          atomicAdd(&s_hi[bk], static_cast<uint32_t>(u >> 16));
-          usum += u;
-        }
+  // the kept window in this thread's local indices: i < wlo or i >= whi
+  const int64_t wlo64 = p.sink - tt0, whi64 = static_cast<int64_t>(L) - p.recent - tt0;
+  const int wlo = static_cast<int>(wlo64 < 0 ? 0 : (wlo64 > 16 ? 16 : wlo64));
+  const int whi = static_cast<int>(whi64 < 0 ? 0 : (whi64 > 16 ? 16 : whi64));
+  uint32_t bkw[8];  // the 16 buckets as 16-bit pairs
+  // one token outside the window: Top-k gives every token unit mass in its topk_bucket; Top-p its
+  // integer mass in its topp_bucket
+  auto hist_token = [&](float x) -> int {
+    if (topk) {
+      const int bk = topk_bucket(x, m);
+      atomicAdd(&s_lo[bk], 1u);
+      usum += 1ull;
+      return bk;
+    }
+    const float tt = topp_t(x, m);
+    const int bk = topp_bucket(tt);
+    {
+      const uint64_t u = topp_mass_t(tt);
+      if (u) {
+        atomicAdd(&s_lo[bk], static_cast<uint32_t>(u & 0xffffu));
+        atomicAdd(&s_hi[bk], static_cast<uint32_t>(u >> 16));
+        usum += u;
       }
     }
-    if (i & 1) bkw[i >> 1] |= static_cast<uint32_t>(bk) << 16;
-    else bkw[i >> 1] = static_cast<uint32_t>(bk);
+    return bk;
+  };
+  if (nv >= 16 && wlo == 0 && whi == 16) {  // all 16 tokens valid and outside the window
+    #pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int bk = hist_token(v[i]);
+      if (i & 1) bkw[i >> 1] |= static_cast<uint32_t>(bk) << 16;
+      else bkw[i >> 1] = static_cast<uint32_t>(bk);
+    }
+  } else {
+    #pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      int bk = kToppBuckets;
+      if (i < nv) {
+        if (i < wlo || i >= whi) {  // kept window: outside the histogram
+          bk = kToppWinBucket;
+          if (!topk) wsum += topp_mass_t(topp_t(v[i], m));
+        } else {
+          bk = hist_token(v[i]);
+        }
+      }
+      if (i & 1) bkw[i >> 1] |= static_cast<uint32_t>(bk) << 16;
+      else bkw[i >> 1] = static_cast<uint32_t>(bk);
+    }
   }
   if (nv > 0) {  // whole 32-byte groups stay inside the row (cap % 128 == 0)
     uint4* bo = reinterpret_cast<uint4*>(p.bk + r * p.c.cap + tt0);
@@ -454,9 +487,16 @@ __global__ void __launch_bounds__(kResolveThreads) topp_resolve_kernel(const Top
   extern __shared__ unsigned long long s_kv[];  // [kResolveSmemCand] keys, then masses
   __shared__ uint32_t h_lo[256], h_hi[256];     // bin masses: wrapping low word + carries
   __shared__ unsigned long long s_prefix, s_rem;
+  __shared__ unsigned s_wsum[kResolveThreads / 32];
+  __shared__ unsigned s_carry;
   const int64_t r = blockIdx.x;
   ToppRowState& rs = p.rows[r];
-  if (rs.bstar < 0) return;
+  const int bstar = rs.bstar;
+  if (bstar == -1) {  // empty row
+    if (threadIdx.x == 0) p.sel_cnt[r] = 0;
+    return;
+  }
+  if (bstar >= 0) {  // block-uniform
   const int n = static_cast<int>(rs.ncand);
   const bool on_chip = n <= kResolveSmemCand;
   const bool topk = p.mode == KV1B_SELECT_TOPK;
@@ -554,6 +594,30 @@ __global__ void __launch_bounds__(kResolveThreads) topp_resolve_kernel(const Top
     const unsigned same = __match_any_sync(kFull, ck);
     if (ck >= 0 && lane == __ffs(same) - 1) atomicAdd(&cc[ck], static_cast<unsigned>(__popc(same)));
   }
+  }
+  // exclusive prefix of the row's sub-chunk counts -> sub_off[r][0 .. nsub]; sel_cnt = the total
+  const int warp_s = threadIdx.x >> 5, lane_s = threadIdx.x & 31;
+  const uint32_t* ccs = p.sub_cnt + r * p.nsub;
+  uint32_t* off = p.sub_off + r * (p.nsub + 1);
+  if (threadIdx.x == 0) s_carry = 0u;
+  __syncthreads();  // the candidate counts are in place
+  for (int k0 = 0; k0 < p.nsub; k0 += kResolveThreads) {  // block-uniform
+    const int k = k0 + threadIdx.x;
+    const unsigned c = k < p.nsub ? ccs[k] : 0u;
+    const unsigned incl = warp_incl_scan(c);
+    if (lane_s == 31) s_wsum[warp_s] = incl;
+    __syncthreads();
+    unsigned before = s_carry;
+    for (int w = 0; w < warp_s; ++w) before += s_wsum[w];
+    if (k < p.nsub) off[k] = before + incl - c;
+    __syncthreads();
+    if (threadIdx.x == kResolveThreads - 1) s_carry = before + incl;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    off[p.nsub] = s_carry;
+    p.sel_cnt[r] = static_cast<int32_t>(s_carry);
+  }
 }
 
 // ---------------------------------------------------------------- 6. ordered writes + gather-attend
@@ -574,7 +638,6 @@ __global__ void __launch_bounds__(kStreamThreads, GM <= 4 ? 3 : 2) topp_write_ga
   static_assert(kTok == 4 && kTok * 32 == 128, "a warp covers one 128-token code tile");
   static_assert(kW * kD == kToppSub, "the weight buffer doubles as the cross-warp reduction buffer");
   __shared__ float s_e[GM][kToppSub];               // weights of the selected tokens, then partial sums
-  __shared__ unsigned s_before[kW][GM];
   __shared__ unsigned s_cnt[kW][kPk];
   __shared__ __align__(16) float s_scl[kW][32][4];  // per slice token: group scales and minima as fp32
   __shared__ __align__(16) float s_mnv[kW][32][4];
@@ -586,25 +649,32 @@ __global__ void __launch_bounds__(kStreamThreads, GM <= 4 ? 3 : 2) topp_write_ga
   const int L = p.len[z / c.Hkv];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int64_t t0 = static_cast<int64_t>(sub) * kToppSub;
+  if (t0 >= L) return;  // block-uniform
   const int64_t t1 = t0 + kToppSub < L ? t0 + kToppSub : L;
   const int64_t tt0 = t0 + kTok * threadIdx.x;
-  // independent global reads first: earlier sub-chunks' counts, row states, this thread's logits
-  unsigned before[GM], mask[GM];
+  // this sub-chunk's first output slot and selected count per head (prefix sums by the resolve)
+  unsigned base[GM], total = 0;
+  #pragma unroll
+  for (int h = 0; h < GM; ++h) {
+    base[h] = 0u;
+    if (h < G) {
+      const uint32_t* off = p.sub_off + (row0 + h) * (p.nsub + 1) + sub;
+      base[h] = off[0];
+      total += off[1] - off[0];
+    }
+  }
+  if (total == 0u) return;  // block-uniform: nothing selected here for any of the G heads
+  unsigned mask[GM];
   uint2 bk4[GM];    // this thread's 4 buckets per head (16 bits each)
   float v[GM][4];   // their logits, loaded where the bucket is at most b*
   float mrow[GM];
   const int nv = static_cast<int>(t1 - tt0);
   #pragma unroll
   for (int h = 0; h < GM; ++h) {
-    before[h] = 0u;
     mask[h] = 0u;
     bk4[h] = make_uint2(0xffffffffu, 0xffffffffu);
     mrow[h] = 0.0f;
-    if (h < G) {
-      const uint32_t* cc = p.sub_cnt + (row0 + h) * p.nsub;
-      for (int k = threadIdx.x; k < sub; k += kStreamThreads) before[h] += cc[k];
-      if (nv > 0) bk4[h] = *reinterpret_cast<const uint2*>(p.bk + (row0 + h) * c.cap + tt0);  // inside the row
-    }
+    if (h < G && nv > 0) bk4[h] = *reinterpret_cast<const uint2*>(p.bk + (row0 + h) * c.cap + tt0);  // inside the row
   }
   #pragma unroll
   for (int h = 0; h < GM; ++h) {
@@ -638,13 +708,6 @@ __global__ void __launch_bounds__(kStreamThreads, GM <= 4 ? 3 : 2) topp_write_ga
     incl[w] = warp_incl_scan(pk[w]);
     if (lane == 31) s_cnt[warp][w] = incl[w];
   }
-  #pragma unroll
-  for (int h = 0; h < GM; ++h) {
-    if (h < G) {
-      const unsigned bsum = warp_sum(before[h]);
-      if (lane == 0) s_before[warp][h] = bsum;
-    }
-  }
   __syncthreads();
   float lsum[GM];
   #pragma unroll
@@ -652,15 +715,11 @@ __global__ void __launch_bounds__(kStreamThreads, GM <= 4 ? 3 : 2) topp_write_ga
     lsum[h] = 0.0f;
     if (h < G) {
       const int sh = 16 * (h & 1);
-      // lane w < kW holds warp w's values: chunk base, this warp's prior count, the block total
-      const unsigned bw = lane < kW ? s_before[lane][h] : 0u;
+      // lane w < kW holds warp w's count: this warp's prior count within the block
       const unsigned cw = lane < kW ? (s_cnt[lane][h >> 1] >> sh) & 0xffffu : 0u;
-      const unsigned base = __reduce_add_sync(kFull, bw);
       const unsigned prior = __reduce_add_sync(kFull, lane < warp ? cw : 0u);
-      const unsigned tot = __reduce_add_sync(kFull, cw);
-      if (sub == p.nsub - 1 && threadIdx.x == 0) p.sel_cnt[row0 + h] = static_cast<int32_t>(base + tot);
       const unsigned cnt = __popc(mask[h]);
-      unsigned off = base + prior + ((incl[h >> 1] >> sh) & 0xffffu) - cnt;
+      unsigned off = base[h] + prior + ((incl[h >> 1] >> sh) & 0xffffu) - cnt;
       int32_t* sel = p.sel_idx + (row0 + h) * c.cap;
       #pragma unroll
       for (int i = 0; i < kTok; ++i) {
@@ -673,7 +732,6 @@ __global__ void __launch_bounds__(kStreamThreads, GM <= 4 ? 3 : 2) topp_write_ga
       }
     }
   }
-  if (t0 >= L) return;  // block-uniform; nothing to gather
   __syncwarp();
   // gather over the warp's slices where any head selects a token
   const int64_t head_tok = static_cast<int64_t>(z) * c.cap;
@@ -807,9 +865,11 @@ __global__ void __launch_bounds__(kD) topp_merge_kernel(const ToppParams p) {
   const int k0 = static_cast<int>(static_cast<int64_t>(n) * j / M);
   const int k1 = static_cast<int>(static_cast<int64_t>(n) * (j + 1) / M);
   const float* base = p.part + r * p.nsub * kPartStride;
+  const uint32_t* off = p.sub_off + r * (p.nsub + 1);
   float num = 0.0f, den = 0.0f;
-  #pragma unroll 8
+  #pragma unroll 4
   for (int k = k0; k < k1; ++k) {
+    if (off[k + 1] == off[k]) continue;  // no selected token of the row there: no partial written
     num += base[k * kPartStride + 2 + ch];
     den += base[k * kPartStride + 1];
   }
@@ -856,7 +916,7 @@ cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t sme
   return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
 }
 struct ToppLayout {
-  size_t planes, qvl, qdl, qsq, s, bk, cand, rows, hist, sub_cnt, part, part2, total, state_bytes;
+  size_t planes, qvl, qdl, qsq, s, bk, cand, rows, hist, sub_cnt, sub_off, part, part2, total, state_bytes;
 };
 ToppLayout topp_layout(int32_t rows, int32_t cap) {
   const size_t R = static_cast<size_t>(rows), C = static_cast<size_t>(cap);
@@ -874,6 +934,7 @@ ToppLayout topp_layout(int32_t rows, int32_t cap) {
   l.hist = o;      o += al256(R * kToppBuckets * 8);
   l.sub_cnt = o;   o += al256(R * nsub * 4);
   l.state_bytes = o - l.rows;
+  l.sub_off = o;   o += al256(R * (nsub + 1) * 4);
   l.part = o;      o += al256(R * nsub * kPartStride * 4);
   l.part2 = o;     o += al256(R * kToppMergeSplit * kPartStride * 4);
   l.total = o;
@@ -897,6 +958,7 @@ void kv1b_topp_carve(ToppParams* p, void* ws, int32_t rows, int32_t cap) {
   p->rows = reinterpret_cast<ToppRowState*>(w + l.rows);
   p->hist = reinterpret_cast<unsigned long long*>(w + l.hist);
   p->sub_cnt = reinterpret_cast<uint32_t*>(w + l.sub_cnt);
+  p->sub_off = reinterpret_cast<uint32_t*>(w + l.sub_off);
   p->part = reinterpret_cast<float*>(w + l.part);
   p->part2 = reinterpret_cast<float*>(w + l.part2);
   p->nchunk = static_cast<int32_t>((static_cast<size_t>(cap) + kToppChunk - 1) / kToppChunk);
@@ -922,14 +984,17 @@ cudaError_t kv1b_launch_topp(const ToppParams& p, int32_t G, int32_t max_len, cu
     const dim3 grid((max_len + kScoreTok - 1) / kScoreTok, p.c.Hkv, p.c.B);
     e = G <= 4 ? launch_pdl(topp_scores_kernel<1>, grid, bs, 0, stream, p, G)
                : launch_pdl(topp_scores_kernel<2>, grid, bs, 0, stream, p, G);
-    if (e == cudaSuccess) e = launch_pdl(topp_mass_kernel, sg, bs, 0, stream, p);
+    if (e == cudaSuccess)
+      e = p.mode == KV1B_SELECT_TOPK ? launch_pdl(topp_mass_kernel<KV1B_SELECT_TOPK>, sg, bs, 0, stream, p)
+                                     : launch_pdl(topp_mass_kernel<KV1B_SELECT_TOPP>, sg, bs, 0, stream, p);
     if (e == cudaSuccess) e = launch_pdl(topp_threshold_kernel, dim3(R), dim3(kThresholdThreads), 0, stream, p);
     if (e == cudaSuccess) e = launch_pdl(topp_cand_kernel, sg, bs, 0, stream, p);
-    if (e == cudaSuccess) e = launch_pdl(topp_resolve_kernel, dim3(R), dim3(kResolveThreads), kResolveSmem, stream, p);
   } else {
     topp_threshold_kernel<<<R, kThresholdThreads, 0, stream>>>(p);  // marks every row empty
     e = cudaGetLastError();
   }
+  // select inside the threshold bucket, then every row's sub-chunk offsets and selected count
+  if (e == cudaSuccess) e = launch_pdl(topp_resolve_kernel, dim3(R), dim3(kResolveThreads), kResolveSmem, stream, p);
   if (e != cudaSuccess) return e;
   const dim3 gg(static_cast<unsigned>(p.nsub), static_cast<unsigned>(p.c.B * p.c.Hkv));
   e = G <= 4 ? launch_pdl(topp_write_gather_kernel<4>, gg, bs, 0, stream, p, G)
