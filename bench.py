@@ -36,8 +36,8 @@ ATTEND_SRC = os.path.join(ROOT, "long_context_decode_kv1b_b200", "csrc", "kv1b_a
 # DRAM bytes (read + write) per token x kv-head of one attend kernel launch, from an ncu capture of
 # the c3 workload (same head grouping, cache 218 MB > L2) scaled by the tokens x kv-heads it
 # processed; valid only for the attend source with this SHA-256 (profiles/attend_ws_c3_ncu_full.txt).
-TRAFFIC = {"bytes_per_token_head": (219242752 + 5809664) / 2097408,
-           "source_sha256": "a7bfa674ff63f953700af44ec4d720085ab271393eef73751d78333ff54f9bef"}
+TRAFFIC = {"bytes_per_token_head": (219243264 + 5559040) / 2097408,
+           "source_sha256": "efe375525ce44c83cd3291730547fd83f804bde7896d3e8521633049ec695e72"}
 
 
 def parse_args():

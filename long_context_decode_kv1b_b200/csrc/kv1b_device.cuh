@@ -65,14 +65,21 @@ __device__ __forceinline__ void rotate128(float x[4], const float sgn[4]) {
 // Several rounds y <- H (D_r (.) y) (a stronger rotation): signs holds KV1B_MAX_ROUNDS x 128 entries
 // and a round whose first sign is 0 ends the rotation (one round unless the cache asked for more).
 __device__ __forceinline__ void rotate_rounds(float x[4], const float* signs) {
+  static_assert(KV1B_MAX_ROUNDS == 3, "three round markers below");
   const int lane = threadIdx.x & 31;
+  // the rounds' first signs (the same addresses for every lane: warp-uniform), read together with
+  // round 0's signs so that the count costs no extra dependent load
+  const float f1 = signs[kD], f2 = signs[2 * kD];
+  float sg[4];
+  #pragma unroll
+  for (int j = 0; j < 4; ++j) sg[j] = signs[4 * lane + j];
+  const int rounds = signs[0] == 0.0f ? 0 : (f1 == 0.0f ? 1 : (f2 == 0.0f ? 2 : 3));
   #pragma unroll 1
-  for (int r = 0; r < KV1B_MAX_ROUNDS; ++r) {
-    const float* sr = signs + r * kD;
-    if (sr[0] == 0.0f) break;  // the same address for every lane: warp-uniform
-    float sg[4];
-    #pragma unroll
-    for (int j = 0; j < 4; ++j) sg[j] = sr[4 * lane + j];
+  for (int r = 0; r < rounds; ++r) {
+    if (r > 0) {
+      #pragma unroll
+      for (int j = 0; j < 4; ++j) sg[j] = signs[r * kD + 4 * lane + j];
+    }
     rotate128(x, sg);
   }
 }

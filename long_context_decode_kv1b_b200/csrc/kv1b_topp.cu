@@ -869,9 +869,12 @@ __global__ void __launch_bounds__(kD) topp_merge_kernel(const ToppParams p) {
   float num = 0.0f, den = 0.0f;
   #pragma unroll 4
   for (int k = k0; k < k1; ++k) {
-    if (off[k + 1] == off[k]) continue;  // no selected token of the row there: no partial written
-    num += base[k * kPartStride + 2 + ch];
-    den += base[k * kPartStride + 1];
+    // a sub-chunk without a selected token of the row wrote no partial: its (allocated, unwritten)
+    // entries are read but not used, so the loads of consecutive sub-chunks stay independent
+    const bool has = off[k + 1] != off[k];
+    const float x = base[k * kPartStride + 2 + ch], y = base[k * kPartStride + 1];
+    num = has ? num + x : num;
+    den = has ? den + y : den;
   }
   float* q2 = p.part2 + (r * M + j) * kPartStride;
   q2[2 + ch] = num;
