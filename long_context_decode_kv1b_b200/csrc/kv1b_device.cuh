@@ -73,13 +73,13 @@ __device__ __forceinline__ void rotate_rounds(float x[4], const float* signs) {
   float sg[4];
   #pragma unroll
   for (int j = 0; j < 4; ++j) sg[j] = signs[4 * lane + j];
-  const int rounds = signs[0] == 0.0f ? 0 : (f1 == 0.0f ? 1 : (f2 == 0.0f ? 2 : 3));
+  if (signs[0] == 0.0f) return;
+  rotate128(x, sg);  // round 0, straight-line (every cache has it)
+  const int rounds = f1 == 0.0f ? 1 : (f2 == 0.0f ? 2 : 3);
   #pragma unroll 1
-  for (int r = 0; r < rounds; ++r) {
-    if (r > 0) {
-      #pragma unroll
-      for (int j = 0; j < 4; ++j) sg[j] = signs[r * kD + 4 * lane + j];
-    }
+  for (int r = 1; r < rounds; ++r) {
+    #pragma unroll
+    for (int j = 0; j < 4; ++j) sg[j] = signs[r * kD + 4 * lane + j];
     rotate128(x, sg);
   }
 }

@@ -34,11 +34,12 @@ __global__ void init_kernel(uint64_t seed, int rounds, float* signs, int32_t* le
   if (blockIdx.x == 0 && threadIdx.x < batch) lengths[threadIdx.x] = 0;
 }
 
-// One block per (16-token tile touched by the append, kv-head, sequence); warp r handles tile
-// slot r.  Keys and v_sm are token-major and written directly; the 4-bit codes of the tile are
-// staged in shared memory and then written as whole 32-bit words of the channel-major code plane
-// (read-modify-write keeps the nibbles of tokens already in the tile).
-__global__ void __launch_bounds__(512) encode_kernel(const EncodeParams p) {
+// One block per (16-token tile touched by the append, kv-head, sequence); warp r < 16 encodes the
+// key of tile slot r and warp 16 + r its value, so the two chains run side by side.  Keys and v_sm
+// are token-major and written directly; the 4-bit codes of the tile are staged in shared memory and
+// then written as whole 32-bit words of the channel-major code plane (read-modify-write keeps the
+// nibbles of tokens already in the tile; the old words are read at the start).
+__global__ void __launch_bounds__(1024) encode_kernel(const EncodeParams p) {
   __shared__ uint8_t codes[16][kD];
   __shared__ int s_new[16];
   const int b = blockIdx.z, h = blockIdx.y;
@@ -47,12 +48,23 @@ __global__ void __launch_bounds__(512) encode_kernel(const EncodeParams p) {
   const int64_t tile = first_tile + blockIdx.x;
   if (tile > last_tile) return;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int64_t pos = tile * 16 + warp;
+  const int slot = warp & 15;
+  const bool value_warp = warp >= 16;
+  const int64_t pos = tile * 16 + slot;
   const bool is_new = pos >= L0 && pos < L0 + p.n_new;
-  if (lane == 0) s_new[warp] = is_new;
+  if (lane == 0 && !value_warp) s_new[slot] = is_new;
   const int64_t head_base = (static_cast<int64_t>(b) * p.Hkv + h) * p.cap;  // token index base
+  // the code words this block rewrites: thread = (channel, half of the 16 tokens)
+  uint32_t* dst = nullptr;
+  uint32_t old_word = 0u;
+  if (threadIdx.x < 256) {
+    const int ch = threadIdx.x >> 1, half = threadIdx.x & 1;
+    const int64_t seg = static_cast<int64_t>(b) * p.Hkv + h;
+    dst = p.v_codes + ((seg * (p.cap / 128) + tile / 8) * kD + ch) * 16 + (tile & 7) * 2 + half;
+    old_word = *dst;
+  }
 
-  if (is_new) {
+  if (is_new && !value_warp) {
     const int64_t t = pos - L0;
     const int64_t row = static_cast<int64_t>(b) * p.sb + t * p.st + static_cast<int64_t>(h) * p.sh;
     int flags = 0;
@@ -81,6 +93,13 @@ __global__ void __launch_bounds__(512) encode_kernel(const EncodeParams p) {
       p.k_norm[head_base + pos] = nrm;
       p.k_cinv[head_base + pos] = cinv;
     }
+    flags = static_cast<int>(__reduce_or_sync(kFull, static_cast<unsigned>(flags)));
+    if (lane == 0 && flags) atomicOr(p.status, flags);
+  }
+  if (is_new && value_warp) {
+    const int64_t t = pos - L0;
+    const int64_t row = static_cast<int64_t>(b) * p.sb + t * p.st + static_cast<int64_t>(h) * p.sh;
+    int flags = 0;
     // ---- value codes
     float v[4];
     load4(p.v, row + 4 * lane, p.dtype, v);
@@ -108,7 +127,7 @@ __global__ void __launch_bounds__(512) encode_kernel(const EncodeParams p) {
         const float fl = floorf(__fadd_rn(__fdiv_rn(__fsub_rn(v[r], mf), sf), 0.5f));
         c = !(fl > 0.0f) ? 0 : (fl >= 15.0f ? 15 : static_cast<int>(fl));
       }
-      codes[warp][4 * lane + r] = static_cast<uint8_t>(c);
+      codes[slot][4 * lane + r] = static_cast<uint8_t>(c);
     }
     if ((lane & 7) == 0) p.v_sm[(head_base + pos) * 4 + (lane >> 3)] = scale_bits | (min_bits << 16);
     flags = static_cast<int>(__reduce_or_sync(kFull, static_cast<unsigned>(flags)));
@@ -120,12 +139,7 @@ __global__ void __launch_bounds__(512) encode_kernel(const EncodeParams p) {
   // of the 8), read-modify-write keeps the nibbles of tokens already in the cache.
   if (threadIdx.x < 256) {
     const int ch = threadIdx.x >> 1, half = threadIdx.x & 1;
-    const int64_t seg = static_cast<int64_t>(b) * p.Hkv + h;
-    uint32_t* dst = p.v_codes + ((seg * (p.cap / 128) + tile / 8) * kD + ch) * 16 + (tile & 7) * 2 + half;
-    bool all_new = true;
-    #pragma unroll
-    for (int j = 0; j < 8; ++j) all_new = all_new && s_new[8 * half + j];
-    uint32_t w = all_new ? 0u : *dst;
+    uint32_t w = old_word;
     #pragma unroll
     for (int j = 0; j < 8; ++j) {
       if (s_new[8 * half + j]) {
@@ -152,6 +166,6 @@ cudaError_t kv1b_launch_init(uint64_t seed, int32_t rounds, float* signs, int32_
 
 cudaError_t kv1b_launch_encode(const EncodeParams& p, int64_t max_tiles, cudaStream_t stream) {
   dim3 grid(static_cast<unsigned>(max_tiles), p.Hkv, p.B);
-  encode_kernel<<<grid, 512, 0, stream>>>(p);
+  encode_kernel<<<grid, 1024, 0, stream>>>(p);
   return cudaGetLastError();
 }
