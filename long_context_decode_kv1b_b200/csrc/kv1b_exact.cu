@@ -8,7 +8,9 @@
 //  1. plan: one block turns the rows' counts n_r into work items of kExactItem selected entries
 //     (item_off[r] = sum over earlier rows of ceil(n_r / kExactItem));
 //  2. a persistent grid (a few blocks per SM) strides over the items: each of a block's 8 warps takes
-//     every 8th entry of the item, 4 tokens in flight; lane l loads channels 4l..4l+3 of the token's
+//     every 8th entry of the item (its 32 token indices fetched at once, one per lane), in rounds of
+//     8 tokens (4 for fp32 rows) with the next round's loads in flight; lane l loads channels
+//     4l..4l+3 of the token's
 //     key and value row (fp32 after exact conversion), the logit z = (scale log2 e) q.k is a butterfly
 //     sum (the same bits in every lane), and an online softmax in log2 units accumulates
 //     sum 2^(z - m) v; the warps combine into one partial (m, l, o[128]) per item;
@@ -16,13 +18,14 @@
 //     set).
 // An index outside [0, min(length[b], kv_tokens)) is skipped and flagged in the cache status word;
 // no memory outside the given rows is read.
+#include <type_traits>
+
 #include "kv1b_device.cuh"
 #include "kv1b_launch.h"
 
 namespace kv1b {
 
 constexpr int kExactWarps = 8;
-constexpr int kExactInFlight = 4;  // tokens per warp loaded before their logits are formed
 constexpr int kPlanThreads = 1024;
 
 __device__ __forceinline__ int row_count(const ExactParams& p, int64_t r) {
@@ -59,7 +62,39 @@ __global__ void __launch_bounds__(kPlanThreads) exact_plan_kernel(const ExactPar
 }
 
 // ---------------------------------------------------------------- 2. items
+// One token's 4 channels of this lane, raw: 8 bytes for 16-bit rows, 16 bytes for fp32 rows.
+template <int KVD>
+struct RawRow {
+  using T = typename std::conditional<KVD == KV1B_DTYPE_F32, float4, uint2>::type;
+  static __device__ __forceinline__ T load(const void* base, int64_t elem_off) {
+    if constexpr (KVD == KV1B_DTYPE_F32) {
+      return __ldg(reinterpret_cast<const float4*>(static_cast<const float*>(base) + elem_off));
+    } else {
+      return __ldg(reinterpret_cast<const uint2*>(static_cast<const uint16_t*>(base) + elem_off));
+    }
+  }
+  static __device__ __forceinline__ void to_f32(const T& r, float x[4]) {
+    if constexpr (KVD == KV1B_DTYPE_F32) {
+      x[0] = r.x; x[1] = r.y; x[2] = r.z; x[3] = r.w;
+    } else {
+      const uint32_t h[4] = {r.x & 0xffffu, r.x >> 16, r.y & 0xffffu, r.y >> 16};
+      #pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        if constexpr (KVD == KV1B_DTYPE_BF16) x[c] = __uint_as_float(h[c] << 16);
+        else x[c] = __half2float(__ushort_as_half(static_cast<unsigned short>(h[c])));
+      }
+    }
+  }
+};
+
+// Each warp takes entries e0 + warp + 8 j (j < 32) of its item: lane j holds entry j's token index;
+// rounds of U tokens are loaded one round ahead of the one being reduced.
+template <int KVD>
 __global__ void __launch_bounds__(kExactWarps * 32) exact_kernel(const ExactParams p, int rows) {
+  constexpr int U = KVD == KV1B_DTYPE_F32 ? 4 : 8;  // tokens per round (registers for 2 rounds in flight)
+  using R = RawRow<KVD>;
+  using Raw = typename R::T;
+  static_assert(kExactItem == kExactWarps * 32, "a warp holds its item entries' indices one per lane");
   __shared__ float s_m[kExactWarps], s_l[kExactWarps];
   __shared__ float s_acc[kExactWarps][kD];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -80,44 +115,55 @@ __global__ void __launch_bounds__(kExactWarps * 32) exact_kernel(const ExactPara
     const int e0 = (item - p.item_off[r]) * kExactItem;
     const int e1 = e0 + kExactItem < n ? e0 + kExactItem : n;
     const int64_t lim = p.len[b] < p.kv_tokens ? p.len[b] : p.kv_tokens;
+    // this warp's entries: e0 + warp + 8 j for j < cnt
+    const int cnt = e1 - e0 - warp > 0 ? (e1 - e0 - warp + kExactWarps - 1) / kExactWarps : 0;
+    const int64_t my_t = lane < cnt ? static_cast<int64_t>(p.sel[r * p.cap + e0 + warp + kExactWarps * lane]) : -1;
+    const bool my_ok = lane < cnt && my_t >= 0 && my_t < lim;
+    bad |= lane < cnt && !my_ok;
     float qv[4];
     load4(p.q, r * kD + 4 * lane, p.q_dtype, qv);
     #pragma unroll
     for (int c = 0; c < 4; ++c) qv[c] = __fmul_rn(qv[c], p.qscale);  // logits in log2 units
-    const int32_t* sl = p.sel + r * p.cap;
     const int64_t kv_off = static_cast<int64_t>(b) * p.sb + static_cast<int64_t>(kvh) * p.sh + 4 * lane;
     float m = -INFINITY, l = 0.0f;
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-    for (int i = e0 + warp; i < e1; i += kExactWarps * kExactInFlight) {  // warp-uniform
-      float kx[kExactInFlight][4], vx[kExactInFlight][4];
-      bool ok[kExactInFlight];
+    Raw kr[U], vr[U];
+    bool ok[U];
+    auto issue = [&](int j0) {  // loads of entries j0 .. j0 + U - 1 of this warp
       #pragma unroll
-      for (int u = 0; u < kExactInFlight; ++u) {
-        const int ii = i + u * kExactWarps;
-        ok[u] = false;
-        #pragma unroll
-        for (int c = 0; c < 4; ++c) kx[u][c] = vx[u][c] = 0.0f;
-        if (ii < e1) {
-          const int64_t t = sl[ii];
-          if (t >= 0 && t < lim) {
-            ok[u] = true;
-            load4(p.k, kv_off + t * p.st, p.kv_dtype, kx[u]);
-            load4(p.v, kv_off + t * p.st, p.kv_dtype, vx[u]);
-          } else {
-            bad = true;
-          }
+      for (int u = 0; u < U; ++u) {
+        const int j = j0 + u;
+        const int64_t t = __shfl_sync(kFull, my_t, j & 31);
+        ok[u] = __shfl_sync(kFull, my_ok, j & 31) && j < cnt;
+        if (ok[u]) {
+          kr[u] = R::load(p.k, kv_off + t * p.st);
+          vr[u] = R::load(p.v, kv_off + t * p.st);
         }
       }
-      float z[kExactInFlight];
+    };
+    if (cnt > 0) issue(0);
+    for (int j0 = 0; j0 < cnt; j0 += U) {  // warp-uniform
+      Raw kc[U], vc[U];
+      bool okc[U];
+      #pragma unroll
+      for (int u = 0; u < U; ++u) {
+        kc[u] = kr[u];
+        vc[u] = vr[u];
+        okc[u] = ok[u];
+      }
+      if (j0 + U < cnt) issue(j0 + U);  // the next round in flight
+      float z[U];
       float mx = m;
       #pragma unroll
-      for (int u = 0; u < kExactInFlight; ++u) {
-        float d = __fmul_rn(qv[0], kx[u][0]);
+      for (int u = 0; u < U; ++u) {
+        float kx[4];
+        R::to_f32(kc[u], kx);
+        float d = __fmul_rn(qv[0], kx[0]);
         #pragma unroll
-        for (int c = 1; c < 4; ++c) d = __fmaf_rn(qv[c], kx[u][c], d);
+        for (int c = 1; c < 4; ++c) d = __fmaf_rn(qv[c], kx[c], d);
         #pragma unroll
         for (int o = 16; o >= 1; o >>= 1) d = __fadd_rn(d, __shfl_xor_sync(kFull, d, o));  // same in every lane
-        z[u] = ok[u] ? d : -INFINITY;
+        z[u] = okc[u] ? d : -INFINITY;
         mx = fmaxf(mx, z[u]);
       }
       if (mx > m) {  // warp-uniform: rescale to the new reference
@@ -128,12 +174,14 @@ __global__ void __launch_bounds__(kExactWarps * 32) exact_kernel(const ExactPara
         m = mx;
       }
       #pragma unroll
-      for (int u = 0; u < kExactInFlight; ++u) {
-        if (ok[u]) {
+      for (int u = 0; u < U; ++u) {
+        if (okc[u]) {
+          float vx[4];
+          R::to_f32(vc[u], vx);
           const float pu = exp2f(__fsub_rn(z[u], m));
           l = __fadd_rn(l, pu);
           #pragma unroll
-          for (int c = 0; c < 4; ++c) acc[c] = __fmaf_rn(pu, vx[u][c], acc[c]);
+          for (int c = 0; c < 4; ++c) acc[c] = __fmaf_rn(pu, vx[c], acc[c]);
         }
       }
     }
@@ -239,7 +287,13 @@ void kv1b_exact_carve(ExactParams* p, void* ws, int32_t rows) {
 cudaError_t kv1b_launch_exact(const ExactParams& p, int32_t rows, int32_t num_sms, cudaStream_t stream) {
   if (rows < 1) return cudaErrorInvalidValue;
   exact_plan_kernel<<<1, kPlanThreads, 0, stream>>>(p, rows);
-  exact_kernel<<<4 * (num_sms > 0 ? num_sms : 1), kExactWarps * 32, 0, stream>>>(p, rows);
+  const unsigned grid = 4u * static_cast<unsigned>(num_sms > 0 ? num_sms : 1);
+  if (p.kv_dtype == KV1B_DTYPE_F32)
+    exact_kernel<KV1B_DTYPE_F32><<<grid, kExactWarps * 32, 0, stream>>>(p, rows);
+  else if (p.kv_dtype == KV1B_DTYPE_BF16)
+    exact_kernel<KV1B_DTYPE_BF16><<<grid, kExactWarps * 32, 0, stream>>>(p, rows);
+  else
+    exact_kernel<KV1B_DTYPE_F16><<<grid, kExactWarps * 32, 0, stream>>>(p, rows);
   exact_merge_kernel<<<rows, kMergeThreads, 0, stream>>>(p);
   return cudaGetLastError();
 }
