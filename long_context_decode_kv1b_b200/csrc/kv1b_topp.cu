@@ -34,7 +34,8 @@ constexpr int kTokPerThread = kToppChunk / kStreamThreads;  // contiguous tokens
 static_assert(kTokPerThread == 16, "the streaming kernels hold 16 tokens per thread");
 constexpr int kScoreTok = 2048;          // tokens per block of the score kernel
 constexpr int kResolveThreads = 1024;
-constexpr int kResolveSmemCand = 12288;  // candidates whose keys and masses the resolve keeps on chip
+constexpr int kResolveSmemCand = 4096;   // candidates whose keys and masses the resolve keeps on chip
+                                         // (64 KB: three resolve blocks per SM)
 constexpr size_t kResolveSmem = static_cast<size_t>(kResolveSmemCand) * 16;
 
 __device__ __forceinline__ float topp_t(float s, float m) { return __fmul_rn(__fsub_rn(s, m), kL2e); }
@@ -489,6 +490,7 @@ __global__ void __launch_bounds__(kResolveThreads) topp_resolve_kernel(const Top
   __shared__ unsigned long long s_prefix, s_rem;
   __shared__ unsigned s_wsum[kResolveThreads / 32];
   __shared__ unsigned s_carry;
+  __shared__ unsigned long long s_diff[kResolveThreads / 32];
   const int64_t r = blockIdx.x;
   ToppRowState& rs = p.rows[r];
   const int bstar = rs.bstar;
@@ -514,11 +516,27 @@ __global__ void __launch_bounds__(kResolveThreads) topp_resolve_kernel(const Top
       smass[i] = topk ? 1ull : topp_mass_t(topp_t(st, m));
     }
   }
+  // leading key bytes shared by every candidate need no pass: start at the highest byte where any
+  // candidate differs from the first (on-chip keys only; otherwise all 8 bytes)
+  int d_top = 7;
+  if (on_chip && n > 0) {
+    __syncthreads();  // the keys are in shared memory
+    unsigned long long x = 0ull;
+    const unsigned long long k0 = skey[0];
+    for (int i = threadIdx.x; i < n; i += kResolveThreads) x |= skey[i] ^ k0;
+    #pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) x |= __shfl_xor_sync(kFull, x, o);
+    if (lane == 0) s_diff[warp] = x;
+    __syncthreads();
+    unsigned long long all = 0ull;
+    for (int w = 0; w < kResolveThreads / 32; ++w) all |= s_diff[w];
+    d_top = all ? (63 - __clzll(static_cast<long long>(all))) / 8 : 0;
+  }
   if (threadIdx.x == 0) {
-    s_prefix = 0;
+    s_prefix = d_top == 7 ? 0ull : (skey[0] >> (8 * (d_top + 1)));  // the bytes every candidate shares
     s_rem = rs.rem;
   }
-  for (int d = 7; d >= 0; --d) {
+  for (int d = d_top; d >= 0; --d) {
     if (threadIdx.x < 256) {
       h_lo[threadIdx.x] = 0u;
       h_hi[threadIdx.x] = 0u;
@@ -536,7 +554,7 @@ __global__ void __launch_bounds__(kResolveThreads) topp_resolve_kernel(const Top
         key = topp_key(st, t);
         u = topk ? 1ull : topp_mass_t(topp_t(st, m));
       }
-      if (u && (d == 7 || (key >> (8 * (d + 1))) == prefix)) {
+      if (u && (d == 7 || (key >> (8 * (d + 1))) == prefix)) {  // (every candidate matches above d_top)
         const int bin = static_cast<int>((key >> (8 * d)) & 255u);
         const uint32_t ulo = static_cast<uint32_t>(u);
         const uint32_t old = atomicAdd(&h_lo[bin], ulo);
