@@ -526,21 +526,27 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
   // < G), ones (g odd, giving Bc) or zeros; k-row 4t + j of k-block kb is channel
   // 32t + 8j + 2kb (+1 for k-rows 16..31), scaled by 2^(3 - ((2kb + hi) & 3)) to undo the
   // in-place bit position.
-  auto prep = [&](int seg) {
+  // Query preparation of segment `seg`'s head h by the calling warp into buffer seg & 1.
+  auto prep_head = [&](int seg, int h) {
     const int par = seg & 1;
-    if (warp < G) {
-      const int b = seg / c.Hkv, kvh = seg - b * c.Hkv;
-      const QueryPrep qp =
-          query_prep_warp(p.q, (static_cast<int64_t>(b) * p.Hq + kvh * G + warp) * kD, p.q_dtype, c.signs);
-      if (lane == 0) {
-        #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          s_planes[par][warp][j] = make_uint4(qp.planes[j][0], qp.planes[j][1], qp.planes[j][2], qp.planes[j][3]);
-        s_vl[par][warp] = qp.vl;
-        s_dl[par][warp] = qp.delta;
-        s_sq[par][warp] = qp.sq;
-      }
+    const int b = seg / c.Hkv, kvh = seg - b * c.Hkv;
+    const QueryPrep qp =
+        query_prep_warp(p.q, (static_cast<int64_t>(b) * p.Hq + kvh * G + h) * kD, p.q_dtype, c.signs);
+    if (lane == 0) {
+      #pragma unroll
+      for (int j = 0; j < 4; ++j)
+        s_planes[par][h][j] = make_uint4(qp.planes[j][0], qp.planes[j][1], qp.planes[j][2], qp.planes[j][3]);
+      s_vl[par][h] = qp.vl;
+      s_dl[par][h] = qp.delta;
+      s_sq[par][h] = qp.sq;
     }
+  };
+  // next_seg >= 0: warps 4 .. 4 + G - 1 also prepare that segment (the CTA's second one) now, so its
+  // switch later skips the preparation (pre = true).
+  auto prep = [&](int seg, bool pre, int next_seg) {
+    const int par = seg & 1;
+    if (!pre && warp < G) prep_head(seg, warp);
+    if (next_seg >= 0 && warp >= 4 && warp < 4 + G) prep_head(next_seg, warp - 4);
     named_bar(1, kThreads);  // reached by every compute warp at the same stage
     const int hb = g >> 1;
     const bool code_col = (g & 1) == 0 && hb < G;
@@ -572,7 +578,9 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
 
   reset();
   int cur_seg = it.seg;
-  if (it.rem > 0) prep(cur_seg);
+  // the CTA's second segment, if its tiles reach one, is prepared at the start with the first
+  const int second_seg = (t_end > t_begin && (t_end - 1) / p.Lt > it.seg) ? it.seg + 1 : -1;
+  if (it.rem > 0) prep(cur_seg, false, second_seg);
   int s = 0;           // stage of the current step
   uint32_t phase = 0;  // parity of the stage's expected completion
   while (it.rem > 0) {
@@ -581,7 +589,7 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
       flush(cur_seg);
       reset();
       cur_seg = it.seg;
-      prep(cur_seg);
+      prep(cur_seg, cur_seg == second_seg, -1);
     }
     if (!mbar_try(&full_bar[s], phase)) mbar_wait(&full_bar[s], phase, &s_abort);
     const uint8_t* st = smem + s * kStageBytes;
