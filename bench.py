@@ -36,8 +36,8 @@ ATTEND_SRC = os.path.join(ROOT, "long_context_decode_kv1b_b200", "csrc", "kv1b_a
 # DRAM bytes (read + write) per token x kv-head of one attend kernel launch, from an ncu capture of
 # the c3 workload (same head grouping, cache 218 MB > L2) scaled by the tokens x kv-heads it
 # processed; valid only for the attend source with this SHA-256 (profiles/attend_ws_c3_ncu_full.txt).
-TRAFFIC = {"bytes_per_token_head": (219243264 + 5559040) / 2097408,
-           "source_sha256": "efe375525ce44c83cd3291730547fd83f804bde7896d3e8521633049ec695e72"}
+TRAFFIC = {"bytes_per_token_head": (219205120 + 5900544) / 2097408,
+           "source_sha256": "8f6aa8ce886d6a38b78738fbf0a649c70d208cd6ac1844a79955be880b1fa892"}
 
 
 def parse_args():
