@@ -11,30 +11,30 @@
 // its "empty" barrier.  The producer's warpgroup gives most of its registers to the compute
 // warpgroups (setmaxnreg), so three compute warps share each SM sub-partition.
 //
-// The compute warps work in 6 pairs; pair p owns 64 tokens of a stage (tile p >> 1, tokens
-// 64 (p & 1) ..), warp half j of the pair owns the 32-token slice j of them for the scores and
-// channels 64 j .. 64 j + 63 for the P.V:
+// The compute warps work in 3 quads; quad q owns tile q of a stage (128 tokens), and warp j of the
+// quad owns the 32-token slice j of it for the scores and value group j (channels 32 j .. 32 j + 31)
+// for the P.V over all 128 tokens:
 //   scores ("RaBitQCache", abstract / key design: binary x INT4 arithmetic): per 16 tokens, four
 //     mma.m16n8k32 s8 products of the key sign bits (A, one AND per register: each byte keeps one
 //     bit in place) with the query's 4-bit codes (B, column 2h = head h scaled to undo the bit
 //     position, column 2h + 1 = ones), so lane (g, t) receives 8 A and 8 Bc of tokens g and g + 8
 //     for head t exactly -- the integers of the popcount form;
 //   softmax: lane (g, t) turns them into head t's logits (log2 units) and probabilities against a
-//     reference maximum shared by the pair and raised only when a logit passes it by kTau (then the
+//     reference maximum shared by the quad and raised only when a logit passes it by kTau (then the
 //     accumulators are rescaled), so every p <= 2^kTau;
 //   weights ("H1B-KV", technical framework: weights from the sketch, then the 4-bit values): lane
 //     (g, t) takes value group t of its tokens for all heads (the heads' p by shuffles within the
 //     lane quad) and forms W = rint(p * scale * 2^E) < 2^32; E is a per-group power of two kept in
-//     step with the largest scale seen (the pair shares it), so the weights of tokens far below the
+//     step with the largest scale seen (the quad shares it), so the weights of tokens far below the
 //     maximum keep many significant bits (a fixed point with fewer bits would round the long tail
 //     of a wide softmax to zero and bias the sum).  stmatrix (.trans, b8) writes the four bytes of
-//     every W into the pair's buffer; ldmatrix gathers them as the A operand (rows = (head, byte));
+//     every W into the quad's buffer; ldmatrix gathers them as the A operand (rows = (head, byte));
 //   P.V: ldmatrix .b8x16.b4x16_p64 expands the staged codes to one byte per code (the B operand,
 //     k = tokens), and mma.m16n8k32 u8 x u8 -> s32 accumulates sum_t W * code per (head, byte,
 //     channel) EXACTLY in 32-bit integers; value = min + scale * code, the min term is summed per
 //     (head, group) in fp32.  The integer accumulators are converted (and rescaled) only when the
 //     reference maximum or a group exponent moves, and at the end of a segment piece.
-// At the end of a segment piece the pairs' partials are combined in shared memory and the CTA
+// At the end of a segment piece the quads' partials are combined in shared memory and the CTA
 // writes one row (m, l, o[128]) per query head; the CTA that writes a segment's last row merges
 // the segment's rows by log-sum-exp into the output (one kernel per attend).
 //
@@ -47,8 +47,8 @@
 namespace kv1b {
 namespace ws {
 
-constexpr int kPairs = 6;
-constexpr int kWarps = 2 * kPairs;          // compute warps
+constexpr int kQuads = 3;
+constexpr int kWarps = 4 * kQuads;          // compute warps
 constexpr int kThreads = kWarps * 32;       // 384 compute threads
 constexpr int kBlock = kThreads + 128;      // + the producer warpgroup
 constexpr int kComputeRegs = 160;           // setmaxnreg: 384 x 160 + 128 x 24 <= 512 x 128 registers (the producer thread may spill)
@@ -62,7 +62,7 @@ constexpr int kTau = 4;                     // lazy-max threshold (log2 units): 
 constexpr int kScaleRoom = 2;               // bits of headroom above the largest scale seen
 constexpr int kNoExp = 100;                 // group exponent before any scale was seen
 constexpr float kNoMax = -1e30f;            // reference maximum before any logit was seen
-constexpr int kMaxAccStages = 8192;         // int32 headroom: 255 * 15 * 64 tokens * 8192 < 2^31
+constexpr int kMaxAccStages = 4096;         // int32 headroom: 255 * 15 * 128 tokens * 4096 < 2^31
 constexpr long long kSpinLimit = 1LL << 24;
 
 // Stage layout (bytes).
@@ -74,16 +74,17 @@ constexpr int kOffCinv = kOffNorm + kStageTok * 4;         // f32 [384]
 constexpr int kOffSm = kOffCinv + kStageTok * 4;           // u32 [384][4]
 constexpr int kStageBytes = (kOffSm + kStageTok * 16 + 1023) / 1024 * 1024;
 constexpr int kWSlice = 16 * 128;                          // one warp's 32 tokens: 16 byte matrices of 8 rows x 16 tokens
-constexpr int kWPair = 2 * kWSlice;
+constexpr int kWQuad = 4 * kWSlice;
 constexpr int kOffW = kStages * kStageBytes;
-constexpr int kRowP = 140;                                 // pair partial row per head: m, l0, l1, -, mid0[4], mid1[4], o[128]
-constexpr int kSmemUsed = kOffW + kPairs * kWPair;
+constexpr int kRowL = 1, kRowMid = 5, kRowO = 24;          // quad partial row per head: m, l[4 warps], mid[4 warps][4 groups], -, o[128]
+constexpr int kRowQ = kRowO + 128;
+constexpr int kSmemUsed = kOffW + kQuads * kWQuad;
 constexpr int kSmemBytes = kSmemUsed + 1024;               // + slack to align the base to 1024 B
 constexpr uint32_t kTxPerTile = kTileTok * 104;            // packed codes 64 B + 40 B of the other planes per token
 static_assert(kSmemBytes <= 227 * 1024, "shared memory per CTA");
 static_assert(kOffW % 1024 == 0 && kStageBytes % 1024 == 0, "TMA 128B-swizzle destinations are 1024-B aligned");
-static_assert(4 * kRowP * 4 <= kWPair, "a pair's partial rows fit its weight buffer");
-static_assert(2 * 4 * 256 * 4 + 64 <= kPairs * kWPair, "the segment merge reuses the weight buffers");
+static_assert(4 * kRowQ * 4 <= kWQuad, "a quad's partial rows fit its weight buffer");
+static_assert(2 * 4 * 256 * 4 + 64 <= kQuads * kWQuad, "the segment merge reuses the weight buffers");
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) { return static_cast<uint32_t>(__cvta_generic_to_shared(p)); }
 
@@ -264,8 +265,8 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
   __shared__ __align__(16) uint4 s_planes[2][4][4];     // double-buffered by segment parity
   __shared__ float s_vl[2][4], s_dl[2][4];
   __shared__ int s_sq[2][4];
-  __shared__ int s_rflag[kPairs][2];                     // a warp of the pair needs a rescale
-  __shared__ float s_xchg[kPairs][2][8];                 // its slice maxima: logits per head, scales per group
+  __shared__ __align__(16) int s_rflag[kQuads][4];      // a warp of the quad needs a rescale
+  __shared__ float s_xchg[kQuads][4][8];                 // its slice maxima: logits per head, scales per group
   __shared__ volatile int s_abort;
   __shared__ int s_merge;
 
@@ -315,43 +316,36 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
   asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kComputeRegs));
 
   const int g = lane >> 2, t = lane & 3;
-  const int pr_ = warp >> 1, jh = warp & 1;  // pair, half
-  const int hh = g & 3;                      // head of this lane's P.V accumulator rows
+  const int qd = warp >> 2, jw = warp & 3;  // quad; slice and value group of this warp
+  const int hh = g & 3;                     // head of this lane's P.V accumulator rows
   const bool lo_bytes = (g >> 2) == 0;       // rows g / g + 8 hold bytes 0 / 2 (else bytes 1 / 3)
   const float qsl = __fmul_rn(__fdiv_rn(p.scale, static_cast<float>(kD)), 0x1.715476p+0f);  // scale/128 * log2 e
-  const int tl = pr_ >> 1;                                  // the pair's tile in the stage
-  const int pbase = tl * kTileTok + (pr_ & 1) * 64;         // the pair's first token in the stage
-  const int sbase = pbase + 32 * jh;                        // this warp's score slice
-  uint8_t* wpair = smem + kOffW + pr_ * kWPair;
-  const uint32_t wpair_s = smem_u32(wpair);
+  const int tl = qd;                                        // the quad's tile in the stage
+  const int sbase = tl * kTileTok + 32 * jw;                // this warp's score slice
+  const uint32_t wq_s = smem_u32(smem + kOffW + qd * kWQuad);
   // stmatrix row address of this lane: matrix (kk, head m = lane >> 3, lo/hi), row rho = lane & 7
   // kept in slot (rho + 2 m) & 7 so that the A-operand gathers below are free of bank conflicts
-  const uint32_t st_addr = wpair_s + jh * kWSlice +
+  const uint32_t st_addr = wq_s + jw * kWSlice +
                            static_cast<uint32_t>((lane >> 3) * 2 * 128 + (((lane & 7) + 2 * (lane >> 3)) & 7) * 16);
-  // A-operand gather for group grp: lane i addresses A row r = (i & 7) + 8 ((i >> 3) & 1) of
-  // k-half kk = i >> 4; row r = (head r & 3, byte r >> 2)
+  // A-operand gather of group jw: lane i addresses A row r = (i & 7) + 8 ((i >> 3) & 1) of k-half
+  // kk = i >> 4 of slice ks; row r = (head r & 3, byte r >> 2)
   const int a_r = (lane & 7) + 8 * ((lane >> 3) & 1), a_kk = lane >> 4;
   const int a_head = a_r & 3, a_byte = a_r >> 2;
-  const uint32_t a_addr = wpair_s + static_cast<uint32_t>(((a_kk * 4 + a_head) * 2 + (a_byte >> 1)) * 128);
-  const int a_rho0 = (a_byte & 1) + 2 * a_head;
-  uint32_t a_pre[2];
-  #pragma unroll
-  for (int gi = 0; gi < 2; ++gi) a_pre[gi] = a_addr + (((a_rho0 + 2 * (2 * jh + gi)) & 7) * 16);
-  // code-tile gathers: lanes 8m .. 8m + 7 address channel rows 64 jh + 8 (2 np + (m >> 1)) + (lane & 7)
-  // of 16-token chunk k16 = (pair chunk) + 2 ks + (m & 1); 128-byte swizzle: chunk ^ (row & 7)
-  const uint32_t c_off = static_cast<uint32_t>(tl * kTileSmem + (64 * jh + 8 * (lane >> 4) + (lane & 7)) * 128);
-  uint32_t c_kx[2];
-  #pragma unroll
-  for (int ks = 0; ks < 2; ++ks) c_kx[ks] = static_cast<uint32_t>(((4 * (pr_ & 1) + 2 * ks + ((lane >> 3) & 1)) ^ (lane & 7)) << 4);
+  const uint32_t a_pre = wq_s + static_cast<uint32_t>(((a_kk * 4 + a_head) * 2 + (a_byte >> 1)) * 128) +
+                         static_cast<uint32_t>((((a_byte & 1) + 2 * a_head + 2 * jw) & 7) * 16);
+  // code-tile gathers: lanes 8m .. 8m + 7 address channel rows 32 jw + 8 (2 np + (m >> 1)) + (lane & 7)
+  // of 16-token chunk 2 ks + (m & 1); 128-byte swizzle: chunk ^ (row & 7) = ((m & 1) ^ (row & 7)) ^ 2 ks
+  const uint32_t c_off = static_cast<uint32_t>(tl * kTileSmem + (32 * jw + 8 * (lane >> 4) + (lane & 7)) * 128);
+  const uint32_t c_kx0 = static_cast<uint32_t>((((lane >> 3) & 1) ^ (lane & 7)) << 4);
 
   // per-lane state
-  float m_w[4], smax_w[4];  // pair-uniform: reference maximum per head, scale bound per group
-  int E_w[4];               // pair-uniform: weight exponent per group
+  float m_w[4], smax_w[4];  // quad-uniform: reference maximum per head, scale bound per group
+  int E_w[4];               // quad-uniform: weight exponent per group
   float m_t, thr_t, s2e_t, smax_t;  // the same for this lane's head t / group t
   float l_t;                // sum p of head t over this lane's tokens
   float mid[4];             // sum p * min of group t, heads 0..3
-  int D[8][4];              // P.V integer accumulators: n-tile (8 channels) x (rows g, g + 8) x 2 channels
-  float F[8][2];            // converted P.V sums of this lane's rows
+  int D[4][4];              // P.V integer accumulators: n-tile (8 channels) x (rows g, g + 8) x 2 channels
+  float F[4][2];            // converted P.V sums of this lane's rows
   uint32_t bq[4][2];        // score-MMA query operand of this segment
   float c1_t, c2_t, c0_t;   // head t logit constants
   bool hv_t;                // head t exists
@@ -371,7 +365,7 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
     smax_t = 0.0f;
     l_t = 0.0f;
     #pragma unroll
-    for (int n = 0; n < 8; ++n) {
+    for (int n = 0; n < 4; ++n) {
       D[n][0] = D[n][1] = D[n][2] = D[n][3] = 0;
       F[n][0] = F[n][1] = 0.0f;
     }
@@ -380,10 +374,9 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
   // Convert the integer accumulators into F (old exponents), then scale F by alpha of this lane's head.
   auto drain = [&](float al) {
     const float wb0 = lo_bytes ? 1.0f : 256.0f, wb2 = lo_bytes ? 65536.0f : 16777216.0f;
-    const float inv0 = exp2i(-(jh ? E_w[2] : E_w[0])), inv1 = exp2i(-(jh ? E_w[3] : E_w[1]));
+    const float inv = exp2i(-sel4(E_w, jw));
     #pragma unroll
-    for (int n = 0; n < 8; ++n) {
-      const float inv = n < 4 ? inv0 : inv1;
+    for (int n = 0; n < 4; ++n) {
       #pragma unroll
       for (int e = 0; e < 2; ++e) {
         const float x = __fmaf_rn(wb2, static_cast<float>(D[n][2 + e]), __fmul_rn(wb0, static_cast<float>(D[n][e])));
@@ -395,7 +388,7 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
     nacc = 0;
   };
 
-  auto prow = [&](int pp, int h) { return reinterpret_cast<float*>(smem + kOffW + pp * kWPair) + h * kRowP; };
+  auto prow = [&](int q, int h) { return reinterpret_cast<float*>(smem + kOffW + q * kWQuad) + h * kRowQ; };
 
   // Log-sum-exp merge of the n CTA rows of segment `seg` (per query head) into the output; uses
   // the weight buffers as scratch.  All heads at once: thread i takes channel i & 127 of heads
@@ -448,14 +441,14 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
     }
   };
 
-  // Segment piece done: each warp puts its share of the pair's partial (m, l, mid, o) per head in
-  // the pair's weight buffer; then thread (head, channel) combines the pairs by log-sum-exp and
+  // Segment piece done: each warp puts its share of the quad's partial (m, l, mid, o) per head in
+  // the quad's weight buffer; then thread (head, channel) combines the quads by log-sum-exp and
   // writes the CTA's row (m, l, o[128] with the mid terms folded in) for slot (segment, piece).
   // Every compute warp reaches this at the same stage.
   auto flush = [&](int seg) {
     drain(1.0f);
     #pragma unroll
-    for (int n = 0; n < 8; ++n)  // rows g (g < 4) and g + 4 of the same head: bytes {0, 2} and {1, 3}
+    for (int n = 0; n < 4; ++n)  // rows g (g < 4) and g + 4 of the same head: bytes {0, 2} and {1, 3}
       #pragma unroll
       for (int e = 0; e < 2; ++e) F[n][e] = __fadd_rn(F[n][e], __shfl_xor_sync(kFull, F[n][e], 16));
     float v[5] = {l_t, mid[0], mid[1], mid[2], mid[3]};
@@ -463,35 +456,38 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
     for (int m = 4; m <= 16; m <<= 1)  // sum over the 8 lanes with the same t
       #pragma unroll
       for (int k = 0; k < 5; ++k) v[k] = __fadd_rn(v[k], __shfl_xor_sync(kFull, v[k], m));
-    named_bar(1, kThreads);  // every pair is done with its weight buffer
+    named_bar(1, kThreads);  // every quad is done with its weight buffer
     if (g == 0) {  // lane t: head t's m and l of this slice, group t's mid of every head
       if (t < G) {
-        if (jh == 0) prow(pr_, t)[0] = m_t == kNoMax ? -INFINITY : m_t;
-        prow(pr_, t)[1 + jh] = v[0];
+        if (jw == 0) prow(qd, t)[0] = m_t == kNoMax ? -INFINITY : m_t;
+        prow(qd, t)[kRowL + jw] = v[0];
       }
       #pragma unroll
-      for (int h = 0; h < G; ++h) prow(pr_, h)[4 + 4 * jh + t] = v[1 + h];
+      for (int h = 0; h < G; ++h) prow(qd, h)[kRowMid + 4 * jw + t] = v[1 + h];
     }
-    if (g < G) {  // head g: channels 64 jh + 8n + 2t + e
-      float* o = prow(pr_, g) + 12 + 64 * jh + 2 * t;
+    if (g < G) {  // head g: channels 32 jw + 8n + 2t + e
+      float* o = prow(qd, g) + kRowO + 32 * jw + 2 * t;
       #pragma unroll
-      for (int n = 0; n < 8; ++n) *reinterpret_cast<float2*>(o + 8 * n) = make_float2(F[n][0], F[n][1]);
+      for (int n = 0; n < 4; ++n) *reinterpret_cast<float2*>(o + 8 * n) = make_float2(F[n][0], F[n][1]);
     }
     named_bar(1, kThreads);
     const int ch = threadIdx.x & 127;
     for (int h = threadIdx.x >> 7; h < G; h += kThreads / 128) {
       float M = -INFINITY;
       #pragma unroll
-      for (int q = 0; q < kPairs; ++q) M = fmaxf(M, prow(q, h)[0]);
+      for (int q = 0; q < kQuads; ++q) M = fmaxf(M, prow(q, h)[0]);
       float num = 0.0f, den = 0.0f;
       if (M != -INFINITY) {
+        const int grp = ch >> 5;
         #pragma unroll
-        for (int q = 0; q < kPairs; ++q) {
+        for (int q = 0; q < kQuads; ++q) {
           const float* r = prow(q, h);
           if (r[0] == -INFINITY) continue;
           const float wt = exp2f(r[0] - M);
-          den = __fmaf_rn(wt, __fadd_rn(r[1], r[2]), den);
-          num = __fmaf_rn(wt, __fadd_rn(r[12 + ch], __fadd_rn(r[4 + (ch >> 5)], r[8 + (ch >> 5)])), num);
+          den = __fmaf_rn(wt, __fadd_rn(__fadd_rn(r[kRowL], r[kRowL + 1]), __fadd_rn(r[kRowL + 2], r[kRowL + 3])), den);
+          const float md = __fadd_rn(__fadd_rn(r[kRowMid + grp], r[kRowMid + 4 + grp]),
+                                     __fadd_rn(r[kRowMid + 8 + grp], r[kRowMid + 12 + grp]));
+          num = __fmaf_rn(wt, __fadd_rn(r[kRowO + ch], md), num);
         }
       }
       const int64_t piece = blockIdx.x - cta_of_tile(wk, static_cast<int64_t>(seg) * wk.Lt);
@@ -594,8 +590,8 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
     if (!mbar_try(&full_bar[s], phase)) mbar_wait(&full_bar[s], phase, &s_abort);
     const uint8_t* st = smem + s * kStageBytes;
     const int rel = it.lt * kTileTok + sbase;          // this slice's first token in the segment
-    const bool pair_on = tl < nt && L > rel - 32 * jh;  // the pair has real tokens in this stage
-    if (pair_on) {
+    const bool quad_on = tl < nt && L > rel - 32 * jw;  // the quad has real tokens in this stage
+    if (quad_on) {
       int lim = L - rel;                                // real tokens of this slice (may be <= 0)
       lim = lim < 32 ? lim : 32;
       if (nacc >= kMaxAccStages) drain(1.0f);
@@ -626,10 +622,11 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
       rare = (fmaxf(fmaxf(s2[0][0], s2[0][1]), fmaxf(s2[1][0], s2[1][1])) > thr_t) |
              (fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1])) > smax_t);
       const bool rare_w = __any_sync(kFull, rare);
-      if (lane == 0) s_rflag[pr_][jh] = rare_w;
-      named_bar(2 + pr_, 64);  // the pair's flags are posted; both warps are done with the weight buffer
-      // ---------------- rare path (pair-uniform): raise a head's reference maximum or a group's scale bound
-      if (rare_w || s_rflag[pr_][jh ^ 1]) {
+      if (lane == 0) s_rflag[qd][jw] = rare_w;
+      named_bar(2 + qd, 128);  // the quad's flags are posted; its warps are done with the weight buffer
+      // ---------------- rare path (quad-uniform): raise a head's reference maximum or a group's scale bound
+      const int4 rf = *reinterpret_cast<const int4*>(s_rflag[qd]);
+      if (rf.x | rf.y | rf.z | rf.w) {
         float mx = fmaxf(fmaxf(s2[0][0], s2[0][1]), fmaxf(s2[1][0], s2[1][1]));
         float sx = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
         #pragma unroll
@@ -638,12 +635,15 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
           sx = fmaxf(sx, __shfl_xor_sync(kFull, sx, m));
         }
         if (g == 0) {
-          s_xchg[pr_][jh][t] = mx;
-          s_xchg[pr_][jh][4 + t] = sx;
+          s_xchg[qd][jw][t] = mx;
+          s_xchg[qd][jw][4 + t] = sx;
         }
-        named_bar(2 + pr_, 64);
-        mx = fmaxf(mx, s_xchg[pr_][jh ^ 1][t]);
-        sx = fmaxf(sx, s_xchg[pr_][jh ^ 1][4 + t]);
+        named_bar(2 + qd, 128);
+        #pragma unroll
+        for (int o = 1; o < 4; ++o) {
+          mx = fmaxf(mx, s_xchg[qd][jw ^ o][t]);
+          sx = fmaxf(sx, s_xchg[qd][jw ^ o][4 + t]);
+        }
         float alpha[4];
         bool changed = false;
         int E_new[4];
@@ -652,13 +652,13 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
           const float mh = __shfl_sync(kFull, mx, h);  // lane h has t = h
           const float sh = __shfl_sync(kFull, sx, h);
           alpha[h] = 1.0f;
-          if (mh > m_w[h] + static_cast<float>(kTau)) {  // pair-uniform
+          if (mh > m_w[h] + static_cast<float>(kTau)) {  // quad-uniform
             alpha[h] = (m_w[h] == kNoMax) ? 0.0f : ex2(m_w[h] - mh);
             m_w[h] = mh;
             changed = true;
           }
           E_new[h] = E_w[h];
-          if (sh > smax_w[h]) {  // pair-uniform; group h
+          if (sh > smax_w[h]) {  // quad-uniform; group h
             const int k = ilog2_pos(sh);
             smax_w[h] = exp2i(k + 1 + kScaleRoom);  // W = p scale 2^E < 2^kTau 2^(k+1+room) 2^E = 2^32
             E_new[h] = 31 - kTau - kScaleRoom - k;
@@ -711,24 +711,20 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
         stsm_x4_t8(st_addr + (kk * 8) * 128, rlo);
         stsm_x4_t8(st_addr + (kk * 8 + 1) * 128, rhi);
       }
-      named_bar(8 + pr_, 64);  // both slices' weights are in the pair's buffer
-      // ---------------- P.V: channels 64 jh .. + 63 over the pair's 64 tokens
+      named_bar(5 + qd, 128);  // the four slices' weights are in the quad's buffer
+      // ---------------- P.V: value group jw (channels 32 jw .. + 31) over the quad's 128 tokens
       const uint32_t ctile = smem_u32(st) + c_off;
       #pragma unroll
-      for (int ks = 0; ks < 2; ++ks) {
-        const uint32_t cks = ctile + c_kx[ks];
+      for (int ks = 0; ks < 4; ++ks) {
+        const uint32_t cks = ctile + (c_kx0 ^ static_cast<uint32_t>(ks << 5));
+        uint32_t a[4];
+        ldsm_x4(a, a_pre + ks * kWSlice);
         #pragma unroll
-        for (int gi = 0; gi < 2; ++gi) {
-          uint32_t a[4];
-          ldsm_x4(a, a_pre[gi] + ks * kWSlice);
-          #pragma unroll
-          for (int np2 = 0; np2 < 2; ++np2) {
-            const int np = 2 * gi + np2;  // n-tiles 2 np, 2 np + 1
-            uint32_t b[4];
-            ldsm_x4_u4(b, cks + np * 2048);
-            imma_u8(D[2 * np], a, b[0], b[1]);
-            imma_u8(D[2 * np + 1], a, b[2], b[3]);
-          }
+        for (int np = 0; np < 2; ++np) {  // n-tiles 2 np, 2 np + 1
+          uint32_t b[4];
+          ldsm_x4_u4(b, cks + np * 2048);
+          imma_u8(D[2 * np], a, b[0], b[1]);
+          imma_u8(D[2 * np + 1], a, b[2], b[3]);
         }
       }
     }
