@@ -36,8 +36,8 @@ ATTEND_SRC = os.path.join(ROOT, "long_context_decode_kv1b_b200", "csrc", "kv1b_a
 # DRAM bytes (read + write) per token x kv-head of one attend kernel launch, from an ncu capture of
 # the c3 workload (same head grouping, cache 218 MB > L2) scaled by the tokens x kv-heads it
 # processed; valid only for the attend source with this SHA-256 (profiles/attend_ws_c3_ncu_full.txt).
-TRAFFIC = {"bytes_per_token_head": (219205120 + 5900544) / 2097408,
-           "source_sha256": "8f6aa8ce886d6a38b78738fbf0a649c70d208cd6ac1844a79955be880b1fa892"}
+TRAFFIC = {"bytes_per_token_head": (219187200 + 7122944) / 2097408,
+           "source_sha256": "5492cc609f5a901ff23d64dde4540e8cd1d2ba8d3af83f8d1e1fe76cc511c423"}
 
 
 def parse_args():
@@ -417,7 +417,7 @@ def run_ours(args):
         result = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": W,
             "ms_per_step": t_max / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-            "dtype": "u1 key bits / u4 value codes; s8 x s8 -> s32 scores; f16 x f16 -> f32 P.V; fp32 softmax",
+            "dtype": "u1 key bits / u4 value codes; s8 x s8 -> s32 scores; fp32 softmax; u8 x u8 -> s32 P.V on 32-bit fixed-point weights",
             "data": "synthetic (seeded torch generators; see long_context_decode_kv1b_b200/workloads.py)",
             "config": {"workload": f"{cfg.name}: {wl.DESCRIPTIONS[cfg.name]}", "batch": cfg.B, "q_heads": cfg.Hq,
                        "kv_heads": cfg.Hkv, "head_dim": 128, "context": cfg.L,
