@@ -143,6 +143,16 @@ __device__ __forceinline__ void tma_codes(void* dst, const CUtensorMap* map, int
       : "memory");
 }
 __device__ __forceinline__ void named_bar(int id, int n) { asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory"); }
+// Named barrier over n threads that also returns the OR of their predicates c.
+__device__ __forceinline__ bool named_bar_or(int id, int n, bool c) {
+  uint32_t r;
+  asm volatile(
+      "{ .reg .pred pc, pr; setp.ne.u32 pc, %3, 0; barrier.cta.red.or.pred pr, %1, %2, pc; selp.u32 %0, 1, 0, pr; }"
+      : "=r"(r)
+      : "r"(id), "r"(n), "r"(static_cast<uint32_t>(c))
+      : "memory");
+  return r != 0;
+}
 
 // Integer tensor-core products (m16n8k32: A 16 x 32, B 32 x 8, D 16 x 8 s32).
 __device__ __forceinline__ void imma_s8(int d[4], const uint32_t a[4], uint32_t b0, uint32_t b1, bool zero) {
@@ -265,7 +275,6 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
   __shared__ __align__(16) uint4 s_planes[2][4][4];     // double-buffered by segment parity
   __shared__ float s_vl[2][4], s_dl[2][4];
   __shared__ int s_sq[2][4];
-  __shared__ __align__(16) int s_rflag[kQuads][4];      // a warp of the quad needs a rescale
   __shared__ float s_xchg[kQuads][4][8];                 // its slice maxima: logits per head, scales per group
   __shared__ volatile int s_abort;
   __shared__ int s_merge;
@@ -621,12 +630,9 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
       }
       rare = (fmaxf(fmaxf(s2[0][0], s2[0][1]), fmaxf(s2[1][0], s2[1][1])) > thr_t) |
              (fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1])) > smax_t);
-      const bool rare_w = __any_sync(kFull, rare);
-      if (lane == 0) s_rflag[qd][jw] = rare_w;
-      named_bar(2 + qd, 128);  // the quad's flags are posted; its warps are done with the weight buffer
-      // ---------------- rare path (quad-uniform): raise a head's reference maximum or a group's scale bound
-      const int4 rf = *reinterpret_cast<const int4*>(s_rflag[qd]);
-      if (rf.x | rf.y | rf.z | rf.w) {
+      // ---------------- rare path (quad-uniform): raise a head's reference maximum or a group's scale
+      // bound.  The barrier also tells that the quad's warps are done with the weight buffer.
+      if (named_bar_or(2 + qd, 128, rare)) {
         float mx = fmaxf(fmaxf(s2[0][0], s2[0][1]), fmaxf(s2[1][0], s2[1][1]));
         float sx = fmaxf(fmaxf(sc[0][0], sc[0][1]), fmaxf(sc[1][0], sc[1][1]));
         #pragma unroll
