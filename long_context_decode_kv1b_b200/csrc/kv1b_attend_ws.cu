@@ -204,15 +204,19 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
 // and 8j + 2kb + 1 (k = 16+4t+j), j = 0..3, each masked in place so that the byte is
 // bit * 2^((2kb + hi) & 3); the query operand carries code * 2^(3 - that), so every product is
 // 8 * bit * code and D = 8 * sum_i bit_i * code_i exactly (the integer A of the popcount form;
-// the columns of ones give 8 * Bc).
+// the columns of ones give 8 * Bc).  K-blocks 0-1 and 2-3 accumulate separately (two chains of two
+// dependent products instead of one of four) and are added at the end.
 __device__ __forceinline__ void score_tile(int d[4], uint32_t wg, uint32_t wg8, const uint32_t (&bq)[4][2]) {
   const uint32_t xg[2] = {wg, __umulhi(wg, 1u << 28)}, xg8[2] = {wg8, __umulhi(wg8, 1u << 28)};  // >> 4
+  int d2[4];
   #pragma unroll
   for (int kb = 0; kb < 4; ++kb) {
     const uint32_t mlo = 0x01010101u << (2 * (kb & 1)), mhi = mlo << 1;
     const uint32_t a[4] = {xg[kb >> 1] & mlo, xg8[kb >> 1] & mlo, xg[kb >> 1] & mhi, xg8[kb >> 1] & mhi};
-    imma_s8(d, a, bq[kb][0], bq[kb][1], kb == 0);
+    imma_s8(kb < 2 ? d : d2, a, bq[kb][0], bq[kb][1], (kb & 1) == 0);
   }
+  #pragma unroll
+  for (int i = 0; i < 4; ++i) d[i] += d2[i];
 }
 __device__ __forceinline__ float exp2i(int e) { return __int_as_float((e + 127) << 23); }
 __device__ __forceinline__ int ilog2_pos(float x) { return static_cast<int>((__float_as_uint(x) >> 23) & 0xff) - 127; }
@@ -717,9 +721,13 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
         stsm_x4_t8(st_addr + (kk * 8) * 128, rlo);
         stsm_x4_t8(st_addr + (kk * 8 + 1) * 128, rhi);
       }
-      named_bar(5 + qd, 128);  // the four slices' weights are in the quad's buffer
-      // ---------------- P.V: value group jw (channels 32 jw .. + 31) over the quad's 128 tokens
+      // ---------------- P.V: value group jw (channels 32 jw .. + 31) over the quad's 128 tokens; the
+      // first slice's codes are in the stage already and load while the quad meets at the barrier
       const uint32_t ctile = smem_u32(st) + c_off;
+      uint32_t bpre[2][4];
+      #pragma unroll
+      for (int np = 0; np < 2; ++np) ldsm_x4_u4(bpre[np], ctile + c_kx0 + np * 2048);
+      named_bar(5 + qd, 128);  // the four slices' weights are in the quad's buffer
       #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
         const uint32_t cks = ctile + (c_kx0 ^ static_cast<uint32_t>(ks << 5));
@@ -728,7 +736,12 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
         #pragma unroll
         for (int np = 0; np < 2; ++np) {  // n-tiles 2 np, 2 np + 1
           uint32_t b[4];
-          ldsm_x4_u4(b, cks + np * 2048);
+          if (ks == 0) {
+            #pragma unroll
+            for (int j = 0; j < 4; ++j) b[j] = bpre[np][j];
+          } else {
+            ldsm_x4_u4(b, cks + np * 2048);
+          }
           imma_u8(D[2 * np], a, b[0], b[1]);
           imma_u8(D[2 * np + 1], a, b[2], b[3]);
         }
