@@ -36,8 +36,8 @@ ATTEND_SRC = os.path.join(ROOT, "long_context_decode_kv1b_b200", "csrc", "kv1b_a
 # DRAM bytes (read + write) per token x kv-head of one attend kernel launch, from an ncu capture of
 # the c3 workload (same head grouping, cache 218 MB > L2) scaled by the tokens x kv-heads it
 # processed; valid only for the attend source with this SHA-256 (profiles/attend_ws_c3_ncu_full.txt).
-TRAFFIC = {"bytes_per_token_head": (219187200 + 7122944) / 2097408,
-           "source_sha256": "5492cc609f5a901ff23d64dde4540e8cd1d2ba8d3af83f8d1e1fe76cc511c423"}
+TRAFFIC = {"bytes_per_token_head": (219180288 + 5096448) / 2097408,
+           "source_sha256": "8edbb7477fc604cbac6f4c384d336e4be2d0e0e3515d4f06fde3727ff6e010ed"}
 
 
 def parse_args():
