@@ -66,6 +66,11 @@ extern "C" {
                                     accumulation) in a persistent kernel, for G in {1, 2, 4}, equal sequence
                                     lengths and an automatic split count; other shapes run the CUDA-core engine */
 #define KV1B_ATTEND_CUDA_CORE 1  /* fp32 FMA on the CUDA cores (split-K grid, any shape) */
+#define KV1B_ATTEND_WS_CLEAN 2   /* OR-ed into the engine: the workspace's merge counters are zero, as every
+                                    kv1b_attend that ran to completion on this workspace leaves them, so the
+                                    call does not zero them first (saves a memset and lets the attend kernel
+                                    start while its predecessor in the stream finishes).  Do not pass it for a
+                                    new workspace, one written by anything else, or after KV1B_STATUS_TIMEOUT. */
 
 /* kv1b_attend_select modes */
 #define KV1B_SELECT_TOPP 0  /* smallest set reaching a fraction p of the estimated attention mass */
@@ -157,7 +162,10 @@ size_t kv1b_attend_workspace_bytes(const kv1b_cache_t* cache, int32_t num_q_head
  * vhat = min + scale_g * code.  A sequence of length 0 gives zeros.
  * ws: device workspace, 256-byte aligned, ws_bytes >= kv1b_attend_workspace_bytes(.., 0).
  * flags: KV1B_ATTEND_TENSOR (default) or KV1B_ATTEND_CUDA_CORE (same result within fp32
- * rounding).  num_splits: 0 chooses the split-K factor; > 0 forces it (testing). */
+ * rounding), optionally | KV1B_ATTEND_WS_CLEAN; any other bit is KV1B_ERR_INVALID_ARG.
+ * num_splits: 0 chooses the split-K factor; > 0 forces it (testing).
+ * The kernels are launched with programmatic stream serialization: they may be scheduled while the
+ * previous kernel in `stream` finishes, and wait for it before touching memory. */
 int kv1b_attend(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,
                 float* out, void* ws, size_t ws_bytes, int32_t flags, int32_t num_splits, void* stream);
 

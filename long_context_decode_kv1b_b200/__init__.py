@@ -19,6 +19,8 @@ HEAD_DIM = 128
 MAX_BATCH = 64
 DTYPE_F32, DTYPE_BF16, DTYPE_F16 = 0, 1, 2
 ATTEND_TENSOR, ATTEND_CUDA_CORE = 0, 1
+ATTEND_WS_CLEAN = 2  # flag: the workspace's merge counters are zero (left so by the previous attend)
+STATUS_TIMEOUT = 4
 STATUS_NONFINITE, STATUS_FP16_SATURATED = 1, 2
 ERRORS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "capacity", -4: "misaligned",
           -5: "workspace too small", -6: "CUDA error"}
@@ -138,6 +140,7 @@ class Cache:
         _check(L.kv1b_cache_init_rounds(ctypes.byref(self.desc), _ptr(self.buffer), nbytes, batch, num_kv_heads,
                                         HEAD_DIM, capacity, seed, rounds, _stream(stream)), "kv1b_cache_init_rounds")
         self._ws = {}
+        self._ws_clean = {}  # num_q_heads -> the attend workspace's merge counters are known to be zero
 
     # ---- views of the device planes (for tests / inspection; layout in include/kv1b.h)
     def _view(self, addr, dtype, shape):
@@ -194,8 +197,11 @@ class Cache:
         if out is None:
             out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
         ws = self.workspace(Hq, 0)
+        # after the first call the workspace's merge counters are zero (each attend leaves them so)
+        flags = engine | (ATTEND_WS_CLEAN if self._ws_clean.get(Hq, False) else 0)
         _check(lib().kv1b_attend(ctypes.byref(self.desc), _ptr(q), _dtype_code(q), Hq, float(scale), _ptr(out),
-                                 _ptr(ws), ws.numel(), engine, num_splits, _stream(stream)), "kv1b_attend")
+                                 _ptr(ws), ws.numel(), flags, num_splits, _stream(stream)), "kv1b_attend")
+        self._ws_clean[Hq] = True
         return out
 
     def attend_topp(self, q: torch.Tensor, scale: float, p: float, out=None, sel=None, cnt=None, stream=None):
@@ -287,6 +293,8 @@ class Cache:
         flags = ctypes.c_int32(0)
         _check(lib().kv1b_read_status(ctypes.byref(self.desc), ctypes.byref(flags), _stream(stream)),
                "kv1b_read_status")
+        if flags.value & STATUS_TIMEOUT:  # a timed-out attend may leave its merge counters set
+            self._ws_clean.clear()
         return flags.value
 
 

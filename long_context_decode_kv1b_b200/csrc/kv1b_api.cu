@@ -221,7 +221,9 @@ int kv1b_attend(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32
   if (!cache_ok(cache) || !q || !out || !ws || !dtype_ok(q_dtype)) return KV1B_ERR_INVALID_ARG;
   const int hc = heads_check(cache, num_q_heads);
   if (hc != KV1B_OK) return hc;
-  if (flags != KV1B_ATTEND_TENSOR && flags != KV1B_ATTEND_CUDA_CORE) return KV1B_ERR_INVALID_ARG;
+  if ((flags & ~(KV1B_ATTEND_CUDA_CORE | KV1B_ATTEND_WS_CLEAN)) != 0) return KV1B_ERR_INVALID_ARG;
+  const bool ws_clean = (flags & KV1B_ATTEND_WS_CLEAN) != 0;
+  flags &= KV1B_ATTEND_CUDA_CORE;  // the engine
   if (num_splits < 0 || num_splits > max_splits(cache)) return KV1B_ERR_INVALID_ARG;
   if (!(scale == scale)) return KV1B_ERR_INVALID_ARG;
   if (!aligned(q, 16) || !aligned(ws, kAlign) || !aligned(out, 16)) return KV1B_ERR_MISALIGNED;
@@ -251,7 +253,14 @@ int kv1b_attend(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32
     w.out = out;
     w.status = cache->d_status;
     w.counters = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + ws_counters_offset(cache, num_q_heads));
-    return cuda_status(kv1b_launch_attend_ws(w, G, static_cast<cudaStream_t>(stream)));
+    return cuda_status(kv1b_launch_attend_ws(w, G, ws_clean, static_cast<cudaStream_t>(stream)));
+  }
+  // this engine does not use the merge counters; they are zeroed here unless the caller says they
+  // are, so that every completed call leaves them zero
+  if (!ws_clean) {
+    const cudaError_t e = cudaMemsetAsync(static_cast<char*>(ws) + ws_counters_offset(cache, num_q_heads), 0,
+                                          ws_counter_bytes(cache), static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) return cuda_status(e);
   }
   kv1b::AttendParams p;
   memset(&p, 0, sizeof(p));

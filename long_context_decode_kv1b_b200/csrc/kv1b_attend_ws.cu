@@ -300,6 +300,7 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
   __syncthreads();
+  pdl_wait();  // every thread, before any global memory access: q and the cache may come from the previous kernel
   TileIt it;  // consume position
   it.seg = static_cast<int>(t_begin / p.Lt);
   it.lt = static_cast<int>(t_begin - static_cast<int64_t>(it.seg) * p.Lt);
@@ -512,14 +513,17 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
       row[2 + ch] = num;
     }
     // The CTA that writes a segment's last piece merges the segment: ticket after the rows are
-    // visible device-wide (the counters are zeroed on the stream before the launch).
+    // visible device-wide.  The counters are zero at launch (a memset on the stream, or left so by
+    // the previous launch on the same workspace): the merging CTA resets its segment's counter.
     __threadfence();
     named_bar(1, kThreads);
     if (threadIdx.x == 0) {
       const int64_t c0 = cta_of_tile(wk, static_cast<int64_t>(seg) * wk.Lt);
       const int64_t c1 = cta_of_tile(wk, static_cast<int64_t>(seg + 1) * wk.Lt - 1);
       const unsigned n = static_cast<unsigned>(c1 - c0 + 1);
-      s_merge = (atomicAdd(p.counters + seg, 1u) == n - 1u) ? static_cast<int>(n) : 0;
+      const bool last = atomicAdd(p.counters + seg, 1u) == n - 1u;
+      s_merge = last ? static_cast<int>(n) : 0;
+      if (last) p.counters[seg] = 0u;  // every piece of the segment has taken its ticket
     }
     named_bar(1, kThreads);
     const int npieces = s_merge;
@@ -761,14 +765,15 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
 }
 
 template <int G>
-static cudaError_t launch_t(const AttendWsParams& p, cudaStream_t stream) {
+static cudaError_t launch_t(const AttendWsParams& p, bool counters_clean, cudaStream_t stream) {
   static std::atomic<unsigned long long> configured{0};  // bit per device
   cudaError_t e = configure_smem(reinterpret_cast<const void*>(attend_ws_kernel<G>), kSmemBytes, &configured);
   if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(p.counters, 0, sizeof(unsigned) * p.c.B * p.c.Hkv, stream);
-  if (e != cudaSuccess) return e;
-  attend_ws_kernel<G><<<p.ncta, kBlock, kSmemBytes, stream>>>(p);
-  return cudaGetLastError();
+  if (!counters_clean) {
+    e = cudaMemsetAsync(p.counters, 0, sizeof(unsigned) * p.c.B * p.c.Hkv, stream);
+    if (e != cudaSuccess) return e;
+  }
+  return launch_pdl(attend_ws_kernel<G>, dim3(p.ncta), dim3(kBlock), kSmemBytes, stream, p);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -818,14 +823,14 @@ void kv1b_ws_plan(int32_t B, int32_t Hkv, int32_t G, int64_t L, int num_sms, int
   (void)G;
 }
 
-cudaError_t kv1b_launch_attend_ws(AttendWsParams& p, int32_t G, cudaStream_t stream) {
+cudaError_t kv1b_launch_attend_ws(AttendWsParams& p, int32_t G, bool counters_clean, cudaStream_t stream) {
   const int64_t tiles = static_cast<int64_t>(p.c.B) * p.c.Hkv * (p.c.cap / ws::kTileTok);
   const cudaError_t e = ws::encode_codes_map(&p.codes_map, p.c.v_codes, tiles);
   if (e != cudaSuccess) return e;
   switch (G) {
-    case 1: return ws::launch_t<1>(p, stream);
-    case 2: return ws::launch_t<2>(p, stream);
-    case 4: return ws::launch_t<4>(p, stream);
+    case 1: return ws::launch_t<1>(p, counters_clean, stream);
+    case 2: return ws::launch_t<2>(p, counters_clean, stream);
+    case 4: return ws::launch_t<4>(p, counters_clean, stream);
     default: return cudaErrorInvalidValue;
   }
 }

@@ -16,6 +16,11 @@
 
 namespace kv1b {
 
+// Programmatic dependent launch: a kernel launched with the programmatic-serialization attribute may
+// be scheduled while its predecessor in the stream is still running; griddepcontrol.wait returns once
+// every prerequisite grid has completed and its memory is visible (a no-op for a plain launch).
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
 constexpr int kD = 128;
 constexpr unsigned kFull = 0xffffffffu;
 

@@ -42,6 +42,7 @@ __global__ void init_kernel(uint64_t seed, int rounds, float* signs, int32_t* le
 __global__ void __launch_bounds__(1024) encode_kernel(const EncodeParams p) {
   __shared__ uint8_t codes[16][kD];
   __shared__ int s_new[16];
+  pdl_wait();  // every block, before any memory access: the inputs may come from the previous kernel
   const int b = blockIdx.z, h = blockIdx.y;
   const int64_t L0 = p.L0[b];
   const int64_t first_tile = L0 / 16, last_tile = (L0 + p.n_new - 1) / 16;
@@ -165,7 +166,6 @@ cudaError_t kv1b_launch_init(uint64_t seed, int32_t rounds, float* signs, int32_
 }
 
 cudaError_t kv1b_launch_encode(const EncodeParams& p, int64_t max_tiles, cudaStream_t stream) {
-  dim3 grid(static_cast<unsigned>(max_tiles), p.Hkv, p.B);
-  encode_kernel<<<grid, 1024, 0, stream>>>(p);
-  return cudaGetLastError();
+  const dim3 grid(static_cast<unsigned>(max_tiles), p.Hkv, p.B);
+  return launch_pdl(encode_kernel, grid, dim3(1024), 0, stream, p);
 }

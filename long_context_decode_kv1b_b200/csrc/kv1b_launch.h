@@ -171,6 +171,24 @@ struct alignas(64) AttendWsParams {
 cudaError_t kv1b_launch_init(uint64_t seed, int32_t rounds, float* signs, int32_t* lengths, int32_t batch,
                              int32_t* status,
                              cudaStream_t stream);
+// Launch with programmatic stream serialization: the kernel may be scheduled while its predecessor
+// in the stream finishes, and must call pdl_wait() before it touches memory.
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                              Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 cudaError_t kv1b_launch_encode(const kv1b::EncodeParams& p, int64_t max_tiles, cudaStream_t stream);
 cudaError_t kv1b_launch_attend(const kv1b::AttendParams& p, int32_t G, int32_t engine, int32_t max_len,
                                cudaStream_t stream);
@@ -188,4 +206,4 @@ cudaError_t kv1b_launch_exact(const kv1b::ExactParams& p, int32_t rows, int32_t 
 bool kv1b_ws_supported(int32_t G);
 void kv1b_ws_plan(int32_t B, int32_t Hkv, int32_t G, int64_t L, int num_sms, int64_t* T, int64_t* Lt, int* ncta,
                   int* max_pieces);
-cudaError_t kv1b_launch_attend_ws(kv1b::AttendWsParams& p, int32_t G, cudaStream_t stream);
+cudaError_t kv1b_launch_attend_ws(kv1b::AttendWsParams& p, int32_t G, bool counters_clean, cudaStream_t stream);

@@ -125,10 +125,6 @@ __device__ __forceinline__ void load16(const float* s, int64_t t0, int64_t t1, f
   }
 }
 
-// Programmatic dependent launch: a kernel launched with the programmatic-serialization attribute may
-// be scheduled while its predecessor in the stream is still running; griddepcontrol.wait returns once
-// every prerequisite grid has completed and its memory is visible (a no-op for a plain launch).
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
 // ---------------------------------------------------------------- 1. logits and row maxima
 // Integer MMA D += A B (16 x 32 s8 by 32 x 8 s8 -> s32).
@@ -920,22 +916,6 @@ using namespace kv1b;
 namespace {
 size_t al256(size_t x) { return (x + 255) / 256 * 256; }
 
-// Launch with programmatic stream serialization (the kernel starts with pdl_wait()).
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
-                       Args... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
-}
 struct ToppLayout {
   size_t planes, qvl, qdl, qsq, s, bk, cand, rows, hist, sub_cnt, sub_off, part, part2, total, state_bytes;
 };

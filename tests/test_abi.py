@@ -68,3 +68,15 @@ def test_init_rejects_bad_arguments_without_launching(lib):
     assert lib.kv1b_cache_init(ctypes.byref(d), ctypes.c_void_p(0x1001), 1 << 20, 1, 1, 128, 128, 0, None) == -4
     assert lib.kv1b_cache_init(ctypes.byref(d), ctypes.c_void_p(0x10000), 16, 1, 1, 128, 128, 0, None) == -5
     assert lib.kv1b_cache_init(ctypes.byref(d), ctypes.c_void_p(0x10000), 1 << 20, 1, 1, 96, 128, 0, None) == -2
+
+
+def test_attend_rejects_unknown_flag_bits_without_launching(lib):
+    # a descriptor that passes the host checks (its pointers are never dereferenced on this path)
+    d = kv.CacheDesc()
+    d.batch, d.num_kv_heads, d.head_dim, d.capacity = 1, 1, 128, 128
+    for name in ("k_bits", "k_norm", "k_cinv", "v_codes", "v_sm", "signs", "d_lengths", "d_status"):
+        setattr(d, name, 0x10000)
+    buf = ctypes.c_void_p(0x20000)
+    for flags in (4, 8, -1):
+        assert lib.kv1b_attend(ctypes.byref(d), buf, kv.DTYPE_F32, 4, ctypes.c_float(0.1), buf, buf, 1 << 20,
+                               flags, 0, None) == -1

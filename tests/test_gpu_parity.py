@@ -3,6 +3,7 @@
 Bit-exact: key bits, N, 1/C, value codes, fp16 scale/min, query planes and grid, popcount
 integers, logits, Top-p index sets.  Attention outputs: <= 1e-3 relative per row (max and l2).
 """
+import ctypes
 import math
 
 import numpy as np
@@ -201,6 +202,30 @@ def test_attend_deterministic_reruns():
     a = cache.attend(q, 0.1).clone()
     b = cache.attend(q, 0.1)
     assert torch.equal(a, b)
+
+
+def test_attend_workspace_counters_left_clean():
+    # a workspace with garbage merge counters: the first call (no flag) zeroes them; every call
+    # leaves them zero, so later calls may pass KV1B_ATTEND_WS_CLEAN and skip the zeroing
+    B, Hkv, G = 2, 2, 4
+    cache, host = build_cache(B, Hkv, [2000, 77], torch.bfloat16, seed=6, data_seed=3)
+    q = torch.randn((B, Hkv * G, 128), device=DEV, generator=torch.Generator(device=DEV).manual_seed(9))
+    ref = oracle_attend_all(host, q, oracle.signs(6), 0.09, G)
+    L = kv.lib()
+    n = L.kv1b_attend_workspace_bytes(ctypes.byref(cache.desc), Hkv * G, 0)
+    ws = torch.full((n,), 0xA5, dtype=torch.uint8, device=DEV)
+    outs = []
+    for flags in (kv.ATTEND_TENSOR, kv.ATTEND_TENSOR | kv.ATTEND_WS_CLEAN, kv.ATTEND_TENSOR | kv.ATTEND_WS_CLEAN,
+                  kv.ATTEND_CUDA_CORE | kv.ATTEND_WS_CLEAN, kv.ATTEND_TENSOR | kv.ATTEND_WS_CLEAN):
+        out = torch.empty((B, Hkv * G, 128), dtype=torch.float32, device=DEV)
+        rc = L.kv1b_attend(ctypes.byref(cache.desc), ctypes.c_void_p(q.data_ptr()), kv.DTYPE_F32, Hkv * G,
+                           ctypes.c_float(0.09), ctypes.c_void_p(out.data_ptr()), ctypes.c_void_p(ws.data_ptr()), n,
+                           flags, 0, None)
+        assert rc == 0
+        assert_rows_close(out.cpu().numpy(), ref, where=f"flags {flags}")
+        outs.append(out)
+    assert torch.equal(outs[0], outs[1]) and torch.equal(outs[0], outs[2]) and torch.equal(outs[0], outs[4])
+    assert cache.status() == 0
 
 
 # ------------------------------------------------------------------------------------- Top-p
