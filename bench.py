@@ -36,8 +36,8 @@ ATTEND_SRC = os.path.join(ROOT, "long_context_decode_kv1b_b200", "csrc", "kv1b_a
 # DRAM bytes (read + write) per token x kv-head of one attend kernel launch, from an ncu capture of
 # the c3 workload (same head grouping, cache 218 MB > L2) scaled by the tokens x kv-heads it
 # processed; valid only for the attend source with this SHA-256 (profiles/attend_ws_c3_ncu_full.txt).
-TRAFFIC = {"bytes_per_token_head": (219180288 + 5096448) / 2097408,
-           "source_sha256": "8edbb7477fc604cbac6f4c384d336e4be2d0e0e3515d4f06fde3727ff6e010ed"}
+TRAFFIC = {"bytes_per_token_head": (219189760 + 5305856) / 2097408,
+           "source_sha256": "30e8db13626aeb70651734a5f5d731fc5d5e7de847c93011d57b17c60fce665b"}
 
 
 def parse_args():
@@ -426,11 +426,11 @@ def run_ours(args):
                              (bytes_per_attend / 1e6), "parallelism": f"independent sequence per GPU x{world}"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
                          "frac": achieved / peak, "traffic": traffic_per_launch(cfg.B * cfg.Hkv * L_mean),
-                         "kernel": "kv1b_attend: counter memset + attend_ws_kernel (merge fused), CUDA events around both",
+                         "kernel": "kv1b_attend: attend_ws_kernel (merge fused; the workspace's merge counters are left zero by the previous call, no memset), CUDA events around the call",
                          "attend_us": att_avg * 1e3, "peak_kind": peak_kind,
                          "frac_of_8tbs": achieved / 8000.0},
             "e2e": e2e,
-            "gpu_launches": 2 * K,  # encode + attend per step (plus one 32-byte counter memset)
+            "gpu_launches": 2 * K,  # encode + attend per step
             "clocks": clocks,
         }
         if alt:
