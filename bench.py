@@ -187,7 +187,7 @@ def barrier(world: int):
 def build_cache(cfg, extra_tokens: int, device, keep_exact: bool = False):
     """The compressed cache of the workload; with keep_exact also the exact bf16 keys / values it
     was built from ([B, capacity, Hkv, 128] in the workload's dtype, for the exact attention over a
-    Top-p set)."""
+    Top-p set); and the CUDA-event time of every prefill kv1b_encode_append (ms, one per chunk)."""
     import torch
 
     import long_context_decode_kv1b_b200 as kv
@@ -199,13 +199,20 @@ def build_cache(cfg, extra_tokens: int, device, keep_exact: bool = False):
     if keep_exact:
         Kx = torch.zeros((cfg.B, cap, cfg.Hkv, 128), dtype=cfg.dtype, device=device)
         Vx = torch.zeros_like(Kx)
+    enc_ms = []
+    stream = torch.cuda.current_stream()
     for start, n in wl.prefill_chunks(cfg):
         K, V = wl.prefill_chunk(cfg, start, n, device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
         cache.append(K, V)
+        e1.record(stream)
+        enc_ms.append((e0, e1))
         if keep_exact:
             Kx[:, start:start + n] = K
             Vx[:, start:start + n] = V
-    return cache, Kx, Vx
+    torch.cuda.synchronize()
+    return cache, Kx, Vx, [a.elapsed_time(b) for a, b in enc_ms]
 
 
 def cpu_baseline(cfg, steps_like: bool):
@@ -256,7 +263,7 @@ def run_ours(args):
     n_alt = 0 if args.no_alt else 5
     extra = W + K + (0 if args.no_e2e else K)
     engine = kv.ATTEND_TENSOR if args.engine == "tensor" else kv.ATTEND_CUDA_CORE
-    cache, Kx, Vx = build_cache(cfg, extra, dev, keep_exact=not args.no_topp)
+    cache, Kx, Vx, enc_ms = build_cache(cfg, extra, dev, keep_exact=not args.no_topp)
     nsteps = W + K
     ks, vs, qs = [], [], []
     for i in range(nsteps + (0 if args.no_e2e else K)):
@@ -433,6 +440,16 @@ def run_ours(args):
             "gpu_launches": 2 * K,  # encode + attend per step
             "clocks": clocks,
         }
+        # the prefill encode (a1-a5 at prefill): K and V rows read, 104 B written per token x kv-head
+        elem = torch.tensor([], dtype=cfg.dtype).element_size()
+        enc_bytes = cfg.B * cfg.Hkv * cfg.L * (2 * 128 * elem + BYTES_PER_TOKEN_HEAD)
+        enc_s = sum(enc_ms) * 1e-3
+        result["encode_prefill"] = {
+            "us": enc_s * 1e6, "calls": len(enc_ms), "tokens_per_call": cfg.chunk,
+            "token_heads_per_s": cfg.B * cfg.Hkv * cfg.L / enc_s, "achieved_gbs": enc_bytes / enc_s / 1e9,
+            "frac": enc_bytes / enc_s / 1e9 / peak, "unit": "GB/s",
+            "bytes_rule": "2 x 128 x element size (K and V rows read) + 104 B written per token x kv-head",
+            "kernel": "kv1b_encode_append over the prefill in chunks, CUDA events around each call"}
         if alt:
             result["alt_engine"] = alt
         if topp:
