@@ -126,7 +126,8 @@ void ref_rotation_signs(uint64_t seed, int d, float* signs) {
   for (int i = 0; i < d; ++i) signs[i] = (ref_splitmix64_next(&st) >> 63) ? -1.0f : 1.0f;
 }
 
-/* Stronger rotation (reading of SURVEY NEXT-4 / RaBitQ's random orthogonal rotation): `rounds`
+/* Stronger rotation (RaBitQCache, abstract / key design: a randomised rotation; RaBitQ proves its
+ * estimator for a random orthogonal one, which several H D rounds approach): `rounds`
  * successive H * diag(D_r), the signs of round r being outputs r d .. r d + d - 1 of the same
  * SplitMix64 stream (round 0 equals ref_rotation_signs).  signs: kRefMaxRounds x d entries, the
  * unused rounds zero. */
