@@ -67,10 +67,12 @@ extern "C" {
                                     lengths and an automatic split count; other shapes run the CUDA-core engine */
 #define KV1B_ATTEND_CUDA_CORE 1  /* fp32 FMA on the CUDA cores (split-K grid, any shape) */
 #define KV1B_ATTEND_WS_CLEAN 2   /* OR-ed into the engine: the workspace's merge counters are zero, as every
-                                    kv1b_attend that ran to completion on this workspace leaves them, so the
-                                    call does not zero them first (saves a memset and lets the attend kernel
-                                    start while its predecessor in the stream finishes).  Do not pass it for a
-                                    new workspace, one written by anything else, or after KV1B_STATUS_TIMEOUT. */
+                                    kv1b_attend that ran to completion on this workspace with the same cache
+                                    shape (batch, kv heads, capacity) and num_q_heads leaves them, so the call
+                                    does not zero them first (saves a memset and lets the attend kernel start
+                                    while its predecessor in the stream finishes).  Do not pass it for a new
+                                    workspace, one used with another shape or written by anything else, or
+                                    after KV1B_STATUS_TIMEOUT. */
 
 /* kv1b_attend_select modes */
 #define KV1B_SELECT_TOPP 0  /* smallest set reaching a fraction p of the estimated attention mass */
