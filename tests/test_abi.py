@@ -1,9 +1,11 @@
 """CPU-only checks of the boundary: the C-ABI library loads and exports every symbol that
-include/kv1b.h declares; host-only size queries behave; the binding's struct mirrors the header.
-No kernel is launched here."""
+include/kv1b.h declares; the header compiles as plain C99 and a C program links against the
+library; host-only size queries behave; the binding's struct mirrors the header.  No kernel is
+launched here."""
 import ctypes
 import os
 import re
+import subprocess
 
 import pytest
 
@@ -80,3 +82,27 @@ def test_attend_rejects_unknown_flag_bits_without_launching(lib):
     for flags in (4, 8, -1):
         assert lib.kv1b_attend(ctypes.byref(d), buf, kv.DTYPE_F32, 4, ctypes.c_float(0.1), buf, buf, 1 << 20,
                                flags, 0, None) == -1
+
+
+def test_header_is_plain_c_and_links(lib, tmp_path):
+    # a C99 program that takes the address of every declared function and calls the host-only ones
+    names = declared_functions()
+    fns = ", ".join(f"(void (*)(void)){n}" for n in names)
+    src = tmp_path / "abi_check.c"
+    src.write_text(f"""#include <stdio.h>
+#include "kv1b.h"
+int main(void) {{
+  void (*fns[])(void) = {{{fns}}};
+  printf("%d %lu %d\\n", kv1b_version(), (unsigned long)kv1b_cache_bytes(1, 1, 128, 128),
+         (int)(sizeof fns / sizeof fns[0]));
+  return 0;
+}}
+""")
+    exe = tmp_path / "abi_check"
+    pkg = os.path.dirname(kv.LIB_PATH)
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I", os.path.join(ROOT, "include"),
+                           "-o", str(exe), str(src), "-L", pkg, "-lkv1b", "-Wl,-rpath," + pkg])
+    out = subprocess.check_output([str(exe)], text=True).split()
+    assert int(out[0]) == lib.kv1b_version()
+    assert int(out[1]) == lib.kv1b_cache_bytes(1, 1, 128, 128)
+    assert int(out[2]) == len(names)
