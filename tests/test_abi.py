@@ -106,3 +106,39 @@ int main(void) {{
     assert int(out[0]) == lib.kv1b_version()
     assert int(out[1]) == lib.kv1b_cache_bytes(1, 1, 128, 128)
     assert int(out[2]) == len(names)
+
+
+def test_binding_passes_workspace_clean_flag_after_first_attend(monkeypatch):
+    # the binding's bookkeeping against a fake library: the first attend on a workspace lets the
+    # library zero the merge counters; later calls say they are clean; a timeout status resets that
+    import types
+
+    import torch
+
+    calls, status = [], [0]
+
+    class FakeLib:
+        def kv1b_attend_workspace_bytes(self, desc, hq, mode):
+            return 4096
+
+        def kv1b_attend(self, desc, q, qdt, hq, scale, out, ws, n, flags, splits, stream):
+            calls.append(flags)
+            return 0
+
+        def kv1b_read_status(self, desc, flags_ref, stream):
+            flags_ref._obj.value = status[0]
+            return 0
+
+    fake = FakeLib()
+    monkeypatch.setattr(kv, "lib", lambda: fake)
+    c = kv.Cache.__new__(kv.Cache)
+    c.desc, c._ws, c._ws_clean, c.device = kv.CacheDesc(), {}, {}, torch.device("cpu")
+    q, out, st = torch.zeros((1, 4, 128)), torch.zeros((1, 4, 128)), types.SimpleNamespace(cuda_stream=0)
+    c.attend(q, 0.1, out=out, stream=st)
+    c.attend(q, 0.1, out=out, stream=st)
+    c.attend(q, 0.1, out=out, engine=kv.ATTEND_CUDA_CORE, stream=st)
+    assert calls == [kv.ATTEND_TENSOR, kv.ATTEND_WS_CLEAN, kv.ATTEND_CUDA_CORE | kv.ATTEND_WS_CLEAN]
+    status[0] = kv.STATUS_TIMEOUT
+    assert c.status(stream=st) == kv.STATUS_TIMEOUT
+    c.attend(q, 0.1, out=out, stream=st)
+    assert calls[-1] == kv.ATTEND_TENSOR
