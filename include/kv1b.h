@@ -252,6 +252,42 @@ int kv1b_query_prep(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, i
 int kv1b_scores(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,
                 int32_t* A, int32_t* Bc, float* s, void* stream);
 
+/* kv1b_scores_probe kernels */
+#define KV1B_PROBE_POPC 0    /* __popc over AND-ed bit-planes (the kv1b_scores hook) */
+#define KV1B_PROBE_ATTEND 1  /* kv1b_attend's persistent tensor-core kernel (the default engine) */
+#define KV1B_PROBE_TOPP 2    /* the score pass of kv1b_attend_topp / kv1b_attend_select */
+
+/* Test hook: the proxy-score integers and logits exactly as one of the library's kernels forms them,
+ * so that the integers of the kernels kv1b_attend and kv1b_attend_topp really run can be compared
+ * bit for bit with A = sum_j 2^j sum_w popc(k_bits_w & P_jw) and Bc = sum_w popc(k_bits_w)
+ * ("RaBitQCache", abstract and key design: binary x INT4 arithmetic).  For every (b, hq) and token
+ * t < length[b], into A, Bc (i32) and s (f32), each [batch][num_q_heads][capacity]:
+ *   KV1B_PROBE_POPC:   A, Bc and the fp32 logit, as kv1b_scores (out, ws, ws_bytes unused);
+ *   KV1B_PROBE_ATTEND: the raw integer tensor-core products 8 A and 8 Bc of the persistent kernel
+ *                      (an exact multiple of 8 when the products are right) and its logit in log2
+ *                      units, s * log2(e) formed in its own fused order (not bit-exact with the fp32
+ *                      logit); the call runs the whole attend and writes out like kv1b_attend.
+ *                      ws: kv1b_attend_workspace_bytes(.., 0) bytes.  KV1B_ERR_UNSUPPORTED unless
+ *                      that kernel would take the call (G in {1, 2, 4}, equal lengths, length > 0);
+ *   KV1B_PROBE_TOPP:   the raw products 8 A and 8 Bc of the Top-p score pass and the fp32 logit it
+ *                      selects with (bit-exact with the oracle's order).  ws: kv1b_attend_workspace_bytes
+ *                      (.., 1) bytes; out unused.
+ * Entries at t >= length[b] are left unspecified.  Asynchronous on `stream`. */
+int kv1b_scores_probe(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,
+                      int32_t kernel, int32_t* A, int32_t* Bc, float* s, float* out, void* ws, size_t ws_bytes,
+                      void* stream);
+
+/* Test hook for the bounded waits of kv1b_attend's persistent kernel: the same call with every
+ * pipeline wait limited to `wait_tries` (1 .. 4096, the product default) suspended tries of at most
+ * 0.5 ms each and, when stall_stage >= 0, each CTA's copy producer stopping before its stage
+ * `stall_stage` as if those copies never arrived.  A CTA whose wait runs out sets
+ * KV1B_STATUS_TIMEOUT, stops issuing copies, lets the copies already in flight land and returns;
+ * out is then invalid, and the next kv1b_attend on this workspace must not pass
+ * KV1B_ATTEND_WS_CLEAN.  KV1B_ERR_UNSUPPORTED unless the persistent kernel would take the call. */
+int kv1b_attend_wait_probe(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads,
+                           float scale, float* out, void* ws, size_t ws_bytes, int32_t wait_tries,
+                           int32_t stall_stage, void* stream);
+
 /* Synchronous: waits for `stream`, then copies the cache's status word to *flags (host). */
 int kv1b_read_status(const kv1b_cache_t* cache, int32_t* flags, void* stream);
 

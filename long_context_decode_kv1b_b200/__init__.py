@@ -21,6 +21,7 @@ DTYPE_F32, DTYPE_BF16, DTYPE_F16 = 0, 1, 2
 ATTEND_TENSOR, ATTEND_CUDA_CORE = 0, 1
 ATTEND_WS_CLEAN = 2  # flag: the workspace's merge counters are zero (left so by the previous attend)
 STATUS_TIMEOUT = 4
+PROBE_POPC, PROBE_ATTEND, PROBE_TOPP = 0, 1, 2
 STATUS_NONFINITE, STATUS_FP16_SATURATED = 1, 2
 ERRORS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "capacity", -4: "misaligned",
           -5: "workspace too small", -6: "CUDA error"}
@@ -29,7 +30,7 @@ ERRORS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "capacity", -4
 SYMBOLS = ("kv1b_cache_bytes", "kv1b_cache_init", "kv1b_cache_init_rounds", "kv1b_encode_append", "kv1b_attend_workspace_bytes",
            "kv1b_attend", "kv1b_attend_noalloc", "kv1b_attend_topp", "kv1b_attend_select",
            "kv1b_attend_selected_exact",
-           "kv1b_query_prep", "kv1b_scores",
+           "kv1b_query_prep", "kv1b_scores", "kv1b_scores_probe", "kv1b_attend_wait_probe",
            "kv1b_read_status", "kv1b_status_string", "kv1b_version")
 
 
@@ -77,6 +78,8 @@ def lib() -> ctypes.CDLL:
                                                           P, P, sz, P]),
             "kv1b_query_prep": (ctypes.c_int, [D, P, i32, i32, P, P, P, P, P]),
             "kv1b_scores": (ctypes.c_int, [D, P, i32, i32, f32, P, P, P, P]),
+            "kv1b_scores_probe": (ctypes.c_int, [D, P, i32, i32, f32, i32, P, P, P, P, P, sz, P]),
+            "kv1b_attend_wait_probe": (ctypes.c_int, [D, P, i32, i32, f32, P, P, sz, i32, i32, P]),
             "kv1b_read_status": (ctypes.c_int, [D, P, P]),
             "kv1b_status_string": (ctypes.c_char_p, [ctypes.c_int]),
             "kv1b_version": (ctypes.c_int, []),
@@ -288,6 +291,36 @@ class Cache:
         _check(lib().kv1b_scores(ctypes.byref(self.desc), _ptr(q), _dtype_code(q), Hq, float(scale), _ptr(A), _ptr(Bc),
                                  _ptr(s), _stream(stream)), "kv1b_scores")
         return {"A": A, "Bc": Bc, "s": s}
+
+    def scores_probe(self, q: torch.Tensor, scale: float, kernel: int, stream=None) -> dict:
+        """The score integers and logits as `kernel` (PROBE_*) forms them (see kv1b_scores_probe):
+        {"A", "Bc", "s"} [B, Hq, capacity], plus "out" for PROBE_ATTEND."""
+        B, Hq, _ = q.shape
+        shape = (B, Hq, self.capacity)
+        A = torch.zeros(shape, dtype=torch.int32, device=q.device)
+        Bc = torch.zeros(shape, dtype=torch.int32, device=q.device)
+        s = torch.zeros(shape, dtype=torch.float32, device=q.device)
+        out = torch.zeros((B, Hq, HEAD_DIM), dtype=torch.float32, device=q.device)
+        ws = self.workspace(Hq, 1 if kernel == PROBE_TOPP else 0) if kernel != PROBE_POPC else None
+        _check(lib().kv1b_scores_probe(ctypes.byref(self.desc), _ptr(q), _dtype_code(q), Hq, float(scale), int(kernel),
+                                       _ptr(A), _ptr(Bc), _ptr(s), _ptr(out), _ptr(ws),
+                                       ws.numel() if ws is not None else 0, _stream(stream)), "kv1b_scores_probe")
+        if kernel == PROBE_ATTEND:  # the probe zeroes the merge counters itself and leaves them zero
+            self._ws_clean[Hq] = True
+        return {"A": A, "Bc": Bc, "s": s, "out": out}
+
+    def attend_wait_probe(self, q: torch.Tensor, scale: float, wait_tries: int, stall_stage: int,
+                          stream=None) -> torch.Tensor:
+        """kv1b_attend's persistent kernel with bounded waits of `wait_tries` tries and, for
+        stall_stage >= 0, the copies of that stage never issued (see kv1b_attend_wait_probe)."""
+        B, Hq, D = q.shape
+        out = torch.zeros((B, Hq, D), dtype=torch.float32, device=q.device)
+        ws = self.workspace(Hq, 0)
+        _check(lib().kv1b_attend_wait_probe(ctypes.byref(self.desc), _ptr(q), _dtype_code(q), Hq, float(scale),
+                                            _ptr(out), _ptr(ws), ws.numel(), int(wait_tries), int(stall_stage),
+                                            _stream(stream)), "kv1b_attend_wait_probe")
+        self._ws_clean[Hq] = stall_stage < 0  # a stalled run may leave the merge counters set
+        return out
 
     def status(self, stream=None) -> int:
         flags = ctypes.c_int32(0)

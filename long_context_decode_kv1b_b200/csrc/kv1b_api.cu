@@ -120,6 +120,55 @@ bool equal_lengths(const kv1b_cache_t* c) {
   return true;
 }
 
+// The persistent tensor-core kernel takes the call: G in {1, 2, 4}, one length for every sequence,
+// a non-empty cache.
+bool ws_engine_applies(const kv1b_cache_t* c, int32_t num_q_heads) {
+  return kv1b_ws_supported(num_q_heads / c->num_kv_heads) && equal_lengths(c) && max_length(c) > 0;
+}
+
+// Parameters of the persistent kernel for this cache and workspace (KV1B_OK or KV1B_ERR_WORKSPACE).
+int ws_params(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale, float* out,
+              void* ws, kv1b::AttendWsParams* w) {
+  const int G = num_q_heads / cache->num_kv_heads;
+  const int64_t maxlen = max_length(cache);
+  memset(w, 0, sizeof(*w));
+  w->c = view(cache);
+  w->q = q;
+  w->q_dtype = q_dtype;
+  w->Hq = num_q_heads;
+  w->scale = scale;
+  w->L = static_cast<int32_t>(maxlen);
+  int ncta = 0, pieces = 0;
+  kv1b_ws_plan(cache->batch, cache->num_kv_heads, G, maxlen, num_sms(), &w->T, &w->Lt, &ncta, &pieces);
+  int64_t Tc, Ltc;
+  int nc, pieces_cap;
+  kv1b_ws_plan(cache->batch, cache->num_kv_heads, G, cache->capacity, num_sms(), &Tc, &Ltc, &nc, &pieces_cap);
+  w->ncta = ncta;
+  w->max_pieces = pieces_cap > pieces ? pieces_cap : pieces;
+  if (w->max_pieces > 256 || static_cast<size_t>(cache->batch) * cache->num_kv_heads * w->max_pieces * G *
+                                    kv1b::kPartStride * 4 > ws_counters_offset(cache, num_q_heads))
+    return KV1B_ERR_WORKSPACE;
+  w->part = static_cast<float*>(ws);
+  w->out = out;
+  w->status = cache->d_status;
+  w->counters = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + ws_counters_offset(cache, num_q_heads));
+  w->wait_tries = kv1b::kWaitTriesDefault;
+  w->stall_stage = -1;
+  return KV1B_OK;
+}
+
+// Shared argument checks of kv1b_attend and its test hooks.
+int attend_args_check(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,
+                      const float* out, const void* ws, size_t ws_bytes) {
+  if (!cache_ok(cache) || !q || !out || !ws || !dtype_ok(q_dtype)) return KV1B_ERR_INVALID_ARG;
+  const int hc = heads_check(cache, num_q_heads);
+  if (hc != KV1B_OK) return hc;
+  if (!(scale == scale)) return KV1B_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(ws, kAlign) || !aligned(out, 16)) return KV1B_ERR_MISALIGNED;
+  if (ws_bytes < kv1b_attend_workspace_bytes(cache, num_q_heads, 0)) return KV1B_ERR_WORKSPACE;
+  return KV1B_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -218,41 +267,18 @@ size_t kv1b_attend_workspace_bytes(const kv1b_cache_t* cache, int32_t num_q_head
 
 int kv1b_attend(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,
                 float* out, void* ws, size_t ws_bytes, int32_t flags, int32_t num_splits, void* stream) {
-  if (!cache_ok(cache) || !q || !out || !ws || !dtype_ok(q_dtype)) return KV1B_ERR_INVALID_ARG;
-  const int hc = heads_check(cache, num_q_heads);
-  if (hc != KV1B_OK) return hc;
+  const int ac = attend_args_check(cache, q, q_dtype, num_q_heads, scale, out, ws, ws_bytes);
+  if (ac != KV1B_OK) return ac;
   if ((flags & ~(KV1B_ATTEND_CUDA_CORE | KV1B_ATTEND_WS_CLEAN)) != 0) return KV1B_ERR_INVALID_ARG;
   const bool ws_clean = (flags & KV1B_ATTEND_WS_CLEAN) != 0;
   flags &= KV1B_ATTEND_CUDA_CORE;  // the engine
   if (num_splits < 0 || num_splits > max_splits(cache)) return KV1B_ERR_INVALID_ARG;
-  if (!(scale == scale)) return KV1B_ERR_INVALID_ARG;
-  if (!aligned(q, 16) || !aligned(ws, kAlign) || !aligned(out, 16)) return KV1B_ERR_MISALIGNED;
-  if (ws_bytes < kv1b_attend_workspace_bytes(cache, num_q_heads, 0)) return KV1B_ERR_WORKSPACE;
   const int64_t maxlen = max_length(cache);
   const int G = num_q_heads / cache->num_kv_heads;
-  if (flags == KV1B_ATTEND_TENSOR && num_splits == 0 && kv1b_ws_supported(G) && equal_lengths(cache) && maxlen > 0) {
+  if (flags == KV1B_ATTEND_TENSOR && num_splits == 0 && ws_engine_applies(cache, num_q_heads)) {
     kv1b::AttendWsParams w;
-    memset(&w, 0, sizeof(w));
-    w.c = view(cache);
-    w.q = q;
-    w.q_dtype = q_dtype;
-    w.Hq = num_q_heads;
-    w.scale = scale;
-    w.L = static_cast<int32_t>(maxlen);
-    int ncta = 0, pieces = 0;
-    kv1b_ws_plan(cache->batch, cache->num_kv_heads, G, maxlen, num_sms(), &w.T, &w.Lt, &ncta, &pieces);
-    int64_t Tc, Ltc;
-    int nc, pieces_cap;
-    kv1b_ws_plan(cache->batch, cache->num_kv_heads, G, cache->capacity, num_sms(), &Tc, &Ltc, &nc, &pieces_cap);
-    w.ncta = ncta;
-    w.max_pieces = pieces_cap > pieces ? pieces_cap : pieces;
-    if (w.max_pieces > 256 || static_cast<size_t>(cache->batch) * cache->num_kv_heads * w.max_pieces * G *
-                                      kv1b::kPartStride * 4 > ws_counters_offset(cache, num_q_heads))
-      return KV1B_ERR_WORKSPACE;
-    w.part = static_cast<float*>(ws);
-    w.out = out;
-    w.status = cache->d_status;
-    w.counters = reinterpret_cast<unsigned*>(static_cast<char*>(ws) + ws_counters_offset(cache, num_q_heads));
+    const int rc = ws_params(cache, q, q_dtype, num_q_heads, scale, out, ws, &w);
+    if (rc != KV1B_OK) return rc;
     return cuda_status(kv1b_launch_attend_ws(w, G, ws_clean, static_cast<cudaStream_t>(stream)));
   }
   // this engine does not use the merge counters; they are zeroed here unless the caller says they
@@ -385,6 +411,69 @@ int kv1b_scores(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32
   for (int b = 0; b < cache->batch; ++b) sp.len[b] = static_cast<int32_t>(cache->h_lengths[b]);
   return cuda_status(kv1b_launch_scores(sp, num_q_heads / cache->num_kv_heads, static_cast<int32_t>(max_length(cache)),
                                         static_cast<cudaStream_t>(stream)));
+}
+
+int kv1b_scores_probe(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,
+                      int32_t kernel, int32_t* A, int32_t* Bc, float* s, float* out, void* ws, size_t ws_bytes,
+                      void* stream) {
+  if (kernel == KV1B_PROBE_POPC) return kv1b_scores(cache, q, q_dtype, num_q_heads, scale, A, Bc, s, stream);
+  if (!cache_ok(cache) || !q || !A || !Bc || !s || !ws || !dtype_ok(q_dtype)) return KV1B_ERR_INVALID_ARG;
+  const int hc = heads_check(cache, num_q_heads);
+  if (hc != KV1B_OK) return hc;
+  if (!(scale == scale)) return KV1B_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int G = num_q_heads / cache->num_kv_heads;
+  if (kernel == KV1B_PROBE_ATTEND) {
+    const int ac = attend_args_check(cache, q, q_dtype, num_q_heads, scale, out, ws, ws_bytes);
+    if (ac != KV1B_OK) return ac;
+    if (!ws_engine_applies(cache, num_q_heads)) return KV1B_ERR_UNSUPPORTED;
+    kv1b::AttendWsParams w;
+    const int rc = ws_params(cache, q, q_dtype, num_q_heads, scale, out, ws, &w);
+    if (rc != KV1B_OK) return rc;
+    w.probe_A = A;
+    w.probe_Bc = Bc;
+    w.probe_s = s;
+    return cuda_status(kv1b_launch_attend_ws(w, G, false, st, true));
+  }
+  if (kernel == KV1B_PROBE_TOPP) {
+    if (!aligned(q, 16) || !aligned(ws, kAlign)) return KV1B_ERR_MISALIGNED;
+    if (ws_bytes < kv1b_attend_workspace_bytes(cache, num_q_heads, 1)) return KV1B_ERR_WORKSPACE;
+    kv1b::ToppParams tp;
+    memset(&tp, 0, sizeof(tp));
+    tp.c = view(cache);
+    tp.q = q;
+    tp.q_dtype = q_dtype;
+    tp.Hq = num_q_heads;
+    tp.p = 1.0f;
+    tp.scale = scale;
+    tp.probe_A = A;
+    tp.probe_Bc = Bc;
+    for (int b = 0; b < cache->batch; ++b) tp.len[b] = static_cast<int32_t>(cache->h_lengths[b]);
+    kv1b_topp_carve(&tp, ws, cache->batch * num_q_heads, cache->capacity);
+    const int64_t maxlen = max_length(cache);
+    cudaError_t e = kv1b_launch_topp_scores_probe(tp, G, static_cast<int32_t>(maxlen), st);
+    if (e == cudaSuccess && maxlen > 0)  // the logits the pass wrote to its plane
+      e = cudaMemcpyAsync(s, tp.s, sizeof(float) * static_cast<size_t>(cache->batch) * num_q_heads * cache->capacity,
+                          cudaMemcpyDeviceToDevice, st);
+    return cuda_status(e);
+  }
+  return KV1B_ERR_INVALID_ARG;
+}
+
+int kv1b_attend_wait_probe(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads,
+                           float scale, float* out, void* ws, size_t ws_bytes, int32_t wait_tries,
+                           int32_t stall_stage, void* stream) {
+  const int ac = attend_args_check(cache, q, q_dtype, num_q_heads, scale, out, ws, ws_bytes);
+  if (ac != KV1B_OK) return ac;
+  if (wait_tries < 1 || wait_tries > kv1b::kWaitTriesDefault || stall_stage < -1) return KV1B_ERR_INVALID_ARG;
+  if (!ws_engine_applies(cache, num_q_heads)) return KV1B_ERR_UNSUPPORTED;
+  kv1b::AttendWsParams w;
+  const int rc = ws_params(cache, q, q_dtype, num_q_heads, scale, out, ws, &w);
+  if (rc != KV1B_OK) return rc;
+  w.wait_tries = wait_tries;
+  w.stall_stage = stall_stage;
+  return cuda_status(kv1b_launch_attend_ws(w, num_q_heads / cache->num_kv_heads, false,
+                                           static_cast<cudaStream_t>(stream)));
 }
 
 int kv1b_read_status(const kv1b_cache_t* cache, int32_t* flags, void* stream) {

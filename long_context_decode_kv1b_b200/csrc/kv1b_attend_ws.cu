@@ -39,8 +39,8 @@
 // the segment's rows by log-sum-exp into the output (one kernel per attend).
 //
 // Every mbarrier wait is bounded: a wait that runs out sets KV1B_STATUS_TIMEOUT in the cache's
-// status word; the CTA then stops issuing copies, later waits return at once, and the producer
-// drains the copies already in flight before the CTA exits.
+// status word; the CTA then stops issuing copies, later waits poll once and return, and the
+// producer drains the copies already in flight before the CTA exits.
 #include "kv1b_device.cuh"
 #include "kv1b_launch.h"
 
@@ -117,11 +117,13 @@ __device__ __forceinline__ bool mbar_try_sleep(uint64_t* bar, uint32_t parity) {
       : "memory");
   return ok != 0;
 }
-constexpr int kWaitTries = 4096;
-// Bounded wait.  Returns false when the CTA has given up (then the caller proceeds on garbage
-// data; the status word records the failure and no further copies are issued).
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
-  for (int tries = 0; tries < kWaitTries; ++tries) {
+// Bounded wait: at most `tries` suspended tries.  Returns false when the CTA has given up (then the
+// caller proceeds on garbage data; the status word records the failure and no further copies are
+// issued); once the CTA has given up, a wait that does not find its phase complete at the first
+// poll returns at once.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag, int tries) {
+  if (*abort_flag) return mbar_try(bar, parity);
+  for (int i = 0; i < tries; ++i) {
     if (mbar_try_sleep(bar, parity)) return true;
     if (*abort_flag) return false;
   }
@@ -270,7 +272,9 @@ __device__ __forceinline__ void issue_stage(const AttendWsParams& p, int seg, in
   bulk_g2s(st + kOffSm, c.v_sm + tok * 4, ntok * 16, bar);
 }
 
-template <int G>
+// PROBE: the test instantiation that also writes every score product and logit it forms
+// (p.probe_A / probe_Bc / probe_s); the product kernel is PROBE = false.
+template <int G, bool PROBE>
 __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_constant__ AttendWsParams p) {
   static_assert(G == 1 || G == 2 || G == 4, "head t of lane (g, t) for t < G");
   extern __shared__ uint8_t smem_raw[];
@@ -311,8 +315,9 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
       TileIt is = it;
       int j = 0;  // stages issued
       while (is.rem > 0 && !s_abort) {
+        if (j == p.stall_stage) break;  // test hook: this stage's copies never arrive
         const int st = j % kStages;
-        if (j >= kStages && !mbar_wait(&empty_bar[st], ((j / kStages) - 1) & 1, &s_abort)) break;
+        if (j >= kStages && !mbar_wait(&empty_bar[st], ((j / kStages) - 1) & 1, &s_abort, p.wait_tries)) break;
         const int n = is.nt(Lt);
         issue_stage(p, is.seg, is.lt, n, smem + st * kStageBytes, &full_bar[st]);
         is.advance(n, Lt);
@@ -351,6 +356,9 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
   // of 16-token chunk 2 ks + (m & 1); 128-byte swizzle: chunk ^ (row & 7) = ((m & 1) ^ (row & 7)) ^ 2 ks
   const uint32_t c_off = static_cast<uint32_t>(tl * kTileSmem + (32 * jw + 8 * (lane >> 4) + (lane & 7)) * 128);
   const uint32_t c_kx0 = static_cast<uint32_t>((((lane >> 3) & 1) ^ (lane & 7)) << 4);
+  // weight-rounding dither: a Weyl sequence over the lane's 32-token slices (top byte of
+  // n * 0x9E3779B9 + lane constant, n = slice index in the segment), offset by a quarter turn per token
+  const uint32_t weyl_c = static_cast<uint32_t>(lane) * 0x6A09E667u;
 
   // per-lane state
   float m_w[4], smax_w[4];  // quad-uniform: reference maximum per head, scale bound per group
@@ -604,7 +612,7 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
       cur_seg = it.seg;
       prep(cur_seg, cur_seg == second_seg, -1);
     }
-    if (!mbar_try(&full_bar[s], phase)) mbar_wait(&full_bar[s], phase, &s_abort);
+    if (!mbar_try(&full_bar[s], phase)) mbar_wait(&full_bar[s], phase, &s_abort, p.wait_tries);
     const uint8_t* st = smem + s * kStageBytes;
     const int rel = it.lt * kTileTok + sbase;          // this slice's first token in the segment
     const bool quad_on = tl < nt && L > rel - 32 * jw;  // the quad has real tokens in this stage
@@ -631,6 +639,15 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
           const float nc = __fmul_rn(knorm[tt], kcinv[tt]);
           const float dot = __fmaf_rn(c1_t, static_cast<float>(d[2 * e]), __fmaf_rn(c2_t, static_cast<float>(d[2 * e + 1]), c0_t));
           s2[kk][e] = valid ? __fmul_rn(dot, nc) : -INFINITY;
+          if constexpr (PROBE) {
+            if (valid) {
+              const int pb = cur_seg / c.Hkv, pkvh = cur_seg - pb * c.Hkv;
+              const int64_t o = (static_cast<int64_t>(pb) * p.Hq + pkvh * G + t) * c.cap + rel + tt;
+              p.probe_A[o] = d[2 * e];
+              p.probe_Bc[o] = d[2 * e + 1];
+              p.probe_s[o] = s2[kk][e];
+            }
+          }
           const uint32_t smw = vsm[tt * 4];  // (scale, min) of group t; zeros past the end of the cache
           sc[kk][e] = __half2float(__ushort_as_half(static_cast<unsigned short>(smw & 0xffffu)));
           mn[kk][e] = tt < lim ? __half2float(__ushort_as_half(static_cast<unsigned short>(smw >> 16))) : 0.0f;
@@ -703,16 +720,22 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
           #pragma unroll
           for (int h = 0; h < 4; ++h) ph[kk][e][h] = (h < G) ? __shfl_sync(kFull, pr, (lane & ~3) | h) : 0.0f;
         }
-      // ---------------- weights of group t: W = rint(p scale 2^E) < 2^32
+      // ---------------- weights of group t: W = rint(p scale 2^E + d) < 2^32, d a dither in [-1/2, 1/2)
+      // that makes the rounding unbiased (weights of a long tail far below the maximum are fractions
+      // of a unit, which plain rounding would send to zero together)
+      const uint32_t weyl = static_cast<uint32_t>(rel >> 5) * 0x9E3779B9u + weyl_c;
       #pragma unroll
       for (int kk = 0; kk < 2; ++kk) {
         uint32_t W[2][4];
         #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const float s2g = __fmul_rn(sc[kk][e], s2e_t);
+          // 2^23 + (top byte of the token's hash) as a float, then / 256 - 1/2 exactly
+          const uint32_t hb = weyl + static_cast<uint32_t>(2 * kk + e) * 0x40000000u;
+          const float dz = __fmaf_rn(__uint_as_float(prmt(hb, 0x4B000000u, 0x7543)), 0x1p-8f, -32768.5f);
           #pragma unroll
           for (int h = 0; h < 4; ++h) {
-            W[e][h] = __float2uint_rn(__fmul_rn(ph[kk][e][h], s2g));
+            W[e][h] = __float2uint_rn(__fmaf_rn(ph[kk][e][h], s2g, dz));
             mid[h] = __fmaf_rn(ph[kk][e][h], mn[kk][e], mid[h]);
           }
         }
@@ -764,16 +787,16 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
   if (s_abort && lane == 0) atomicOr(p.status, KV1B_STATUS_TIMEOUT);
 }
 
-template <int G>
+template <int G, bool PROBE>
 static cudaError_t launch_t(const AttendWsParams& p, bool counters_clean, cudaStream_t stream) {
   static std::atomic<unsigned long long> configured{0};  // bit per device
-  cudaError_t e = configure_smem(reinterpret_cast<const void*>(attend_ws_kernel<G>), kSmemBytes, &configured);
+  cudaError_t e = configure_smem(reinterpret_cast<const void*>(attend_ws_kernel<G, PROBE>), kSmemBytes, &configured);
   if (e != cudaSuccess) return e;
   if (!counters_clean) {
     e = cudaMemsetAsync(p.counters, 0, sizeof(unsigned) * p.c.B * p.c.Hkv, stream);
     if (e != cudaSuccess) return e;
   }
-  return launch_pdl(attend_ws_kernel<G>, dim3(p.ncta), dim3(kBlock), kSmemBytes, stream, p);
+  return launch_pdl(attend_ws_kernel<G, PROBE>, dim3(p.ncta), dim3(kBlock), kSmemBytes, stream, p);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -823,14 +846,20 @@ void kv1b_ws_plan(int32_t B, int32_t Hkv, int32_t G, int64_t L, int num_sms, int
   (void)G;
 }
 
-cudaError_t kv1b_launch_attend_ws(AttendWsParams& p, int32_t G, bool counters_clean, cudaStream_t stream) {
+cudaError_t kv1b_launch_attend_ws(AttendWsParams& p, int32_t G, bool counters_clean, cudaStream_t stream,
+                                  bool probe) {
   const int64_t tiles = static_cast<int64_t>(p.c.B) * p.c.Hkv * (p.c.cap / ws::kTileTok);
   const cudaError_t e = ws::encode_codes_map(&p.codes_map, p.c.v_codes, tiles);
   if (e != cudaSuccess) return e;
-  switch (G) {
-    case 1: return ws::launch_t<1>(p, counters_clean, stream);
-    case 2: return ws::launch_t<2>(p, counters_clean, stream);
-    case 4: return ws::launch_t<4>(p, counters_clean, stream);
+  if (p.wait_tries < 1) return cudaErrorInvalidValue;
+  if (probe && (!p.probe_A || !p.probe_Bc || !p.probe_s)) return cudaErrorInvalidValue;
+  switch (G * 2 + (probe ? 1 : 0)) {
+    case 2: return ws::launch_t<1, false>(p, counters_clean, stream);
+    case 4: return ws::launch_t<2, false>(p, counters_clean, stream);
+    case 8: return ws::launch_t<4, false>(p, counters_clean, stream);
+    case 3: return ws::launch_t<1, true>(p, counters_clean, stream);
+    case 5: return ws::launch_t<2, true>(p, counters_clean, stream);
+    case 9: return ws::launch_t<4, true>(p, counters_clean, stream);
     default: return cudaErrorInvalidValue;
   }
 }

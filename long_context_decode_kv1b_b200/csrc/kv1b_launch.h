@@ -107,6 +107,8 @@ struct ToppParams {
   float* out;
   int32_t* sel_idx;
   int32_t* sel_cnt;
+  int32_t* probe_A;          // test hook (probe instantiation of the score pass only): [R][cap] raw
+  int32_t* probe_Bc;         //   score products 8 A and 8 Bc
   int32_t len[KV1B_MAX_BATCH];
 };
 
@@ -164,7 +166,13 @@ struct alignas(64) AttendWsParams {
   float* out;          // [B][Hq][128]
   int32_t* status;     // cache status word (timeout flag)
   unsigned* counters;  // [B * Hkv] pieces of each segment written so far (zeroed before the launch)
+  int32_t wait_tries;  // suspended tries (<= 0.5 ms each) before a pipeline wait gives up
+  int32_t stall_stage; // test hook: each CTA's producer stops before this stage (-1: never)
+  int32_t* probe_A;    // test hook (probe instantiation only): [B][Hq][cap] raw score products 8 A,
+  int32_t* probe_Bc;   //   8 Bc and the log2-unit logits as the kernel forms them
+  float* probe_s;
 };
+constexpr int kWaitTriesDefault = 4096;
 
 }  // namespace kv1b
 
@@ -196,6 +204,9 @@ cudaError_t kv1b_launch_query_prep(const kv1b::CacheView& c, const void* q, int3
                                    uint32_t* planes, float* vl, float* delta, int32_t* sq, cudaStream_t stream);
 cudaError_t kv1b_launch_scores(const kv1b::ScoresParams& p, int32_t G, int32_t max_len, cudaStream_t stream);
 cudaError_t kv1b_launch_topp(const kv1b::ToppParams& p, int32_t G, int32_t max_len, cudaStream_t stream);
+// The Top-p pipeline's first two passes only (query preparation, scores), with the score pass writing
+// its raw integer products to p.probe_A / probe_Bc and its logits to p.s.
+cudaError_t kv1b_launch_topp_scores_probe(const kv1b::ToppParams& p, int32_t G, int32_t max_len, cudaStream_t stream);
 size_t kv1b_topp_workspace_bytes(int32_t rows, int32_t cap);
 void kv1b_topp_carve(kv1b::ToppParams* p, void* ws, int32_t rows, int32_t cap);
 int kv1b_pick_splits(int32_t B, int32_t Hkv, int64_t max_len, int num_sms);
@@ -206,4 +217,5 @@ cudaError_t kv1b_launch_exact(const kv1b::ExactParams& p, int32_t rows, int32_t 
 bool kv1b_ws_supported(int32_t G);
 void kv1b_ws_plan(int32_t B, int32_t Hkv, int32_t G, int64_t L, int num_sms, int64_t* T, int64_t* Lt, int* ncta,
                   int* max_pieces);
-cudaError_t kv1b_launch_attend_ws(kv1b::AttendWsParams& p, int32_t G, bool counters_clean, cudaStream_t stream);
+cudaError_t kv1b_launch_attend_ws(kv1b::AttendWsParams& p, int32_t G, bool counters_clean, cudaStream_t stream,
+                                  bool probe = false);

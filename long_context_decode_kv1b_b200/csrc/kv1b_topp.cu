@@ -173,8 +173,9 @@ __device__ __forceinline__ void build_bq(uint32_t (&bq)[4][2], const uint32_t* p
 }
 
 // grid (token blocks of kScoreTok, kv-heads, sequences); warp = 64 tokens at a time, up to 4 NG
-// heads as NG groups of 4 operand-column pairs.
-template <int NG>
+// heads as NG groups of 4 operand-column pairs.  PROBE: the test instantiation that also writes the
+// raw products 8 A and 8 Bc of every token (p.probe_A / probe_Bc).
+template <int NG, bool PROBE>
 __global__ void __launch_bounds__(kStreamThreads, NG == 1 ? 4 : 2) topp_scores_kernel(const ToppParams p, int G) {
   pdl_wait();
   __shared__ float s_max[kStreamWarps][8];
@@ -236,6 +237,11 @@ __global__ void __launch_bounds__(kStreamThreads, NG == 1 ? 4 : 2) topp_scores_k
             const float sv =
                 logit_from_ints(d[2 * e] >> 3, d[2 * e + 1] >> 3, csq[hg], cvl[hg], cdl[hg], nc[i], qs);
             srow[hg][base + g + 8 * i] = sv;
+            if constexpr (PROBE) {
+              const int64_t o = (srow[hg] - p.s) + base + g + 8 * i;
+              p.probe_A[o] = d[2 * e];
+              p.probe_Bc[o] = d[2 * e + 1];
+            }
             mx[hg] = fmaxf(mx[hg], sv);
           }
         }
@@ -983,8 +989,8 @@ cudaError_t kv1b_launch_topp(const ToppParams& p, int32_t G, int32_t max_len, cu
     e = kv1b_launch_query_prep(p.c, p.q, p.q_dtype, p.Hq, p.planes, p.qvl, p.qdl, p.qsq, stream);
     if (e != cudaSuccess) return e;
     const dim3 grid((max_len + kScoreTok - 1) / kScoreTok, p.c.Hkv, p.c.B);
-    e = G <= 4 ? launch_pdl(topp_scores_kernel<1>, grid, bs, 0, stream, p, G)
-               : launch_pdl(topp_scores_kernel<2>, grid, bs, 0, stream, p, G);
+    e = G <= 4 ? launch_pdl(topp_scores_kernel<1, false>, grid, bs, 0, stream, p, G)
+               : launch_pdl(topp_scores_kernel<2, false>, grid, bs, 0, stream, p, G);
     if (e == cudaSuccess)
       e = p.mode == KV1B_SELECT_TOPK ? launch_pdl(topp_mass_kernel<KV1B_SELECT_TOPK>, sg, bs, 0, stream, p)
                                      : launch_pdl(topp_mass_kernel<KV1B_SELECT_TOPP>, sg, bs, 0, stream, p);
@@ -1005,6 +1011,20 @@ cudaError_t kv1b_launch_topp(const ToppParams& p, int32_t G, int32_t max_len, cu
   int msplit = (nsub_used + 15) / 16;
   msplit = msplit < 1 ? 1 : (msplit > kToppMergeSplit ? kToppMergeSplit : msplit);
   if (e == cudaSuccess) e = launch_pdl(topp_merge_kernel, dim3(msplit, R), dim3(kD), 0, stream, p);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+cudaError_t kv1b_launch_topp_scores_probe(const ToppParams& p, int32_t G, int32_t max_len, cudaStream_t stream) {
+  if (G > 8 || !p.probe_A || !p.probe_Bc) return cudaErrorInvalidValue;
+  if (max_len <= 0) return cudaSuccess;
+  const ToppLayout l = topp_layout(p.c.B * p.Hq, p.c.cap);
+  cudaError_t e = cudaMemsetAsync(p.rows, 0, l.state_bytes, stream);
+  if (e == cudaSuccess) e = kv1b_launch_query_prep(p.c, p.q, p.q_dtype, p.Hq, p.planes, p.qvl, p.qdl, p.qsq, stream);
+  if (e != cudaSuccess) return e;
+  const dim3 grid((max_len + kScoreTok - 1) / kScoreTok, p.c.Hkv, p.c.B);
+  e = G <= 4 ? launch_pdl(topp_scores_kernel<1, true>, grid, dim3(kStreamThreads), 0, stream, p, G)
+             : launch_pdl(topp_scores_kernel<2, true>, grid, dim3(kStreamThreads), 0, stream, p, G);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
 }

@@ -56,6 +56,7 @@ def lib() -> ctypes.CDLL:
             "ref_half_to_double": (ctypes.c_double, [ctypes.c_uint16]),
             "ref_query_prep": (None, [P, P, ctypes.c_int, P, P, P, P, P, P]),
             "ref_score_ints": (None, [P, P, ctypes.c_int, P, P]),
+            "ref_score_ints_n": (None, [P, i64, P, ctypes.c_int, P, P]),
             "ref_logit": (f32, [i32, i32, i32, f32, f32, f32, f32, f32, ctypes.c_int]),
             "ref_logits": (None, [P, P, P, i64, P, f32, f32, i32, f32, ctypes.c_int, P]),
             "ref_attend_head": (None, [P, P, P, P, P, i64, P, P, f32, ctypes.c_int, P]),
@@ -194,10 +195,7 @@ def score_ints(bits, planes):
     d = bits.shape[1] * 32
     A = np.empty(bits.shape[0], np.int32)
     Bc = np.empty(bits.shape[0], np.int32)
-    for t in range(bits.shape[0]):
-        a, b = ctypes.c_int32(), ctypes.c_int32()
-        lib().ref_score_ints(_p(bits[t]), _p(planes), d, ctypes.byref(a), ctypes.byref(b))
-        A[t], Bc[t] = a.value, b.value
+    lib().ref_score_ints_n(_p(bits), bits.shape[0], _p(planes), d, _p(A), _p(Bc))
     return A, Bc
 
 

@@ -307,6 +307,12 @@ void ref_score_ints(const uint32_t* bits, const uint32_t* planes, int d, int32_t
   *Bc = b;
 }
 
+/* The same integers for L consecutive tokens (one call instead of L). */
+void ref_score_ints_n(const uint32_t* bits, int64_t L, const uint32_t* planes, int d, int32_t* A, int32_t* Bc) {
+  const int nw = d / 32;
+  for (int64_t t = 0; t < L; ++t) ref_score_ints(bits + t * nw, planes, d, A + t, Bc + t);
+}
+
 /* RaBitQ estimator in unnormalised variables: q.k ~ N cinv sum_i (2 b_i - 1) z_i / d, with the
  * quantised z_i = vl + delta code_i, so sum_i (2b_i - 1) z_i = delta (2A - Sq) + vl (2Bc - d).
  * The logit is that estimate times the softmax scale. */

@@ -81,6 +81,9 @@ void ref_query_prep(const float* q, const float* signs, int d, uint32_t* planes,
  * Bc = sum_w popc(bits_w). */
 void ref_score_ints(const uint32_t* bits, const uint32_t* planes, int d, int32_t* A, int32_t* Bc);
 
+/* ref_score_ints for L consecutive tokens: bits [L][d/32], A and Bc [L]. */
+void ref_score_ints_n(const uint32_t* bits, int64_t L, const uint32_t* planes, int d, int32_t* A, int32_t* Bc);
+
 /* Estimated logit from the integers, fp32, fixed op order:
  * I1 = 2Bc - d, I2 = 2A - Sq, dot = fl(fl(delta*I2) + fl(vl*I1)), s = fl(fl(dot * fl(norm*cinv)) * (scale/d)). */
 float ref_logit(int32_t A, int32_t Bc, int32_t Sq, float vl, float delta, float norm, float cinv, float scale, int d);

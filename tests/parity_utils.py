@@ -86,3 +86,34 @@ def oracle_attend_all(host: HostKV, q: torch.Tensor, signs, scale, G, heads=None
                 encs[(b, kvh)] = host.encode(b, kvh, signs)
             out[b, hq] = oracle.attend(encs[(b, kvh)], qn[b, hq], signs, scale)
     return out
+
+
+L2E = 1.4426950408889634
+
+
+def check_probe_row(pr: dict, b: int, hq: int, enc: dict, q_row: np.ndarray, signs, scale: float, kernel: int,
+                    n: int, where: str = ""):
+    """One (b, hq) row of a kv1b_scores_probe result against the oracle: the integers bit for bit
+    (8 A and 8 Bc from the tensor-core kernels, A and Bc from the popcount hook); the fp32 logits bit
+    for bit (popcount hook, Top-p score pass); the persistent attend kernel's log2-unit logits within
+    16 roundings of the magnitude of their terms (it forms them in its own fused order)."""
+    mult = 1 if kernel == kv.PROBE_POPC else 8
+    r = oracle.query_prep(q_row, signs)
+    A, Bc = oracle.score_ints(enc["bits"][:n], r["planes"])
+    gA, gB = pr["A"][b, hq, :n].cpu().numpy(), pr["Bc"][b, hq, :n].cpu().numpy()
+    bad = np.flatnonzero((gA != mult * A) | (gB != mult * Bc))
+    assert bad.size == 0, f"{where} b{b} hq{hq}: {bad.size} integer mismatches, first at {bad[:4].tolist()}"
+    gs = pr["s"][b, hq, :n].cpu().numpy()
+    if kernel == kv.PROBE_ATTEND:
+        dl, vl, sq = float(r["delta"]), float(r["vl"]), int(r["Sq"])
+        nc = enc["norm"][:n].astype(np.float64) * enc["cinv"][:n].astype(np.float64)
+        qs = scale / 128.0 * L2E
+        exact = (dl * (2.0 * A - sq) + vl * (2.0 * Bc - 128.0)) * nc * qs
+        mag = (abs(dl) * (2.0 * A + sq) + abs(vl) * (2.0 * Bc + 128.0)) * np.abs(nc) * qs
+        err = np.abs(gs.astype(np.float64) - exact)
+        assert (err <= 16 * 2.0 ** -24 * mag + 1e-30).all(), \
+            f"{where} b{b} hq{hq}: log2 logit off by {np.max(err / (mag + 1e-30)):.2e} of its terms"
+    else:
+        enc_n = {k: v[:n] for k, v in enc.items() if k != "flags"}
+        s = oracle.logits(enc_n, r, scale)
+        assert np.array_equal(gs.view(np.uint32), s.view(np.uint32)), f"{where} b{b} hq{hq}: logits differ"

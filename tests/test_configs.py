@@ -16,7 +16,7 @@ import torch
 import oracle
 import long_context_decode_kv1b_b200 as kv
 from long_context_decode_kv1b_b200 import workloads as wl
-from parity_utils import assert_planes_equal, assert_rows_close, gpu_head_planes, to_np32
+from parity_utils import assert_planes_equal, assert_rows_close, check_probe_row, gpu_head_planes, to_np32
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -114,6 +114,20 @@ def test_c2_mha_outlier_channels():
     assert run.cache.status() == 0
 
 
+def probe_rows(run: Run, q, kernel, heads_per_pair=None):
+    """kv1b_scores_probe of `kernel` on the run's cache; the sampled segments' query heads (all G of
+    them, or the first heads_per_pair) checked against the oracle over every token."""
+    cfg = run.cfg
+    pr = run.cache.scores_probe(q, cfg.scale, kernel)
+    torch.cuda.synchronize()
+    qn = to_np32(q)
+    for (b, h) in run.pairs:
+        for j in range(heads_per_pair or cfg.G):
+            check_probe_row(pr, b, h * cfg.G + j, run.encoded((b, h)), qn[b, h * cfg.G + j], run.signs, cfg.scale,
+                            kernel, run.n, where=cfg.name)
+    return pr
+
+
 def test_c3_gqa_batch8_decode_steps():
     cfg = wl.CONFIGS["c3"]
     run = Run(cfg, [(0, 0), (0, 7), (5, 3), (7, 7)])
@@ -122,6 +136,10 @@ def test_c3_gqa_batch8_decode_steps():
     q = wl.queries(cfg, cfg.steps - 1, DEV)
     again = run.cache.attend(q, cfg.scale)
     assert torch.equal(out, again)
+    # the integers of the kernels this workload runs, bit for bit over every token of the sampled segments
+    pr = probe_rows(run, q, kv.PROBE_ATTEND)
+    assert torch.equal(pr["out"], out)  # the probe instantiation computes the same attention
+    probe_rows(run, q, kv.PROBE_TOPP)
 
 
 def test_c4_topp_heavy_tokens():
@@ -169,4 +187,25 @@ def test_c5_one_million_tokens():
     run.check_planes()
     assert run.cache.lengths == [cfg.L + cfg.steps]
     assert not torch.equal(first, out)  # the appended tokens and new queries changed the result
+    assert run.cache.status() == 0
+    # the score integers of both tensor-core kernels over all 1,048,608 tokens of kv-head 0's heads
+    saved = run.pairs
+    run.pairs = [(0, 0)]
+    probe_rows(run, q, kv.PROBE_ATTEND)
+    probe_rows(run, q, kv.PROBE_TOPP)
+    run.pairs = saved
+    # adaptive Top-p (p = 0.9) on the same cache: sampled heads of kv-heads 0 and 5, selected sets and
+    # counts bit for bit, outputs at the bar
+    out_p, sel, cnt = run.cache.attend_topp(q, cfg.scale, 0.9)
+    torch.cuda.synchronize()
+    qn, cnt_h = to_np32(q), cnt.cpu().numpy()
+    for (b, h), heads in (((0, 0), (0, 3)), ((0, 5), (21, 22))):
+        enc = {k: v[:run.n] for k, v in run.encoded((b, h)).items() if k != "flags"}
+        for hq in heads:
+            ref_sel, ref_out = oracle.attend_topp(enc, qn[b, hq], run.signs, cfg.scale, 0.9)
+            n = int(cnt_h[b, hq])
+            assert n == len(ref_sel), f"c5 Top-p hq{hq}: |S| {n} vs {len(ref_sel)}"
+            assert np.array_equal(sel[b, hq, :n].cpu().numpy(), ref_sel), f"c5 Top-p hq{hq}: selected sets differ"
+            assert_rows_close(out_p[b, hq].cpu().numpy(), ref_out, where=f"c5 Top-p hq{hq}")
+    assert (cnt_h >= 1).all() and (cnt_h <= run.n).all()
     assert run.cache.status() == 0

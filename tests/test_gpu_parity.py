@@ -12,7 +12,8 @@ import torch
 
 import oracle
 import long_context_decode_kv1b_b200 as kv
-from parity_utils import HostKV, assert_planes_equal, assert_rows_close, gpu_head_planes, oracle_attend_all, to_np32
+from parity_utils import (L2E, HostKV, assert_planes_equal, assert_rows_close, check_probe_row, gpu_head_planes,
+                          oracle_attend_all, to_np32)
 
 pytestmark = pytest.mark.gpu
 DEV = "cuda"
@@ -463,4 +464,126 @@ def test_three_rounds_encode_bit_exact_and_attend(dtype):
     for engine in (kv.ATTEND_TENSOR, kv.ATTEND_CUDA_CORE):
         assert_rows_close(cache.attend(q, 0.3, engine=engine).cpu().numpy(), ref, where=f"3 rounds e{engine}")
     topp_check(cache, host, q, 0.3, 0.9, G, D)
+    assert cache.status() == 0
+
+
+# ------------------------------------------------- score integers of the kernels kv1b_attend / kv1b_attend_topp run
+def probe_check(cache, host, q, scale, G, signs, kernel, where=""):
+    """Every (b, hq) row of a kv1b_scores_probe result against the oracle (check_probe_row)."""
+    pr = cache.scores_probe(q, scale, kernel)
+    torch.cuda.synchronize()
+    qn = to_np32(q)
+    B, Hq, _ = qn.shape
+    encs = {}
+    for b in range(B):
+        for hq in range(Hq):
+            kvh = hq // G
+            if (b, kvh) not in encs:
+                encs[(b, kvh)] = host.encode(b, kvh, signs)
+            check_probe_row(pr, b, hq, encs[(b, kvh)], qn[b, hq], signs, scale, kernel, cache.lengths[b], where)
+    return pr
+
+
+@pytest.mark.parametrize("G", [1, 2, 4])
+def test_attend_kernel_score_integers_bit_exact(G):
+    # a tile-boundary length (4099 = 32 tiles + 3) and two sequences x two kv-heads
+    B, Hkv = 2, 2
+    cache, host = build_cache(B, Hkv, [4000, 99], torch.bfloat16, seed=19, data_seed=G)
+    q = torch.randn((B, Hkv * G, 128), device=DEV, generator=torch.Generator(device=DEV).manual_seed(40 + G))
+    pr = probe_check(cache, host, q, 0.3, G, oracle.signs(19), kv.PROBE_ATTEND, where=f"attend G{G}")
+    # the probe runs the whole attend: its output is the default engine's
+    ref = oracle_attend_all(host, q, oracle.signs(19), 0.3, G)
+    assert_rows_close(pr["out"].cpu().numpy(), ref, where=f"probe out G{G}")
+    assert cache.status() == 0
+
+
+@pytest.mark.parametrize("G,L", [(1, 300), (3, 4099), (4, 9000), (8, 2049)])
+def test_topp_score_pass_integers_and_logits_bit_exact(G, L):
+    B, Hkv = 1, 2
+    cache, host = build_cache(B, Hkv, [L], torch.float32, seed=29, data_seed=L)
+    q = torch.randn((B, Hkv * G, 128), device=DEV, generator=torch.Generator(device=DEV).manual_seed(G))
+    probe_check(cache, host, q, 0.2, G, oracle.signs(29), kv.PROBE_TOPP, where=f"topp G{G} L{L}")
+
+
+def test_popc_probe_matches_kv1b_scores():
+    B, Hkv, G = 1, 1, 4
+    cache, host = build_cache(B, Hkv, [777], torch.bfloat16, seed=3, data_seed=3)
+    q = torch.randn((B, Hkv * G, 128), device=DEV, generator=torch.Generator(device=DEV).manual_seed(1))
+    pr = probe_check(cache, host, q, 0.1, G, oracle.signs(3), kv.PROBE_POPC, where="popc")
+    sc = cache.scores(q, 0.1)
+    for k in ("A", "Bc", "s"):
+        assert torch.equal(pr[k][..., :777], sc[k][..., :777])
+
+
+# ------------------------------------------------------------------ bounded pipeline waits of the persistent kernel
+def test_attend_wait_runs_out_and_reports_timeout():
+    # Each CTA's copy producer stops before its stage `stall` (70,000 tokens x 2 kv-heads = 1,094 tiles:
+    # 7-8 tiles, i.e. 3 stages, per CTA): the consumers' wait (2 tries of at most 0.5 ms) runs out, the
+    # kernel records KV1B_STATUS_TIMEOUT and returns; the next call, which zeroes the merge counters
+    # again, matches the oracle.  A fresh cache per case: the status word keeps its bits.
+    B, Hkv, G, L = 1, 2, 4, 70000
+    for stall in (-1, 0, 1):
+        cache, host = build_cache(B, Hkv, [L], torch.bfloat16, seed=14, data_seed=2)
+        q = torch.randn((B, Hkv * G, 128), device=DEV, generator=torch.Generator(device=DEV).manual_seed(3))
+        if stall == -1:
+            ref = oracle_attend_all(host, q, oracle.signs(14), 0.2, G)
+        out = cache.attend_wait_probe(q, 0.2, wait_tries=2, stall_stage=stall)
+        torch.cuda.synchronize()
+        if stall == -1:  # a short limit alone changes nothing
+            assert_rows_close(out.cpu().numpy(), ref, where="short limit, no stall")
+            assert cache.status() == 0
+            continue
+        assert cache.status() & kv.STATUS_TIMEOUT, f"stall at stage {stall}: no timeout reported"
+        out = cache.attend(q, 0.2)  # the binding drops WS_CLEAN after a stalled run
+        torch.cuda.synchronize()
+        assert_rows_close(out.cpu().numpy(), ref, where=f"after a stall at stage {stall}")
+
+
+# ------------------------------------------------------------------ a long tail far below one dominant token
+def tail_cache(L: int, gap_lo: float, gap_hi: float, seed: int):
+    """One kv-head, 4 query heads, L + 1 tokens.  Every key is a positive multiple a_t of one vector u,
+    so all tokens share the sign bits and the estimated logit is linear in a_t; the dominant token
+    (position 777, a = 1) sits gap_t log2 units above token t for the head-0 query q = u, with gap_t
+    uniform in [gap_lo, gap_hi].  Tail values have mean +1, the dominant value mean -1, so the output
+    depends directly on how much of the mass the tail carries."""
+    g = torch.Generator(device=DEV).manual_seed(seed)
+    u = torch.randn((128,), generator=g, device=DEV)
+    n = L + 1
+    cache = kv.Cache(1, 1, (n + 127) // 128 * 128, seed=seed)
+    host = HostKV(1, 1, cache.capacity)
+    # the logit of a key a * u at scale 1 (the oracle's estimate; the same sign bits for every a > 0)
+    D = oracle.signs(seed)
+    enc1 = oracle.encode(u.cpu().numpy()[None, :], np.zeros((1, 128), np.float32), D)
+    s1 = float(oracle.logits(enc1, oracle.query_prep(u.cpu().numpy(), D), 1.0)[0])
+    assert s1 > 0
+    span = 40.0  # log2-unit logit of the dominant token: gap = (1 - a) * span
+    scale = span / (s1 * L2E)
+    a = 1.0 - (gap_lo + (gap_hi - gap_lo) * torch.rand((n,), generator=g, device=DEV)) / span
+    a[777] = 1.0
+    K = (a[:, None] * u[None, :]).view(1, n, 1, 128)
+    V = torch.randn((1, n, 1, 128), generator=g, device=DEV) + 1.0
+    V[0, 777] -= 2.0
+    for t0 in range(0, n, 1 << 18):
+        t1 = min(n, t0 + (1 << 18))
+        cache.append(K[:, t0:t1].contiguous(), V[:, t0:t1].contiguous())
+        host.add(K[:, t0:t1], V[:, t0:t1])
+    q = torch.stack([u * f for f in (1.0, 1.05, 0.95, 1.1)]).view(1, 4, 128)
+    return cache, host, q, scale, D
+
+
+@pytest.mark.parametrize("gap_lo,gap_hi", [(20.0, 28.0), (26.6, 27.4)])
+def test_attend_long_tail_below_a_dominant_token(gap_lo, gap_hi):
+    # 2^20 tail tokens 2^-20 .. 2^-28 below the dominant one carry ~15 % of the mass (head 0); a tail
+    # packed at 2^-27 carries ~0.7 %: with 32-bit fixed-point weights these are fractions of a unit,
+    # which the dithered rounding keeps unbiased
+    cache, host, q, scale, D = tail_cache(1 << 20, gap_lo, gap_hi, seed=61)
+    ref = oracle_attend_all(host, q, D, scale, 4)
+    enc = host.encode(0, 0, D)
+    s = oracle.logits(enc, oracle.query_prep(q[0, 0].cpu().numpy(), D), scale).astype(np.float64)
+    w = np.exp2((s - s.max()) * L2E)
+    frac = (w.sum() - 1.0) / w.sum()
+    assert (0.05 <= frac <= 0.30) if gap_lo < 25 else (0.003 <= frac <= 0.02), frac
+    for engine in (kv.ATTEND_TENSOR, kv.ATTEND_CUDA_CORE):
+        out = cache.attend(q, scale, engine=engine)
+        assert_rows_close(out.cpu().numpy(), ref, where=f"tail {gap_lo}-{gap_hi} e{engine}")
     assert cache.status() == 0

@@ -11,6 +11,13 @@ values).  The model follows those steps tile by tile (128 tokens) and shows why 
 32 bits: when a long tail far below the maximum holds a few percent of the softmax mass or more,
 a 23-bit fixed point rounds the tail's weights to a unit or none and biases the output beyond the
 1e-3 bar, while 32 bits stay near 1e-6.
+
+The engine adds a dither d in [-1/2, 1/2) before rounding, W = rint(p * scale * 2^E + d): tokens
+2^-26.6 or more below the reference maximum get weights under half a unit, which plain rounding sends
+to zero all together -- a bias that grows with the number of such tokens one reference covers.  d is
+the top byte of a Weyl sequence (n * 0x9E3779B9 + lane * 0x6A09E667 + j * 2^30, n the 32-token slice,
+lane = 4 (token & 7) + group, j = 2 ((token & 31) >> 4) + ((token >> 3) & 1)), so over many tokens
+every fractional weight keeps its expected value; the model reproduces that mapping.
 """
 import math
 
@@ -34,8 +41,20 @@ def decode_values(enc: dict):
     return codes, fp16_bits_to_f32(sm & 0xFFFF), fp16_bits_to_f32(sm >> 16)
 
 
-def model_attend(s2: np.ndarray, codes, scale, mn, bits: int = 32) -> np.ndarray:
-    """One head: s2 log2-unit logits [L] (fp32).  Returns fp64 out [128]."""
+def dither(t0: int, t1: int, group: int) -> np.ndarray:
+    """The engine's rounding offsets of tokens t0 .. t1 - 1 (segment positions) for one value group."""
+    t = np.arange(t0, t1, dtype=np.uint64)
+    n = t >> np.uint64(5)
+    tau = t & np.uint64(31)
+    lane = (tau & np.uint64(7)) * np.uint64(4) + np.uint64(group)
+    j = np.uint64(2) * (tau >> np.uint64(4)) + ((tau >> np.uint64(3)) & np.uint64(1))
+    h = (n * np.uint64(0x9E3779B9) + lane * np.uint64(0x6A09E667) + j * np.uint64(0x40000000)) & np.uint64(0xFFFFFFFF)
+    return ((h >> np.uint64(24)).astype(np.float64) / 256.0 - 0.5).astype(np.float32)
+
+
+def model_attend(s2: np.ndarray, codes, scale, mn, bits: int = 32, dithered: bool = True) -> np.ndarray:
+    """One head: s2 log2-unit logits [L] (fp32).  Returns fp64 out [128].  dithered=False rounds the
+    weights without the dither (the form the dither replaced)."""
     L = s2.shape[0]
     m = -math.inf
     E = [None] * 4
@@ -79,7 +98,11 @@ def model_attend(s2: np.ndarray, codes, scale, mn, bits: int = 32) -> np.ndarray
         lsum += float(p.astype(np.float64).sum())
         for g in range(4):
             s2g = (scale[t0:t1, g] * np.float32(2.0 ** E[g])).astype(np.float32)
-            W = np.rint((p * s2g).astype(np.float32)).astype(np.int64)
+            if dithered:  # one rounding of p * s2g + d (a fused multiply-add), negative results to 0
+                x = (p.astype(np.float64) * s2g.astype(np.float64) + dither(t0, t1, g)).astype(np.float32)
+            else:
+                x = (p * s2g).astype(np.float32)
+            W = np.maximum(np.rint(x), 0).astype(np.int64)
             assert W.max(initial=0) < 2 ** bits
             D[32 * g:32 * g + 32] += W @ codes[t0:t1, 32 * g:32 * g + 32]
             mid[g] += float((p.astype(np.float64) * mn[t0:t1, g].astype(np.float64)).sum())
@@ -145,3 +168,41 @@ def test_32_bit_weights_on_gaussian_logits_with_a_late_maximum():
     s2[-1] = s2.max() + 12.0
     ref = reference(s2, codes, scale, mn)
     assert rel_err(model_attend(s2, codes, scale, mn, 32), ref) < 2e-5
+
+
+def packed_tail_case(L: int = 1 << 20, vmean: float = 3.0):
+    """One dominant token at position 0 and L tail tokens 2^-27.2 .. 2^-28 below it (log2 units) --
+    weights of 0.2 .. 0.5 units at 32 bits; tail values of mean +vmean, the dominant value -vmean."""
+    rng = np.random.default_rng(11)
+    K = rng.standard_normal((L, 128)).astype(np.float32)
+    V = (rng.standard_normal((L, 128)) + vmean).astype(np.float32)
+    V[0] -= 2 * vmean
+    enc = oracle.encode(K, V, oracle.signs(11))
+    codes, scale, mn = decode_values(enc)
+    s2 = rng.uniform(-28.0, -27.2, L).astype(np.float32)
+    s2[0] = 0.0
+    return s2, codes, scale, mn
+
+
+def test_dither_keeps_a_tail_of_sub_unit_weights_unbiased():
+    # one reference maximum over 2^20 tokens whose weights are fractions of a unit (as one quad of
+    # the engine sees when a very large cache gives it that many tokens): plain rounding drops most
+    # of them and misses the bar; the dithered rounding stays far inside it
+    s2, codes, scale, mn = packed_tail_case()
+    ref = reference(s2, codes, scale, mn)
+    w = np.exp2(s2.astype(np.float64))
+    assert 3e-3 < (w.sum() - 1.0) / w.sum() < 8e-3
+    e_plain = rel_err(model_attend(s2, codes, scale, mn, dithered=False), ref)
+    e_dith = rel_err(model_attend(s2, codes, scale, mn), ref)
+    assert e_plain > 1e-3, e_plain
+    assert e_dith < 1e-4, e_dith
+
+
+def test_dither_offsets_are_uniform_per_group():
+    # the offsets of any 8192 consecutive tokens cover [-1/2, 1/2) evenly for every value group
+    for g in range(4):
+        d = dither(4096, 4096 + 8192, g).astype(np.float64)
+        assert d.min() >= -0.5 and d.max() < 0.5
+        assert abs(d.mean()) < 0.01
+        hist = np.histogram(d, bins=16, range=(-0.5, 0.5))[0]
+        assert hist.min() > 0.8 * 8192 / 16 and hist.max() < 1.2 * 8192 / 16
