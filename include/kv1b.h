@@ -73,6 +73,13 @@ extern "C" {
                                     while its predecessor in the stream finishes).  Do not pass it for a new
                                     workspace, one used with another shape or written by anything else, or
                                     after KV1B_STATUS_TIMEOUT. */
+#define KV1B_ATTEND_PARTIAL 4    /* OR-ed into the engine: out receives log-sum-exp partial rows instead of the
+                                    normalised output, f32 [batch][num_q_heads][2 + 128] = (m, l, o[128]) with
+                                    l = sum_t 2^(s_t log2(e) - m) and o = sum_t 2^(s_t log2(e) - m) vhat_t for a
+                                    reference m in log2 units (the row's largest s_t log2(e), or at most 4 below
+                                    it; m = -inf, l = 0, o = 0 for an empty sequence): the attention of this
+                                    cache's tokens in a form that kv1b_merge_partials combines with the rows of
+                                    other token ranges of the same sequences (a context split over GPUs). */
 
 /* kv1b_attend_select modes */
 #define KV1B_SELECT_TOPP 0  /* smallest set reaching a fraction p of the estimated attention mass */
@@ -164,7 +171,8 @@ size_t kv1b_attend_workspace_bytes(const kv1b_cache_t* cache, int32_t num_q_head
  * vhat = min + scale_g * code.  A sequence of length 0 gives zeros.
  * ws: device workspace, 256-byte aligned, ws_bytes >= kv1b_attend_workspace_bytes(.., 0).
  * flags: KV1B_ATTEND_TENSOR (default) or KV1B_ATTEND_CUDA_CORE (same result within fp32
- * rounding), optionally | KV1B_ATTEND_WS_CLEAN; any other bit is KV1B_ERR_INVALID_ARG.
+ * rounding), optionally | KV1B_ATTEND_WS_CLEAN and | KV1B_ATTEND_PARTIAL (then out is
+ * [batch][num_q_heads][2 + 128], see above); any other bit is KV1B_ERR_INVALID_ARG.
  * num_splits: 0 chooses the split-K factor; > 0 forces it (testing).
  * The kernels are launched with programmatic stream serialization: they may be scheduled while the
  * previous kernel in `stream` finishes, and wait for it before touching memory. */
@@ -179,14 +187,20 @@ int kv1b_attend(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32
  * it; it exists for this library's users.)  For callers that can neither allocate device memory
  * (their framework's allocator owns it, or cudaMalloc/cudaFree would synchronise a
  * latency-critical decode loop) nor pass a workspace buffer (a fixed ABI with inputs and outputs
- * only).  Same arguments, result and rules as kv1b_attend minus ws / ws_bytes / num_splits; the
- * split-K partials go to a file-scope device array of KV1B_NOALLOC_SCRATCH_BYTES instead.
- * The first call on a device looks up that array's device address (cudaGetSymbolAddress, with
- * the device current) and caches it; make that first call before any stream capture.
- * Every call shares the array: calls whose kernels may overlap on the GPU race, so order them on
- * one stream (or otherwise).  The split count is lowered when needed to fit the array; a shape
- * whose partials do not fit even unsplit (batch * num_q_heads * 520 bytes > the array) returns
- * KV1B_ERR_WORKSPACE before launching anything.  Calls no cudaMalloc / cudaFree. */
+ * only).  Same arguments and result as kv1b_attend minus ws / ws_bytes / num_splits; flags is
+ * KV1B_ATTEND_TENSOR or KV1B_ATTEND_CUDA_CORE (KV1B_ATTEND_WS_CLEAN is not accepted).
+ * KV1B_ATTEND_TENSOR runs the persistent tensor-core kernel where kv1b_attend would (G in {1, 2, 4},
+ * equal sequence lengths) and its partial rows fit the array, otherwise the CUDA-core split-K
+ * engine, which KV1B_ATTEND_CUDA_CORE always runs.  The partial rows and merge counters go to a
+ * file-scope device array of KV1B_NOALLOC_SCRATCH_BYTES instead of a workspace; each call zeroes
+ * the counters it uses with one small memset on `stream`.
+ * The first call on a device (and the first after a new context replaced the old one) looks up that
+ * array's device address (cudaGetSymbolAddress, with the device current) and caches it; make that
+ * first call before any stream capture.  Every call shares the array: calls whose kernels may
+ * overlap on the GPU race, so order them on one stream (or otherwise).  A shape whose split-K
+ * partials do not fit (batch * num_q_heads * splits * 520 bytes > the array; splits <= 2 * SMs /
+ * (batch * num_kv_heads)) returns KV1B_ERR_WORKSPACE before launching anything.  Calls no
+ * cudaMalloc / cudaFree. */
 int kv1b_attend_noalloc(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,
                         float* out, int32_t flags, void* stream);
 
@@ -251,6 +265,15 @@ int kv1b_query_prep(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, i
  * entries at t >= length[b] are left unspecified. */
 int kv1b_scores(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,
                 int32_t* A, int32_t* Bc, float* s, void* stream);
+
+/* Log-sum-exp merge of partial attention rows (KV1B_ATTEND_PARTIAL) of disjoint token ranges of the
+ * same sequences -- e.g. one context split over several GPUs, whose rows were gathered into one
+ * array: out[r] = sum_k 2^(m_k - M) o_k / sum_k 2^(m_k - M) l_k, M = max_k m_k, in a fixed order
+ * (zeros when every l_k is 0).  parts: f32 [nparts][rows][2 + 128] (device, 4-byte aligned), out:
+ * f32 [rows][128] (device, 16-byte aligned); 1 <= nparts <= 1024.  Asynchronous on `stream`.
+ * (No page describes a multi-GPU split; this is the merge the split-K engines already use, across
+ * ranks.) */
+int kv1b_merge_partials(const float* parts, int32_t nparts, int64_t rows, float* out, void* stream);
 
 /* kv1b_scores_probe kernels */
 #define KV1B_PROBE_POPC 0    /* __popc over AND-ed bit-planes (the kv1b_scores hook) */

@@ -20,6 +20,8 @@ MAX_BATCH = 64
 DTYPE_F32, DTYPE_BF16, DTYPE_F16 = 0, 1, 2
 ATTEND_TENSOR, ATTEND_CUDA_CORE = 0, 1
 ATTEND_WS_CLEAN = 2  # flag: the workspace's merge counters are zero (left so by the previous attend)
+ATTEND_PARTIAL = 4   # flag: log-sum-exp partial rows (m, l, o[128]) instead of the normalised output
+PART_ROW = 2 + 128
 STATUS_TIMEOUT = 4
 PROBE_POPC, PROBE_ATTEND, PROBE_TOPP = 0, 1, 2
 STATUS_NONFINITE, STATUS_FP16_SATURATED = 1, 2
@@ -30,7 +32,7 @@ ERRORS = {0: "ok", -1: "invalid argument", -2: "unsupported", -3: "capacity", -4
 SYMBOLS = ("kv1b_cache_bytes", "kv1b_cache_init", "kv1b_cache_init_rounds", "kv1b_encode_append", "kv1b_attend_workspace_bytes",
            "kv1b_attend", "kv1b_attend_noalloc", "kv1b_attend_topp", "kv1b_attend_select",
            "kv1b_attend_selected_exact",
-           "kv1b_query_prep", "kv1b_scores", "kv1b_scores_probe", "kv1b_attend_wait_probe",
+           "kv1b_merge_partials", "kv1b_query_prep", "kv1b_scores", "kv1b_scores_probe", "kv1b_attend_wait_probe",
            "kv1b_read_status", "kv1b_status_string", "kv1b_version")
 
 
@@ -76,6 +78,7 @@ def lib() -> ctypes.CDLL:
             "kv1b_attend_select": (ctypes.c_int, [D, P, i32, i32, f32, i32, f32, i32, i32, i32, P, P, P, P, sz, P]),
             "kv1b_attend_selected_exact": (ctypes.c_int, [D, P, i32, i32, f32, P, P, i32, i64, i64, i64, i64, P, P,
                                                           P, P, sz, P]),
+            "kv1b_merge_partials": (ctypes.c_int, [P, i32, i64, P, P]),
             "kv1b_query_prep": (ctypes.c_int, [D, P, i32, i32, P, P, P, P, P]),
             "kv1b_scores": (ctypes.c_int, [D, P, i32, i32, f32, P, P, P, P]),
             "kv1b_scores_probe": (ctypes.c_int, [D, P, i32, i32, f32, i32, P, P, P, P, P, sz, P]),
@@ -192,16 +195,19 @@ class Cache:
         return self._ws[key]
 
     def attend(self, q: torch.Tensor, scale: float, out: torch.Tensor | None = None, engine: int = ATTEND_TENSOR,
-               num_splits: int = 0, stream=None) -> torch.Tensor:
-        """q: [batch, num_q_heads, 128] contiguous.  Returns fp32 [batch, num_q_heads, 128]."""
+               num_splits: int = 0, stream=None, partial: bool = False) -> torch.Tensor:
+        """q: [batch, num_q_heads, 128] contiguous.  Returns fp32 [batch, num_q_heads, 128], or with
+        partial=True the log-sum-exp rows [batch, num_q_heads, 130] = (m, l, o[128]) for merge_partials."""
         B, Hq, D = q.shape
         if not q.is_contiguous():
             raise ValueError("q must be contiguous")
+        width = PART_ROW if partial else D
         if out is None:
-            out = torch.empty((B, Hq, D), dtype=torch.float32, device=q.device)
+            out = torch.empty((B, Hq, width), dtype=torch.float32, device=q.device)
+        _check_buf(out, (B, Hq, width), torch.float32, "out")
         ws = self.workspace(Hq, 0)
         # after the first call the workspace's merge counters are zero (each attend leaves them so)
-        flags = engine | (ATTEND_WS_CLEAN if self._ws_clean.get(Hq, False) else 0)
+        flags = engine | (ATTEND_WS_CLEAN if self._ws_clean.get(Hq, False) else 0) | (ATTEND_PARTIAL if partial else 0)
         _check(lib().kv1b_attend(ctypes.byref(self.desc), _ptr(q), _dtype_code(q), Hq, float(scale), _ptr(out),
                                  _ptr(ws), ws.numel(), flags, num_splits, _stream(stream)), "kv1b_attend")
         self._ws_clean[Hq] = True
@@ -329,6 +335,23 @@ class Cache:
         if flags.value & STATUS_TIMEOUT:  # a timed-out attend may leave its merge counters set
             self._ws_clean.clear()
         return flags.value
+
+
+def merge_partials(parts: torch.Tensor, out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Log-sum-exp merge of partial rows [n, ..., 130] (Cache.attend(partial=True) of n disjoint token
+    ranges of the same sequences) into fp32 [..., 128] (kv1b_merge_partials)."""
+    if parts.dtype != torch.float32 or not parts.is_contiguous() or parts.shape[-1] != PART_ROW or parts.dim() < 2:
+        raise ValueError("parts must be a contiguous fp32 tensor [n, ..., 130]")
+    lead = tuple(parts.shape[1:-1])
+    rows = 1
+    for x in lead:
+        rows *= x
+    if out is None:
+        out = torch.empty(lead + (HEAD_DIM,), dtype=torch.float32, device=parts.device)
+    _check_buf(out, lead + (HEAD_DIM,), torch.float32, "out")
+    _check(lib().kv1b_merge_partials(_ptr(parts), parts.shape[0], rows, _ptr(out), _stream(stream)),
+           "kv1b_merge_partials")
+    return out
 
 
 def attend_from_host(cache: Cache, q_host: torch.Tensor, k_new_host: torch.Tensor | None, v_new_host: torch.Tensor | None,

@@ -171,6 +171,42 @@ int attend_args_check(const kv1b_cache_t* cache, const void* q, int32_t q_dtype,
 
 }  // namespace
 
+// The persistent tensor-core attend with caller-given partial-row and merge-counter buffers (used by
+// kv1b_attend_noalloc).  KV1B_ERR_UNSUPPORTED when that kernel does not take the call,
+// KV1B_ERR_WORKSPACE when its partial rows need more than part_bytes.
+int kv1b_attend_ws_buffers(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads,
+                           float scale, float* out, float* part, size_t part_bytes, unsigned* counters,
+                           cudaStream_t stream) {
+  if (!cache_ok(cache) || !q || !out || !part || !counters || !dtype_ok(q_dtype)) return KV1B_ERR_INVALID_ARG;
+  const int hc = heads_check(cache, num_q_heads);
+  if (hc != KV1B_OK) return hc;
+  if (!ws_engine_applies(cache, num_q_heads)) return KV1B_ERR_UNSUPPORTED;
+  const int G = num_q_heads / cache->num_kv_heads;
+  kv1b::AttendWsParams w;
+  memset(&w, 0, sizeof(w));
+  w.c = view(cache);
+  w.q = q;
+  w.q_dtype = q_dtype;
+  w.Hq = num_q_heads;
+  w.scale = scale;
+  const int64_t maxlen = max_length(cache);
+  w.L = static_cast<int32_t>(maxlen);
+  int ncta = 0, pieces = 0;
+  kv1b_ws_plan(cache->batch, cache->num_kv_heads, G, maxlen, num_sms(), &w.T, &w.Lt, &ncta, &pieces);
+  w.ncta = ncta;
+  w.max_pieces = pieces;
+  if (pieces > 256 ||
+      static_cast<size_t>(cache->batch) * cache->num_kv_heads * pieces * G * kv1b::kPartStride * 4 > part_bytes)
+    return KV1B_ERR_WORKSPACE;
+  w.part = part;
+  w.out = out;
+  w.status = cache->d_status;
+  w.counters = counters;
+  w.wait_tries = kv1b::kWaitTriesDefault;
+  w.stall_stage = -1;
+  return cuda_status(kv1b_launch_attend_ws(w, G, false, stream));
+}
+
 extern "C" {
 
 size_t kv1b_cache_bytes(int32_t batch, int32_t num_kv_heads, int32_t head_dim, int32_t capacity) {
@@ -269,8 +305,9 @@ int kv1b_attend(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32
                 float* out, void* ws, size_t ws_bytes, int32_t flags, int32_t num_splits, void* stream) {
   const int ac = attend_args_check(cache, q, q_dtype, num_q_heads, scale, out, ws, ws_bytes);
   if (ac != KV1B_OK) return ac;
-  if ((flags & ~(KV1B_ATTEND_CUDA_CORE | KV1B_ATTEND_WS_CLEAN)) != 0) return KV1B_ERR_INVALID_ARG;
+  if ((flags & ~(KV1B_ATTEND_CUDA_CORE | KV1B_ATTEND_WS_CLEAN | KV1B_ATTEND_PARTIAL)) != 0) return KV1B_ERR_INVALID_ARG;
   const bool ws_clean = (flags & KV1B_ATTEND_WS_CLEAN) != 0;
+  const bool partial = (flags & KV1B_ATTEND_PARTIAL) != 0;
   flags &= KV1B_ATTEND_CUDA_CORE;  // the engine
   if (num_splits < 0 || num_splits > max_splits(cache)) return KV1B_ERR_INVALID_ARG;
   const int64_t maxlen = max_length(cache);
@@ -279,6 +316,7 @@ int kv1b_attend(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32
     kv1b::AttendWsParams w;
     const int rc = ws_params(cache, q, q_dtype, num_q_heads, scale, out, ws, &w);
     if (rc != KV1B_OK) return rc;
+    w.partial_out = partial ? 1 : 0;
     return cuda_status(kv1b_launch_attend_ws(w, G, ws_clean, static_cast<cudaStream_t>(stream)));
   }
   // this engine does not use the merge counters; they are zeroed here unless the caller says they
@@ -298,6 +336,7 @@ int kv1b_attend(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32
   p.nsplit = num_splits > 0 ? num_splits : kv1b_pick_splits(cache->batch, cache->num_kv_heads, maxlen, num_sms());
   p.part = static_cast<float*>(ws);
   p.out = out;
+  p.partial_out = partial ? 1 : 0;
   for (int b = 0; b < cache->batch; ++b) p.len[b] = static_cast<int32_t>(cache->h_lengths[b]);
   return cuda_status(kv1b_launch_attend(p, G, flags, static_cast<int32_t>(maxlen), static_cast<cudaStream_t>(stream)));
 }
@@ -474,6 +513,13 @@ int kv1b_attend_wait_probe(const kv1b_cache_t* cache, const void* q, int32_t q_d
   w.stall_stage = stall_stage;
   return cuda_status(kv1b_launch_attend_ws(w, num_q_heads / cache->num_kv_heads, false,
                                            static_cast<cudaStream_t>(stream)));
+}
+
+int kv1b_merge_partials(const float* parts, int32_t nparts, int64_t rows, float* out, void* stream) {
+  if (!parts || !out || nparts < 1 || nparts > 1024 || rows < 1 || rows > 0x7fffffff) return KV1B_ERR_INVALID_ARG;
+  if (!aligned(parts, 4) || !aligned(out, 16)) return KV1B_ERR_MISALIGNED;
+  return cuda_status(kv1b_launch_merge_strided(parts, out, rows, nparts, kv1b::kPartStride, rows * kv1b::kPartStride,
+                                               false, static_cast<cudaStream_t>(stream)));
 }
 
 int kv1b_read_status(const kv1b_cache_t* cache, int32_t* flags, void* stream) {

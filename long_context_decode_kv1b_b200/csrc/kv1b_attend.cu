@@ -239,16 +239,18 @@ __global__ void __launch_bounds__(kThreads, 2) attend_kernel(const AttendParams 
 
 // log-sum-exp merge of the split partials; one block of 128 threads (channels) per (b, hq).
 // Split maxima and weights are formed in parallel, then each channel sums the splits with
-// independent loads (nsplit <= 1024).
+// independent loads (nsplit <= 1024).  Partial row k of output row r sits at part + r * row_stride +
+// k * split_stride; with partial_out the merged row (m, l, o[128]) is written instead of o / l.
 __global__ void __launch_bounds__(128) merge_kernel(const float* __restrict__ part, float* __restrict__ out,
-                                                    int nsplit) {
+                                                    int nsplit, int64_t row_stride, int64_t split_stride,
+                                                    int partial_out) {
   __shared__ float s_w[1024];
   __shared__ float s_red[4];
   const int64_t row = blockIdx.x;  // b * Hq + hq
-  const float* pr = part + row * nsplit * kPartStride;
+  const float* pr = part + row * row_stride;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   float M = -INFINITY;
-  for (int k = threadIdx.x; k < nsplit; k += 128) M = fmaxf(M, pr[k * kPartStride]);
+  for (int k = threadIdx.x; k < nsplit; k += 128) M = fmaxf(M, pr[k * split_stride]);
   #pragma unroll
   for (int m = 16; m >= 1; m >>= 1) M = fmaxf(M, __shfl_xor_sync(kFull, M, m));
   if (lane == 0) s_red[warp] = M;
@@ -257,10 +259,10 @@ __global__ void __launch_bounds__(128) merge_kernel(const float* __restrict__ pa
   __syncthreads();
   float den = 0.0f;
   for (int k = threadIdx.x; k < nsplit; k += 128) {
-    const float ms = pr[k * kPartStride];
+    const float ms = pr[k * split_stride];
     const float w = (ms != -INFINITY && M != -INFINITY) ? exp2f(ms - M) : 0.0f;
     s_w[k] = w;
-    den = __fmaf_rn(w, pr[k * kPartStride + 1], den);
+    den = __fmaf_rn(w, pr[k * split_stride + 1], den);
   }
   #pragma unroll
   for (int m = 16; m >= 1; m >>= 1) den += __shfl_xor_sync(kFull, den, m);
@@ -269,8 +271,17 @@ __global__ void __launch_bounds__(128) merge_kernel(const float* __restrict__ pa
   den = (s_red[0] + s_red[1]) + (s_red[2] + s_red[3]);
   float num = 0.0f;
   #pragma unroll 8
-  for (int k = 0; k < nsplit; ++k) num = __fmaf_rn(s_w[k], pr[k * kPartStride + 2 + threadIdx.x], num);
-  out[row * kD + threadIdx.x] = den > 0.0f ? __fdiv_rn(num, den) : 0.0f;
+  for (int k = 0; k < nsplit; ++k) num = __fmaf_rn(s_w[k], pr[k * split_stride + 2 + threadIdx.x], num);
+  if (partial_out) {
+    float* o = out + row * kPartStride;
+    if (threadIdx.x == 0) {
+      o[0] = M;
+      o[1] = den;
+    }
+    o[2 + threadIdx.x] = num;
+  } else {
+    out[row * kD + threadIdx.x] = den > 0.0f ? __fdiv_rn(num, den) : 0.0f;
+  }
 }
 
 // ---------------------------------------------------------------------------------------------
@@ -375,14 +386,23 @@ cudaError_t kv1b_launch_attend(const AttendParams& p, int32_t G, int32_t engine,
   }
 #undef KV1B_CASE
   if (e != cudaSuccess) return e;
-  merge_kernel<<<p.c.B * p.Hq, 128, 0, stream>>>(p.part, p.out, p.nsplit);
+  merge_kernel<<<p.c.B * p.Hq, 128, 0, stream>>>(p.part, p.out, p.nsplit, static_cast<int64_t>(p.nsplit) * kPartStride,
+                                                  kPartStride, p.partial_out);
   return cudaGetLastError();
 }
 
 // Log-sum-exp merge of nsplit partial rows (m in log2 units, l, o[128]) per row: [rows][nsplit][2 + 128].
 cudaError_t kv1b_launch_merge(const float* part, float* out, int32_t rows, int32_t nsplit, cudaStream_t stream) {
   if (nsplit < 1 || nsplit > 1024 || rows < 1) return cudaErrorInvalidValue;
-  merge_kernel<<<rows, 128, 0, stream>>>(part, out, nsplit);
+  merge_kernel<<<rows, 128, 0, stream>>>(part, out, nsplit, static_cast<int64_t>(nsplit) * kPartStride, kPartStride, 0);
+  return cudaGetLastError();
+}
+
+cudaError_t kv1b_launch_merge_strided(const float* part, float* out, int64_t rows, int32_t nsplit, int64_t row_stride,
+                                      int64_t split_stride, bool partial_out, cudaStream_t stream) {
+  if (nsplit < 1 || nsplit > 1024 || rows < 1 || rows > 0x7fffffff) return cudaErrorInvalidValue;
+  merge_kernel<<<static_cast<unsigned>(rows), 128, 0, stream>>>(part, out, nsplit, row_stride, split_stride,
+                                                                partial_out ? 1 : 0);
   return cudaGetLastError();
 }
 

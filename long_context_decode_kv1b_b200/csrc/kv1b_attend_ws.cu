@@ -357,7 +357,7 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
   const uint32_t c_off = static_cast<uint32_t>(tl * kTileSmem + (32 * jw + 8 * (lane >> 4) + (lane & 7)) * 128);
   const uint32_t c_kx0 = static_cast<uint32_t>((((lane >> 3) & 1) ^ (lane & 7)) << 4);
   // weight-rounding dither: a Weyl sequence over the lane's 32-token slices (top byte of
-  // n * 0x9E3779B9 + lane constant, n = slice index in the segment), offset by a quarter turn per token
+  // n * 0x9E3779B9 + lane * 0x6A09E667, n = slice index in the segment), one value per lane and slice
   const uint32_t weyl_c = static_cast<uint32_t>(lane) * 0x6A09E667u;
 
   // per-lane state
@@ -419,6 +419,7 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
     float* sm_m = reinterpret_cast<float*>(smem + kOffW);  // [G][256] piece maxima, then weights
     float* sm_l = sm_m + 4 * 256;                          // [G][256] piece sums
     float* sm_d = sm_l + 4 * 256;                          // [G] denominators
+    float* sm_M = sm_d + 4;                                // [G] maxima
     const int b = seg / c.Hkv, kvh = seg - b * c.Hkv;
     const int64_t stride = static_cast<int64_t>(G) * kPartStride;  // between pieces
     const float* base = p.part + static_cast<int64_t>(seg) * p.max_pieces * G * kPartStride;
@@ -443,7 +444,10 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
       }
       #pragma unroll
       for (int m = 16; m >= 1; m >>= 1) den += __shfl_xor_sync(kFull, den, m);
-      if (lane == 0) sm_d[warp] = den;
+      if (lane == 0) {
+        sm_d[warp] = den;
+        sm_M[warp] = M;
+      }
     }
     named_bar(1, kThreads);
     const int ch = threadIdx.x & 127;
@@ -458,8 +462,18 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
       }
       for (; k < n; ++k) acc[0] = __fmaf_rn(w[k], o[k * stride], acc[0]);
       const float den = sm_d[h];
-      p.out[(static_cast<int64_t>(b) * p.Hq + kvh * G + h) * kD + ch] =
-          den > 0.0f ? __fdiv_rn(__fadd_rn(__fadd_rn(acc[0], acc[1]), __fadd_rn(acc[2], acc[3])), den) : 0.0f;
+      const float num = __fadd_rn(__fadd_rn(acc[0], acc[1]), __fadd_rn(acc[2], acc[3]));
+      const int64_t orow = static_cast<int64_t>(b) * p.Hq + kvh * G + h;
+      if (p.partial_out) {  // the segment's log-sum-exp row (m, l, o[128]) for a later merge
+        float* o = p.out + orow * kPartStride;
+        if (ch == 0) {
+          o[0] = sm_M[h];
+          o[1] = den;
+        }
+        o[2 + ch] = num;
+      } else {
+        p.out[orow * kD + ch] = den > 0.0f ? __fdiv_rn(num, den) : 0.0f;
+      }
     }
   };
 
@@ -723,16 +737,16 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
       // ---------------- weights of group t: W = rint(p scale 2^E + d) < 2^32, d a dither in [-1/2, 1/2)
       // that makes the rounding unbiased (weights of a long tail far below the maximum are fractions
       // of a unit, which plain rounding would send to zero together)
+      // 2^23 + (top byte of the lane's hash for this slice) as a float, then / 256 - 1/2 exactly; the
+      // lane's four tokens (and all heads) share it, each draw uniform over the slices
       const uint32_t weyl = static_cast<uint32_t>(rel >> 5) * 0x9E3779B9u + weyl_c;
+      const float dz = __fmaf_rn(__uint_as_float(prmt(weyl, 0x4B000000u, 0x7543)), 0x1p-8f, -32768.5f);
       #pragma unroll
       for (int kk = 0; kk < 2; ++kk) {
         uint32_t W[2][4];
         #pragma unroll
         for (int e = 0; e < 2; ++e) {
           const float s2g = __fmul_rn(sc[kk][e], s2e_t);
-          // 2^23 + (top byte of the token's hash) as a float, then / 256 - 1/2 exactly
-          const uint32_t hb = weyl + static_cast<uint32_t>(2 * kk + e) * 0x40000000u;
-          const float dz = __fmaf_rn(__uint_as_float(prmt(hb, 0x4B000000u, 0x7543)), 0x1p-8f, -32768.5f);
           #pragma unroll
           for (int h = 0; h < 4; ++h) {
             W[e][h] = __float2uint_rn(__fmaf_rn(ph[kk][e][h], s2g, dz));

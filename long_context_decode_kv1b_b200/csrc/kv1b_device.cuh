@@ -202,17 +202,78 @@ __device__ __forceinline__ double half_bits_to_double(uint32_t hb) {
 }
 
 // Smallest non-negative finite binary16 h with 15*h >= D (15*h is exact in fp64); 0x7bff and
-// *sat on overflow.  Starts next to the answer and walks at most a few steps.
-__device__ __forceinline__ uint32_t half_scale_up(double D, int* sat) {
+// *sat on overflow.  Starts next to the answer (a float estimate of D / 15, within a binary16 step
+// of it) and walks at most a few steps, each checked exactly in fp64.
+__device__ __forceinline__ uint32_t half_scale_up_f64(double D, int* sat) {
   if (!(D > 0.0)) return 0u;
   if (D > 15.0 * 65504.0) { *sat = 1; return 0x7bffu; }
-  uint32_t hb = __half_as_ushort(__float2half_rz(__double2float_rz(D / 15.0)));
+  uint32_t hb = __half_as_ushort(__float2half_rz(__fmul_rz(__double2float_rz(D), 0x1.111112p-4f)));
   if (hb > 0x7bffu) hb = 0x7bffu;
   #pragma unroll 1
   for (int i = 0; i < 8 && 15.0 * half_bits_to_double(hb) < D; ++i) ++hb;
   #pragma unroll 1
-  for (int i = 0; i < 8 && hb > 0u && 15.0 * half_bits_to_double(hb - 1u) >= D; ++i) --hb;
+  for (int i = 0; i < 8 && hb > 0u && 15.0 * half_bits_to_double(hb - 1u) >= D; --hb, ++i) {}
   return hb;
+}
+
+// The same for D = fl64(mx - mn) (mn a binary16 value, mx >= mn), in fp32 arithmetic: TwoSum (Knuth)
+// gives D = hi + lo exactly; when that sum fits the 53 bits of a double (always, unless lo is below
+// hi's 29th bit: then the fp64 rounding of D matters and the fp64 form runs), 15 h >= D is decided
+// exactly as 15 h - hi >= lo: 15 h is exact, and 15 h - hi is exact whenever 15 h and hi are within a
+// factor of two (Sterbenz) and otherwise far from lo on the right side.
+__device__ __forceinline__ uint32_t half_scale_up(float mx, float mn, int* sat) {
+  const float hi = __fsub_rn(mx, mn);
+  const float bb = __fsub_rn(hi, mx);
+  const float lo = __fadd_rn(__fsub_rn(mx, __fsub_rn(hi, bb)), __fsub_rn(-mn, bb));
+  if (lo != 0.0f && fabsf(lo) < __fmul_rn(hi, 0x1p-28f))
+    return half_scale_up_f64(static_cast<double>(mx) - static_cast<double>(mn), sat);
+  if (!(hi > 0.0f)) return 0u;
+  if (hi > 982560.0f || (hi == 982560.0f && lo > 0.0f)) { *sat = 1; return 0x7bffu; }  // 15 * 65504
+  auto covers = [&](uint32_t hb) {
+    const float h15 = __fmul_rn(15.0f, __half2float(__ushort_as_half(static_cast<unsigned short>(hb))));
+    return __fsub_rn(h15, hi) >= lo;
+  };
+  uint32_t hb = __half_as_ushort(__float2half_rz(__fmul_rz(hi, 0x1.111112p-4f)));
+  if (hb > 0x7bffu) hb = 0x7bffu;
+  #pragma unroll 1
+  for (int i = 0; i < 8 && !covers(hb); ++i) ++hb;
+  #pragma unroll 1
+  for (int i = 0; i < 8 && hb > 0u && covers(hb - 1u); --hb, ++i) {}
+  return hb;
+}
+
+// The smallest non-negative finite binary16 h with 15 h >= D for D = fl64(mx - mn), as half_scale_up,
+// without a data-dependent loop in the common case: the float estimate e of D / 15 is at most two
+// binary16 steps below the answer and never above it, so the answer is e, e + 1 or e + 2 unless
+// e - 1 already covers D; only then (or for e + 2 failing) does the warp take the walking form.
+__device__ __forceinline__ uint32_t half_scale_up_fast(float mx, float mn, int* sat) {
+  const float hi = __fsub_rn(mx, mn);
+  const float bb = __fsub_rn(hi, mx);
+  const float lo = __fadd_rn(__fsub_rn(mx, __fsub_rn(hi, bb)), __fsub_rn(-mn, bb));
+  const bool exact = !(lo != 0.0f && fabsf(lo) < __fmul_rn(hi, 0x1p-28f));
+  auto covers = [&](uint32_t hb) {
+    const float h15 = __fmul_rn(15.0f, __half2float(__ushort_as_half(static_cast<unsigned short>(hb))));
+    return __fsub_rn(h15, hi) >= lo;
+  };
+  uint32_t e = __half_as_ushort(__float2half_rz(__fmul_rz(hi, 0x1.111112p-4f)));
+  e = e > 0x7bfdu ? 0x7bfdu : e;
+  const bool cm = e > 0u && covers(e - 1u), c0 = covers(e), c1 = covers(e + 1u), c2 = covers(e + 2u);
+  const bool normal = exact && hi > 0.0f && hi < 982560.0f && !cm && c2;
+  uint32_t hb = c0 ? e : (c1 ? e + 1u : e + 2u);
+  if (__any_sync(kFull, !normal)) {  // rare: saturation, an inexact fp64 range, or an estimate off by more
+    const uint32_t slow = half_scale_up(mx, mn, sat);
+    hb = normal ? hb : slow;
+  }
+  return hb;
+}
+
+// Correctly rounded x / y from r = RN(1 / y): q0 = RN(x r) is within an ulp of x / y, the residual
+// x - y q0 is exact in a fused multiply-add, and RN(q0 + (x - y q0) r) = RN(x / y) when nothing
+// underflows or overflows (Markstein's correction theorem: P. Markstein, "Computation of elementary
+// functions on the IBM RISC System/6000 processor", IBM J. Res. Dev. 34 (1), 1990).
+__device__ __forceinline__ float div_markstein(float x, float y, float r) {
+  const float q0 = __fmul_rn(x, r);
+  return __fmaf_rn(__fmaf_rn(-y, q0, x), r, q0);
 }
 
 // Largest finite binary16 <= x (saturates at -65504 with *sat).

@@ -45,7 +45,8 @@ struct AttendParams {
   float scale;
   int32_t nsplit;
   float* part;   // [B][Hq][nsplit][2 + 128]: m (log2 units), l, o[128]
-  float* out;    // [B][Hq][128]
+  float* out;    // [B][Hq][128], or [B][Hq][2 + 128] partial rows when partial_out
+  int32_t partial_out;
   int32_t len[KV1B_MAX_BATCH];
 };
 
@@ -166,6 +167,7 @@ struct alignas(64) AttendWsParams {
   float* out;          // [B][Hq][128]
   int32_t* status;     // cache status word (timeout flag)
   unsigned* counters;  // [B * Hkv] pieces of each segment written so far (zeroed before the launch)
+  int32_t partial_out; // the merge writes log-sum-exp rows (m, l, o[128]) to out instead of o / l
   int32_t wait_tries;  // suspended tries (<= 0.5 ms each) before a pipeline wait gives up
   int32_t stall_stage; // test hook: each CTA's producer stops before this stage (-1: never)
   int32_t* probe_A;    // test hook (probe instantiation only): [B][Hq][cap] raw score products 8 A,
@@ -211,10 +213,17 @@ size_t kv1b_topp_workspace_bytes(int32_t rows, int32_t cap);
 void kv1b_topp_carve(kv1b::ToppParams* p, void* ws, int32_t rows, int32_t cap);
 int kv1b_pick_splits(int32_t B, int32_t Hkv, int64_t max_len, int num_sms);
 cudaError_t kv1b_launch_merge(const float* part, float* out, int32_t rows, int32_t nsplit, cudaStream_t stream);
+// Log-sum-exp merge of nsplit partial rows per output row; partial row k of output row r at
+// part + r * row_stride + k * split_stride (floats).  partial_out: write (m, l, o[128]) rows.
+cudaError_t kv1b_launch_merge_strided(const float* part, float* out, int64_t rows, int32_t nsplit, int64_t row_stride,
+                                      int64_t split_stride, bool partial_out, cudaStream_t stream);
 size_t kv1b_exact_workspace_bytes(int32_t rows, int32_t cap);
 void kv1b_exact_carve(kv1b::ExactParams* p, void* ws, int32_t rows);
 cudaError_t kv1b_launch_exact(const kv1b::ExactParams& p, int32_t rows, int32_t num_sms, cudaStream_t stream);
 bool kv1b_ws_supported(int32_t G);
+int kv1b_attend_ws_buffers(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads,
+                           float scale, float* out, float* part, size_t part_bytes, unsigned* counters,
+                           cudaStream_t stream);
 void kv1b_ws_plan(int32_t B, int32_t Hkv, int32_t G, int64_t L, int num_sms, int64_t* T, int64_t* Lt, int* ncta,
                   int* max_pieces);
 cudaError_t kv1b_launch_attend_ws(kv1b::AttendWsParams& p, int32_t G, bool counters_clean, cudaStream_t stream,

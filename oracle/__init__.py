@@ -11,6 +11,7 @@ the web page and section it follows (RaBitQCache; H1B-KV; the H1IB-KV news artic
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import subprocess
 
@@ -234,6 +235,22 @@ def attend(enc: dict, q, sgn, scale: float) -> np.ndarray:
     out = np.empty(d, np.float64)
     lib().ref_attend_head(*ptrs, L, _p(q), _p(sgn), float(scale), d, _p(out))
     return out
+
+
+def attend_partial(enc: dict, q, sgn, scale: float):
+    """The attention sums of one query head over one encoded token range, before normalisation:
+    (m, l, o[d]) with m = max_t s_t log2(e), l = sum_t 2^(s_t log2(e) - m), o = sum_t 2^(s_t log2(e) - m)
+    vhat_t in fp64 from the fp32 logits (the same logits and dequantised values as `attend`); an empty
+    range gives (-inf, 0, 0).  Ranges merge by log-sum-exp: out = sum_k 2^(m_k - M) o_k / sum_k
+    2^(m_k - M) l_k, M = max_k m_k -- the split of one context over several devices."""
+    L = np.shape(enc["bits"])[0]
+    d = np.shape(enc["bits"])[1] * 32
+    if L == 0:
+        return -math.inf, 0.0, np.zeros(d)
+    s = logits(enc, query_prep(q, sgn), scale).astype(np.float64) * (1.0 / math.log(2.0))
+    m = float(s.max())
+    w = np.exp2(s - m)
+    return m, float(w.sum()), w @ dequant(enc["codes"], enc["sm"])
 
 
 def exp2_coef(k: int) -> float:

@@ -56,6 +56,81 @@ def test_encode_bit_exact_ragged_appends(dtype):
     assert cache.status() == 0
 
 
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
+def test_prefill_encode_bit_exact_ragged_groups(dtype):
+    # appends of >= 64 tokens take the prefill form (one warp per 8-token code word): starts and ends
+    # inside an 8-token group and inside a 128-token tile, whole tiles, single tokens in between
+    B, H = 2, 3
+    appends = [100, 200, 64, 1, 65, 300, 7, 129]
+    cache, host = build_cache(B, H, appends, dtype, seed=321, data_seed=4)
+    torch.cuda.synchronize()
+    D = oracle.signs(321)
+    assert cache.lengths == [sum(appends)] * B
+    for b in range(B):
+        for h in range(H):
+            assert_planes_equal(gpu_head_planes(cache, b, h, host.n), host.encode(b, h, D), f"prefill b{b} h{h}")
+    assert cache.status() == 0
+
+
+def test_prefill_encode_strided_rows_and_special_values():
+    B, H, n = 2, 2, 200
+    g = torch.Generator(device=DEV).manual_seed(15)
+    wide = torch.randn((B, n, H, 2, 128), generator=g, device=DEV)
+    wide[0, 3, 0, 0, :] = 0.0                     # zero key: every sign bit 1, cinv = 1
+    wide[1, 77, 1, 0, 5:40] = 0.0                 # exact zeros inside a key
+    wide[0, 9, 1, 1, :] = 0.25                    # a constant (binary16-exact) value row
+    wide[1, 150, 0, 1, 32:64] = -3.0e4            # large but representable
+    K, V = wide[:, :, :, 0, :], wide[:, :, :, 1, :]  # token stride 512, head stride 256 elements
+    cache = kv.Cache(B, H, 256, seed=99)
+    cache.append(K[:, :5], V[:, :5])                  # decode form first, then prefill from mid-group
+    cache.append(K[:, 5:], V[:, 5:])
+    host = HostKV(B, H, 256)
+    host.add(K, V)
+    D = oracle.signs(99)
+    for b in range(B):
+        for h in range(H):
+            assert_planes_equal(gpu_head_planes(cache, b, h, n), host.encode(b, h, D), f"strided prefill b{b} h{h}")
+    assert cache.status() == 0
+    V2 = V[:, :80].clone()
+    V2[1, 70, 0, 3] = float("nan")
+    cache2 = kv.Cache(B, H, 128, seed=1)
+    cache2.append(K[:, :80].contiguous(), V2.contiguous())
+    assert cache2.status() & kv.STATUS_NONFINITE
+
+
+def edge_value_rows(n: int, seed: int) -> torch.Tensor:
+    """[n, 128] fp32 rows whose first 32-channel group is a scale-search edge case, cycling through:
+    a range D = fl64(max - min) that fp64 rounds (min = -15 * 2^-24, max = 2^-140), a range of exactly
+    15 h (h = 0.5 and a subnormal binary16), the saturation boundary 15 * 65504 and just above it, a
+    constant group, and a range of one subnormal binary16 step; the other groups are random."""
+    g = torch.Generator().manual_seed(seed)
+    rows = torch.randn((n, 128), generator=g)
+    cases = [(-15 * 2.0 ** -24, 2.0 ** -140), (0.0, 7.5), (0.0, 15 * 3 * 2.0 ** -24), (0.0, 982560.0),
+             (0.0, 982560.0625), (1.25, 1.25), (-2.0 ** -24, 0.0), (-3.0, 2.0 ** -149)]
+    for i in range(n):
+        lo, hi = cases[i % len(cases)]
+        grp = torch.full((32,), lo)
+        grp[7] = hi
+        rows[i, :32] = grp
+    return rows
+
+
+@pytest.mark.parametrize("n", [5, 100])
+def test_value_scale_search_edge_groups(n):
+    # n = 5 takes the decode form of the encode, n = 100 the prefill form
+    B, H = 1, 2
+    V = torch.stack([edge_value_rows(n, 1), edge_value_rows(n, 2)], dim=1).view(B, n, H, 128).to(DEV)
+    K = torch.randn((B, n, H, 128), device=DEV, generator=torch.Generator(device=DEV).manual_seed(3))
+    cache = kv.Cache(B, H, 128, seed=5)
+    cache.append(K, V)
+    host = HostKV(B, H, 128)
+    host.add(K, V)
+    D = oracle.signs(5)
+    for h in range(H):
+        assert_planes_equal(gpu_head_planes(cache, 0, h, n), host.encode(0, h, D), f"scale edges n{n} h{h}")
+    assert cache.status() & kv.STATUS_FP16_SATURATED  # the group just above 15 * 65504
+
+
 def test_encode_strided_inputs_and_special_values():
     B, H, n = 1, 2, 48
     g = torch.Generator(device=DEV).manual_seed(5)
@@ -381,6 +456,37 @@ def test_exact_kv_dtypes_and_strides(dtype):
     exact_check(cache, q, 0.25, Kc, Vc, sel, cnt, G, where=f"{dtype} contiguous")
 
 
+def device_address_of_host(t: torch.Tensor) -> int:
+    """The device address of pinned host memory (0 when the device cannot address it)."""
+    from cuda.bindings import runtime as rt
+
+    err, attr = rt.cudaPointerGetAttributes(t.data_ptr())
+    if err != rt.cudaError_t.cudaSuccess or attr.type != rt.cudaMemoryType.cudaMemoryTypeHost:
+        return 0
+    return int(attr.devicePointer)
+
+
+def test_exact_kv_from_pinned_host_memory():
+    # the exact keys / values stay in host memory (RaBitQCache, core idea: full-precision KV kept off
+    # the GPU); the kernel reads the selected rows through the device's mapping of pinned memory
+    B, Hkv, G, L = 2, 2, 4, 3000
+    cache, K, V = cache_with_exact(B, Hkv, L, torch.bfloat16, seed=44, data_seed=8)
+    q = torch.randn((B, Hkv * G, 128), device=DEV, generator=torch.Generator(device=DEV).manual_seed(12))
+    _, sel, cnt = cache.attend_topp(q, 0.3, 0.9)
+    Kh = torch.empty(K.shape, dtype=K.dtype, pin_memory=True)
+    Vh = torch.empty(V.shape, dtype=V.dtype, pin_memory=True)
+    Kh.copy_(K)
+    Vh.copy_(V)
+    torch.cuda.synchronize()
+    for t in (Kh, Vh):
+        if device_address_of_host(t) != t.data_ptr():
+            pytest.skip("pinned host memory is not addressable at its host address on this device")
+    out_dev = cache.attend_selected_exact(q, 0.3, K, V, sel, cnt)
+    out_host = exact_check(cache, q, 0.3, Kh, Vh, sel, cnt, G, where="host KV")
+    assert torch.allclose(out_host, out_dev, rtol=0, atol=0)  # the same arithmetic on the same rows
+    assert cache.status() == 0
+
+
 # ------------------------------------------------------------------ Top-k budget and the kept window
 def select_check(cache, host, q, scale, G, signs, mode, p=1.0, k=0, sink=0, recent=0, where=""):
     out, sel, cnt = cache.attend_select(q, scale, mode, p=p, k=k, sink=sink, recent=recent)
@@ -587,3 +693,43 @@ def test_attend_long_tail_below_a_dominant_token(gap_lo, gap_hi):
         out = cache.attend(q, scale, engine=engine)
         assert_rows_close(out.cpu().numpy(), ref, where=f"tail {gap_lo}-{gap_hi} e{engine}")
     assert cache.status() == 0
+
+
+# ------------------------------------------------------------------ a context split: partial rows + merge
+@pytest.mark.parametrize("engine", [kv.ATTEND_TENSOR, kv.ATTEND_CUDA_CORE])
+def test_context_split_partial_rows_merge_to_the_whole_attention(engine):
+    # one sequence's 9,100 tokens in three caches (three ranks of a context split, emulated one after
+    # another on this GPU) plus an empty fourth: each cache's log-sum-exp rows, merged by
+    # kv1b_merge_partials, equal the oracle's attention over the whole context; every partial row
+    # normalised equals the oracle's attention over its own range
+    from long_context_decode_kv1b_b200 import context_split as cs
+
+    B, Hkv, G, L, world = 2, 2, 4, 9100, 3
+    g = torch.Generator(device=DEV).manual_seed(77)
+    K = torch.randn((B, L, Hkv, 128), generator=g, device=DEV).to(torch.bfloat16)
+    V = torch.randn((B, L, Hkv, 128), generator=g, device=DEV).to(torch.bfloat16)
+    q = torch.randn((B, Hkv * G, 128), generator=g, device=DEV).to(torch.bfloat16)
+    D = oracle.signs(8)
+    parts, hosts = [], []
+    for r in range(world + 1):
+        t0, t1 = cs.shard_bounds(L, world, r) if r < world else (L, L)
+        cap = max(128, (t1 - t0 + 127) // 128 * 128)
+        cache = kv.Cache(B, Hkv, cap, seed=8)
+        host = HostKV(B, Hkv, cap)
+        if t1 > t0:
+            cache.append(K[:, t0:t1].contiguous(), V[:, t0:t1].contiguous())
+            host.add(K[:, t0:t1], V[:, t0:t1])
+        parts.append(cache.attend(q, 0.3, engine=engine, partial=True))
+        hosts.append(host)
+    allp = torch.stack(parts)  # [world + 1, B, Hq, 130], the gathered rows
+    out = kv.merge_partials(allp)
+    torch.cuda.synchronize()
+    whole = HostKV(B, Hkv, L)
+    whole.add(K, V)
+    ref = oracle_attend_all(whole, q, D, 0.3, G)
+    assert_rows_close(out.cpu().numpy(), ref, where=f"split merge e{engine}")
+    P = allp.cpu().numpy()
+    assert np.all(P[world, :, :, 0] == -np.inf) and not P[world, :, :, 1:].any()  # the empty range
+    for r in range(world):
+        sub = oracle_attend_all(hosts[r], q, D, 0.3, G)
+        assert_rows_close(P[r, :, :, 2:] / P[r, :, :, 1:2], sub, where=f"range {r} e{engine}")

@@ -680,3 +680,26 @@ def test_three_round_estimator_nearly_unbiased_and_scale_free():
     kk = (R.T @ np.ones(d) / d ** 3).astype(np.float32)  # R kk = (1, ..., 1) up to fp32 rounding
     enc = oracle.encode(kk[None, :], np.zeros((1, d), np.float32), S)
     assert abs(1.0 / enc["cinv"][0] - d) <= 1e-4 * d
+
+
+def test_attend_partial_sums_normalise_to_attend_and_merge_by_log_sum_exp():
+    # the unnormalised sums of a token range: o / l is the range's attention; two ranges merged by
+    # log-sum-exp give the attention over both (a context split over devices); an empty range is the
+    # identity of the merge
+    rng = np.random.default_rng(4)
+    K = rng.standard_normal((900, 128)).astype(np.float32)
+    V = rng.standard_normal((900, 128)).astype(np.float32)
+    q = rng.standard_normal(128).astype(np.float32)
+    D = oracle.signs(2)
+    whole = oracle.encode(K, V, D)
+    ref = oracle.attend(whole, q, D, 0.4)
+    m, l, o = oracle.attend_partial(whole, q, D, 0.4)
+    assert np.abs(o / l - ref).max() <= 1e-12 * np.abs(ref).max()
+    parts = [oracle.attend_partial(oracle.encode(K[a:b], V[a:b], D), q, D, 0.4) for a, b in ((0, 333), (333, 900))]
+    M = max(p[0] for p in parts)
+    num = sum(2.0 ** (p[0] - M) * p[2] for p in parts)
+    den = sum(2.0 ** (p[0] - M) * p[1] for p in parts)
+    assert np.abs(num / den - ref).max() <= 1e-12 * np.abs(ref).max()
+    assert abs(M - m) == 0.0  # the larger range maximum is the whole maximum
+    me, le, oe = oracle.attend_partial(oracle.encode(K[:0], V[:0], D), q, D, 0.4)
+    assert me == -math.inf and le == 0.0 and not oe.any()

@@ -15,9 +15,9 @@ a 23-bit fixed point rounds the tail's weights to a unit or none and biases the 
 The engine adds a dither d in [-1/2, 1/2) before rounding, W = rint(p * scale * 2^E + d): tokens
 2^-26.6 or more below the reference maximum get weights under half a unit, which plain rounding sends
 to zero all together -- a bias that grows with the number of such tokens one reference covers.  d is
-the top byte of a Weyl sequence (n * 0x9E3779B9 + lane * 0x6A09E667 + j * 2^30, n the 32-token slice,
-lane = 4 (token & 7) + group, j = 2 ((token & 31) >> 4) + ((token >> 3) & 1)), so over many tokens
-every fractional weight keeps its expected value; the model reproduces that mapping.
+the top byte of a Weyl sequence (n * 0x9E3779B9 + lane * 0x6A09E667, n the 32-token slice, lane =
+4 (token & 7) + group: the lane that forms the weights of those tokens), so over many tokens every
+fractional weight keeps its expected value; the model reproduces that mapping.
 """
 import math
 
@@ -45,10 +45,8 @@ def dither(t0: int, t1: int, group: int) -> np.ndarray:
     """The engine's rounding offsets of tokens t0 .. t1 - 1 (segment positions) for one value group."""
     t = np.arange(t0, t1, dtype=np.uint64)
     n = t >> np.uint64(5)
-    tau = t & np.uint64(31)
-    lane = (tau & np.uint64(7)) * np.uint64(4) + np.uint64(group)
-    j = np.uint64(2) * (tau >> np.uint64(4)) + ((tau >> np.uint64(3)) & np.uint64(1))
-    h = (n * np.uint64(0x9E3779B9) + lane * np.uint64(0x6A09E667) + j * np.uint64(0x40000000)) & np.uint64(0xFFFFFFFF)
+    lane = (t & np.uint64(7)) * np.uint64(4) + np.uint64(group)
+    h = (n * np.uint64(0x9E3779B9) + lane * np.uint64(0x6A09E667)) & np.uint64(0xFFFFFFFF)
     return ((h >> np.uint64(24)).astype(np.float64) / 256.0 - 0.5).astype(np.float32)
 
 

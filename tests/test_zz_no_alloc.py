@@ -1,18 +1,20 @@
 """kv1b_attend_noalloc: attention for callers that cannot allocate device memory or pass a
 workspace (e.g. a framework whose allocator owns all device memory, or a decode loop where
-cudaMalloc / cudaFree would synchronise the device).  The entry point keeps its split partials in
-a fixed device array inside the library.  Called through the C ABI with ctypes; its output must
-match kv1b_attend's within the parity tolerance, on two calls in a row.  This file sorts last so a
-run that stops at the first failure has already run every other test."""
+cudaMalloc / cudaFree would synchronise the device).  The entry point keeps its split partials and
+merge counters in a fixed device array inside the library.  Called through the C ABI with ctypes;
+its output must match the CPU oracle within the parity tolerance, on two calls in a row, with the
+persistent tensor-core kernel (G = 4, equal lengths) and the CUDA-core split engine (G = 8, ragged
+lengths, or asked for).  This file sorts last so a run that stops at the first failure has already
+run every other test."""
 import ctypes
 import math
 
-import numpy as np
 import pytest
 import torch
 
+import oracle
 import long_context_decode_kv1b_b200 as kv
-from parity_utils import assert_rows_close
+from parity_utils import HostKV, assert_rows_close, oracle_attend_all
 
 pytestmark = pytest.mark.gpu
 
@@ -36,26 +38,30 @@ def call_noalloc(cache, q, scale, engine=kv.ATTEND_TENSOR):
     return rc, out
 
 
-def test_noalloc_matches_attend_on_two_calls_in_a_row():
+@pytest.mark.parametrize("G,appends", [(4, [6000]), (8, [3000]), (4, [2500, 1])])
+def test_noalloc_matches_the_oracle_on_two_calls_in_a_row(G, appends):
     dev = "cuda"
-    g = torch.Generator(device=dev).manual_seed(31)
-    B, Hkv, G = 2, 4, 4
-    cache = kv.Cache(B, Hkv, 8192, seed=3)
-    K = torch.randn((B, 6000, Hkv, 128), generator=g, device=dev).to(torch.bfloat16)
-    V = torch.randn((B, 6000, Hkv, 128), generator=g, device=dev).to(torch.bfloat16)
-    cache.append(K, V)
+    g = torch.Generator(device=dev).manual_seed(31 + G)
+    B, Hkv = 2, 4
+    total = sum(appends)
+    cache = kv.Cache(B, Hkv, (total + 127) // 128 * 128, seed=3)
+    host = HostKV(B, Hkv, cache.capacity)
+    for n in appends:
+        K = torch.randn((B, n, Hkv, 128), generator=g, device=dev).to(torch.bfloat16)
+        V = torch.randn((B, n, Hkv, 128), generator=g, device=dev).to(torch.bfloat16)
+        cache.append(K, V)
+        host.add(K, V)
     scale = 1.0 / math.sqrt(128)
+    D = oracle.signs(3)
     for call in range(2):
         q = torch.randn((B, Hkv * G, 128), generator=g, device=dev).to(torch.bfloat16)
-        ref = cache.attend(q, scale).cpu().numpy()
-        rc, out = call_noalloc(cache, q, scale)
-        assert rc == 0, f"call {call}: {kv.lib().kv1b_status_string(rc)}"
-        torch.cuda.synchronize()
-        assert_rows_close(out.cpu().numpy(), ref, where=f"noalloc call {call}")
-        # the CUDA-core engine through the same fixed scratch
-        rc, out_c = call_noalloc(cache, q, scale, engine=kv.ATTEND_CUDA_CORE)
-        assert rc == 0
-        assert_rows_close(out_c.cpu().numpy(), ref, where=f"noalloc cuda-core call {call}")
+        ref = oracle_attend_all(host, q, D, scale, G)
+        for engine in (kv.ATTEND_TENSOR, kv.ATTEND_CUDA_CORE):
+            rc, out = call_noalloc(cache, q, scale, engine=engine)
+            assert rc == 0, f"call {call}: {kv.lib().kv1b_status_string(rc)}"
+            torch.cuda.synchronize()
+            assert_rows_close(out.cpu().numpy(), ref, where=f"noalloc G{G} engine {engine} call {call}")
+    assert cache.status() == 0
 
 
 def test_noalloc_refuses_shapes_beyond_its_scratch():
@@ -63,7 +69,7 @@ def test_noalloc_refuses_shapes_beyond_its_scratch():
     cache = kv.Cache(64, 16, 128, seed=0)
     q = torch.zeros((64, 128, 128), dtype=torch.float32, device="cuda")
     assert 64 * 128 * 520 > SCRATCH_BYTES
-    rc, out = call_noalloc(cache, q, 0.1)
+    rc, out = call_noalloc(cache, q, 0.1, engine=kv.ATTEND_CUDA_CORE)
     assert rc == -5
     torch.cuda.synchronize()
     assert torch.isnan(out).all()  # nothing was launched or written
