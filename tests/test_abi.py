@@ -79,7 +79,7 @@ def test_attend_rejects_unknown_flag_bits_without_launching(lib):
     for name in ("k_bits", "k_norm", "k_cinv", "v_codes", "v_sm", "signs", "d_lengths", "d_status"):
         setattr(d, name, 0x10000)
     buf = ctypes.c_void_p(0x20000)
-    for flags in (4, 8, -1):
+    for flags in (8, 16, 1 << 30, -1):  # bits 0-2 are the engine, KV1B_ATTEND_WS_CLEAN and KV1B_ATTEND_PARTIAL
         assert lib.kv1b_attend(ctypes.byref(d), buf, kv.DTYPE_F32, 4, ctypes.c_float(0.1), buf, buf, 1 << 20,
                                flags, 0, None) == -1
 
