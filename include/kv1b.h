@@ -63,8 +63,9 @@ extern "C" {
 
 /* kv1b_attend flags: which engine forms the probability-weighted sum of values */
 #define KV1B_ATTEND_TENSOR 0     /* default: integer mma.sync (u8 codes x 32-bit fixed-point weights, exact s32
-                                    accumulation) in a persistent kernel, for G in {1, 2, 4}, equal sequence
-                                    lengths and an automatic split count; other shapes run the CUDA-core engine */
+                                    accumulation) in a persistent kernel, for equal sequence lengths and an
+                                    automatic split count (G > 4 as launches of at most 4 query heads, each
+                                    streaming the cache); other shapes run the CUDA-core engine */
 #define KV1B_ATTEND_CUDA_CORE 1  /* fp32 FMA on the CUDA cores (split-K grid, any shape) */
 #define KV1B_ATTEND_WS_CLEAN 2   /* OR-ed into the engine: the workspace's merge counters are zero, as every
                                     kv1b_attend that ran to completion on this workspace with the same cache
@@ -189,8 +190,8 @@ int kv1b_attend(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32
  * latency-critical decode loop) nor pass a workspace buffer (a fixed ABI with inputs and outputs
  * only).  Same arguments and result as kv1b_attend minus ws / ws_bytes / num_splits; flags is
  * KV1B_ATTEND_TENSOR or KV1B_ATTEND_CUDA_CORE (KV1B_ATTEND_WS_CLEAN is not accepted).
- * KV1B_ATTEND_TENSOR runs the persistent tensor-core kernel where kv1b_attend would (G in {1, 2, 4},
- * equal sequence lengths) and its partial rows fit the array, otherwise the CUDA-core split-K
+ * KV1B_ATTEND_TENSOR runs the persistent tensor-core kernel where kv1b_attend would (equal sequence
+ * lengths) and its partial rows fit the array, otherwise the CUDA-core split-K
  * engine, which KV1B_ATTEND_CUDA_CORE always runs.  The partial rows and merge counters go to a
  * file-scope device array of KV1B_NOALLOC_SCRATCH_BYTES instead of a workspace; each call zeroes
  * the counters it uses with one small memset on `stream`.
@@ -291,7 +292,7 @@ int kv1b_merge_partials(const float* parts, int32_t nparts, int64_t rows, float*
  *                      units, s * log2(e) formed in its own fused order (not bit-exact with the fp32
  *                      logit); the call runs the whole attend and writes out like kv1b_attend.
  *                      ws: kv1b_attend_workspace_bytes(.., 0) bytes.  KV1B_ERR_UNSUPPORTED unless
- *                      that kernel would take the call (G in {1, 2, 4}, equal lengths, length > 0);
+ *                      that kernel would take the call (equal lengths, length > 0);
  *   KV1B_PROBE_TOPP:   the raw products 8 A and 8 Bc of the Top-p score pass and the fp32 logit it
  *                      selects with (bit-exact with the oracle's order).  ws: kv1b_attend_workspace_bytes
  *                      (.., 1) bytes; out unused.

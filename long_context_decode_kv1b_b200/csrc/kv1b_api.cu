@@ -96,8 +96,9 @@ int cuda_status(cudaError_t e) { return e == cudaSuccess ? KV1B_OK : KV1B_ERR_CU
 // Partial slots of the persistent kernel: segments x pieces x G x (6 + 128) floats; the piece
 // count per segment does not depend on the length, so the capacity-sized plan bounds every call.
 size_t ws_bytes_needed(const kv1b_cache_t* c, int32_t num_q_heads) {
-  const int G = num_q_heads / c->num_kv_heads;
-  if (!kv1b_ws_supported(G)) return 0;
+  const int Gq = num_q_heads / c->num_kv_heads;
+  if (!kv1b_ws_supported(Gq)) return 0;
+  const int G = kv1b_ws_template_group(Gq < 4 ? Gq : 4);  // head slots of one launch
   int64_t T, Lt;
   int ncta, pieces;
   kv1b_ws_plan(c->batch, c->num_kv_heads, G, c->capacity, num_sms(), &T, &Lt, &ncta, &pieces);
@@ -120,8 +121,8 @@ bool equal_lengths(const kv1b_cache_t* c) {
   return true;
 }
 
-// The persistent tensor-core kernel takes the call: G in {1, 2, 4}, one length for every sequence,
-// a non-empty cache.
+// The persistent tensor-core kernel takes the call: one length for every sequence, a non-empty cache
+// (G up to 8: launches of at most 4 query heads).
 bool ws_engine_applies(const kv1b_cache_t* c, int32_t num_q_heads) {
   return kv1b_ws_supported(num_q_heads / c->num_kv_heads) && equal_lengths(c) && max_length(c) > 0;
 }
@@ -129,7 +130,8 @@ bool ws_engine_applies(const kv1b_cache_t* c, int32_t num_q_heads) {
 // Parameters of the persistent kernel for this cache and workspace (KV1B_OK or KV1B_ERR_WORKSPACE).
 int ws_params(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale, float* out,
               void* ws, kv1b::AttendWsParams* w) {
-  const int G = num_q_heads / cache->num_kv_heads;
+  const int Gq = num_q_heads / cache->num_kv_heads;
+  const int G = kv1b_ws_template_group(Gq < 4 ? Gq : 4);  // head slots of one launch
   const int64_t maxlen = max_length(cache);
   memset(w, 0, sizeof(*w));
   w->c = view(cache);
@@ -181,7 +183,8 @@ int kv1b_attend_ws_buffers(const kv1b_cache_t* cache, const void* q, int32_t q_d
   const int hc = heads_check(cache, num_q_heads);
   if (hc != KV1B_OK) return hc;
   if (!ws_engine_applies(cache, num_q_heads)) return KV1B_ERR_UNSUPPORTED;
-  const int G = num_q_heads / cache->num_kv_heads;
+  const int Gq = num_q_heads / cache->num_kv_heads;
+  const int G = kv1b_ws_template_group(Gq < 4 ? Gq : 4);  // head slots of one launch
   kv1b::AttendWsParams w;
   memset(&w, 0, sizeof(w));
   w.c = view(cache);
@@ -204,7 +207,7 @@ int kv1b_attend_ws_buffers(const kv1b_cache_t* cache, const void* q, int32_t q_d
   w.counters = counters;
   w.wait_tries = kv1b::kWaitTriesDefault;
   w.stall_stage = -1;
-  return cuda_status(kv1b_launch_attend_ws(w, G, false, stream));
+  return cuda_status(kv1b_launch_attend_ws(w, Gq, false, stream));
 }
 
 extern "C" {

@@ -277,6 +277,10 @@ __device__ __forceinline__ void issue_stage(const AttendWsParams& p, int seg, in
 template <int G, bool PROBE>
 __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_constant__ AttendWsParams p) {
   static_assert(G == 1 || G == 2 || G == 4, "head t of lane (g, t) for t < G");
+  // this launch serves query heads head_base .. head_base + NH - 1 of each kv-head's G_all (NH <= G;
+  // lanes of absent heads carry no probability, so their weights and sums are zero)
+  const int NH = p.heads;
+  const int GA = p.G_all, HB = p.head_base;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kStages];
   __shared__ __align__(8) uint64_t empty_bar[kStages];  // all compute warps released the stage
@@ -423,13 +427,13 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
     const int b = seg / c.Hkv, kvh = seg - b * c.Hkv;
     const int64_t stride = static_cast<int64_t>(G) * kPartStride;  // between pieces
     const float* base = p.part + static_cast<int64_t>(seg) * p.max_pieces * G * kPartStride;
-    for (int i = threadIdx.x; i < G * n; i += kThreads) {
+    for (int i = threadIdx.x; i < NH * n; i += kThreads) {
       const int h = i / n, k = i - h * n;
       sm_m[h * 256 + k] = base[k * stride + h * kPartStride];
       sm_l[h * 256 + k] = base[k * stride + h * kPartStride + 1];
     }
     named_bar(1, kThreads);
-    if (warp < G) {
+    if (warp < NH) {
       float* mw = sm_m + warp * 256;
       const float* lw = sm_l + warp * 256;
       float M = -INFINITY;
@@ -451,7 +455,7 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
     }
     named_bar(1, kThreads);
     const int ch = threadIdx.x & 127;
-    for (int h = threadIdx.x >> 7; h < G; h += kThreads / 128) {
+    for (int h = threadIdx.x >> 7; h < NH; h += kThreads / 128) {
       const float* w = sm_m + h * 256;
       const float* o = base + h * kPartStride + 2 + ch;
       float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
@@ -463,7 +467,7 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
       for (; k < n; ++k) acc[0] = __fmaf_rn(w[k], o[k * stride], acc[0]);
       const float den = sm_d[h];
       const float num = __fadd_rn(__fadd_rn(acc[0], acc[1]), __fadd_rn(acc[2], acc[3]));
-      const int64_t orow = static_cast<int64_t>(b) * p.Hq + kvh * G + h;
+      const int64_t orow = static_cast<int64_t>(b) * p.Hq + kvh * GA + HB + h;
       if (p.partial_out) {  // the segment's log-sum-exp row (m, l, o[128]) for a later merge
         float* o = p.out + orow * kPartStride;
         if (ch == 0) {
@@ -494,21 +498,22 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
       for (int k = 0; k < 5; ++k) v[k] = __fadd_rn(v[k], __shfl_xor_sync(kFull, v[k], m));
     named_bar(1, kThreads);  // every quad is done with its weight buffer
     if (g == 0) {  // lane t: head t's m and l of this slice, group t's mid of every head
-      if (t < G) {
+      if (t < NH) {
         if (jw == 0) prow(qd, t)[0] = m_t == kNoMax ? -INFINITY : m_t;
         prow(qd, t)[kRowL + jw] = v[0];
       }
       #pragma unroll
-      for (int h = 0; h < G; ++h) prow(qd, h)[kRowMid + 4 * jw + t] = v[1 + h];
+      for (int h = 0; h < G; ++h)
+        if (h < NH) prow(qd, h)[kRowMid + 4 * jw + t] = v[1 + h];
     }
-    if (g < G) {  // head g: channels 32 jw + 8n + 2t + e
+    if (g < NH) {  // head g: channels 32 jw + 8n + 2t + e
       float* o = prow(qd, g) + kRowO + 32 * jw + 2 * t;
       #pragma unroll
       for (int n = 0; n < 4; ++n) *reinterpret_cast<float2*>(o + 8 * n) = make_float2(F[n][0], F[n][1]);
     }
     named_bar(1, kThreads);
     const int ch = threadIdx.x & 127;
-    for (int h = threadIdx.x >> 7; h < G; h += kThreads / 128) {
+    for (int h = threadIdx.x >> 7; h < NH; h += kThreads / 128) {
       float M = -INFINITY;
       #pragma unroll
       for (int q = 0; q < kQuads; ++q) M = fmaxf(M, prow(q, h)[0]);
@@ -566,7 +571,7 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
     const int par = seg & 1;
     const int b = seg / c.Hkv, kvh = seg - b * c.Hkv;
     const QueryPrep qp =
-        query_prep_warp(p.q, (static_cast<int64_t>(b) * p.Hq + kvh * G + h) * kD, p.q_dtype, c.signs);
+        query_prep_warp(p.q, (static_cast<int64_t>(b) * p.Hq + kvh * GA + HB + h) * kD, p.q_dtype, c.signs);
     if (lane == 0) {
       #pragma unroll
       for (int j = 0; j < 4; ++j)
@@ -580,11 +585,11 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
   // switch later skips the preparation (pre = true).
   auto prep = [&](int seg, bool pre, int next_seg) {
     const int par = seg & 1;
-    if (!pre && warp < G) prep_head(seg, warp);
-    if (next_seg >= 0 && warp >= 4 && warp < 4 + G) prep_head(next_seg, warp - 4);
+    if (!pre && warp < NH) prep_head(seg, warp);
+    if (next_seg >= 0 && warp >= 4 && warp < 4 + NH) prep_head(next_seg, warp - 4);
     named_bar(1, kThreads);  // reached by every compute warp at the same stage
     const int hb = g >> 1;
-    const bool code_col = (g & 1) == 0 && hb < G;
+    const bool code_col = (g & 1) == 0 && hb < NH;
     uint32_t pw[4] = {0u, 0u, 0u, 0u};
     if (code_col) {
       #pragma unroll
@@ -601,7 +606,7 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
         for (int j = 0; j < 4; ++j) code |= ((pw[j] >> r) & 0x01010101u) << j;
         bq[kb][hi] = code_col ? (code << sh) : ((g & 1) ? (0x01010101u << sh) : 0u);
       }
-    hv_t = t < G;
+    hv_t = t < NH;
     const int hs = hv_t ? t : 0;
     const float dl = hv_t ? s_dl[par][hs] : 0.0f, vl = hv_t ? s_vl[par][hs] : 0.0f;
     const float sq = hv_t ? static_cast<float>(s_sq[par][hs]) : 0.0f;
@@ -656,7 +661,7 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
           if constexpr (PROBE) {
             if (valid) {
               const int pb = cur_seg / c.Hkv, pkvh = cur_seg - pb * c.Hkv;
-              const int64_t o = (static_cast<int64_t>(pb) * p.Hq + pkvh * G + t) * c.cap + rel + tt;
+              const int64_t o = (static_cast<int64_t>(pb) * p.Hq + pkvh * GA + HB + t) * c.cap + rel + tt;
               p.probe_A[o] = d[2 * e];
               p.probe_Bc[o] = d[2 * e + 1];
               p.probe_s[o] = s2[kk][e];
@@ -843,7 +848,11 @@ static cudaError_t encode_codes_map(CUtensorMap* map, const uint32_t* v_codes, i
 
 using namespace kv1b;
 
-bool kv1b_ws_supported(int32_t G) { return G == 1 || G == 2 || G == 4; }
+// Any G up to KV1B_MAX_GROUP: launches of at most 4 query heads each (one for G <= 4), every one
+// streaming the whole cache -- the kernel is bound by its per-stage work, not by HBM, so a fused
+// 8-head form would not be faster than two 4-head launches.
+bool kv1b_ws_supported(int32_t G) { return G >= 1 && G <= KV1B_MAX_GROUP; }
+int kv1b_ws_template_group(int32_t G) { return G >= 3 ? 4 : G; }
 
 // CTAs = SMs (fewer when there are fewer tiles); T, Lt in 128-token tiles; partial rows per
 // segment = the most CTAs one segment can touch.
@@ -865,15 +874,27 @@ cudaError_t kv1b_launch_attend_ws(AttendWsParams& p, int32_t G, bool counters_cl
   const int64_t tiles = static_cast<int64_t>(p.c.B) * p.c.Hkv * (p.c.cap / ws::kTileTok);
   const cudaError_t e = ws::encode_codes_map(&p.codes_map, p.c.v_codes, tiles);
   if (e != cudaSuccess) return e;
-  if (p.wait_tries < 1) return cudaErrorInvalidValue;
+  if (p.wait_tries < 1 || G < 1 || G > KV1B_MAX_GROUP) return cudaErrorInvalidValue;
   if (probe && (!p.probe_A || !p.probe_Bc || !p.probe_s)) return cudaErrorInvalidValue;
-  switch (G * 2 + (probe ? 1 : 0)) {
-    case 2: return ws::launch_t<1, false>(p, counters_clean, stream);
-    case 4: return ws::launch_t<2, false>(p, counters_clean, stream);
-    case 8: return ws::launch_t<4, false>(p, counters_clean, stream);
-    case 3: return ws::launch_t<1, true>(p, counters_clean, stream);
-    case 5: return ws::launch_t<2, true>(p, counters_clean, stream);
-    case 9: return ws::launch_t<4, true>(p, counters_clean, stream);
-    default: return cudaErrorInvalidValue;
+  p.G_all = G;
+  // launches of up to 4 heads; the merge counters are zero after each (the first may clear them)
+  for (int base = 0; base < G; base += 4) {
+    const int nh = G - base < 4 ? G - base : 4;
+    const int tg = kv1b_ws_template_group(nh);
+    p.head_base = base;
+    p.heads = nh;
+    const bool clean = counters_clean || base > 0;
+    cudaError_t e2;
+    switch (tg * 2 + (probe ? 1 : 0)) {
+      case 2: e2 = ws::launch_t<1, false>(p, clean, stream); break;
+      case 4: e2 = ws::launch_t<2, false>(p, clean, stream); break;
+      case 8: e2 = ws::launch_t<4, false>(p, clean, stream); break;
+      case 3: e2 = ws::launch_t<1, true>(p, clean, stream); break;
+      case 5: e2 = ws::launch_t<2, true>(p, clean, stream); break;
+      case 9: e2 = ws::launch_t<4, true>(p, clean, stream); break;
+      default: e2 = cudaErrorInvalidValue;
+    }
+    if (e2 != cudaSuccess) return e2;
   }
+  return cudaSuccess;
 }

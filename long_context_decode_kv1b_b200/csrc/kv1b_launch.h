@@ -168,6 +168,9 @@ struct alignas(64) AttendWsParams {
   int32_t* status;     // cache status word (timeout flag)
   unsigned* counters;  // [B * Hkv] pieces of each segment written so far (zeroed before the launch)
   int32_t partial_out; // the merge writes log-sum-exp rows (m, l, o[128]) to out instead of o / l
+  int32_t G_all;       // query heads per kv-head of the call (set by the launcher)
+  int32_t head_base;   // first query head (within the kv-head's group) of this launch
+  int32_t heads;       // query heads this launch serves (<= the kernel's G)
   int32_t wait_tries;  // suspended tries (<= 0.5 ms each) before a pipeline wait gives up
   int32_t stall_stage; // test hook: each CTA's producer stops before this stage (-1: never)
   int32_t* probe_A;    // test hook (probe instantiation only): [B][Hq][cap] raw score products 8 A,
@@ -221,6 +224,7 @@ size_t kv1b_exact_workspace_bytes(int32_t rows, int32_t cap);
 void kv1b_exact_carve(kv1b::ExactParams* p, void* ws, int32_t rows);
 cudaError_t kv1b_launch_exact(const kv1b::ExactParams& p, int32_t rows, int32_t num_sms, cudaStream_t stream);
 bool kv1b_ws_supported(int32_t G);
+int kv1b_ws_template_group(int32_t G);  // query heads per launch slot of the persistent kernel for G (1, 2 or 4)
 int kv1b_attend_ws_buffers(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads,
                            float scale, float* out, float* part, size_t part_bytes, unsigned* counters,
                            cudaStream_t stream);

@@ -53,6 +53,9 @@ CONFIGS = {
     "c3": Config("c3", B=8, Hq=32, Hkv=8, L=32768, dtype=torch.bfloat16, seed=3, steps=16, token_scale=True),
     "c4": Config("c4", B=8, Hq=32, Hkv=8, L=32768, dtype=torch.bfloat16, seed=4, heavy=64, p=0.9),
     "c5": Config("c5", B=1, Hq=32, Hkv=8, L=1048576, dtype=torch.bfloat16, seed=5, steps=32, outliers=True),
+    # not one of the five parity configurations: the long context with 64 query heads per 8 kv heads
+    # (G = 8, a common grouping), for measurement only
+    "c5g8": Config("c5g8", B=1, Hq=64, Hkv=8, L=1048576, dtype=torch.bfloat16, seed=5, steps=32, outliers=True),
 }
 
 DESCRIPTIONS = {
@@ -61,6 +64,7 @@ DESCRIPTIONS = {
     "c3": "Llama-3-8B-shaped GQA decode: 32q/8kv, batch 8, context 32768, 16 append+attend steps, token scales",
     "c4": "Top-p p=0.9 on 32q/8kv, batch 8, context 32768, 64 heavy tokens per head",
     "c5": "long context: 32q/8kv, batch 1, context 1,048,576, 32 append+attend steps, outlier key channels",
+    "c5g8": "long context with G = 8: 64q/8kv, batch 1, context 1,048,576, 32 append+attend steps, outlier key channels",
 }
 
 

@@ -214,9 +214,11 @@ def test_query_prep_and_scores_bit_exact(dtype):
 
 
 # ------------------------------------------------------------------------------------- attend
-@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("G", [1, 2, 3, 4, 5, 6, 8])
 @pytest.mark.parametrize("engine", [kv.ATTEND_TENSOR, kv.ATTEND_CUDA_CORE])
 def test_attend_parity_group_sizes(G, engine):
+    # the persistent engine serves G > 4 as launches of at most 4 query heads (G = 3, 5, 6: a launch
+    # with absent head slots)
     B, Hkv = 2, 2
     cache, host = build_cache(B, Hkv, [700, 3], torch.bfloat16, seed=5, data_seed=G)
     g = torch.Generator(device=DEV).manual_seed(100 + G)
@@ -590,7 +592,7 @@ def probe_check(cache, host, q, scale, G, signs, kernel, where=""):
     return pr
 
 
-@pytest.mark.parametrize("G", [1, 2, 4])
+@pytest.mark.parametrize("G", [1, 2, 3, 4, 8])
 def test_attend_kernel_score_integers_bit_exact(G):
     # a tile-boundary length (4099 = 32 tiles + 3) and two sequences x two kv-heads
     B, Hkv = 2, 2
