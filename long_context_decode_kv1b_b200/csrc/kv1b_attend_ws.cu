@@ -273,13 +273,14 @@ __device__ __forceinline__ void issue_stage(const AttendWsParams& p, int seg, in
 }
 
 // PROBE: the test instantiation that also writes every score product and logit it forms
-// (p.probe_A / probe_Bc / probe_s); the product kernel is PROBE = false.
-template <int G, bool PROBE>
+// (p.probe_A / probe_Bc / probe_s); the product kernel is PROBE = false.  FULL: the launch fills all
+// G head slots (the head count is then a compile-time constant); otherwise p.heads < G of them.
+template <int G, bool PROBE, bool FULL>
 __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_constant__ AttendWsParams p) {
   static_assert(G == 1 || G == 2 || G == 4, "head t of lane (g, t) for t < G");
   // this launch serves query heads head_base .. head_base + NH - 1 of each kv-head's G_all (NH <= G;
   // lanes of absent heads carry no probability, so their weights and sums are zero)
-  const int NH = p.heads;
+  const int NH = FULL ? G : p.heads;
   const int GA = p.G_all, HB = p.head_base;
   extern __shared__ uint8_t smem_raw[];
   __shared__ __align__(8) uint64_t full_bar[kStages];
@@ -806,16 +807,17 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
   if (s_abort && lane == 0) atomicOr(p.status, KV1B_STATUS_TIMEOUT);
 }
 
-template <int G, bool PROBE>
+template <int G, bool PROBE, bool FULL = true>
 static cudaError_t launch_t(const AttendWsParams& p, bool counters_clean, cudaStream_t stream) {
   static std::atomic<unsigned long long> configured{0};  // bit per device
-  cudaError_t e = configure_smem(reinterpret_cast<const void*>(attend_ws_kernel<G, PROBE>), kSmemBytes, &configured);
+  cudaError_t e = configure_smem(reinterpret_cast<const void*>(attend_ws_kernel<G, PROBE, FULL>), kSmemBytes,
+                                 &configured);
   if (e != cudaSuccess) return e;
   if (!counters_clean) {
     e = cudaMemsetAsync(p.counters, 0, sizeof(unsigned) * p.c.B * p.c.Hkv, stream);
     if (e != cudaSuccess) return e;
   }
-  return launch_pdl(attend_ws_kernel<G, PROBE>, dim3(p.ncta), dim3(kBlock), kSmemBytes, stream, p);
+  return launch_pdl(attend_ws_kernel<G, PROBE, FULL>, dim3(p.ncta), dim3(kBlock), kSmemBytes, stream, p);
 }
 
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
@@ -885,13 +887,15 @@ cudaError_t kv1b_launch_attend_ws(AttendWsParams& p, int32_t G, bool counters_cl
     p.heads = nh;
     const bool clean = counters_clean || base > 0;
     cudaError_t e2;
-    switch (tg * 2 + (probe ? 1 : 0)) {
+    switch (tg * 2 + (probe ? 1 : 0) + (nh < tg ? 16 : 0)) {
       case 2: e2 = ws::launch_t<1, false>(p, clean, stream); break;
       case 4: e2 = ws::launch_t<2, false>(p, clean, stream); break;
       case 8: e2 = ws::launch_t<4, false>(p, clean, stream); break;
       case 3: e2 = ws::launch_t<1, true>(p, clean, stream); break;
       case 5: e2 = ws::launch_t<2, true>(p, clean, stream); break;
       case 9: e2 = ws::launch_t<4, true>(p, clean, stream); break;
+      case 24: e2 = ws::launch_t<4, false, false>(p, clean, stream); break;  // 3 heads in 4 slots
+      case 25: e2 = ws::launch_t<4, true, false>(p, clean, stream); break;
       default: e2 = cudaErrorInvalidValue;
     }
     if (e2 != cudaSuccess) return e2;
