@@ -37,6 +37,7 @@ constexpr int kResolveThreads = 1024;
 constexpr int kResolveSmemCand = 4096;   // candidates whose keys and masses the resolve keeps on chip
                                          // (64 KB: three resolve blocks per SM)
 constexpr size_t kResolveSmem = static_cast<size_t>(kResolveSmemCand) * 16;
+constexpr int kResolveSmallCand = 128;   // up to this many candidates: direct ranking, no radix passes
 
 __device__ __forceinline__ float topp_t(float s, float m) { return __fmul_rn(__fsub_rn(s, m), kL2e); }
 
@@ -518,6 +519,33 @@ __global__ void __launch_bounds__(kResolveThreads) topp_resolve_kernel(const Top
       smass[i] = topk ? 1ull : topp_mass_t(topp_t(st, m));
     }
   }
+  if (on_chip && n <= kResolveSmallCand) {  // block-uniform: few candidates (concentrated attention)
+    // thread i ranks candidate i: the mass of every candidate whose key is not larger (keys are
+    // unique); K* = the smallest key whose cumulative mass reaches rem -- the same key the radix
+    // passes below find
+    __syncthreads();  // keys and masses are in shared memory
+    const unsigned long long rem = rs.rem;
+    unsigned long long best = ~0ull;
+    if (threadIdx.x < n) {
+      const unsigned long long ki = skey[threadIdx.x];
+      unsigned long long cum = 0ull;
+      for (int j = 0; j < n; ++j) cum += skey[j] <= ki ? smass[j] : 0ull;
+      if (cum >= rem) best = ki;
+    }
+    #pragma unroll
+    for (int o = 16; o >= 1; o >>= 1) {
+      const unsigned long long x = __shfl_xor_sync(kFull, best, o);
+      best = x < best ? x : best;
+    }
+    if (lane == 0) s_diff[warp] = best;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      unsigned long long b0 = ~0ull;
+      for (int w = 0; w < kResolveThreads / 32; ++w) b0 = s_diff[w] < b0 ? s_diff[w] : b0;
+      s_prefix = b0;
+    }
+    __syncthreads();
+  } else {
   // leading key bytes shared by every candidate need no pass: start at the highest byte where any
   // candidate differs from the first (on-chip keys only; otherwise all 8 bytes)
   int d_top = 7;
@@ -599,6 +627,7 @@ __global__ void __launch_bounds__(kResolveThreads) topp_resolve_kernel(const Top
     }
     __syncthreads();
   }
+  }  // radix passes
   const unsigned long long kstar = s_prefix;
   if (threadIdx.x == 0) rs.kstar = kstar;
   // selected candidates join their sub-chunks' counts (one atomic per sub-chunk and warp)
