@@ -205,6 +205,9 @@ def build_cache(cfg, extra_tokens: int, device, keep_exact: bool = False):
         K, V = wl.prefill_chunk(cfg, start, n, device)
         torch.cuda.synchronize()  # the chunk's generation is not part of the encode's time
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        # a short device-side wait ahead of the first event: the host's call overhead then overlaps
+        # it and the events bracket the encode's device time alone
+        torch.cuda._sleep(HOST_SHADOW_CYCLES)
         e0.record(stream)
         cache.append(K, V)
         e1.record(stream)
@@ -215,6 +218,8 @@ def build_cache(cfg, extra_tokens: int, device, keep_exact: bool = False):
     torch.cuda.synchronize()
     return cache, Kx, Vx, [a.elapsed_time(b) for a, b in enc_ms]
 
+
+HOST_SHADOW_CYCLES = 200_000  # about 0.1 ms at the B200's clock
 
 CPU_SAMPLE_TOKENS = 1 << 15  # tokens of kv-head 0 / sequence 0 the oracle attends per call
 
@@ -519,7 +524,8 @@ def run_ours(args):
             "frac": enc_bytes / enc_s / 1e9 / peak, "unit": "GB/s",
             "bytes_rule": "2 x 128 x element size (K and V rows read) + 104 B written per token x kv-head",
             "kernel": "kv1b_encode_append over the prefill in chunks (each chunk generated and synchronized "
-                      "first), CUDA events around each call"}
+                      "first), CUDA events around each call with a 0.1 ms device wait queued ahead so that "
+                      "the host's call overhead is off the clock"}
         if alt:
             result["alt_engine"] = alt
         if topp:

@@ -258,7 +258,7 @@ __device__ __forceinline__ uint32_t half_scale_up_fast(float mx, float mn, int* 
   uint32_t e = __half_as_ushort(__float2half_rz(__fmul_rz(hi, 0x1.111112p-4f)));
   e = e > 0x7bfdu ? 0x7bfdu : e;
   const bool cm = e > 0u && covers(e - 1u), c0 = covers(e), c1 = covers(e + 1u), c2 = covers(e + 2u);
-  const bool normal = exact && hi > 0.0f && hi < 982560.0f && !cm && c2;
+  const bool normal = exact && hi >= 0.0f && hi < 982560.0f && !cm && c2;  // hi = 0: a constant group, scale 0
   uint32_t hb = c0 ? e : (c1 ? e + 1u : e + 2u);
   if (__any_sync(kFull, !normal)) {  // rare: saturation, an inexact fp64 range, or an estimate off by more
     const uint32_t slow = half_scale_up(mx, mn, sat);

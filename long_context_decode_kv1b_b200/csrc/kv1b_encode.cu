@@ -156,176 +156,244 @@ __global__ void __launch_bounds__(1024) encode_kernel(const EncodeParams p) {
 
 // ---------------------------------------------------------------------------------------------
 // Prefill form (appends of many tokens): one warp per 8-token group of one (sequence, kv-head) --
-// the tokens whose codes share one 32-bit word of every channel row -- encoding its tokens one after
-// another, the next token's rows in flight while the current one is encoded.
-//  - Key: lane l holds channels l + 32 r (r = 0..3).  The fixed tree sums take their two widest
-//    levels (h = 64, 32) inside the lane, the rotation its two widest stages (h = 32, 64), and sign
-//    word r is the warp's ballot of channel l + 32 r: bit i of word r = channel 32 r + i.  The
-//    cross-lane butterfly is one fused multiply-add, sgn * x + partner (sgn = -1 on the upper lane):
-//    a single rounding of a + c or a - c, the same value as the sum or difference.
-//  - Value: lane l holds channels 4 l .. 4 l + 3 (a 32-channel group on 8 lanes), as the decode form.
-//  - Codes: each lane keeps its 4 channels' code words of the group in registers and writes them once
-//    (nibbles of tokens outside the append are kept from the old word).
+// the tokens whose codes share one 32-bit word of every channel row -- with 4 lanes per token
+// (lane = 4 tau + j: token tau of the group, part j) and all 8 tokens at once.
+//  - Key: lane j holds channels j + 4 r (r = 0..31).  The fixed tree sums take levels h = 64 .. 4
+//    inside the lane (pairs r, r + h / 4) and h = 2, 1 across the token's lanes; the rotation takes
+//    stages h = 1, 2 across them (one fused multiply-add, sgn * x + partner: a single rounding of
+//    a + c or a - c) and h = 4 .. 64 inside (pairs r, r + h / 4), in the order h = 1, 2, 4, ..., 64.
+//    Sign word w of a token: bit i is channel 32 w + i, i.e. lane i & 3 at r = 8 w + (i >> 2) -- one
+//    ballot per r gives every token's bits, and lane j assembles word j of its token.
+//  - Value: lane j holds value group j (channels 32 j .. 32 j + 31): min / max and the binary16
+//    searches inside the lane; codes from one correctly rounded reciprocal per group and Markstein's
+//    correction, packed 8 per word token-major, then an 8 x 8 transpose of nibbles across the group's
+//    8 token lanes turns them into the channel-major code words (nibble tau = token tau).
 // Every stored bit, code and scalar equals the decode form's (the same operations in the same order).
 constexpr int kPrefillWarps = 4;
 constexpr int kPrefillMinTokens = 64;  // appends of at least this many tokens per sequence take the prefill form
-constexpr int kPrefillGroup = 8;  // tokens per code word
+constexpr int kPrefillGroup = 8;       // tokens per code word
 
-// Fixed pairwise tree over the 128 channels in the strided layout (lane l: channels l + 32 r):
-// h = 64 and 32 inside the lane, then h = 16 .. 1 across lanes.  Returns a[0] on every lane.
-__device__ __forceinline__ float tree_sum128_strided(const float a[4]) {
-  float x = __fadd_rn(__fadd_rn(a[0], a[2]), __fadd_rn(a[1], a[3]));  // h = 64 (r, r + 2), then h = 32
-  #pragma unroll
-  for (int off = 16; off >= 1; off >>= 1) x = __fadd_rn(x, __shfl_down_sync(kFull, x, off));
-  return __shfl_sync(kFull, x, 0);
-}
-
-// One round y <- H (D (.) y) in the strided layout: stages h = 1 .. 16 across lanes, 32 and 64 inside.
-__device__ __forceinline__ void rotate128_strided(float x[4], const float sg[4]) {
+// 32-bit mask of the rotation signs of lane j's key channels j + 4 r (bit r set: D = -1) for round rd:
+// four coalesced loads, one ballot each (bit l of ballot i = channel 32 i + l), then the stride-4
+// bits j, j + 4, .., j + 28 of each ballot packed into byte i.
+__device__ __forceinline__ uint32_t sign_mask(const float* signs, int rd, int j) {
   const int lane = threadIdx.x & 31;
+  uint32_t m = 0u;
   #pragma unroll
-  for (int r = 0; r < 4; ++r) x[r] = (sg[r] < 0.0f) ? -x[r] : x[r];
-  #pragma unroll
-  for (int h = 1; h < 32; h <<= 1) {
-    const float sgn = (lane & h) ? -1.0f : 1.0f;
-    #pragma unroll
-    for (int r = 0; r < 4; ++r) x[r] = __fmaf_rn(sgn, x[r], __shfl_xor_sync(kFull, x[r], h));
+  for (int i = 0; i < 4; ++i) {
+    uint32_t x = (__ballot_sync(kFull, __ldg(signs + rd * kD + 32 * i + lane) < 0.0f) >> j) & 0x11111111u;
+    x = (x | (x >> 3)) & 0x03030303u;
+    x = (x | (x >> 6)) & 0x000F000Fu;
+    x = (x | (x >> 12)) & 0x000000FFu;
+    m |= x << (8 * i);
   }
-  const float a0 = __fadd_rn(x[0], x[1]), a1 = __fsub_rn(x[0], x[1]);  // h = 32: (r, r + 1)
-  const float a2 = __fadd_rn(x[2], x[3]), a3 = __fsub_rn(x[2], x[3]);
-  x[0] = __fadd_rn(a0, a2);  // h = 64: (r, r + 2)
-  x[2] = __fsub_rn(a0, a2);
-  x[1] = __fadd_rn(a1, a3);
-  x[3] = __fsub_rn(a1, a3);
+  return m;
 }
 
-// Channels l + 32 r (r = 0..3) of an fp32 / bf16 / fp16 row as fp32.
-__device__ __forceinline__ void load_strided(const void* base, int64_t off, int dtype, float x[4]) {
-  const int lane = threadIdx.x & 31;
+// One round y <- H (D (.) y): stages h = 1, 2 across the token's 4 lanes, h = 4 .. 64 inside.
+__device__ __forceinline__ void rotate_q4(float x[32], uint32_t smask, int j) {
   #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int64_t o = off + lane + 32 * r;
-    if (dtype == KV1B_DTYPE_F32) {
-      x[r] = __ldg(static_cast<const float*>(base) + o);
-    } else {
-      const uint32_t h = __ldg(static_cast<const unsigned short*>(base) + o);
-      x[r] = dtype == KV1B_DTYPE_BF16 ? __uint_as_float(h << 16)
-                                      : __half2float(__ushort_as_half(static_cast<unsigned short>(h)));
+  for (int r = 0; r < 32; ++r)  // D: flip the sign bit where the mask has a 1
+    x[r] = __int_as_float(__float_as_int(x[r]) ^ static_cast<int>((smask << (31 - r)) & 0x80000000u));
+  #pragma unroll
+  for (int h = 1; h <= 2; h <<= 1) {
+    const float sgn = (j & h) ? -1.0f : 1.0f;  // the lane of the pair's upper element forms a - c
+    #pragma unroll
+    for (int r = 0; r < 32; ++r) x[r] = __fmaf_rn(sgn, x[r], __shfl_xor_sync(kFull, x[r], h));
+  }
+  #pragma unroll
+  for (int hr = 1; hr <= 16; hr <<= 1) {
+    #pragma unroll
+    for (int r = 0; r < 32; ++r) {
+      if (r & hr) continue;
+      const float a = x[r], c = x[r + hr];
+      x[r] = __fadd_rn(a, c);
+      x[r + hr] = __fsub_rn(a, c);
     }
   }
 }
 
-__global__ void __launch_bounds__(32 * kPrefillWarps) encode_prefill_kernel(const EncodeParams p) {
+// Fixed pairwise tree over the token's 128 channels (lane j: channels j + 4 r); h = 64 .. 4 inside
+// the lane, 2 and 1 across lanes.  Returns the sum on each of the token's lanes.  a is overwritten.
+__device__ __forceinline__ float tree_sum_q4(float a[32]) {
+  #pragma unroll
+  for (int hr = 16; hr >= 1; hr >>= 1)
+    #pragma unroll
+    for (int r = 0; r < hr; ++r) a[r] = __fadd_rn(a[r], a[r + hr]);
+  float x = a[0];
+  x = __fadd_rn(x, __shfl_xor_sync(kFull, x, 2));  // h = 2: lanes j < 2 add lane j + 2
+  x = __fadd_rn(x, __shfl_xor_sync(kFull, x, 1));  // h = 1: lane 0 adds lane 1
+  return __shfl_sync(kFull, x, (threadIdx.x & 31) & ~3);
+}
+
+// Element types of the K / V rows (the kernel is compiled once per type).
+template <int DT> struct Elem;
+template <> struct Elem<KV1B_DTYPE_F32> {
+  typedef float T;
+  static __device__ __forceinline__ float get(float x) { return x; }
+};
+template <> struct Elem<KV1B_DTYPE_BF16> {
+  typedef unsigned short T;
+  static __device__ __forceinline__ float get(unsigned short x) { return __uint_as_float(static_cast<uint32_t>(x) << 16); }
+};
+template <> struct Elem<KV1B_DTYPE_F16> {
+  typedef unsigned short T;
+  static __device__ __forceinline__ float get(unsigned short x) { return __half2float(__ushort_as_half(x)); }
+};
+
+// sum over i = 0..7 of (0x4B000000 << 4 i) modulo 2^32: the exponent bits of 2^23 + code, shifted
+// into each nibble's place (only i = 0, 1 keep any bits)
+constexpr uint32_t kMagicPacked = 0x4B000000u + (0x4B000000u << 4);
+constexpr int kPrefillMaxGroupsPerWarp = 4;  // 8-token groups a warp encodes one after another, at most
+
+template <int DT>
+__global__ void __launch_bounds__(32 * kPrefillWarps, 4) encode_prefill_kernel(const EncodeParams p) {
+  typedef typename Elem<DT>::T T;
   pdl_wait();
   const int b = blockIdx.z, h = blockIdx.y;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int tau = lane >> 2, j = lane & 3;
   if (blockIdx.x == 0 && blockIdx.y == 0 && blockIdx.z == 0 && threadIdx.x < p.B)
     p.lengths[threadIdx.x] = static_cast<int32_t>(p.L0[threadIdx.x] + p.n_new);
   const int64_t L0 = p.L0[b], L1 = L0 + p.n_new;
-  const int64_t g0 = ((L0 >> 3) + static_cast<int64_t>(blockIdx.x) * kPrefillWarps + warp) * kPrefillGroup;
-  if (g0 >= L1) return;  // warp-uniform
-  const int64_t t_lo = g0 > L0 ? g0 : L0, t_hi = g0 + kPrefillGroup < L1 ? g0 + kPrefillGroup : L1;
-  const int64_t tok0 = (static_cast<int64_t>(b) * p.Hkv + h) * p.cap + t_lo;  // first token's index in the planes
-  // rotation signs of the lane's key channels, round 0; later rounds (rare) are read per token
-  float sg[4];
-  #pragma unroll
-  for (int r = 0; r < 4; ++r) sg[r] = p.signs[lane + 32 * r];
+  const int gpw = p.groups_per_warp;
+  const int64_t gw = ((L0 >> 3) + (static_cast<int64_t>(blockIdx.x) * kPrefillWarps + warp) * gpw) *
+                     kPrefillGroup;  // the warp's first group
+  if (gw >= L1) return;  // warp-uniform
+  // rotation: round 0's sign mask of this lane's key channels (the rounds and their masks are the
+  // same for every token)
   const bool rotate = p.signs[0] != 0.0f;
   const int rounds = !rotate ? 0 : (p.signs[kD] == 0.0f ? 1 : (p.signs[2 * kD] == 0.0f ? 2 : 3));
-  uint32_t cw[4] = {0u, 0u, 0u, 0u};  // code words of channels 4 lane + j for this group
+  const uint32_t smask0 = sign_mask(p.signs, 0, j);
+  const int64_t seg = static_cast<int64_t>(b) * p.Hkv + h;
   int flags = 0;
-  const int n = static_cast<int>(t_hi - t_lo);
-  int64_t row = static_cast<int64_t>(b) * p.sb + (t_lo - L0) * p.st + static_cast<int64_t>(h) * p.sh;
-  uint32_t* kbits = p.k_bits + tok0 * 4;
-  float* knorm = p.k_norm + tok0;
-  float* kcinv = p.k_cinv + tok0;
-  uint32_t* vsm = p.v_sm + tok0 * 4 + (lane >> 3);
-  float kx[4], vx[4];
-  load_strided(p.k, row, p.dtype, kx);
-  load4(p.v, row + 4 * lane, p.dtype, vx);
   #pragma unroll 1
-  for (int i = 0; i < n; ++i) {
-    float x[4], v[4];
-    #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      x[r] = kx[r];
-      v[r] = vx[r];
-    }
-    row += p.st;
-    if (i + 1 < n) {  // the next token's rows in flight
-      load_strided(p.k, row, p.dtype, kx);
-      load4(p.v, row + 4 * lane, p.dtype, vx);
-    }
+  for (int gi = 0; gi < gpw; ++gi) {
+    const int64_t g0 = gw + gi * kPrefillGroup;
+    if (g0 >= L1) break;  // warp-uniform
+    const int64_t pos = g0 + tau;
+    const bool full = g0 >= L0 && g0 + kPrefillGroup <= L1;  // warp-uniform: every token of the group is new
+    const bool on = pos >= L0 && pos < L1;                   // this token is appended now (its 4 lanes agree)
+    const int64_t rowk = static_cast<int64_t>(b) * p.sb + (pos - L0) * p.st + static_cast<int64_t>(h) * p.sh;
+    const T* krow = static_cast<const T*>(p.k) + rowk + j;       // channels j + 4 r at krow[4 r]
+    const int64_t tok = seg * p.cap + pos;                       // the token's index in the planes
+
     // ---- key sketch: N, rotation, sign words, 1/C
-    float sq[4], ab[4];
-    #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      sq[r] = __fmul_rn(x[r], x[r]);
-      flags |= isfinite(x[r]) ? 0 : KV1B_STATUS_NONFINITE;
-    }
-    const float nrm = __fsqrt_rn(tree_sum128_strided(sq));
-    if (rotate) {
-      rotate128_strided(x, sg);
-      #pragma unroll 1
-      for (int rd = 1; rd < rounds; ++rd) {
-        float s2[4];
+    {
+      float x[32], a[32];
+      if (full) {
         #pragma unroll
-        for (int r = 0; r < 4; ++r) s2[r] = p.signs[rd * kD + lane + 32 * r];
-        rotate128_strided(x, s2);
+        for (int r = 0; r < 32; ++r) x[r] = Elem<DT>::get(__ldg(krow + 4 * r));
+      } else {
+        #pragma unroll
+        for (int r = 0; r < 32; ++r) x[r] = on ? Elem<DT>::get(__ldg(krow + 4 * r)) : 0.0f;
+      }
+      bool fin = true;
+      #pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        fin &= isfinite(x[r]);
+        a[r] = __fmul_rn(x[r], x[r]);
+      }
+      flags |= fin ? 0 : KV1B_STATUS_NONFINITE;
+      const float nrm = __fsqrt_rn(tree_sum_q4(a));
+      if (rotate) {  // a zero first sign: no rotation (as the decode form)
+        rotate_q4(x, smask0, j);
+        #pragma unroll 1
+        for (int rd = 1; rd < rounds; ++rd) rotate_q4(x, sign_mask(p.signs, rd, j), j);
+      }
+      uint32_t word = 0u;  // sign word j of this lane's token
+      #pragma unroll
+      for (int r = 0; r < 32; ++r) {
+        const uint32_t bal = __ballot_sync(kFull, x[r] >= 0.0f);  // bit 4 tau' + j' = channel j' + 4 r of token tau'
+        if ((r >> 3) == j) word |= ((bal >> (4 * tau)) & 0xFu) << (4 * (r & 7));
+        a[r] = fabsf(x[r]);
+      }
+      const float sabs = tree_sum_q4(a);
+      const float cinv = (sabs > 0.0f) ? __fdiv_rn(__fmul_rn(static_cast<float>(kD), nrm), sabs) : 1.0f;
+      if (on) {
+        p.k_bits[tok * 4 + j] = word;
+        if (j == 0) {
+          p.k_norm[tok] = nrm;
+          p.k_cinv[tok] = cinv;
+        }
       }
     }
-    uint32_t word[4];
+
+    // ---- value codes: group j
+    float v[32];
+    if (full) {
+      #pragma unroll
+      for (int q = 0; q < 8; ++q) load4(p.v, rowk + 32 * j + 4 * q, DT, v + 4 * q);
+    } else {
+      #pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (on) {
+          load4(p.v, rowk + 32 * j + 4 * q, DT, v + 4 * q);
+        } else {
+          v[4 * q] = v[4 * q + 1] = v[4 * q + 2] = v[4 * q + 3] = 0.0f;
+        }
+      }
+    }
+    float mn = v[0], mx = v[0];
+    bool fin = true;
     #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      word[r] = __ballot_sync(kFull, x[r] >= 0.0f);
-      ab[r] = fabsf(x[r]);
+    for (int i = 0; i < 32; ++i) {
+      fin &= isfinite(v[i]);
+      mn = fminf(mn, v[i]);
+      mx = fmaxf(mx, v[i]);
     }
-    const float sabs = tree_sum128_strided(ab);
-    const float cinv = (sabs > 0.0f) ? __fdiv_rn(__fmul_rn(static_cast<float>(kD), nrm), sabs) : 1.0f;
-    if (lane < 4) kbits[lane] = lane == 0 ? word[0] : (lane == 1 ? word[1] : (lane == 2 ? word[2] : word[3]));
-    if (lane == 0) {
-      *knorm = nrm;
-      *kcinv = cinv;
-    }
-    kbits += 4;
-    ++knorm;
-    ++kcinv;
-    // ---- value codes: group lane >> 3
-    float mn = fminf(fminf(v[0], v[1]), fminf(v[2], v[3]));
-    float mx = fmaxf(fmaxf(v[0], v[1]), fmaxf(v[2], v[3]));
-    #pragma unroll
-    for (int m = 1; m <= 4; m <<= 1) {  // reduce over the 8 lanes of this 32-channel group
-      mn = fminf(mn, __shfl_xor_sync(kFull, mn, m));
-      mx = fmaxf(mx, __shfl_xor_sync(kFull, mx, m));
-    }
+    flags |= fin ? 0 : KV1B_STATUS_NONFINITE;
     int sat = 0;
-    #pragma unroll
-    for (int r = 0; r < 4; ++r) flags |= isfinite(v[r]) ? 0 : KV1B_STATUS_NONFINITE;
     const uint32_t min_bits = half_round_down(mn, &sat);
     const float mf = __half2float(__ushort_as_half(static_cast<unsigned short>(min_bits)));
     const uint32_t scale_bits = half_scale_up_fast(mx, mf, &sat);
-    flags |= sat ? KV1B_STATUS_FP16_SATURATED : 0;
+    flags |= (sat && on) ? KV1B_STATUS_FP16_SATURATED : 0;
     const float sf = __half2float(__ushort_as_half(static_cast<unsigned short>(scale_bits)));
     const float rs = __frcp_rn(sf);  // correctly rounded; +inf for a zero scale (codes 0 below)
-    const uint32_t nsh = 4u * static_cast<uint32_t>((t_lo + i) & 7);
+    uint32_t cw[4];  // token-major: nibble i of word k = channel 32 j + 8 k + i of this token
     #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-      // code = clamp(floor(fl(fl(v - min) / scale) + 0.5), 0, 15), 0 for a zero scale
-      const float fl = floorf(__fadd_rn(div_markstein(__fsub_rn(v[r], mf), sf, rs), 0.5f));
-      const float cl = sf > 0.0f ? fminf(fmaxf(fl, 0.0f), 15.0f) : 0.0f;  // NaN -> 0
-      cw[r] |= (__float_as_uint(__fadd_rn(cl, 8388608.0f)) & 0xFu) << nsh;  // the integer in the mantissa
+    for (int k = 0; k < 4; ++k) {
+      // code = clamp(floor(y), 0, 15) with y = fl(fl(v - min) / scale) + 0.5, 0 for a zero scale.
+      // floor(clamp(y, 0, 15.5)) is the same integer (NaN -> 0), and adding 2^23 rounded toward
+      // -inf leaves it exactly in the low mantissa bits: the float's bits are 0x4B000000 + code.
+      // Shifted by 4 i and summed modulo 2^32, the eight words give the packed codes plus the
+      // shifted constants, which one subtraction removes.
+      uint32_t w = 0u - kMagicPacked;
+      #pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const float y = __fadd_rn(div_markstein(__fsub_rn(v[8 * k + i], mf), sf, rs), 0.5f);
+        const float c = fminf(fmaxf(y, 0.0f), 15.5f);
+        w += __float_as_uint(__fadd_rd(c, 8388608.0f)) << (4 * i);
+      }
+      cw[k] = (on && sf > 0.0f) ? w : 0u;  // sf NaN or 0: codes 0
     }
-    if ((lane & 7) == 0) *vsm = scale_bits | (min_bits << 16);
-    vsm += 4;
+    if (on) p.v_sm[tok * 4 + j] = scale_bits | (min_bits << 16);
+    // transpose the 8 x 8 nibbles of each word across the 8 token lanes of group j: afterwards
+    // nibble tau' of lane tau's word k is the code of channel 32 j + 8 k + tau of token tau'
+    #pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      uint32_t x = cw[k];
+      uint32_t y = __shfl_xor_sync(kFull, x, 16);  // token tau ^ 4
+      x = (tau & 4) ? ((x & 0xFFFF0000u) | (y >> 16)) : ((x & 0x0000FFFFu) | (y << 16));
+      y = __shfl_xor_sync(kFull, x, 8);            // token tau ^ 2
+      x = (tau & 2) ? ((x & 0xFF00FF00u) | ((y >> 8) & 0x00FF00FFu)) : ((x & 0x00FF00FFu) | ((y & 0x00FF00FFu) << 8));
+      y = __shfl_xor_sync(kFull, x, 4);            // token tau ^ 1
+      x = (tau & 1) ? ((x & 0xF0F0F0F0u) | ((y >> 4) & 0x0F0F0F0Fu)) : ((x & 0x0F0F0F0Fu) | ((y & 0x0F0F0F0Fu) << 4));
+      cw[k] = x;
+    }
+    // ---- code words: word (g0 & 127) / 8 of channel rows 32 j + 8 k + tau in the group's 128-token
+    // tile; nibbles of tokens outside the append keep the old word's
+    uint32_t* dst = p.v_codes + ((seg * (p.cap / 128) + (g0 >> 7)) * kD + 32 * j + tau) * 16 + ((g0 & 127) >> 3);
+    if (full) {
+      #pragma unroll
+      for (int k = 0; k < 4; ++k) dst[8 * 16 * k] = cw[k];
+    } else {
+      const int n0 = static_cast<int>((g0 > L0 ? g0 : L0) - g0), n1 = static_cast<int>((g0 + 8 < L1 ? g0 + 8 : L1) - g0);
+      const uint32_t keep = ~(((n1 == 8 ? 0u : (~0u << (4 * n1))) ^ ~0u) & (~0u << (4 * n0)));
+      #pragma unroll
+      for (int k = 0; k < 4; ++k) dst[8 * 16 * k] = (dst[8 * 16 * k] & keep) | cw[k];
+    }
   }
-  // ---- code words: word (g0 & 127) / 8 of channel rows 4 lane + j in the group's 128-token tile;
-  // nibbles of tokens outside [t_lo, t_hi) keep the old word's
-  const int64_t seg = static_cast<int64_t>(b) * p.Hkv + h;
-  uint32_t* dst = p.v_codes + ((seg * (p.cap / 128) + (g0 >> 7)) * kD + 4 * lane) * 16 + ((g0 & 127) >> 3);
-  const int n0 = static_cast<int>(t_lo - g0), n1 = static_cast<int>(t_hi - g0);
-  const uint32_t keep = (n0 == 0 && n1 == kPrefillGroup) ? 0u : ~(((n1 == 8 ? 0u : (~0u << (4 * n1))) ^ ~0u) & (~0u << (4 * n0)));
-  #pragma unroll
-  for (int j = 0; j < 4; ++j) dst[16 * j] = keep ? ((dst[16 * j] & keep) | cw[j]) : cw[j];
   flags = static_cast<int>(__reduce_or_sync(kFull, static_cast<unsigned>(flags)));
   if (lane == 0 && flags) atomicOr(p.status, flags);
 }
@@ -348,8 +416,20 @@ cudaError_t kv1b_launch_encode(const EncodeParams& p, int64_t max_tiles, cudaStr
       const int64_t g = ((p.L0[b] + p.n_new - 1) >> 3) - (p.L0[b] >> 3) + 1;
       groups = g > groups ? g : groups;
     }
-    const dim3 grid(static_cast<unsigned>((groups + kPrefillWarps - 1) / kPrefillWarps), p.Hkv, p.B);
-    return launch_pdl(encode_prefill_kernel, grid, dim3(32 * kPrefillWarps), 0, stream, p);
+    // several groups per warp amortise the warp's set-up (sign masks, row bases) once there are
+    // about two waves of warps at 16 resident per SM without it
+    const int64_t warps = groups * p.Hkv * p.B;
+    const int64_t wave2 = 2LL * 148 * 16;
+    EncodeParams q = p;
+    q.groups_per_warp = static_cast<int32_t>(warps >= kPrefillMaxGroupsPerWarp * wave2 ? kPrefillMaxGroupsPerWarp
+                                             : (warps >= 2 * wave2 ? 2 : 1));
+    const int64_t per_block = static_cast<int64_t>(kPrefillWarps) * q.groups_per_warp;
+    const dim3 grid(static_cast<unsigned>((groups + per_block - 1) / per_block), p.Hkv, p.B);
+    switch (p.dtype) {
+      case KV1B_DTYPE_F32: return launch_pdl(encode_prefill_kernel<KV1B_DTYPE_F32>, grid, dim3(32 * kPrefillWarps), 0, stream, q);
+      case KV1B_DTYPE_BF16: return launch_pdl(encode_prefill_kernel<KV1B_DTYPE_BF16>, grid, dim3(32 * kPrefillWarps), 0, stream, q);
+      default: return launch_pdl(encode_prefill_kernel<KV1B_DTYPE_F16>, grid, dim3(32 * kPrefillWarps), 0, stream, q);
+    }
   }
   const dim3 grid(static_cast<unsigned>(max_tiles), p.Hkv, p.B);
   return launch_pdl(encode_kernel, grid, dim3(1024), 0, stream, p);

@@ -16,6 +16,7 @@ struct EncodeParams {
   int32_t n_new;
   int64_t sb, st, sh;  // element strides of K/V: sequence, token, kv-head
   int32_t B, Hkv, cap;
+  int32_t groups_per_warp;  // prefill form: 8-token groups a warp encodes in turn (set by the launcher)
   uint32_t* k_bits;
   float* k_norm;
   float* k_cinv;
