@@ -375,6 +375,34 @@ def test_topp_group_sizes(G, qdt):
         topp_check(cache, host, q, 0.4, p, G, oracle.signs(13))
 
 
+@pytest.mark.parametrize("G", [4, 8])
+def test_topp_flat_and_peaked_sequences(G):
+    # one call over two very different selections: sequence 0 has flat attention (a large share of
+    # the tokens is needed to reach p), sequence 1 a few planted tokens that carry the mass
+    B, Hkv, L = 2, 2, 6000
+    cap = (L + 127) // 128 * 128
+    cache = kv.Cache(B, Hkv, cap, seed=17)
+    host = HostKV(B, Hkv, cap)
+    g = torch.Generator(device=DEV).manual_seed(31)
+    K = torch.randn((B, L, Hkv, 128), generator=g, device=DEV)
+    V = torch.randn((B, L, Hkv, 128), generator=g, device=DEV)
+    dirs = torch.nn.functional.normalize(torch.randn((Hkv, 128), generator=g, device=DEV), dim=-1)
+    heavy = torch.randperm(L, generator=g, device=DEV)[:12]
+    for h in range(Hkv):
+        K[1, heavy, h, :] = 6.0 * math.sqrt(128.0) * dirs[h] + 0.1 * torch.randn((12, 128), generator=g, device=DEV)
+    K, V = K.to(torch.bfloat16), V.to(torch.bfloat16)
+    cache.append(K, V)
+    host.add(K, V)
+    q = torch.randn((B, Hkv * G, 128), generator=g, device=DEV)
+    for h in range(Hkv):
+        q[1, h * G:(h + 1) * G] = 4.0 * dirs[h] + 0.3 * torch.randn((G, 128), generator=g, device=DEV)
+    for p in (0.6, 0.9):
+        cnt = topp_check(cache, host, q, 0.05, p, G, oracle.signs(17))  # sequence 0: logits of std ~0.6
+        assert int(cnt[0].min().item()) > L // 10, f"p {p}: flat rows select {cnt[0].tolist()}"
+        assert int(cnt[1].max().item()) <= 12, f"p {p}: peaked rows select {cnt[1].tolist()}"
+    assert cache.status() == 0
+
+
 # ------------------------------------------------------------------ exact attention over a selected set
 def cache_with_exact(B, Hkv, L, dtype, seed, data_seed):
     """A compressed cache plus the exact keys / values it was built from ([B, L, Hkv, 128] on the GPU)."""
