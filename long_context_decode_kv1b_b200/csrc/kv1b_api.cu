@@ -341,7 +341,7 @@ int kv1b_attend(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32
   p.out = out;
   p.partial_out = partial ? 1 : 0;
   for (int b = 0; b < cache->batch; ++b) p.len[b] = static_cast<int32_t>(cache->h_lengths[b]);
-  return cuda_status(kv1b_launch_attend(p, G, flags, static_cast<int32_t>(maxlen), static_cast<cudaStream_t>(stream)));
+  return cuda_status(kv1b_launch_attend(p, G, static_cast<cudaStream_t>(stream)));
 }
 
 int kv1b_attend_select(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads, float scale,

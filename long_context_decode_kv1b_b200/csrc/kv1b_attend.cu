@@ -363,10 +363,7 @@ int kv1b_pick_splits(int32_t B, int32_t Hkv, int64_t max_len, int num_sms) {
   return static_cast<int>(ns);
 }
 
-cudaError_t kv1b_launch_attend(const AttendParams& p, int32_t G, int32_t engine, int32_t max_len,
-                               cudaStream_t stream) {
-  (void)max_len;
-  (void)engine;
+cudaError_t kv1b_launch_attend(const AttendParams& p, int32_t G, cudaStream_t stream) {
   cudaError_t e = cudaSuccess;
 #define KV1B_CASE(GG)                      \
   case GG:                                 \

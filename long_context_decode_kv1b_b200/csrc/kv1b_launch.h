@@ -204,8 +204,8 @@ inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, siz
 }
 
 cudaError_t kv1b_launch_encode(const kv1b::EncodeParams& p, int64_t max_tiles, cudaStream_t stream);
-cudaError_t kv1b_launch_attend(const kv1b::AttendParams& p, int32_t G, int32_t engine, int32_t max_len,
-                               cudaStream_t stream);
+// The CUDA-core split-K engine (split kernel + merge); the tensor-core engine is kv1b_launch_attend_ws.
+cudaError_t kv1b_launch_attend(const kv1b::AttendParams& p, int32_t G, cudaStream_t stream);
 cudaError_t kv1b_launch_query_prep(const kv1b::CacheView& c, const void* q, int32_t q_dtype, int32_t Hq,
                                    uint32_t* planes, float* vl, float* delta, int32_t* sq, cudaStream_t stream);
 cudaError_t kv1b_launch_scores(const kv1b::ScoresParams& p, int32_t G, int32_t max_len, cudaStream_t stream);

@@ -152,6 +152,6 @@ extern "C" int kv1b_attend_noalloc(const kv1b_cache_t* cache, const void* q, int
   p.part = static_cast<float*>(scratch);
   p.out = out;
   for (int b = 0; b < cache->batch; ++b) p.len[b] = static_cast<int32_t>(cache->h_lengths[b]);
-  const cudaError_t e = kv1b_launch_attend(p, G, KV1B_ATTEND_CUDA_CORE, static_cast<int32_t>(maxlen), st);
+  const cudaError_t e = kv1b_launch_attend(p, G, st);
   return e == cudaSuccess ? KV1B_OK : KV1B_ERR_CUDA;
 }
