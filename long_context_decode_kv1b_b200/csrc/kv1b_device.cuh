@@ -20,6 +20,9 @@ namespace kv1b {
 // be scheduled while its predecessor in the stream is still running; griddepcontrol.wait returns once
 // every prerequisite grid has completed and its memory is visible (a no-op for a plain launch).
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+// Let the next kernel in the stream be scheduled now (its CTAs take free SM slots and run up to
+// their own griddepcontrol.wait, which still waits for this whole grid to complete).
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" :::); }
 
 constexpr int kD = 128;
 constexpr unsigned kFull = 0xffffffffu;

@@ -43,6 +43,7 @@ __global__ void __launch_bounds__(1024) encode_kernel(const EncodeParams p) {
   __shared__ uint8_t codes[16][kD];
   __shared__ int s_new[16];
   pdl_wait();  // every block, before any memory access: the inputs may come from the previous kernel
+  pdl_launch_dependents();  // the attend that usually follows sets up on the SMs this grid leaves free
   const int b = blockIdx.z, h = blockIdx.y;
   const int64_t L0 = p.L0[b];
   const int64_t first_tile = L0 / 16, last_tile = (L0 + p.n_new - 1) / 16;
