@@ -358,14 +358,17 @@ def attend_from_host(cache: Cache, q_host: torch.Tensor, k_new_host: torch.Tenso
                      scale: float, out_host: torch.Tensor, q_dev: torch.Tensor, k_dev: torch.Tensor | None,
                      v_dev: torch.Tensor | None, stream=None) -> torch.Tensor:
     """One decode step with HOST buffers: copy the new token's K/V and the query from pinned host
-    memory to the device, append, attend, copy the output back (all on one stream)."""
+    memory to the device, append, attend, copy the output back (all on one stream).  The copies in
+    come first, so that the append and the attend follow each other directly (the attend is then
+    scheduled while the append runs)."""
     s = stream if stream is not None else torch.cuda.current_stream()
     with torch.cuda.stream(s):
         if k_new_host is not None:
             k_dev.copy_(k_new_host, non_blocking=True)
             v_dev.copy_(v_new_host, non_blocking=True)
-            cache.append(k_dev, v_dev, stream=s)
         q_dev.copy_(q_host, non_blocking=True)
+        if k_new_host is not None:
+            cache.append(k_dev, v_dev, stream=s)
         out = cache.attend(q_dev, scale, stream=s)
         out_host.copy_(out, non_blocking=True)
     return out_host
