@@ -93,7 +93,7 @@ int32_t max_splits(const kv1b_cache_t* c) {
 
 int cuda_status(cudaError_t e) { return e == cudaSuccess ? KV1B_OK : KV1B_ERR_CUDA; }
 
-// Partial slots of the persistent kernel: segments x pieces x G x (6 + 128) floats; the piece
+// Partial slots of the persistent kernel: segments x pieces x G x (2 + 128) floats; the piece
 // count per segment does not depend on the length, so the capacity-sized plan bounds every call.
 size_t ws_bytes_needed(const kv1b_cache_t* c, int32_t num_q_heads) {
   const int Gq = num_q_heads / c->num_kv_heads;
@@ -101,7 +101,7 @@ size_t ws_bytes_needed(const kv1b_cache_t* c, int32_t num_q_heads) {
   const int G = kv1b_ws_template_group(Gq < 4 ? Gq : 4);  // head slots of one launch
   int64_t T, Lt;
   int ncta, pieces;
-  kv1b_ws_plan(c->batch, c->num_kv_heads, G, c->capacity, num_sms(), &T, &Lt, &ncta, &pieces);
+  kv1b_ws_plan(c->batch, c->num_kv_heads, c->capacity, num_sms(), &T, &Lt, &ncta, &pieces);
   return static_cast<size_t>(c->batch) * c->num_kv_heads * pieces * G * kv1b::kPartStride * 4;
 }
 
@@ -141,10 +141,10 @@ int ws_params(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t
   w->scale = scale;
   w->L = static_cast<int32_t>(maxlen);
   int ncta = 0, pieces = 0;
-  kv1b_ws_plan(cache->batch, cache->num_kv_heads, G, maxlen, num_sms(), &w->T, &w->Lt, &ncta, &pieces);
+  kv1b_ws_plan(cache->batch, cache->num_kv_heads, maxlen, num_sms(), &w->T, &w->Lt, &ncta, &pieces);
   int64_t Tc, Ltc;
   int nc, pieces_cap;
-  kv1b_ws_plan(cache->batch, cache->num_kv_heads, G, cache->capacity, num_sms(), &Tc, &Ltc, &nc, &pieces_cap);
+  kv1b_ws_plan(cache->batch, cache->num_kv_heads, cache->capacity, num_sms(), &Tc, &Ltc, &nc, &pieces_cap);
   w->ncta = ncta;
   w->max_pieces = pieces_cap > pieces ? pieces_cap : pieces;
   if (w->max_pieces > 256 || static_cast<size_t>(cache->batch) * cache->num_kv_heads * w->max_pieces * G *
@@ -195,7 +195,7 @@ int kv1b_attend_ws_buffers(const kv1b_cache_t* cache, const void* q, int32_t q_d
   const int64_t maxlen = max_length(cache);
   w.L = static_cast<int32_t>(maxlen);
   int ncta = 0, pieces = 0;
-  kv1b_ws_plan(cache->batch, cache->num_kv_heads, G, maxlen, num_sms(), &w.T, &w.Lt, &ncta, &pieces);
+  kv1b_ws_plan(cache->batch, cache->num_kv_heads, maxlen, num_sms(), &w.T, &w.Lt, &ncta, &pieces);
   w.ncta = ncta;
   w.max_pieces = pieces;
   if (pieces > 256 ||

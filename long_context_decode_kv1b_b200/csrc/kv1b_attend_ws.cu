@@ -858,7 +858,7 @@ int kv1b_ws_template_group(int32_t G) { return G >= 3 ? 4 : G; }
 
 // CTAs = SMs (fewer when there are fewer tiles); T, Lt in 128-token tiles; partial rows per
 // segment = the most CTAs one segment can touch.
-void kv1b_ws_plan(int32_t B, int32_t Hkv, int32_t G, int64_t L, int num_sms, int64_t* T, int64_t* Lt, int* ncta,
+void kv1b_ws_plan(int32_t B, int32_t Hkv, int64_t L, int num_sms, int64_t* T, int64_t* Lt, int* ncta,
                   int* max_pieces) {
   const int64_t lt = (L + ws::kTileTok - 1) / ws::kTileTok;
   const int64_t tot = static_cast<int64_t>(B) * Hkv * lt;
@@ -868,7 +868,6 @@ void kv1b_ws_plan(int32_t B, int32_t Hkv, int32_t G, int64_t L, int num_sms, int
   *Lt = lt;
   *ncta = n;
   *max_pieces = tot > 0 ? static_cast<int>((lt * n + tot - 1) / tot + 1) : 1;
-  (void)G;
 }
 
 cudaError_t kv1b_launch_attend_ws(AttendWsParams& p, int32_t G, bool counters_clean, cudaStream_t stream,

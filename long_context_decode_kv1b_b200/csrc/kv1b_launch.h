@@ -229,7 +229,7 @@ int kv1b_ws_template_group(int32_t G);  // query heads per launch slot of the pe
 int kv1b_attend_ws_buffers(const kv1b_cache_t* cache, const void* q, int32_t q_dtype, int32_t num_q_heads,
                            float scale, float* out, float* part, size_t part_bytes, unsigned* counters,
                            cudaStream_t stream);
-void kv1b_ws_plan(int32_t B, int32_t Hkv, int32_t G, int64_t L, int num_sms, int64_t* T, int64_t* Lt, int* ncta,
+void kv1b_ws_plan(int32_t B, int32_t Hkv, int64_t L, int num_sms, int64_t* T, int64_t* Lt, int* ncta,
                   int* max_pieces);
 cudaError_t kv1b_launch_attend_ws(kv1b::AttendWsParams& p, int32_t G, bool counters_clean, cudaStream_t stream,
                                   bool probe = false);
