@@ -327,6 +327,9 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
         issue_stage(p, is.seg, is.lt, n, smem + st * kStageBytes, &full_bar[st]);
         is.advance(n, Lt);
         ++j;
+        // the first stage alone first: every CTA's first stage then lands at once instead of with
+        // the ring's other stages, and the compute warps start about 3 us earlier
+        if (j == 1 && !mbar_wait(&full_bar[0], 0, &s_abort, p.wait_tries)) break;
       }
       // the CTA's shared memory must outlive every copy issued into it (the compute warps wait
       // for all of them unless the CTA gave up)
@@ -455,17 +458,12 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
       }
     }
     named_bar(1, kThreads);
+    // thread (h, ch) for h = threadIdx.x >> 7 and h + 3: the pieces' o[ch] of both heads are loaded
+    // 16 pieces at a time, all loads issued before the sums (one round trip to L2 per 16 pieces)
     const int ch = threadIdx.x & 127;
-    for (int h = threadIdx.x >> 7; h < NH; h += kThreads / 128) {
-      const float* w = sm_m + h * 256;
-      const float* o = base + h * kPartStride + 2 + ch;
-      float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
-      int k = 0;
-      for (; k + 4 <= n; k += 4) {
-        #pragma unroll
-        for (int u = 0; u < 4; ++u) acc[u] = __fmaf_rn(w[k + u], o[(k + u) * stride], acc[u]);
-      }
-      for (; k < n; ++k) acc[0] = __fmaf_rn(w[k], o[k * stride], acc[0]);
+    const int ha = threadIdx.x >> 7, hb = ha + kThreads / 128;
+    const bool two = hb < NH;
+    auto emit = [&](int h, const float (&acc)[4]) {
       const float den = sm_d[h];
       const float num = __fadd_rn(__fadd_rn(acc[0], acc[1]), __fadd_rn(acc[2], acc[3]));
       const int64_t orow = static_cast<int64_t>(b) * p.Hq + kvh * GA + HB + h;
@@ -479,6 +477,31 @@ __global__ void __launch_bounds__(kBlock, 1) attend_ws_kernel(const __grid_const
       } else {
         p.out[orow * kD + ch] = den > 0.0f ? __fdiv_rn(num, den) : 0.0f;
       }
+    };
+    if (ha < NH) {
+      const float* oa = base + ha * kPartStride + 2 + ch;
+      const float* ob = base + (two ? hb : ha) * kPartStride + 2 + ch;
+      const float* wa = sm_m + ha * 256;
+      const float* wb = sm_m + (two ? hb : ha) * 256;
+      float acca[4] = {0.0f, 0.0f, 0.0f, 0.0f}, accb[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      for (int k0 = 0; k0 < n; k0 += 16) {
+        float xa[16], xb[16];
+        #pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          const bool in = k0 + u < n;
+          xa[u] = in ? oa[(k0 + u) * stride] : 0.0f;
+          xb[u] = (in && two) ? ob[(k0 + u) * stride] : 0.0f;
+        }
+        #pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          if (k0 + u < n) {
+            acca[u & 3] = __fmaf_rn(wa[k0 + u], xa[u], acca[u & 3]);
+            accb[u & 3] = __fmaf_rn(wb[k0 + u], xb[u], accb[u & 3]);
+          }
+        }
+      }
+      emit(ha, acca);
+      if (two) emit(hb, accb);
     }
   };
 
