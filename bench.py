@@ -36,8 +36,8 @@ ATTEND_SRC = os.path.join(ROOT, "long_context_decode_kv1b_b200", "csrc", "kv1b_a
 # DRAM bytes (read + write) per token x kv-head of one attend kernel launch, from an ncu capture of
 # the c3 workload (same head grouping, cache 218 MB > L2) scaled by the tokens x kv-heads it
 # processed; valid only for the attend source with this SHA-256 (profiles/attend_ws_c3_ncu_full.txt).
-TRAFFIC = {"bytes_per_token_head": (219227136 + 5009920) / 2097408,
-           "source_sha256": "09e0bee4ac21bc2fc49b53d873e41110f58db71fba44487b559403fc016700cf"}
+TRAFFIC = {"bytes_per_token_head": (219185920 + 6267136) / 2097408,
+           "source_sha256": "a52ede72530e4b5b3da5c7ef6d5a19320f6fe40d9978fed1bf36cba0411d2740"}
 
 
 def parse_args():
