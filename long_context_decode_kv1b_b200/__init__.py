@@ -374,6 +374,41 @@ def attend_from_host(cache: Cache, q_host: torch.Tensor, k_new_host: torch.Tenso
     return out_host
 
 
+def step_block_views(block: torch.Tensor, batch: int, num_kv_heads: int, num_q_heads: int, dtype):
+    """Views of one decode step's inputs packed in a uint8 block: the new token's K
+    [batch, 1, num_kv_heads, 128], then its V, then the query [batch, num_q_heads, 128], all in
+    `dtype`, each starting on a 256-byte multiple.  Returns (k, v, q)."""
+    esz = torch.empty((), dtype=dtype).element_size()
+    nk = batch * num_kv_heads * HEAD_DIM * esz
+    nq = batch * num_q_heads * HEAD_DIM * esz
+    if block.dtype != torch.uint8 or block.numel() < 2 * nk + nq or not block.is_contiguous():
+        raise ValueError("block must be a contiguous uint8 tensor of at least step_block_bytes() bytes")
+    k = block[:nk].view(dtype).view(batch, 1, num_kv_heads, HEAD_DIM)
+    v = block[nk:2 * nk].view(dtype).view(batch, 1, num_kv_heads, HEAD_DIM)
+    q = block[2 * nk:2 * nk + nq].view(dtype).view(batch, num_q_heads, HEAD_DIM)
+    return k, v, q
+
+
+def step_block_bytes(batch: int, num_kv_heads: int, num_q_heads: int, dtype) -> int:
+    esz = torch.empty((), dtype=dtype).element_size()
+    return (2 * batch * num_kv_heads + batch * num_q_heads) * HEAD_DIM * esz
+
+
+def attend_from_host_block(cache: Cache, host_block: torch.Tensor, dev_block: torch.Tensor, num_q_heads: int, dtype,
+                           scale: float, out_host: torch.Tensor, stream=None) -> torch.Tensor:
+    """One decode step whose inputs (the new token's K and V and the query, laid out as
+    step_block_views describes) sit in ONE pinned host block: one copy in, append, attend, the
+    output copied back -- two copies per step instead of four."""
+    s = stream if stream is not None else torch.cuda.current_stream()
+    with torch.cuda.stream(s):
+        dev_block.copy_(host_block, non_blocking=True)
+        k, v, q = step_block_views(dev_block, cache.batch, cache.num_kv_heads, num_q_heads, dtype)
+        cache.append(k, v, stream=s)
+        out = cache.attend(q, scale, stream=s)
+        out_host.copy_(out, non_blocking=True)
+    return out_host
+
+
 def unpack_codes(v_codes: torch.Tensor, length: int) -> torch.Tensor:
     """Logical codes [length, 128] (uint8) of one (sequence, kv-head) from the code plane
     [capacity/128, 128, 16] (128-token tiles, channel-major rows; nibble j of word w of a row is

@@ -306,6 +306,33 @@ def test_attend_workspace_counters_left_clean():
     assert cache.status() == 0
 
 
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+def test_decode_step_from_one_pinned_block(dtype):
+    # a decode step whose new K/V and query come in one pinned host block (one copy in) against the
+    # same step from device tensors, on two caches built alike; and against the oracle
+    B, Hkv, G = 2, 2, 4
+    c1, host = build_cache(B, Hkv, [900], dtype, seed=12, data_seed=2, cap=1024)
+    c2, _ = build_cache(B, Hkv, [900], dtype, seed=12, data_seed=2, cap=1024)
+    g = torch.Generator(device=DEV).manual_seed(77)
+    k, v = rand_kv(g, B, 1, Hkv, dtype)
+    q = torch.randn((B, Hkv * G, 128), generator=g, device=DEV).to(dtype)
+    nblk = kv.step_block_bytes(B, Hkv, Hkv * G, dtype)
+    hb = torch.empty(nblk, dtype=torch.uint8).pin_memory()
+    hk, hv, hq = kv.step_block_views(hb, B, Hkv, Hkv * G, dtype)
+    hk.copy_(k.cpu()), hv.copy_(v.cpu()), hq.copy_(q.cpu())
+    db = torch.empty(nblk, dtype=torch.uint8, device=DEV)
+    outh = torch.empty((B, Hkv * G, 128), dtype=torch.float32).pin_memory()
+    kv.attend_from_host_block(c1, hb, db, Hkv * G, dtype, 0.2, outh)
+    c2.append(k, v)
+    ref_dev = c2.attend(q, 0.2)
+    torch.cuda.synchronize()
+    assert torch.equal(outh, ref_dev.cpu())
+    host.add(k, v)
+    ref = oracle_attend_all(host, q, oracle.signs(12), 0.2, G)
+    assert_rows_close(outh.numpy(), ref, where="one-block step")
+    assert c1.status() == 0
+
+
 # ------------------------------------------------------------------------------------- Top-p
 def topp_check(cache, host, q, scale, p, G, signs, rows=None):
     out, sel, cnt = cache.attend_topp(q, scale, p)
