@@ -142,3 +142,25 @@ def test_binding_passes_workspace_clean_flag_after_first_attend(monkeypatch):
     assert c.status(stream=st) == kv.STATUS_TIMEOUT
     c.attend(q, 0.1, out=out, stream=st)
     assert calls[-1] == kv.ATTEND_TENSOR
+
+
+def test_step_block_views_layout():
+    # one decode step's inputs in one block: K, then V, then q, each at a 256-byte multiple, each a
+    # view of the block (a write through a view lands at the documented offset)
+    import torch
+
+    for dtype, esz in ((torch.bfloat16, 2), (torch.float32, 4)):
+        B, Hkv, Hq = 3, 2, 8
+        n = kv.step_block_bytes(B, Hkv, Hq, dtype)
+        assert n == (2 * B * Hkv + B * Hq) * 128 * esz
+        blk = torch.zeros(n, dtype=torch.uint8)
+        k, v, q = kv.step_block_views(blk, B, Hkv, Hq, dtype)
+        assert k.shape == (B, 1, Hkv, 128) and v.shape == (B, 1, Hkv, 128) and q.shape == (B, Hq, 128)
+        nk = B * Hkv * 128 * esz
+        assert v.data_ptr() - blk.data_ptr() == nk and q.data_ptr() - blk.data_ptr() == 2 * nk
+        assert nk % 256 == 0
+        v.fill_(1)
+        assert blk[:nk].count_nonzero() == 0 and blk[nk:2 * nk].count_nonzero() > 0
+        assert blk[2 * nk:].count_nonzero() == 0
+        with pytest.raises(ValueError):
+            kv.step_block_views(blk[:-1], B, Hkv, Hq, dtype)
