@@ -5,7 +5,7 @@ import torch
 import oracle
 import long_context_decode_kv1b_b200 as kv
 
-TOL = 1e-3  # the benchmark spec: <= 1e-3 relative error for attention outputs (fp32 accumulation)
+TOL = 1e-3  # the output bar: <= 1e-3 relative error for attention outputs (fp32 accumulation)
 
 
 def to_np32(t: torch.Tensor) -> np.ndarray:
