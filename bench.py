@@ -295,7 +295,7 @@ class OracleSample:
 
 
 def cpu_baseline(cfg, budget_s: float = 20.0):
-    """The oracle, as it stands, on the machine's host cores: the same bounded sample the reference arm
+    """The oracle, as it stands, on this machine's host cores: the same bounded sample the reference arm
     times, first on one thread, then on every core; about budget_s seconds in all."""
     smp = OracleSample(cfg)
     qs = smp.queries(0)
